@@ -1,0 +1,401 @@
+#!/usr/bin/env python
+"""Benchmark of the hybrid-head KV attention path on B200.
+
+Headline workload (N = 1): decode attention of a Llama-3-8B-shaped GQA layer (32 q /
+8 kv heads, d 128, 4 retrieval + 4 streaming kv heads, S 16, W 512, bf16) at a
+128K-token context, batch 1.  One step = for each of 4 layer caches in turn (4 x
+1.08 GB of K/V, larger than L2, so no L2 flush is needed): append the new token's
+K/V and run decode attention -- the whole decode path (append/evict, retrieval
+split-KV, streaming sink+ring, merge).  value = algorithmic HBM bytes of the decode
+attention per step / step time (GB/s).  The chunked pre-fill workload (256K prompt
+in 32K chunks, same shape) is timed after it and reported under "prefill".
+
+--impl reference times the fp64 CPU oracle on the host cores on a bounded sample of
+the same workload (the reference arm).  Under torchrun every rank runs an
+independent replica (the path does not shard); value sums the ranks' bytes over
+the slowest rank's time.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "decode-attn achieved HBM GB/s + μs/token/layer at 128K; prefill TFLOP/s"
+WORKLOAD = "llama3-8b-gqa-decode-128k-b1"
+HQ, HKV, D, NRET, S, W = 32, 8, 128, 4, 16, 512
+CTX = 131072
+ROT_LAYERS = 4
+PREFILL_LEN, PREFILL_CHUNK = 262144, 32768
+
+
+def decode_bytes(len_, B=1, Hr=NRET, Hs=HKV - NRET, Hq=HQ, d=D):
+    """Algorithmic HBM bytes of one decode-attention call: every visible K and V row
+    once (bf16), the queries, the outputs and the lse."""
+    kv = 2 * d * 2
+    return B * (Hr * len_ * kv + Hs * min(len_, S + W) * kv) + B * Hq * d * 2 * 2 + B * Hq * 4
+
+
+def prefill_flops(L=PREFILL_LEN, Hq=HQ, d=D, G=HQ // HKV, nret=NRET):
+    """Algorithmic FLOPs of the full pre-fill: 4 d per visible (query, key) pair."""
+    retr_pairs = L * (L + 1) // 2
+    sw = S + W
+    # streaming rows: i+1 keys while i < S+W, then S+W
+    strm_pairs = sw * (sw + 1) // 2 + (L - sw) * sw if L > sw else L * (L + 1) // 2
+    return 4 * d * G * (nret * retr_pairs + (HKV - nret) * strm_pairs)
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        p = json.load(open(path))
+        return p["hbm_gbs"], p["bf16_tflops"], p.get("bf16_tflops_sustained", p["bf16_tflops"]), "measured"
+    return 6650.0, 1590.0, 1400.0, "fallback"
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle samples during the timed region."""
+
+    def __init__(self, index=0):
+        self.index, self.proc, self.lines = index, None, []
+
+    def __enter__(self):
+        q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", f"--id={self.index}", f"--query-gpu={q}",
+                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.t = threading.Thread(target=self._read, daemon=True)
+            self.t.start()
+        except (FileNotFoundError, OSError):
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def __exit__(self, *a):
+        if self.proc:
+            time.sleep(0.25)
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in self.lines:
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx = float(f[2])
+            except ValueError:
+                continue
+            for n, val in zip(names, f[5:9]):
+                if val.lower() == "active":
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def kernel_hash():
+    h = hashlib.sha256()
+    for f in ("k_decode.cu", "device_common.cuh", "duo_internal.h"):
+        h.update(open(os.path.join(ROOT, "head_split_kv_duo_b200", "csrc", f), "rb").read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic():
+    """DRAM bytes per decode launch from the committed ncu summary, when it was taken
+    on the current kernel source."""
+    path = os.path.join(ROOT, "profiles", "decode_traffic.json")
+    if not os.path.exists(path):
+        return None
+    rec = json.load(open(path))
+    if rec.get("kernel_hash") != kernel_hash():
+        return None
+    return rec.get("dram_bytes_per_launch_full_size")
+
+
+# ---------------------------------------------------------------- our arm
+
+def run_ours(args, rank, world, dist):
+    import torch
+
+    from head_split_kv_duo_b200 import inputs
+    from head_split_kv_duo_b200.duo import DuoCache
+
+    dev = torch.device("cuda", int(os.environ.get("LOCAL_RANK", 0)))
+    torch.cuda.set_device(dev)
+    hbm_peak, tc_peak, tc_sust, peak_src = peaks()
+    steps, warmup = args.steps, args.warmup
+    total_tokens = warmup + steps + 1
+    max_len = CTX + warmup + 2 * steps + 16
+    mask = inputs.retrieval_mask(ROT_LAYERS, HKV, NRET, seed=1)
+    cache = DuoCache(ROT_LAYERS, HKV, D, mask, S, W, max_len, q_heads=HQ, dtype=torch.bfloat16, device=dev)
+    # fill each layer to CTX tokens (seeded N(0,1) K/V)
+    for layer in range(ROT_LAYERS):
+        k = inputs.randn((1, CTX, HKV, D), 100 + 2 * layer, device=dev)
+        v = inputs.randn((1, CTX, HKV, D), 101 + 2 * layer, device=dev)
+        cache.append_kv(layer, k, v)
+        del k, v
+    torch.cuda.synchronize()
+    # per-step inputs: q, k, v of the new token for every layer
+    nstep_in = warmup + steps
+    qs = inputs.randn((nstep_in, ROT_LAYERS, 1, HQ, D), 7, device=dev)
+    ks = inputs.randn((nstep_in, ROT_LAYERS, 1, 1, HKV, D), 8, device=dev)
+    vs = inputs.randn((nstep_in, ROT_LAYERS, 1, 1, HKV, D), 9, device=dev)
+    out = torch.empty(ROT_LAYERS, 1, HQ, D, dtype=torch.bfloat16, device=dev)
+    lse = torch.empty(ROT_LAYERS, 1, HQ, dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def step(i, ev=None):
+        nbytes = 0
+        for layer in range(ROT_LAYERS):
+            cache.append_kv(layer, ks[i, layer], vs[i, layer], stream=stream)
+            n = cache.len(layer)
+            if ev is not None:
+                ev[0].record(stream)
+            cache.decode_attention(layer, qs[i, layer], out=out[layer], lse=lse[layer], stream=stream)
+            if ev is not None:
+                ev[1].record(stream)
+                ev[2].append((ev[0], ev[1]))
+                ev[0] = torch.cuda.Event(enable_timing=True)
+                ev[1] = torch.cuda.Event(enable_timing=True)
+            nbytes += decode_bytes(n)
+        return nbytes
+
+    for i in range(warmup):
+        step(i)
+    torch.cuda.synchronize()
+    if dist:
+        dist.barrier()
+    kev = [torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True), []]
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    nbytes = 0
+    with ClockSampler(dev.index) as clk:
+        torch.cuda.synchronize()
+        t0.record(stream)
+        for i in range(warmup, warmup + steps):
+            nbytes += step(i, kev)
+        t1.record(stream)
+        torch.cuda.synchronize()
+    if dist:
+        dist.barrier()
+    ms = t0.elapsed_time(t1)
+    dec_ms = [a.elapsed_time(b) for a, b in kev[2]]
+    assert cache.device_status() == 0, "device status word set"
+    ms_max, bytes_sum = ms, nbytes
+    if dist:
+        t = torch.tensor([ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms_max = float(t.item())
+        b = torch.tensor([float(nbytes)], device=dev, dtype=torch.float64)
+        dist.all_reduce(b)
+        bytes_sum = float(b.item())
+    value = bytes_sum / (ms_max * 1e-3) / 1e9
+    us_per_token_layer = ms * 1e3 / (steps * ROT_LAYERS)
+    dec_avg_ms = statistics.mean(dec_ms)
+    per_launch_bytes = nbytes / (steps * ROT_LAYERS)
+    achieved = per_launch_bytes / (dec_avg_ms * 1e-3) / 1e9
+
+    # ---- end-to-end through the public API with host buffers ----
+    e2e = None
+    if not args.skip_e2e:
+        hq = qs.cpu().pin_memory()
+        hk = ks.cpu().pin_memory()
+        hv = vs.cpu().pin_memory()
+        hout = torch.empty(ROT_LAYERS, 1, HQ, D, dtype=torch.bfloat16).pin_memory()
+        dq = torch.empty_like(qs[0])
+        dk = torch.empty_like(ks[0])
+        dv = torch.empty_like(vs[0])
+        # rewind lengths is not possible; continue appending (lengths grow by `steps`)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        eb = 0
+        torch.cuda.synchronize()
+        e0.record(stream)
+        for i in range(warmup, warmup + steps):
+            dq.copy_(hq[i], non_blocking=True)
+            dk.copy_(hk[i], non_blocking=True)
+            dv.copy_(hv[i], non_blocking=True)
+            for layer in range(ROT_LAYERS):
+                cache.append_kv(layer, dk[layer], dv[layer], stream=stream)
+                eb += decode_bytes(cache.len(layer))
+                cache.decode_attention(layer, dq[layer], out=out[layer], lse=lse[layer], stream=stream)
+            hout.copy_(out, non_blocking=True)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        ems = e0.elapsed_time(e1)
+        h2d = (dq.numel() + dk.numel() + dv.numel()) * 2
+        e2e = {"value": round(eb / (ems * 1e-3) / 1e9, 1), "unit": "GB/s", "h2d_bytes_per_step": h2d,
+               "d2h_bytes_per_step": hout.numel() * 2, "ms_per_step": round(ems / steps, 4)}
+
+    # ---- chunked pre-fill (Llama-3-8B GQA, 256K in 32K chunks) ----
+    prefill = None
+    if not args.skip_prefill:
+        prefill = run_prefill(args, dev, tc_peak, tc_sust, peak_src)
+
+    res = {
+        "metric": METRIC, "value": round(value, 1), "unit": "GB/s", "n_gpus": world, "steps": steps,
+        "warmup": warmup, "ms_per_step": round(ms_max / steps, 4), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": WORKLOAD, "q_heads": HQ, "kv_heads": HKV, "head_dim": D, "retrieval_kv_heads": NRET,
+                   "S": S, "W": W, "context": CTX, "batch": 1, "layers_rotated": ROT_LAYERS,
+                   "l2": "inputs larger than L2: 4 rotating layer caches of 1.08 GB", "parallelism": f"replicas{world}"},
+        "us_per_token_layer": round(us_per_token_layer, 3),
+        "roofline": {"bound": "hbm", "kernel": "decode_kernel", "achieved": round(achieved, 1),
+                     "peak": hbm_peak, "peak_source": f"{peak_src} hbm_gbs (burst copy)", "unit": "GB/s",
+                     "frac": round(achieved / hbm_peak, 4), "traffic": recorded_traffic(),
+                     "algorithmic_bytes_per_launch": int(per_launch_bytes), "avg_launch_us": round(dec_avg_ms * 1e3, 3)},
+        "gpu_launches": steps * ROT_LAYERS * 2,
+        "clocks": clk.summary(),
+        "e2e": e2e,
+        "prefill": prefill,
+    }
+    return res
+
+
+def run_prefill(args, dev, tc_peak, tc_sust, peak_src):
+    import torch
+
+    from head_split_kv_duo_b200 import inputs
+    from head_split_kv_duo_b200.duo import DuoCache
+
+    mask = inputs.retrieval_mask(1, HKV, NRET, seed=1)
+    k = inputs.randn((1, PREFILL_LEN, HKV, D), 200, device=dev)
+    v = inputs.randn((1, PREFILL_LEN, HKV, D), 201, device=dev)
+    q = inputs.randn((1, PREFILL_CHUNK, HQ, D), 202, device=dev)  # same queries for every chunk
+    out = torch.empty_like(q)
+    nchunks = PREFILL_LEN // PREFILL_CHUNK
+    stream = torch.cuda.current_stream()
+
+    def one():
+        cache = DuoCache(1, HKV, D, mask, S, W, PREFILL_LEN, q_heads=HQ, dtype=torch.bfloat16, device=dev)
+        evs = []
+        for c in range(nchunks):
+            sl = slice(c * PREFILL_CHUNK, (c + 1) * PREFILL_CHUNK)
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            cache.prefill_chunk(0, q, k[:, sl], v[:, sl], out=out, want_lse=False, stream=stream)
+            b.record(stream)
+            evs.append((a, b))
+        torch.cuda.synchronize()
+        assert cache.device_status() == 0
+        cache.close()
+        return sum(x.elapsed_time(y) for x, y in evs)
+
+    for _ in range(args.prefill_warmup):
+        one()
+    times = [one() for _ in range(args.prefill_steps)]
+    ms = statistics.mean(times)
+    fl = prefill_flops()
+    tflops = fl / (ms * 1e-3) / 1e12
+    return {"workload": "llama3-8b-gqa-prefill-256k-chunk32k", "tflops": round(tflops, 1), "ms": round(ms, 2),
+            "steps": args.prefill_steps, "algorithmic_tflop": round(fl / 1e12, 2),
+            "roofline": {"bound": "tensor", "achieved": round(tflops, 1), "peak": tc_peak,
+                         "peak_source": f"{peak_src} bf16_tflops (burst)", "unit": "TFLOP/s",
+                         "frac": round(tflops / tc_peak, 4), "frac_of_sustained": round(tflops / tc_sust, 4)}}
+
+
+# ---------------------------------------------------------- reference arm
+
+def oracle_sample(args):
+    """Time the fp64 oracle on decode steps of the headline workload (one layer at
+    128K context; each step = one query token, all 32 query heads)."""
+    import numpy as np
+    import torch
+
+    import oracle
+    from head_split_kv_duo_b200 import inputs
+
+    mask = inputs.retrieval_mask(1, HKV, NRET, seed=1)[0].numpy().astype(bool)
+    k = inputs.randn((1, CTX, HKV, D), 100).view(torch.int16).numpy().view(np.uint16)
+    v = inputs.randn((1, CTX, HKV, D), 101).view(torch.int16).numpy().view(np.uint16)
+    q = inputs.randn((1, 1, HQ, D), 7).view(torch.int16).numpy().view(np.uint16)
+    oracle.attend(q, k[:, :1024], v[:, :1024], mask, S, W, pos0=1023)  # load / warm
+    n, t_total = 0, 0.0
+    budget = args.oracle_seconds
+    while t_total < budget and n < args.oracle_max_steps:
+        t = time.perf_counter()
+        oracle.attend(q, k, v, mask, S, W, pos0=CTX - 1)
+        t_total += time.perf_counter() - t
+        n += 1
+    gbs = n * decode_bytes(CTX) / t_total / 1e9
+    return {"value": round(gbs, 3), "unit": "GB/s", "cores": oracle.num_threads(), "kind": "oracle",
+            "sample": f"{n} decode steps of one layer at context {CTX} (all 32 query heads), "
+                      f"{t_total:.1f} s wall on {oracle.num_threads()} threads",
+            "seconds": round(t_total, 2), "steps": n}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--skip-prefill", action="store_true")
+    ap.add_argument("--skip-e2e", action="store_true")
+    ap.add_argument("--skip-cpu-baseline", action="store_true")
+    ap.add_argument("--prefill-steps", type=int, default=2)
+    ap.add_argument("--prefill-warmup", type=int, default=1)
+    ap.add_argument("--oracle-seconds", type=float, default=6.0)
+    ap.add_argument("--oracle-max-steps", type=int, default=40)
+    args = ap.parse_args()
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+
+    if args.impl == "reference":
+        if rank != 0:
+            return 0
+        t0 = time.perf_counter()
+        for _ in range(args.warmup):
+            pass
+        cb = oracle_sample(args)
+        res = {"impl": "reference", "metric": METRIC, "value": cb["value"], "unit": "GB/s", "n_gpus": args.gpus,
+               "steps": cb["steps"], "warmup": args.warmup, "ms_per_step": round(cb["seconds"] * 1e3 / max(cb["steps"], 1), 3),
+               "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+               "config": {"workload": WORKLOAD, "q_heads": HQ, "kv_heads": HKV, "head_dim": D,
+                          "retrieval_kv_heads": NRET, "S": S, "W": W, "context": CTX, "batch": 1},
+               "cpu_baseline": cb,
+               "e2e": {"value": cb["value"], "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+               "wall_s": round(time.perf_counter() - t0, 1)}
+        print(json.dumps(res))
+        return 0
+
+    dist = None
+    if world > 1:
+        import datetime
+
+        import torch.distributed as tdist
+        tdist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+        dist = tdist
+    res = run_ours(args, rank, world, dist)
+    if rank == 0 and not args.skip_cpu_baseline:
+        res["cpu_baseline"] = oracle_sample(args)
+    if dist:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(res))
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

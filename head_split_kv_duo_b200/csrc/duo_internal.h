@@ -1,0 +1,134 @@
+// duo_internal.h -- host/device shared structures of the hybrid-head KV cache.
+// Not part of the public ABI (include/duo.h is).
+#pragma once
+
+#include <cstddef>
+#include <cstdint>
+#include <vector>
+
+#include <cuda_runtime.h>
+
+#include "duo.h"
+
+namespace duo {
+
+constexpr int kMaxKvHeads = 128;
+constexpr int kAlign = 1024;          // every carved region starts on a 1 KiB boundary
+constexpr int kMinSplitTokens = 256;  // shortest split of a retrieval head in decode
+constexpr int kMaxSplits = 512;       // most splits of one retrieval head in decode
+
+// Device status word bits (latched, cleared by duo_get_device_status).
+constexpr uint32_t kDevTimeout = 1u;
+
+// Head partition of one layer, passed to kernels by value.
+struct HeadMap {
+  uint8_t is_retr[kMaxKvHeads];   // kv head -> 1 retrieval / 0 streaming
+  uint8_t kind_idx[kMaxKvHeads];  // kv head -> index among heads of its kind
+  uint8_t retr_head[kMaxKvHeads]; // retrieval index -> kv head
+  uint8_t strm_head[kMaxKvHeads]; // streaming index -> kv head
+};
+
+struct Layer {
+  int Hr = 0, Hs = 0;
+  HeadMap hm{};
+  // retrieval K/V: [B][Hr][max_len][row] (row = d elements, or d/2 INT4 bytes)
+  char *rk = nullptr, *rv = nullptr;
+  // INT4 scale/zero: [B][Hr][max_len][2] fp16
+  char *rk_sz = nullptr, *rv_sz = nullptr;
+  // streaming K/V: [B][Hs][S+W][d]
+  char *sk = nullptr, *sv = nullptr;
+  int64_t len = 0;
+};
+
+}  // namespace duo
+
+struct duo_cache {
+  int layers = 0, Hkv = 0, Hq = 0, G = 0, D = 0, B = 0, S = 0, W = 0;
+  int64_t max_len = 0;  // capacity in tokens
+  int64_t cap = 0;      // row stride of retrieval arrays: max_len rounded up to 256
+  duo_dtype dtype = DUO_BF16;
+  duo_kv_fmt fmt = DUO_KV_SAME;
+  float scale = 0.f;
+  int esize = 2;
+  char *buf = nullptr;
+  size_t bytes = 0;
+  bool initialised = false;
+  int num_sms = 0;
+  // scratch
+  uint32_t *status = nullptr;    // device status word
+  uint32_t *counters = nullptr;  // [B][Hq] split-merge tickets
+  float *partials = nullptr;     // [B][Hkv][max_splits][G][d+2]
+  int max_splits = 1;
+  char *hist_k = nullptr, *hist_v = nullptr;  // [B][HsMax][S+W][d] pre-fill staging
+  int hs_max = 0;
+  std::vector<duo::Layer> L;
+};
+
+namespace duo {
+
+// ---- kernel parameter blocks ----
+
+struct AppendParams {
+  const char *k, *v;  // [B][n][Hkv][d]
+  char *rk, *rv, *rk_sz, *rv_sz, *sk, *sv;
+  int B, n, Hkv, D, Hr, Hs, S, W;
+  int64_t len, max_len;  // max_len: row stride of retrieval arrays (capacity rounded up to 256)
+  int64_t ring_from;  // first non-sink position that reaches the ring
+  int int4;           // retrieval rows stored INT4
+  HeadMap hm;
+};
+
+struct HistParams {
+  const char *sk, *sv;  // streaming cache of the layer
+  char *hk, *hv;        // staging [B][HsMax][S+W][d]
+  int B, Hs, HsMax, D, S, W;
+  int hs, hw;           // sink rows, window rows staged
+  int64_t wstart;       // position of the first window row
+};
+
+struct DecodeParams {
+  const char *q;
+  char *out;
+  float *lse;
+  const char *rk, *rv, *rk_sz, *rv_sz, *sk, *sv;
+  float *partials;
+  uint32_t *counters, *status;
+  int B, Hq, Hkv, G, D, Hr, Hs, S, W;
+  int64_t len, max_len;  // max_len: row stride of retrieval arrays
+  int nsplit;
+  int64_t split_len;
+  int qg, nqg;        // query heads per CTA, CTAs per KV head
+  int max_splits;
+  int n_retr_ctas;
+  float scale_log2;   // softmax scale * log2(e)
+  HeadMap hm;
+};
+
+struct PrefillParams {
+  const char *q, *k, *v;  // q [B][n][Hq][d]; k, v [B][n][Hkv][d] (the chunk)
+  char *out;
+  float *lse;
+  const char *rk, *rv;    // retrieval cache (chunk already appended)
+  const char *hk, *hv;    // streaming history staging
+  uint32_t *status;
+  int B, n, Hq, Hkv, G, D, Hr, Hs, HsMax, S, W;
+  int64_t len, max_len;  // max_len: row stride of retrieval arrays
+  int hs, hw;
+  int64_t wstart;
+  float scale_log2;
+  HeadMap hm;
+};
+
+// ---- launchers (return cudaSuccess or the launch error) ----
+cudaError_t launch_append(const AppendParams &p, duo_dtype dt, cudaStream_t st);
+cudaError_t launch_hist(const HistParams &p, duo_dtype dt, cudaStream_t st);
+cudaError_t launch_decode(const DecodeParams &p, duo_dtype dt, bool int4, cudaStream_t st);
+cudaError_t launch_prefill_simt(const PrefillParams &p, duo_dtype dt, cudaStream_t st);
+// tcgen05 pre-fill (bf16, d = 128); returns cudaErrorNotSupported when it does not apply
+cudaError_t launch_prefill_tc(const PrefillParams &p, cudaStream_t st);
+bool prefill_tc_supported(const PrefillParams &p, duo_dtype dt);
+
+// decode tiling shared by host (split sizing) and device
+int decode_tokens_per_stage(duo_dtype dt, int D, bool int4);
+
+}  // namespace duo

@@ -1,0 +1,212 @@
+/*
+ * duo.h -- C ABI of the B200 (sm_100a) hybrid-head KV attention library.
+ *
+ * The operation is DuoAttention's deployment path ("DuoAttention: Efficient
+ * Long-Context LLM Inference with Retrieval and Streaming Heads", arXiv 2410.10819,
+ * as explained on the paper-graph-ui page, section "Deployment Architecture"):
+ * each KV head of a layer is either a retrieval head, which keeps every token and
+ * attends with the causal mask, or a streaming head, which keeps only the first S
+ * "attention sink" tokens plus the W most recent tokens and attends with the
+ * Lambda-shaped mask ("The Full and Streaming Attention Masks").
+ *
+ * Conventions shared by every call
+ * ---------------------------------
+ * Notation: B batch, Hq query heads, Hkv KV heads, G = Hq / Hkv, d head_dim,
+ * S sinks, W recent window, len = tokens already in a layer's cache, n = tokens in
+ * one call.  Query head h reads KV head h / G (contiguous GQA grouping); the cache
+ * is kept per KV head, so no K/V row is ever repeated per query head.
+ *
+ * Mask: query at absolute position i sees key j iff j <= i and, for a streaming
+ * head, (j < S or i - j < W).  W counts the query's own token, so a streaming
+ * head holds exactly S + W tokens once len >= S + W, and W >= 1.
+ *
+ * Tensors are dense, row-major, device-resident, 16-byte aligned, in the dtype
+ * chosen at creation (bf16 or fp32):
+ *     decode q, out   [B][Hq][d]          decode lse   [B][Hq]      (fp32)
+ *     prefill q, out  [B][n][Hq][d]       prefill lse  [B][n][Hq]   (fp32)
+ *     k, v            [B][n][Hkv][d]
+ * lse is the natural log of the sum of exp(scaled logits) over the visible keys.
+ * Heads keep the caller's order; the library groups retrieval and streaming heads
+ * internally through index tables, so no weight permutation is needed.
+ *
+ * Ownership: the caller owns every device buffer, the cache storage included
+ * (one buffer of duo_cache_bytes() bytes, 256-byte aligned).  The handle owns only
+ * host metadata.  No pointer is kept beyond the call that receives it, except the
+ * cache buffer, which must outlive the handle.
+ *
+ * Ordering: calls are asynchronous on the given CUDA stream (NULL = legacy default
+ * stream).  Calls on one handle must be ordered on one stream (or externally
+ * synchronised): they share the cache's scratch space.  A handle is not thread-safe.
+ *
+ * Errors: every argument is checked before any launch; on error nothing is
+ * launched and the cache (lengths included) is unchanged.  len advances only when
+ * every launch of the call was accepted.  A failed launch returns DUO_ERR_CUDA.
+ * Conditions detected on the device (a bounded wait that ran out) are latched in a
+ * status word and reported by duo_get_device_status().
+ */
+#ifndef DUO_H
+#define DUO_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define DUO_API __attribute__((visibility("default")))
+#else
+#define DUO_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct duo_cache duo_cache; /* opaque host handle */
+
+typedef enum {
+  DUO_OK = 0,
+  DUO_ERR_INVALID = 1,     /* bad argument (NULL, range, alignment, shape)      */
+  DUO_ERR_CAPACITY = 2,    /* the call would grow a layer past max_len          */
+  DUO_ERR_CUDA = 3,        /* a CUDA runtime call or launch failed              */
+  DUO_ERR_TIMEOUT = 4,     /* a kernel's bounded wait ran out (device status)   */
+  DUO_ERR_UNSUPPORTED = 5  /* valid request this build does not implement       */
+} duo_status;
+
+typedef enum { DUO_BF16 = 0, DUO_FP32 = 1 } duo_dtype;
+
+/* Storage of retrieval-head K/V.  DUO_KV_INT4_G128: 4-bit asymmetric codes, one
+ * group per token row of a head (head_dim must be 128), fp16 scale and zero per
+ * group: scale = fp16((max-min)/15), zero = fp16(min), code = clamp(rint((x - zero)
+ * / scale), 0, 15) in fp32, element 2t in the low nibble of byte t, value =
+ * code*scale + zero.  bf16 only.  Streaming heads always keep the working dtype. */
+typedef enum { DUO_KV_SAME = 0, DUO_KV_INT4_G128 = 1 } duo_kv_fmt;
+
+typedef struct {
+  int batch;           /* B >= 1                                               */
+  int q_heads;         /* Hq, a multiple of kv_heads; 0 means kv_heads (MHA)   */
+  duo_dtype dtype;     /* activations and K/V                                  */
+  duo_kv_fmt retr_fmt; /* retrieval-head storage                               */
+  float softmax_scale; /* logit scale; 0 means 1/sqrt(head_dim)                */
+} duo_opts;            /* NULL opts = {1, 0, DUO_BF16, DUO_KV_SAME, 0}         */
+
+/*
+ * Bytes of device memory a cache needs: the per-layer K/V arrays (retrieval heads
+ * [B][H_r][max_len][d], streaming heads [B][H_s][S+W][d]; the KV memory
+ * (H_r L + H_s (S+R)) d of "Decoding Procedure" at L = max_len) plus scratch for
+ * split-KV decode partials and the pre-fill staging of streaming heads.
+ * Returns 0 when the arguments are invalid (same checks as duo_cache_create).
+ */
+DUO_API size_t duo_cache_bytes(int layers, int kv_heads, int head_dim, const uint8_t *retrieval_head_mask, int S, int W,
+                       int64_t max_len, const duo_opts *opts);
+
+/*
+ * Creates a cache handle over caller-owned device memory ("Deployment
+ * Architecture": two KV caches per layer, pre-allocated).
+ *   layers, kv_heads      >= 1; kv_heads <= 128
+ *   head_dim              64 or 128
+ *   retrieval_head_mask   host [layers][kv_heads], 1 = retrieval, 0 = streaming
+ *                         (the binarised gates of "Optimization-Based Retrieval
+ *                         Head Identification"); copied, not kept
+ *   S >= 0, W >= 1        sinks and recent window of streaming heads
+ *   max_len >= 1          capacity of every retrieval head, in tokens
+ *   dev_buf, dev_bytes    device buffer of >= duo_cache_bytes() bytes, 256-byte
+ *                         aligned; it is zero-filled by the first call that
+ *                         launches work
+ * No device work happens here.  *out receives the handle.
+ */
+DUO_API duo_status duo_cache_create(int layers, int kv_heads, int head_dim, const uint8_t *retrieval_head_mask, int S,
+                            int W, int64_t max_len, const duo_opts *opts, void *dev_buf, size_t dev_bytes,
+                            duo_cache **out);
+
+/* Frees the host handle only; the caller frees dev_buf.  NULL is a no-op. */
+DUO_API void duo_cache_destroy(duo_cache *cache);
+
+/*
+ * Appends n >= 1 tokens (positions len .. len+n-1) of one layer ("Decoding
+ * Procedure", step 4: update both caches).  Retrieval heads store every row
+ * (INT4-quantised when configured).  Streaming heads store position p in slot p
+ * when p < S, else in ring slot S + (p mod W), which evicts position p - W; of an
+ * n-token append only the sinks and the last min(n, W) positions are written
+ * (earlier ones would be evicted within the same call).
+ *   k, v   device [B][n][Hkv][d]
+ * DUO_ERR_CAPACITY if len + n > max_len.
+ */
+DUO_API duo_status duo_append_kv(duo_cache *cache, int layer, const void *k, const void *v, int n, void *cuda_stream);
+
+/*
+ * Chunked pre-fill of one layer ("Chunked Pre-filling", Figure 5 right): the n
+ * queries at positions len .. len+n-1 attend to the layer's cache plus the
+ * chunk itself -- causal mask for retrieval heads, Lambda mask for streaming heads
+ * -- and the chunk is then appended as by duo_append_kv.
+ *   q, out  device [B][n][Hq][d];  k, v device [B][n][Hkv][d]
+ *   lse     device [B][n][Hq] fp32, or NULL
+ * DUO_ERR_UNSUPPORTED for an INT4 retrieval cache.
+ */
+DUO_API duo_status duo_prefill_chunk(duo_cache *cache, int layer, const void *q, const void *k, const void *v, int n,
+                             void *out, float *lse, void *cuda_stream);
+
+/*
+ * Single-token decode attention of one layer ("Decoding Procedure", steps 2, 3
+ * and 5): the query of the newest token, at position len-1, attends to every
+ * cached token of its retrieval head, or to the sinks and ring of its streaming
+ * head.  The token must have been appended first (it attends to itself).
+ *   q, out  device [B][Hq][d];  lse device [B][Hq] fp32, or NULL
+ * DUO_ERR_INVALID if the layer is empty.
+ */
+DUO_API duo_status duo_decode_attention(duo_cache *cache, int layer, const void *q, void *out, float *lse,
+                                void *cuda_stream);
+
+/* Tokens in a layer's cache (host value, no synchronisation). */
+DUO_API duo_status duo_cache_len(const duo_cache *cache, int layer, int64_t *len);
+
+/*
+ * KV memory of the configured cache at sequence length L, in bytes of K plus V:
+ * *retained = what the hybrid cache keeps, (H_r L + H_s min(L, S+W)) d per layer
+ * ("Decoding Procedure"), INT4 codes and scale/zero counted when configured;
+ * *full = what full attention would keep in the working dtype, 2 D H L d elements
+ * ("The Core Problem").  Either pointer may be NULL.
+ */
+DUO_API duo_status duo_kv_bytes(const duo_cache *cache, int64_t L, uint64_t *retained, uint64_t *full);
+
+/*
+ * Position held by a cache slot of one KV head, from the host's bookkeeping
+ * (no device access): retrieval heads hold position `slot` iff slot < len;
+ * streaming heads follow the slot rule of duo_append_kv.  *pos = -1 when empty.
+ */
+DUO_API duo_status duo_debug_slot_position(const duo_cache *cache, int layer, int kv_head, int slot, int64_t *pos);
+
+/*
+ * Device address and size of one storage array of a layer, for inspection and
+ * tests (no device access).  which:
+ *   DUO_REGION_RETR_K / _RETR_V   retrieval heads [B][H_r][cap][row], row = d
+ *                                 elements, or d/2 code bytes for INT4
+ *   DUO_REGION_RETR_KSZ / _VSZ    INT4 only: [B][H_r][cap][2] fp16 (scale, zero)
+ *   DUO_REGION_STRM_K / _STRM_V   streaming heads [B][H_s][S+W][d]
+ * Heads of a kind are in increasing KV-head order.  *cap receives the token stride
+ * of retrieval arrays (max_len rounded up to a multiple of 256).  Any output
+ * pointer may be NULL.  An array with no heads reports 0 bytes.
+ */
+typedef enum {
+  DUO_REGION_RETR_K = 0,
+  DUO_REGION_RETR_V = 1,
+  DUO_REGION_RETR_KSZ = 2,
+  DUO_REGION_RETR_VSZ = 3,
+  DUO_REGION_STRM_K = 4,
+  DUO_REGION_STRM_V = 5
+} duo_region;
+DUO_API duo_status duo_debug_region(const duo_cache *cache, int layer, duo_region which, void **ptr, uint64_t *bytes,
+                                    int64_t *cap);
+
+/*
+ * Synchronises `cuda_stream`, reads and clears the device status word.
+ * DUO_ERR_TIMEOUT if a kernel's bounded wait ran out since the last check.
+ */
+DUO_API duo_status duo_get_device_status(duo_cache *cache, void *cuda_stream);
+
+/* Static description of a status code. */
+DUO_API const char *duo_status_str(duo_status status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* DUO_H */

@@ -1,0 +1,163 @@
+"""CPU tests of the C ABI: the library loads, exports every declared symbol, and its
+host-side checks and bookkeeping behave as include/duo.h states.  No kernel is
+launched; a fake (never dereferenced) device address stands in for the buffer."""
+import ctypes
+import os
+import re
+import subprocess
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from head_split_kv_duo_b200 import duo
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+FAKE = 1 << 40  # 256-byte aligned address that is never touched without a GPU
+
+
+def _declared():
+    text = open(os.path.join(ROOT, "include", "duo.h")).read()
+    return re.findall(r"DUO_API\s+[\w\s\*]*?\b(duo_\w+)\s*\(", text)
+
+
+def test_library_exports_every_declared_symbol():
+    names = _declared()
+    assert len(names) >= 12
+    lib = duo.lib()
+    for n in names:
+        assert hasattr(lib, n), n
+    out = subprocess.run(["nm", "-D", "--defined-only", duo._build.LIB], capture_output=True, text=True).stdout
+    exported = set(re.findall(r"\bT (duo_\w+)", out))
+    assert set(names) <= exported
+    assert exported <= set(names), f"undeclared exports: {exported - set(names)}"
+
+
+def _create(layers=2, Hkv=4, d=128, mask=None, S=4, W=16, max_len=1000, opts=None, buf=FAKE, nbytes=None):
+    if mask is None:
+        mask = np.array([[1, 0, 1, 0]] * layers, dtype=np.uint8)
+    if opts is None:
+        opts = duo._opts(batch=2, q_heads=8)
+    need = duo.duo_cache_bytes(layers, Hkv, d, mask, S, W, max_len, opts)
+    st, h = duo.duo_cache_create(layers, Hkv, d, mask, S, W, max_len, opts, buf, need if nbytes is None else nbytes)
+    return st, h, need
+
+
+def test_create_is_host_only_and_reports_lengths():
+    st, h, need = _create()
+    assert st == duo.DUO_OK and need > 0
+    for layer in range(2):
+        assert duo.duo_cache_len(h, layer) == (duo.DUO_OK, 0)
+    assert duo.duo_cache_len(h, 2)[0] == duo.DUO_ERR_INVALID
+    duo.duo_cache_destroy(h)
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(layers=0), duo.DUO_ERR_INVALID),
+    (dict(d=96), duo.DUO_ERR_INVALID),
+    (dict(W=0), duo.DUO_ERR_INVALID),
+    (dict(S=-1), duo.DUO_ERR_INVALID),
+    (dict(max_len=0), duo.DUO_ERR_INVALID),
+    (dict(opts=duo._opts(q_heads=6)), duo.DUO_ERR_INVALID),
+    (dict(opts=duo._opts(batch=0)), duo.DUO_ERR_INVALID),
+    (dict(opts=duo._opts(dtype=7)), duo.DUO_ERR_INVALID),
+    (dict(opts=duo._opts(dtype=duo.DUO_FP32, retr_fmt=duo.DUO_KV_INT4_G128)), duo.DUO_ERR_UNSUPPORTED),
+    (dict(d=64, opts=duo._opts(retr_fmt=duo.DUO_KV_INT4_G128)), duo.DUO_ERR_UNSUPPORTED),
+    (dict(buf=FAKE + 16), duo.DUO_ERR_INVALID),
+    (dict(buf=0), duo.DUO_ERR_INVALID),
+])
+def test_create_rejects(kw, status):
+    if "d" in kw and kw["d"] == 96:
+        st, h = duo.duo_cache_create(2, 4, 96, np.zeros((2, 4), np.uint8), 4, 16, 100, None, FAKE, 1 << 30)
+    else:
+        st, h, _ = _create(**kw)
+    assert st == status
+    assert not h.value
+
+
+def test_create_rejects_small_buffer_and_bad_mask():
+    st, _, need = _create()
+    st, h, _ = _create(nbytes=need - 1)
+    assert st == duo.DUO_ERR_INVALID
+    st, h, _ = _create(mask=np.array([[1, 2, 0, 0]] * 2, dtype=np.uint8))
+    assert st == duo.DUO_ERR_INVALID
+
+
+def test_calls_check_arguments_before_any_launch():
+    st, h, _ = _create(max_len=100)
+    p = FAKE  # aligned stand-in pointers: every call below must fail before touching them
+    assert duo.duo_append_kv(h, 0, p, p, 0) == duo.DUO_ERR_INVALID
+    assert duo.duo_append_kv(h, 5, p, p, 1) == duo.DUO_ERR_INVALID
+    assert duo.duo_append_kv(h, 0, p + 8, p, 1) == duo.DUO_ERR_INVALID
+    assert duo.duo_append_kv(h, 0, None, p, 1) == duo.DUO_ERR_INVALID
+    assert duo.duo_append_kv(h, 0, p, p, 101) == duo.DUO_ERR_CAPACITY
+    assert duo.duo_prefill_chunk(h, 0, p, p, p, 101, p, None) == duo.DUO_ERR_CAPACITY
+    assert duo.duo_prefill_chunk(h, 0, p, p, p, 0, p, None) == duo.DUO_ERR_INVALID
+    assert duo.duo_prefill_chunk(h, 0, p, p, p, 4, p, p + 2) == duo.DUO_ERR_INVALID
+    assert duo.duo_decode_attention(h, 0, p, p, None) == duo.DUO_ERR_INVALID  # empty layer
+    assert duo.duo_cache_len(h, 0) == (duo.DUO_OK, 0)
+    duo.duo_cache_destroy(h)
+
+
+def test_int4_prefill_is_unsupported():
+    st, h, _ = _create(opts=duo._opts(retr_fmt=duo.DUO_KV_INT4_G128))
+    assert st == duo.DUO_OK
+    assert duo.duo_prefill_chunk(h, 0, FAKE, FAKE, FAKE, 4, FAKE, None) == duo.DUO_ERR_UNSUPPORTED
+    duo.duo_cache_destroy(h)
+
+
+@pytest.mark.skipif(torch.cuda.is_available(), reason="checks the no-device failure path")
+def test_launch_without_device_fails_cleanly():
+    st, h, _ = _create(max_len=100)
+    assert duo.duo_append_kv(h, 0, FAKE, FAKE, 3) == duo.DUO_ERR_CUDA
+    assert duo.duo_cache_len(h, 0) == (duo.DUO_OK, 0)
+    duo.duo_cache_destroy(h)
+
+
+def test_kv_bytes_closed_forms():
+    """duo_kv_bytes against the oracle's (H_r L + H_s min(L, S+W)) d and 2 D H L d."""
+    mask = np.array([[1, 0, 0, 0, 1, 0, 0, 0]] * 3, dtype=np.uint8)
+    st, h, _ = _create(layers=3, Hkv=8, mask=mask, S=16, W=512, max_len=1 << 20, opts=duo._opts(batch=2))
+    for L in [1, 100, 528, 529, 32768, 1 << 20]:
+        st, r, f = duo.duo_kv_bytes(h, L)
+        assert st == duo.DUO_OK
+        assert r == 2 * 2 * 3 * 2 * oracle.layer_kv_elems(2, 6, L, 16, 512, 128)
+        assert f == 2 * 3 * oracle.full_kv_bytes(1, 8, 128, L, 2)
+    duo.duo_cache_destroy(h)
+
+
+def test_kv_bytes_int4_counts_codes_and_scales():
+    st, h, _ = _create(layers=1, Hkv=4, mask=np.array([[1, 1, 0, 0]], np.uint8), S=16, W=512, max_len=1 << 20,
+                       opts=duo._opts(retr_fmt=duo.DUO_KV_INT4_G128))
+    st, r, f = duo.duo_kv_bytes(h, 1 << 20)
+    assert r == 2 * (2 * (1 << 20) * (64 + 4) + 2 * 528 * 256)
+    duo.duo_cache_destroy(h)
+
+
+def test_slot_positions_before_any_token():
+    st, h, _ = _create()
+    for slot in range(20):
+        assert duo.duo_debug_slot_position(h, 0, 1, slot) == (duo.DUO_OK, -1)
+    assert duo.duo_debug_slot_position(h, 0, 1, 20)[0] == duo.DUO_ERR_INVALID  # S + W slots
+    assert duo.duo_debug_slot_position(h, 0, 0, 999) == (duo.DUO_OK, -1)
+    duo.duo_cache_destroy(h)
+
+
+def test_regions_are_disjoint_and_inside_the_buffer():
+    st, h, need = _create(opts=duo._opts(batch=2, q_heads=8, retr_fmt=duo.DUO_KV_INT4_G128))
+    spans = []
+    for layer in range(2):
+        for which in range(6):
+            st, ptr, nb, cap = duo.duo_debug_region(h, layer, which)
+            assert st == duo.DUO_OK and cap == 1024
+            assert FAKE <= ptr and ptr + nb <= FAKE + need and ptr % 1024 == 0
+            spans.append((ptr, ptr + nb))
+    spans.sort()
+    assert all(a[1] <= b[0] for a, b in zip(spans, spans[1:]))
+    duo.duo_cache_destroy(h)
+
+
+def test_status_strings():
+    for s in range(6):
+        assert duo.duo_status_str(s)

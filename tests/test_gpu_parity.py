@@ -1,0 +1,332 @@
+"""GPU parity: the C-ABI path (libduo.so kernels) against the fp64 oracle, element
+by element on seeded inputs, for the five workloads (reduced sizes that span
+several tiles and a ragged tail, plus sampled outputs at full size) and the
+degenerate cases of the method."""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from head_split_kv_duo_b200 import inputs
+from head_split_kv_duo_b200 import duo
+from head_split_kv_duo_b200.duo import DuoCache, DuoError
+from parity import assert_close, bits, errors, oracle_rows
+
+pytestmark = pytest.mark.gpu
+
+DEV = "cuda"
+
+
+def _seq(B, T, Hq, Hkv, d, dtype, seed):
+    q = inputs.randn((B, T, Hq, d), seed, dtype, DEV)
+    k = inputs.randn((B, T, Hkv, d), seed + 1, dtype, DEV)
+    v = inputs.randn((B, T, Hkv, d), seed + 2, dtype, DEV)
+    return q, k, v
+
+
+def _run(cache, q, k, v, chunks, decode_steps):
+    """Pre-fill the first sum(chunks) tokens in the given chunks, then decode
+    `decode_steps` tokens (append then attend).  Returns per-position outputs
+    [B][T][Hq][d] (fp32) and lse [B][T][Hq]."""
+    outs, lses = [], []
+    pos = 0
+    for n in chunks:
+        o, l = cache.prefill_chunk(0, q[:, pos:pos + n].contiguous(), k[:, pos:pos + n].contiguous(),
+                                   v[:, pos:pos + n].contiguous())
+        outs.append(o.float())
+        lses.append(l)
+        pos += n
+    for _ in range(decode_steps):
+        cache.append_kv(0, k[:, pos:pos + 1].contiguous(), v[:, pos:pos + 1].contiguous())
+        o, l = cache.decode_attention(0, q[:, pos].contiguous())
+        outs.append(o.float()[:, None])
+        lses.append(l[:, None])
+        pos += 1
+    torch.cuda.synchronize()
+    assert cache.device_status() == 0
+    return torch.cat(outs, 1).cpu().numpy(), torch.cat(lses, 1).cpu().numpy()
+
+
+# ------------------------------------------------------------ tiny hybrid MHA
+
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+@pytest.mark.parametrize("chunks", [[256], [37] * 6 + [34], [1] * 40 + [216]])
+def test_tiny_mha_prefill_then_decode(dtype, chunks):
+    """8 heads, d 64, heads {1,5} retrieval, S 4, W 16; pre-fill 256 tokens (whole,
+    in chunks of 37, token by token), then 16 decode steps."""
+    B, Hq, Hkv, d, S, W, steps = 1, 8, 8, 64, 4, 16, 16
+    mask = inputs.fixed_mask(8, (1, 5))
+    T = 256 + steps
+    q, k, v = _seq(B, T, Hq, Hkv, d, dtype, 0)
+    cache = DuoCache(1, Hkv, d, mask, S, W, T, q_heads=Hq, dtype=dtype)
+    got, got_lse = _run(cache, q, k, v, chunks, steps)
+    want, want_lse = oracle_rows(q, k, v, mask[0], S, W, 0)
+    assert_close(got, want, dtype, got_lse, want_lse, f"tiny {dtype} {chunks[:2]}")
+
+
+def test_chunking_does_not_change_results():
+    """Chunked pre-fill with any partition equals single-chunk pre-fill (reading: every
+    query row uses the Lambda mask of its own position)."""
+    B, Hq, Hkv, d, S, W = 2, 8, 4, 128, 8, 100
+    mask = torch.tensor([[0, 1, 0, 0]], dtype=torch.uint8)
+    T = 700
+    q, k, v = _seq(B, T, Hq, Hkv, d, torch.float32, 5)
+    res = []
+    for chunks in ([700], [128, 200, 1, 371], [99] * 7 + [7]):
+        cache = DuoCache(1, Hkv, d, mask, S, W, T, batch=B, q_heads=Hq, dtype=torch.float32)
+        res.append(_run(cache, q, k, v, chunks, 0))
+    for o, l in res[1:]:
+        np.testing.assert_allclose(o, res[0][0], atol=2e-6, rtol=0)
+        np.testing.assert_allclose(l, res[0][1], atol=2e-6, rtol=0)
+
+
+# ------------------------------------------------------ cache bookkeeping
+
+def _check_cache_rows(cache, k, v, T):
+    """Every retrieval row equals its input row; every streaming slot holds the input
+    row of the position the host bookkeeping reports, bit for bit; slot positions
+    match the oracle's replay."""
+    B, Hkv, d = cache.batch, cache.kv_heads, cache.head_dim
+    esize = 2 if cache.dtype == torch.bfloat16 else 4
+    mask = cache.mask[0].tolist()
+    ridx = [g for g in range(Hkv) if mask[g]]
+    sidx = [g for g in range(Hkv) if not mask[g]]
+    rk, cap = cache.region(0, duo.DUO_REGION_RETR_K)
+    rv, _ = cache.region(0, duo.DUO_REGION_RETR_V)
+    sk, _ = cache.region(0, duo.DUO_REGION_STRM_K)
+    sv, _ = cache.region(0, duo.DUO_REGION_STRM_V)
+    tdt = cache.dtype
+    kb = k.view(torch.int16) if esize == 2 else k.view(torch.int32)
+    vb = v.view(torch.int16) if esize == 2 else v.view(torch.int32)
+    idt = torch.int16 if esize == 2 else torch.int32
+    if ridx:
+        R = rk.view(idt).view(B, len(ridx), cap, d)
+        RV = rv.view(idt).view(B, len(ridx), cap, d)
+        for i, g in enumerate(ridx):
+            assert torch.equal(R[:, i, :T], kb[:, :T, g]) and torch.equal(RV[:, i, :T], vb[:, :T, g])
+    if sidx:
+        nsl = cache.S + cache.W
+        SK = sk.view(idt).view(B, len(sidx), nsl, d)
+        SV = sv.view(idt).view(B, len(sidx), nsl, d)
+        replay = oracle.ring_replay(cache.S, cache.W, [T])[0]
+        for i, g in enumerate(sidx):
+            for slot in range(nsl):
+                pos = cache.slot_position(0, g, slot)
+                assert pos == replay[slot], (slot, pos, replay[slot])
+                if pos >= 0:
+                    assert torch.equal(SK[:, i, slot], kb[:, pos, g]) and torch.equal(SV[:, i, slot], vb[:, pos, g])
+
+
+@pytest.mark.parametrize("chunks", [[5], [3, 4, 9], [1] * 23, [64, 1, 1, 70], [600]])
+@pytest.mark.parametrize("S,W", [(1, 2), (4, 16), (0, 7), (16, 64)])
+def test_cache_rows_and_slots_bit_exact(chunks, S, W):
+    B, Hkv, d = 2, 4, 64
+    mask = torch.tensor([[1, 0, 0, 1]], dtype=torch.uint8)
+    T = sum(chunks)
+    _, k, v = _seq(B, T, Hkv, Hkv, d, torch.bfloat16, 9)
+    cache = DuoCache(1, Hkv, d, mask, S, W, T + 3, batch=B, dtype=torch.bfloat16)
+    pos = 0
+    for n in chunks:
+        cache.append_kv(0, k[:, pos:pos + n].contiguous(), v[:, pos:pos + n].contiguous())
+        pos += n
+        torch.cuda.synchronize()
+        _check_cache_rows(cache, k, v, pos)
+    assert cache.len(0) == T
+
+
+def test_fig5_worked_example_on_device():
+    """'Chunked Pre-filling', Figure 5 (right): S 1, W 2, chunks of 4 -> the streaming
+    head holds {0, 2, 3} after chunk 1 and {0, 6, 7} after chunk 2."""
+    d = 64
+    mask = torch.tensor([[0]], dtype=torch.uint8)
+    q, k, v = _seq(1, 8, 1, 1, d, torch.float32, 3)
+    cache = DuoCache(1, 1, d, mask, 1, 2, 8, dtype=torch.float32)
+    held = []
+    for c in range(2):
+        sl = slice(4 * c, 4 * c + 4)
+        cache.prefill_chunk(0, q[:, sl].contiguous(), k[:, sl].contiguous(), v[:, sl].contiguous())
+        torch.cuda.synchronize()
+        held.append(sorted(p for p in (cache.slot_position(0, 0, s) for s in range(3)) if p >= 0))
+        _check_cache_rows(cache, k, v, 4 * c + 4)
+    assert held == [[0, 2, 3], [0, 6, 7]]
+
+
+# ------------------------------------------------------------- decode shapes
+
+def _fill_and_decode(Hq, Hkv, d, mask, S, W, B, ctx, steps, seed, dtype=torch.bfloat16, retr_fmt="same",
+                     rows_per_check=None):
+    T = ctx + steps
+    q = inputs.randn((B, steps, Hq, d), seed, dtype, DEV)
+    k = inputs.randn((B, T, Hkv, d), seed + 1, dtype, DEV)
+    v = inputs.randn((B, T, Hkv, d), seed + 2, dtype, DEV)
+    cache = DuoCache(1, Hkv, d, mask, S, W, T, batch=B, q_heads=Hq, dtype=dtype, retr_fmt=retr_fmt)
+    if ctx > 0:
+        cache.append_kv(0, k[:, :ctx].contiguous(), v[:, :ctx].contiguous())
+    outs, lses = [], []
+    for t in range(steps):
+        cache.append_kv(0, k[:, ctx + t:ctx + t + 1].contiguous(), v[:, ctx + t:ctx + t + 1].contiguous())
+        o, l = cache.decode_attention(0, q[:, t].contiguous())
+        outs.append(o.float()[:, None])
+        lses.append(l[:, None])
+    torch.cuda.synchronize()
+    assert cache.device_status() == 0
+    return cache, q, k, v, torch.cat(outs, 1).cpu().numpy(), torch.cat(lses, 1).cpu().numpy()
+
+
+def _decode_oracle(q, k, v, mask_row, S, W, ctx, steps):
+    """Oracle for each decode step t (query position ctx + t, history 0..ctx+t)."""
+    ws, ls = [], []
+    for t in range(steps):
+        w, l = oracle_rows(q[:, t:t + 1], k[:, :ctx + t + 1], v[:, :ctx + t + 1], mask_row, S, W, ctx + t)
+        ws.append(w)
+        ls.append(l)
+    return np.concatenate(ws, 1), np.concatenate(ls, 1)
+
+
+@pytest.mark.parametrize("B,ctx", [(1, 4095), (8, 3000), (1, 32768), (8, 32768)])
+def test_llama2_mha_decode(B, ctx):
+    """Llama-2-7B-shaped layer: 32 heads, d 128, 8 retrieval (seeded), S 16, W 512."""
+    mask = inputs.retrieval_mask(1, 32, 8, seed=0)
+    steps = 2
+    _, q, k, v, got, got_lse = _fill_and_decode(32, 32, 128, mask, 16, 512, B, ctx, steps, 10)
+    want, want_lse = _decode_oracle(q, k, v, mask[0], 16, 512, ctx, steps)
+    assert_close(got, want, torch.bfloat16, got_lse, want_lse, f"llama2 B{B} ctx{ctx}")
+
+
+@pytest.mark.parametrize("B,ctx", [(1, 5000), (4, 1 << 17), (1, 1 << 17)])
+def test_llama3_gqa_decode(B, ctx):
+    """Llama-3-8B-shaped layer: 32 q / 8 kv heads (group 4), d 128, 4 retrieval, S 16, W 512."""
+    mask = inputs.retrieval_mask(1, 8, 4, seed=1)
+    steps = 2
+    _, q, k, v, got, got_lse = _fill_and_decode(32, 8, 128, mask, 16, 512, B, ctx, steps, 20)
+    want, want_lse = _decode_oracle(q, k, v, mask[0], 16, 512, ctx, steps)
+    assert_close(got, want, torch.bfloat16, got_lse, want_lse, f"llama3 B{B} ctx{ctx}")
+
+
+@pytest.mark.parametrize("ctx", [1, 2, 15, 16, 17, 527, 528, 529, 1000])
+def test_decode_short_contexts_and_boundaries(ctx):
+    """len around S and S + W; the first query sees only itself."""
+    mask = torch.tensor([[1, 0]], dtype=torch.uint8)
+    _, q, k, v, got, got_lse = _fill_and_decode(4, 2, 128, mask, 16, 512, 2, ctx - 1, 1, 30)
+    want, want_lse = _decode_oracle(q, k, v, mask[0], 16, 512, ctx - 1, 1)
+    assert_close(got, want, torch.bfloat16, got_lse, want_lse, f"ctx {ctx}")
+
+
+@pytest.mark.parametrize("S,W,mask", [(0, 1, [0, 0]), (0, 64, [0, 0]), (3, 1, [0, 1]), (0, 5, [1, 1]),
+                                      (700, 9, [0, 0]), (2, 3000, [0, 0])])
+def test_degenerate_settings(S, W, mask):
+    """S = 0 (pure sliding window), W = 1 (only the current token), all-retrieval,
+    all-streaming, S or W beyond the sequence."""
+    m = torch.tensor([mask], dtype=torch.uint8)
+    for dtype in (torch.bfloat16, torch.float32):
+        T = 1200
+        q, k, v = _seq(1, T, 4, 2, 64, dtype, 40)
+        cache = DuoCache(1, 2, 64, m, S, W, T, q_heads=4, dtype=dtype)
+        got, got_lse = _run(cache, q, k, v, [500, 300, 390], 10)
+        want, want_lse = oracle_rows(q, k, v, m[0], S, W, 0)
+        assert_close(got, want, dtype, got_lse, want_lse, f"S{S} W{W} {mask} {dtype}")
+
+
+def test_capacity_is_enforced_on_device():
+    mask = torch.tensor([[1, 0]], dtype=torch.uint8)
+    q, k, v = _seq(1, 10, 2, 2, 64, torch.bfloat16, 50)
+    cache = DuoCache(1, 2, 64, mask, 2, 4, 8, dtype=torch.bfloat16, q_heads=2)
+    cache.append_kv(0, k[:, :8].contiguous(), v[:, :8].contiguous())
+    with pytest.raises(DuoError) as e:
+        cache.append_kv(0, k[:, 8:9].contiguous(), v[:, 8:9].contiguous())
+    assert e.value.status == duo.DUO_ERR_CAPACITY and cache.len(0) == 8
+    o, _ = cache.decode_attention(0, q[:, 7].contiguous())  # still usable at capacity
+    want, _ = oracle_rows(q[:, 7:8], k[:, :8], v[:, :8], mask[0], 2, 4, 7)
+    assert_close(o.float().cpu().numpy()[:, None], want, torch.bfloat16)
+
+
+# ------------------------------------------------------ planted needle, masks
+
+def _planted(ctx, d=128, seed=60):
+    """GQA 8 q / 2 kv heads (kv 0 retrieval, kv 1 streaming), S 16, W 512: keys at a
+    middle position and at the window / sink boundaries planted to dominate."""
+    Hq, Hkv, S, W = 8, 2, 16, 512
+    mask = torch.tensor([[1, 0]], dtype=torch.uint8)
+    g = torch.Generator(device="cpu").manual_seed(seed)
+    q = torch.randn(1, 1, Hq, d, generator=g)
+    k = torch.randn(1, ctx, Hkv, d, generator=g)
+    v = torch.randn(1, ctx, Hkv, d, generator=g)
+    i = ctx - 1
+    needles = {"middle": ctx // 2, "window_edge": i - W + 1, "outside": i - W, "sink_edge": S - 1, "post_sink": S}
+    values = {"middle": 3.0, "window_edge": 7.0, "outside": 11.0, "sink_edge": 17.0, "post_sink": 23.0}
+    for name, j in needles.items():
+        for kv in range(Hkv):
+            qq = q[0, 0, kv * 4]
+            k[0, j, kv] = 6.0 * qq / qq.norm() * math.sqrt(d) * (1.05 if name == "outside" else 1.0)
+            v[0, j, kv] = values[name]
+    return [t.to(torch.bfloat16).to(DEV) for t in (q, k, v)], mask, needles, S, W
+
+
+def test_planted_needle_and_mask_discrimination():
+    ctx = 9000
+    (q, k, v), mask, needles, S, W = _planted(ctx)
+    cache = DuoCache(1, 2, 128, mask, S, W, ctx, q_heads=8, dtype=torch.bfloat16)
+    cache.append_kv(0, k.contiguous(), v.contiguous())
+    o, lse = cache.decode_attention(0, q[:, 0].contiguous())
+    torch.cuda.synchronize()
+    got = o.float().cpu().numpy()[:, None]
+    want, want_lse = oracle_rows(q, k, v, mask[0], S, W, ctx - 1)
+    assert_close(got, want, torch.bfloat16, lse.cpu().numpy()[:, None], want_lse, "planted")
+    # retrieval query head 0 recovers the strongest needle (value 11, outside the
+    # window); streaming query head 4 sees only the window-edge and sink needles
+    # (values 7 and 17, equal logits) and nothing of the middle or outside ones
+    assert abs(got[0, 0, 0].mean() - 11.0) < 1.0
+    assert abs(got[0, 0, 4].mean() - 12.0) < 1.0
+    # each wrong reading of the mask moves the answer by far more than the tolerance
+    for wrong in [dict(W=W + 1), dict(W=W - 1), dict(S=S + 1), dict(S=S - 1), dict(mask=[1, 1]), dict(mask=[0, 0])]:
+        m = wrong.get("mask", mask[0].tolist())
+        w2, _ = oracle_rows(q, k, v, m, wrong.get("S", S), wrong.get("W", W), ctx - 1)
+        assert np.abs(w2 - got).max() > 0.2, f"reading {wrong} is not distinguishable"
+
+
+# ------------------------------------------------------------------- INT4
+
+def _int4_reference(k_rows):
+    """oracle quantisation of bf16 rows [..., 128] -> codes, scale bits, zero bits, dequantised fp64."""
+    b = bits(k_rows).reshape(-1, 128)
+    codes, sb, zb = oracle.int4_quantize(b)
+    return codes, sb, zb, oracle.int4_dequantize(codes, sb, zb)
+
+
+@pytest.mark.parametrize("B,ctx", [(1, 3000), (2, 20000)])
+def test_int4_codes_bit_exact_and_decode(B, ctx):
+    Hq, Hkv, d, S, W = 32, 8, 128, 16, 512
+    mask = inputs.retrieval_mask(1, 8, 4, seed=2)
+    steps = 2
+    cache, q, k, v, got, got_lse = _fill_and_decode(Hq, Hkv, d, mask, S, W, B, ctx, steps, 70, retr_fmt="int4")
+    T = ctx + steps
+    ridx = [g for g in range(Hkv) if mask[0, g]]
+    rk, cap = cache.region(0, duo.DUO_REGION_RETR_K)
+    rv, _ = cache.region(0, duo.DUO_REGION_RETR_V)
+    ks, _ = cache.region(0, duo.DUO_REGION_RETR_KSZ)
+    vs, _ = cache.region(0, duo.DUO_REGION_RETR_VSZ)
+    RK = rk.view(B, len(ridx), cap, 64)[:, :, :T].cpu().numpy()
+    RV = rv.view(B, len(ridx), cap, 64)[:, :, :T].cpu().numpy()
+    KS = ks.view(torch.int16).view(B, len(ridx), cap, 2)[:, :, :T].cpu().numpy().view(np.uint16)
+    VS = vs.view(torch.int16).view(B, len(ridx), cap, 2)[:, :, :T].cpu().numpy().view(np.uint16)
+    # the oracle's own quantisation, dequantised in fp64, stands in for the retrieval rows
+    kq = k.float().cpu().numpy().astype(np.float64)
+    vq = v.float().cpu().numpy().astype(np.float64)
+    for i, g in enumerate(ridx):
+        for src, C, Z, dst in ((k, RK, KS, kq), (v, RV, VS, vq)):
+            codes, sb, zb, deq = _int4_reference(src[:, :, g])
+            assert np.array_equal(C[:, i].reshape(-1, 64), codes), "INT4 codes differ"
+            assert np.array_equal(Z[:, i, :, 0].reshape(-1), sb) and np.array_equal(Z[:, i, :, 1].reshape(-1), zb)
+            dst[:, :, g] = deq.reshape(B, T, 128)
+    ws, ls = [], []
+    for t in range(steps):
+        w, l = oracle.attend(bits(q[:, t:t + 1]), kq[:, :ctx + t + 1], vq[:, :ctx + t + 1], mask[0].numpy().astype(bool),
+                             S, W, pos0=ctx + t)
+        ws.append(w)
+        ls.append(l)
+    assert_close(got, np.concatenate(ws, 1), torch.bfloat16, got_lse, np.concatenate(ls, 1), "int4 decode")
+    # for information: distance to attention over the unquantised bf16 values
+    ref, _ = _decode_oracle(q, k, v, mask[0], S, W, ctx, steps)
+    print("int4 vs unquantised:", errors(got, ref))
