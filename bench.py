@@ -272,24 +272,25 @@ def run_ours(args, rank, world, dist):
 
 
 def run_prefill(args, dev, tc_peak, tc_sust, peak_src):
+    L, C = args.prefill_len, args.prefill_chunk
     import torch
 
     from head_split_kv_duo_b200 import inputs
     from head_split_kv_duo_b200.duo import DuoCache
 
     mask = inputs.retrieval_mask(1, HKV, NRET, seed=1)
-    k = inputs.randn((1, PREFILL_LEN, HKV, D), 200, device=dev)
-    v = inputs.randn((1, PREFILL_LEN, HKV, D), 201, device=dev)
-    q = inputs.randn((1, PREFILL_CHUNK, HQ, D), 202, device=dev)  # same queries for every chunk
+    k = inputs.randn((1, L, HKV, D), 200, device=dev)
+    v = inputs.randn((1, L, HKV, D), 201, device=dev)
+    q = inputs.randn((1, C, HQ, D), 202, device=dev)  # same queries for every chunk
     out = torch.empty_like(q)
-    nchunks = PREFILL_LEN // PREFILL_CHUNK
+    nchunks = L // C
     stream = torch.cuda.current_stream()
 
     def one():
-        cache = DuoCache(1, HKV, D, mask, S, W, PREFILL_LEN, q_heads=HQ, dtype=torch.bfloat16, device=dev)
+        cache = DuoCache(1, HKV, D, mask, S, W, L, q_heads=HQ, dtype=torch.bfloat16, device=dev)
         evs = []
         for c in range(nchunks):
-            sl = slice(c * PREFILL_CHUNK, (c + 1) * PREFILL_CHUNK)
+            sl = slice(c * C, (c + 1) * C)
             a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
             a.record(stream)
             cache.prefill_chunk(0, q, k[:, sl], v[:, sl], out=out, want_lse=False, stream=stream)
@@ -304,9 +305,10 @@ def run_prefill(args, dev, tc_peak, tc_sust, peak_src):
         one()
     times = [one() for _ in range(args.prefill_steps)]
     ms = statistics.mean(times)
-    fl = prefill_flops()
+    fl = prefill_flops(L)
     tflops = fl / (ms * 1e-3) / 1e12
-    return {"workload": "llama3-8b-gqa-prefill-256k-chunk32k", "tflops": round(tflops, 1), "ms": round(ms, 2),
+    name = f"llama3-8b-gqa-prefill-{L // 1024}k-chunk{C // 1024}k"
+    return {"workload": name, "tflops": round(tflops, 1), "ms": round(ms, 2),
             "steps": args.prefill_steps, "algorithmic_tflop": round(fl / 1e12, 2),
             "roofline": {"bound": "tensor", "achieved": round(tflops, 1), "peak": tc_peak,
                          "peak_source": f"{peak_src} bf16_tflops (burst)", "unit": "TFLOP/s",
@@ -350,6 +352,9 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--skip-prefill", action="store_true")
+    ap.add_argument("--skip-decode", action="store_true", help="time only the pre-fill workload")
+    ap.add_argument("--prefill-len", type=int, default=PREFILL_LEN)
+    ap.add_argument("--prefill-chunk", type=int, default=PREFILL_CHUNK)
     ap.add_argument("--skip-e2e", action="store_true")
     ap.add_argument("--skip-cpu-baseline", action="store_true")
     ap.add_argument("--prefill-steps", type=int, default=2)
@@ -386,6 +391,14 @@ def main():
         import torch.distributed as tdist
         tdist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
         dist = tdist
+    if args.skip_decode:
+        import torch
+        dev = torch.device("cuda", int(os.environ.get("LOCAL_RANK", 0)))
+        torch.cuda.set_device(dev)
+        _, tc_peak, tc_sust, src = peaks()
+        if rank == 0:
+            print(json.dumps({"prefill": run_prefill(args, dev, tc_peak, tc_sust, src)}))
+        return 0
     res = run_ours(args, rank, world, dist)
     if rank == 0 and not args.skip_cpu_baseline:
         res["cpu_baseline"] = oracle_sample(args)

@@ -1,10 +1,557 @@
-// k_prefill_tc.cu -- tcgen05 / TMEM pre-fill attention (bf16, head_dim 128).
+// k_prefill_tc.cu -- chunked pre-fill attention on the 5th-generation tensor cores
+// (tcgen05 + TMEM), bf16 in, fp32 accumulate, head_dim 128.
+//
+// Operation ("Chunked Pre-filling", masks of "The Full and Streaming Attention
+// Masks"): the n chunk queries at positions len .. len+n-1 attend to
+//   * retrieval heads: every key 0 .. i (causal), read from the full cache, into
+//     which the chunk has already been appended;
+//   * streaming heads: the staged history (sinks, then positions wstart..len-1) and
+//     the chunk's own keys, with the Lambda mask j < S or i - j < W.  Key tiles that
+//     hold no visible key for any row of a query tile are never loaded (tile skip).
+//
+// One CTA = one 128-row query tile of one (batch, query head); 6 warps:
+//   warp 0      TMA producer: Q once, then K/V tiles of 128 keys into a 2-stage ring
+//   warp 1      TMEM allocator; lane 0 issues every tcgen05.mma
+//   warps 2..5  softmax warpgroup: thread t owns query row t (TMEM lane t)
+// TMEM (512 columns): S double buffer at columns 0 and 128, O tile at 256.
+//   S_j = Q K_j^T      (M 128, N 128, K 128: 8 MMAs of K 16), into S[j % 2]
+//   O_j = P_j V_j      (M 128, N 128, K 128 keys), P_j from shared memory
+// The softmax warps read S_j twice from TMEM (row max, then probabilities), write
+// P_j (bf16) to shared memory in the 128B-swizzled K-major layout, and fold each
+// O_j into fp32 registers with the online-softmax rescale.  The tensor core computes
+// S_{j+1} while the softmax warps work on tile j.
+//
+// Every mbarrier wait is bounded; a wait that runs out latches kDevTimeout in the
+// status word and sets an abort flag so that every role drains and exits.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
 #include "device_common.cuh"
 
 namespace duo {
 
-bool prefill_tc_supported(const PrefillParams &, duo_dtype) { return false; }
+namespace {
 
-cudaError_t launch_prefill_tc(const PrefillParams &, cudaStream_t) { return cudaErrorNotSupported; }
+constexpr int kTcThreads = 192;
+constexpr int kBM = 128;  // query rows per tile
+constexpr int kBN = 128;  // keys per tile
+constexpr int kD = 128;
+constexpr int kKvStages = 2;
+constexpr int kMaxStrmTiles = 48;
+
+// shared memory map (bytes from the 1 KiB-aligned base)
+constexpr int kSmQ = 0;                    // 2 x [128][64] bf16, 128B swizzle
+constexpr int kSmKV = 32768;               // stage s: K at +s*65536, V at +s*65536+32768
+constexpr int kSmP = kSmKV + kKvStages * 65536;  // 2 x [128][64] bf16
+constexpr int kSmBar = kSmP + 32768;
+constexpr int kSmMisc = kSmBar + 256;
+constexpr int kSmTotal = kSmMisc + 1024 + kMaxStrmTiles * 16;
+constexpr int kSmemAlloc = kSmTotal + 1024;  // slack for aligning the base to 1 KiB
+
+// barrier indices (8 bytes each)
+constexpr int kBarQ = 0, kBarKvFull = 1, kBarKvEmpty = 3, kBarSFull = 5, kBarSFree = 7, kBarPFull = 9, kBarOFull = 10,
+              kBarDrain = 11, kNumBars = 12;
+
+struct TileDesc {
+  int src;      // 0 retrieval cache, 1 streaming history, 2 chunk input
+  int y;        // first row in the source
+};
+
+struct TcArgs {
+  PrefillParams p;
+  CUtensorMap tm_q, tm_kc, tm_vc, tm_kh, tm_vh, tm_kn, tm_vn;
+};
+
+// ---------------------------------------------------------------- PTX wrappers
+
+__device__ __forceinline__ void tma_3d(uint32_t dst, const CUtensorMap *m, int x, int y, int z, uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4}], [%5];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(m)), "r"(x), "r"(y), "r"(z), "r"(bar)
+      : "memory");
+}
+__device__ __forceinline__ void tma_4d(uint32_t dst, const CUtensorMap *m, int x, int y, int z, int w, uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.4d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4, %5}], [%6];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(m)), "r"(x), "r"(y), "r"(z), "r"(w), "r"(bar)
+      : "memory");
+}
+__device__ __forceinline__ void prefetch_map(const CUtensorMap *m) {
+  asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(m)) : "memory");
+}
+
+__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void fence_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
+
+__device__ __forceinline__ void tc_commit(uint32_t bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar) : "memory");
+}
+
+__device__ __forceinline__ void tc_mma(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc, uint32_t acc) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(acc)
+      : "memory");
+}
+
+// 32 consecutive fp32 columns of this thread's TMEM lane
+__device__ __forceinline__ void tc_ld32(uint32_t taddr, float (&v)[32]) {
+  uint32_t r[32];
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+      "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, "
+      "%16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]), "=r"(r[8]),
+        "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]), "=r"(r[16]),
+        "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]),
+        "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+      : "r"(taddr));
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+  for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+// Shared-memory matrix descriptor, 128-byte swizzle (sm_100 layout: start >> 4 at
+// bit 0, leading byte offset >> 4 at bit 16, stride byte offset >> 4 at bit 32,
+// version 1 at bit 46, swizzle mode 2 at bit 61).
+__device__ __forceinline__ uint64_t sdesc(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
+  return static_cast<uint64_t>((saddr >> 4) & 0x3FFFu) | (static_cast<uint64_t>((lbo >> 4) & 0x3FFFu) << 16) |
+         (static_cast<uint64_t>((sbo >> 4) & 0x3FFFu) << 32) | (1ull << 46) | (2ull << 61);
+}
+
+// Instruction descriptor of kind::f16: fp32 accumulator, bf16 A and B, M 128, N 128.
+constexpr uint32_t idesc_bf16(bool b_mn_major) {
+  return (1u << 4) | (1u << 7) | (1u << 10) | ((b_mn_major ? 1u : 0u) << 16) | ((128u >> 3) << 17) | ((128u >> 4) << 24);
+}
+
+// Bounded wait that also gives up at once after another role aborted.
+__device__ __forceinline__ bool wait_bar(uint32_t bar, uint32_t parity, uint32_t *status, volatile int *abort_flag) {
+#pragma unroll 1
+  for (int i = 0; i < 64; ++i)
+    if (mbar_try_wait(bar, parity)) return true;
+  const unsigned long long t0 = globaltimer();
+#pragma unroll 1
+  while (true) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if (*abort_flag) return false;
+    if (globaltimer() - t0 > kWaitLimitNs) {
+      flag_status(status, kDevTimeout);
+      *abort_flag = 1;
+      return false;
+    }
+  }
+}
+
+// ---------------------------------------------------------------- tile lists
+
+struct Plan {
+  bool retr;
+  int nt;          // key tiles to visit
+  int64_t q0;      // absolute position of query row 0 of this tile
+  int kvrow;       // retrieval: z index of the head in the cache map / streaming: in the hist map
+};
+
+// Streaming heads: which history / chunk tiles hold a visible key for some row of
+// the query tile.  Writes the list into `tl` and returns its length.
+__device__ int streaming_tiles(const PrefillParams &p, int r0, TileDesc *tl) {
+  int nt = 0;
+  const int64_t qlo = p.len + r0;                                      // smallest query position
+  const int rows_hi = (r0 + kBM < p.n) ? r0 + kBM : p.n;                // chunk rows this tile needs
+  const int hrows = p.hs + p.hw;
+  const int nh = (hrows + kBN - 1) / kBN;
+  for (int t = 0; t < nh && nt < kMaxStrmTiles; ++t) {
+    const int a = t * kBN, b = ((t + 1) * kBN < hrows ? (t + 1) * kBN : hrows) - 1;
+    const bool sinks = a < p.hs;
+    const int64_t maxpos = b < p.hs ? b : p.wstart + (b - p.hs);
+    // the smallest query position reaches furthest back: pos > qlo - W
+    const bool recent = maxpos > qlo - p.W;
+    if (sinks || recent) tl[nt++] = {1, a};
+  }
+  const int nc = (rows_hi + kBN - 1) / kBN;
+  int c0 = r0 - p.W + 1;
+  c0 = c0 < 0 ? 0 : c0 / kBN;
+  // chunk tiles holding sinks (positions < S) that lie before the window tiles
+  const int sink_rows = p.len < p.S ? static_cast<int>(p.S - p.len) : 0;
+  const int ns = (sink_rows + kBN - 1) / kBN;
+  for (int t = 0; t < ns && t < c0 && t < nc && nt < kMaxStrmTiles; ++t) tl[nt++] = {2, t * kBN};
+  for (int t = c0; t < nc && nt < kMaxStrmTiles; ++t) tl[nt++] = {2, t * kBN};
+  return nt;
+}
+
+__device__ __forceinline__ TileDesc tile_of(const Plan &pl, const TileDesc *tl, int j) {
+  if (pl.retr) return {0, j * kBN};
+  return tl[j];
+}
+
+// ---------------------------------------------------------------- the kernel
+
+__global__ void __launch_bounds__(kTcThreads, 1) prefill_tc_kernel(const __grid_constant__ TcArgs a) {
+  const PrefillParams &p = a.p;
+  extern __shared__ char smem_raw[];
+  char *smem = reinterpret_cast<char *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const uint32_t sbase = smem_u32(smem);
+  const uint32_t bar0 = sbase + kSmBar;
+  auto bar = [&](int i) { return bar0 + 8u * i; };
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + kSmMisc);
+  volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + kSmMisc + 4);
+  int *ntiles_sm = reinterpret_cast<int *>(smem + kSmMisc + 8);
+  TileDesc *tl = reinterpret_cast<TileDesc *>(smem + kSmMisc + 1024);
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+
+  // ---- which query tile ----
+  const int ntq = (p.n + kBM - 1) / kBM;
+  const int bh = blockIdx.x % (p.B * p.Hq);
+  const int qt = ntq - 1 - blockIdx.x / (p.B * p.Hq);  // heaviest (latest) tiles first
+  const int b = bh / p.Hq, h = bh % p.Hq;
+  const int g = h / p.G;
+  const int r0 = qt * kBM;
+  Plan pl;
+  pl.retr = p.hm.is_retr[g] != 0;
+  pl.q0 = p.len + r0;
+  pl.kvrow = b * (pl.retr ? p.Hr : p.HsMax) + p.hm.kind_idx[g];
+
+  if (tid == 0) {
+    for (int i = 0; i < kNumBars; ++i) mbar_init(bar(i), (i == kBarSFree || i == kBarSFree + 1 || i == kBarPFull) ? 128 : 1);
+    fence_mbar_init();
+    *abort_flag = 0;
+    int nt;
+    if (pl.retr) {
+      const int64_t last = pl.q0 + ((r0 + kBM < p.n) ? kBM : p.n - r0) - 1;  // last key position needed
+      nt = static_cast<int>(last / kBN) + 1;
+    } else {
+      nt = streaming_tiles(p, r0, tl);
+    }
+    *ntiles_sm = nt;
+  }
+  if (warp == 1) {  // TMEM: 512 columns
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_slot)),
+                 "r"(512));
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const int nt = *ntiles_sm;
+
+  if (warp == 0) {
+    // ================= TMA producer =================
+    if (lane == 0) {
+      prefetch_map(&a.tm_q);
+      const CUtensorMap *mk = pl.retr ? &a.tm_kc : &a.tm_kh;
+      prefetch_map(mk);
+      mbar_expect_tx(bar(kBarQ), 32768);
+      tma_4d(sbase + kSmQ, &a.tm_q, 0, h, r0, b, bar(kBarQ));
+      tma_4d(sbase + kSmQ + 16384, &a.tm_q, 64, h, r0, b, bar(kBarQ));
+      for (int j = 0; j < nt; ++j) {
+        const int s = j % kKvStages;
+        if (j >= kKvStages && !wait_bar(bar(kBarKvEmpty + s), ((j / kKvStages) - 1) & 1, p.status, abort_flag)) break;
+        const TileDesc t = tile_of(pl, tl, j);
+        const uint32_t kd = sbase + kSmKV + s * 65536, vd = kd + 32768;
+        mbar_expect_tx(bar(kBarKvFull + s), 65536);
+        if (t.src == 0) {
+          tma_3d(kd, &a.tm_kc, 0, t.y, pl.kvrow, bar(kBarKvFull + s));
+          tma_3d(kd + 16384, &a.tm_kc, 64, t.y, pl.kvrow, bar(kBarKvFull + s));
+          tma_3d(vd, &a.tm_vc, 0, t.y, pl.kvrow, bar(kBarKvFull + s));
+          tma_3d(vd + 16384, &a.tm_vc, 64, t.y, pl.kvrow, bar(kBarKvFull + s));
+        } else if (t.src == 1) {
+          tma_3d(kd, &a.tm_kh, 0, t.y, pl.kvrow, bar(kBarKvFull + s));
+          tma_3d(kd + 16384, &a.tm_kh, 64, t.y, pl.kvrow, bar(kBarKvFull + s));
+          tma_3d(vd, &a.tm_vh, 0, t.y, pl.kvrow, bar(kBarKvFull + s));
+          tma_3d(vd + 16384, &a.tm_vh, 64, t.y, pl.kvrow, bar(kBarKvFull + s));
+        } else {
+          tma_4d(kd, &a.tm_kn, 0, g, t.y, b, bar(kBarKvFull + s));
+          tma_4d(kd + 16384, &a.tm_kn, 64, g, t.y, b, bar(kBarKvFull + s));
+          tma_4d(vd, &a.tm_vn, 0, g, t.y, b, bar(kBarKvFull + s));
+          tma_4d(vd + 16384, &a.tm_vn, 64, g, t.y, b, bar(kBarKvFull + s));
+        }
+      }
+    }
+  } else if (warp == 1) {
+    // ================= MMA issuer =================
+    if (lane == 0) {
+      constexpr uint32_t kIdS = idesc_bf16(false);
+      constexpr uint32_t kIdPV = idesc_bf16(true);
+      bool ok = wait_bar(bar(kBarQ), 0, p.status, abort_flag);
+      auto issue_pv = [&](int jj) {
+        // O = P_jj V_jj : K = 128 keys in 8 steps of 16; V is N-major (d contiguous)
+        const int s = jj % kKvStages;
+        const uint32_t vbase = sbase + kSmKV + s * 65536 + 32768;
+        for (int kk = 0; kk < 8; ++kk) {
+          const uint64_t ad = sdesc(sbase + kSmP + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024);
+          const uint64_t bd = sdesc(vbase + kk * 2048, 16384, 1024);
+          tc_mma(tmem + 256, ad, bd, kIdPV, kk > 0 ? 1u : 0u);
+        }
+        tc_commit(bar(kBarOFull));
+        tc_commit(bar(kBarKvEmpty + s));
+      };
+      for (int j = 0; j < nt && ok; ++j) {
+        const int s = j % kKvStages;
+        if (!wait_bar(bar(kBarKvFull + s), (j / kKvStages) & 1, p.status, abort_flag)) { ok = false; break; }
+        if (j >= 2 && !wait_bar(bar(kBarSFree + (j & 1)), ((j - 2) >> 1) & 1, p.status, abort_flag)) { ok = false; break; }
+        tc_fence_after();
+        // S_j = Q K_j^T : K = d 128 in 8 steps of 16; Q and K are K-major
+        const uint32_t kbase = sbase + kSmKV + s * 65536;
+        for (int kk = 0; kk < 8; ++kk) {
+          const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
+          tc_mma(tmem + (j & 1) * 128, sdesc(sbase + kSmQ + off, 16, 1024), sdesc(kbase + off, 16, 1024), kIdS,
+                 kk > 0 ? 1u : 0u);
+        }
+        tc_commit(bar(kBarSFull + (j & 1)));
+        if (j >= 1) {
+          if (!wait_bar(bar(kBarPFull), (j - 1) & 1, p.status, abort_flag)) { ok = false; break; }
+          tc_fence_after();
+          issue_pv(j - 1);
+        }
+      }
+      if (ok && nt > 0 && wait_bar(bar(kBarPFull), (nt - 1) & 1, p.status, abort_flag)) {
+        tc_fence_after();
+        issue_pv(nt - 1);
+      }
+      // drain: every MMA this thread issued has completed before TMEM is freed
+      tc_commit(bar(kBarDrain));
+      mbar_wait(bar(kBarDrain), 0, p.status);
+    }
+  } else {
+    // ================= softmax warpgroup =================
+    const int row = ((warp & 3) << 5) | lane;             // TMEM lane == query row of the tile
+    const uint32_t lane_base = tmem + (static_cast<uint32_t>((warp & 3) << 5) << 16);
+    const int64_t i = pl.q0 + row;                         // absolute query position
+    const float c = p.scale_log2;
+    float o[kD];
+#pragma unroll
+    for (int e = 0; e < kD; ++e) o[e] = 0.f;
+    float m = -INFINITY, l = 0.f, alpha_prev = 1.f;
+    char *prow = smem + kSmP + row * 128;
+    const int rsw = row & 7;
+    bool ok = true;
+
+    for (int j = 0; j < nt; ++j) {
+      const TileDesc t = tile_of(pl, tl, j);
+      // positions of the 128 keys of this tile, and whether the whole tile is visible
+      int64_t pos0;
+      bool full_vis;
+      int valid_rows = kBN;
+      if (t.src == 0) {
+        pos0 = t.y;
+        full_vis = pos0 + kBN - 1 <= pl.q0;  // below the diagonal for every row
+      } else if (t.src == 2) {
+        pos0 = p.len + t.y;
+        valid_rows = p.n - t.y;
+        full_vis = false;
+      } else {
+        pos0 = -1;  // history: positions are not contiguous
+        valid_rows = p.hs + p.hw - t.y;
+        full_vis = false;
+      }
+      auto key_pos = [&](int col) -> int64_t {
+        if (pos0 >= 0) return pos0 + col;
+        const int r = t.y + col;
+        return r < p.hs ? r : p.wstart + (r - p.hs);
+      };
+      auto visible = [&](int col) -> bool {
+        if (col >= valid_rows) return false;
+        const int64_t kp = key_pos(col);
+        if (kp > i) return false;
+        if (pl.retr) return true;
+        return kp < p.S || i - kp < p.W;
+      };
+
+      if (ok) ok = wait_bar(bar(kBarSFull + (j & 1)), (j >> 1) & 1, p.status, abort_flag);
+      tc_fence_after();
+      const uint32_t sbuf = lane_base + (j & 1) * 128;
+      // pass 1: row max of the visible logits
+      float mx = -INFINITY;
+#pragma unroll
+      for (int cc = 0; cc < 4; ++cc) {
+        float v[32];
+        tc_ld32(sbuf + cc * 32, v);
+#pragma unroll
+        for (int e = 0; e < 32; ++e) {
+          const bool vis = full_vis || visible(cc * 32 + e);
+          mx = vis ? fmaxf(mx, v[e]) : mx;
+        }
+      }
+      const float m_new = fmaxf(m, mx * c);
+      const bool none = (m_new == -INFINITY);
+      const float alpha = none ? 1.f : ex2(m - m_new);
+
+      // fold O_{j-1} into the register accumulator (P_{j-1} in shared memory is free after)
+      if (j >= 1) {
+        if (ok) ok = wait_bar(bar(kBarOFull), (j - 1) & 1, p.status, abort_flag);
+        tc_fence_after();
+#pragma unroll
+        for (int cc = 0; cc < 4; ++cc) {
+          float v[32];
+          tc_ld32(lane_base + 256 + cc * 32, v);
+#pragma unroll
+          for (int e = 0; e < 32; ++e) o[cc * 32 + e] = fmaf(o[cc * 32 + e], alpha_prev, v[e]);
+        }
+      }
+      // pass 2: probabilities, row sum, bf16 P into the swizzled K-major tile
+      float rs = 0.f;
+      const float mc = none ? 0.f : m_new;
+#pragma unroll
+      for (int cc = 0; cc < 4; ++cc) {
+        float v[32];
+        tc_ld32(sbuf + cc * 32, v);
+        uint32_t pk[16];
+#pragma unroll
+        for (int e = 0; e < 32; e += 2) {
+          const bool v0 = full_vis || visible(cc * 32 + e);
+          const bool v1 = full_vis || visible(cc * 32 + e + 1);
+          const float p0 = v0 ? ex2(fmaf(v[e], c, -mc)) : 0.f;
+          const float p1 = v1 ? ex2(fmaf(v[e + 1], c, -mc)) : 0.f;
+          rs += p0 + p1;
+          const __nv_bfloat162 pb = __floats2bfloat162_rn(p0, p1);
+          pk[e >> 1] = *reinterpret_cast<const uint32_t *>(&pb);
+        }
+        // columns cc*32 .. cc*32+31 -> half (cc >> 1), 16-byte chunks 4*(cc&1) .. +3
+        char *half = prow + (cc >> 1) * 16384;
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const int chunk = ((cc & 1) * 4 + q) ^ rsw;
+          *reinterpret_cast<uint4 *>(half + chunk * 16) = make_uint4(pk[4 * q], pk[4 * q + 1], pk[4 * q + 2], pk[4 * q + 3]);
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(bar(kBarSFree + (j & 1)));  // S buffer j % 2 may be overwritten
+      l = fmaf(l, alpha, rs);
+      m = m_new;
+      alpha_prev = alpha;
+      fence_async_smem();  // P visible to the tensor core
+      tc_fence_before();
+      mbar_arrive(bar(kBarPFull));
+    }
+    // last O tile
+    if (nt > 0) {
+      if (ok) ok = wait_bar(bar(kBarOFull), (nt - 1) & 1, p.status, abort_flag);
+      tc_fence_after();
+#pragma unroll
+      for (int cc = 0; cc < 4; ++cc) {
+        float v[32];
+        tc_ld32(lane_base + 256 + cc * 32, v);
+#pragma unroll
+        for (int e = 0; e < 32; ++e) o[cc * 32 + e] = fmaf(o[cc * 32 + e], alpha_prev, v[e]);
+      }
+    }
+    // epilogue: normalise and store the row (bf16) and its lse
+    if (r0 + row < p.n) {
+      const float inv = 1.f / l;
+      char *orow = p.out + ((static_cast<int64_t>(b) * p.n + r0 + row) * p.Hq + h) * (kD * 2);
+#pragma unroll
+      for (int q = 0; q < kD / 8; ++q) {
+        uint32_t w[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const __nv_bfloat162 pb = __floats2bfloat162_rn(o[8 * q + 2 * e] * inv, o[8 * q + 2 * e + 1] * inv);
+          w[e] = *reinterpret_cast<const uint32_t *>(&pb);
+        }
+        *reinterpret_cast<uint4 *>(orow + q * 16) = make_uint4(w[0], w[1], w[2], w[3]);
+      }
+      if (p.lse) p.lse[(static_cast<int64_t>(b) * p.n + r0 + row) * p.Hq + h] = (m + lg2(l)) * kLn2;
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 1) asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(512));
+}
+
+// ---------------------------------------------------------------- host side
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static bool tried = false;
+  if (!tried) {
+    tried = true;
+    void *ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+  }
+  return fn;
+}
+
+// bf16 map of `rank` dims (innermost first), box {64, ...}, 128-byte swizzle.
+bool make_map(CUtensorMap *m, const void *base, int rank, const uint64_t *dims, const uint64_t *strides_bytes,
+              const uint32_t *box) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t gd[5], gs[4];
+  cuuint32_t bx[5], es[5];
+  for (int r = 0; r < rank; ++r) {
+    gd[r] = dims[r];
+    bx[r] = box[r];
+    es[r] = 1;
+  }
+  for (int r = 0; r < rank - 1; ++r) gs[r] = strides_bytes[r];
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, rank, const_cast<void *>(base), gd, gs, bx, es,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+}  // namespace
+
+bool prefill_tc_supported(const PrefillParams &p, duo_dtype dt) {
+  if (dt != DUO_BF16 || p.D != kD) return false;
+  if (encode_fn() == nullptr) return false;
+  // streaming tile list must fit: history tiles + window tiles + a sink tile
+  const int hist_tiles = (p.hs + p.hw + kBN - 1) / kBN;
+  const int win_tiles = (p.W + 2 * kBN - 2) / kBN + 1;
+  const int sink_tiles = (p.S + kBN - 1) / kBN;
+  return hist_tiles + win_tiles + sink_tiles <= kMaxStrmTiles;
+}
+
+cudaError_t launch_prefill_tc(const PrefillParams &p, cudaStream_t st) {
+  static TcArgs a;  // host staging only; copied into the launch's parameter buffer
+  a.p = p;
+  const uint64_t row = kD * 2;
+  bool ok = true;
+  {  // q [B][n][Hq][d]
+    const uint64_t d[4] = {kD, static_cast<uint64_t>(p.Hq), static_cast<uint64_t>(p.n), static_cast<uint64_t>(p.B)};
+    const uint64_t s[3] = {row, row * p.Hq, row * p.Hq * p.n};
+    const uint32_t bx[4] = {64, 1, kBM, 1};
+    ok &= make_map(&a.tm_q, p.q, 4, d, s, bx);
+  }
+  {  // chunk k, v [B][n][Hkv][d]
+    const uint64_t d[4] = {kD, static_cast<uint64_t>(p.Hkv), static_cast<uint64_t>(p.n), static_cast<uint64_t>(p.B)};
+    const uint64_t s[3] = {row, row * p.Hkv, row * p.Hkv * p.n};
+    const uint32_t bx[4] = {64, 1, kBN, 1};
+    ok &= make_map(&a.tm_kn, p.k, 4, d, s, bx);
+    ok &= make_map(&a.tm_vn, p.v, 4, d, s, bx);
+  }
+  {  // retrieval cache [B*Hr][cap][d]
+    const uint64_t d[3] = {kD, static_cast<uint64_t>(p.max_len), static_cast<uint64_t>(p.B) * (p.Hr > 0 ? p.Hr : 1)};
+    const uint64_t s[2] = {row, row * p.max_len};
+    const uint32_t bx[3] = {64, kBN, 1};
+    ok &= make_map(&a.tm_kc, p.rk, 3, d, s, bx);
+    ok &= make_map(&a.tm_vc, p.rv, 3, d, s, bx);
+  }
+  {  // streaming history [B*HsMax][S+W][d]
+    const uint64_t d[3] = {kD, static_cast<uint64_t>(p.S + p.W), static_cast<uint64_t>(p.B) * (p.HsMax > 0 ? p.HsMax : 1)};
+    const uint64_t s[2] = {row, row * (p.S + p.W)};
+    const uint32_t bx[3] = {64, kBN, 1};
+    ok &= make_map(&a.tm_kh, p.hk, 3, d, s, bx);
+    ok &= make_map(&a.tm_vh, p.hv, 3, d, s, bx);
+  }
+  if (!ok) return cudaErrorInvalidValue;
+  static bool attr = false;
+  if (!attr) {
+    cudaError_t e = cudaFuncSetAttribute(prefill_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemAlloc);
+    if (e != cudaSuccess) return e;
+    attr = true;
+  }
+  const int ntq = (p.n + kBM - 1) / kBM;
+  const int grid = ntq * p.B * p.Hq;
+  prefill_tc_kernel<<<grid, kTcThreads, kSmemAlloc, st>>>(a);
+  return cudaGetLastError();
+}
 
 }  // namespace duo

@@ -255,7 +255,7 @@ def _planted(ctx, d=128, seed=60):
     v = torch.randn(1, ctx, Hkv, d, generator=g)
     i = ctx - 1
     needles = {"middle": ctx // 2, "window_edge": i - W + 1, "outside": i - W, "sink_edge": S - 1, "post_sink": S}
-    values = {"middle": 3.0, "window_edge": 7.0, "outside": 11.0, "sink_edge": 17.0, "post_sink": 23.0}
+    values = {"middle": 0.2, "window_edge": 0.6, "outside": 1.0, "sink_edge": 1.8, "post_sink": 2.6}
     for name, j in needles.items():
         for kv in range(Hkv):
             qq = q[0, 0, kv * 4]
@@ -274,16 +274,17 @@ def test_planted_needle_and_mask_discrimination():
     got = o.float().cpu().numpy()[:, None]
     want, want_lse = oracle_rows(q, k, v, mask[0], S, W, ctx - 1)
     assert_close(got, want, torch.bfloat16, lse.cpu().numpy()[:, None], want_lse, "planted")
-    # retrieval query head 0 recovers the strongest needle (value 11, outside the
+    # retrieval query head 0 recovers the strongest needle (value 1.0, outside the
     # window); streaming query head 4 sees only the window-edge and sink needles
-    # (values 7 and 17, equal logits) and nothing of the middle or outside ones
-    assert abs(got[0, 0, 0].mean() - 11.0) < 1.0
-    assert abs(got[0, 0, 4].mean() - 12.0) < 1.0
+    # (values 0.6 and 1.8, equal logits) and nothing of the middle or outside ones
+    # (planted values stay O(1) so that bf16 output rounding is within tolerance)
+    assert abs(got[0, 0, 0].mean() - 1.0) < 0.1
+    assert abs(got[0, 0, 4].mean() - 1.2) < 0.1
     # each wrong reading of the mask moves the answer by far more than the tolerance
     for wrong in [dict(W=W + 1), dict(W=W - 1), dict(S=S + 1), dict(S=S - 1), dict(mask=[1, 1]), dict(mask=[0, 0])]:
         m = wrong.get("mask", mask[0].tolist())
         w2, _ = oracle_rows(q, k, v, m, wrong.get("S", S), wrong.get("W", W), ctx - 1)
-        assert np.abs(w2 - got).max() > 0.2, f"reading {wrong} is not distinguishable"
+        assert np.abs(w2 - got).max() > 0.1, f"reading {wrong} is not distinguishable"
 
 
 # ------------------------------------------------------------------- INT4
@@ -330,3 +331,67 @@ def test_int4_codes_bit_exact_and_decode(B, ctx):
     # for information: distance to attention over the unquantised bf16 values
     ref, _ = _decode_oracle(q, k, v, mask[0], S, W, ctx, steps)
     print("int4 vs unquantised:", errors(got, ref))
+
+
+# -------------------------------------------------- tensor-core pre-fill (bf16, d 128)
+
+@pytest.mark.parametrize("B,Hq,Hkv,mask,S,W,chunks", [
+    (1, 8, 2, [1, 0], 4, 32, [300]),
+    (2, 4, 4, [1, 0, 1, 0], 16, 512, [1000, 129, 1, 500]),
+    (1, 32, 8, [1, 0, 0, 1, 1, 0, 0, 1], 16, 512, [1024, 1024, 1024, 1024]),
+    (1, 4, 2, [0, 0], 0, 1, [257, 255]),
+    (1, 4, 2, [0, 0], 200, 3, [130, 140, 90]),
+    (1, 4, 2, [1, 1], 3, 7, [640, 17]),
+    (1, 8, 1, [0], 5, 300, [77, 600, 129]),
+])
+def test_tc_prefill_parity(B, Hq, Hkv, mask, S, W, chunks):
+    """Chunked pre-fill through the tensor-core kernel against the oracle, rows of
+    every chunk; shapes cover ragged tails, sinks inside and beyond one tile,
+    windows narrower and wider than a tile, MHA and GQA, B > 1."""
+    m = torch.tensor([mask], dtype=torch.uint8)
+    T = sum(chunks)
+    q, k, v = _seq(B, T, Hq, Hkv, 128, torch.bfloat16, 80)
+    cache = DuoCache(1, Hkv, 128, m, S, W, T, batch=B, q_heads=Hq, dtype=torch.bfloat16)
+    got, got_lse = _run(cache, q, k, v, chunks, 0)
+    want, want_lse = oracle_rows(q, k, v, m[0], S, W, 0)
+    assert_close(got, want, torch.bfloat16, got_lse, want_lse, f"tc prefill {chunks}")
+
+
+def test_llama3_prefill_reduced():
+    """Llama-3-8B GQA shape (32 q / 8 kv, 4 retrieval, S 16, W 512), 8K prompt in 2K
+    chunks, every output row against the oracle."""
+    mask = inputs.retrieval_mask(1, 8, 4, seed=1)
+    T, chunk = 8192, 2048
+    q, k, v = _seq(1, T, 32, 8, 128, torch.bfloat16, 90)
+    cache = DuoCache(1, 8, 128, mask, 16, 512, T, q_heads=32, dtype=torch.bfloat16)
+    got, got_lse = _run(cache, q, k, v, [chunk] * (T // chunk), 0)
+    want, want_lse = oracle_rows(q, k, v, mask[0], 16, 512, 0)
+    assert_close(got, want, torch.bfloat16, got_lse, want_lse, "llama3 prefill 8K")
+
+
+def test_llama3_prefill_full_size_sampled():
+    """The benchmarked workload: 256K-token prompt in 32K chunks, Llama-3-8B GQA shape.
+    Sampled rows of the first, a middle and the last chunk (first/last rows, rows at
+    the S and W boundaries, random rows; all 32 heads) against the oracle."""
+    mask = inputs.retrieval_mask(1, 8, 4, seed=1)
+    T, chunk = 262144, 32768
+    k = inputs.randn((1, T, 8, 128), 200, device=DEV)
+    v = inputs.randn((1, T, 8, 128), 201, device=DEV)
+    q = inputs.randn((1, chunk, 32, 128), 202, device=DEV)
+    cache = DuoCache(1, 8, 128, mask, 16, 512, T, q_heads=32, dtype=torch.bfloat16)
+    kb, vb = bits(k), bits(v)
+    rng = np.random.default_rng(0)
+    for c in range(T // chunk):
+        sl = slice(c * chunk, (c + 1) * chunk)
+        o, lse = cache.prefill_chunk(0, q, k[:, sl], v[:, sl])
+        if c not in (0, 3, 7):
+            continue
+        torch.cuda.synchronize()
+        rows_r = sorted(set([0, 1, 15, 16, 17, 510, 511, 512, 513, chunk - 1] + rng.integers(0, chunk, 12).tolist()))
+        ids = [r * 32 + h for r in rows_r for h in range(32)]
+        want, want_lse = oracle.attend(bits(q), kb[:, :(c + 1) * chunk], vb[:, :(c + 1) * chunk],
+                                       mask[0].numpy().astype(bool), 16, 512, pos0=c * chunk, rows=ids)
+        got = o.float()[0, rows_r].reshape(-1, 128).cpu().numpy()
+        got_lse = lse[0, rows_r].reshape(-1).cpu().numpy()
+        assert_close(got, want, torch.bfloat16, got_lse, want_lse, f"256K prefill chunk {c}")
+    assert cache.device_status() == 0
