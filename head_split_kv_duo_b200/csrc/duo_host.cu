@@ -79,8 +79,10 @@ bool make_layout(const Cfg &c, const uint8_t *mask, Layout *L) {
                      c.D * c.esize * 2.0;
   if (est > static_cast<double>(kMaxBytes)) return false;
   L->cap = static_cast<int64_t>(align_up(static_cast<size_t>(c.max_len), 256));
-  L->max_splits = static_cast<int>(
-      std::min<int64_t>(kMaxSplits, std::max<int64_t>(1, (c.max_len + kMinSplitTokens - 1) / kMinSplitTokens)));
+  // partial slots per head: enough for every 128-token unit of a retrieval head (or of
+  // the sink+ring slots), capped at kMaxSplits
+  const int64_t units = std::max<int64_t>((c.max_len + 127) / 128, (static_cast<int64_t>(c.S) + c.W + 127) / 128);
+  L->max_splits = static_cast<int>(std::min<int64_t>(kMaxSplits, std::max<int64_t>(1, units)));
   const size_t row = static_cast<size_t>(c.D) * c.esize;
   const size_t rrow = c.fmt == DUO_KV_INT4_G128 ? static_cast<size_t>(c.D / 2) : row;
   const size_t nslots = static_cast<size_t>(c.S) + c.W;
@@ -391,7 +393,9 @@ duo_status duo_decode_attention(duo_cache *c, int layer, const void *q, void *ou
   p.nsplit = static_cast<int>(nsplit);
   p.split_len = split_len;
   p.n_retr_ctas = static_cast<int>(heads * nsplit);
-  if (launch_decode(p, c->dtype, int4, st) != cudaSuccess) return DUO_ERR_CUDA;
+  const cudaError_t e = decode_tc_supported(p, c->dtype, int4) ? launch_decode_tc(p, c->num_sms, st)
+                                                                : launch_decode(p, c->dtype, int4, st);
+  if (e != cudaSuccess) return DUO_ERR_CUDA;
   return DUO_OK;
 }
 

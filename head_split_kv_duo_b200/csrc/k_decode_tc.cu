@@ -1,0 +1,518 @@
+// k_decode_tc.cu -- single-token decode attention on the tcgen05 tensor cores
+// (bf16, head_dim 128, up to 16 query heads per KV head).
+//
+// Operation ("Decoding Procedure", steps 2, 3 and 5): the newest query (position
+// len-1) of every query head attends to all cached tokens of its retrieval KV head,
+// or to the valid sink and ring slots of its streaming KV head.
+//
+// Tokens sit on the M side of the MMA, so a GQA group of G query heads costs one
+// N = 16 column block instead of G passes over the cache:
+//   S^T (128 tokens x 16)  = K_tile (128 x d)   . Qpad^T (d x 16)      A K-major, B K-major
+//   O^T (d 128 x 16)       = V_tile^T (d x 128) . P^T (128 tokens x 16) A MN-major, B K-major
+// Each K/V tile (128 rows, 64 KiB) and the group's queries (16 rows, 4 KiB) arrive by
+// TMA (128-byte swizzle) into a 3-stage ring.  Thread t of the softmax warpgroup owns
+// token t of S^T (TMEM lane t) and dimension t of O^T.
+//
+// Work balance: every (batch, KV head) is an item of 128-token units (retrieval:
+// ceil(len/128), streaming: ceil((S+W)/128)); the units of all items are laid end to
+// end and cut into one equal range per CTA (one CTA per SM).  A CTA flushes a partial
+// (max, sum, unnormalised output) whenever an item ends inside its range; the last
+// CTA to finish an item (atomic ticket, no waiting) merges its partials.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
+#include "device_common.cuh"
+
+namespace duo {
+
+namespace {
+
+constexpr int kThreads = 192;  // warp 0 TMA, warp 1 MMA + TMEM, warps 2-5 softmax
+constexpr int kTile = 128;
+constexpr int kD = 128;
+constexpr int kN = 16;         // padded query heads per item
+constexpr int kStages = 3;
+// shared memory map per stage: K [128][128] (2 swizzle atoms of 16 KiB), V likewise, Q [16][128]
+constexpr int kStK = 0, kStV = 32768, kStQ = 65536, kStage = 65536 + 4096;
+constexpr int kSmP = kStages * kStage;     // P^T [16][128] bf16: 2 atoms of 2 KiB
+constexpr int kSmRed = kSmP + 4096;        // cross-warp reductions [4][16] floats x 2
+constexpr int kSmBar = kSmRed + 1024;
+constexpr int kSmMisc = kSmBar + 256;
+constexpr int kSmemAlloc = kSmMisc + 64 + 1024;
+constexpr int kBarFull = 0, kBarEmpty = 3, kBarSFull = 6, kBarSFree = 8, kBarPFull = 10, kBarOFull = 11,
+              kBarDrain = 12, kNumBars = 13;
+
+struct TcDecodeArgs {
+  DecodeParams p;
+  int units_r, units_s;    // units per retrieval / streaming item
+  int n_items_r;           // B * Hr
+  int64_t total_units;
+  int num_ctas;
+  CUtensorMap tm_q, tm_kr, tm_vr, tm_ks, tm_vs;
+};
+
+__device__ __forceinline__ void tma_2d(uint32_t dst, const CUtensorMap *m, int x, int y, uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(m)), "r"(x), "r"(y), "r"(bar)
+      : "memory");
+}
+__device__ __forceinline__ void tma_3d(uint32_t dst, const CUtensorMap *m, int x, int y, int z, uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4}], [%5];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(m)), "r"(x), "r"(y), "r"(z), "r"(bar)
+      : "memory");
+}
+__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tc_commit(uint32_t bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar) : "memory");
+}
+__device__ __forceinline__ void tc_mma(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc, uint32_t acc) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(acc)
+      : "memory");
+}
+// 16 consecutive fp32 columns of this thread's TMEM lane
+__device__ __forceinline__ void tc_ld16(uint32_t taddr, float (&v)[16]) {
+  uint32_t r[16];
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+      "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15}, [%16];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]), "=r"(r[8]),
+        "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+      : "r"(taddr));
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+  for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
+}
+__device__ __forceinline__ uint64_t sdesc(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
+  return static_cast<uint64_t>((saddr >> 4) & 0x3FFFu) | (static_cast<uint64_t>((lbo >> 4) & 0x3FFFu) << 16) |
+         (static_cast<uint64_t>((sbo >> 4) & 0x3FFFu) << 32) | (1ull << 46) | (2ull << 61);
+}
+// kind::f16, fp32 accumulator, bf16 operands, M 128, N 16
+constexpr uint32_t idesc_m128n16(bool a_mn_major) {
+  return (1u << 4) | (1u << 7) | (1u << 10) | ((a_mn_major ? 1u : 0u) << 15) | ((16u >> 3) << 17) | ((128u >> 4) << 24);
+}
+__device__ __forceinline__ void named_sync(int id, int n) { asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory"); }
+
+__device__ __forceinline__ bool wait_bar(uint32_t bar, uint32_t parity, uint32_t *status, volatile int *abort_flag) {
+#pragma unroll 1
+  for (int i = 0; i < 64; ++i)
+    if (mbar_try_wait(bar, parity)) return true;
+  const unsigned long long t0 = globaltimer();
+#pragma unroll 1
+  while (true) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if (*abort_flag) return false;
+    if (globaltimer() - t0 > kWaitLimitNs) {
+      flag_status(status, kDevTimeout);
+      *abort_flag = 1;
+      return false;
+    }
+  }
+}
+
+// unit u -> (item, tile within item)
+struct Unit {
+  int item, tile;
+  bool retr;
+};
+__device__ __forceinline__ Unit unit_of(const TcDecodeArgs &a, int64_t u) {
+  const int64_t ur = static_cast<int64_t>(a.n_items_r) * a.units_r;
+  if (u < ur) return {static_cast<int>(u / a.units_r), static_cast<int>(u % a.units_r), true};
+  const int64_t us = u - ur;
+  return {a.n_items_r + static_cast<int>(us / a.units_s), static_cast<int>(us % a.units_s), false};
+}
+// first unit of CTA c: floor(c * U / C); the CTA holding unit u: ceil((u+1) C / U) - 1
+__device__ __forceinline__ int64_t cta_begin(const TcDecodeArgs &a, int c) {
+  return static_cast<int64_t>(c) * a.total_units / a.num_ctas;
+}
+__device__ __forceinline__ int cta_of(const TcDecodeArgs &a, int64_t u) {
+  return static_cast<int>(((u + 1) * a.num_ctas + a.total_units - 1) / a.total_units) - 1;
+}
+
+__global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_constant__ TcDecodeArgs a) {
+  const DecodeParams &p = a.p;
+  extern __shared__ char smem_raw[];
+  char *smem = reinterpret_cast<char *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const uint32_t sbase = smem_u32(smem);
+  auto bar = [&](int i) { return sbase + kSmBar + 8u * i; };
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + kSmMisc);
+  volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + kSmMisc + 4);
+  int *last_flag = reinterpret_cast<int *>(smem + kSmMisc + 8);
+  float *red = reinterpret_cast<float *>(smem + kSmRed);  // [4 warps][16]
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int64_t u0 = cta_begin(a, blockIdx.x), u1 = cta_begin(a, blockIdx.x + 1);
+  const int nu = static_cast<int>(u1 - u0);
+  const int G = p.G;
+
+  if (tid == 0) {
+    for (int i = 0; i < kNumBars; ++i)
+      mbar_init(bar(i), (i == kBarSFree || i == kBarSFree + 1 || i == kBarPFull) ? 128 : 1);
+    fence_mbar_init();
+    *abort_flag = 0;
+  }
+  // P^T rows >= G stay zero for the whole kernel
+  for (int i = tid; i < 4096 / 16; i += kThreads) reinterpret_cast<uint4 *>(smem + kSmP)[i] = make_uint4(0, 0, 0, 0);
+  if (warp == 1) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_slot)), "r"(64));
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
+  }
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0) {
+    // ================= TMA producer =================
+    if (lane == 0) {
+      for (int j = 0; j < nu; ++j) {
+        const int s = j % kStages;
+        if (j >= kStages && !wait_bar(bar(kBarEmpty + s), ((j / kStages) - 1) & 1, p.status, abort_flag)) break;
+        const Unit un = unit_of(a, u0 + j);
+        const uint32_t dst = sbase + s * kStage;
+        const uint32_t fb = bar(kBarFull + s);
+        mbar_expect_tx(fb, 65536 + 4096);
+        int b, g, z;
+        const CUtensorMap *mk, *mv;
+        if (un.retr) {
+          b = un.item / p.Hr;
+          const int ri = un.item % p.Hr;
+          g = p.hm.retr_head[ri];
+          z = b * p.Hr + ri;
+          mk = &a.tm_kr;
+          mv = &a.tm_vr;
+        } else {
+          const int it = un.item - a.n_items_r;
+          b = it / p.Hs;
+          const int si = it % p.Hs;
+          g = p.hm.strm_head[si];
+          z = b * p.Hs + si;
+          mk = &a.tm_ks;
+          mv = &a.tm_vs;
+        }
+        const int y = un.tile * kTile;
+        tma_3d(dst + kStK, mk, 0, y, z, fb);
+        tma_3d(dst + kStK + 16384, mk, 64, y, z, fb);
+        tma_3d(dst + kStV, mv, 0, y, z, fb);
+        tma_3d(dst + kStV + 16384, mv, 64, y, z, fb);
+        const int qrow = b * p.Hq + g * G;  // rows beyond this group's G heads are never used
+        tma_2d(dst + kStQ, &a.tm_q, 0, qrow, fb);
+        tma_2d(dst + kStQ + 2048, &a.tm_q, 64, qrow, fb);
+      }
+    }
+  } else if (warp == 1) {
+    // ================= MMA issuer =================
+    if (lane == 0) {
+      constexpr uint32_t kIdS = idesc_m128n16(false);
+      constexpr uint32_t kIdO = idesc_m128n16(true);
+      bool ok = true;
+      auto issue_o = [&](int jj) {
+        const int s = jj % kStages;
+        const uint32_t vb = sbase + s * kStage + kStV;
+        for (int kk = 0; kk < 8; ++kk) {  // K = 128 tokens in steps of 16
+          const uint64_t ad = sdesc(vb + kk * 2048, 16384, 1024);                                  // V^T, MN-major
+          const uint64_t bd = sdesc(sbase + kSmP + (kk >> 2) * 2048 + (kk & 3) * 32, 16, 1024);   // P^T, K-major
+          tc_mma(tmem + 32, ad, bd, kIdO, kk > 0 ? 1u : 0u);
+        }
+        tc_commit(bar(kBarOFull));
+        tc_commit(bar(kBarEmpty + s));
+      };
+      for (int j = 0; j < nu && ok; ++j) {
+        const int s = j % kStages;
+        if (!wait_bar(bar(kBarFull + s), (j / kStages) & 1, p.status, abort_flag)) { ok = false; break; }
+        if (j >= 2 && !wait_bar(bar(kBarSFree + (j & 1)), ((j - 2) >> 1) & 1, p.status, abort_flag)) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t st = sbase + s * kStage;
+        for (int kk = 0; kk < 8; ++kk) {  // K = d 128 in steps of 16
+          const uint64_t ad = sdesc(st + kStK + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024);  // K tile, K-major
+          const uint64_t bd = sdesc(st + kStQ + (kk >> 2) * 2048 + (kk & 3) * 32, 16, 1024);   // Qpad, K-major
+          tc_mma(tmem + (j & 1) * 16, ad, bd, kIdS, kk > 0 ? 1u : 0u);
+        }
+        tc_commit(bar(kBarSFull + (j & 1)));
+        if (j >= 1) {
+          if (!wait_bar(bar(kBarPFull), (j - 1) & 1, p.status, abort_flag)) { ok = false; break; }
+          tc_fence_after();
+          issue_o(j - 1);
+        }
+      }
+      if (ok && nu > 0 && wait_bar(bar(kBarPFull), (nu - 1) & 1, p.status, abort_flag)) {
+        tc_fence_after();
+        issue_o(nu - 1);
+      }
+      tc_commit(bar(kBarDrain));
+      mbar_wait(bar(kBarDrain), 0, p.status);
+    }
+  } else {
+    // ================= softmax warpgroup =================
+    const int t = ((warp & 3) << 5) | lane;  // token of S^T / dimension of O^T (TMEM lane)
+    const int wq = warp & 3;
+    const uint32_t lane_base = tmem + (static_cast<uint32_t>(wq << 5) << 16);
+    const float c = p.scale_log2;
+    float m[kN], l[kN], o[kN], alpha[kN];
+#pragma unroll
+    for (int q = 0; q < kN; ++q) {
+      m[q] = -INFINITY;
+      l[q] = 0.f;
+      o[q] = 0.f;
+      alpha[q] = 1.f;
+    }
+    bool ok = true;
+    int cur_item = -1;
+    int64_t item_u0 = 0;  // first unit of the current item (global index)
+
+    // Writes this CTA's result for `item` (partial or final) and merges when last.
+    auto flush = [&](int item) {
+      // row sums over the 128 threads
+#pragma unroll
+      for (int q = 0; q < kN; ++q) {
+        float v = warp_sum(l[q]);
+        if (lane == 0) red[wq * kN + q] = v;
+      }
+      named_sync(1, 128);
+      float lt[kN];
+#pragma unroll
+      for (int q = 0; q < kN; ++q) lt[q] = red[q] + red[kN + q] + red[2 * kN + q] + red[3 * kN + q];
+      named_sync(1, 128);
+      const bool retr = item < a.n_items_r;
+      const int units = retr ? a.units_r : a.units_s;
+      const int64_t ia = retr ? static_cast<int64_t>(item) * a.units_r
+                              : static_cast<int64_t>(a.n_items_r) * a.units_r +
+                                    static_cast<int64_t>(item - a.n_items_r) * a.units_s;
+      const int cfirst = cta_of(a, ia), clast = cta_of(a, ia + units - 1);
+      const int nseg = clast - cfirst + 1;
+      int b, g;
+      if (retr) {
+        b = item / p.Hr;
+        g = p.hm.retr_head[item % p.Hr];
+      } else {
+        const int it = item - a.n_items_r;
+        b = it / p.Hs;
+        g = p.hm.strm_head[it % p.Hs];
+      }
+      const int h0 = g * G;
+      if (nseg == 1) {
+        _Pragma("unroll") for (int q = 0; q < kN; ++q) if (q < G) {
+          Elem<__nv_bfloat16>::store(p.out, (static_cast<int64_t>(b) * p.Hq + h0 + q) * kD + t, o[q] / lt[q]);
+          if (t == 0 && p.lse) p.lse[b * p.Hq + h0 + q] = (m[q] + lg2(lt[q])) * kLn2;
+        }
+        return;
+      }
+      const int seg = blockIdx.x - cfirst;
+      const int64_t pitem = static_cast<int64_t>(b) * p.Hkv + g;
+      float *part = p.partials + (pitem * p.max_splits) * G * (kD + 2);
+      _Pragma("unroll") for (int q = 0; q < kN; ++q) if (q < G) {
+        float *dst = part + (static_cast<int64_t>(seg) * G + q) * (kD + 2);
+        dst[2 + t] = o[q];
+        if (t == 0) {
+          dst[0] = m[q];
+          dst[1] = lt[q];
+        }
+      }
+      __threadfence();
+      named_sync(1, 128);
+      if (t == 0) {
+        const uint32_t prev = atomicAdd(p.counters + pitem, 1u);
+        *last_flag = (prev == static_cast<uint32_t>(nseg - 1)) ? 1 : 0;
+      }
+      named_sync(1, 128);
+      if (!*last_flag) return;
+      __threadfence();
+      _Pragma("unroll") for (int q = 0; q < kN; ++q) if (q < G) {
+        float M = -INFINITY;
+        for (int sg = 0; sg < nseg; ++sg) M = fmaxf(M, __ldcg(part + (static_cast<int64_t>(sg) * G + q) * (kD + 2)));
+        float num = 0.f, den = 0.f;
+        for (int sg = 0; sg < nseg; ++sg) {
+          const float *r = part + (static_cast<int64_t>(sg) * G + q) * (kD + 2);
+          const float ms = __ldcg(r);
+          const float w = (ms == -INFINITY) ? 0.f : ex2(ms - M);
+          den = fmaf(w, __ldcg(r + 1), den);
+          num = fmaf(w, __ldcg(r + 2 + t), num);
+        }
+        Elem<__nv_bfloat16>::store(p.out, (static_cast<int64_t>(b) * p.Hq + h0 + q) * kD + t, num / den);
+        if (t == 0 && p.lse) p.lse[b * p.Hq + h0 + q] = (M + lg2(den)) * kLn2;
+      }
+      if (t == 0) p.counters[pitem] = 0u;
+    };
+
+    auto fold = [&](int jj) {  // o = o * alpha + O^T(jj) for this thread's dimension t
+      if (ok) ok = wait_bar(bar(kBarOFull), jj & 1, p.status, abort_flag);
+      tc_fence_after();
+      float v[16];
+      tc_ld16(lane_base + 32, v);
+#pragma unroll
+      for (int q = 0; q < kN; ++q) o[q] = fmaf(o[q], alpha[q], v[q]);
+    };
+
+    for (int j = 0; j < nu; ++j) {
+      const Unit un = unit_of(a, u0 + j);
+      if (ok) ok = wait_bar(bar(kBarSFull + (j & 1)), (j >> 1) & 1, p.status, abort_flag);
+      tc_fence_after();
+      float sv[16];
+      tc_ld16(lane_base + (j & 1) * 16, sv);
+      // this token's validity
+      bool valid;
+      const int64_t tok = static_cast<int64_t>(un.tile) * kTile + t;
+      if (un.retr) {
+        valid = tok < p.len;
+      } else {
+        const int S = p.S, W = p.W;
+        const int64_t len = p.len;
+        const int64_t rstart = (len - W > S) ? len - W : S;
+        const int64_t rcount = len > rstart ? len - rstart : 0;
+        if (tok >= S + W) valid = false;
+        else if (tok < S) valid = tok < len;
+        else if (rcount >= W) valid = true;
+        else valid = (((tok - S) - (S % W)) % W + W) % W < rcount;
+      }
+      // fold the previous unit's O^T (its P is then free), flush at item boundaries
+      if (j >= 1) fold(j - 1);
+      if (un.item != cur_item) {
+        if (cur_item >= 0) flush(cur_item);
+#pragma unroll
+        for (int q = 0; q < kN; ++q) {
+          m[q] = -INFINITY;
+          l[q] = 0.f;
+          o[q] = 0.f;
+          alpha[q] = 1.f;
+        }
+        cur_item = un.item;
+      }
+      // tile max per query head over the 128 tokens
+#pragma unroll
+      for (int q = 0; q < kN; ++q) {
+        float x = (valid && q < G) ? sv[q] : -INFINITY;
+        x = warp_max(x);
+        if (lane == 0) red[wq * kN + q] = x;
+      }
+      named_sync(1, 128);
+      uint16_t pb[kN];
+#pragma unroll
+      for (int q = 0; q < kN; ++q) {
+        const float mt = fmaxf(fmaxf(red[q], red[kN + q]), fmaxf(red[2 * kN + q], red[3 * kN + q])) * c;
+        const float mn = fmaxf(m[q], mt);
+        const bool none = mn == -INFINITY;
+        alpha[q] = none ? 1.f : ex2(m[q] - mn);
+        m[q] = mn;
+        const float pv = (valid && q < G && !none) ? ex2(fmaf(sv[q], c, -mn)) : 0.f;
+        l[q] = fmaf(l[q], alpha[q], pv);
+        const __nv_bfloat16 hb = __float2bfloat16_rn(pv);
+        pb[q] = *reinterpret_cast<const uint16_t *>(&hb);
+      }
+      named_sync(1, 128);  // red reused next tile
+      // P^T[q][t] into the 128B-swizzled K-major tile (rows q < G)
+      {
+        const int atom = t >> 6, col = t & 63;
+        char *pbase = smem + kSmP + atom * 2048;
+        _Pragma("unroll") for (int q = 0; q < kN; ++q) if (q < G) {
+          const int chunk = (col >> 3) ^ (q & 7);
+          *reinterpret_cast<uint16_t *>(pbase + q * 128 + chunk * 16 + (col & 7) * 2) = pb[q];
+        }
+      }
+      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+      tc_fence_before();
+      mbar_arrive(bar(kBarSFree + (j & 1)));
+      mbar_arrive(bar(kBarPFull));
+    }
+    if (nu > 0) {
+      fold(nu - 1);
+      flush(cur_item);
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 1) asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(64));
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static bool tried = false;
+  if (!tried) {
+    tried = true;
+    void *ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+  }
+  return fn;
+}
+
+bool map_bf16(CUtensorMap *m, const void *base, int rank, const uint64_t *dims, const uint64_t *strides,
+              const uint32_t *box) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t gd[3], gs[2];
+  cuuint32_t bx[3], es[3] = {1, 1, 1};
+  for (int r = 0; r < rank; ++r) {
+    gd[r] = dims[r];
+    bx[r] = box[r];
+  }
+  for (int r = 0; r < rank - 1; ++r) gs[r] = strides[r];
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, rank, const_cast<void *>(base), gd, gs, bx, es,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+}  // namespace
+
+bool decode_tc_supported(const DecodeParams &p, duo_dtype dt, bool int4) {
+  return dt == DUO_BF16 && !int4 && p.D == kD && p.G >= 1 && p.G <= kN && encode_fn() != nullptr;
+}
+
+cudaError_t launch_decode_tc(const DecodeParams &p, int num_sms, cudaStream_t st) {
+  static TcDecodeArgs a;
+  a.p = p;
+  a.units_r = static_cast<int>((p.len + kTile - 1) / kTile);
+  const int64_t slots = static_cast<int64_t>(p.S) + p.W;
+  const int64_t used = p.len < slots ? p.len : slots;  // streaming slots that can hold a token
+  a.units_s = static_cast<int>((used + kTile - 1) / kTile);
+  a.n_items_r = p.B * p.Hr;
+  a.total_units = static_cast<int64_t>(a.n_items_r) * a.units_r + static_cast<int64_t>(p.B) * p.Hs * a.units_s;
+  // at most one CTA per SM, and never more segments per item than partial slots
+  int64_t ctas = num_sms;
+  if (ctas > a.total_units) ctas = a.total_units;
+  if (ctas > kMaxSplits) ctas = kMaxSplits;
+  a.num_ctas = static_cast<int>(ctas);
+  const uint64_t row = kD * 2;
+  bool ok = true;
+  {  // queries [B*Hq][d]
+    const uint64_t d[2] = {kD, static_cast<uint64_t>(p.B) * p.Hq};
+    const uint64_t s[1] = {row};
+    const uint32_t bx[2] = {64, kN};
+    ok &= map_bf16(&a.tm_q, p.q, 2, d, s, bx);
+  }
+  {  // retrieval [B*Hr][cap][d]
+    const uint64_t d[3] = {kD, static_cast<uint64_t>(p.max_len), static_cast<uint64_t>(p.B) * (p.Hr > 0 ? p.Hr : 1)};
+    const uint64_t s[2] = {row, row * p.max_len};
+    const uint32_t bx[3] = {64, kTile, 1};
+    ok &= map_bf16(&a.tm_kr, p.rk, 3, d, s, bx);
+    ok &= map_bf16(&a.tm_vr, p.rv, 3, d, s, bx);
+  }
+  {  // streaming [B*Hs][S+W][d]
+    const uint64_t d[3] = {kD, static_cast<uint64_t>(slots), static_cast<uint64_t>(p.B) * (p.Hs > 0 ? p.Hs : 1)};
+    const uint64_t s[2] = {row, row * slots};
+    const uint32_t bx[3] = {64, kTile, 1};
+    ok &= map_bf16(&a.tm_ks, p.sk, 3, d, s, bx);
+    ok &= map_bf16(&a.tm_vs, p.sv, 3, d, s, bx);
+  }
+  if (!ok) return cudaErrorInvalidValue;
+  static bool attr = false;
+  if (!attr) {
+    cudaError_t e = cudaFuncSetAttribute(decode_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemAlloc);
+    if (e != cudaSuccess) return e;
+    attr = true;
+  }
+  decode_tc_kernel<<<a.num_ctas, kThreads, kSmemAlloc, st>>>(a);
+  return cudaGetLastError();
+}
+
+}  // namespace duo

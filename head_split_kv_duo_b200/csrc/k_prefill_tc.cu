@@ -181,6 +181,9 @@ __device__ int streaming_tiles(const PrefillParams &p, int r0, TileDesc *tl) {
   return nt;
 }
 
+// A key offset relative to a tile start, clamped to [-1, 127].
+__device__ __forceinline__ int clamp_col(int64_t x) { return static_cast<int>(x < -1 ? -1 : (x > kBN - 1 ? kBN - 1 : x)); }
+
 __device__ __forceinline__ TileDesc tile_of(const Plan &pl, const TileDesc *tl, int j) {
   if (pl.retr) return {0, j * kBN};
   return tl[j];
@@ -332,48 +335,51 @@ __global__ void __launch_bounds__(kTcThreads, 1) prefill_tc_kernel(const __grid_
 
     for (int j = 0; j < nt; ++j) {
       const TileDesc t = tile_of(pl, tl, j);
-      // positions of the 128 keys of this tile, and whether the whole tile is visible
-      int64_t pos0;
-      bool full_vis;
-      int valid_rows = kBN;
-      if (t.src == 0) {
-        pos0 = t.y;
-        full_vis = pos0 + kBN - 1 <= pl.q0;  // below the diagonal for every row
-      } else if (t.src == 2) {
-        pos0 = p.len + t.y;
-        valid_rows = p.n - t.y;
-        full_vis = false;
+      // Mask of this row over the tile's 128 keys, as three column bounds: key col is
+      // visible iff col <= hi && (col < sink_c || col > win_c).
+      int hi, sink_c = kBN, win_c = -1;
+      if (t.src == 0) {  // retrieval cache: positions y + col, causal only
+        hi = clamp_col(i - t.y);
       } else {
-        pos0 = -1;  // history: positions are not contiguous
-        valid_rows = p.hs + p.hw - t.y;
-        full_vis = false;
+        int64_t base, sink_rel, win_rel;
+        int valid;
+        if (t.src == 2) {  // chunk rows: positions len + y + col
+          base = p.len + t.y;
+          valid = p.n - t.y;
+          hi = clamp_col(i - base);
+          sink_rel = p.S - base;
+          win_rel = i - p.W - base;
+        } else {  // history rows: col < hs - y are sinks, later rows are wstart + (row - hs)
+          valid = p.hs + p.hw - t.y;
+          hi = kBN - 1;
+          sink_rel = p.hs - t.y;
+          win_rel = i - p.W - p.wstart + p.hs - t.y;
+        }
+        hi = min(hi, valid - 1);
+        sink_c = static_cast<int>(sink_rel < 0 ? 0 : (sink_rel > kBN ? kBN : sink_rel));
+        win_c = clamp_col(win_rel);
       }
-      auto key_pos = [&](int col) -> int64_t {
-        if (pos0 >= 0) return pos0 + col;
-        const int r = t.y + col;
-        return r < p.hs ? r : p.wstart + (r - p.hs);
-      };
-      auto visible = [&](int col) -> bool {
-        if (col >= valid_rows) return false;
-        const int64_t kp = key_pos(col);
-        if (kp > i) return false;
-        if (pl.retr) return true;
-        return kp < p.S || i - kp < p.W;
-      };
+      const bool full_vis = hi >= kBN - 1 && (sink_c >= kBN || win_c < 0);
 
       if (ok) ok = wait_bar(bar(kBarSFull + (j & 1)), (j >> 1) & 1, p.status, abort_flag);
       tc_fence_after();
       const uint32_t sbuf = lane_base + (j & 1) * 128;
       // pass 1: row max of the visible logits
       float mx = -INFINITY;
-#pragma unroll
+#pragma unroll 1
       for (int cc = 0; cc < 4; ++cc) {
         float v[32];
         tc_ld32(sbuf + cc * 32, v);
+        if (full_vis) {
 #pragma unroll
-        for (int e = 0; e < 32; ++e) {
-          const bool vis = full_vis || visible(cc * 32 + e);
-          mx = vis ? fmaxf(mx, v[e]) : mx;
+          for (int e = 0; e < 32; ++e) mx = fmaxf(mx, v[e]);
+        } else {
+#pragma unroll
+          for (int e = 0; e < 32; ++e) {
+            const int col = cc * 32 + e;
+            const bool vis = col <= hi && (col < sink_c || col > win_c);
+            mx = vis ? fmaxf(mx, v[e]) : mx;
+          }
         }
       }
       const float m_new = fmaxf(m, mx * c);
@@ -395,20 +401,31 @@ __global__ void __launch_bounds__(kTcThreads, 1) prefill_tc_kernel(const __grid_
       // pass 2: probabilities, row sum, bf16 P into the swizzled K-major tile
       float rs = 0.f;
       const float mc = none ? 0.f : m_new;
-#pragma unroll
+#pragma unroll 1
       for (int cc = 0; cc < 4; ++cc) {
         float v[32];
         tc_ld32(sbuf + cc * 32, v);
         uint32_t pk[16];
+        if (full_vis) {
 #pragma unroll
-        for (int e = 0; e < 32; e += 2) {
-          const bool v0 = full_vis || visible(cc * 32 + e);
-          const bool v1 = full_vis || visible(cc * 32 + e + 1);
-          const float p0 = v0 ? ex2(fmaf(v[e], c, -mc)) : 0.f;
-          const float p1 = v1 ? ex2(fmaf(v[e + 1], c, -mc)) : 0.f;
-          rs += p0 + p1;
-          const __nv_bfloat162 pb = __floats2bfloat162_rn(p0, p1);
-          pk[e >> 1] = *reinterpret_cast<const uint32_t *>(&pb);
+          for (int e = 0; e < 32; e += 2) {
+            const float p0 = ex2(fmaf(v[e], c, -mc)), p1 = ex2(fmaf(v[e + 1], c, -mc));
+            rs += p0 + p1;
+            const __nv_bfloat162 pb = __floats2bfloat162_rn(p0, p1);
+            pk[e >> 1] = *reinterpret_cast<const uint32_t *>(&pb);
+          }
+        } else {
+#pragma unroll
+          for (int e = 0; e < 32; e += 2) {
+            const int c0 = cc * 32 + e, c1 = c0 + 1;
+            const bool v0 = c0 <= hi && (c0 < sink_c || c0 > win_c);
+            const bool v1 = c1 <= hi && (c1 < sink_c || c1 > win_c);
+            const float p0 = v0 ? ex2(fmaf(v[e], c, -mc)) : 0.f;
+            const float p1 = v1 ? ex2(fmaf(v[e + 1], c, -mc)) : 0.f;
+            rs += p0 + p1;
+            const __nv_bfloat162 pb = __floats2bfloat162_rn(p0, p1);
+            pk[e >> 1] = *reinterpret_cast<const uint32_t *>(&pb);
+          }
         }
         // columns cc*32 .. cc*32+31 -> half (cc >> 1), 16-byte chunks 4*(cc&1) .. +3
         char *half = prow + (cc >> 1) * 16384;

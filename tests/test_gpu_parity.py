@@ -395,3 +395,20 @@ def test_llama3_prefill_full_size_sampled():
         got_lse = lse[0, rows_r].reshape(-1).cpu().numpy()
         assert_close(got, want, torch.bfloat16, got_lse, want_lse, f"256K prefill chunk {c}")
     assert cache.device_status() == 0
+
+
+@pytest.mark.parametrize("B,Hq,Hkv,mask,S,W,ctx", [
+    (3, 24, 3, [1, 0, 1], 4, 100, 777),
+    (2, 16, 2, [0, 1], 16, 512, 20000),
+    (1, 16, 1, [1], 0, 8, 300),
+    (2, 32, 2, [1, 0], 2, 129, 4097),
+    (5, 10, 5, [0, 0, 1, 0, 1], 3, 300, 2500),
+])
+def test_decode_group_sizes_and_batches(B, Hq, Hkv, mask, S, W, ctx):
+    """Query groups of 2, 8, 16 (and 8 on one KV head), odd batch sizes: every item of
+    the work split (retrieval and streaming heads of every sequence) against the oracle."""
+    m = torch.tensor([mask], dtype=torch.uint8)
+    steps = 2
+    _, q, k, v, got, got_lse = _fill_and_decode(Hq, Hkv, 128, m, S, W, B, ctx, steps, 110)
+    want, want_lse = _decode_oracle(q, k, v, m[0], S, W, ctx, steps)
+    assert_close(got, want, torch.bfloat16, got_lse, want_lse, f"decode B{B} G{Hq // Hkv}")
