@@ -34,13 +34,15 @@ constexpr int kN = 16;         // padded query heads per item
 constexpr int kStages = 3;
 // shared memory map per stage: K [128][128] (2 swizzle atoms of 16 KiB), V likewise, Q [16][128]
 constexpr int kStK = 0, kStV = 32768, kStQ = 65536, kStage = 65536 + 4096;
-constexpr int kSmP = kStages * kStage;     // P^T [16][128] bf16: 2 atoms of 2 KiB
-constexpr int kSmRed = kSmP + 4096;        // cross-warp reductions [4][16] floats x 2
+constexpr int kSmP = kStages * kStage;     // 2 x P^T [16][128] bf16 (2 atoms of 2 KiB each)
+constexpr int kSmRed = kSmP + 8192;        // cross-warp reductions [4][16] floats
 constexpr int kSmBar = kSmRed + 1024;
 constexpr int kSmMisc = kSmBar + 256;
 constexpr int kSmemAlloc = kSmMisc + 64 + 1024;
-constexpr int kBarFull = 0, kBarEmpty = 3, kBarSFull = 6, kBarSFree = 8, kBarPFull = 10, kBarOFull = 11,
-              kBarDrain = 12, kNumBars = 13;
+// Double-buffered resources (S, P, O) each have one barrier per buffer, so that no
+// barrier can complete two phases ahead of the thread waiting on it (parity waits).
+constexpr int kBarFull = 0, kBarEmpty = 3, kBarSFull = 6, kBarSFree = 8, kBarPFull = 10, kBarOFull = 12,
+              kBarDrain = 14, kNumBars = 15;
 
 struct TcDecodeArgs {
   DecodeParams p;
@@ -89,6 +91,43 @@ __device__ __forceinline__ void tc_ld16(uint32_t taddr, float (&v)[16]) {
 #pragma unroll
   for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
 }
+// N (1, 2, 4, 8 or 16) consecutive fp32 columns of this thread's TMEM lane
+template <int N>
+__device__ __forceinline__ void tc_ld(uint32_t taddr, float (&v)[N]) {
+  if constexpr (N == 16) {
+    tc_ld16(taddr, v);
+  } else {
+    uint32_t r[8];
+    if constexpr (N == 1)
+      asm volatile("tcgen05.ld.sync.aligned.32x32b.x1.b32 {%0}, [%1];" : "=r"(r[0]) : "r"(taddr));
+    else if constexpr (N == 2)
+      asm volatile("tcgen05.ld.sync.aligned.32x32b.x2.b32 {%0, %1}, [%2];" : "=r"(r[0]), "=r"(r[1]) : "r"(taddr));
+    else if constexpr (N == 4)
+      asm volatile("tcgen05.ld.sync.aligned.32x32b.x4.b32 {%0, %1, %2, %3}, [%4];"
+                   : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+                   : "r"(taddr));
+    else
+      asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];"
+                   : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7])
+                   : "r"(taddr));
+    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+    for (int i = 0; i < N; ++i) v[i] = __uint_as_float(r[i]);
+  }
+}
+// OR of `v` over the threads of named barrier `id` (all `n` threads receive it)
+__device__ __forceinline__ int bar_or(int id, int n, int v) {
+  int r;
+  asm volatile(
+      "{\n\t.reg .pred pi, po;\n\t"
+      "setp.ne.u32 pi, %1, 0;\n\t"
+      "bar.red.or.pred po, %2, %3, pi;\n\t"
+      "selp.u32 %0, 1, 0, po;\n\t}"
+      : "=r"(r)
+      : "r"(v), "r"(id), "r"(n)
+      : "memory");
+  return r;
+}
 __device__ __forceinline__ uint64_t sdesc(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
   return static_cast<uint64_t>((saddr >> 4) & 0x3FFFu) | (static_cast<uint64_t>((lbo >> 4) & 0x3FFFu) << 16) |
          (static_cast<uint64_t>((sbo >> 4) & 0x3FFFu) << 32) | (1ull << 46) | (2ull << 61);
@@ -135,6 +174,7 @@ __device__ __forceinline__ int cta_of(const TcDecodeArgs &a, int64_t u) {
   return static_cast<int>(((u + 1) * a.num_ctas + a.total_units - 1) / a.total_units) - 1;
 }
 
+template <int NQ>
 __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_constant__ TcDecodeArgs a) {
   const DecodeParams &p = a.p;
   extern __shared__ char smem_raw[];
@@ -153,12 +193,12 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
 
   if (tid == 0) {
     for (int i = 0; i < kNumBars; ++i)
-      mbar_init(bar(i), (i == kBarSFree || i == kBarSFree + 1 || i == kBarPFull) ? 128 : 1);
+      mbar_init(bar(i), (i == kBarSFree || i == kBarSFree + 1 || i == kBarPFull || i == kBarPFull + 1) ? 128 : 1);
     fence_mbar_init();
     *abort_flag = 0;
   }
   // P^T rows >= G stay zero for the whole kernel
-  for (int i = tid; i < 4096 / 16; i += kThreads) reinterpret_cast<uint4 *>(smem + kSmP)[i] = make_uint4(0, 0, 0, 0);
+  for (int i = tid; i < 8192 / 16; i += kThreads) reinterpret_cast<uint4 *>(smem + kSmP)[i] = make_uint4(0, 0, 0, 0);
   if (warp == 1) {
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_slot)), "r"(64));
     asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
@@ -216,12 +256,13 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
       auto issue_o = [&](int jj) {
         const int s = jj % kStages;
         const uint32_t vb = sbase + s * kStage + kStV;
+        const uint32_t pb = sbase + kSmP + (jj & 1) * 4096;
         for (int kk = 0; kk < 8; ++kk) {  // K = 128 tokens in steps of 16
-          const uint64_t ad = sdesc(vb + kk * 2048, 16384, 1024);                                  // V^T, MN-major
-          const uint64_t bd = sdesc(sbase + kSmP + (kk >> 2) * 2048 + (kk & 3) * 32, 16, 1024);   // P^T, K-major
-          tc_mma(tmem + 32, ad, bd, kIdO, kk > 0 ? 1u : 0u);
+          const uint64_t ad = sdesc(vb + kk * 2048, 16384, 1024);                    // V^T, MN-major
+          const uint64_t bd = sdesc(pb + (kk >> 2) * 2048 + (kk & 3) * 32, 16, 1024);  // P^T, K-major
+          tc_mma(tmem + 32 + (jj & 1) * 16, ad, bd, kIdO, kk > 0 ? 1u : 0u);
         }
-        tc_commit(bar(kBarOFull));
+        tc_commit(bar(kBarOFull + (jj & 1)));
         tc_commit(bar(kBarEmpty + s));
       };
       for (int j = 0; j < nu && ok; ++j) {
@@ -237,12 +278,12 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
         }
         tc_commit(bar(kBarSFull + (j & 1)));
         if (j >= 1) {
-          if (!wait_bar(bar(kBarPFull), (j - 1) & 1, p.status, abort_flag)) { ok = false; break; }
+          if (!wait_bar(bar(kBarPFull + ((j - 1) & 1)), ((j - 1) >> 1) & 1, p.status, abort_flag)) { ok = false; break; }
           tc_fence_after();
           issue_o(j - 1);
         }
       }
-      if (ok && nu > 0 && wait_bar(bar(kBarPFull), (nu - 1) & 1, p.status, abort_flag)) {
+      if (ok && nu > 0 && wait_bar(bar(kBarPFull + ((nu - 1) & 1)), ((nu - 1) >> 1) & 1, p.status, abort_flag)) {
         tc_fence_after();
         issue_o(nu - 1);
       }
@@ -251,34 +292,36 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
     }
   } else {
     // ================= softmax warpgroup =================
-    const int t = ((warp & 3) << 5) | lane;  // token of S^T / dimension of O^T (TMEM lane)
+    // Thread t owns token t of each S^T tile and dimension t of each O^T tile.  The
+    // running max m[q] is a reference: a tile's probabilities are exp2(s*c - m[q]);
+    // m is raised (and everything before rescaled) only when some logit of the tile
+    // exceeds it by more than kSlack, decided by one barrier-reduction vote.
+    constexpr float kSlack = 8.0f;
+    const int t = ((warp & 3) << 5) | lane;
     const int wq = warp & 3;
     const uint32_t lane_base = tmem + (static_cast<uint32_t>(wq << 5) << 16);
     const float c = p.scale_log2;
-    float m[kN], l[kN], o[kN], alpha[kN];
+    float m[NQ], l[NQ], o[NQ];
 #pragma unroll
-    for (int q = 0; q < kN; ++q) {
+    for (int q = 0; q < NQ; ++q) {
       m[q] = -INFINITY;
       l[q] = 0.f;
       o[q] = 0.f;
-      alpha[q] = 1.f;
     }
     bool ok = true;
     int cur_item = -1;
-    int64_t item_u0 = 0;  // first unit of the current item (global index)
 
     // Writes this CTA's result for `item` (partial or final) and merges when last.
     auto flush = [&](int item) {
-      // row sums over the 128 threads
 #pragma unroll
-      for (int q = 0; q < kN; ++q) {
-        float v = warp_sum(l[q]);
+      for (int q = 0; q < NQ; ++q) {
+        const float v = warp_sum(l[q]);
         if (lane == 0) red[wq * kN + q] = v;
       }
       named_sync(1, 128);
-      float lt[kN];
+      float lt[NQ];
 #pragma unroll
-      for (int q = 0; q < kN; ++q) lt[q] = red[q] + red[kN + q] + red[2 * kN + q] + red[3 * kN + q];
+      for (int q = 0; q < NQ; ++q) lt[q] = red[q] + red[kN + q] + red[2 * kN + q] + red[3 * kN + q];
       named_sync(1, 128);
       const bool retr = item < a.n_items_r;
       const int units = retr ? a.units_r : a.units_s;
@@ -298,23 +341,27 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
       }
       const int h0 = g * G;
       if (nseg == 1) {
-        _Pragma("unroll") for (int q = 0; q < kN; ++q) if (q < G) {
-          Elem<__nv_bfloat16>::store(p.out, (static_cast<int64_t>(b) * p.Hq + h0 + q) * kD + t, o[q] / lt[q]);
-          if (t == 0 && p.lse) p.lse[b * p.Hq + h0 + q] = (m[q] + lg2(lt[q])) * kLn2;
-        }
+#pragma unroll
+        for (int q = 0; q < NQ; ++q)
+          if (q < G) {
+            Elem<__nv_bfloat16>::store(p.out, (static_cast<int64_t>(b) * p.Hq + h0 + q) * kD + t, o[q] / lt[q]);
+            if (t == 0 && p.lse) p.lse[b * p.Hq + h0 + q] = (m[q] + lg2(lt[q])) * kLn2;
+          }
         return;
       }
       const int seg = blockIdx.x - cfirst;
       const int64_t pitem = static_cast<int64_t>(b) * p.Hkv + g;
       float *part = p.partials + (pitem * p.max_splits) * G * (kD + 2);
-      _Pragma("unroll") for (int q = 0; q < kN; ++q) if (q < G) {
-        float *dst = part + (static_cast<int64_t>(seg) * G + q) * (kD + 2);
-        dst[2 + t] = o[q];
-        if (t == 0) {
-          dst[0] = m[q];
-          dst[1] = lt[q];
+#pragma unroll
+      for (int q = 0; q < NQ; ++q)
+        if (q < G) {
+          float *dst = part + (static_cast<int64_t>(seg) * G + q) * (kD + 2);
+          dst[2 + t] = o[q];
+          if (t == 0) {
+            dst[0] = m[q];
+            dst[1] = lt[q];
+          }
         }
-      }
       __threadfence();
       named_sync(1, 128);
       if (t == 0) {
@@ -324,38 +371,47 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
       named_sync(1, 128);
       if (!*last_flag) return;
       __threadfence();
-      _Pragma("unroll") for (int q = 0; q < kN; ++q) if (q < G) {
-        float M = -INFINITY;
-        for (int sg = 0; sg < nseg; ++sg) M = fmaxf(M, __ldcg(part + (static_cast<int64_t>(sg) * G + q) * (kD + 2)));
-        float num = 0.f, den = 0.f;
-        for (int sg = 0; sg < nseg; ++sg) {
-          const float *r = part + (static_cast<int64_t>(sg) * G + q) * (kD + 2);
-          const float ms = __ldcg(r);
-          const float w = (ms == -INFINITY) ? 0.f : ex2(ms - M);
-          den = fmaf(w, __ldcg(r + 1), den);
-          num = fmaf(w, __ldcg(r + 2 + t), num);
+#pragma unroll
+      for (int q = 0; q < NQ; ++q)
+        if (q < G) {
+          float M = -INFINITY;
+          for (int sg = 0; sg < nseg; ++sg) M = fmaxf(M, __ldcg(part + (static_cast<int64_t>(sg) * G + q) * (kD + 2)));
+          float num = 0.f, den = 0.f;
+          for (int sg = 0; sg < nseg; ++sg) {
+            const float *r = part + (static_cast<int64_t>(sg) * G + q) * (kD + 2);
+            const float ms = __ldcg(r);
+            const float w = (ms == -INFINITY) ? 0.f : ex2(ms - M);
+            den = fmaf(w, __ldcg(r + 1), den);
+            num = fmaf(w, __ldcg(r + 2 + t), num);
+          }
+          Elem<__nv_bfloat16>::store(p.out, (static_cast<int64_t>(b) * p.Hq + h0 + q) * kD + t, num / den);
+          if (t == 0 && p.lse) p.lse[b * p.Hq + h0 + q] = (M + lg2(den)) * kLn2;
         }
-        Elem<__nv_bfloat16>::store(p.out, (static_cast<int64_t>(b) * p.Hq + h0 + q) * kD + t, num / den);
-        if (t == 0 && p.lse) p.lse[b * p.Hq + h0 + q] = (M + lg2(den)) * kLn2;
-      }
       if (t == 0) p.counters[pitem] = 0u;
     };
 
-    auto fold = [&](int jj) {  // o = o * alpha + O^T(jj) for this thread's dimension t
-      if (ok) ok = wait_bar(bar(kBarOFull), jj & 1, p.status, abort_flag);
+    // o = (o + O^T(jj)) * alpha for this thread's dimension t
+    auto fold = [&](int jj, const float (&alpha)[NQ]) {
+      if (ok) ok = wait_bar(bar(kBarOFull + (jj & 1)), (jj >> 1) & 1, p.status, abort_flag);
       tc_fence_after();
-      float v[16];
-      tc_ld16(lane_base + 32, v);
+      float v[NQ];
+      tc_ld<NQ>(lane_base + 32 + (jj & 1) * 16, v);
 #pragma unroll
-      for (int q = 0; q < kN; ++q) o[q] = fmaf(o[q], alpha[q], v[q]);
+      for (int q = 0; q < NQ; ++q) o[q] = (o[q] + v[q]) * alpha[q];
     };
+    float one[NQ];
+#pragma unroll
+    for (int q = 0; q < NQ; ++q) one[q] = 1.f;
 
+    bool pending = false;  // O^T of the previous unit still to be folded
     for (int j = 0; j < nu; ++j) {
       const Unit un = unit_of(a, u0 + j);
       if (ok) ok = wait_bar(bar(kBarSFull + (j & 1)), (j >> 1) & 1, p.status, abort_flag);
       tc_fence_after();
-      float sv[16];
-      tc_ld16(lane_base + (j & 1) * 16, sv);
+      float sv[NQ];
+      tc_ld<NQ>(lane_base + (j & 1) * 16, sv);
+      tc_fence_before();
+      mbar_arrive(bar(kBarSFree + (j & 1)));  // S buffer j % 2 is free again
       // this token's validity
       bool valid;
       const int64_t tok = static_cast<int64_t>(un.tile) * kTile + t;
@@ -371,57 +427,78 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
         else if (rcount >= W) valid = true;
         else valid = (((tok - S) - (S % W)) % W + W) % W < rcount;
       }
-      // fold the previous unit's O^T (its P is then free), flush at item boundaries
-      if (j >= 1) fold(j - 1);
       if (un.item != cur_item) {
-        if (cur_item >= 0) flush(cur_item);
+        if (cur_item >= 0) {
+          if (pending) fold(j - 1, one);
+          flush(cur_item);
+        }
 #pragma unroll
-        for (int q = 0; q < kN; ++q) {
+        for (int q = 0; q < NQ; ++q) {
           m[q] = -INFINITY;
           l[q] = 0.f;
           o[q] = 0.f;
-          alpha[q] = 1.f;
         }
+        pending = false;
         cur_item = un.item;
       }
-      // tile max per query head over the 128 tokens
+      // does any logit of this tile exceed the reference max by more than kSlack?
+      int need = 0;
 #pragma unroll
-      for (int q = 0; q < kN; ++q) {
-        float x = (valid && q < G) ? sv[q] : -INFINITY;
-        x = warp_max(x);
-        if (lane == 0) red[wq * kN + q] = x;
+      for (int q = 0; q < NQ; ++q)
+        if (q < G && valid && sv[q] * c > m[q] + kSlack) need = 1;
+      need = bar_or(1, 128, need);
+      float alpha[NQ];
+#pragma unroll
+      for (int q = 0; q < NQ; ++q) alpha[q] = 1.f;
+      if (need) {  // uniform over the warpgroup
+#pragma unroll
+        for (int q = 0; q < NQ; ++q) {
+          const float x = warp_max((valid && q < G) ? sv[q] : -INFINITY);
+          if (lane == 0) red[wq * kN + q] = x;
+        }
+        named_sync(1, 128);
+#pragma unroll
+        for (int q = 0; q < NQ; ++q) {
+          const float mt = fmaxf(fmaxf(red[q], red[kN + q]), fmaxf(red[2 * kN + q], red[3 * kN + q])) * c;
+          const float mn = fmaxf(m[q], mt);
+          alpha[q] = (mn == -INFINITY) ? 1.f : ex2(m[q] - mn);
+          m[q] = mn;
+        }
+        named_sync(1, 128);  // red is reused later
       }
-      named_sync(1, 128);
-      uint16_t pb[kN];
+      uint16_t pb[NQ];
 #pragma unroll
-      for (int q = 0; q < kN; ++q) {
-        const float mt = fmaxf(fmaxf(red[q], red[kN + q]), fmaxf(red[2 * kN + q], red[3 * kN + q])) * c;
-        const float mn = fmaxf(m[q], mt);
-        const bool none = mn == -INFINITY;
-        alpha[q] = none ? 1.f : ex2(m[q] - mn);
-        m[q] = mn;
-        const float pv = (valid && q < G && !none) ? ex2(fmaf(sv[q], c, -mn)) : 0.f;
+      for (int q = 0; q < NQ; ++q) {
+        const float pv = (valid && q < G && m[q] != -INFINITY) ? ex2(fmaf(sv[q], c, -m[q])) : 0.f;
         l[q] = fmaf(l[q], alpha[q], pv);
         const __nv_bfloat16 hb = __float2bfloat16_rn(pv);
         pb[q] = *reinterpret_cast<const uint16_t *>(&hb);
       }
-      named_sync(1, 128);  // red reused next tile
-      // P^T[q][t] into the 128B-swizzled K-major tile (rows q < G)
+      // P^T[q][t] into buffer j % 2 (its previous reader, unit j-2, was folded at j-1)
       {
         const int atom = t >> 6, col = t & 63;
-        char *pbase = smem + kSmP + atom * 2048;
-        _Pragma("unroll") for (int q = 0; q < kN; ++q) if (q < G) {
-          const int chunk = (col >> 3) ^ (q & 7);
-          *reinterpret_cast<uint16_t *>(pbase + q * 128 + chunk * 16 + (col & 7) * 2) = pb[q];
-        }
+        char *pbase = smem + kSmP + (j & 1) * 4096 + atom * 2048;
+#pragma unroll
+        for (int q = 0; q < NQ; ++q)
+          if (q < G) {
+            const int chunk = (col >> 3) ^ (q & 7);
+            *reinterpret_cast<uint16_t *>(pbase + q * 128 + chunk * 16 + (col & 7) * 2) = pb[q];
+          }
       }
       asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
       tc_fence_before();
-      mbar_arrive(bar(kBarSFree + (j & 1)));
-      mbar_arrive(bar(kBarPFull));
+      mbar_arrive(bar(kBarPFull + (j & 1)));
+      // fold the previous unit of the same item, bringing it to this unit's scale
+      if (pending) {
+        fold(j - 1, alpha);
+      } else {
+#pragma unroll
+        for (int q = 0; q < NQ; ++q) o[q] *= alpha[q];
+      }
+      pending = true;
     }
     if (nu > 0) {
-      fold(nu - 1);
+      if (pending) fold(nu - 1, one);
       flush(cur_item);
     }
   }
@@ -460,6 +537,18 @@ bool map_bf16(CUtensorMap *m, const void *base, int rank, const uint64_t *dims, 
   return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, rank, const_cast<void *>(base), gd, gs, bx, es,
             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <int NQ>
+cudaError_t launch_nq(const TcDecodeArgs &a, cudaStream_t st) {
+  static bool attr = false;
+  if (!attr) {
+    cudaError_t e = cudaFuncSetAttribute(decode_tc_kernel<NQ>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemAlloc);
+    if (e != cudaSuccess) return e;
+    attr = true;
+  }
+  decode_tc_kernel<NQ><<<a.num_ctas, kThreads, kSmemAlloc, st>>>(a);
+  return cudaGetLastError();
 }
 
 }  // namespace
@@ -505,14 +594,11 @@ cudaError_t launch_decode_tc(const DecodeParams &p, int num_sms, cudaStream_t st
     ok &= map_bf16(&a.tm_vs, p.sv, 3, d, s, bx);
   }
   if (!ok) return cudaErrorInvalidValue;
-  static bool attr = false;
-  if (!attr) {
-    cudaError_t e = cudaFuncSetAttribute(decode_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemAlloc);
-    if (e != cudaSuccess) return e;
-    attr = true;
-  }
-  decode_tc_kernel<<<a.num_ctas, kThreads, kSmemAlloc, st>>>(a);
-  return cudaGetLastError();
+  if (p.G <= 1) return launch_nq<1>(a, st);
+  if (p.G <= 2) return launch_nq<2>(a, st);
+  if (p.G <= 4) return launch_nq<4>(a, st);
+  if (p.G <= 8) return launch_nq<8>(a, st);
+  return launch_nq<16>(a, st);
 }
 
 }  // namespace duo

@@ -13,13 +13,13 @@
 //   warp 0      TMA producer: Q once, then K/V tiles of 128 keys into a 2-stage ring
 //   warp 1      TMEM allocator; lane 0 issues every tcgen05.mma
 //   warps 2..5  softmax warpgroup: thread t owns query row t (TMEM lane t)
-// TMEM (512 columns): S double buffer at columns 0 and 128, O tile at 256.
+// TMEM (512 columns): S double buffer at columns 0 and 128, O double buffer at 256 and 384.
 //   S_j = Q K_j^T      (M 128, N 128, K 128: 8 MMAs of K 16), into S[j % 2]
-//   O_j = P_j V_j      (M 128, N 128, K 128 keys), P_j from shared memory
+//   O_j = P_j V_j      (M 128, N 128, K 128 keys) into O[j % 2], P_j from shared memory
 // The softmax warps read S_j twice from TMEM (row max, then probabilities), write
-// P_j (bf16) to shared memory in the 128B-swizzled K-major layout, and fold each
-// O_j into fp32 registers with the online-softmax rescale.  The tensor core computes
-// S_{j+1} while the softmax warps work on tile j.
+// P_j (bf16) over K_j in its stage (128B-swizzled K-major), and only then fold O_{j-1}
+// into fp32 registers with the online-softmax rescale, so the tensor core computes
+// S_{j+1} and P_j V_j while the softmax warps work.
 //
 // Every mbarrier wait is bounded; a wait that runs out latches kDevTimeout in the
 // status word and sets an abort flag so that every role drains and exits.
@@ -42,15 +42,18 @@ constexpr int kMaxStrmTiles = 48;
 // shared memory map (bytes from the 1 KiB-aligned base)
 constexpr int kSmQ = 0;                    // 2 x [128][64] bf16, 128B swizzle
 constexpr int kSmKV = 32768;               // stage s: K at +s*65536, V at +s*65536+32768
-constexpr int kSmP = kSmKV + kKvStages * 65536;  // 2 x [128][64] bf16
-constexpr int kSmBar = kSmP + 32768;
+// P_j (bf16, 128B-swizzled K-major) is written over K_j in its own stage once S_j has
+// been computed, so P is double-buffered along with the K/V stages.
+constexpr int kSmBar = kSmKV + kKvStages * 65536;
 constexpr int kSmMisc = kSmBar + 256;
 constexpr int kSmTotal = kSmMisc + 1024 + kMaxStrmTiles * 16;
 constexpr int kSmemAlloc = kSmTotal + 1024;  // slack for aligning the base to 1 KiB
 
 // barrier indices (8 bytes each)
-constexpr int kBarQ = 0, kBarKvFull = 1, kBarKvEmpty = 3, kBarSFull = 5, kBarSFree = 7, kBarPFull = 9, kBarOFull = 10,
-              kBarDrain = 11, kNumBars = 12;
+// Double-buffered resources (S, P, O) have one barrier per buffer, so that no barrier
+// can complete two phases ahead of a thread waiting on it (parity waits).
+constexpr int kBarQ = 0, kBarKvFull = 1, kBarKvEmpty = 3, kBarSFull = 5, kBarSFree = 7, kBarPFull = 9, kBarOFull = 11,
+              kBarDrain = 13, kNumBars = 14;
 
 struct TileDesc {
   int src;      // 0 retrieval cache, 1 streaming history, 2 chunk input
@@ -218,7 +221,8 @@ __global__ void __launch_bounds__(kTcThreads, 1) prefill_tc_kernel(const __grid_
   pl.kvrow = b * (pl.retr ? p.Hr : p.HsMax) + p.hm.kind_idx[g];
 
   if (tid == 0) {
-    for (int i = 0; i < kNumBars; ++i) mbar_init(bar(i), (i == kBarSFree || i == kBarSFree + 1 || i == kBarPFull) ? 128 : 1);
+    for (int i = 0; i < kNumBars; ++i)
+      mbar_init(bar(i), (i == kBarSFree || i == kBarSFree + 1 || i == kBarPFull || i == kBarPFull + 1) ? 128 : 1);
     fence_mbar_init();
     *abort_flag = 0;
     int nt;
@@ -285,11 +289,11 @@ __global__ void __launch_bounds__(kTcThreads, 1) prefill_tc_kernel(const __grid_
         const int s = jj % kKvStages;
         const uint32_t vbase = sbase + kSmKV + s * 65536 + 32768;
         for (int kk = 0; kk < 8; ++kk) {
-          const uint64_t ad = sdesc(sbase + kSmP + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024);
+          const uint64_t ad = sdesc(sbase + kSmKV + s * 65536 + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024);
           const uint64_t bd = sdesc(vbase + kk * 2048, 16384, 1024);
-          tc_mma(tmem + 256, ad, bd, kIdPV, kk > 0 ? 1u : 0u);
+          tc_mma(tmem + 256 + (jj & 1) * 128, ad, bd, kIdPV, kk > 0 ? 1u : 0u);
         }
-        tc_commit(bar(kBarOFull));
+        tc_commit(bar(kBarOFull + (jj & 1)));
         tc_commit(bar(kBarKvEmpty + s));
       };
       for (int j = 0; j < nt && ok; ++j) {
@@ -306,12 +310,12 @@ __global__ void __launch_bounds__(kTcThreads, 1) prefill_tc_kernel(const __grid_
         }
         tc_commit(bar(kBarSFull + (j & 1)));
         if (j >= 1) {
-          if (!wait_bar(bar(kBarPFull), (j - 1) & 1, p.status, abort_flag)) { ok = false; break; }
+          if (!wait_bar(bar(kBarPFull + ((j - 1) & 1)), ((j - 1) >> 1) & 1, p.status, abort_flag)) { ok = false; break; }
           tc_fence_after();
           issue_pv(j - 1);
         }
       }
-      if (ok && nt > 0 && wait_bar(bar(kBarPFull), (nt - 1) & 1, p.status, abort_flag)) {
+      if (ok && nt > 0 && wait_bar(bar(kBarPFull + ((nt - 1) & 1)), ((nt - 1) >> 1) & 1, p.status, abort_flag)) {
         tc_fence_after();
         issue_pv(nt - 1);
       }
@@ -329,7 +333,6 @@ __global__ void __launch_bounds__(kTcThreads, 1) prefill_tc_kernel(const __grid_
 #pragma unroll
     for (int e = 0; e < kD; ++e) o[e] = 0.f;
     float m = -INFINITY, l = 0.f, alpha_prev = 1.f;
-    char *prow = smem + kSmP + row * 128;
     const int rsw = row & 7;
     bool ok = true;
 
@@ -386,19 +389,8 @@ __global__ void __launch_bounds__(kTcThreads, 1) prefill_tc_kernel(const __grid_
       const bool none = (m_new == -INFINITY);
       const float alpha = none ? 1.f : ex2(m - m_new);
 
-      // fold O_{j-1} into the register accumulator (P_{j-1} in shared memory is free after)
-      if (j >= 1) {
-        if (ok) ok = wait_bar(bar(kBarOFull), (j - 1) & 1, p.status, abort_flag);
-        tc_fence_after();
-#pragma unroll
-        for (int cc = 0; cc < 4; ++cc) {
-          float v[32];
-          tc_ld32(lane_base + 256 + cc * 32, v);
-#pragma unroll
-          for (int e = 0; e < 32; ++e) o[cc * 32 + e] = fmaf(o[cc * 32 + e], alpha_prev, v[e]);
-        }
-      }
-      // pass 2: probabilities, row sum, bf16 P into the swizzled K-major tile
+      // pass 2: probabilities, row sum, bf16 P over K_j in stage j % 2
+      char *prow = smem + kSmKV + (j % kKvStages) * 65536 + row * 128;
       float rs = 0.f;
       const float mc = none ? 0.f : m_new;
 #pragma unroll 1
@@ -437,21 +429,33 @@ __global__ void __launch_bounds__(kTcThreads, 1) prefill_tc_kernel(const __grid_
       }
       tc_fence_before();
       mbar_arrive(bar(kBarSFree + (j & 1)));  // S buffer j % 2 may be overwritten
+      fence_async_smem();  // P visible to the tensor core
+      tc_fence_before();
+      mbar_arrive(bar(kBarPFull + (j & 1)));
+      // fold O_{j-1} (scale m_{j-1}) into the registers while the tensor core works on P_j
+      if (j >= 1) {
+        if (ok) ok = wait_bar(bar(kBarOFull + ((j - 1) & 1)), ((j - 1) >> 1) & 1, p.status, abort_flag);
+        tc_fence_after();
+#pragma unroll
+        for (int cc = 0; cc < 4; ++cc) {
+          float v[32];
+          tc_ld32(lane_base + 256 + ((j - 1) & 1) * 128 + cc * 32, v);
+#pragma unroll
+          for (int e = 0; e < 32; ++e) o[cc * 32 + e] = fmaf(o[cc * 32 + e], alpha_prev, v[e]);
+        }
+      }
       l = fmaf(l, alpha, rs);
       m = m_new;
       alpha_prev = alpha;
-      fence_async_smem();  // P visible to the tensor core
-      tc_fence_before();
-      mbar_arrive(bar(kBarPFull));
     }
     // last O tile
     if (nt > 0) {
-      if (ok) ok = wait_bar(bar(kBarOFull), (nt - 1) & 1, p.status, abort_flag);
+      if (ok) ok = wait_bar(bar(kBarOFull + ((nt - 1) & 1)), ((nt - 1) >> 1) & 1, p.status, abort_flag);
       tc_fence_after();
 #pragma unroll
       for (int cc = 0; cc < 4; ++cc) {
         float v[32];
-        tc_ld32(lane_base + 256 + cc * 32, v);
+        tc_ld32(lane_base + 256 + ((nt - 1) & 1) * 128 + cc * 32, v);
 #pragma unroll
         for (int e = 0; e < 32; ++e) o[cc * 32 + e] = fmaf(o[cc * 32 + e], alpha_prev, v[e]);
       }
