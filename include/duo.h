@@ -202,6 +202,31 @@ DUO_API duo_status duo_debug_region(const duo_cache *cache, int layer, duo_regio
  */
 DUO_API duo_status duo_get_device_status(duo_cache *cache, void *cuda_stream);
 
+/*
+ * duo_decode_attention for callers that cannot allocate device memory when they
+ * decode -- for instance code running while a CUDA graph is being captured, where
+ * cudaMalloc is not allowed, or a runtime whose device memory belongs to a pool sized
+ * once at start-up.  The paper has no counterpart: this is a property of the library,
+ * not of the method.
+ *
+ * Same arguments, layouts and result as duo_decode_attention.  It calls no cudaMalloc,
+ * cudaFree or allocating library routine and does not use the scratch area of the
+ * cache buffer: the split-KV partial results and merge tickets go to one 4 MiB array
+ * of static device memory that every GPU which loads this library holds until the
+ * process exits.  The tickets are cleared (cudaMemsetAsync on `cuda_stream`) at every
+ * call; the rest of the array keeps the previous call's contents, so calls that
+ * overlap on the GPU (other streams, other threads) race and must be ordered by the
+ * caller.  The first call on each device looks up the array's device address with
+ * cudaGetSymbolAddress, with that device current; make that first call before any
+ * stream capture.
+ * Limits: bf16 caches with head_dim 128, not INT4, at most 16 query heads per KV head
+ * (else DUO_ERR_UNSUPPORTED).  The partials of B*kv_heads heads must fit the array at
+ * one CTA: B*kv_heads*G*(head_dim+2)*4 bytes <= 4 MiB less the tickets, else
+ * DUO_ERR_CAPACITY; larger head counts still fit but run on fewer CTAs.
+ */
+DUO_API duo_status duo_decode_attention_static_scratch(duo_cache *cache, int layer, const void *q, void *out,
+                                                       float *lse, void *cuda_stream);
+
 /* Static description of a status code. */
 DUO_API const char *duo_status_str(duo_status status);
 
