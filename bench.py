@@ -37,12 +37,25 @@ CTX = 131072
 ROT_LAYERS = 4
 PREFILL_LEN, PREFILL_CHUNK = 262144, 32768
 
+# decode workloads: (q heads, kv heads, retrieval kv heads, context, batch, layers, retrieval format);
+# `layers` caches are visited in turn each step (the headline rotates 4 so that a step
+# touches more K/V than L2 holds; the INT4 stack is the 32-layer model itself)
+DECODE_WORKLOADS = {
+    "llama3-8b-gqa-decode-128k-b1": (32, 8, 4, 131072, 1, 4, "same"),
+    "llama3-8b-gqa-decode-128k-b4": (32, 8, 4, 131072, 4, 2, "same"),
+    "llama2-7b-mha-decode-32k-b1": (32, 32, 8, 32768, 1, 8, "same"),
+    "llama2-7b-mha-decode-32k-b8": (32, 32, 8, 32768, 8, 2, "same"),
+    "llama3-8b-gqa-decode-1m-int4-32l": (32, 8, 4, 1 << 20, 1, 32, "int4"),
+}
 
-def decode_bytes(len_, B=1, Hr=NRET, Hs=HKV - NRET, Hq=HQ, d=D):
+
+def decode_bytes(len_, B=1, Hr=NRET, Hs=HKV - NRET, Hq=HQ, d=D, fmt="same"):
     """Algorithmic HBM bytes of one decode-attention call: every visible K and V row
-    once (bf16), the queries, the outputs and the lse."""
+    once (bf16 rows, or INT4 codes plus fp16 scale/zero), the queries, the outputs and
+    the lse."""
     kv = 2 * d * 2
-    return B * (Hr * len_ * kv + Hs * min(len_, S + W) * kv) + B * Hq * d * 2 * 2 + B * Hq * 4
+    rkv = 2 * (d // 2 + 4) if fmt == "int4" else kv
+    return B * (Hr * len_ * rkv + Hs * min(len_, S + W) * kv) + B * Hq * d * 2 * 2 + B * Hq * 4
 
 
 def prefill_flops(L=PREFILL_LEN, Hq=HQ, d=D, G=HQ // HKV, nret=NRET):
@@ -115,22 +128,23 @@ class ClockSampler:
 
 
 def kernel_hash():
+    """Hash of the decode kernels' sources: recorded DRAM traffic is void once they change."""
     h = hashlib.sha256()
-    for f in ("k_decode.cu", "device_common.cuh", "duo_internal.h"):
+    for f in ("k_decode.cu", "k_decode_tc.cu", "device_common.cuh", "duo_internal.h"):
         h.update(open(os.path.join(ROOT, "head_split_kv_duo_b200", "csrc", f), "rb").read())
     return h.hexdigest()[:16]
 
 
-def recorded_traffic():
-    """DRAM bytes per decode launch from the committed ncu summary, when it was taken
-    on the current kernel source."""
+def recorded_traffic(workload):
+    """DRAM bytes (read + write) per decode launch from the committed ncu summary of
+    this workload, when it was taken on the current kernel source."""
     path = os.path.join(ROOT, "profiles", "decode_traffic.json")
     if not os.path.exists(path):
         return None
-    rec = json.load(open(path))
-    if rec.get("kernel_hash") != kernel_hash():
+    rec = json.load(open(path)).get(workload)
+    if not rec or rec.get("kernel_hash") != kernel_hash():
         return None
-    return rec.get("dram_bytes_per_launch_full_size")
+    return rec.get("dram_bytes_per_launch")
 
 
 # ---------------------------------------------------------------- our arm
@@ -145,29 +159,37 @@ def run_ours(args, rank, world, dist):
     torch.cuda.set_device(dev)
     hbm_peak, tc_peak, tc_sust, peak_src = peaks()
     steps, warmup = args.steps, args.warmup
-    total_tokens = warmup + steps + 1
-    max_len = CTX + warmup + 2 * steps + 16
-    mask = inputs.retrieval_mask(ROT_LAYERS, HKV, NRET, seed=1)
-    cache = DuoCache(ROT_LAYERS, HKV, D, mask, S, W, max_len, q_heads=HQ, dtype=torch.bfloat16, device=dev)
-    # fill each layer to CTX tokens (seeded N(0,1) K/V)
-    for layer in range(ROT_LAYERS):
-        k = inputs.randn((1, CTX, HKV, D), 100 + 2 * layer, device=dev)
-        v = inputs.randn((1, CTX, HKV, D), 101 + 2 * layer, device=dev)
-        cache.append_kv(layer, k, v)
-        del k, v
+    Hq, Hkv, nret, ctx, B, nlayers, fmt = DECODE_WORKLOADS[args.workload]
+    Hr, Hs = nret, Hkv - nret
+    max_len = ctx + warmup + 2 * steps + 16
+    mask = inputs.retrieval_mask(nlayers, Hkv, nret, seed=1)
+    cache = DuoCache(nlayers, Hkv, D, mask, S, W, max_len, batch=B, q_heads=Hq, dtype=torch.bfloat16,
+                     retr_fmt=fmt, device=dev)
+    # fill each layer to `ctx` tokens (seeded N(0,1) K/V), in pieces of at most 2^18 tokens
+    piece = min(ctx, 1 << 18)
+    for layer in range(nlayers):
+        for t0 in range(0, ctx, piece):
+            n = min(piece, ctx - t0)
+            k = inputs.randn((B, n, Hkv, D), 100 + 1000 * layer + 2 * t0 // piece, device=dev)
+            v = inputs.randn((B, n, Hkv, D), 101 + 1000 * layer + 2 * t0 // piece, device=dev)
+            cache.append_kv(layer, k, v)
+            del k, v
     torch.cuda.synchronize()
     # per-step inputs: q, k, v of the new token for every layer
     nstep_in = warmup + steps
-    qs = inputs.randn((nstep_in, ROT_LAYERS, 1, HQ, D), 7, device=dev)
-    ks = inputs.randn((nstep_in, ROT_LAYERS, 1, 1, HKV, D), 8, device=dev)
-    vs = inputs.randn((nstep_in, ROT_LAYERS, 1, 1, HKV, D), 9, device=dev)
-    out = torch.empty(ROT_LAYERS, 1, HQ, D, dtype=torch.bfloat16, device=dev)
-    lse = torch.empty(ROT_LAYERS, 1, HQ, dtype=torch.float32, device=dev)
+    qs = inputs.randn((nstep_in, nlayers, B, Hq, D), 7, device=dev)
+    ks = inputs.randn((nstep_in, nlayers, B, 1, Hkv, D), 8, device=dev)
+    vs = inputs.randn((nstep_in, nlayers, B, 1, Hkv, D), 9, device=dev)
+    out = torch.empty(nlayers, B, Hq, D, dtype=torch.bfloat16, device=dev)
+    lse = torch.empty(nlayers, B, Hq, dtype=torch.float32, device=dev)
     stream = torch.cuda.current_stream()
+
+    def nbytes_of(n):
+        return decode_bytes(n, B=B, Hr=Hr, Hs=Hs, Hq=Hq, fmt=fmt)
 
     def step(i, ev=None):
         nbytes = 0
-        for layer in range(ROT_LAYERS):
+        for layer in range(nlayers):
             cache.append_kv(layer, ks[i, layer], vs[i, layer], stream=stream)
             n = cache.len(layer)
             if ev is not None:
@@ -178,7 +200,7 @@ def run_ours(args, rank, world, dist):
                 ev[2].append((ev[0], ev[1]))
                 ev[0] = torch.cuda.Event(enable_timing=True)
                 ev[1] = torch.cuda.Event(enable_timing=True)
-            nbytes += decode_bytes(n)
+            nbytes += nbytes_of(n)
         return nbytes
 
     for i in range(warmup):
@@ -210,9 +232,9 @@ def run_ours(args, rank, world, dist):
         dist.all_reduce(b)
         bytes_sum = float(b.item())
     value = bytes_sum / (ms_max * 1e-3) / 1e9
-    us_per_token_layer = ms * 1e3 / (steps * ROT_LAYERS)
+    us_per_token_layer = ms * 1e3 / (steps * nlayers)
     dec_avg_ms = statistics.mean(dec_ms)
-    per_launch_bytes = nbytes / (steps * ROT_LAYERS)
+    per_launch_bytes = nbytes / (steps * nlayers)
     achieved = per_launch_bytes / (dec_avg_ms * 1e-3) / 1e9
 
     # ---- end-to-end through the public API with host buffers ----
@@ -221,11 +243,11 @@ def run_ours(args, rank, world, dist):
         hq = qs.cpu().pin_memory()
         hk = ks.cpu().pin_memory()
         hv = vs.cpu().pin_memory()
-        hout = torch.empty(ROT_LAYERS, 1, HQ, D, dtype=torch.bfloat16).pin_memory()
+        hout = torch.empty(nlayers, B, Hq, D, dtype=torch.bfloat16).pin_memory()
         dq = torch.empty_like(qs[0])
         dk = torch.empty_like(ks[0])
         dv = torch.empty_like(vs[0])
-        # rewind lengths is not possible; continue appending (lengths grow by `steps`)
+        # lengths cannot be rewound: this pass keeps appending (max_len has room for it)
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         eb = 0
         torch.cuda.synchronize()
@@ -234,9 +256,9 @@ def run_ours(args, rank, world, dist):
             dq.copy_(hq[i], non_blocking=True)
             dk.copy_(hk[i], non_blocking=True)
             dv.copy_(hv[i], non_blocking=True)
-            for layer in range(ROT_LAYERS):
+            for layer in range(nlayers):
                 cache.append_kv(layer, dk[layer], dv[layer], stream=stream)
-                eb += decode_bytes(cache.len(layer))
+                eb += nbytes_of(cache.len(layer))
                 cache.decode_attention(layer, dq[layer], out=out[layer], lse=lse[layer], stream=stream)
             hout.copy_(out, non_blocking=True)
         e1.record(stream)
@@ -245,25 +267,30 @@ def run_ours(args, rank, world, dist):
         h2d = (dq.numel() + dk.numel() + dv.numel()) * 2
         e2e = {"value": round(eb / (ems * 1e-3) / 1e9, 1), "unit": "GB/s", "h2d_bytes_per_step": h2d,
                "d2h_bytes_per_step": hout.numel() * 2, "ms_per_step": round(ems / steps, 4)}
+    cache.close()
+    del cache
+    torch.cuda.empty_cache()
 
     # ---- chunked pre-fill (Llama-3-8B GQA, 256K in 32K chunks) ----
     prefill = None
     if not args.skip_prefill:
         prefill = run_prefill(args, dev, tc_peak, tc_sust, peak_src)
 
+    kv_gb = nlayers * nbytes_of(ctx) / 1e9
     res = {
         "metric": METRIC, "value": round(value, 1), "unit": "GB/s", "n_gpus": world, "steps": steps,
         "warmup": warmup, "ms_per_step": round(ms_max / steps, 4), "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-        "config": {"workload": WORKLOAD, "q_heads": HQ, "kv_heads": HKV, "head_dim": D, "retrieval_kv_heads": NRET,
-                   "S": S, "W": W, "context": CTX, "batch": 1, "layers_rotated": ROT_LAYERS,
-                   "l2": "inputs larger than L2: 4 rotating layer caches of 1.08 GB", "parallelism": f"replicas{world}"},
+        "vs_baseline": None, "dtype": "bf16" if fmt == "same" else "bf16+int4kv", "data": "synthetic",
+        "config": {"workload": args.workload, "q_heads": Hq, "kv_heads": Hkv, "head_dim": D, "retrieval_kv_heads": nret,
+                   "S": S, "W": W, "context": ctx, "batch": B, "layers": nlayers, "retrieval_kv": fmt,
+                   "l2": f"inputs larger than L2: {nlayers} layer caches of {kv_gb / nlayers:.2f} GB visited per step",
+                   "parallelism": f"replicas{world}"},
         "us_per_token_layer": round(us_per_token_layer, 3),
-        "roofline": {"bound": "hbm", "kernel": "decode_kernel", "achieved": round(achieved, 1),
+        "roofline": {"bound": "hbm", "kernel": "decode", "achieved": round(achieved, 1),
                      "peak": hbm_peak, "peak_source": f"{peak_src} hbm_gbs (burst copy)", "unit": "GB/s",
-                     "frac": round(achieved / hbm_peak, 4), "traffic": recorded_traffic(),
+                     "frac": round(achieved / hbm_peak, 4), "traffic": recorded_traffic(args.workload),
                      "algorithmic_bytes_per_launch": int(per_launch_bytes), "avg_launch_us": round(dec_avg_ms * 1e3, 3)},
-        "gpu_launches": steps * ROT_LAYERS * 2,
+        "gpu_launches": steps * nlayers * 2,
         "clocks": clk.summary(),
         "e2e": e2e,
         "prefill": prefill,
@@ -348,6 +375,7 @@ def oracle_sample(args):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--workload", default=WORKLOAD, choices=sorted(DECODE_WORKLOADS))
     ap.add_argument("--steps", type=int, default=50)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])

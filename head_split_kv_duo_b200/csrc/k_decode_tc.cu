@@ -32,6 +32,12 @@ constexpr int kTile = 128;
 constexpr int kD = 128;
 constexpr int kN = 16;         // padded query heads per item
 constexpr int kStages = 3;
+// Each contraction (over d for S^T, over tokens for O^T) is split into kAcc partial
+// accumulators in separate TMEM columns, so the tensor core runs kAcc independent
+// chains of 8 / kAcc MMAs instead of one chain of 8; the softmax warps add them up.
+constexpr int kAcc = 4;
+constexpr int kTmO = 2 * kAcc * 16;         // TMEM column of the O^T double buffer
+constexpr int kTmemCols = 4 * kAcc * 16;    // S^T x 2 and O^T x 2, kAcc blocks of 16 each
 // shared memory map per stage: K [128][128] (2 swizzle atoms of 16 KiB), V likewise, Q [16][128]
 constexpr int kStK = 0, kStV = 32768, kStQ = 65536, kStage = 65536 + 4096;
 constexpr int kSmP = kStages * kStage;     // 2 x P^T [16][128] bf16 (2 atoms of 2 KiB each)
@@ -113,6 +119,18 @@ __device__ __forceinline__ void tc_ld(uint32_t taddr, float (&v)[N]) {
     asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 #pragma unroll
     for (int i = 0; i < N; ++i) v[i] = __uint_as_float(r[i]);
+  }
+}
+// Sum of kAcc partial accumulators, 16 columns apart
+template <int N>
+__device__ __forceinline__ void tc_ld_sum(uint32_t taddr, float (&v)[N]) {
+  tc_ld<N>(taddr, v);
+#pragma unroll
+  for (int a = 1; a < kAcc; ++a) {
+    float w[N];
+    tc_ld<N>(taddr + a * 16, w);
+#pragma unroll
+    for (int q = 0; q < N; ++q) v[q] += w[q];
   }
 }
 // OR of `v` over the threads of named barrier `id` (all `n` threads receive it)
@@ -200,7 +218,8 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
   // P^T rows >= G stay zero for the whole kernel
   for (int i = tid; i < 8192 / 16; i += kThreads) reinterpret_cast<uint4 *>(smem + kSmP)[i] = make_uint4(0, 0, 0, 0);
   if (warp == 1) {
-    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_slot)), "r"(64));
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_slot)),
+                 "r"(kTmemCols));
     asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
   }
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
@@ -257,10 +276,11 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
         const int s = jj % kStages;
         const uint32_t vb = sbase + s * kStage + kStV;
         const uint32_t pb = sbase + kSmP + (jj & 1) * 4096;
-        for (int kk = 0; kk < 8; ++kk) {  // K = 128 tokens in steps of 16
+        for (int i = 0; i < 8; ++i) {  // K = 128 tokens in steps of 16, kAcc independent chains
+          const int kk = (i % kAcc) * (8 / kAcc) + i / kAcc;
           const uint64_t ad = sdesc(vb + kk * 2048, 16384, 1024);                    // V^T, MN-major
           const uint64_t bd = sdesc(pb + (kk >> 2) * 2048 + (kk & 3) * 32, 16, 1024);  // P^T, K-major
-          tc_mma(tmem + 32 + (jj & 1) * 16, ad, bd, kIdO, kk > 0 ? 1u : 0u);
+          tc_mma(tmem + kTmO + (jj & 1) * kAcc * 16 + (i % kAcc) * 16, ad, bd, kIdO, i >= kAcc ? 1u : 0u);
         }
         tc_commit(bar(kBarOFull + (jj & 1)));
         tc_commit(bar(kBarEmpty + s));
@@ -271,10 +291,11 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
         if (j >= 2 && !wait_bar(bar(kBarSFree + (j & 1)), ((j - 2) >> 1) & 1, p.status, abort_flag)) { ok = false; break; }
         tc_fence_after();
         const uint32_t st = sbase + s * kStage;
-        for (int kk = 0; kk < 8; ++kk) {  // K = d 128 in steps of 16
+        for (int i = 0; i < 8; ++i) {  // K = d 128 in steps of 16, kAcc independent chains
+          const int kk = (i % kAcc) * (8 / kAcc) + i / kAcc;
           const uint64_t ad = sdesc(st + kStK + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024);  // K tile, K-major
           const uint64_t bd = sdesc(st + kStQ + (kk >> 2) * 2048 + (kk & 3) * 32, 16, 1024);   // Qpad, K-major
-          tc_mma(tmem + (j & 1) * 16, ad, bd, kIdS, kk > 0 ? 1u : 0u);
+          tc_mma(tmem + (j & 1) * kAcc * 16 + (i % kAcc) * 16, ad, bd, kIdS, i >= kAcc ? 1u : 0u);
         }
         tc_commit(bar(kBarSFull + (j & 1)));
         if (j >= 1) {
@@ -395,7 +416,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
       if (ok) ok = wait_bar(bar(kBarOFull + (jj & 1)), (jj >> 1) & 1, p.status, abort_flag);
       tc_fence_after();
       float v[NQ];
-      tc_ld<NQ>(lane_base + 32 + (jj & 1) * 16, v);
+      tc_ld_sum<NQ>(lane_base + kTmO + (jj & 1) * kAcc * 16, v);
 #pragma unroll
       for (int q = 0; q < NQ; ++q) o[q] = (o[q] + v[q]) * alpha[q];
     };
@@ -409,7 +430,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
       if (ok) ok = wait_bar(bar(kBarSFull + (j & 1)), (j >> 1) & 1, p.status, abort_flag);
       tc_fence_after();
       float sv[NQ];
-      tc_ld<NQ>(lane_base + (j & 1) * 16, sv);
+      tc_ld_sum<NQ>(lane_base + (j & 1) * kAcc * 16, sv);
       tc_fence_before();
       mbar_arrive(bar(kBarSFree + (j & 1)));  // S buffer j % 2 is free again
       // this token's validity
@@ -506,7 +527,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  if (warp == 1) asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(64));
+  if (warp == 1) asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kTmemCols));
 }
 
 PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
