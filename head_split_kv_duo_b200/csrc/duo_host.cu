@@ -94,7 +94,7 @@ bool make_layout(const Cfg &c, const uint8_t *mask, Layout *L) {
   };
   L->status = take(256);
   L->counters = take(static_cast<size_t>(c.B) * c.Hq * 4);
-  L->partials = take(static_cast<size_t>(c.B) * c.Hkv * L->max_splits * c.G * (c.D + 2) * 4);
+  L->partials = take(static_cast<size_t>(c.B) * c.Hkv * L->max_splits * c.G * (c.D + 4) * 4);
   L->hs_max = 0;
   L->layer.resize(c.layers);
   for (int l = 0; l < c.layers; ++l) {

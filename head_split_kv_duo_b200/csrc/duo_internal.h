@@ -57,7 +57,7 @@ struct duo_cache {
   // scratch
   uint32_t *status = nullptr;    // device status word
   uint32_t *counters = nullptr;  // [B][Hq] split-merge tickets
-  float *partials = nullptr;     // [B][Hkv][max_splits][G][d+2]
+  float *partials = nullptr;     // [B][Hkv][max_splits][G][d+4]
   int max_splits = 1;
   char *hist_k = nullptr, *hist_v = nullptr;  // [B][HsMax][S+W][d] pre-fill staging
   int hs_max = 0;

@@ -41,8 +41,8 @@ constexpr int kTmemCols = 4 * kAcc * 16;    // S^T x 2 and O^T x 2, kAcc blocks 
 // shared memory map per stage: K [128][128] (2 swizzle atoms of 16 KiB), V likewise, Q [16][128]
 constexpr int kStK = 0, kStV = 32768, kStQ = 65536, kStage = 65536 + 4096;
 constexpr int kSmP = kStages * kStage;     // 2 x P^T [16][128] bf16 (2 atoms of 2 KiB each)
-constexpr int kSmRed = kSmP + 8192;        // cross-warp reductions [4][16] floats
-constexpr int kSmBar = kSmRed + 1024;
+constexpr int kSmRed = kSmP + 8192;        // cross-warp reductions [4][16] + merge weights [4][kMaxSplits]
+constexpr int kSmBar = kSmRed + (4 * 16 + 4 * kMaxSplits) * 4;
 constexpr int kSmMisc = kSmBar + 256;
 constexpr int kSmemAlloc = kSmMisc + 64 + 1024;
 // Double-buffered resources (S, P, O) each have one barrier per buffer, so that no
@@ -372,15 +372,17 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
       }
       const int seg = blockIdx.x - cfirst;
       const int64_t pitem = static_cast<int64_t>(b) * p.Hkv + g;
-      float *part = p.partials + (pitem * p.max_splits) * G * (kD + 2);
+      // partial row of (segment, query head): o[0..d), m at d, l at d+1 (16-byte aligned rows)
+      constexpr int kRow = kD + 4;
+      float *part = p.partials + (pitem * p.max_splits) * G * kRow;
 #pragma unroll
       for (int q = 0; q < NQ; ++q)
         if (q < G) {
-          float *dst = part + (static_cast<int64_t>(seg) * G + q) * (kD + 2);
-          dst[2 + t] = o[q];
+          float *dst = part + (static_cast<int64_t>(seg) * G + q) * kRow;
+          dst[t] = o[q];
           if (t == 0) {
-            dst[0] = m[q];
-            dst[1] = lt[q];
+            dst[kD] = m[q];
+            dst[kD + 1] = lt[q];
           }
         }
       __threadfence();
@@ -392,22 +394,44 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
       named_sync(1, 128);
       if (!*last_flag) return;
       __threadfence();
-#pragma unroll
-      for (int q = 0; q < NQ; ++q)
-        if (q < G) {
-          float M = -INFINITY;
-          for (int sg = 0; sg < nseg; ++sg) M = fmaxf(M, __ldcg(part + (static_cast<int64_t>(sg) * G + q) * (kD + 2)));
-          float num = 0.f, den = 0.f;
-          for (int sg = 0; sg < nseg; ++sg) {
-            const float *r = part + (static_cast<int64_t>(sg) * G + q) * (kD + 2);
-            const float ms = __ldcg(r);
-            const float w = (ms == -INFINITY) ? 0.f : ex2(ms - M);
-            den = fmaf(w, __ldcg(r + 1), den);
-            num = fmaf(w, __ldcg(r + 2 + t), num);
-          }
-          Elem<__nv_bfloat16>::store(p.out, (static_cast<int64_t>(b) * p.Hq + h0 + q) * kD + t, num / den);
-          if (t == 0 && p.lse) p.lse[b * p.Hq + h0 + q] = (M + lg2(den)) * kLn2;
+      // merge: warp wq takes query heads wq, wq+4, ...; its lanes read segments in
+      // parallel for the max and the normaliser, then stream the output rows (4 dims a lane)
+      float *wts = red + 4 * kN + wq * kMaxSplits;
+      for (int q = wq; q < G; q += 4) {
+        const float *base = part + static_cast<int64_t>(q) * kRow;
+        const int64_t sstride = static_cast<int64_t>(G) * kRow;
+        float M = -INFINITY;
+        for (int sg = lane; sg < nseg; sg += 32) M = fmaxf(M, __ldcg(base + sg * sstride + kD));
+        M = warp_max(M);
+        float den = 0.f;
+        for (int sg = lane; sg < nseg; sg += 32) {
+          const float ms = __ldcg(base + sg * sstride + kD);
+          const float e = (ms == -INFINITY) ? 0.f : ex2(ms - M);
+          wts[sg] = e;
+          den = fmaf(e, __ldcg(base + sg * sstride + kD + 1), den);
         }
+        den = warp_sum(den);
+        __syncwarp();
+        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll 4
+        for (int sg = 0; sg < nseg; ++sg) {
+          const float w = wts[sg];
+          const float4 v = __ldcg(reinterpret_cast<const float4 *>(base + sg * sstride) + lane);
+          acc.x = fmaf(w, v.x, acc.x);
+          acc.y = fmaf(w, v.y, acc.y);
+          acc.z = fmaf(w, v.z, acc.z);
+          acc.w = fmaf(w, v.w, acc.w);
+        }
+        const float inv = 1.f / den;
+        const __nv_bfloat162 lo = __floats2bfloat162_rn(acc.x * inv, acc.y * inv);
+        const __nv_bfloat162 hi = __floats2bfloat162_rn(acc.z * inv, acc.w * inv);
+        uint2 pk;
+        pk.x = *reinterpret_cast<const uint32_t *>(&lo);
+        pk.y = *reinterpret_cast<const uint32_t *>(&hi);
+        *reinterpret_cast<uint2 *>(p.out + ((static_cast<int64_t>(b) * p.Hq + h0 + q) * kD + 4 * lane) * 2) = pk;
+        if (lane == 0 && p.lse) p.lse[b * p.Hq + h0 + q] = (M + lg2(den)) * kLn2;
+        __syncwarp();
+      }
       if (t == 0) p.counters[pitem] = 0u;
     };
 

@@ -9,17 +9,17 @@
 //     the chunk's own keys, with the Lambda mask j < S or i - j < W.  Key tiles that
 //     hold no visible key for any row of a query tile are never loaded (tile skip).
 //
-// One CTA = one 128-row query tile of one (batch, query head); 6 warps:
+// One CTA = one 128-row query tile of one (batch, query head); 10 warps:
 //   warp 0      TMA producer: Q once, then K/V tiles of 128 keys into a 2-stage ring
 //   warp 1      TMEM allocator; lane 0 issues every tcgen05.mma
-//   warps 2..5  softmax warpgroup: thread t owns query row t (TMEM lane t)
-// TMEM (512 columns): S double buffer at columns 0 and 128, O double buffer at 256 and 384.
+//   warps 2..9  softmax: two threads per query row (TMEM lane), 64 columns each
+// TMEM (512 columns): S double buffer at columns 0 and 128, O accumulator at 256.
 //   S_j = Q K_j^T      (M 128, N 128, K 128: 8 MMAs of K 16), into S[j % 2]
-//   O_j = P_j V_j      (M 128, N 128, K 128 keys) into O[j % 2], P_j from shared memory
-// The softmax warps read S_j twice from TMEM (row max, then probabilities), write
-// P_j (bf16) over K_j in its stage (128B-swizzled K-major), and only then fold O_{j-1}
-// into fp32 registers with the online-softmax rescale, so the tensor core computes
-// S_{j+1} and P_j V_j while the softmax warps work.
+//   O += P_j V_j       (M 128, N 128, K 128 keys), P_j from shared memory
+// The softmax warps read S_j twice from TMEM (row max, then probabilities) and write
+// P_j (bf16) over K_j in its stage (128B-swizzled K-major); O stays in TMEM and is
+// rescaled there only when a row's maximum grows past its reference by 2^8, so the
+// tensor core computes S_{j+1} and P_j V_j while the softmax warps work.
 //
 // Every mbarrier wait is bounded; a wait that runs out latches kDevTimeout in the
 // status word and sets an abort flag so that every role drains and exits.
@@ -32,7 +32,7 @@ namespace duo {
 
 namespace {
 
-constexpr int kTcThreads = 192;
+constexpr int kTcThreads = 320;  // warp 0 TMA, warp 1 MMA + TMEM, warps 2-9 softmax
 constexpr int kBM = 128;  // query rows per tile
 constexpr int kBN = 128;  // keys per tile
 constexpr int kD = 128;
@@ -46,14 +46,15 @@ constexpr int kSmKV = 32768;               // stage s: K at +s*65536, V at +s*65
 // been computed, so P is double-buffered along with the K/V stages.
 constexpr int kSmBar = kSmKV + kKvStages * 65536;
 constexpr int kSmMisc = kSmBar + 256;
-constexpr int kSmTotal = kSmMisc + 1024 + kMaxStrmTiles * 16;
+constexpr int kSmXchg = kSmMisc + 1024 + kMaxStrmTiles * 16;  // row max / sum exchange, 6 x 128 floats
+constexpr int kSmTotal = kSmXchg + 6 * 128 * 4;
 constexpr int kSmemAlloc = kSmTotal + 1024;  // slack for aligning the base to 1 KiB
 
 // barrier indices (8 bytes each)
 // Double-buffered resources (S, P, O) have one barrier per buffer, so that no barrier
 // can complete two phases ahead of a thread waiting on it (parity waits).
 constexpr int kBarQ = 0, kBarKvFull = 1, kBarKvEmpty = 3, kBarSFull = 5, kBarSFree = 7, kBarPFull = 9, kBarOFull = 11,
-              kBarDrain = 13, kNumBars = 14;
+              kBarDrain = 12, kNumBars = 13;
 
 struct TileDesc {
   int src;      // 0 retrieval cache, 1 streaming history, 2 chunk input
@@ -116,6 +117,25 @@ __device__ __forceinline__ void tc_ld32(uint32_t taddr, float (&v)[32]) {
 #pragma unroll
   for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
 }
+
+// store 32 consecutive fp32 columns of this thread's TMEM lane, and wait for it
+__device__ __forceinline__ void tc_st32(uint32_t taddr, const float (&v)[32]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "
+      "{%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16, "
+      "%17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31, %32};" ::"r"(taddr),
+      "r"(__float_as_uint(v[0])), "r"(__float_as_uint(v[1])), "r"(__float_as_uint(v[2])), "r"(__float_as_uint(v[3])),
+      "r"(__float_as_uint(v[4])), "r"(__float_as_uint(v[5])), "r"(__float_as_uint(v[6])), "r"(__float_as_uint(v[7])),
+      "r"(__float_as_uint(v[8])), "r"(__float_as_uint(v[9])), "r"(__float_as_uint(v[10])), "r"(__float_as_uint(v[11])),
+      "r"(__float_as_uint(v[12])), "r"(__float_as_uint(v[13])), "r"(__float_as_uint(v[14])), "r"(__float_as_uint(v[15])),
+      "r"(__float_as_uint(v[16])), "r"(__float_as_uint(v[17])), "r"(__float_as_uint(v[18])), "r"(__float_as_uint(v[19])),
+      "r"(__float_as_uint(v[20])), "r"(__float_as_uint(v[21])), "r"(__float_as_uint(v[22])), "r"(__float_as_uint(v[23])),
+      "r"(__float_as_uint(v[24])), "r"(__float_as_uint(v[25])), "r"(__float_as_uint(v[26])), "r"(__float_as_uint(v[27])),
+      "r"(__float_as_uint(v[28])), "r"(__float_as_uint(v[29])), "r"(__float_as_uint(v[30])), "r"(__float_as_uint(v[31]))
+      : "memory");
+  asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void named_sync(int id, int n) { asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory"); }
 
 // Shared-memory matrix descriptor, 128-byte swizzle (sm_100 layout: start >> 4 at
 // bit 0, leading byte offset >> 4 at bit 16, stride byte offset >> 4 at bit 32,
@@ -234,7 +254,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) prefill_tc_kernel(const __grid_
 
   if (tid == 0) {
     for (int i = 0; i < kNumBars; ++i)
-      mbar_init(bar(i), (i == kBarSFree || i == kBarSFree + 1 || i == kBarPFull || i == kBarPFull + 1) ? 128 : 1);
+      mbar_init(bar(i), (i == kBarSFree || i == kBarSFree + 1 || i == kBarPFull || i == kBarPFull + 1) ? 256 : 1);
     fence_mbar_init();
     *abort_flag = 0;
     int nt;
@@ -303,9 +323,9 @@ __global__ void __launch_bounds__(kTcThreads, 1) prefill_tc_kernel(const __grid_
         for (int kk = 0; kk < 8; ++kk) {
           const uint64_t ad = sdesc(sbase + kSmKV + s * 65536 + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024);
           const uint64_t bd = sdesc(vbase + kk * 2048, 16384, 1024);
-          tc_mma(tmem + 256 + (jj & 1) * 128, ad, bd, kIdPV, kk > 0 ? 1u : 0u);
+          tc_mma(tmem + 256, ad, bd, kIdPV, (jj > 0 || kk > 0) ? 1u : 0u);  // O accumulates over tiles
         }
-        tc_commit(bar(kBarOFull + (jj & 1)));
+        tc_commit(bar(kBarOFull));
         tc_commit(bar(kBarKvEmpty + s));
       };
       for (int j = 0; j < nt && ok; ++j) {
@@ -336,16 +356,21 @@ __global__ void __launch_bounds__(kTcThreads, 1) prefill_tc_kernel(const __grid_
       mbar_wait(bar(kBarDrain), 0, p.status);
     }
   } else {
-    // ================= softmax warpgroup =================
-    const int row = ((warp & 3) << 5) | lane;             // TMEM lane == query row of the tile
-    const uint32_t lane_base = tmem + (static_cast<uint32_t>((warp & 3) << 5) << 16);
-    const int64_t i = pl.q0 + row;                         // absolute query position
+    // ================= softmax: 8 warps, two threads per query row =================
+    // Warp w reads TMEM lanes 32*(w%4).. (rows) and columns [64*half, 64*half+64) of S
+    // and of O.  The running max m is a reference: P = exp2(s*c - m) may exceed 1 by up to
+    // 2^kSlack, and m (with O in TMEM and l) is rescaled only when a row's tile maximum
+    // passes m + kSlack.  O accumulates in TMEM across tiles.
+    constexpr float kSlack = 8.0f;
+    const int wq = warp & 3;
+    const int half = (warp - 2) >> 2;
+    const int row = (wq << 5) | lane;
+    const uint32_t lane_base = tmem + (static_cast<uint32_t>(wq << 5) << 16);
+    const int64_t i = pl.q0 + row;  // absolute query position
     const float c = p.scale_log2;
-    float o[kD];
-#pragma unroll
-    for (int e = 0; e < kD; ++e) o[e] = 0.f;
-    float m = -INFINITY, l = 0.f, alpha_prev = 1.f;
+    float m = -INFINITY, l = 0.f;
     const int rsw = row & 7;
+    float *xch = reinterpret_cast<float *>(smem + kSmXchg);  // [tile parity][half][row] partial maxima
     bool ok = true;
 
     for (int j = 0; j < nt; ++j) {
@@ -378,13 +403,13 @@ __global__ void __launch_bounds__(kTcThreads, 1) prefill_tc_kernel(const __grid_
 
       if (ok) ok = wait_bar(bar(kBarSFull + (j & 1)), (j >> 1) & 1, p.status, abort_flag);
       tc_fence_after();
-      const uint32_t sbuf = lane_base + (j & 1) * 128;
-      // pass 1: row max of the visible logits (8 independent partial maxima)
+      const uint32_t sbuf = lane_base + (j & 1) * 128 + half * 64;
+      // pass 1: maximum of the visible logits in this thread's 64 columns
       float mx8[8];
 #pragma unroll
       for (int u = 0; u < 8; ++u) mx8[u] = -INFINITY;
 #pragma unroll 1
-      for (int cc = 0; cc < 4; ++cc) {
+      for (int cc = 0; cc < 2; ++cc) {
         float v[32];
         tc_ld32(sbuf + cc * 32, v);
         if (full_vis) {
@@ -393,41 +418,74 @@ __global__ void __launch_bounds__(kTcThreads, 1) prefill_tc_kernel(const __grid_
         } else {
 #pragma unroll
           for (int e = 0; e < 32; ++e) {
-            const int col = cc * 32 + e;
+            const int col = half * 64 + cc * 32 + e;
             const bool vis = col <= hi && (col < sink_c || col > win_c);
             mx8[e & 7] = vis ? fmaxf(mx8[e & 7], v[e]) : mx8[e & 7];
           }
         }
       }
-      const float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
-                             fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
-      const float m_new = fmaxf(m, mx * c);
-      const bool none = (m_new == -INFINITY);
-      const float alpha = none ? 1.f : ex2(m - m_new);
-
-      // pass 2: probabilities, row sum, bf16 P over K_j in stage j % 2
-      char *prow = smem + kSmKV + (j % kKvStages) * 65536 + row * 128;
+      float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
+                       fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
+      xch[((j & 1) * 2 + half) * kBM + row] = mx;
+      named_sync(1, 256);
+      mx = fmaxf(mx, xch[((j & 1) * 2 + (half ^ 1)) * kBM + row]);
+      const float tmax = mx * c;  // -inf when nothing in the tile is visible
+      const bool need = tmax > m + kSlack;
+      float alpha = 1.f;
+      if (need) {
+        alpha = ex2(m - tmax);  // 0 while m is -inf
+        m = tmax;
+      }
+      l *= alpha;
+      bool waited = false;
+      if (j >= 1 && __any_sync(0xffffffffu, need)) {
+        // rescale this thread's 64 columns of O once P_{j-1} V_{j-1} has landed
+        if (ok) ok = wait_bar(bar(kBarOFull), (j - 1) & 1, p.status, abort_flag);
+        tc_fence_after();
+#pragma unroll 1
+        for (int cc = 0; cc < 2; ++cc) {
+          float v[32];
+          const uint32_t oa = lane_base + 256 + half * 64 + cc * 32;
+          tc_ld32(oa, v);
+#pragma unroll
+          for (int e = 0; e < 32; ++e) v[e] *= alpha;
+          tc_st32(oa, v);
+        }
+        waited = true;
+      }
+      // pass 2: probabilities, row sum, bf16 P over K_j in stage j % 2 (this thread's half)
+      char *prow = smem + kSmKV + (j % kKvStages) * 65536 + half * 16384 + row * 128;
       float rs8[8];
 #pragma unroll
       for (int u = 0; u < 8; ++u) rs8[u] = 0.f;
-      const float mc = none ? 0.f : m_new;
+      const float mc = (m == -INFINITY) ? 0.f : m;
 #pragma unroll 1
-      for (int cc = 0; cc < 4; ++cc) {
+      for (int cc = 0; cc < 2; ++cc) {
         float v[32];
         tc_ld32(sbuf + cc * 32, v);
         uint32_t pk[16];
-        if (full_vis && cc == 3) {
-          // a quarter of the exponentials on the FMA pipe, the rest on the MUFU unit
+        if (full_vis) {
+          // a quarter of the exponentials (16 of this thread's 64) on the FMA pipe, the rest
+          // on the MUFU unit
+          if (cc == half) {
 #pragma unroll
-          for (int e = 0; e < 32; e += 2) {
-            const float p0 = exp2_poly(fmaf(v[e], c, -mc)), p1 = exp2_poly(fmaf(v[e + 1], c, -mc));
-            rs8[(e >> 1) & 7] += p0 + p1;
-            const __nv_bfloat162 pb = __floats2bfloat162_rn(p0, p1);
-            pk[e >> 1] = *reinterpret_cast<const uint32_t *>(&pb);
+            for (int e = 0; e < 16; e += 2) {
+              const float p0 = exp2_poly(fmaf(v[e], c, -mc)), p1 = exp2_poly(fmaf(v[e + 1], c, -mc));
+              rs8[(e >> 1) & 7] += p0 + p1;
+              const __nv_bfloat162 pb = __floats2bfloat162_rn(p0, p1);
+              pk[e >> 1] = *reinterpret_cast<const uint32_t *>(&pb);
+            }
+          } else {
+#pragma unroll
+            for (int e = 0; e < 16; e += 2) {
+              const float p0 = ex2(fmaf(v[e], c, -mc)), p1 = ex2(fmaf(v[e + 1], c, -mc));
+              rs8[(e >> 1) & 7] += p0 + p1;
+              const __nv_bfloat162 pb = __floats2bfloat162_rn(p0, p1);
+              pk[e >> 1] = *reinterpret_cast<const uint32_t *>(&pb);
+            }
           }
-        } else if (full_vis) {
 #pragma unroll
-          for (int e = 0; e < 32; e += 2) {
+          for (int e = 16; e < 32; e += 2) {
             const float p0 = ex2(fmaf(v[e], c, -mc)), p1 = ex2(fmaf(v[e + 1], c, -mc));
             rs8[(e >> 1) & 7] += p0 + p1;
             const __nv_bfloat162 pb = __floats2bfloat162_rn(p0, p1);
@@ -436,7 +494,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) prefill_tc_kernel(const __grid_
         } else {
 #pragma unroll
           for (int e = 0; e < 32; e += 2) {
-            const int c0 = cc * 32 + e, c1 = c0 + 1;
+            const int c0 = half * 64 + cc * 32 + e, c1 = c0 + 1;
             const bool v0 = c0 <= hi && (c0 < sink_c || c0 > win_c);
             const bool v1 = c1 <= hi && (c1 < sink_c || c1 > win_c);
             const float p0 = v0 ? ex2(fmaf(v[e], c, -mc)) : 0.f;
@@ -446,64 +504,53 @@ __global__ void __launch_bounds__(kTcThreads, 1) prefill_tc_kernel(const __grid_
             pk[e >> 1] = *reinterpret_cast<const uint32_t *>(&pb);
           }
         }
-        // columns cc*32 .. cc*32+31 -> half (cc >> 1), 16-byte chunks 4*(cc&1) .. +3
-        char *half = prow + (cc >> 1) * 16384;
+        // columns 64*half + 32*cc .. +31 -> 16-byte chunks 4*cc .. 4*cc+3 of this half
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
-          const int chunk = ((cc & 1) * 4 + q) ^ rsw;
-          *reinterpret_cast<uint4 *>(half + chunk * 16) = make_uint4(pk[4 * q], pk[4 * q + 1], pk[4 * q + 2], pk[4 * q + 3]);
+          const int chunk = (cc * 4 + q) ^ rsw;
+          *reinterpret_cast<uint4 *>(prow + chunk * 16) = make_uint4(pk[4 * q], pk[4 * q + 1], pk[4 * q + 2], pk[4 * q + 3]);
         }
       }
       tc_fence_before();
       mbar_arrive(bar(kBarSFree + (j & 1)));  // S buffer j % 2 may be overwritten
+      // one wait per P V product, in order (here unless the rescale already waited)
+      if (j >= 1 && !waited) {
+        if (ok) ok = wait_bar(bar(kBarOFull), (j - 1) & 1, p.status, abort_flag);
+      }
+      l += ((rs8[0] + rs8[1]) + (rs8[2] + rs8[3])) + ((rs8[4] + rs8[5]) + (rs8[6] + rs8[7]));
       fence_async_smem();  // P visible to the tensor core
       tc_fence_before();
       mbar_arrive(bar(kBarPFull + (j & 1)));
-      // fold O_{j-1} (scale m_{j-1}) into the registers while the tensor core works on P_j
-      if (j >= 1) {
-        if (ok) ok = wait_bar(bar(kBarOFull + ((j - 1) & 1)), ((j - 1) >> 1) & 1, p.status, abort_flag);
-        tc_fence_after();
+    }
+    // the last product, then the row's normaliser from both halves
+    if (nt > 0 && ok) ok = wait_bar(bar(kBarOFull), (nt - 1) & 1, p.status, abort_flag);
+    tc_fence_after();
+    float *xl = xch + 4 * kBM;  // [half][row]
+    xl[half * kBM + row] = l;
+    named_sync(1, 256);
+    const float lrow = l + xl[(half ^ 1) * kBM + row];
+    // epilogue: normalise and store this thread's 64 dims of the row (bf16) and its lse
+    const bool store = r0 + row < p.n;
+    char *orow = p.out + ((static_cast<int64_t>(b) * p.n + r0 + row) * p.Hq + h) * (kD * 2) + half * 128;
+    const float inv = 1.f / lrow;
+#pragma unroll 1
+    for (int cc = 0; cc < 2; ++cc) {
+      float v[32];
+      tc_ld32(lane_base + 256 + half * 64 + cc * 32, v);
+      if (store) {
 #pragma unroll
-        for (int cc = 0; cc < 4; ++cc) {
-          float v[32];
-          tc_ld32(lane_base + 256 + ((j - 1) & 1) * 128 + cc * 32, v);
+        for (int q = 0; q < 4; ++q) {
+          uint32_t w[4];
 #pragma unroll
-          for (int e = 0; e < 32; ++e) o[cc * 32 + e] = fmaf(o[cc * 32 + e], alpha_prev, v[e]);
+          for (int e = 0; e < 4; ++e) {
+            const __nv_bfloat162 pb = __floats2bfloat162_rn(v[8 * q + 2 * e] * inv, v[8 * q + 2 * e + 1] * inv);
+            w[e] = *reinterpret_cast<const uint32_t *>(&pb);
+          }
+          *reinterpret_cast<uint4 *>(orow + cc * 64 + q * 16) = make_uint4(w[0], w[1], w[2], w[3]);
         }
       }
-      const float rs = ((rs8[0] + rs8[1]) + (rs8[2] + rs8[3])) + ((rs8[4] + rs8[5]) + (rs8[6] + rs8[7]));
-      l = fmaf(l, alpha, rs);
-      m = m_new;
-      alpha_prev = alpha;
     }
-    // last O tile
-    if (nt > 0) {
-      if (ok) ok = wait_bar(bar(kBarOFull + ((nt - 1) & 1)), ((nt - 1) >> 1) & 1, p.status, abort_flag);
-      tc_fence_after();
-#pragma unroll
-      for (int cc = 0; cc < 4; ++cc) {
-        float v[32];
-        tc_ld32(lane_base + 256 + ((nt - 1) & 1) * 128 + cc * 32, v);
-#pragma unroll
-        for (int e = 0; e < 32; ++e) o[cc * 32 + e] = fmaf(o[cc * 32 + e], alpha_prev, v[e]);
-      }
-    }
-    // epilogue: normalise and store the row (bf16) and its lse
-    if (r0 + row < p.n) {
-      const float inv = 1.f / l;
-      char *orow = p.out + ((static_cast<int64_t>(b) * p.n + r0 + row) * p.Hq + h) * (kD * 2);
-#pragma unroll
-      for (int q = 0; q < kD / 8; ++q) {
-        uint32_t w[4];
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const __nv_bfloat162 pb = __floats2bfloat162_rn(o[8 * q + 2 * e] * inv, o[8 * q + 2 * e + 1] * inv);
-          w[e] = *reinterpret_cast<const uint32_t *>(&pb);
-        }
-        *reinterpret_cast<uint4 *>(orow + q * 16) = make_uint4(w[0], w[1], w[2], w[3]);
-      }
-      if (p.lse) p.lse[(static_cast<int64_t>(b) * p.n + r0 + row) * p.Hq + h] = (m + lg2(l)) * kLn2;
-    }
+    if (store && half == 0 && p.lse) p.lse[(static_cast<int64_t>(b) * p.n + r0 + row) * p.Hq + h] = (m + lg2(lrow)) * kLn2;
   }
 
   tc_fence_before();

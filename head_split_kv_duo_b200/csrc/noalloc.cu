@@ -86,11 +86,11 @@ extern "C" duo_status duo_decode_attention_static_scratch(duo_cache *c, int laye
   if (!decode_tc_supported(p, c->dtype, int4)) return DUO_ERR_UNSUPPORTED;
 
   // Scratch layout: tickets [B][Hkv] (256-byte padded), then partials
-  // [B][Hkv][ctas][G][d+2] floats.  Fewer CTAs are used when the partials of one
+  // [B][Hkv][ctas][G][d+4] floats.  Fewer CTAs are used when the partials of one
   // CTA per SM would not fit; a cache with more heads than fit at one CTA is refused.
   const size_t items = static_cast<size_t>(c->B) * c->Hkv;
   const size_t ticket_bytes = (items * 4 + 255) / 256 * 256;
-  const size_t per_cta = items * c->G * (static_cast<size_t>(c->D) + 2) * 4;
+  const size_t per_cta = items * c->G * (static_cast<size_t>(c->D) + 4) * 4;
   if (ticket_bytes >= kStaticScratchBytes || per_cta > kStaticScratchBytes - ticket_bytes) return DUO_ERR_CAPACITY;
   size_t ctas = (kStaticScratchBytes - ticket_bytes) / per_cta;
   if (ctas > static_cast<size_t>(c->num_sms)) ctas = static_cast<size_t>(c->num_sms);
