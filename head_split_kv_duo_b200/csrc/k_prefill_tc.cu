@@ -179,10 +179,10 @@ struct Plan {
 
 // Streaming heads: which history / chunk tiles hold a visible key for some row of
 // the query tile.  Writes the list into `tl` and returns its length.
-__device__ int streaming_tiles(const PrefillParams &p, int r0, TileDesc *tl) {
+__device__ int streaming_tiles(const PrefillParams &p, int r0, int npos, TileDesc *tl) {
   int nt = 0;
   const int64_t qlo = p.len + r0;                                      // smallest query position
-  const int rows_hi = (r0 + kBM < p.n) ? r0 + kBM : p.n;                // chunk rows this tile needs
+  const int rows_hi = (r0 + npos < p.n) ? r0 + npos : p.n;              // chunk rows this block needs
   const int hrows = p.hs + p.hw;
   const int nh = (hrows + kBN - 1) / kBN;
   for (int t = 0; t < nh && nt < kMaxStrmTiles; ++t) {
@@ -241,12 +241,16 @@ __global__ void __launch_bounds__(kTcThreads, 1) prefill_tc_kernel(const __grid_
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
 
   // ---- which query tile ----
-  const int ntq = (p.n + kBM - 1) / kBM;
-  const int bh = blockIdx.x % (p.B * p.Hq);
-  const int qt = ntq - 1 - blockIdx.x / (p.B * p.Hq);  // heaviest (latest) tiles first
-  const int b = bh / p.Hq, h = bh % p.Hq;
-  const int g = h / p.G;
-  const int r0 = qt * kBM;
+  // GQA packing: the 128 rows of the tile are npos = 128 / G consecutive positions x the
+  // G query heads of one KV head (row r = position r / G, head r % G), so every K/V tile
+  // a CTA loads serves the whole group.
+  const int G = p.G;
+  const int npos = kBM / G;
+  const int ntq = (p.n + npos - 1) / npos;
+  const int bg = blockIdx.x % (p.B * p.Hkv);
+  const int qt = ntq - 1 - blockIdx.x / (p.B * p.Hkv);  // heaviest (latest) blocks first
+  const int b = bg / p.Hkv, g = bg % p.Hkv;
+  const int r0 = qt * npos;  // first chunk row (position offset) of the block
   Plan pl;
   pl.retr = p.hm.is_retr[g] != 0;
   pl.q0 = p.len + r0;
@@ -259,10 +263,10 @@ __global__ void __launch_bounds__(kTcThreads, 1) prefill_tc_kernel(const __grid_
     *abort_flag = 0;
     int nt;
     if (pl.retr) {
-      const int64_t last = pl.q0 + ((r0 + kBM < p.n) ? kBM : p.n - r0) - 1;  // last key position needed
+      const int64_t last = pl.q0 + ((r0 + npos < p.n) ? npos : p.n - r0) - 1;  // last key position needed
       nt = static_cast<int>(last / kBN) + 1;
     } else {
-      nt = streaming_tiles(p, r0, tl);
+      nt = streaming_tiles(p, r0, npos, tl);
     }
     *ntiles_sm = nt;
   }
@@ -284,8 +288,8 @@ __global__ void __launch_bounds__(kTcThreads, 1) prefill_tc_kernel(const __grid_
       const CUtensorMap *mk = pl.retr ? &a.tm_kc : &a.tm_kh;
       prefetch_map(mk);
       mbar_expect_tx(bar(kBarQ), 32768);
-      tma_4d(sbase + kSmQ, &a.tm_q, 0, h, r0, b, bar(kBarQ));
-      tma_4d(sbase + kSmQ + 16384, &a.tm_q, 64, h, r0, b, bar(kBarQ));
+      tma_4d(sbase + kSmQ, &a.tm_q, 0, g * G, r0, b, bar(kBarQ));  // box: 64 dims x G heads x npos positions
+      tma_4d(sbase + kSmQ + 16384, &a.tm_q, 64, g * G, r0, b, bar(kBarQ));
       for (int j = 0; j < nt; ++j) {
         const int s = j % kKvStages;
         if (j >= kKvStages && !wait_bar(bar(kBarKvEmpty + s), ((j / kKvStages) - 1) & 1, p.status, abort_flag)) break;
@@ -366,7 +370,9 @@ __global__ void __launch_bounds__(kTcThreads, 1) prefill_tc_kernel(const __grid_
     const int half = (warp - 2) >> 2;
     const int row = (wq << 5) | lane;
     const uint32_t lane_base = tmem + (static_cast<uint32_t>(wq << 5) << 16);
-    const int64_t i = pl.q0 + row;  // absolute query position
+    const int rpos = row / G;                  // position offset of this row within the block
+    const int h = g * G + row % G;             // its query head
+    const int64_t i = pl.q0 + rpos;            // absolute query position
     const float c = p.scale_log2;
     float m = -INFINITY, l = 0.f;
     const int rsw = row & 7;
@@ -530,8 +536,8 @@ __global__ void __launch_bounds__(kTcThreads, 1) prefill_tc_kernel(const __grid_
     named_sync(1, 256);
     const float lrow = l + xl[(half ^ 1) * kBM + row];
     // epilogue: normalise and store this thread's 64 dims of the row (bf16) and its lse
-    const bool store = r0 + row < p.n;
-    char *orow = p.out + ((static_cast<int64_t>(b) * p.n + r0 + row) * p.Hq + h) * (kD * 2) + half * 128;
+    const bool store = r0 + rpos < p.n;
+    char *orow = p.out + ((static_cast<int64_t>(b) * p.n + r0 + rpos) * p.Hq + h) * (kD * 2) + half * 128;
     const float inv = 1.f / lrow;
 #pragma unroll 1
     for (int cc = 0; cc < 2; ++cc) {
@@ -550,7 +556,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) prefill_tc_kernel(const __grid_
         }
       }
     }
-    if (store && half == 0 && p.lse) p.lse[(static_cast<int64_t>(b) * p.n + r0 + row) * p.Hq + h] = (m + lg2(lrow)) * kLn2;
+    if (store && half == 0 && p.lse) p.lse[(static_cast<int64_t>(b) * p.n + r0 + rpos) * p.Hq + h] = (m + lg2(lrow)) * kLn2;
   }
 
   tc_fence_before();
@@ -597,6 +603,7 @@ bool make_map(CUtensorMap *m, const void *base, int rank, const uint64_t *dims, 
 
 bool prefill_tc_supported(const PrefillParams &p, duo_dtype dt) {
   if (dt != DUO_BF16 || p.D != kD) return false;
+  if (p.G < 1 || p.G > kBM || (p.G & (p.G - 1)) != 0) return false;  // the group must tile 128 rows
   if (encode_fn() == nullptr) return false;
   // streaming tile list must fit: history tiles + window tiles + a sink tile
   const int hist_tiles = (p.hs + p.hw + kBN - 1) / kBN;
@@ -610,10 +617,10 @@ cudaError_t launch_prefill_tc(const PrefillParams &p, cudaStream_t st) {
   a.p = p;
   const uint64_t row = kD * 2;
   bool ok = true;
-  {  // q [B][n][Hq][d]
+  {  // q [B][n][Hq][d]; box = 64 dims x G heads x 128/G positions (one GQA group)
     const uint64_t d[4] = {kD, static_cast<uint64_t>(p.Hq), static_cast<uint64_t>(p.n), static_cast<uint64_t>(p.B)};
     const uint64_t s[3] = {row, row * p.Hq, row * p.Hq * p.n};
-    const uint32_t bx[4] = {64, 1, kBM, 1};
+    const uint32_t bx[4] = {64, static_cast<uint32_t>(p.G), static_cast<uint32_t>(kBM / p.G), 1};
     ok &= make_map(&a.tm_q, p.q, 4, d, s, bx);
   }
   {  // chunk k, v [B][n][Hkv][d]
@@ -644,8 +651,9 @@ cudaError_t launch_prefill_tc(const PrefillParams &p, cudaStream_t st) {
     if (e != cudaSuccess) return e;
     attr = true;
   }
-  const int ntq = (p.n + kBM - 1) / kBM;
-  const int grid = ntq * p.B * p.Hq;
+  const int npos = kBM / p.G;
+  const int ntq = (p.n + npos - 1) / npos;
+  const int grid = ntq * p.B * p.Hkv;
   prefill_tc_kernel<<<grid, kTcThreads, kSmemAlloc, st>>>(a);
   return cudaGetLastError();
 }
