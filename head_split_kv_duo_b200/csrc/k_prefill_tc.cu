@@ -9,17 +9,20 @@
 //     the chunk's own keys, with the Lambda mask j < S or i - j < W.  Key tiles that
 //     hold no visible key for any row of a query tile are never loaded (tile skip).
 //
-// One CTA = one 128-row query tile of one (batch, query head); 10 warps:
-//   warp 0      TMA producer: Q once, then K/V tiles of 128 keys into a 2-stage ring
+// One CTA = one 128-row query tile (a GQA group of heads x 128/G positions); 11 warps:
+//   warp 0      TMA producer: Q once, then K tiles of 128 keys into a 3-stage ring
+//   warp 10     TMA producer: V tiles into a 2-stage ring
 //   warp 1      TMEM allocator; lane 0 issues every tcgen05.mma
 //   warps 2..9  softmax: two threads per query row (TMEM lane), 64 columns each
-// TMEM (512 columns): S double buffer at columns 0 and 128, O accumulator at 256.
+// TMEM (512 columns): S double buffer at 0 and 128, O accumulator at 256, P (bf16
+// pairs) double buffer at 384 and 448.
 //   S_j = Q K_j^T      (M 128, N 128, K 128: 8 MMAs of K 16), into S[j % 2]
-//   O += P_j V_j       (M 128, N 128, K 128 keys), P_j from shared memory
-// The softmax warps read S_j twice from TMEM (row max, then probabilities) and write
-// P_j (bf16) over K_j in its stage (128B-swizzled K-major); O stays in TMEM and is
-// rescaled there only when a row's maximum grows past its reference by 2^8, so the
-// tensor core computes S_{j+1} and P_j V_j while the softmax warps work.
+//   O += P_j V_j       (M 128, N 128, K 128 keys), A = P_j from TMEM, B = V_j (smem)
+// The softmax warps read S_j once from TMEM, release it, and write P_j (bf16) back
+// into TMEM; O stays in TMEM and is rescaled there only when a row's maximum grows
+// past its reference by 2^8.  K stages are released as soon as S_j is computed and V
+// stages once P_j V_j is, so the tensor core computes S_{j+1} and P_j V_j while the
+// softmax warps work.
 //
 // Every mbarrier wait is bounded; a wait that runs out latches kDevTimeout in the
 // status word and sets an abort flag so that every role drains and exits.
@@ -32,29 +35,33 @@ namespace duo {
 
 namespace {
 
-constexpr int kTcThreads = 320;  // warp 0 TMA, warp 1 MMA + TMEM, warps 2-9 softmax
+constexpr int kTcThreads = 352;  // warp 0 K/Q TMA, warp 1 MMA + TMEM, warps 2-9 softmax, warp 10 V TMA
 constexpr int kBM = 128;  // query rows per tile
 constexpr int kBN = 128;  // keys per tile
 constexpr int kD = 128;
-constexpr int kKvStages = 2;
+constexpr int kKStages = 3;  // K ring: a stage is free once S_j is computed
+constexpr int kVStages = 2;  // V ring: a stage is free once P_j V_j is computed
 constexpr int kMaxStrmTiles = 48;
 
-// shared memory map (bytes from the 1 KiB-aligned base)
-constexpr int kSmQ = 0;                    // 2 x [128][64] bf16, 128B swizzle
-constexpr int kSmKV = 32768;               // stage s: K at +s*65536, V at +s*65536+32768
-// P_j (bf16, 128B-swizzled K-major) is written over K_j in its own stage once S_j has
-// been computed, so P is double-buffered along with the K/V stages.
-constexpr int kSmBar = kSmKV + kKvStages * 65536;
+// shared memory map (bytes from the 1 KiB-aligned base); every tile is two 128B-swizzled
+// [128][64] bf16 halves of 16 KiB
+constexpr int kSmQ = 0;
+constexpr int kSmK = 32768;                         // K stage s at kSmK + s * 32 KiB
+constexpr int kSmV = kSmK + kKStages * 32768;       // V stage s at kSmV + s * 32 KiB
+constexpr int kSmBar = kSmV + kVStages * 32768;
 constexpr int kSmMisc = kSmBar + 256;
 constexpr int kSmXchg = kSmMisc + 1024 + kMaxStrmTiles * 16;  // row max / sum exchange, 6 x 128 floats
 constexpr int kSmTotal = kSmXchg + 6 * 128 * 4;
 constexpr int kSmemAlloc = kSmTotal + 1024;  // slack for aligning the base to 1 KiB
 
-// barrier indices (8 bytes each)
-// Double-buffered resources (S, P, O) have one barrier per buffer, so that no barrier
-// can complete two phases ahead of a thread waiting on it (parity waits).
-constexpr int kBarQ = 0, kBarKvFull = 1, kBarKvEmpty = 3, kBarSFull = 5, kBarSFree = 7, kBarPFull = 9, kBarOFull = 11,
-              kBarDrain = 12, kNumBars = 13;
+// TMEM columns: S double buffer, O accumulator, P double buffer (bf16 pairs, A operand)
+constexpr int kTmS = 0, kTmO = 256, kTmP = 384;
+
+// barrier indices (8 bytes each).  Double-buffered resources (S, P) have one barrier
+// per buffer, so that no barrier can complete two phases ahead of a thread waiting on
+// it (parity waits).
+constexpr int kBarQ = 0, kBarKFull = 1, kBarKEmpty = 4, kBarVFull = 7, kBarVEmpty = 9, kBarSFull = 11,
+              kBarSFree = 13, kBarPFull = 15, kBarOFull = 17, kBarDrain = 18, kNumBars = 19;
 
 struct TileDesc {
   int src;      // 0 retrieval cache, 1 streaming history, 2 chunk input
@@ -116,6 +123,54 @@ __device__ __forceinline__ void tc_ld32(uint32_t taddr, float (&v)[32]) {
   asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 #pragma unroll
   for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+// 64 consecutive fp32 columns of this thread's TMEM lane (two loads, one wait)
+__device__ __forceinline__ void tc_ld64(uint32_t taddr, float (&v)[64]) {
+  uint32_t r[64];
+#define DUO_LD32(OFF, B)                                                                                        \
+  asm volatile(                                                                                                 \
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 "                                                                 \
+      "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, "                                 \
+      "%16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];"                \
+      : "=r"(r[B + 0]), "=r"(r[B + 1]), "=r"(r[B + 2]), "=r"(r[B + 3]), "=r"(r[B + 4]), "=r"(r[B + 5]),          \
+        "=r"(r[B + 6]), "=r"(r[B + 7]), "=r"(r[B + 8]), "=r"(r[B + 9]), "=r"(r[B + 10]), "=r"(r[B + 11]),        \
+        "=r"(r[B + 12]), "=r"(r[B + 13]), "=r"(r[B + 14]), "=r"(r[B + 15]), "=r"(r[B + 16]), "=r"(r[B + 17]),    \
+        "=r"(r[B + 18]), "=r"(r[B + 19]), "=r"(r[B + 20]), "=r"(r[B + 21]), "=r"(r[B + 22]), "=r"(r[B + 23]),    \
+        "=r"(r[B + 24]), "=r"(r[B + 25]), "=r"(r[B + 26]), "=r"(r[B + 27]), "=r"(r[B + 28]), "=r"(r[B + 29]),    \
+        "=r"(r[B + 30]), "=r"(r[B + 31])                                                                       \
+      : "r"(taddr + OFF))
+  DUO_LD32(0, 0);
+  DUO_LD32(32, 32);
+#undef DUO_LD32
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+  for (int i = 0; i < 64; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+// store 32 consecutive 32-bit columns of this thread's TMEM lane, and wait for it
+__device__ __forceinline__ void tc_st32u(uint32_t taddr, const uint32_t (&v)[32]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "
+      "{%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16, "
+      "%17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31, %32};" ::"r"(taddr),
+      "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]), "r"(v[8]), "r"(v[9]),
+      "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]), "r"(v[15]), "r"(v[16]), "r"(v[17]), "r"(v[18]),
+      "r"(v[19]), "r"(v[20]), "r"(v[21]), "r"(v[22]), "r"(v[23]), "r"(v[24]), "r"(v[25]), "r"(v[26]), "r"(v[27]),
+      "r"(v[28]), "r"(v[29]), "r"(v[30]), "r"(v[31])
+      : "memory");
+  asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+}
+
+// MMA with A read from tensor memory (bf16 pairs per 32-bit column, K-major)
+__device__ __forceinline__ void tc_mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
+                                          uint32_t acc) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(acc)
+      : "memory");
 }
 
 // store 32 consecutive fp32 columns of this thread's TMEM lane, and wait for it
@@ -216,12 +271,52 @@ __device__ __forceinline__ float exp2_poly(float x) {
   return __int_as_float(__float_as_int(p) + (__float_as_int(t) << 23));
 }
 
+// exp2(v*c - mc) of 64 logits, their sum into rs8 and bf16 pairs into pk; logits
+// [POLY, POLY+16) use the FMA-pipe polynomial (POLY < 0: none)
+template <int POLY>
+__device__ __forceinline__ void probabilities(const float (&v)[64], float c, float mc, float (&rs8)[8],
+                                              uint32_t (&pk)[32]) {
+#pragma unroll
+  for (int e = 0; e < 64; e += 2) {
+    const float x0 = fmaf(v[e], c, -mc), x1 = fmaf(v[e + 1], c, -mc);
+    float p0, p1;
+    if (POLY >= 0 && e >= POLY && e < POLY + 16) {
+      p0 = exp2_poly(x0);
+      p1 = exp2_poly(x1);
+    } else {
+      p0 = ex2(x0);
+      p1 = ex2(x1);
+    }
+    rs8[(e >> 1) & 7] += p0 + p1;
+    const __nv_bfloat162 pb = __floats2bfloat162_rn(p0, p1);
+    pk[e >> 1] = *reinterpret_cast<const uint32_t *>(&pb);
+  }
+}
+
 // A key offset relative to a tile start, clamped to [-1, 127].
 __device__ __forceinline__ int clamp_col(int64_t x) { return static_cast<int>(x < -1 ? -1 : (x > kBN - 1 ? kBN - 1 : x)); }
 
 __device__ __forceinline__ TileDesc tile_of(const Plan &pl, const TileDesc *tl, int j) {
   if (pl.retr) return {0, j * kBN};
   return tl[j];
+}
+
+// TMA of one 128-key tile (K when is_k, else V) from its source into two swizzled halves
+__device__ __forceinline__ void load_tile(const TcArgs &a, const TileDesc &t, const Plan &pl, int g, int b,
+                                          uint32_t dst, uint32_t fb, bool is_k) {
+  if (t.src == 0) {
+    const CUtensorMap *m = is_k ? &a.tm_kc : &a.tm_vc;
+    tma_3d(dst, m, 0, t.y, pl.kvrow, fb);
+    tma_3d(dst + 16384, m, 64, t.y, pl.kvrow, fb);
+  } else if (t.src == 1) {
+    const CUtensorMap *m = is_k ? &a.tm_kh : &a.tm_vh;
+    tma_3d(dst, m, 0, t.y, pl.kvrow, fb);
+    tma_3d(dst + 16384, m, 64, t.y, pl.kvrow, fb);
+  } else {
+    const CUtensorMap *m = is_k ? &a.tm_kn : &a.tm_vn;
+    tma_4d(dst, m, 0, g, t.y, b, fb);
+    tma_4d(dst + 16384, m, 64, g, t.y, b, fb);
+  }
 }
 
 // ---------------------------------------------------------------- the kernel
@@ -259,6 +354,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) prefill_tc_kernel(const __grid_
   if (tid == 0) {
     for (int i = 0; i < kNumBars; ++i)
       mbar_init(bar(i), (i == kBarSFree || i == kBarSFree + 1 || i == kBarPFull || i == kBarPFull + 1) ? 256 : 1);
+    if (smem_u32(smem) & 1023u) flag_status(p.status, kDevTimeout);  // layout assumption (never expected)
     fence_mbar_init();
     *abort_flag = 0;
     int nt;
@@ -282,36 +378,31 @@ __global__ void __launch_bounds__(kTcThreads, 1) prefill_tc_kernel(const __grid_
   const int nt = *ntiles_sm;
 
   if (warp == 0) {
-    // ================= TMA producer =================
+    // ================= TMA producer: Q, then the K ring =================
     if (lane == 0) {
       prefetch_map(&a.tm_q);
-      const CUtensorMap *mk = pl.retr ? &a.tm_kc : &a.tm_kh;
-      prefetch_map(mk);
       mbar_expect_tx(bar(kBarQ), 32768);
       tma_4d(sbase + kSmQ, &a.tm_q, 0, g * G, r0, b, bar(kBarQ));  // box: 64 dims x G heads x npos positions
       tma_4d(sbase + kSmQ + 16384, &a.tm_q, 64, g * G, r0, b, bar(kBarQ));
       for (int j = 0; j < nt; ++j) {
-        const int s = j % kKvStages;
-        if (j >= kKvStages && !wait_bar(bar(kBarKvEmpty + s), ((j / kKvStages) - 1) & 1, p.status, abort_flag)) break;
+        const int s = j % kKStages;
+        if (j >= kKStages && !wait_bar(bar(kBarKEmpty + s), ((j / kKStages) - 1) & 1, p.status, abort_flag)) break;
         const TileDesc t = tile_of(pl, tl, j);
-        const uint32_t kd = sbase + kSmKV + s * 65536, vd = kd + 32768;
-        mbar_expect_tx(bar(kBarKvFull + s), 65536);
-        if (t.src == 0) {
-          tma_3d(kd, &a.tm_kc, 0, t.y, pl.kvrow, bar(kBarKvFull + s));
-          tma_3d(kd + 16384, &a.tm_kc, 64, t.y, pl.kvrow, bar(kBarKvFull + s));
-          tma_3d(vd, &a.tm_vc, 0, t.y, pl.kvrow, bar(kBarKvFull + s));
-          tma_3d(vd + 16384, &a.tm_vc, 64, t.y, pl.kvrow, bar(kBarKvFull + s));
-        } else if (t.src == 1) {
-          tma_3d(kd, &a.tm_kh, 0, t.y, pl.kvrow, bar(kBarKvFull + s));
-          tma_3d(kd + 16384, &a.tm_kh, 64, t.y, pl.kvrow, bar(kBarKvFull + s));
-          tma_3d(vd, &a.tm_vh, 0, t.y, pl.kvrow, bar(kBarKvFull + s));
-          tma_3d(vd + 16384, &a.tm_vh, 64, t.y, pl.kvrow, bar(kBarKvFull + s));
-        } else {
-          tma_4d(kd, &a.tm_kn, 0, g, t.y, b, bar(kBarKvFull + s));
-          tma_4d(kd + 16384, &a.tm_kn, 64, g, t.y, b, bar(kBarKvFull + s));
-          tma_4d(vd, &a.tm_vn, 0, g, t.y, b, bar(kBarKvFull + s));
-          tma_4d(vd + 16384, &a.tm_vn, 64, g, t.y, b, bar(kBarKvFull + s));
-        }
+        const uint32_t dst = sbase + kSmK + s * 32768, fb = bar(kBarKFull + s);
+        mbar_expect_tx(fb, 32768);
+        load_tile(a, t, pl, g, b, dst, fb, true);
+      }
+    }
+  } else if (warp == 10) {
+    // ================= TMA producer: the V ring =================
+    if (lane == 0) {
+      for (int j = 0; j < nt; ++j) {
+        const int s = j % kVStages;
+        if (j >= kVStages && !wait_bar(bar(kBarVEmpty + s), ((j / kVStages) - 1) & 1, p.status, abort_flag)) break;
+        const TileDesc t = tile_of(pl, tl, j);
+        const uint32_t dst = sbase + kSmV + s * 32768, fb = bar(kBarVFull + s);
+        mbar_expect_tx(fb, 32768);
+        load_tile(a, t, pl, g, b, dst, fb, false);
       }
     }
   } else if (warp == 1) {
@@ -321,37 +412,41 @@ __global__ void __launch_bounds__(kTcThreads, 1) prefill_tc_kernel(const __grid_
       constexpr uint32_t kIdPV = idesc_bf16(true);
       bool ok = wait_bar(bar(kBarQ), 0, p.status, abort_flag);
       auto issue_pv = [&](int jj) {
-        // O = P_jj V_jj : K = 128 keys in 8 steps of 16; V is N-major (d contiguous)
-        const int s = jj % kKvStages;
-        const uint32_t vbase = sbase + kSmKV + s * 65536 + 32768;
+        // O += P_jj V_jj : K = 128 keys in 8 steps of 16; P from TMEM (bf16 pairs, K-major),
+        // V from shared memory (d contiguous, MN-major)
+        const int sv = jj % kVStages;
+        const uint32_t vbase = sbase + kSmV + sv * 32768;
+        const uint32_t pcol = tmem + kTmP + (jj & 1) * 64;
         for (int kk = 0; kk < 8; ++kk) {
-          const uint64_t ad = sdesc(sbase + kSmKV + s * 65536 + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024);
           const uint64_t bd = sdesc(vbase + kk * 2048, 16384, 1024);
-          tc_mma(tmem + 256, ad, bd, kIdPV, (jj > 0 || kk > 0) ? 1u : 0u);  // O accumulates over tiles
+          tc_mma_ts(tmem + kTmO, pcol + kk * 8, bd, kIdPV, (jj > 0 || kk > 0) ? 1u : 0u);
         }
         tc_commit(bar(kBarOFull));
-        tc_commit(bar(kBarKvEmpty + s));
+        tc_commit(bar(kBarVEmpty + sv));
       };
       for (int j = 0; j < nt && ok; ++j) {
-        const int s = j % kKvStages;
-        if (!wait_bar(bar(kBarKvFull + s), (j / kKvStages) & 1, p.status, abort_flag)) { ok = false; break; }
+        const int sk = j % kKStages;
+        if (!wait_bar(bar(kBarKFull + sk), (j / kKStages) & 1, p.status, abort_flag)) { ok = false; break; }
         if (j >= 2 && !wait_bar(bar(kBarSFree + (j & 1)), ((j - 2) >> 1) & 1, p.status, abort_flag)) { ok = false; break; }
         tc_fence_after();
         // S_j = Q K_j^T : K = d 128 in 8 steps of 16; Q and K are K-major
-        const uint32_t kbase = sbase + kSmKV + s * 65536;
+        const uint32_t kbase = sbase + kSmK + sk * 32768;
         for (int kk = 0; kk < 8; ++kk) {
           const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
-          tc_mma(tmem + (j & 1) * 128, sdesc(sbase + kSmQ + off, 16, 1024), sdesc(kbase + off, 16, 1024), kIdS,
+          tc_mma(tmem + kTmS + (j & 1) * 128, sdesc(sbase + kSmQ + off, 16, 1024), sdesc(kbase + off, 16, 1024), kIdS,
                  kk > 0 ? 1u : 0u);
         }
         tc_commit(bar(kBarSFull + (j & 1)));
+        tc_commit(bar(kBarKEmpty + sk));
         if (j >= 1) {
           if (!wait_bar(bar(kBarPFull + ((j - 1) & 1)), ((j - 1) >> 1) & 1, p.status, abort_flag)) { ok = false; break; }
+          if (!wait_bar(bar(kBarVFull + ((j - 1) % kVStages)), ((j - 1) / kVStages) & 1, p.status, abort_flag)) { ok = false; break; }
           tc_fence_after();
           issue_pv(j - 1);
         }
       }
-      if (ok && nt > 0 && wait_bar(bar(kBarPFull + ((nt - 1) & 1)), ((nt - 1) >> 1) & 1, p.status, abort_flag)) {
+      if (ok && nt > 0 && wait_bar(bar(kBarPFull + ((nt - 1) & 1)), ((nt - 1) >> 1) & 1, p.status, abort_flag) &&
+          wait_bar(bar(kBarVFull + ((nt - 1) % kVStages)), ((nt - 1) / kVStages) & 1, p.status, abort_flag)) {
         tc_fence_after();
         issue_pv(nt - 1);
       }
@@ -361,10 +456,10 @@ __global__ void __launch_bounds__(kTcThreads, 1) prefill_tc_kernel(const __grid_
     }
   } else {
     // ================= softmax: 8 warps, two threads per query row =================
-    // Warp w reads TMEM lanes 32*(w%4).. (rows) and columns [64*half, 64*half+64) of S
-    // and of O.  The running max m is a reference: P = exp2(s*c - m) may exceed 1 by up to
+    // Warp w reads TMEM lanes 32*(w%4).. (rows) and columns [64*half, 64*half+64) of S,
+    // O and P.  The running max m is a reference: P = exp2(s*c - m) may exceed 1 by up to
     // 2^kSlack, and m (with O in TMEM and l) is rescaled only when a row's tile maximum
-    // passes m + kSlack.  O accumulates in TMEM across tiles.
+    // passes m + kSlack.  S is read from TMEM once per tile.
     constexpr float kSlack = 8.0f;
     const int wq = warp & 3;
     const int half = (warp - 2) >> 2;
@@ -375,7 +470,6 @@ __global__ void __launch_bounds__(kTcThreads, 1) prefill_tc_kernel(const __grid_
     const int64_t i = pl.q0 + rpos;            // absolute query position
     const float c = p.scale_log2;
     float m = -INFINITY, l = 0.f;
-    const int rsw = row & 7;
     float *xch = reinterpret_cast<float *>(smem + kSmXchg);  // [tile parity][half][row] partial maxima
     bool ok = true;
 
@@ -409,27 +503,24 @@ __global__ void __launch_bounds__(kTcThreads, 1) prefill_tc_kernel(const __grid_
 
       if (ok) ok = wait_bar(bar(kBarSFull + (j & 1)), (j >> 1) & 1, p.status, abort_flag);
       tc_fence_after();
-      const uint32_t sbuf = lane_base + (j & 1) * 128 + half * 64;
-      // pass 1: maximum of the visible logits in this thread's 64 columns
-      float mx8[8];
+      // this thread's 64 logits of S_j, then the S buffer is released
+      float v[64];
+      tc_ld64(lane_base + kTmS + (j & 1) * 128 + half * 64, v);
+      tc_fence_before();
+      mbar_arrive(bar(kBarSFree + (j & 1)));
+      if (!full_vis) {
 #pragma unroll
-      for (int u = 0; u < 8; ++u) mx8[u] = -INFINITY;
-#pragma unroll 1
-      for (int cc = 0; cc < 2; ++cc) {
-        float v[32];
-        tc_ld32(sbuf + cc * 32, v);
-        if (full_vis) {
-#pragma unroll
-          for (int e = 0; e < 32; ++e) mx8[e & 7] = fmaxf(mx8[e & 7], v[e]);
-        } else {
-#pragma unroll
-          for (int e = 0; e < 32; ++e) {
-            const int col = half * 64 + cc * 32 + e;
-            const bool vis = col <= hi && (col < sink_c || col > win_c);
-            mx8[e & 7] = vis ? fmaxf(mx8[e & 7], v[e]) : mx8[e & 7];
-          }
+        for (int e = 0; e < 64; ++e) {
+          const int col = half * 64 + e;
+          const bool vis = col <= hi && (col < sink_c || col > win_c);
+          v[e] = vis ? v[e] : -INFINITY;
         }
       }
+      float mx8[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) mx8[u] = v[u];
+#pragma unroll
+      for (int e = 8; e < 64; ++e) mx8[e & 7] = fmaxf(mx8[e & 7], v[e]);
       float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
                        fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
       xch[((j & 1) * 2 + half) * kBM + row] = mx;
@@ -450,81 +541,32 @@ __global__ void __launch_bounds__(kTcThreads, 1) prefill_tc_kernel(const __grid_
         tc_fence_after();
 #pragma unroll 1
         for (int cc = 0; cc < 2; ++cc) {
-          float v[32];
-          const uint32_t oa = lane_base + 256 + half * 64 + cc * 32;
-          tc_ld32(oa, v);
+          float w[32];
+          const uint32_t oa = lane_base + kTmO + half * 64 + cc * 32;
+          tc_ld32(oa, w);
 #pragma unroll
-          for (int e = 0; e < 32; ++e) v[e] *= alpha;
-          tc_st32(oa, v);
+          for (int e = 0; e < 32; ++e) w[e] *= alpha;
+          tc_st32(oa, w);
         }
         waited = true;
       }
-      // pass 2: probabilities, row sum, bf16 P over K_j in stage j % 2 (this thread's half)
-      char *prow = smem + kSmKV + (j % kKvStages) * 65536 + half * 16384 + row * 128;
+      // probabilities (masked logits are -inf and give 0), row sum, bf16 pairs of P_j
       float rs8[8];
 #pragma unroll
       for (int u = 0; u < 8; ++u) rs8[u] = 0.f;
       const float mc = (m == -INFINITY) ? 0.f : m;
-#pragma unroll 1
-      for (int cc = 0; cc < 2; ++cc) {
-        float v[32];
-        tc_ld32(sbuf + cc * 32, v);
-        uint32_t pk[16];
-        if (full_vis) {
-          // a quarter of the exponentials (16 of this thread's 64) on the FMA pipe, the rest
-          // on the MUFU unit
-          if (cc == half) {
-#pragma unroll
-            for (int e = 0; e < 16; e += 2) {
-              const float p0 = exp2_poly(fmaf(v[e], c, -mc)), p1 = exp2_poly(fmaf(v[e + 1], c, -mc));
-              rs8[(e >> 1) & 7] += p0 + p1;
-              const __nv_bfloat162 pb = __floats2bfloat162_rn(p0, p1);
-              pk[e >> 1] = *reinterpret_cast<const uint32_t *>(&pb);
-            }
-          } else {
-#pragma unroll
-            for (int e = 0; e < 16; e += 2) {
-              const float p0 = ex2(fmaf(v[e], c, -mc)), p1 = ex2(fmaf(v[e + 1], c, -mc));
-              rs8[(e >> 1) & 7] += p0 + p1;
-              const __nv_bfloat162 pb = __floats2bfloat162_rn(p0, p1);
-              pk[e >> 1] = *reinterpret_cast<const uint32_t *>(&pb);
-            }
-          }
-#pragma unroll
-          for (int e = 16; e < 32; e += 2) {
-            const float p0 = ex2(fmaf(v[e], c, -mc)), p1 = ex2(fmaf(v[e + 1], c, -mc));
-            rs8[(e >> 1) & 7] += p0 + p1;
-            const __nv_bfloat162 pb = __floats2bfloat162_rn(p0, p1);
-            pk[e >> 1] = *reinterpret_cast<const uint32_t *>(&pb);
-          }
-        } else {
-#pragma unroll
-          for (int e = 0; e < 32; e += 2) {
-            const int c0 = half * 64 + cc * 32 + e, c1 = c0 + 1;
-            const bool v0 = c0 <= hi && (c0 < sink_c || c0 > win_c);
-            const bool v1 = c1 <= hi && (c1 < sink_c || c1 > win_c);
-            const float p0 = v0 ? ex2(fmaf(v[e], c, -mc)) : 0.f;
-            const float p1 = v1 ? ex2(fmaf(v[e + 1], c, -mc)) : 0.f;
-            rs8[(e >> 1) & 7] += p0 + p1;
-            const __nv_bfloat162 pb = __floats2bfloat162_rn(p0, p1);
-            pk[e >> 1] = *reinterpret_cast<const uint32_t *>(&pb);
-          }
-        }
-        // columns 64*half + 32*cc .. +31 -> 16-byte chunks 4*cc .. 4*cc+3 of this half
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          const int chunk = (cc * 4 + q) ^ rsw;
-          *reinterpret_cast<uint4 *>(prow + chunk * 16) = make_uint4(pk[4 * q], pk[4 * q + 1], pk[4 * q + 2], pk[4 * q + 3]);
-        }
-      }
-      tc_fence_before();
-      mbar_arrive(bar(kBarSFree + (j & 1)));  // S buffer j % 2 may be overwritten
+      uint32_t pk[32];
+      // a quarter of the exponentials of interior tiles on the FMA pipe, the rest on MUFU
+      if (!full_vis) probabilities<-1>(v, c, mc, rs8, pk);
+      else if (half == 0) probabilities<16>(v, c, mc, rs8, pk);
+      else probabilities<48>(v, c, mc, rs8, pk);
+      // P_j into TMEM buffer j % 2 (its previous reader P_{j-2} V_{j-2} was waited for at j-1)
+      tc_st32u(lane_base + kTmP + (j & 1) * 64 + half * 32, pk);
       // one wait per P V product, in order (here unless the rescale already waited)
       if (j >= 1 && !waited) {
         if (ok) ok = wait_bar(bar(kBarOFull), (j - 1) & 1, p.status, abort_flag);
       }
       l += ((rs8[0] + rs8[1]) + (rs8[2] + rs8[3])) + ((rs8[4] + rs8[5]) + (rs8[6] + rs8[7]));
-      fence_async_smem();  // P visible to the tensor core
       tc_fence_before();
       mbar_arrive(bar(kBarPFull + (j & 1)));
     }
@@ -541,18 +583,18 @@ __global__ void __launch_bounds__(kTcThreads, 1) prefill_tc_kernel(const __grid_
     const float inv = 1.f / lrow;
 #pragma unroll 1
     for (int cc = 0; cc < 2; ++cc) {
-      float v[32];
-      tc_ld32(lane_base + 256 + half * 64 + cc * 32, v);
+      float w[32];
+      tc_ld32(lane_base + kTmO + half * 64 + cc * 32, w);
       if (store) {
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
-          uint32_t w[4];
+          uint32_t wd[4];
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
-            const __nv_bfloat162 pb = __floats2bfloat162_rn(v[8 * q + 2 * e] * inv, v[8 * q + 2 * e + 1] * inv);
-            w[e] = *reinterpret_cast<const uint32_t *>(&pb);
+            const __nv_bfloat162 pb = __floats2bfloat162_rn(w[8 * q + 2 * e] * inv, w[8 * q + 2 * e + 1] * inv);
+            wd[e] = *reinterpret_cast<const uint32_t *>(&pb);
           }
-          *reinterpret_cast<uint4 *>(orow + cc * 64 + q * 16) = make_uint4(w[0], w[1], w[2], w[3]);
+          *reinterpret_cast<uint4 *>(orow + cc * 64 + q * 16) = make_uint4(wd[0], wd[1], wd[2], wd[3]);
         }
       }
     }
