@@ -393,7 +393,8 @@ duo_status duo_decode_attention(duo_cache *c, int layer, const void *q, void *ou
   p.nsplit = static_cast<int>(nsplit);
   p.split_len = split_len;
   p.n_retr_ctas = static_cast<int>(heads * nsplit);
-  const cudaError_t e = decode_tc_supported(p, c->dtype, int4) ? launch_decode_tc(p, c->num_sms, st)
+  // the tcgen05 decode overlaps its start-up with the previous kernel on the stream
+  const cudaError_t e = decode_tc_supported(p, c->dtype, int4) ? launch_decode_tc(p, c->num_sms, true, st)
                                                                 : launch_decode(p, c->dtype, int4, st);
   if (e != cudaSuccess) return DUO_ERR_CUDA;
   return DUO_OK;

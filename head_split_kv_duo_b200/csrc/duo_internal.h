@@ -128,9 +128,11 @@ cudaError_t launch_prefill_simt(const PrefillParams &p, duo_dtype dt, cudaStream
 cudaError_t launch_prefill_tc(const PrefillParams &p, cudaStream_t st);
 bool prefill_tc_supported(const PrefillParams &p, duo_dtype dt);
 
-// tcgen05 decode (bf16, d = 128, up to 16 query heads per KV head), one CTA per SM
+// tcgen05 decode (bf16, d = 128, up to 16 query heads per KV head), one CTA per SM.
+// overlap_previous: launch as a programmatic dependent of the previous kernel on the
+// stream; the kernel waits for it (griddepcontrol.wait) before its first global read.
 bool decode_tc_supported(const DecodeParams &p, duo_dtype dt, bool int4);
-cudaError_t launch_decode_tc(const DecodeParams &p, int num_sms, cudaStream_t st);
+cudaError_t launch_decode_tc(const DecodeParams &p, int num_sms, bool overlap_previous, cudaStream_t st);
 
 // decode tiling shared by host (split sizing) and device
 int decode_tokens_per_stage(duo_dtype dt, int D, bool int4);

@@ -55,6 +55,9 @@ __device__ __forceinline__ void quantize_row_int4(const char *src, uint8_t *code
 
 template <typename T>
 __global__ void __launch_bounds__(256) append_kernel(const AppendParams p) {
+  // a decode launched right after may start its set-up now; it waits for this grid to
+  // finish before its first global read
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   const int64_t warp = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
   const int lane = threadIdx.x & 31;
   const int64_t total = static_cast<int64_t>(p.B) * p.n * p.Hkv;

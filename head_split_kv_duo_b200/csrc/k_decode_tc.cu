@@ -231,6 +231,10 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
   if (warp == 0) {
     // ================= TMA producer =================
     if (lane == 0) {
+      // Launched as a programmatic dependent, this grid's set-up overlaps the previous
+      // kernel on the stream; nothing is read from global memory before that kernel has
+      // finished (every other read and every write of this grid follows these loads).
+      asm volatile("griddepcontrol.wait;" ::: "memory");
       for (int j = 0; j < nu; ++j) {
         const int s = j % kStages;
         if (j >= kStages && !wait_bar(bar(kBarEmpty + s), ((j / kStages) - 1) & 1, p.status, abort_flag)) break;
@@ -585,15 +589,25 @@ bool map_bf16(CUtensorMap *m, const void *base, int rank, const uint64_t *dims, 
 }
 
 template <int NQ>
-cudaError_t launch_nq(const TcDecodeArgs &a, cudaStream_t st) {
+cudaError_t launch_nq(const TcDecodeArgs &a, bool overlap_previous, cudaStream_t st) {
   static bool attr = false;
   if (!attr) {
     cudaError_t e = cudaFuncSetAttribute(decode_tc_kernel<NQ>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemAlloc);
     if (e != cudaSuccess) return e;
     attr = true;
   }
-  decode_tc_kernel<NQ><<<a.num_ctas, kThreads, kSmemAlloc, st>>>(a);
-  return cudaGetLastError();
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(a.num_ctas);
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = kSmemAlloc;
+  cfg.stream = st;
+  cudaLaunchAttribute attrs[1];
+  attrs[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attrs[0].val.programmaticStreamSerializationAllowed = overlap_previous ? 1 : 0;
+  cfg.attrs = attrs;
+  cfg.numAttrs = 1;
+  cudaError_t e = cudaLaunchKernelEx(&cfg, decode_tc_kernel<NQ>, a);
+  return e != cudaSuccess ? e : cudaGetLastError();
 }
 
 }  // namespace
@@ -602,7 +616,7 @@ bool decode_tc_supported(const DecodeParams &p, duo_dtype dt, bool int4) {
   return dt == DUO_BF16 && !int4 && p.D == kD && p.G >= 1 && p.G <= kN && encode_fn() != nullptr;
 }
 
-cudaError_t launch_decode_tc(const DecodeParams &p, int num_sms, cudaStream_t st) {
+cudaError_t launch_decode_tc(const DecodeParams &p, int num_sms, bool overlap_previous, cudaStream_t st) {
   static TcDecodeArgs a;
   a.p = p;
   a.units_r = static_cast<int>((p.len + kTile - 1) / kTile);
@@ -639,11 +653,11 @@ cudaError_t launch_decode_tc(const DecodeParams &p, int num_sms, cudaStream_t st
     ok &= map_bf16(&a.tm_vs, p.sv, 3, d, s, bx);
   }
   if (!ok) return cudaErrorInvalidValue;
-  if (p.G <= 1) return launch_nq<1>(a, st);
-  if (p.G <= 2) return launch_nq<2>(a, st);
-  if (p.G <= 4) return launch_nq<4>(a, st);
-  if (p.G <= 8) return launch_nq<8>(a, st);
-  return launch_nq<16>(a, st);
+  if (p.G <= 1) return launch_nq<1>(a, overlap_previous, st);
+  if (p.G <= 2) return launch_nq<2>(a, overlap_previous, st);
+  if (p.G <= 4) return launch_nq<4>(a, overlap_previous, st);
+  if (p.G <= 8) return launch_nq<8>(a, overlap_previous, st);
+  return launch_nq<16>(a, overlap_previous, st);
 }
 
 }  // namespace duo

@@ -106,6 +106,6 @@ extern "C" duo_status duo_decode_attention_static_scratch(duo_cache *c, int laye
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   // tickets must start at zero; the previous call's contents are still in the array
   if (cudaMemsetAsync(p.counters, 0, items * 4, st) != cudaSuccess) return DUO_ERR_CUDA;
-  if (launch_decode_tc(p, static_cast<int>(ctas), st) != cudaSuccess) return DUO_ERR_CUDA;
+  if (launch_decode_tc(p, static_cast<int>(ctas), false, st) != cudaSuccess) return DUO_ERR_CUDA;
   return DUO_OK;
 }
