@@ -290,7 +290,8 @@ def run_ours(args, rank, world, dist):
                      "peak": hbm_peak, "peak_source": f"{peak_src} hbm_gbs (burst copy)", "unit": "GB/s",
                      "frac": round(achieved / hbm_peak, 4), "traffic": recorded_traffic(args.workload),
                      "algorithmic_bytes_per_launch": int(per_launch_bytes), "avg_launch_us": round(dec_avg_ms * 1e3, 3)},
-        "gpu_launches": steps * nlayers * 2,
+        # per layer and step: append + decode (+ the split merge on the tcgen05 path)
+        "gpu_launches": steps * nlayers * (3 if fmt == "same" else 2),
         "clocks": clk.summary(),
         "e2e": e2e,
         "prefill": prefill,

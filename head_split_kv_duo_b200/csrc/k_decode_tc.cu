@@ -16,8 +16,9 @@
 // Work balance: every (batch, KV head) is an item of 128-token units (retrieval:
 // ceil(len/128), streaming: ceil((S+W)/128)); the units of all items are laid end to
 // end and cut into one equal range per CTA (one CTA per SM).  A CTA flushes a partial
-// (max, sum, unnormalised output) whenever an item ends inside its range; the last
-// CTA to finish an item (atomic ticket, no waiting) merges its partials.
+// (max, sum, unnormalised output) whenever an item ends inside its range; the
+// partials are merged by decode_merge_kernel, launched right behind as a programmatic
+// dependent (one block per query head; items held by a single CTA are written directly).
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
@@ -201,10 +202,11 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
   auto bar = [&](int i) { return sbase + kSmBar + 8u * i; };
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + kSmMisc);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + kSmMisc + 4);
-  int *last_flag = reinterpret_cast<int *>(smem + kSmMisc + 8);
   float *red = reinterpret_cast<float *>(smem + kSmRed);  // [4 warps][16]
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  // the split merge (decode_merge_kernel) may be scheduled now; it waits for this grid
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   const int64_t u0 = cta_begin(a, blockIdx.x), u1 = cta_begin(a, blockIdx.x + 1);
   const int nu = static_cast<int>(u1 - u0);
   const int G = p.G;
@@ -389,54 +391,6 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
             dst[kD + 1] = lt[q];
           }
         }
-      __threadfence();
-      named_sync(1, 128);
-      if (t == 0) {
-        const uint32_t prev = atomicAdd(p.counters + pitem, 1u);
-        *last_flag = (prev == static_cast<uint32_t>(nseg - 1)) ? 1 : 0;
-      }
-      named_sync(1, 128);
-      if (!*last_flag) return;
-      __threadfence();
-      // merge: warp wq takes query heads wq, wq+4, ...; its lanes read segments in
-      // parallel for the max and the normaliser, then stream the output rows (4 dims a lane)
-      float *wts = red + 4 * kN + wq * kMaxSplits;
-      for (int q = wq; q < G; q += 4) {
-        const float *base = part + static_cast<int64_t>(q) * kRow;
-        const int64_t sstride = static_cast<int64_t>(G) * kRow;
-        float M = -INFINITY;
-        for (int sg = lane; sg < nseg; sg += 32) M = fmaxf(M, __ldcg(base + sg * sstride + kD));
-        M = warp_max(M);
-        float den = 0.f;
-        for (int sg = lane; sg < nseg; sg += 32) {
-          const float ms = __ldcg(base + sg * sstride + kD);
-          const float e = (ms == -INFINITY) ? 0.f : ex2(ms - M);
-          wts[sg] = e;
-          den = fmaf(e, __ldcg(base + sg * sstride + kD + 1), den);
-        }
-        den = warp_sum(den);
-        __syncwarp();
-        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll 4
-        for (int sg = 0; sg < nseg; ++sg) {
-          const float w = wts[sg];
-          const float4 v = __ldcg(reinterpret_cast<const float4 *>(base + sg * sstride) + lane);
-          acc.x = fmaf(w, v.x, acc.x);
-          acc.y = fmaf(w, v.y, acc.y);
-          acc.z = fmaf(w, v.z, acc.z);
-          acc.w = fmaf(w, v.w, acc.w);
-        }
-        const float inv = 1.f / den;
-        const __nv_bfloat162 lo = __floats2bfloat162_rn(acc.x * inv, acc.y * inv);
-        const __nv_bfloat162 hi = __floats2bfloat162_rn(acc.z * inv, acc.w * inv);
-        uint2 pk;
-        pk.x = *reinterpret_cast<const uint32_t *>(&lo);
-        pk.y = *reinterpret_cast<const uint32_t *>(&hi);
-        *reinterpret_cast<uint2 *>(p.out + ((static_cast<int64_t>(b) * p.Hq + h0 + q) * kD + 4 * lane) * 2) = pk;
-        if (lane == 0 && p.lse) p.lse[b * p.Hq + h0 + q] = (M + lg2(den)) * kLn2;
-        __syncwarp();
-      }
-      if (t == 0) p.counters[pitem] = 0u;
     };
 
     // o = (o + O^T(jj)) * alpha for this thread's dimension t
@@ -558,6 +512,63 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
   if (warp == 1) asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kTmemCols));
 }
 
+// Merges the split partials of every (batch, KV head) whose units were cut over more
+// than one CTA: block = (item, query head of the group), thread t = head dimension t.
+// Launched as a programmatic dependent of decode_tc_kernel; waits for it to finish.
+__global__ void __launch_bounds__(kTile) decode_merge_kernel(const __grid_constant__ TcDecodeArgs a) {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  const DecodeParams &p = a.p;
+  const int G = p.G;
+  const int item = blockIdx.x / G, q = blockIdx.x % G;
+  const bool retr = item < a.n_items_r;
+  const int units = retr ? a.units_r : a.units_s;
+  const int64_t ia = retr ? static_cast<int64_t>(item) * a.units_r
+                          : static_cast<int64_t>(a.n_items_r) * a.units_r +
+                                static_cast<int64_t>(item - a.n_items_r) * a.units_s;
+  const int nseg = cta_of(a, ia + units - 1) - cta_of(a, ia) + 1;
+  if (nseg == 1) return;  // written directly by its only CTA
+  int b, g;
+  if (retr) {
+    b = item / p.Hr;
+    g = p.hm.retr_head[item % p.Hr];
+  } else {
+    const int it = item - a.n_items_r;
+    b = it / p.Hs;
+    g = p.hm.strm_head[it % p.Hs];
+  }
+  constexpr int kRow = kD + 4;
+  const int64_t pitem = static_cast<int64_t>(b) * p.Hkv + g;
+  const float *base = p.partials + (pitem * p.max_splits) * G * kRow + static_cast<int64_t>(q) * kRow;
+  const int64_t sstride = static_cast<int64_t>(G) * kRow;
+  __shared__ float wts[kMaxSplits];
+  __shared__ float red[4];
+  const int t = threadIdx.x, lane = t & 31, w = t >> 5;
+  float M = -INFINITY;
+  for (int sg = t; sg < nseg; sg += kTile) M = fmaxf(M, base[sg * sstride + kD]);
+  M = warp_max(M);
+  if (lane == 0) red[w] = M;
+  __syncthreads();
+  M = fmaxf(fmaxf(red[0], red[1]), fmaxf(red[2], red[3]));
+  __syncthreads();
+  float den = 0.f;
+  for (int sg = t; sg < nseg; sg += kTile) {
+    const float ms = base[sg * sstride + kD];
+    const float e = (ms == -INFINITY) ? 0.f : ex2(ms - M);
+    wts[sg] = e;
+    den = fmaf(e, base[sg * sstride + kD + 1], den);
+  }
+  den = warp_sum(den);
+  if (lane == 0) red[w] = den;
+  __syncthreads();
+  den = (red[0] + red[1]) + (red[2] + red[3]);
+  float acc = 0.f;
+#pragma unroll 8
+  for (int sg = 0; sg < nseg; ++sg) acc = fmaf(wts[sg], base[sg * sstride + t], acc);
+  const int h = g * G + q;
+  Elem<__nv_bfloat16>::store(p.out, (static_cast<int64_t>(b) * p.Hq + h) * kD + t, acc / den);
+  if (t == 0 && p.lse) p.lse[b * p.Hq + h] = (M + lg2(den)) * kLn2;
+}
+
 PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
   static bool tried = false;
@@ -607,7 +618,23 @@ cudaError_t launch_nq(const TcDecodeArgs &a, bool overlap_previous, cudaStream_t
   cfg.attrs = attrs;
   cfg.numAttrs = 1;
   cudaError_t e = cudaLaunchKernelEx(&cfg, decode_tc_kernel<NQ>, a);
-  return e != cudaSuccess ? e : cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  // split merge: only needed when some item spans more than one CTA
+  if (a.num_ctas > 1) {
+    cudaLaunchConfig_t mc = {};
+    mc.gridDim = dim3((a.n_items_r + a.p.B * a.p.Hs) * a.p.G);
+    mc.blockDim = dim3(kTile);
+    mc.dynamicSmemBytes = 0;
+    mc.stream = st;
+    cudaLaunchAttribute ma[1];
+    ma[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    ma[0].val.programmaticStreamSerializationAllowed = 1;
+    mc.attrs = ma;
+    mc.numAttrs = 1;
+    e = cudaLaunchKernelEx(&mc, decode_merge_kernel, a);
+    if (e != cudaSuccess) return e;
+  }
+  return cudaGetLastError();
 }
 
 }  // namespace
