@@ -16,9 +16,9 @@
 // Work balance: every (batch, KV head) is an item of 128-token units (retrieval:
 // ceil(len/128), streaming: ceil((S+W)/128)); the units of all items are laid end to
 // end and cut into one equal range per CTA (one CTA per SM).  A CTA flushes a partial
-// (max, sum, unnormalised output) whenever an item ends inside its range; the
-// partials are merged by decode_merge_kernel, launched right behind as a programmatic
-// dependent (one block per query head; items held by a single CTA are written directly).
+// (max, sum, unnormalised output) whenever an item ends inside its range; the last CTA
+// of an item to flush (a ticket per item) merges the item's partials.  Items held by a
+// single CTA are written directly.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
@@ -42,8 +42,8 @@ constexpr int kTmemCols = 4 * kAcc * 16;    // S^T x 2 and O^T x 2, kAcc blocks 
 // shared memory map per stage: K [128][128] (2 swizzle atoms of 16 KiB), V likewise, Q [16][128]
 constexpr int kStK = 0, kStV = 32768, kStQ = 65536, kStage = 65536 + 4096;
 constexpr int kSmP = kStages * kStage;     // 2 x P^T [16][128] bf16 (2 atoms of 2 KiB each)
-constexpr int kSmRed = kSmP + 8192;        // cross-warp reductions [4][16] + merge weights [4][kMaxSplits]
-constexpr int kSmBar = kSmRed + (4 * 16 + 4 * kMaxSplits) * 4;
+constexpr int kSmRed = kSmP + 8192;        // cross-warp reductions [4][16] + merge exchange [128][6]
+constexpr int kSmBar = kSmRed + (4 * 16 + 128 * 6) * 4;
 constexpr int kSmMisc = kSmBar + 256;
 constexpr int kSmemAlloc = kSmMisc + 64 + 1024;
 // Double-buffered resources (S, P, O) each have one barrier per buffer, so that no
@@ -202,11 +202,10 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
   auto bar = [&](int i) { return sbase + kSmBar + 8u * i; };
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + kSmMisc);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + kSmMisc + 4);
+  volatile int *last_flag = reinterpret_cast<volatile int *>(smem + kSmMisc + 8);
   float *red = reinterpret_cast<float *>(smem + kSmRed);  // [4 warps][16]
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  // the split merge (decode_merge_kernel) may be scheduled now; it waits for this grid
-  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   const int64_t u0 = cta_begin(a, blockIdx.x), u1 = cta_begin(a, blockIdx.x + 1);
   const int nu = static_cast<int>(u1 - u0);
   const int G = p.G;
@@ -338,6 +337,106 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
     bool ok = true;
     int cur_item = -1;
 
+    // Merges the nseg partial rows of one item (run by the item's last CTA).  A row is one
+    // float4 column c of query head c / 32's output; with fewer than 128 columns the
+    // threads split the segments into nsl interleaved lanes, combined through shared
+    // memory at the end.  Loads are issued in batches of 8 segments, so the merge costs
+    // about ceil(nseg / (8 nsl)) round trips to L2.
+    auto merge = [&](const float *part, int nseg, int b, int h0) {
+      constexpr int kRow = kD + 4;
+      constexpr int kBatch = 8;
+      const int cols = G * (kD / 4);
+      const int nsl = cols >= 128 ? 1 : 128 / cols;
+      float *cmb = red + 4 * kN;  // [128][6]: M, den, acc
+      for (int c0 = 0; c0 < cols; c0 += 128) {
+        const int col = cols >= 128 ? c0 + t : t % cols;
+        const int sl = cols >= 128 ? 0 : t / cols;
+        const bool active = col < cols && sl < nsl;
+        const int q = col >> 5, c4 = col & 31;
+        float M = -INFINITY, den = 0.f;
+        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (active) {
+          for (int s0 = sl; s0 < nseg; s0 += kBatch * nsl) {
+            float mm[kBatch], ll[kBatch];
+            float4 vv[kBatch];
+#pragma unroll
+            for (int i = 0; i < kBatch; ++i) {
+              const int sg = s0 + i * nsl;
+              if (sg < nseg) {
+                const float *row = part + (static_cast<int64_t>(sg) * G + q) * kRow;
+                mm[i] = __ldcg(row + kD);
+                ll[i] = __ldcg(row + kD + 1);
+                vv[i] = __ldcg(reinterpret_cast<const float4 *>(row) + c4);
+              } else {
+                mm[i] = -INFINITY;
+                ll[i] = 0.f;
+                vv[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+              }
+            }
+            float Mb = M;
+#pragma unroll
+            for (int i = 0; i < kBatch; ++i) Mb = fmaxf(Mb, mm[i]);
+            if (Mb == -INFINITY) continue;  // nothing visible so far
+            const float r = (M == -INFINITY) ? 0.f : ex2(M - Mb);
+            den *= r;
+            acc.x *= r;
+            acc.y *= r;
+            acc.z *= r;
+            acc.w *= r;
+#pragma unroll
+            for (int i = 0; i < kBatch; ++i) {
+              const float w = (mm[i] == -INFINITY) ? 0.f : ex2(mm[i] - Mb);
+              den = fmaf(w, ll[i], den);
+              acc.x = fmaf(w, vv[i].x, acc.x);
+              acc.y = fmaf(w, vv[i].y, acc.y);
+              acc.z = fmaf(w, vv[i].z, acc.z);
+              acc.w = fmaf(w, vv[i].w, acc.w);
+            }
+            M = Mb;
+          }
+        }
+        if (nsl > 1) {
+          if (active) {
+            float *e = cmb + t * 6;
+            e[0] = M;
+            e[1] = den;
+            e[2] = acc.x;
+            e[3] = acc.y;
+            e[4] = acc.z;
+            e[5] = acc.w;
+          }
+          named_sync(1, 128);
+          if (active && sl == 0) {
+            for (int k = 1; k < nsl; ++k) {
+              const float *e = cmb + (t + k * cols) * 6;
+              const float Mn = fmaxf(M, e[0]);
+              if (Mn == -INFINITY) continue;
+              const float ra = (M == -INFINITY) ? 0.f : ex2(M - Mn);
+              const float rb = (e[0] == -INFINITY) ? 0.f : ex2(e[0] - Mn);
+              den = den * ra + e[1] * rb;
+              acc.x = acc.x * ra + e[2] * rb;
+              acc.y = acc.y * ra + e[3] * rb;
+              acc.z = acc.z * ra + e[4] * rb;
+              acc.w = acc.w * ra + e[5] * rb;
+              M = Mn;
+            }
+          }
+        }
+        if (active && sl == 0) {
+          const float inv = 1.f / den;
+          const __nv_bfloat162 lo = __floats2bfloat162_rn(acc.x * inv, acc.y * inv);
+          const __nv_bfloat162 hi = __floats2bfloat162_rn(acc.z * inv, acc.w * inv);
+          uint2 pk;
+          pk.x = *reinterpret_cast<const uint32_t *>(&lo);
+          pk.y = *reinterpret_cast<const uint32_t *>(&hi);
+          const int h = h0 + q;
+          *reinterpret_cast<uint2 *>(p.out + ((static_cast<int64_t>(b) * p.Hq + h) * kD + 4 * c4) * 2) = pk;
+          if (c4 == 0 && p.lse) p.lse[b * p.Hq + h] = (M + lg2(den)) * kLn2;
+        }
+      }
+      named_sync(1, 128);  // cmb and red are reused by the next flush
+    };
+
     // Writes this CTA's result for `item` (partial or final) and merges when last.
     auto flush = [&](int item) {
 #pragma unroll
@@ -391,6 +490,17 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
             dst[kD + 1] = lt[q];
           }
         }
+      __threadfence();
+      named_sync(1, 128);
+      if (t == 0) {
+        const uint32_t prev = atomicAdd(p.counters + pitem, 1u);
+        *last_flag = (prev == static_cast<uint32_t>(nseg - 1)) ? 1 : 0;
+      }
+      named_sync(1, 128);
+      if (!*last_flag) return;
+      __threadfence();
+      merge(part, nseg, b, h0);
+      if (t == 0) p.counters[pitem] = 0u;  // ready for the next call
     };
 
     // o = (o + O^T(jj)) * alpha for this thread's dimension t
@@ -512,63 +622,6 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
   if (warp == 1) asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kTmemCols));
 }
 
-// Merges the split partials of every (batch, KV head) whose units were cut over more
-// than one CTA: block = (item, query head of the group), thread t = head dimension t.
-// Launched as a programmatic dependent of decode_tc_kernel; waits for it to finish.
-__global__ void __launch_bounds__(kTile) decode_merge_kernel(const __grid_constant__ TcDecodeArgs a) {
-  asm volatile("griddepcontrol.wait;" ::: "memory");
-  const DecodeParams &p = a.p;
-  const int G = p.G;
-  const int item = blockIdx.x / G, q = blockIdx.x % G;
-  const bool retr = item < a.n_items_r;
-  const int units = retr ? a.units_r : a.units_s;
-  const int64_t ia = retr ? static_cast<int64_t>(item) * a.units_r
-                          : static_cast<int64_t>(a.n_items_r) * a.units_r +
-                                static_cast<int64_t>(item - a.n_items_r) * a.units_s;
-  const int nseg = cta_of(a, ia + units - 1) - cta_of(a, ia) + 1;
-  if (nseg == 1) return;  // written directly by its only CTA
-  int b, g;
-  if (retr) {
-    b = item / p.Hr;
-    g = p.hm.retr_head[item % p.Hr];
-  } else {
-    const int it = item - a.n_items_r;
-    b = it / p.Hs;
-    g = p.hm.strm_head[it % p.Hs];
-  }
-  constexpr int kRow = kD + 4;
-  const int64_t pitem = static_cast<int64_t>(b) * p.Hkv + g;
-  const float *base = p.partials + (pitem * p.max_splits) * G * kRow + static_cast<int64_t>(q) * kRow;
-  const int64_t sstride = static_cast<int64_t>(G) * kRow;
-  __shared__ float wts[kMaxSplits];
-  __shared__ float red[4];
-  const int t = threadIdx.x, lane = t & 31, w = t >> 5;
-  float M = -INFINITY;
-  for (int sg = t; sg < nseg; sg += kTile) M = fmaxf(M, base[sg * sstride + kD]);
-  M = warp_max(M);
-  if (lane == 0) red[w] = M;
-  __syncthreads();
-  M = fmaxf(fmaxf(red[0], red[1]), fmaxf(red[2], red[3]));
-  __syncthreads();
-  float den = 0.f;
-  for (int sg = t; sg < nseg; sg += kTile) {
-    const float ms = base[sg * sstride + kD];
-    const float e = (ms == -INFINITY) ? 0.f : ex2(ms - M);
-    wts[sg] = e;
-    den = fmaf(e, base[sg * sstride + kD + 1], den);
-  }
-  den = warp_sum(den);
-  if (lane == 0) red[w] = den;
-  __syncthreads();
-  den = (red[0] + red[1]) + (red[2] + red[3]);
-  float acc = 0.f;
-#pragma unroll 8
-  for (int sg = 0; sg < nseg; ++sg) acc = fmaf(wts[sg], base[sg * sstride + t], acc);
-  const int h = g * G + q;
-  Elem<__nv_bfloat16>::store(p.out, (static_cast<int64_t>(b) * p.Hq + h) * kD + t, acc / den);
-  if (t == 0 && p.lse) p.lse[b * p.Hq + h] = (M + lg2(den)) * kLn2;
-}
-
 PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
   static bool tried = false;
@@ -617,23 +670,8 @@ cudaError_t launch_nq(const TcDecodeArgs &a, bool overlap_previous, cudaStream_t
   attrs[0].val.programmaticStreamSerializationAllowed = overlap_previous ? 1 : 0;
   cfg.attrs = attrs;
   cfg.numAttrs = 1;
-  cudaError_t e = cudaLaunchKernelEx(&cfg, decode_tc_kernel<NQ>, a);
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, decode_tc_kernel<NQ>, a);
   if (e != cudaSuccess) return e;
-  // split merge: only needed when some item spans more than one CTA
-  if (a.num_ctas > 1) {
-    cudaLaunchConfig_t mc = {};
-    mc.gridDim = dim3((a.n_items_r + a.p.B * a.p.Hs) * a.p.G);
-    mc.blockDim = dim3(kTile);
-    mc.dynamicSmemBytes = 0;
-    mc.stream = st;
-    cudaLaunchAttribute ma[1];
-    ma[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    ma[0].val.programmaticStreamSerializationAllowed = 1;
-    mc.attrs = ma;
-    mc.numAttrs = 1;
-    e = cudaLaunchKernelEx(&mc, decode_merge_kernel, a);
-    if (e != cudaSuccess) return e;
-  }
   return cudaGetLastError();
 }
 
@@ -644,7 +682,7 @@ bool decode_tc_supported(const DecodeParams &p, duo_dtype dt, bool int4) {
 }
 
 cudaError_t launch_decode_tc(const DecodeParams &p, int num_sms, bool overlap_previous, cudaStream_t st) {
-  static TcDecodeArgs a;
+  TcDecodeArgs a{};
   a.p = p;
   a.units_r = static_cast<int>((p.len + kTile - 1) / kTile);
   const int64_t slots = static_cast<int64_t>(p.S) + p.W;
