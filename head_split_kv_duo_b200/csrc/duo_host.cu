@@ -394,8 +394,13 @@ duo_status duo_decode_attention(duo_cache *c, int layer, const void *q, void *ou
   p.split_len = split_len;
   p.n_retr_ctas = static_cast<int>(heads * nsplit);
   // the tcgen05 decode overlaps its start-up with the previous kernel on the stream
-  const cudaError_t e = decode_tc_supported(p, c->dtype, int4) ? launch_decode_tc(p, c->num_sms, true, st)
-                                                                : launch_decode(p, c->dtype, int4, st);
+  cudaError_t e;
+  if (int4 && decode_int4_tc_supported(p, c->dtype))
+    e = launch_decode_int4_tc(p, c->num_sms, true, st);
+  else if (decode_tc_supported(p, c->dtype, int4))
+    e = launch_decode_tc(p, c->num_sms, true, st);
+  else
+    e = launch_decode(p, c->dtype, int4, st);
   if (e != cudaSuccess) return DUO_ERR_CUDA;
   return DUO_OK;
 }

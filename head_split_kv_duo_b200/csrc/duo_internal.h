@@ -133,6 +133,9 @@ bool prefill_tc_supported(const PrefillParams &p, duo_dtype dt);
 // stream; the kernel waits for it (griddepcontrol.wait) before its first global read.
 bool decode_tc_supported(const DecodeParams &p, duo_dtype dt, bool int4);
 cudaError_t launch_decode_tc(const DecodeParams &p, int num_sms, bool overlap_previous, cudaStream_t st);
+// tcgen05 decode over an INT4 retrieval cache (bf16, head_dim 128, G <= 16)
+bool decode_int4_tc_supported(const DecodeParams &p, duo_dtype dt);
+cudaError_t launch_decode_int4_tc(const DecodeParams &p, int num_sms, bool overlap_previous, cudaStream_t st);
 
 // decode tiling shared by host (split sizing) and device
 int decode_tokens_per_stage(duo_dtype dt, int D, bool int4);

@@ -333,6 +333,77 @@ def test_int4_codes_bit_exact_and_decode(B, ctx):
     print("int4 vs unquantised:", errors(got, ref))
 
 
+def _int4_decode_check(Hq, Hkv, mask_row, S, W, B, ctx, steps, seed, plant=False):
+    """Append ctx tokens, then `steps` decode steps, on an INT4 retrieval cache; compare
+    with the oracle over the oracle's own dequantisation of the retrieval rows.  With
+    `plant`, one middle key of every retrieval head is set to 3x the first query of its
+    group (so that query's attention concentrates there) and its value to a ramp."""
+    d, T, G = 128, ctx + steps, Hq // Hkv
+    mask = torch.tensor([mask_row], dtype=torch.uint8)
+    q = inputs.randn((B, steps, Hq, d), seed, torch.bfloat16, DEV)
+    k = inputs.randn((B, T, Hkv, d), seed + 1, torch.bfloat16, DEV)
+    v = inputs.randn((B, T, Hkv, d), seed + 2, torch.bfloat16, DEV)
+    ridx = [g for g in range(Hkv) if mask_row[g]]
+    if plant and ctx > 2:
+        P = ctx // 2
+        ramp = torch.linspace(-2.0, 2.0, d, device=DEV).to(torch.bfloat16)
+        for g in ridx:
+            k[:, P, g] = (3.0 * q[:, 0, g * G].float()).to(torch.bfloat16)
+            v[:, P, g] = ramp
+    cache = DuoCache(1, Hkv, d, mask, S, W, T, batch=B, q_heads=Hq, dtype=torch.bfloat16, retr_fmt="int4")
+    if ctx > 0:
+        cache.append_kv(0, k[:, :ctx].contiguous(), v[:, :ctx].contiguous())
+    outs, lses = [], []
+    for t in range(steps):
+        cache.append_kv(0, k[:, ctx + t:ctx + t + 1].contiguous(), v[:, ctx + t:ctx + t + 1].contiguous())
+        o, l = cache.decode_attention(0, q[:, t].contiguous())
+        outs.append(o.float()[:, None])
+        lses.append(l[:, None])
+    torch.cuda.synchronize()
+    assert cache.device_status() == 0
+    got, got_lse = torch.cat(outs, 1).cpu().numpy(), torch.cat(lses, 1).cpu().numpy()
+    kq = k.float().cpu().numpy().astype(np.float64)
+    vq = v.float().cpu().numpy().astype(np.float64)
+    for g in ridx:
+        for src, dst in ((k, kq), (v, vq)):
+            dst[:, :, g] = _int4_reference(src[:, :, g])[3].reshape(B, T, d)
+    ws, ls = [], []
+    for t in range(steps):
+        w, l = oracle.attend(bits(q[:, t:t + 1]), kq[:, :ctx + t + 1], vq[:, :ctx + t + 1],
+                             np.asarray(mask_row, dtype=bool), S, W, pos0=ctx + t)
+        ws.append(w)
+        ls.append(l)
+    want, want_lse = np.concatenate(ws, 1), np.concatenate(ls, 1)
+    assert_close(got, want, torch.bfloat16, got_lse, want_lse, f"int4 decode Hq{Hq} Hkv{Hkv} B{B} ctx{ctx}")
+    return got, want
+
+
+@pytest.mark.parametrize("Hq,Hkv,mask_row,S,W,B,ctx", [
+    (8, 8, [1, 0, 1, 0, 0, 0, 0, 1], 4, 32, 1, 0),        # first token: sees only itself
+    (8, 8, [1, 0, 1, 0, 0, 0, 0, 1], 4, 32, 2, 37),       # MHA, one ragged tile
+    (16, 8, [1] * 8, 16, 64, 1, 3000),                     # all retrieval, group 2
+    (32, 4, [0, 0, 0, 0], 16, 512, 2, 2000),               # all streaming (bf16 pieces only)
+    (64, 4, [1, 0, 1, 1], 16, 512, 1, 5000),               # group 16
+    (32, 4, [0, 1, 1, 0], 0, 100, 3, 1000),                # group 8, no sinks
+    (32, 8, [0, 1, 0, 1, 1, 0, 0, 1], 16, 512, 1, 1 << 18),  # Llama-3 shape, 256K
+])
+def test_int4_tc_decode_shapes(Hq, Hkv, mask_row, S, W, B, ctx):
+    _int4_decode_check(Hq, Hkv, mask_row, S, W, B, ctx, 2, 90)
+
+
+@pytest.mark.parametrize("Hq,Hkv,B,ctx", [(32, 8, 1, 20000), (8, 8, 2, 5000)])
+def test_int4_tc_decode_planted_needle(Hq, Hkv, B, ctx):
+    """Concentrated attention: the bf16 rounding of p s_v that the MMA sees is
+    compensated exactly, so the output still matches the oracle to bf16 accuracy."""
+    mask_row = [1, 0] * (Hkv // 2)
+    got, want = _int4_decode_check(Hq, Hkv, mask_row, 16, 512, B, ctx, 1, 95, plant=True)
+    G = Hq // Hkv
+    ramp = np.linspace(-2.0, 2.0, 128)
+    for g in range(0, Hkv, 2):  # retrieval heads recover the planted ramp
+        assert np.abs(want[:, 0, g * G] - ramp).max() < 0.3
+        assert np.abs(got[:, 0, g * G] - ramp).max() < 0.3
+
+
 # -------------------------------------------------- tensor-core pre-fill (bf16, d 128)
 
 @pytest.mark.parametrize("B,Hq,Hkv,mask,S,W,chunks", [
