@@ -130,7 +130,8 @@ class ClockSampler:
 def kernel_hash():
     """Hash of the decode kernels' sources: recorded DRAM traffic is void once they change."""
     h = hashlib.sha256()
-    for f in ("k_decode.cu", "k_decode_tc.cu", "device_common.cuh", "duo_internal.h"):
+    for f in ("k_decode.cu", "k_decode_tc.cu", "k_decode_int4_tc.cu", "tcgen05.cuh", "decode_merge.cuh",
+              "device_common.cuh", "duo_internal.h"):
         h.update(open(os.path.join(ROOT, "head_split_kv_duo_b200", "csrc", f), "rb").read())
     return h.hexdigest()[:16]
 
@@ -160,6 +161,8 @@ def run_ours(args, rank, world, dist):
     hbm_peak, tc_peak, tc_sust, peak_src = peaks()
     steps, warmup = args.steps, args.warmup
     Hq, Hkv, nret, ctx, B, nlayers, fmt = DECODE_WORKLOADS[args.workload]
+    if args.layers:
+        nlayers = args.layers
     Hr, Hs = nret, Hkv - nret
     max_len = ctx + warmup + 2 * steps + 16
     mask = inputs.retrieval_mask(nlayers, Hkv, nret, seed=1)
@@ -288,10 +291,11 @@ def run_ours(args, rank, world, dist):
         "us_per_token_layer": round(us_per_token_layer, 3),
         "roofline": {"bound": "hbm", "kernel": "decode", "achieved": round(achieved, 1),
                      "peak": hbm_peak, "peak_source": f"{peak_src} hbm_gbs (burst copy)", "unit": "GB/s",
-                     "frac": round(achieved / hbm_peak, 4), "traffic": recorded_traffic(args.workload),
+                     "frac": round(achieved / hbm_peak, 4), "frac_of_8tbs_spec": round(achieved / 8000.0, 4),
+                     "traffic": recorded_traffic(args.workload),
                      "algorithmic_bytes_per_launch": int(per_launch_bytes), "avg_launch_us": round(dec_avg_ms * 1e3, 3)},
-        # per layer and step: append + decode (+ the split merge on the tcgen05 path)
-        "gpu_launches": steps * nlayers * (3 if fmt == "same" else 2),
+        # per layer and step: append + decode (the split merge runs inside the decode kernel)
+        "gpu_launches": steps * nlayers * 2,
         "clocks": clk.summary(),
         "e2e": e2e,
         "prefill": prefill,
@@ -377,6 +381,8 @@ def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--workload", default=WORKLOAD, choices=sorted(DECODE_WORKLOADS))
+    ap.add_argument("--layers", type=int, default=0,
+                    help="layer caches to rotate through instead of the workload's (small profiling captures)")
     ap.add_argument("--steps", type=int, default=50)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])

@@ -184,14 +184,14 @@ __device__ __forceinline__ int bar_or(int id, int n, int v) {
 
 // Bounded parity wait shared by the roles of a CTA: gives up at once when another role
 // has already given up (abort_flag), or after kWaitLimitNs, latching kDevTimeout.
+// The thread sleeps inside try_wait (woken when the phase completes, or after the
+// hint) instead of spinning, so waiting warps leave the issue slots to working ones.
 __device__ __forceinline__ bool wait_bar(uint32_t bar, uint32_t parity, uint32_t *status, volatile int *abort_flag) {
-#pragma unroll 1
-  for (int i = 0; i < 64; ++i)
-    if (mbar_try_wait(bar, parity)) return true;
+  if (mbar_try_wait_ns(bar, parity, 20000)) return true;
   const unsigned long long t0 = globaltimer();
 #pragma unroll 1
   while (true) {
-    if (mbar_try_wait(bar, parity)) return true;
+    if (mbar_try_wait_ns(bar, parity, 20000)) return true;
     if (*abort_flag) return false;
     if (globaltimer() - t0 > kWaitLimitNs) {
       flag_status(status, kDevTimeout);
