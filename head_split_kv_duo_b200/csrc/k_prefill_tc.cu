@@ -9,11 +9,12 @@
 //     the chunk's own keys, with the Lambda mask j < S or i - j < W.  Key tiles that
 //     hold no visible key for any row of a query tile are never loaded (tile skip).
 //
-// One CTA = one 128-row query tile (a GQA group of heads x 128/G positions); 11 warps:
+// One CTA = one 128-row query tile (a GQA group of heads x 128/G positions); 19 warps:
 //   warp 0      TMA producer: Q once, then K tiles of 128 keys into a 3-stage ring
-//   warp 10     TMA producer: V tiles into a 2-stage ring
+//   warp 18     TMA producer: V tiles into a 2-stage ring
 //   warp 1      TMEM allocator; lane 0 issues every tcgen05.mma
-//   warps 2..9  softmax: two threads per query row (TMEM lane), 64 columns each
+//   warps 2..17 softmax: four threads per query row (TMEM lane), 32 columns each, so
+//               that 16 warps hide the latency of the tensor-memory loads
 // TMEM (512 columns): S double buffer at 0 and 128, O accumulator at 256, P (bf16
 // pairs) double buffer at 384 and 448.
 //   S_j = Q K_j^T      (M 128, N 128, K 128: 8 MMAs of K 16), into S[j % 2]
@@ -30,14 +31,18 @@
 #include <cudaTypedefs.h>
 
 #include "device_common.cuh"
+#include "tcgen05.cuh"
 
 namespace duo {
 
 namespace {
 
-constexpr int kTcThreads = 352;  // warp 0 K/Q TMA, warp 1 MMA + TMEM, warps 2-9 softmax, warp 10 V TMA
 constexpr int kBM = 128;  // query rows per tile
 constexpr int kBN = 128;  // keys per tile
+constexpr int kSplit = 4;                      // softmax threads per query row
+constexpr int kCols = kBN / kSplit;            // S, P and O columns per softmax thread
+constexpr int kVWarp = 2 + 4 * kSplit;         // the V producer follows the softmax warps
+constexpr int kTcThreads = 32 * (kVWarp + 1);  // warp 0 K/Q TMA, warp 1 MMA + TMEM, softmax, V TMA
 constexpr int kD = 128;
 constexpr int kKStages = 3;  // K ring: a stage is free once S_j is computed
 constexpr int kVStages = 2;  // V ring: a stage is free once P_j V_j is computed
@@ -50,8 +55,8 @@ constexpr int kSmK = 32768;                         // K stage s at kSmK + s * 3
 constexpr int kSmV = kSmK + kKStages * 32768;       // V stage s at kSmV + s * 32 KiB
 constexpr int kSmBar = kSmV + kVStages * 32768;
 constexpr int kSmMisc = kSmBar + 256;
-constexpr int kSmXchg = kSmMisc + 1024 + kMaxStrmTiles * 16;  // row max / sum exchange, 6 x 128 floats
-constexpr int kSmTotal = kSmXchg + 6 * 128 * 4;
+constexpr int kSmXchg = kSmMisc + 1024 + kMaxStrmTiles * 16;  // row max / sum exchange, 3 kSplit x 128 floats
+constexpr int kSmTotal = kSmXchg + 3 * kSplit * 128 * 4;
 constexpr int kSmemAlloc = kSmTotal + 1024;  // slack for aligning the base to 1 KiB
 
 // TMEM columns: S double buffer, O accumulator, P double buffer (bf16 pairs, A operand)
@@ -93,7 +98,6 @@ __device__ __forceinline__ void prefetch_map(const CUtensorMap *m) {
 
 __device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
 __device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
-__device__ __forceinline__ void fence_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
 
 __device__ __forceinline__ void tc_commit(uint32_t bar) {
   asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar) : "memory");
@@ -123,43 +127,6 @@ __device__ __forceinline__ void tc_ld32(uint32_t taddr, float (&v)[32]) {
   asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 #pragma unroll
   for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
-}
-
-// 64 consecutive fp32 columns of this thread's TMEM lane (two loads, one wait)
-__device__ __forceinline__ void tc_ld64(uint32_t taddr, float (&v)[64]) {
-  uint32_t r[64];
-#define DUO_LD32(OFF, B)                                                                                        \
-  asm volatile(                                                                                                 \
-      "tcgen05.ld.sync.aligned.32x32b.x32.b32 "                                                                 \
-      "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, "                                 \
-      "%16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];"                \
-      : "=r"(r[B + 0]), "=r"(r[B + 1]), "=r"(r[B + 2]), "=r"(r[B + 3]), "=r"(r[B + 4]), "=r"(r[B + 5]),          \
-        "=r"(r[B + 6]), "=r"(r[B + 7]), "=r"(r[B + 8]), "=r"(r[B + 9]), "=r"(r[B + 10]), "=r"(r[B + 11]),        \
-        "=r"(r[B + 12]), "=r"(r[B + 13]), "=r"(r[B + 14]), "=r"(r[B + 15]), "=r"(r[B + 16]), "=r"(r[B + 17]),    \
-        "=r"(r[B + 18]), "=r"(r[B + 19]), "=r"(r[B + 20]), "=r"(r[B + 21]), "=r"(r[B + 22]), "=r"(r[B + 23]),    \
-        "=r"(r[B + 24]), "=r"(r[B + 25]), "=r"(r[B + 26]), "=r"(r[B + 27]), "=r"(r[B + 28]), "=r"(r[B + 29]),    \
-        "=r"(r[B + 30]), "=r"(r[B + 31])                                                                       \
-      : "r"(taddr + OFF))
-  DUO_LD32(0, 0);
-  DUO_LD32(32, 32);
-#undef DUO_LD32
-  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
-#pragma unroll
-  for (int i = 0; i < 64; ++i) v[i] = __uint_as_float(r[i]);
-}
-
-// store 32 consecutive 32-bit columns of this thread's TMEM lane, and wait for it
-__device__ __forceinline__ void tc_st32u(uint32_t taddr, const uint32_t (&v)[32]) {
-  asm volatile(
-      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "
-      "{%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16, "
-      "%17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31, %32};" ::"r"(taddr),
-      "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]), "r"(v[8]), "r"(v[9]),
-      "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]), "r"(v[15]), "r"(v[16]), "r"(v[17]), "r"(v[18]),
-      "r"(v[19]), "r"(v[20]), "r"(v[21]), "r"(v[22]), "r"(v[23]), "r"(v[24]), "r"(v[25]), "r"(v[26]), "r"(v[27]),
-      "r"(v[28]), "r"(v[29]), "r"(v[30]), "r"(v[31])
-      : "memory");
-  asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
 }
 
 // MMA with A read from tensor memory (bf16 pairs per 32-bit column, K-major)
@@ -205,15 +172,14 @@ constexpr uint32_t idesc_bf16(bool b_mn_major) {
   return (1u << 4) | (1u << 7) | (1u << 10) | ((b_mn_major ? 1u : 0u) << 16) | ((128u >> 3) << 17) | ((128u >> 4) << 24);
 }
 
-// Bounded wait that also gives up at once after another role aborted.
+// Bounded wait that also gives up at once after another role aborted; the thread
+// sleeps inside try_wait (woken when the phase completes) instead of spinning.
 __device__ __forceinline__ bool wait_bar(uint32_t bar, uint32_t parity, uint32_t *status, volatile int *abort_flag) {
-#pragma unroll 1
-  for (int i = 0; i < 64; ++i)
-    if (mbar_try_wait(bar, parity)) return true;
+  if (mbar_try_wait_ns(bar, parity, 20000)) return true;
   const unsigned long long t0 = globaltimer();
 #pragma unroll 1
   while (true) {
-    if (mbar_try_wait(bar, parity)) return true;
+    if (mbar_try_wait_ns(bar, parity, 20000)) return true;
     if (*abort_flag) return false;
     if (globaltimer() - t0 > kWaitLimitNs) {
       flag_status(status, kDevTimeout);
@@ -271,16 +237,16 @@ __device__ __forceinline__ float exp2_poly(float x) {
   return __int_as_float(__float_as_int(p) + (__float_as_int(t) << 23));
 }
 
-// exp2(v*c - mc) of 64 logits, their sum into rs8 and bf16 pairs into pk; logits
-// [POLY, POLY+16) use the FMA-pipe polynomial (POLY < 0: none)
-template <int POLY>
-__device__ __forceinline__ void probabilities(const float (&v)[64], float c, float mc, float (&rs8)[8],
-                                              uint32_t (&pk)[32]) {
+// exp2(v*c - mc) of N logits, their sum into rs8 and bf16 pairs into pk; logits
+// [P0, P0+PN) use the FMA-pipe polynomial (which needs finite arguments), the rest MUFU
+template <int N, int P0, int PN>
+__device__ __forceinline__ void probabilities(const float (&v)[N], float c, float mc, float (&rs8)[8],
+                                              uint32_t (&pk)[N / 2]) {
 #pragma unroll
-  for (int e = 0; e < 64; e += 2) {
+  for (int e = 0; e < N; e += 2) {
     const float x0 = fmaf(v[e], c, -mc), x1 = fmaf(v[e + 1], c, -mc);
     float p0, p1;
-    if (POLY >= 0 && e >= POLY && e < POLY + 16) {
+    if (e >= P0 && e < P0 + PN) {
       p0 = exp2_poly(x0);
       p1 = exp2_poly(x1);
     } else {
@@ -353,7 +319,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) prefill_tc_kernel(const __grid_
 
   if (tid == 0) {
     for (int i = 0; i < kNumBars; ++i)
-      mbar_init(bar(i), (i == kBarSFree || i == kBarSFree + 1 || i == kBarPFull || i == kBarPFull + 1) ? 256 : 1);
+      mbar_init(bar(i), (i == kBarSFree || i == kBarSFree + 1 || i == kBarPFull || i == kBarPFull + 1) ? 128 * kSplit : 1);
     if (smem_u32(smem) & 1023u) flag_status(p.status, kDevTimeout);  // layout assumption (never expected)
     fence_mbar_init();
     *abort_flag = 0;
@@ -393,7 +359,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) prefill_tc_kernel(const __grid_
         load_tile(a, t, pl, g, b, dst, fb, true);
       }
     }
-  } else if (warp == 10) {
+  } else if (warp == kVWarp) {
     // ================= TMA producer: the V ring =================
     if (lane == 0) {
       for (int j = 0; j < nt; ++j) {
@@ -455,14 +421,15 @@ __global__ void __launch_bounds__(kTcThreads, 1) prefill_tc_kernel(const __grid_
       mbar_wait(bar(kBarDrain), 0, p.status);
     }
   } else {
-    // ================= softmax: 8 warps, two threads per query row =================
-    // Warp w reads TMEM lanes 32*(w%4).. (rows) and columns [64*half, 64*half+64) of S,
-    // O and P.  The running max m is a reference: P = exp2(s*c - m) may exceed 1 by up to
-    // 2^kSlack, and m (with O in TMEM and l) is rescaled only when a row's tile maximum
-    // passes m + kSlack.  S is read from TMEM once per tile.
+    // ================= softmax: 4 kSplit warps, kSplit threads per query row =================
+    // Warp w reads TMEM lanes 32*(w%4).. (rows) and columns [kCols*part, kCols*part+kCols)
+    // of S, O and P.  The running max m is a reference: P = exp2(s*c - m) may exceed 1 by
+    // up to 2^kSlack, and m (with O in TMEM and l) is rescaled only when a row's tile
+    // maximum passes m + kSlack.  S is read from TMEM once per tile.
     constexpr float kSlack = 8.0f;
+    constexpr int kSoft = 128 * kSplit;  // softmax threads (named barrier 1)
     const int wq = warp & 3;
-    const int half = (warp - 2) >> 2;
+    const int part = (warp - 2) >> 2;
     const int row = (wq << 5) | lane;
     const uint32_t lane_base = tmem + (static_cast<uint32_t>(wq << 5) << 16);
     const int rpos = row / G;                  // position offset of this row within the block
@@ -470,7 +437,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) prefill_tc_kernel(const __grid_
     const int64_t i = pl.q0 + rpos;            // absolute query position
     const float c = p.scale_log2;
     float m = -INFINITY, l = 0.f;
-    float *xch = reinterpret_cast<float *>(smem + kSmXchg);  // [tile parity][half][row] partial maxima
+    float *xch = reinterpret_cast<float *>(smem + kSmXchg);  // [tile parity][part][row] partial maxima
     bool ok = true;
 
     for (int j = 0; j < nt; ++j) {
@@ -503,15 +470,15 @@ __global__ void __launch_bounds__(kTcThreads, 1) prefill_tc_kernel(const __grid_
 
       if (ok) ok = wait_bar(bar(kBarSFull + (j & 1)), (j >> 1) & 1, p.status, abort_flag);
       tc_fence_after();
-      // this thread's 64 logits of S_j, then the S buffer is released
-      float v[64];
-      tc_ld64(lane_base + kTmS + (j & 1) * 128 + half * 64, v);
+      // this thread's kCols logits of S_j, then the S buffer is released
+      float v[kCols];
+      tc_ld32(lane_base + kTmS + (j & 1) * 128 + part * kCols, v);
       tc_fence_before();
       mbar_arrive(bar(kBarSFree + (j & 1)));
       if (!full_vis) {
 #pragma unroll
-        for (int e = 0; e < 64; ++e) {
-          const int col = half * 64 + e;
+        for (int e = 0; e < kCols; ++e) {
+          const int col = part * kCols + e;
           const bool vis = col <= hi && (col < sink_c || col > win_c);
           v[e] = vis ? v[e] : -INFINITY;
         }
@@ -520,12 +487,13 @@ __global__ void __launch_bounds__(kTcThreads, 1) prefill_tc_kernel(const __grid_
 #pragma unroll
       for (int u = 0; u < 8; ++u) mx8[u] = v[u];
 #pragma unroll
-      for (int e = 8; e < 64; ++e) mx8[e & 7] = fmaxf(mx8[e & 7], v[e]);
+      for (int e = 8; e < kCols; ++e) mx8[e & 7] = fmaxf(mx8[e & 7], v[e]);
       float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
                        fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
-      xch[((j & 1) * 2 + half) * kBM + row] = mx;
-      named_sync(1, 256);
-      mx = fmaxf(mx, xch[((j & 1) * 2 + (half ^ 1)) * kBM + row]);
+      xch[((j & 1) * kSplit + part) * kBM + row] = mx;
+      named_sync(1, kSoft);
+#pragma unroll
+      for (int o = 1; o < kSplit; ++o) mx = fmaxf(mx, xch[((j & 1) * kSplit + ((part + o) % kSplit)) * kBM + row]);
       const float tmax = mx * c;  // -inf when nothing in the tile is visible
       const bool need = tmax > m + kSlack;
       float alpha = 1.f;
@@ -536,18 +504,15 @@ __global__ void __launch_bounds__(kTcThreads, 1) prefill_tc_kernel(const __grid_
       l *= alpha;
       bool waited = false;
       if (j >= 1 && __any_sync(0xffffffffu, need)) {
-        // rescale this thread's 64 columns of O once P_{j-1} V_{j-1} has landed
+        // rescale this thread's kCols columns of O once P_{j-1} V_{j-1} has landed
         if (ok) ok = wait_bar(bar(kBarOFull), (j - 1) & 1, p.status, abort_flag);
         tc_fence_after();
-#pragma unroll 1
-        for (int cc = 0; cc < 2; ++cc) {
-          float w[32];
-          const uint32_t oa = lane_base + kTmO + half * 64 + cc * 32;
-          tc_ld32(oa, w);
+        float w[kCols];
+        const uint32_t oa = lane_base + kTmO + part * kCols;
+        tc_ld32(oa, w);
 #pragma unroll
-          for (int e = 0; e < 32; ++e) w[e] *= alpha;
-          tc_st32(oa, w);
-        }
+        for (int e = 0; e < kCols; ++e) w[e] *= alpha;
+        tc_st32(oa, w);
         waited = true;
       }
       // probabilities (masked logits are -inf and give 0), row sum, bf16 pairs of P_j
@@ -555,13 +520,13 @@ __global__ void __launch_bounds__(kTcThreads, 1) prefill_tc_kernel(const __grid_
 #pragma unroll
       for (int u = 0; u < 8; ++u) rs8[u] = 0.f;
       const float mc = (m == -INFINITY) ? 0.f : m;
-      uint32_t pk[32];
-      // a quarter of the exponentials of interior tiles on the FMA pipe, the rest on MUFU
-      if (!full_vis) probabilities<-1>(v, c, mc, rs8, pk);
-      else if (half == 0) probabilities<16>(v, c, mc, rs8, pk);
-      else probabilities<48>(v, c, mc, rs8, pk);
+      uint32_t pk[kCols / 2];
+      // 3/8 of the exponentials of interior tiles on the FMA pipe, the rest on MUFU
+      if (!full_vis) probabilities<kCols, 0, 0>(v, c, mc, rs8, pk);
+      else probabilities<kCols, 0, kCols * 3 / 8>(v, c, mc, rs8, pk);
       // P_j into TMEM buffer j % 2 (its previous reader P_{j-2} V_{j-2} was waited for at j-1)
-      tc_st32u(lane_base + kTmP + (j & 1) * 64 + half * 32, pk);
+      tc::st16(lane_base + kTmP + (j & 1) * 64 + part * (kCols / 2), pk);
+      tc::st_wait();
       // one wait per P V product, in order (here unless the rescale already waited)
       if (j >= 1 && !waited) {
         if (ok) ok = wait_bar(bar(kBarOFull), (j - 1) & 1, p.status, abort_flag);
@@ -570,35 +535,36 @@ __global__ void __launch_bounds__(kTcThreads, 1) prefill_tc_kernel(const __grid_
       tc_fence_before();
       mbar_arrive(bar(kBarPFull + (j & 1)));
     }
-    // the last product, then the row's normaliser from both halves
+    // the last product, then the row's normaliser from all parts
     if (nt > 0 && ok) ok = wait_bar(bar(kBarOFull), (nt - 1) & 1, p.status, abort_flag);
     tc_fence_after();
-    float *xl = xch + 4 * kBM;  // [half][row]
-    xl[half * kBM + row] = l;
-    named_sync(1, 256);
-    const float lrow = l + xl[(half ^ 1) * kBM + row];
-    // epilogue: normalise and store this thread's 64 dims of the row (bf16) and its lse
+    float *xl = xch + 2 * kSplit * kBM;  // [part][row]
+    xl[part * kBM + row] = l;
+    named_sync(1, kSoft);
+    float lrow = 0.f;
+#pragma unroll
+    for (int o = 0; o < kSplit; ++o) lrow += xl[o * kBM + row];
+    // epilogue: normalise and store this thread's kCols dims of the row (bf16) and its lse
     const bool store = r0 + rpos < p.n;
-    char *orow = p.out + ((static_cast<int64_t>(b) * p.n + r0 + rpos) * p.Hq + h) * (kD * 2) + half * 128;
+    char *orow = p.out + ((static_cast<int64_t>(b) * p.n + r0 + rpos) * p.Hq + h) * (kD * 2) + part * (kCols * 2);
     const float inv = 1.f / lrow;
-#pragma unroll 1
-    for (int cc = 0; cc < 2; ++cc) {
-      float w[32];
-      tc_ld32(lane_base + kTmO + half * 64 + cc * 32, w);
+    {
+      float w[kCols];
+      tc_ld32(lane_base + kTmO + part * kCols, w);
       if (store) {
 #pragma unroll
-        for (int q = 0; q < 4; ++q) {
+        for (int q = 0; q < kCols / 8; ++q) {
           uint32_t wd[4];
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
             const __nv_bfloat162 pb = __floats2bfloat162_rn(w[8 * q + 2 * e] * inv, w[8 * q + 2 * e + 1] * inv);
             wd[e] = *reinterpret_cast<const uint32_t *>(&pb);
           }
-          *reinterpret_cast<uint4 *>(orow + cc * 64 + q * 16) = make_uint4(wd[0], wd[1], wd[2], wd[3]);
+          *reinterpret_cast<uint4 *>(orow + q * 16) = make_uint4(wd[0], wd[1], wd[2], wd[3]);
         }
       }
     }
-    if (store && half == 0 && p.lse) p.lse[(static_cast<int64_t>(b) * p.n + r0 + rpos) * p.Hq + h] = (m + lg2(lrow)) * kLn2;
+    if (store && part == 0 && p.lse) p.lse[(static_cast<int64_t>(b) * p.n + r0 + rpos) * p.Hq + h] = (m + lg2(lrow)) * kLn2;
   }
 
   tc_fence_before();
