@@ -225,38 +225,80 @@ __device__ int streaming_tiles(const PrefillParams &p, int r0, int npos, TileDes
   return nt;
 }
 
-// 2^x for x <= 0 on the FMA pipe: x = n + f with n the nearest integer (|f| <= 1/2),
-// 2^f by a cubic fitted for this kernel by weighted least squares on [-1/2, 1/2]
-// (maximum relative error 1.0e-4, below bf16's 2^-9), and n added to the exponent.
-__device__ __forceinline__ float exp2_poly(float x) {
-  x = fmaxf(x, -126.0f);
-  const float t = x + 12582912.0f;  // 1.5 * 2^23: the integer nearest x lands in t's low bits
-  const float n = t - 12582912.0f;
-  const float f = x - n;
-  const float p = fmaf(fmaf(fmaf(0.05500858f, f, 0.24221036f), f, 0.6932829f), f, 1.0f);
-  return __int_as_float(__float_as_int(p) + (__float_as_int(t) << 23));
+// ---- packed fp32 pairs (sm_100 f32x2 arithmetic: two lanes per instruction) ----
+__device__ __forceinline__ uint64_t pack2(float a, float b) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(a), "f"(b));
+  return r;
+}
+__device__ __forceinline__ void unpack2(uint64_t v, float &a, float &b) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(a), "=f"(b) : "l"(v));
+}
+__device__ __forceinline__ uint64_t ffma2(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+__device__ __forceinline__ uint64_t fadd2(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
 }
 
-// exp2(v*c - mc) of N logits, their sum into rs8 and bf16 pairs into pk; logits
-// [P0, P0+PN) use the FMA-pipe polynomial (which needs finite arguments), the rest MUFU
+// 2^x of a pair on the FMA pipe: x = n + f with n the nearest integer (|f| <= 1/2),
+// 2^f by a cubic fitted for this kernel by weighted least squares on [-1/2, 1/2]
+// (maximum relative error 1.0e-4, below bf16's 2^-9), and n added to the exponent
+// field.  Arguments below -126 give 2^-126 (the callers' tiles hold no -inf).
+__device__ __forceinline__ void exp2_poly2(uint64_t x2, float &r0, float &r1) {
+  float x0, x1;
+  unpack2(x2, x0, x1);
+  x2 = pack2(fmaxf(x0, -126.0f), fmaxf(x1, -126.0f));
+  const uint64_t t = fadd2(x2, pack2(12582912.0f, 12582912.0f));  // 1.5 * 2^23: rounds to an integer
+  const uint64_t n = fadd2(t, pack2(-12582912.0f, -12582912.0f));
+  const uint64_t f = ffma2(n, pack2(-1.0f, -1.0f), x2);  // x - n, exact
+  uint64_t q = ffma2(pack2(0.05500858f, 0.05500858f), f, pack2(0.24221036f, 0.24221036f));
+  q = ffma2(q, f, pack2(0.6932829f, 0.6932829f));
+  q = ffma2(q, f, pack2(1.0f, 1.0f));
+  float q0, q1, t0, t1;
+  unpack2(q, q0, q1);
+  unpack2(t, t0, t1);
+  r0 = __int_as_float(__float_as_int(q0) + (__float_as_int(t0) << 23));
+  r1 = __int_as_float(__float_as_int(q1) + (__float_as_int(t1) << 23));
+}
+
+// exp2(v*c - mc) of N logits, their sum into rowsum and bf16 pairs into pk; logits
+// [P0, P0+PN) use the FMA-pipe polynomial (which needs finite arguments), the rest MUFU.
+// The scaling and the sums run on packed fp32 pairs.
 template <int N, int P0, int PN>
-__device__ __forceinline__ void probabilities(const float (&v)[N], float c, float mc, float (&rs8)[8],
+__device__ __forceinline__ void probabilities(const float (&v)[N], float c, float mc, float &rowsum,
                                               uint32_t (&pk)[N / 2]) {
+  const uint64_t cc = pack2(c, c), mm = pack2(-mc, -mc);
+  uint64_t acc[2] = {pack2(0.f, 0.f), pack2(0.f, 0.f)};
 #pragma unroll
   for (int e = 0; e < N; e += 2) {
-    const float x0 = fmaf(v[e], c, -mc), x1 = fmaf(v[e + 1], c, -mc);
+    const uint64_t x = ffma2(pack2(v[e], v[e + 1]), cc, mm);
     float p0, p1;
     if (e >= P0 && e < P0 + PN) {
-      p0 = exp2_poly(x0);
-      p1 = exp2_poly(x1);
+      exp2_poly2(x, p0, p1);
     } else {
+      float x0, x1;
+      unpack2(x, x0, x1);
       p0 = ex2(x0);
       p1 = ex2(x1);
     }
-    rs8[(e >> 1) & 7] += p0 + p1;
+    acc[(e >> 1) & 1] = fadd2(acc[(e >> 1) & 1], pack2(p0, p1));
     const __nv_bfloat162 pb = __floats2bfloat162_rn(p0, p1);
     pk[e >> 1] = *reinterpret_cast<const uint32_t *>(&pb);
   }
+  float a0, a1, b0, b1;
+  unpack2(acc[0], a0, a1);
+  unpack2(acc[1], b0, b1);
+  rowsum = (a0 + a1) + (b0 + b1);
 }
 
 // A key offset relative to a tile start, clamped to [-1, 127].
@@ -483,13 +525,12 @@ __global__ void __launch_bounds__(kTcThreads, 1) prefill_tc_kernel(const __grid_
           v[e] = vis ? v[e] : -INFINITY;
         }
       }
-      float mx8[8];
+      float mx4[4];  // four independent chains of three-input maxima
 #pragma unroll
-      for (int u = 0; u < 8; ++u) mx8[u] = v[u];
+      for (int u = 0; u < 4; ++u) mx4[u] = fmaxf(v[2 * u], v[2 * u + 1]);
 #pragma unroll
-      for (int e = 8; e < kCols; ++e) mx8[e & 7] = fmaxf(mx8[e & 7], v[e]);
-      float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
-                       fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
+      for (int e = 8; e < kCols; e += 2) mx4[(e >> 1) & 3] = fmax3(mx4[(e >> 1) & 3], v[e], v[e + 1]);
+      float mx = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3]));
       xch[((j & 1) * kSplit + part) * kBM + row] = mx;
       named_sync(1, kSoft);
 #pragma unroll
@@ -516,14 +557,12 @@ __global__ void __launch_bounds__(kTcThreads, 1) prefill_tc_kernel(const __grid_
         waited = true;
       }
       // probabilities (masked logits are -inf and give 0), row sum, bf16 pairs of P_j
-      float rs8[8];
-#pragma unroll
-      for (int u = 0; u < 8; ++u) rs8[u] = 0.f;
+      float rsum;
       const float mc = (m == -INFINITY) ? 0.f : m;
       uint32_t pk[kCols / 2];
       // 3/8 of the exponentials of interior tiles on the FMA pipe, the rest on MUFU
-      if (!full_vis) probabilities<kCols, 0, 0>(v, c, mc, rs8, pk);
-      else probabilities<kCols, 0, kCols * 3 / 8>(v, c, mc, rs8, pk);
+      if (!full_vis) probabilities<kCols, 0, 0>(v, c, mc, rsum, pk);
+      else probabilities<kCols, 0, kCols * 3 / 8>(v, c, mc, rsum, pk);
       // P_j into TMEM buffer j % 2 (its previous reader P_{j-2} V_{j-2} was waited for at j-1)
       tc::st16(lane_base + kTmP + (j & 1) * 64 + part * (kCols / 2), pk);
       tc::st_wait();
@@ -531,7 +570,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) prefill_tc_kernel(const __grid_
       if (j >= 1 && !waited) {
         if (ok) ok = wait_bar(bar(kBarOFull), (j - 1) & 1, p.status, abort_flag);
       }
-      l += ((rs8[0] + rs8[1]) + (rs8[2] + rs8[3])) + ((rs8[4] + rs8[5]) + (rs8[6] + rs8[7]));
+      l += rsum;
       tc_fence_before();
       mbar_arrive(bar(kBarPFull + (j & 1)));
     }
