@@ -60,6 +60,9 @@ def _load():
             lib.oracle_attend.restype = i32
             lib.oracle_attend.argtypes = [i32, i64, i32, i32, i32, vp, i32, i64, vp, vp, i32, i64, vp, i64, i64,
                                           dbl, vp, i64, vp, vp, i32]
+            lib.oracle_gated.restype = i32
+            lib.oracle_gated.argtypes = [i32, i64, i32, i32, i32, vp, i32, vp, vp, i32, vp, i64, i64, dbl, vp, i64,
+                                         vp]
             lib.oracle_visible.restype = i32
             lib.oracle_visible.argtypes = [i64, i64, i32, i64, i64]
             lib.oracle_retained.restype = None
@@ -146,6 +149,38 @@ def attend(q, k, v, retrieval, S: int, W: int, pos0: int, scale: float | None = 
     if rows is None:
         return out.reshape(B, nq, Hq, d), lse.reshape(B, nq, Hq)
     return out, lse
+
+
+def gated(q, k, v, alpha, S: int, W: int, scale: float | None = None, rows=None):
+    """Gated mixed attention over whole sequences: alpha[g] * causal attention +
+    (1 - alpha[g]) * Lambda-masked attention, per KV head g (the plain definition).
+
+    q: [B][L][Hq][d], k, v: [B][L][Hkv][d] (positions 0..L-1); alpha: [Hkv] floats.
+    Returns out [rows][d] or [B][L][Hq][d] float64.
+    """
+    qa, qt = _as_input(q)
+    ka, kt = _as_input(k)
+    va, vt = _as_input(v)
+    if kt != vt:
+        raise TypeError("k and v must share a dtype")
+    B, L, Hq, d = qa.shape
+    if ka.shape[:2] != (B, L) or ka.shape[3] != d or va.shape != ka.shape or Hq % ka.shape[2]:
+        raise ValueError("shape mismatch")
+    Hkv = ka.shape[2]
+    al = np.ascontiguousarray(np.asarray(alpha, dtype=np.float64).reshape(Hkv))
+    if rows is None:
+        n = B * L * Hq
+        rows_arr = None
+    else:
+        rows_arr = np.ascontiguousarray(np.asarray(rows, dtype=np.int64))
+        n = rows_arr.size
+    out = np.empty((n, d), dtype=np.float64)
+    rc = _load().oracle_gated(B, L, Hq, Hkv, d, _ptr(qa), qt, _ptr(ka), _ptr(va), kt, _ptr(al), S, W,
+                              0.0 if scale is None else float(scale),
+                              None if rows_arr is None else _ptr(rows_arr), n, _ptr(out))
+    if rc != 0:
+        raise ValueError(f"oracle_gated failed ({rc})")
+    return out.reshape(B, L, Hq, d) if rows is None else out
 
 
 def retained(length: int, S: int, W: int) -> np.ndarray:

@@ -170,6 +170,77 @@ int oracle_attend(int B, int64_t nq, int Hq, int Hkv, int d, const void *q, int 
 }
 
 /*
+ * Gated mixed attention of the identification phase ("Gate Parameterization"): for
+ * KV head g with gate alpha[g] in [0, 1], the output of each of its query heads is
+ *   alpha[g] * full_attn + (1 - alpha[g]) * streaming_attn
+ * with full_attn under the causal mask and streaming_attn under the Lambda mask ("The
+ * Full and Streaming Attention Masks"), both over the same scaled logits.
+ *
+ *   q [B][L][Hq][d], k, v [B][L][Hkv][d]: one sequence per batch entry, positions 0..L-1
+ *   alpha [Hkv] fp64; rows / nrows / out as in oracle_attend (row id = (b*L + i)*Hq + h)
+ */
+int oracle_gated(int B, int64_t L, int Hq, int Hkv, int d, const void *q, int q_dtype, const void *k,
+                 const void *v, int kv_dtype, const double *alpha, int64_t S, int64_t W, double scale,
+                 const int64_t *rows, int64_t nrows, double *out) {
+  if (scale <= 0.0) scale = 1.0 / sqrt((double)d);
+  const int G = Hq / Hkv;
+  const int64_t total = rows ? nrows : (int64_t)B * L * Hq;
+  int bad = 0;
+
+#pragma omp parallel
+  {
+    double *s = (double *)malloc(sizeof(double) * (size_t)(L > 0 ? L : 1));
+    double *of = (double *)malloc(sizeof(double) * (size_t)d);
+    double *os = (double *)malloc(sizeof(double) * (size_t)d);
+    if (!s || !of || !os) {
+#pragma omp atomic write
+      bad = 1;
+    }
+#pragma omp for schedule(dynamic, 1)
+    for (int64_t t = 0; t < total; ++t) {
+      if (!s || !of || !os) continue;
+      const int64_t id = rows ? rows[t] : t;
+      const int h = (int)(id % Hq);
+      const int64_t i = (id / Hq) % L;
+      const int64_t b = id / ((int64_t)Hq * L);
+      const int g = h / G;
+      const int64_t qoff = ((b * L + i) * Hq + h) * (int64_t)d;
+
+      /* the scaled logits of every key the causal mask admits, and both maxima */
+      double mf = -INFINITY, ms = -INFINITY;
+      for (int64_t j = 0; j <= i; ++j) {
+        const int64_t koff = ((b * L + j) * Hkv + g) * (int64_t)d;
+        double dot = 0.0;
+        for (int e = 0; e < d; ++e) dot += load_elem(q, q_dtype, qoff + e) * load_elem(k, kv_dtype, koff + e);
+        s[j] = scale * dot;
+        if (s[j] > mf) mf = s[j];
+        if (oracle_visible(i, j, 0, S, W) && s[j] > ms) ms = s[j];
+      }
+      /* two softmax normalisers and two weighted sums of the value rows */
+      double Zf = 0.0, Zs = 0.0;
+      for (int e = 0; e < d; ++e) of[e] = os[e] = 0.0;
+      for (int64_t j = 0; j <= i; ++j) {
+        const int64_t voff = ((b * L + j) * Hkv + g) * (int64_t)d;
+        const double wf = exp(s[j] - mf);
+        Zf += wf;
+        for (int e = 0; e < d; ++e) of[e] += wf * load_elem(v, kv_dtype, voff + e);
+        if (oracle_visible(i, j, 0, S, W)) {
+          const double ws = exp(s[j] - ms);
+          Zs += ws;
+          for (int e = 0; e < d; ++e) os[e] += ws * load_elem(v, kv_dtype, voff + e);
+        }
+      }
+      const double a = alpha[g];
+      for (int e = 0; e < d; ++e) out[t * d + e] = a * (of[e] / Zf) + (1.0 - a) * (os[e] / Zs);
+    }
+    free(s);
+    free(of);
+    free(os);
+  }
+  return bad ? -2 : 0;
+}
+
+/*
  * Retained set of a streaming head after `len` tokens, in closed form:
  * the sinks {p < min(S, len)} and the recent tokens {max(S, len-W) <= p < len}
  * ("Decoding Procedure" step 3 and Figure 5, reading R1).

@@ -167,6 +167,53 @@ def test_streaming_without_sinks_is_sliding_window(W):
     np.testing.assert_allclose(out, _sdpa(q, k, v, band), rtol=0, atol=1e-12)
 
 
+# ------------------------------------------------------- gated mixed attention
+
+def _lambda_mask(L, S, W):
+    """The Lambda mask of 'The Full and Streaming Attention Masks' as a union of a
+    causal band of width W (query included) and the first S columns, below the diagonal."""
+    causal = np.tril(np.ones((L, L), dtype=bool))
+    band = causal & np.triu(np.ones((L, L), dtype=bool), k=-(W - 1))
+    sinks = causal & (np.arange(L)[None, :] < S)
+    return band | sinks
+
+
+@pytest.mark.parametrize("B,Hq,Hkv,d,L,S,W", [(1, 4, 2, 16, 40, 3, 7), (2, 6, 3, 8, 25, 0, 4), (1, 2, 1, 32, 19, 5, 1)])
+def test_gated_is_mixture_of_causal_and_lambda_sdpa(B, Hq, Hkv, d, L, S, W):
+    """'Gate Parameterization': attn = alpha * full_attn + (1 - alpha) * streaming_attn
+    per KV head; both terms from torch SDPA (float64) under the two masks."""
+    q, k, v = _rand((B, L, Hq, d), 31), _rand((B, L, Hkv, d), 32), _rand((B, L, Hkv, d), 33)
+    alpha = np.linspace(0.0, 1.0, Hkv) if Hkv > 1 else np.array([0.37])
+    full = _sdpa(q, k, v, np.tril(np.ones((L, L), dtype=bool)))
+    lam = _sdpa(q, k, v, _lambda_mask(L, S, W))
+    a = np.repeat(alpha, Hq // Hkv)[None, None, :, None]
+    want = a * full + (1.0 - a) * lam
+    np.testing.assert_allclose(oracle.gated(q, k, v, alpha, S, W), want, rtol=0, atol=1e-12)
+
+
+def test_gated_end_points_and_sampled_rows():
+    """alpha = 1 is the retrieval (causal) head and alpha = 0 the streaming head of the
+    cache attention; sampled rows equal the same rows of the full evaluation."""
+    B, Hq, Hkv, d, L, S, W = 1, 4, 2, 16, 30, 2, 5
+    q, k, v = _rand((B, L, Hq, d), 34), _rand((B, L, Hkv, d), 35), _rand((B, L, Hkv, d), 36)
+    g = oracle.gated(q, k, v, [1.0, 0.0], S, W)
+    att, _ = oracle.attend(q, k, v, [True, False], S=S, W=W, pos0=0)
+    np.testing.assert_allclose(g, att, rtol=0, atol=1e-12)
+    rows = np.array([0, 7, 33, L * Hq - 1])
+    np.testing.assert_array_equal(oracle.gated(q, k, v, [0.2, 0.9], S, W, rows=rows),
+                                  oracle.gated(q, k, v, [0.2, 0.9], S, W).reshape(-1, d)[rows])
+
+
+def test_gated_wrong_gate_is_caught():
+    """A gate applied to the wrong KV head (or swapped terms) moves the output far
+    outside any tolerance on these inputs."""
+    B, Hq, Hkv, d, L, S, W = 1, 4, 2, 16, 60, 2, 5
+    q, k, v = _rand((B, L, Hq, d), 37), _rand((B, L, Hkv, d), 38), _rand((B, L, Hkv, d), 39)
+    good = oracle.gated(q, k, v, [0.1, 0.8], S, W)
+    assert np.abs(oracle.gated(q, k, v, [0.8, 0.1], S, W) - good).max() > 0.05
+    assert np.abs(oracle.gated(q, k, v, [0.9, 0.2], S, W) - good).max() > 0.05
+
+
 def _enumerated_visible(i, is_retrieval, S, W):
     """Visible keys of query i as a union of ranges: all earlier keys for a retrieval
     head; the first S tokens plus the W newest (query included) for a streaming head."""
