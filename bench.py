@@ -67,6 +67,15 @@ def prefill_flops(L=PREFILL_LEN, Hq=HQ, d=D, G=HQ // HKV, nret=NRET):
     return 4 * d * G * (nret * retr_pairs + (HKV - nret) * strm_pairs)
 
 
+def gated_flops(L, Hq=HQ, d=D):
+    """Algorithmic FLOPs of the gated forward over one sequence: every query head pays
+    4 d per causally visible pair (full term) plus 4 d per Lambda-visible pair."""
+    causal = L * (L + 1) // 2
+    sw = S + W
+    lam = sw * (sw + 1) // 2 + (L - sw) * sw if L > sw else causal
+    return 4 * d * Hq * (causal + lam)
+
+
 def peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(path):
@@ -278,6 +287,9 @@ def run_ours(args, rank, world, dist):
     prefill = None
     if not args.skip_prefill:
         prefill = run_prefill(args, dev, tc_peak, tc_sust, peak_src)
+    gated = None
+    if not args.skip_gated:
+        gated = run_gated(args, dev, tc_peak, tc_sust, peak_src)
 
     kv_gb = nlayers * nbytes_of(ctx) / 1e9
     res = {
@@ -299,6 +311,7 @@ def run_ours(args, rank, world, dist):
         "clocks": clk.summary(),
         "e2e": e2e,
         "prefill": prefill,
+        "gated": gated,
     }
     return res
 
@@ -342,6 +355,40 @@ def run_prefill(args, dev, tc_peak, tc_sust, peak_src):
     name = f"llama3-8b-gqa-prefill-{L // 1024}k-chunk{C // 1024}k"
     return {"workload": name, "tflops": round(tflops, 1), "ms": round(ms, 2),
             "steps": args.prefill_steps, "algorithmic_tflop": round(fl / 1e12, 2),
+            "roofline": {"bound": "tensor", "achieved": round(tflops, 1), "peak": tc_peak,
+                         "peak_source": f"{peak_src} bf16_tflops (burst)", "unit": "TFLOP/s",
+                         "frac": round(tflops / tc_peak, 4), "frac_of_sustained": round(tflops / tc_sust, 4)}}
+
+
+def run_gated(args, dev, tc_peak, tc_sust, peak_src):
+    """Gated mixed attention of the identification phase on a Llama-3-8B-shaped layer
+    (32 q / 8 kv heads, d 128, S 16, W 512) over one sequence of args.gated_len tokens."""
+    import torch
+
+    from head_split_kv_duo_b200 import inputs
+    from head_split_kv_duo_b200.duo import gated_attention
+
+    L = args.gated_len
+    q = inputs.randn((1, L, HQ, D), 300, device=dev)
+    k = inputs.randn((1, L, HKV, D), 301, device=dev)
+    v = inputs.randn((1, L, HKV, D), 302, device=dev)
+    alpha = torch.rand(HKV, generator=torch.Generator().manual_seed(3)).to(dev)
+    out = torch.empty_like(q)
+    stream = torch.cuda.current_stream()
+    times = []
+    for i in range(4):
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        gated_attention(q, k, v, alpha, S, W, out=out, stream=stream)
+        b.record(stream)
+        torch.cuda.synchronize()
+        if i > 0:
+            times.append(a.elapsed_time(b))
+    ms = statistics.mean(times)
+    fl = gated_flops(L)
+    tflops = fl / (ms * 1e-3) / 1e12
+    return {"workload": f"llama3-8b-gqa-gated-{L // 1024}k", "tflops": round(tflops, 1), "ms": round(ms, 3),
+            "steps": len(times), "algorithmic_tflop": round(fl / 1e12, 3),
             "roofline": {"bound": "tensor", "achieved": round(tflops, 1), "peak": tc_peak,
                          "peak_source": f"{peak_src} bf16_tflops (burst)", "unit": "TFLOP/s",
                          "frac": round(tflops / tc_peak, 4), "frac_of_sustained": round(tflops / tc_sust, 4)}}
@@ -391,6 +438,8 @@ def main():
     ap.add_argument("--prefill-len", type=int, default=PREFILL_LEN)
     ap.add_argument("--prefill-chunk", type=int, default=PREFILL_CHUNK)
     ap.add_argument("--skip-e2e", action="store_true")
+    ap.add_argument("--skip-gated", action="store_true", help="skip the gated (identification-phase) forward")
+    ap.add_argument("--gated-len", type=int, default=32768)
     ap.add_argument("--skip-cpu-baseline", action="store_true")
     ap.add_argument("--prefill-steps", type=int, default=2)
     ap.add_argument("--prefill-warmup", type=int, default=1)
@@ -432,7 +481,10 @@ def main():
         torch.cuda.set_device(dev)
         _, tc_peak, tc_sust, src = peaks()
         if rank == 0:
-            print(json.dumps({"prefill": run_prefill(args, dev, tc_peak, tc_sust, src)}))
+            res = {"prefill": run_prefill(args, dev, tc_peak, tc_sust, src)}
+            if not args.skip_gated:
+                res["gated"] = run_gated(args, dev, tc_peak, tc_sust, src)
+            print(json.dumps(res))
         return 0
     res = run_ours(args, rank, world, dist)
     if rank == 0 and not args.skip_cpu_baseline:

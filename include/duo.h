@@ -221,11 +221,37 @@ DUO_API duo_status duo_get_device_status(duo_cache *cache, void *cuda_stream);
  * stream capture.
  * Limits: bf16 caches with head_dim 128, not INT4, at most 16 query heads per KV head
  * (else DUO_ERR_UNSUPPORTED).  The partials of B*kv_heads heads must fit the array at
- * one CTA: B*kv_heads*G*(head_dim+2)*4 bytes <= 4 MiB less the tickets, else
+ * one CTA: B*kv_heads*G*(head_dim+4)*4 bytes <= 4 MiB less the tickets, else
  * DUO_ERR_CAPACITY; larger head counts still fit but run on fewer CTAs.
  */
 DUO_API duo_status duo_decode_attention_static_scratch(duo_cache *cache, int layer, const void *q, void *out,
                                                        float *lse, void *cuda_stream);
+
+/*
+ * Gated mixed attention of the identification phase ("Gate Parameterization"): over
+ * whole sequences (positions 0..L-1, no cache), the output of every query head of KV
+ * head g is
+ *     alpha[g] * full_attn + (1 - alpha[g]) * streaming_attn
+ * with full_attn under the causal mask and streaming_attn under the Lambda mask of
+ * sinks S and window W ("The Full and Streaming Attention Masks"; same mask reading as
+ * the cache calls).  Training the gates is not part of this library.
+ *   q, out   device [B][L][Hq][d];  k, v  device [B][L][Hkv][d]  (dtype bf16 or fp32)
+ *   alpha    device [Hkv] fp32, one gate per KV head (values outside [0, 1] are used
+ *            as given)
+ *   softmax_scale  0 means 1/sqrt(head_dim)
+ *   workspace      caller-owned device buffer of >= duo_gated_workspace_bytes() bytes,
+ *                  256-byte aligned; its contents are scratch (the K/V copy and the
+ *                  streaming term); it must not be used by another call meanwhile.
+ * The causal term is written to `out`, the Lambda term to the workspace, and one
+ * elementwise kernel mixes them in place.  Launches on `cuda_stream`; arguments are
+ * checked before any launch (DUO_ERR_INVALID; DUO_ERR_CAPACITY for a short workspace).
+ */
+DUO_API size_t duo_gated_workspace_bytes(int batch, int seq_len, int q_heads, int kv_heads, int head_dim,
+                                         duo_dtype dtype, int S, int W);
+DUO_API duo_status duo_gated_attention(const void *q, const void *k, const void *v, int batch, int seq_len,
+                                       int q_heads, int kv_heads, int head_dim, duo_dtype dtype, const float *alpha,
+                                       int S, int W, float softmax_scale, void *out, void *workspace,
+                                       size_t workspace_bytes, void *cuda_stream);
 
 /* Static description of a status code. */
 DUO_API const char *duo_status_str(duo_status status);

@@ -161,3 +161,38 @@ def test_regions_are_disjoint_and_inside_the_buffer():
 def test_status_strings():
     for s in range(6):
         assert duo.duo_status_str(s)
+
+
+# ------------------------------------------------------- gated mixed attention
+
+def test_gated_workspace_bytes():
+    """Two one-layer caches (all retrieval, all streaming) plus the streaming term."""
+    B, L, Hq, Hkv, d, S, W = 2, 1000, 8, 4, 128, 4, 16
+    n = duo.duo_gated_workspace_bytes(B, L, Hq, Hkv, d, duo.DUO_BF16, S, W)
+    full = duo.duo_cache_bytes(1, Hkv, d, np.ones(Hkv, np.uint8), S, W, L, duo._opts(batch=B, q_heads=Hq))
+    strm = duo.duo_cache_bytes(1, Hkv, d, np.zeros(Hkv, np.uint8), S, W, L, duo._opts(batch=B, q_heads=Hq))
+    assert n >= full + strm + B * L * Hq * d * 2
+    assert duo.duo_gated_workspace_bytes(B, L, Hq, Hkv, 96, duo.DUO_BF16, S, W) == 0  # head_dim
+    assert duo.duo_gated_workspace_bytes(B, L, 6, 4, d, duo.DUO_BF16, S, W) == 0       # Hq % Hkv
+    assert duo.duo_gated_workspace_bytes(B, 0, Hq, Hkv, d, duo.DUO_BF16, S, W) == 0    # empty sequence
+    assert duo.duo_gated_workspace_bytes(B, L, Hq, Hkv, d, duo.DUO_BF16, S, 0) == 0    # W >= 1
+
+
+def test_gated_checks_arguments_before_any_launch():
+    B, L, Hq, Hkv, d, S, W = 1, 100, 4, 2, 64, 2, 8
+    n = duo.duo_gated_workspace_bytes(B, L, Hq, Hkv, d, duo.DUO_FP32, S, W)
+    p = FAKE
+
+    def call(**kw):
+        a = dict(q=p, k=p, v=p, alpha=p, out=p, ws=p, nb=n, scale=0.0, L=L)
+        a.update(kw)
+        return duo.duo_gated_attention(a["q"], a["k"], a["v"], B, a["L"], Hq, Hkv, d, duo.DUO_FP32, a["alpha"], S, W,
+                                       a["scale"], a["out"], a["ws"], a["nb"])
+
+    assert call(q=0) == duo.DUO_ERR_INVALID
+    assert call(alpha=0) == duo.DUO_ERR_INVALID
+    assert call(out=p + 8) == duo.DUO_ERR_INVALID       # 16-byte alignment
+    assert call(ws=p + 16) == duo.DUO_ERR_INVALID       # 256-byte alignment
+    assert call(scale=-1.0) == duo.DUO_ERR_INVALID
+    assert call(L=0) == duo.DUO_ERR_INVALID
+    assert call(nb=n - 1) == duo.DUO_ERR_CAPACITY

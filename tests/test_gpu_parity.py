@@ -483,3 +483,35 @@ def test_decode_group_sizes_and_batches(B, Hq, Hkv, mask, S, W, ctx):
     _, q, k, v, got, got_lse = _fill_and_decode(Hq, Hkv, 128, m, S, W, B, ctx, steps, 110)
     want, want_lse = _decode_oracle(q, k, v, m[0], S, W, ctx, steps)
     assert_close(got, want, torch.bfloat16, got_lse, want_lse, f"decode B{B} G{Hq // Hkv}")
+
+
+# ------------------------------------------------- gated mixed attention
+
+@pytest.mark.parametrize("dtype,B,L,Hq,Hkv,d,S,W", [
+    (torch.float32, 1, 200, 8, 8, 64, 4, 16),        # SIMT pre-fill path
+    (torch.bfloat16, 2, 1500, 8, 2, 128, 16, 64),    # tcgen05 pre-fill path, GQA
+    (torch.bfloat16, 1, 700, 4, 4, 128, 0, 33),      # no sinks, ragged tiles
+])
+def test_gated_attention(dtype, B, L, Hq, Hkv, d, S, W):
+    """alpha * causal + (1 - alpha) * Lambda per KV head against the oracle, gates
+    including the end points 0 and 1."""
+    q, k, v = _seq(B, L, Hq, Hkv, d, dtype, 120)
+    alpha = torch.linspace(0.0, 1.0, Hkv, dtype=torch.float32)
+    got = duo.gated_attention(q, k, v, alpha.to(DEV), S, W)
+    torch.cuda.synchronize()
+    want = oracle.gated(bits(q), bits(k), bits(v), alpha.numpy(), S, W)
+    assert_close(got.float().cpu().numpy(), want, dtype, what=f"gated {dtype} L{L}")
+
+
+def test_gated_attention_llama3_sampled():
+    """Llama-3-8B shape (32 q / 8 kv heads, d 128, S 16, W 512) over an 8K sequence;
+    sampled rows: first and last positions, around S and W, and random rows."""
+    B, L, Hq, Hkv, d, S, W = 1, 8192, 32, 8, 128, 16, 512
+    q, k, v = _seq(B, L, Hq, Hkv, d, torch.bfloat16, 130)
+    alpha = torch.rand(Hkv, generator=torch.Generator().manual_seed(5))
+    got = duo.gated_attention(q, k, v, alpha.to(DEV), S, W).float().cpu().numpy().reshape(-1, d)
+    pos = np.unique(np.concatenate([[0, 1, S - 1, S, S + 1, W - 1, W, W + 1, S + W, L - 1],
+                                    np.random.default_rng(7).integers(0, L, 24)]))
+    rows = (pos[:, None] * Hq + np.arange(Hq)[None, :]).reshape(-1)
+    want = oracle.gated(bits(q), bits(k), bits(v), alpha.numpy(), S, W, rows=rows)
+    assert_close(got[rows], want, torch.bfloat16, what="gated llama3 8K sampled")
