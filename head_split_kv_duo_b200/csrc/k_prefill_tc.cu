@@ -65,8 +65,10 @@ constexpr int kTmS = 0, kTmO = 256, kTmP = 384;
 // barrier indices (8 bytes each).  Double-buffered resources (S, P) have one barrier
 // per buffer, so that no barrier can complete two phases ahead of a thread waiting on
 // it (parity waits).
-constexpr int kBarQ = 0, kBarKFull = 1, kBarKEmpty = 4, kBarVFull = 7, kBarVEmpty = 9, kBarSFull = 11,
-              kBarSFree = 13, kBarPFull = 15, kBarOFull = 17, kBarDrain = 18, kNumBars = 19;
+constexpr int kBarQ = 0, kBarKFull = 1, kBarKEmpty = kBarKFull + kKStages, kBarVFull = kBarKEmpty + kKStages,
+              kBarVEmpty = kBarVFull + kVStages, kBarSFull = kBarVEmpty + kVStages, kBarSFree = kBarSFull + 2,
+              kBarPFull = kBarSFree + 2, kBarOFull = kBarPFull + 2, kBarDrain = kBarOFull + 1, kNumBars = kBarDrain + 1;
+static_assert(kNumBars * 8 <= 256, "barrier area");
 
 struct TileDesc {
   int src;      // 0 retrieval cache, 1 streaming history, 2 chunk input
