@@ -7,8 +7,13 @@ Headline workload (N = 1): decode attention of a Llama-3-8B-shaped GQA layer (32
 1.08 GB of K/V, larger than L2, so no L2 flush is needed): append the new token's
 K/V and run decode attention -- the whole decode path (append/evict, retrieval
 split-KV, streaming sink+ring, merge).  value = algorithmic HBM bytes of the decode
-attention per step / step time (GB/s).  The chunked pre-fill workload (256K prompt
-in 32K chunks, same shape) is timed after it and reported under "prefill".
+attention per step / step time (GB/s), the step timed with no events between its
+launches; each append + attend goes through duo_append_decode (one fused launch at
+batch 1).  roofline.achieved divides the same bytes by the timed region's time per
+decode call; a second pass of the same steps with an event pair around every call
+gives event_bracketed_call_us for reference.  The chunked pre-fill workload (256K
+prompt in 32K chunks, same shape) is timed after it and reported under "prefill",
+and the identification-phase gated forward (32K tokens) under "gated".
 
 --impl reference times the fp64 CPU oracle on the host cores on a bounded sample of
 the same workload (the reference arm).  Under torchrun every rank runs an
@@ -173,7 +178,7 @@ def run_ours(args, rank, world, dist):
     if args.layers:
         nlayers = args.layers
     Hr, Hs = nret, Hkv - nret
-    max_len = ctx + warmup + 2 * steps + 16
+    max_len = ctx + warmup + 3 * steps + 16  # warm-up, timed and event passes, e2e pass
     mask = inputs.retrieval_mask(nlayers, Hkv, nret, seed=1)
     cache = DuoCache(nlayers, Hkv, D, mask, S, W, max_len, batch=B, q_heads=Hq, dtype=torch.bfloat16,
                      retr_fmt=fmt, device=dev)
@@ -188,7 +193,7 @@ def run_ours(args, rank, world, dist):
             del k, v
     torch.cuda.synchronize()
     # per-step inputs: q, k, v of the new token for every layer
-    nstep_in = warmup + steps
+    nstep_in = warmup + 2 * steps
     qs = inputs.randn((nstep_in, nlayers, B, Hq, D), 7, device=dev)
     ks = inputs.randn((nstep_in, nlayers, B, 1, Hkv, D), 8, device=dev)
     vs = inputs.randn((nstep_in, nlayers, B, 1, Hkv, D), 9, device=dev)
@@ -202,11 +207,12 @@ def run_ours(args, rank, world, dist):
     def step(i, ev=None):
         nbytes = 0
         for layer in range(nlayers):
-            cache.append_kv(layer, ks[i, layer], vs[i, layer], stream=stream)
-            n = cache.len(layer)
+            n = cache.len(layer) + 1
             if ev is not None:
                 ev[0].record(stream)
-            cache.decode_attention(layer, qs[i, layer], out=out[layer], lse=lse[layer], stream=stream)
+            # append the step's token and attend: one launch on the bf16 tcgen05 path
+            cache.append_decode(layer, qs[i, layer], ks[i, layer], vs[i, layer], out=out[layer], lse=lse[layer],
+                                stream=stream)
             if ev is not None:
                 ev[1].record(stream)
                 ev[2].append((ev[0], ev[1]))
@@ -220,19 +226,25 @@ def run_ours(args, rank, world, dist):
     torch.cuda.synchronize()
     if dist:
         dist.barrier()
-    kev = [torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True), []]
+    # timed region: the steps alone (no events between launches)
     t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     nbytes = 0
     with ClockSampler(dev.index) as clk:
         torch.cuda.synchronize()
         t0.record(stream)
         for i in range(warmup, warmup + steps):
-            nbytes += step(i, kev)
+            nbytes += step(i)
         t1.record(stream)
         torch.cuda.synchronize()
     if dist:
         dist.barrier()
     ms = t0.elapsed_time(t1)
+    # per-call durations of the decode call for the roofline: the same steps again, with
+    # an event pair around every call (the events add a little time between launches)
+    kev = [torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True), []]
+    for i in range(warmup + steps, warmup + 2 * steps):
+        step(i, kev)
+    torch.cuda.synchronize()
     dec_ms = [a.elapsed_time(b) for a, b in kev[2]]
     assert cache.device_status() == 0, "device status word set"
     ms_max, bytes_sum = ms, nbytes
@@ -247,7 +259,10 @@ def run_ours(args, rank, world, dist):
     us_per_token_layer = ms * 1e3 / (steps * nlayers)
     dec_avg_ms = statistics.mean(dec_ms)
     per_launch_bytes = nbytes / (steps * nlayers)
-    achieved = per_launch_bytes / (dec_avg_ms * 1e-3) / 1e9
+    # the decode call's duration over the timed region: every launch in it belongs to a
+    # decode call (one fused launch at batch 1), so this includes the gaps between them
+    call_ms = ms / (steps * nlayers)
+    achieved = per_launch_bytes / (call_ms * 1e-3) / 1e9
 
     # ---- end-to-end through the public API with host buffers ----
     e2e = None
@@ -269,9 +284,9 @@ def run_ours(args, rank, world, dist):
             dk.copy_(hk[i], non_blocking=True)
             dv.copy_(hv[i], non_blocking=True)
             for layer in range(nlayers):
-                cache.append_kv(layer, dk[layer], dv[layer], stream=stream)
-                eb += nbytes_of(cache.len(layer))
-                cache.decode_attention(layer, dq[layer], out=out[layer], lse=lse[layer], stream=stream)
+                eb += nbytes_of(cache.len(layer) + 1)
+                cache.append_decode(layer, dq[layer], dk[layer], dv[layer], out=out[layer], lse=lse[layer],
+                                    stream=stream)
             hout.copy_(out, non_blocking=True)
         e1.record(stream)
         torch.cuda.synchronize()
@@ -305,9 +320,11 @@ def run_ours(args, rank, world, dist):
                      "peak": hbm_peak, "peak_source": f"{peak_src} hbm_gbs (burst copy)", "unit": "GB/s",
                      "frac": round(achieved / hbm_peak, 4), "frac_of_8tbs_spec": round(achieved / 8000.0, 4),
                      "traffic": recorded_traffic(args.workload),
-                     "algorithmic_bytes_per_launch": int(per_launch_bytes), "avg_launch_us": round(dec_avg_ms * 1e3, 3)},
-        # per layer and step: append + decode (the split merge runs inside the decode kernel)
-        "gpu_launches": steps * nlayers * 2,
+                     "algorithmic_bytes_per_launch": int(per_launch_bytes), "avg_launch_us": round(call_ms * 1e3, 3),
+                     "event_bracketed_call_us": round(dec_avg_ms * 1e3, 3),
+                     "launch": "fused append+decode" if fmt == "same" and B == 1 else "append, then decode"},
+        # per layer and step: one fused append + decode launch (bf16, batch 1), else append then decode
+        "gpu_launches": steps * nlayers * (1 if fmt == "same" and B == 1 else 2),
         "clocks": clk.summary(),
         "e2e": e2e,
         "prefill": prefill,

@@ -102,6 +102,10 @@ struct DecodeParams {
   int n_retr_ctas;
   float scale_log2;   // softmax scale * log2(e)
   HeadMap hm;
+  // fused append: the new token's rows [B][Hkv][d] (nullptr: already in the cache), at
+  // position npos = len - 1; the CTA that reads a row's tile writes it first
+  const char *nk, *nv;
+  int64_t npos;
 };
 
 struct PrefillParams {

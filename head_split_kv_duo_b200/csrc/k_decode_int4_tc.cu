@@ -209,6 +209,10 @@ __global__ void __launch_bounds__(kThreads, 1) decode_int4_kernel(const __grid_c
   const float *qsum_all = reinterpret_cast<const float *>(smem + kSmQsum);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  // A decode launched next on the stream may start its set-up on the SMs this grid
+  // frees; it touches global memory only after its own griddepcontrol.wait, which
+  // returns once this whole grid has completed.
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   const int64_t u0 = cta_begin(a, blockIdx.x), u1 = cta_begin(a, blockIdx.x + 1);
   const int nu = static_cast<int>(u1 - u0);
   const int G = p.G;

@@ -106,6 +106,10 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
   float *red = reinterpret_cast<float *>(smem + kSmRed);  // [4 warps][16]
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  // A decode launched next on the stream may start its set-up on the SMs this grid
+  // frees; it touches global memory only after its own griddepcontrol.wait, which
+  // returns once this whole grid has completed.
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   const int64_t u0 = cta_begin(a, blockIdx.x), u1 = cta_begin(a, blockIdx.x + 1);
   const int nu = static_cast<int>(u1 - u0);
   const int G = p.G;
@@ -129,11 +133,49 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
 
   if (warp == 0) {
     // ================= TMA producer =================
+    // Launched as a programmatic dependent, this grid's set-up overlaps the previous
+    // kernel on the stream; nothing is read from global memory before that kernel has
+    // finished (every other read and every write of this grid follows this warp's loads).
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    if (p.nk) {
+      // Fused append ("Decoding Procedure", step 4): the token at position npos goes to
+      // row npos of every retrieval head and to slot npos < S ? npos : S + npos mod W of
+      // every streaming head.  The only CTA that reads the tile holding that row writes
+      // it here (lanes 0-15 the K row, 16-31 the V row), before its TMA loads the tile.
+      const int64_t slot = p.npos < p.S ? p.npos : p.S + p.npos % p.W;
+      const int first_item = unit_of(a, u0).item, last_item = nu > 0 ? unit_of(a, u1 - 1).item : first_item - 1;
+      const int64_t ur = static_cast<int64_t>(a.n_items_r) * a.units_r;
+      for (int item = first_item; item <= last_item; ++item) {
+        // the unit of this item whose tile holds the new row, if this CTA owns it
+        const bool retr = item < a.n_items_r;
+        const int64_t row = retr ? p.npos : slot;
+        const int64_t u = retr ? static_cast<int64_t>(item) * a.units_r + row / kTile
+                               : ur + static_cast<int64_t>(item - a.n_items_r) * a.units_s + row / kTile;
+        if (u < u0 || u >= u1) continue;
+        int b, g;
+        char *dst;
+        if (retr) {
+          b = item / p.Hr;
+          const int ri = item % p.Hr;
+          g = p.hm.retr_head[ri];
+          dst = const_cast<char *>(lane < 16 ? p.rk : p.rv) + ((static_cast<int64_t>(b) * p.Hr + ri) * p.max_len + row) * kD * 2;
+        } else {
+          const int it2 = item - a.n_items_r;
+          b = it2 / p.Hs;
+          const int si = it2 % p.Hs;
+          g = p.hm.strm_head[si];
+          dst = const_cast<char *>(lane < 16 ? p.sk : p.sv) +
+                ((static_cast<int64_t>(b) * p.Hs + si) * (p.S + p.W) + row) * kD * 2;
+        }
+        const char *src = (lane < 16 ? p.nk : p.nv) + (static_cast<int64_t>(b) * p.Hkv + g) * kD * 2;
+        reinterpret_cast<uint4 *>(dst)[lane & 15] = reinterpret_cast<const uint4 *>(src)[lane & 15];
+      }
+      // the rows are read back through the TMA (async proxy) by lane 0 below
+      asm volatile("fence.proxy.async.global;" ::: "memory");
+      __syncwarp();
+      asm volatile("fence.proxy.async.global;" ::: "memory");
+    }
     if (lane == 0) {
-      // Launched as a programmatic dependent, this grid's set-up overlaps the previous
-      // kernel on the stream; nothing is read from global memory before that kernel has
-      // finished (every other read and every write of this grid follows these loads).
-      asm volatile("griddepcontrol.wait;" ::: "memory");
       UnitIter it(a, u0);
       for (int j = 0; j < nu; ++j, it.next(a)) {
         const int s = j % kStages;

@@ -60,6 +60,8 @@ def lib() -> ctypes.CDLL:
             L.duo_append_kv.argtypes = [vp, i32, vp, vp, i32, vp]
             L.duo_prefill_chunk.restype = i32
             L.duo_prefill_chunk.argtypes = [vp, i32, vp, vp, vp, i32, vp, vp, vp]
+            L.duo_append_decode.restype = i32
+            L.duo_append_decode.argtypes = [vp, i32, vp, vp, vp, vp, vp, vp]
             L.duo_decode_attention.restype = i32
             L.duo_decode_attention.argtypes = [vp, i32, vp, vp, vp, vp]
             L.duo_cache_len.restype = i32
@@ -140,6 +142,10 @@ def duo_prefill_chunk(handle, layer, q, k, v, n, out, lse, stream=None) -> int:
 
 def duo_decode_attention(handle, layer, q, out, lse, stream=None) -> int:
     return lib().duo_decode_attention(handle, layer, _ptr(q), _ptr(out), _ptr(lse), _ptr(stream))
+
+
+def duo_append_decode(handle, layer, q, k, v, out, lse, stream=None) -> int:
+    return lib().duo_append_decode(handle, layer, _ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), _ptr(stream))
 
 
 def duo_cache_len(handle, layer):
@@ -267,6 +273,21 @@ class DuoCache:
             self._want(lse, (self.batch, self.q_heads), "lse", torch.float32)
         self._check(duo_decode_attention(self.handle, layer, q, out, lse, _stream_ptr(stream)),
                     "duo_decode_attention")
+        return out, lse
+
+    def append_decode(self, layer, q, k, v, out=None, lse=None, want_lse=True, stream=None):
+        """duo_append_decode: append one token (k, v [B][1][Hkv][d]) and attend with q."""
+        self._want(q, (self.batch, self.q_heads, self.head_dim), "q")
+        self._want(k, (self.batch, 1, self.kv_heads, self.head_dim), "k")
+        self._want(v, (self.batch, 1, self.kv_heads, self.head_dim), "v")
+        if out is None:
+            out = torch.empty_like(q)
+        if lse is None and want_lse:
+            lse = torch.empty(self.batch, self.q_heads, dtype=torch.float32, device=q.device)
+        self._want(out, q.shape, "out")
+        if lse is not None:
+            self._want(lse, (self.batch, self.q_heads), "lse", torch.float32)
+        self._check(duo_append_decode(self.handle, layer, q, k, v, out, lse, _stream_ptr(stream)), "duo_append_decode")
         return out, lse
 
     def len(self, layer) -> int:

@@ -155,6 +155,19 @@ DUO_API duo_status duo_prefill_chunk(duo_cache *cache, int layer, const void *q,
 DUO_API duo_status duo_decode_attention(duo_cache *cache, int layer, const void *q, void *out, float *lse,
                                 void *cuda_stream);
 
+/*
+ * duo_append_kv of one token followed by duo_decode_attention, as one call: k, v
+ * device [B][1][Hkv][d] (the token at position len), q / out / lse as for
+ * duo_decode_attention ("Decoding Procedure", steps 2-4, in the order of reading R6).
+ * For bf16 caches with head_dim 128 (not INT4) and batch 1 it is one launch: the decode
+ * kernel writes the token's rows into the cache itself, each by the CTA that then reads
+ * the tile holding it; other caches get the two launches (the faster choice measured).  The cache afterwards holds
+ * exactly what duo_append_kv would have written, and len advances by one.
+ * DUO_ERR_CAPACITY if len + 1 > max_len.
+ */
+DUO_API duo_status duo_append_decode(duo_cache *cache, int layer, const void *q, const void *k, const void *v,
+                                     void *out, float *lse, void *cuda_stream);
+
 /* Tokens in a layer's cache (host value, no synchronisation). */
 DUO_API duo_status duo_cache_len(const duo_cache *cache, int layer, int64_t *len);
 

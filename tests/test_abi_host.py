@@ -196,3 +196,18 @@ def test_gated_checks_arguments_before_any_launch():
     assert call(scale=-1.0) == duo.DUO_ERR_INVALID
     assert call(L=0) == duo.DUO_ERR_INVALID
     assert call(nb=n - 1) == duo.DUO_ERR_CAPACITY
+
+
+def test_append_decode_checks_arguments_before_any_launch():
+    st, h, _ = _create(max_len=10)
+    assert st == duo.DUO_OK
+    p = FAKE
+    try:
+        assert duo.duo_append_decode(h, 0, 0, p, p, p, None) == duo.DUO_ERR_INVALID   # no q
+        assert duo.duo_append_decode(h, 0, p, 0, p, p, None) == duo.DUO_ERR_INVALID   # no k
+        assert duo.duo_append_decode(h, 0, p, p, p + 8, p, None) == duo.DUO_ERR_INVALID  # unaligned v
+        assert duo.duo_append_decode(h, 5, p, p, p, p, None) == duo.DUO_ERR_INVALID   # no such layer
+        assert duo.duo_append_decode(h, 0, p, p, p, p, p + 2) == duo.DUO_ERR_INVALID  # unaligned lse
+        assert duo.duo_cache_len(h, 0) == (duo.DUO_OK, 0)
+    finally:
+        duo.duo_cache_destroy(h)

@@ -515,3 +515,48 @@ def test_gated_attention_llama3_sampled():
     rows = (pos[:, None] * Hq + np.arange(Hq)[None, :]).reshape(-1)
     want = oracle.gated(bits(q), bits(k), bits(v), alpha.numpy(), S, W, rows=rows)
     assert_close(got[rows], want, torch.bfloat16, what="gated llama3 8K sampled")
+
+
+# ---------------------------------------------- fused append + decode (one launch)
+
+@pytest.mark.parametrize("Hq,Hkv,mask_row,S,W,B,ctx,dtype,fmt", [
+    (32, 8, [0, 1, 0, 1, 1, 0, 0, 1], 16, 64, 2, 300, torch.bfloat16, "same"),   # tcgen05 path, ring wraps
+    (8, 8, [1, 0, 0, 0, 0, 0, 0, 1], 4, 16, 1, 0, torch.bfloat16, "same"),       # from the first token
+    (32, 32, [1] * 8 + [0] * 24, 16, 512, 1, 2000, torch.bfloat16, "same"),       # MHA
+    (8, 8, [1, 0, 1, 0, 0, 0, 0, 1], 4, 16, 1, 50, torch.float32, "same"),       # CUDA-core path (two launches)
+    (32, 8, [0, 1, 1, 0, 0, 1, 0, 1], 16, 64, 1, 400, torch.bfloat16, "int4"),   # INT4 path (two launches)
+])
+def test_append_decode_equals_append_then_decode(Hq, Hkv, mask_row, S, W, B, ctx, dtype, fmt):
+    """duo_append_decode leaves exactly the cache duo_append_kv writes and returns exactly
+    what duo_decode_attention returns, step after step across ring wrap-around."""
+    d = 128 if dtype == torch.bfloat16 else 64
+    steps = 70
+    T = ctx + steps
+    mask = torch.tensor([mask_row], dtype=torch.uint8)
+    q = inputs.randn((B, steps, Hq, d), 140, dtype, DEV)
+    k = inputs.randn((B, T, Hkv, d), 141, dtype, DEV)
+    v = inputs.randn((B, T, Hkv, d), 142, dtype, DEV)
+    c1 = DuoCache(1, Hkv, d, mask, S, W, T, batch=B, q_heads=Hq, dtype=dtype, retr_fmt=fmt)
+    c2 = DuoCache(1, Hkv, d, mask, S, W, T, batch=B, q_heads=Hq, dtype=dtype, retr_fmt=fmt)
+    if ctx > 0:
+        for c in (c1, c2):
+            c.append_kv(0, k[:, :ctx].contiguous(), v[:, :ctx].contiguous())
+    for t in range(steps):
+        kt, vt = k[:, ctx + t:ctx + t + 1].contiguous(), v[:, ctx + t:ctx + t + 1].contiguous()
+        c1.append_kv(0, kt, vt)
+        o1, l1 = c1.decode_attention(0, q[:, t].contiguous())
+        o2, l2 = c2.append_decode(0, q[:, t].contiguous(), kt, vt)
+        assert torch.equal(o1, o2) and torch.equal(l1, l2), f"step {t}"
+    torch.cuda.synchronize()
+    assert c1.len(0) == c2.len(0) == T and c1.device_status() == 0 and c2.device_status() == 0
+    regions = [duo.DUO_REGION_RETR_K, duo.DUO_REGION_RETR_V, duo.DUO_REGION_STRM_K, duo.DUO_REGION_STRM_V]
+    if fmt == "int4":
+        regions += [duo.DUO_REGION_RETR_KSZ, duo.DUO_REGION_RETR_VSZ]
+    for r in regions:
+        a, _ = c1.region(0, r)
+        b, _ = c2.region(0, r)
+        assert torch.equal(a, b), f"region {r}"
+    # and the last step matches the oracle
+    want, want_lse = _decode_oracle(q[:, steps - 1:], k, v, mask[0], S, W, T - 1, 1)
+    if fmt == "same":
+        assert_close(o2.float().cpu().numpy()[:, None], want, dtype, l2.cpu().numpy()[:, None], want_lse, "append_decode")
