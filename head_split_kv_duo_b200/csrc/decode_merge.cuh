@@ -117,4 +117,85 @@ __device__ __forceinline__ void merge_partials(const float *part, int nseg, int 
   asm volatile("bar.sync %0, 128;" ::"r"(bar_id) : "memory");  // cmb is reused by the caller
 }
 
+// merge_partials for rows already copied into (writable) shared memory: the per-head
+// maxima are found first and each row's m is replaced by its weight exp2(m - max), so
+// the weighted sums that follow are independent (no rescaling chain).
+__device__ __forceinline__ void merge_partials_smem(float *rows, int nseg, int G, int b, int h0, int Hq, char *out,
+                                                    float *lse, float *cmb, int t, int bar_id) {
+  constexpr int kD = 128;
+  if (t < G) {
+    float M0 = -INFINITY, M1 = -INFINITY;
+    int s = 0;
+    for (; s + 1 < nseg; s += 2) {
+      M0 = fmaxf(M0, rows[(s * G + t) * kPartRow + kD]);
+      M1 = fmaxf(M1, rows[((s + 1) * G + t) * kPartRow + kD]);
+    }
+    if (s < nseg) M0 = fmaxf(M0, rows[(s * G + t) * kPartRow + kD]);
+    cmb[t] = fmaxf(M0, M1);
+  }
+  asm volatile("bar.sync %0, 128;" ::"r"(bar_id) : "memory");
+  for (int i = t; i < nseg * G; i += 128) {
+    float *r = rows + i * kPartRow;
+    r[kD] = (r[kD] == -INFINITY) ? 0.f : ex2(r[kD] - cmb[i % G]);
+  }
+  asm volatile("bar.sync %0, 128;" ::"r"(bar_id) : "memory");
+  const int cols = G * (kD / 4);
+  const int nsl = cols >= 128 ? 1 : 128 / cols;
+  float *lanes = cmb + 16;  // [128][5] per segment lane: den, acc
+  for (int c0 = 0; c0 < cols; c0 += 128) {
+    const int col = cols >= 128 ? c0 + t : t % cols;
+    const int sl = cols >= 128 ? 0 : t / cols;
+    const bool active = col < cols && sl < nsl;
+    const int q = col >> 5, c4 = col & 31;
+    float den = 0.f;
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (active) {
+#pragma unroll 4
+      for (int sg = sl; sg < nseg; sg += nsl) {
+        const float *r = rows + (sg * G + q) * kPartRow;
+        const float w = r[kD];
+        const float4 v = reinterpret_cast<const float4 *>(r)[c4];
+        den = fmaf(w, r[kD + 1], den);
+        acc.x = fmaf(w, v.x, acc.x);
+        acc.y = fmaf(w, v.y, acc.y);
+        acc.z = fmaf(w, v.z, acc.z);
+        acc.w = fmaf(w, v.w, acc.w);
+      }
+    }
+    if (nsl > 1) {
+      if (active) {
+        float *e = lanes + t * 5;
+        e[0] = den;
+        e[1] = acc.x;
+        e[2] = acc.y;
+        e[3] = acc.z;
+        e[4] = acc.w;
+      }
+      asm volatile("bar.sync %0, 128;" ::"r"(bar_id) : "memory");
+      if (active && sl == 0) {
+        for (int k = 1; k < nsl; ++k) {
+          const float *e = lanes + (t + k * cols) * 5;
+          den += e[0];
+          acc.x += e[1];
+          acc.y += e[2];
+          acc.z += e[3];
+          acc.w += e[4];
+        }
+      }
+    }
+    if (active && sl == 0) {
+      const float inv = 1.f / den;
+      const __nv_bfloat162 lo = __floats2bfloat162_rn(acc.x * inv, acc.y * inv);
+      const __nv_bfloat162 hi = __floats2bfloat162_rn(acc.z * inv, acc.w * inv);
+      uint2 pk;
+      pk.x = *reinterpret_cast<const uint32_t *>(&lo);
+      pk.y = *reinterpret_cast<const uint32_t *>(&hi);
+      const int h = h0 + q;
+      *reinterpret_cast<uint2 *>(out + ((static_cast<int64_t>(b) * Hq + h) * kD + 4 * c4) * 2) = pk;
+      if (c4 == 0 && lse) lse[b * Hq + h] = (cmb[q] + lg2(den)) * kLn2;
+    }
+  }
+  asm volatile("bar.sync %0, 128;" ::"r"(bar_id) : "memory");  // cmb is reused by the caller
+}
+
 }  // namespace duo

@@ -163,4 +163,11 @@ __device__ __forceinline__ void bulk_g2s(uint32_t dst, const void *src, uint32_t
       : "memory");
 }
 
+// Prefetch into L2 (untiled bulk form); addr 16-byte aligned, bytes a positive multiple
+// of 16.  A hint only: L2 is the point of coherence for device memory, so a line brought
+// in early is still updated by any later write before a load reads it.
+__device__ __forceinline__ void prefetch_l2(const void *addr, uint32_t bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(addr), "r"(bytes) : "memory");
+}
+
 }  // namespace duo

@@ -740,7 +740,10 @@ cudaError_t launch_decode_int4_tc(const DecodeParams &p, int num_sms, bool overl
   a.p = p;
   a.units_r = static_cast<int>((p.len + kTile - 1) / kTile);
   const int64_t slots = static_cast<int64_t>(p.S) + p.W;
-  const int64_t used = p.len < slots ? p.len : slots;  // streaming slots that can hold a token
+  // highest ring slot in use + 1: position p >= S sits in slot S + p mod W, so before the
+  // ring wraps (len <= W) the slots reach S + len - 1, beyond len itself
+  const int64_t reach = static_cast<int64_t>(p.S) + p.len;
+  const int64_t used = reach < slots ? reach : slots;
   a.units_s = static_cast<int>((used + kTile - 1) / kTile);
   a.n_items_r = p.B * p.Hr;
   a.ur = static_cast<int64_t>(a.n_items_r) * a.units_r;

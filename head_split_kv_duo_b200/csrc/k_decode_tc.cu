@@ -26,11 +26,14 @@ namespace duo {
 
 namespace {
 
-constexpr int kThreads = 192;  // warp 0 TMA, warp 1 MMA + TMEM, warps 2-5 softmax
+constexpr int kThreads = 224;  // warp 0 TMA, warp 1 MMA + TMEM, warps 2-5 softmax, warp 6 append
 constexpr int kTile = 128;
 constexpr int kD = 128;
 constexpr int kN = 16;         // padded query heads per item
 constexpr int kStages = 3;
+// Tiles of its range a CTA asks L2 to fetch before the previous grid on the stream has
+// finished: that grid's tail (its last CTAs and their merges) leaves HBM mostly idle.
+constexpr int kPrefetch = 4;
 // Each contraction (over d for S^T, over tokens for O^T) is split into kAcc partial
 // accumulators in separate TMEM columns, so the tensor core runs kAcc independent
 // chains of 8 / kAcc MMAs instead of one chain of 8; the softmax warps add them up.
@@ -47,7 +50,7 @@ constexpr int kSmemAlloc = kSmMisc + 64 + 1024;
 // Double-buffered resources (S, P, O) each have one barrier per buffer, so that no
 // barrier can complete two phases ahead of the thread waiting on it (parity waits).
 constexpr int kBarFull = 0, kBarEmpty = 3, kBarSFull = 6, kBarSFree = 8, kBarPFull = 10, kBarOFull = 12,
-              kBarDrain = 14, kNumBars = 15;
+              kBarDrain = 14, kBarAppend = 15, kBarMerge = 16, kNumBars = 17;
 
 struct TcDecodeArgs {
   DecodeParams p;
@@ -133,54 +136,53 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
 
   if (warp == 0) {
     // ================= TMA producer =================
-    // Launched as a programmatic dependent, this grid's set-up overlaps the previous
-    // kernel on the stream; nothing is read from global memory before that kernel has
-    // finished (every other read and every write of this grid follows this warp's loads).
-    asm volatile("griddepcontrol.wait;" ::: "memory");
-    if (p.nk) {
-      // Fused append ("Decoding Procedure", step 4): the token at position npos goes to
-      // row npos of every retrieval head and to slot npos < S ? npos : S + npos mod W of
-      // every streaming head.  The only CTA that reads the tile holding that row writes
-      // it here (lanes 0-15 the K row, 16-31 the V row), before its TMA loads the tile.
-      const int64_t slot = p.npos < p.S ? p.npos : p.S + p.npos % p.W;
-      const int first_item = unit_of(a, u0).item, last_item = nu > 0 ? unit_of(a, u1 - 1).item : first_item - 1;
-      const int64_t ur = static_cast<int64_t>(a.n_items_r) * a.units_r;
-      for (int item = first_item; item <= last_item; ++item) {
-        // the unit of this item whose tile holds the new row, if this CTA owns it
-        const bool retr = item < a.n_items_r;
-        const int64_t row = retr ? p.npos : slot;
-        const int64_t u = retr ? static_cast<int64_t>(item) * a.units_r + row / kTile
-                               : ur + static_cast<int64_t>(item - a.n_items_r) * a.units_s + row / kTile;
-        if (u < u0 || u >= u1) continue;
-        int b, g;
-        char *dst;
-        if (retr) {
-          b = item / p.Hr;
-          const int ri = item % p.Hr;
-          g = p.hm.retr_head[ri];
-          dst = const_cast<char *>(lane < 16 ? p.rk : p.rv) + ((static_cast<int64_t>(b) * p.Hr + ri) * p.max_len + row) * kD * 2;
-        } else {
-          const int it2 = item - a.n_items_r;
-          b = it2 / p.Hs;
-          const int si = it2 % p.Hs;
-          g = p.hm.strm_head[si];
-          dst = const_cast<char *>(lane < 16 ? p.sk : p.sv) +
-                ((static_cast<int64_t>(b) * p.Hs + si) * (p.S + p.W) + row) * kD * 2;
+    if (lane == 0) {
+      for (const CUtensorMap *m : {&a.tm_q, &a.tm_kr, &a.tm_vr, &a.tm_ks, &a.tm_vs})
+        asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(m)) : "memory");
+      {  // L2 prefetch of the first tiles; no data is consumed before the wait below
+        UnitIter it(a, u0);
+        for (int j = 0; j < nu && j < kPrefetch; ++j, it.next(a)) {
+          const Unit un = it.un;
+          const int64_t y = static_cast<int64_t>(un.tile) * kTile;
+          const char *kb, *vb;
+          int64_t rows, base;
+          if (un.retr) {
+            base = (static_cast<int64_t>(un.item) * p.max_len + y) * kD * 2;  // item = b * Hr + retrieval index
+            rows = p.max_len - y;
+            kb = p.rk;
+            vb = p.rv;
+          } else {
+            base = (static_cast<int64_t>(un.item - a.n_items_r) * (p.S + p.W) + y) * kD * 2;
+            rows = p.S + p.W - y;
+            kb = p.sk;
+            vb = p.sv;
+          }
+          const uint32_t bytes = static_cast<uint32_t>((rows < kTile ? rows : kTile) * kD * 2);
+          prefetch_l2(kb + base, bytes);
+          prefetch_l2(vb + base, bytes);
         }
-        const char *src = (lane < 16 ? p.nk : p.nv) + (static_cast<int64_t>(b) * p.Hkv + g) * kD * 2;
-        reinterpret_cast<uint4 *>(dst)[lane & 15] = reinterpret_cast<const uint4 *>(src)[lane & 15];
       }
-      // the rows are read back through the TMA (async proxy) by lane 0 below
-      asm volatile("fence.proxy.async.global;" ::: "memory");
-      __syncwarp();
-      asm volatile("fence.proxy.async.global;" ::: "memory");
+      // Launched as a programmatic dependent, this grid's set-up overlaps the previous
+      // kernel on the stream; nothing is read from global memory before that kernel has
+      // finished (every other read and every write of this grid follows this wait or the
+      // append warp's).
+      asm volatile("griddepcontrol.wait;" ::: "memory");
     }
     if (lane == 0) {
+      // the tile of each item that holds the appended row: its TMA load waits for the
+      // append warp (retrieval: row npos; streaming: the row's slot)
+      const int64_t tile_r = p.npos / kTile, tile_s = (p.npos < p.S ? p.npos : p.S + p.npos % p.W) / kTile;
+      bool appended = p.nk == nullptr;
       UnitIter it(a, u0);
       for (int j = 0; j < nu; ++j, it.next(a)) {
         const int s = j % kStages;
         if (j >= kStages && !tc::wait_bar(bar(kBarEmpty + s), ((j / kStages) - 1) & 1, p.status, abort_flag)) break;
         const Unit un = it.un;
+        if (!appended && un.tile == (un.retr ? tile_r : tile_s)) {
+          if (!tc::wait_bar(bar(kBarAppend), 0, p.status, abort_flag)) break;
+          asm volatile("fence.proxy.async.global;" ::: "memory");
+          appended = true;
+        }
         const uint32_t dst = sbase + s * kStage;
         const uint32_t fb = bar(kBarFull + s);
         mbar_expect_tx(fb, 65536 + 4096);
@@ -263,6 +265,48 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
       tc::commit(bar(kBarDrain));
       mbar_wait(bar(kBarDrain), 0, p.status);
     }
+  } else if (warp == 6) {
+    // ================= append =================
+    if (p.nk) {
+      // Fused append ("Decoding Procedure", step 4): the token at position npos goes to
+      // row npos of every retrieval head and to slot npos < S ? npos : S + npos mod W of
+      // every streaming head.  The only CTA that reads the tile holding that row writes
+      // it (lanes 0-15 the K row, 16-31 the V row); the producer loads that tile only
+      // after this warp's barrier, so its other loads are not held up by these writes.
+      asm volatile("griddepcontrol.wait;" ::: "memory");
+      const int64_t slot = p.npos < p.S ? p.npos : p.S + p.npos % p.W;
+      const int first_item = unit_of(a, u0).item, last_item = nu > 0 ? unit_of(a, u1 - 1).item : first_item - 1;
+      const int64_t ur = static_cast<int64_t>(a.n_items_r) * a.units_r;
+      for (int item = first_item; item <= last_item; ++item) {
+        // the unit of this item whose tile holds the new row, if this CTA owns it
+        const bool retr = item < a.n_items_r;
+        const int64_t row = retr ? p.npos : slot;
+        const int64_t u = retr ? static_cast<int64_t>(item) * a.units_r + row / kTile
+                               : ur + static_cast<int64_t>(item - a.n_items_r) * a.units_s + row / kTile;
+        if (u < u0 || u >= u1) continue;
+        int b, g;
+        char *dst;
+        if (retr) {
+          b = item / p.Hr;
+          const int ri = item % p.Hr;
+          g = p.hm.retr_head[ri];
+          dst = const_cast<char *>(lane < 16 ? p.rk : p.rv) + ((static_cast<int64_t>(b) * p.Hr + ri) * p.max_len + row) * kD * 2;
+        } else {
+          const int it2 = item - a.n_items_r;
+          b = it2 / p.Hs;
+          const int si = it2 % p.Hs;
+          g = p.hm.strm_head[si];
+          dst = const_cast<char *>(lane < 16 ? p.sk : p.sv) +
+                ((static_cast<int64_t>(b) * p.Hs + si) * (p.S + p.W) + row) * kD * 2;
+        }
+        const char *src = (lane < 16 ? p.nk : p.nv) + (static_cast<int64_t>(b) * p.Hkv + g) * kD * 2;
+        reinterpret_cast<uint4 *>(dst)[lane & 15] = reinterpret_cast<const uint4 *>(src)[lane & 15];
+      }
+      // the rows are read back through the TMA (async proxy)
+      asm volatile("fence.proxy.async.global;" ::: "memory");
+      __syncwarp();
+    }
+    if (lane == 0) mbar_arrive(bar(kBarAppend));
   } else {
     // ================= softmax warpgroup =================
     // Thread t owns token t of each S^T tile and dimension t of each O^T tile.  The
@@ -284,8 +328,10 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
     bool ok = true;
     int cur_item = -1;
 
-    // Writes this CTA's result for `item` (partial or final) and merges when last.
-    auto flush = [&](int item) {
+    // Writes this CTA's result for `item` (partial or final) and merges when last.  At
+    // the CTA's final flush the stage buffers are idle: the merge then brings the item's
+    // partial rows in with one bulk copy instead of a chain of round trips to L2.
+    auto flush = [&](int item, bool final_flush) {
 #pragma unroll
       for (int q = 0; q < NQ; ++q) {
         const float v = warp_sum(l[q]);
@@ -346,7 +392,18 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
       tc::named_sync(1, 128);
       if (!*last_flag) return;
       __threadfence();
-      merge_partials(part, nseg, G, b, h0, p.Hq, p.out, p.lse, red + 4 * kN, t, 1);
+      const uint32_t bytes = static_cast<uint32_t>(nseg) * G * kRow * 4;
+      if (final_flush && bytes <= kStages * kStage) {
+        if (t == 0) {
+          asm volatile("fence.proxy.async.global;" ::: "memory");  // the rows are read by the async proxy
+          mbar_expect_tx(bar(kBarMerge), bytes);
+          bulk_g2s(sbase, part, bytes, bar(kBarMerge));
+        }
+        if (ok) ok = tc::wait_bar(bar(kBarMerge), 0, p.status, abort_flag);
+        merge_partials_smem(reinterpret_cast<float *>(smem), nseg, G, b, h0, p.Hq, p.out, p.lse, red + 4 * kN, t, 1);
+      } else {
+        merge_partials(part, nseg, G, b, h0, p.Hq, p.out, p.lse, red + 4 * kN, t, 1);
+      }
       if (t == 0) p.counters[pitem] = 0u;  // ready for the next call
     };
 
@@ -391,7 +448,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
       if (un.item != cur_item) {
         if (cur_item >= 0) {
           if (pending) fold(j - 1, one);
-          flush(cur_item);
+          flush(cur_item, false);
         }
 #pragma unroll
         for (int q = 0; q < NQ; ++q) {
@@ -460,7 +517,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
     }
     if (nu > 0) {
       if (pending) fold(nu - 1, one);
-      flush(cur_item);
+      flush(cur_item, true);
     }
   }
 
@@ -504,7 +561,10 @@ cudaError_t launch_decode_tc(const DecodeParams &p, int num_sms, bool overlap_pr
   a.p = p;
   a.units_r = static_cast<int>((p.len + kTile - 1) / kTile);
   const int64_t slots = static_cast<int64_t>(p.S) + p.W;
-  const int64_t used = p.len < slots ? p.len : slots;  // streaming slots that can hold a token
+  // highest ring slot in use + 1: position p >= S sits in slot S + p mod W, so before the
+  // ring wraps (len <= W) the slots reach S + len - 1, beyond len itself
+  const int64_t reach = static_cast<int64_t>(p.S) + p.len;
+  const int64_t used = reach < slots ? reach : slots;
   a.units_s = static_cast<int>((used + kTile - 1) / kTile);
   a.n_items_r = p.B * p.Hr;
   a.total_units = static_cast<int64_t>(a.n_items_r) * a.units_r + static_cast<int64_t>(p.B) * p.Hs * a.units_s;

@@ -205,9 +205,13 @@ def test_llama3_gqa_decode(B, ctx):
     assert_close(got, want, torch.bfloat16, got_lse, want_lse, f"llama3 B{B} ctx{ctx}")
 
 
-@pytest.mark.parametrize("ctx", [1, 2, 15, 16, 17, 527, 528, 529, 1000])
+@pytest.mark.parametrize("ctx", [1, 2, 15, 16, 17, 113, 120, 128, 250, 256, 400, 500, 512, 513, 527, 528, 529,
+                                 1000])
 def test_decode_short_contexts_and_boundaries(ctx):
-    """len around S and S + W; the first query sees only itself."""
+    """len around S and S + W; the first query sees only itself.  Before the ring wraps
+    (S < len <= W) position p sits in slot S + p, so the newest tokens lie in slots past
+    len: lengths whose last slots cross into a further 128-slot tile (113..128, 250,
+    256, 400, 500, 512) catch a kernel that scans only the first len slots."""
     mask = torch.tensor([[1, 0]], dtype=torch.uint8)
     _, q, k, v, got, got_lse = _fill_and_decode(4, 2, 128, mask, 16, 512, 2, ctx - 1, 1, 30)
     want, want_lse = _decode_oracle(q, k, v, mask[0], 16, 512, ctx - 1, 1)
@@ -386,6 +390,8 @@ def _int4_decode_check(Hq, Hkv, mask_row, S, W, B, ctx, steps, seed, plant=False
     (64, 4, [1, 0, 1, 1], 16, 512, 1, 5000),               # group 16
     (32, 4, [0, 1, 1, 0], 0, 100, 3, 1000),                # group 8, no sinks
     (32, 8, [0, 1, 0, 1, 1, 0, 0, 1], 16, 512, 1, 1 << 18),  # Llama-3 shape, 256K
+    (32, 8, [0, 1, 0, 1, 1, 0, 0, 1], 16, 512, 1, 250),      # ring slots past len (tile 2)
+    (32, 8, [1, 0, 1, 0, 1, 0, 1, 0], 16, 512, 2, 118),      # ring slots past len (tile 1)
 ])
 def test_int4_tc_decode_shapes(Hq, Hkv, mask_row, S, W, B, ctx):
     _int4_decode_check(Hq, Hkv, mask_row, S, W, B, ctx, 2, 90)
