@@ -307,6 +307,14 @@ def run_ours(args, rank, world, dist):
         gated = run_gated(args, dev, tc_peak, tc_sust, peak_src)
 
     kv_gb = nlayers * nbytes_of(ctx) / 1e9
+    # per layer and step: one fused append + decode launch (bf16, batch 1), else the append
+    # then the decode; an INT4 layer decodes its bf16 streaming heads and its INT4
+    # retrieval heads in two launches
+    if fmt == "same":
+        launches_per_layer, launch_desc = (1, "fused append+decode") if B == 1 else (2, "append, then decode")
+    else:
+        launches_per_layer = 3 if Hkv > nret else 2
+        launch_desc = "append, bf16 streaming-head decode, INT4 retrieval-head decode"
     res = {
         "metric": METRIC, "value": round(value, 1), "unit": "GB/s", "n_gpus": world, "steps": steps,
         "warmup": warmup, "ms_per_step": round(ms_max / steps, 4), "higher_is_better": True, "scaling": "weak",
@@ -322,9 +330,8 @@ def run_ours(args, rank, world, dist):
                      "traffic": recorded_traffic(args.workload),
                      "algorithmic_bytes_per_launch": int(per_launch_bytes), "avg_launch_us": round(call_ms * 1e3, 3),
                      "event_bracketed_call_us": round(dec_avg_ms * 1e3, 3),
-                     "launch": "fused append+decode" if fmt == "same" and B == 1 else "append, then decode"},
-        # per layer and step: one fused append + decode launch (bf16, batch 1), else append then decode
-        "gpu_launches": steps * nlayers * (1 if fmt == "same" and B == 1 else 2),
+                     "launch": launch_desc},
+        "gpu_launches": steps * nlayers * launches_per_layer,
         "clocks": clk.summary(),
         "e2e": e2e,
         "prefill": prefill,

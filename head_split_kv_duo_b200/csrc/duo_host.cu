@@ -397,7 +397,18 @@ DecodeParams decode_params(const duo_cache *c, const Layer &ly, const void *q, v
 cudaError_t launch_decode_any(const duo_cache *c, const DecodeParams &p, cudaStream_t st) {
   const bool int4 = c->fmt == DUO_KV_INT4_G128;
   // the tcgen05 decodes overlap their start-up with the previous kernel on the stream
-  if (int4 && decode_int4_tc_supported(p, c->dtype)) return launch_decode_int4_tc(p, c->num_sms, true, st);
+  if (int4 && decode_int4_tc_supported(p, c->dtype)) {
+    // the bf16 streaming heads on the bf16 kernel (a few tiles), then the INT4 retrieval
+    // heads; the two write disjoint heads, partial rows and tickets
+    // (decode_int4_tc_supported implies decode_tc_supported for that view)
+    if (p.Hs > 0) {
+      DecodeParams ps = p;
+      ps.Hr = 0;
+      const cudaError_t e = launch_decode_tc(ps, c->num_sms, true, st);
+      if (e != cudaSuccess) return e;
+    }
+    return launch_decode_int4_tc(p, c->num_sms, true, st);
+  }
   if (decode_tc_supported(p, c->dtype, int4)) return launch_decode_tc(p, c->num_sms, true, st);
   return launch_decode(p, c->dtype, int4, st);
 }

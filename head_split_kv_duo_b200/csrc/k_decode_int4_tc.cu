@@ -1,44 +1,40 @@
-// k_decode_int4_tc.cu -- single-token decode attention when the retrieval heads keep
-// K and V as 4-bit codes ("Combination with Quantization", Figure 12: DuoAttention
-// with a 4-bit KV cache), on the tcgen05 tensor cores.  bf16 queries, head_dim 128,
-// up to 16 query heads per KV head; the streaming heads stay bf16.
+// k_decode_int4_tc.cu -- single-token decode attention over the retrieval heads when
+// they keep K and V as 4-bit codes ("Combination with Quantization", Figure 12:
+// DuoAttention with a 4-bit KV cache), on the tcgen05 integer tensor cores.  bf16
+// queries, head_dim 128, up to 16 query heads per KV head.  The streaming heads (bf16)
+// of such a layer run on the bf16 decode kernel.
 //
 // Operation ("Decoding Procedure", steps 2, 3 and 5) as in k_decode_tc.cu.  A stored
-// element is c s + z (code c in 0..15, per-token fp16 scale s and zero z).  K codes
-// become c' = c + 128, exact in bf16 (bit pattern 0x4300 | c); V codes c" = c + 1024,
-// exact in fp16 (0x6400 | c).  For token t
-//   q . k_t       = s_t (q . c'_t) + (z_t - 128 s_t) sum(q)
-//   sum_t p_t v_t = sum_t (p_t s_t) c"_t + sum_t (p_t z_t - 1024 (p_t s_t))
-// so both contractions run on the tensor cores (Q . K' in bf16, V" . P' in fp16), and
-// the scale and zero enter as a row scale of S^T and one scalar correction per query
-// head of O.  The correction uses the fp16-rounded p_t s_t that the MMA consumes, so
-// the offset cancels exactly; fp16 keeps that product to 11 bits.  INT4 items keep the
-// running max exact (p <= 1), so p_t s_t <= s_t stays in fp16 range.
+// element is c s + z (code c in 0..15, per-token fp16 scale s and zero z).  A token's
+// 64 code bytes are read by the tensor core as they are stored: byte j is
+// U_j = c_{2j} + 16 c_{2j+1} (kind::i8, unsigned); the only conversion is the low
+// nibble L_j = c_{2j}, one AND per four bytes.  Then
+//   sum_d q_d c_d = sum_j (q_{2j+1} / 16) U_j + (q_{2j} - q_{2j+1} / 16) L_j
+// so S^T = [U | L] . Qx^T over K = 128 bytes, with Qx the two coefficient rows above,
+// and for the output (dimension pair j of one query head)
+//   sum_t p'_t L_tj = O_{2j},  sum_t p'_t U_tj = O_{2j} + 16 O_{2j+1}
+// so O^T = [U_V | L_V]^T . P'^T (M = 128: 64 byte rows, 64 low-nibble rows).  The fp32
+// operands Qx and P' = p s_v enter as signed 8-bit limbs with a scale: Qx per query
+// head as three limbs (21 bits below the row's largest coefficient), P' per tile as two
+// (15 bits below the tile's largest s_v, which bounds p s_v since INT4 items keep the
+// running max exact, p <= 1).  The int32 accumulators are exact; the limbs are split
+// and recombined in fp32 by exact magic-number adds (no conversion instructions).  Per token the scale and zero then give
+//   q . k_t = s_t (q . c_t) + z_t sum(q),   sum_t p_t v_t = sum_t p'_t c_t + sum_t p_t z_t.
 //
-// One 32-bit word of codes holds elements e0..e7 (e0 in the low nibble); the pair
-// ((w >> 4i) & 0x000F000F) | 0x43004300 (or 0x64006400) is (c'_i, c'_{4+i}).  An
-// expanded row is thus
-// stored in the order perm(x) = (x & ~7) | ((x & 7) >> 1) | ((x & 1) << 2): position x
-// holds element perm(x).  K rows and the queries are both expanded in that order, which
-// leaves q . k unchanged; V rows too, so lane x of O^T holds output element perm(x).
+// Roles of a CTA (one per SM, 320 threads):
+//   warp 0     TMA producer: per 128-token tile the K and V code rows (64 B each,
+//              64-byte swizzle) and their scale/zero rows, at an item's first tile the
+//              group's bf16 queries; a ring of kStages stages.
+//   warp 1     MMA issuer and TMEM owner (4 MMAs for S^T and 4 for O^T per tile; the
+//              K low nibbles are read from tensor memory).
+//   warps 2-5  softmax: thread t owns token t of S^T and row t of O^T.
+//   warps 6-9  prep: a thread writes the low nibbles of token t's K row into TMEM lane
+//              t and those of its V row beside the V codes, and the token's {s_k, z_k,
+//              s_v, z_v}; warp 6 also turns an item's queries into limbs.
 //
-// Roles of a CTA (one per SM, 448 threads):
-//   warp 0     TMA producer.  INT4 tile: the codes of 128 K rows and 128 V rows (64 B
-//              each, 64-byte swizzle), their scale/zero rows (2 x 512 B) and, at the
-//              first tile of an item, the group's queries.  bf16 (streaming) tile: four
-//              pieces of 32 K and V rows (128-byte swizzle).  Raw ring of kRaw stages.
-//   warp 1     MMA issuer and TMEM owner.  S^T = K'_tile . Qpad^T with K' read from
-//              tensor memory; O^T = V'^T . P'^T with V' from shared memory.
-//   warps 2-5  softmax: thread t owns token t of S^T and position t of O^T.
-//   warps 6-13 expansion: a thread expands one half (64 elements) of token t's K row into
-//              TMEM lane t and of its V row into the swizzled V tile; warps 6-9 also
-//              stage the scale and zero, warp 12 the queries.  Expanded ring of kCvt
-//              stages.
-//
-// Work balance: every (batch, KV head) is an item of 128-token tiles; the tiles of all
-// items are laid end to end (retrieval first) and cut into one range per CTA, an INT4
-// tile counting 1 and a bf16 tile kWs (about 4x the bytes).  Split partials are merged
-// by the last CTA of each item, as in the bf16 kernel.
+// Work balance: every (batch, retrieval head) is an item of 128-token tiles; the tiles
+// of all items are laid end to end and cut into one equal range per CTA.  Split partials
+// are merged by the last CTA of each item, as in the bf16 kernel.
 #include "decode_merge.cuh"
 #include "tcgen05.cuh"
 
@@ -46,157 +42,172 @@ namespace duo {
 
 namespace {
 
-constexpr int kThreads = 448;
+constexpr int kThreads = 320;
 constexpr int kTile = 128;
 constexpr int kD = 128;
-constexpr int kN = 16;  // padded query heads per item
-constexpr int kAcc = 4;  // independent accumulator chains per contraction (as in the bf16 kernel)
-constexpr int kRaw = 4;  // raw stages
-constexpr int kCvt = 3;  // expanded stages
-constexpr int kWs = 4;   // cost of a bf16 tile in INT4 tiles
-
-// raw stage: INT4 tile -- K codes [128][64 B], V codes, K scale/zero [128][4 B], V
-// scale/zero, queries [16][128] bf16 (2 atoms); bf16 piece -- K rows 32 x 256 B as two
-// 64-column halves [32][128 B] at 0 / 4096, V halves at 8192 / 12288, queries as above
-constexpr int kRawKc = 0, kRawVc = 8192, kRawKsz = 16384, kRawVsz = 16896, kRawQ = 17408, kRawStage = 21504;
-// expanded stage: V" [128][128] fp16 (bf16 for streaming tiles; 2 atoms of 16 KiB),
-// per-token {s_k, z_k - 128 s_k, s_v, z_v}
-constexpr int kCvtV = 0, kCvtMisc = 32768, kCvtStage = 32768 + 2048;
-constexpr int kSmRaw = 0;
-constexpr int kSmCvt = kSmRaw + kRaw * kRawStage;
-constexpr int kSmQ = kSmCvt + kCvt * kCvtStage;  // 2 x expanded queries [16][128] bf16 (one per item parity)
-constexpr int kSmP = kSmQ + 2 * 4096;         // 2 x P'^T [16][128] bf16
-constexpr int kSmQsum = kSmP + 8192;          // [2][16] fp32 sums of the queries
-constexpr int kSmRed = kSmQsum + 128;         // [4][16] l sums, [4][16] correction sums, [128][6] merge
+constexpr int kStages = 6;
+constexpr int kPrefetch = 4;  // tiles asked of L2 before the previous grid has finished
+// stage: K and V codes [128][64 B] (64-byte swizzle, as the TMA writes them), the V low
+// nibbles in the same layout, the scale/zero rows [128][4 B], per token {s_k, z_k, s_v,
+// z_v}, per prep warp the largest s_v, at an item's first tile the queries [16][128]
+// bf16 (two 128-byte-swizzled atoms)
+constexpr int kStKc = 0, kStVc = 8192, kStLv = 16384, kStKsz = 24576, kStVsz = 25088, kStMisc = 25600,
+              kStTmax = 27648, kStQ = 28672, kStage = 32768;
+constexpr int kQlBytes = 6144;                 // query limbs [48][128 B] s8, 128-byte swizzle
+constexpr int kSmQl = kStages * kStage;        // 2 x query limbs (item parity)
+constexpr int kSmP = kSmQl + 2 * kQlBytes;     // 2 x P' limbs [32][128 B] u8; flush exchange
+constexpr int kSmQinfo = kSmP + 8192;          // [2][32]: sigma[16], sum(q)[16] per query head
+constexpr int kSmRed = kSmQinfo + 256;         // [4][16] l, [4][16] zc, [128][6] merge
 constexpr int kSmBar = kSmRed + (2 * 4 * 16 + 128 * 6) * 4;
 constexpr int kSmMisc = kSmBar + 256;
 constexpr int kSmemAlloc = kSmMisc + 64 + 1024;
-static_assert(kSmCvt % 1024 == 0 && kSmQ % 1024 == 0 && kSmP % 1024 == 0, "swizzle atoms need 1 KiB alignment");
-static_assert(kRawStage % 1024 == 0 && kCvtStage % 1024 == 0 && kRawQ % 1024 == 0, "stage alignment");
+static_assert(kStage % 1024 == 0 && kStQ % 1024 == 0 && kSmQl % 1024 == 0 && kSmP % 1024 == 0 &&
+                  kQlBytes % 1024 == 0, "alignment");
+static_assert(kSmemAlloc <= 232448, "shared memory");
 
-// tensor memory columns: S^T x 2, O^T x 2 (64 columns each), K' x kCvt (64 each)
-constexpr int kTmS = 0, kTmO = 128, kTmK = 256, kTmemCols = 512;
-static_assert(kTmK + kCvt * 64 <= kTmemCols, "tensor memory");
-
-constexpr int kBarRawFull = 0, kBarRawEmpty = kRaw, kBarCvtFull = 2 * kRaw, kBarCvtEmpty = 2 * kRaw + kCvt,
-              kBarSFull = 2 * kRaw + 2 * kCvt, kBarSFree = kBarSFull + 2, kBarPFull = kBarSFull + 4,
-              kBarOFull = kBarSFull + 6, kBarDrain = kBarSFull + 8, kNumBars = kBarSFull + 9;
+constexpr int kBarFull = 0, kBarEmpty = kStages, kBarCvt = 2 * kStages, kBarSFull = 3 * kStages,
+              kBarSFree = kBarSFull + 2, kBarPFull = kBarSFull + 4, kBarOFull = kBarSFull + 6,
+              kBarQFree = kBarSFull + 8, kBarDrain = kBarSFull + 10, kNumBars = kBarSFull + 11;
 static_assert(kNumBars * 8 <= 256, "barrier area");
+
+// tensor memory columns: S^T (three limbs per query head) x 2, O^T (two limbs) x 2, and
+// per stage the K low nibbles (16 columns: 4 bytes each)
+template <int NQ>
+struct Cols {
+  static constexpr int kS = (3 * NQ + 15) / 16 * 16;
+  static constexpr int kO = (2 * NQ + 15) / 16 * 16;
+  static constexpr int kLk = 2 * kS + 2 * kO;
+  static constexpr int kUsed = kLk + kStages * 16;
+  static constexpr int kAlloc = kUsed <= 128 ? 128 : kUsed <= 256 ? 256 : 512;
+};
 
 struct Int4DecodeArgs {
   DecodeParams p;
-  int units_r, units_s;  // tiles per retrieval / streaming item
-  int n_items_r;         // B * Hr
-  int64_t ur;            // retrieval tiles in total
-  int64_t total_units;   // ur + streaming tiles
-  int64_t total_cost;    // ur + kWs * streaming tiles
+  int units_r;          // tiles per item
+  int n_items;          // B * Hr
+  int64_t total_units;  // n_items * units_r
   int num_ctas;
-  CUtensorMap tm_q, tm_kc, tm_vc, tm_ks, tm_vs;
+  CUtensorMap tm_q, tm_kc, tm_vc;
 };
+
+// shared-memory matrix descriptor with an explicit layout (2: 128-byte swizzle, 4: 64-byte)
+__device__ __forceinline__ uint64_t sdesc_l(uint32_t saddr, uint32_t lbo, uint32_t sbo, uint32_t layout) {
+  return static_cast<uint64_t>((saddr >> 4) & 0x3FFFu) | (static_cast<uint64_t>((lbo >> 4) & 0x3FFFu) << 16) |
+         (static_cast<uint64_t>((sbo >> 4) & 0x3FFFu) << 32) | (1ull << 46) | (static_cast<uint64_t>(layout) << 61);
+}
+// kind::i8 instruction descriptor: int32 accumulator, A unsigned, B signed or unsigned
+constexpr uint32_t idesc_i8(int M, int N, bool b_signed, bool a_mn_major) {
+  return (2u << 4) | ((b_signed ? 1u : 0u) << 10) | ((a_mn_major ? 1u : 0u) << 15) |
+         ((static_cast<uint32_t>(N) >> 3) << 17) | ((static_cast<uint32_t>(M) >> 4) << 24);
+}
+__device__ __forceinline__ void mma_i8(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc, uint32_t acc) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::i8 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(acc)
+      : "memory");
+}
+// same with A read from tensor memory (lane = row, one column = 4 consecutive K bytes)
+__device__ __forceinline__ void mma_i8_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc, uint32_t acc) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::i8 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(acc)
+      : "memory");
+}
+// Exact int <-> float for |x| < 2^22 on the ALU and FMA pipes: 1.5 * 2^23 has unit
+// mantissa steps, so x + 1.5 * 2^23 holds x in its low mantissa bits.
+constexpr float kMagic = 12582912.0f;
+constexpr int kMagicBits = 0x4B400000;
+__device__ __forceinline__ float to_float(int x) { return __int_as_float(x + kMagicBits) - kMagic; }  // exact
+// x rounded to the nearest integer: its low byte (two's complement) and its value
+__device__ __forceinline__ uint32_t round_byte(float x, float &rounded) {
+  const float t = x + kMagic;
+  rounded = t - kMagic;
+  return static_cast<uint32_t>(__float_as_int(t)) & 0xFFu;
+}
+// N (a multiple of 16) int32 columns of this thread's TMEM lane
+template <int N>
+__device__ __forceinline__ void ld_i32(uint32_t taddr, int (&v)[N]) {
+#pragma unroll
+  for (int c = 0; c < N; c += 16) {
+    float f[16];
+    tc::ld<16>(taddr + c, f);
+#pragma unroll
+    for (int i = 0; i < 16; ++i) v[c + i] = __float_as_int(f[i]);
+  }
+}
+// byte (row n, column k) of a [rows][128 B] K-major operand with 128-byte swizzle
+__device__ __forceinline__ int sw128(int n, int k) { return (n >> 3) * 1024 + (n & 7) * 128 + (((k >> 4) ^ (n & 7)) << 4) + (k & 15); }
 
 struct Unit {
   int item, tile;
-  bool retr;
 };
-__device__ __forceinline__ Unit unit_of(const Int4DecodeArgs &a, int64_t u) {
-  if (u < a.ur) return {static_cast<int>(u / a.units_r), static_cast<int>(u % a.units_r), true};
-  const int64_t us = u - a.ur;
-  return {a.n_items_r + static_cast<int>(us / a.units_s), static_cast<int>(us % a.units_s), false};
-}
 // Walks a CTA's units in order without a division per step.
 struct UnitIter {
   Unit un;
-  int units;  // tiles of the current item
-  __device__ __forceinline__ UnitIter(const Int4DecodeArgs &a, int64_t u) : un(unit_of(a, u)) {
-    units = un.retr ? a.units_r : a.units_s;
-  }
-  __device__ __forceinline__ void next(const Int4DecodeArgs &a) {
+  int units;
+  __device__ __forceinline__ UnitIter(const Int4DecodeArgs &a, int64_t u)
+      : un{static_cast<int>(u / a.units_r), static_cast<int>(u % a.units_r)}, units(a.units_r) {}
+  __device__ __forceinline__ void next() {
     if (++un.tile == units) {
       ++un.item;
       un.tile = 0;
-      un.retr = un.item < a.n_items_r;
-      units = un.retr ? a.units_r : a.units_s;
     }
   }
 };
-__device__ __forceinline__ int64_t start_cost(const Int4DecodeArgs &a, int64_t u) {
-  return u < a.ur ? u : a.ur + (u - a.ur) * kWs;
-}
-// CTA c takes the units whose start cost lies in [floor(c T / C), floor((c+1) T / C))
 __device__ __forceinline__ int64_t cta_begin(const Int4DecodeArgs &a, int c) {
-  const int64_t x = static_cast<int64_t>(c) * a.total_cost / a.num_ctas;
-  return x <= a.ur ? x : a.ur + (x - a.ur + kWs - 1) / kWs;
+  return static_cast<int64_t>(c) * a.total_units / a.num_ctas;
 }
 __device__ __forceinline__ int cta_of(const Int4DecodeArgs &a, int64_t u) {
-  return static_cast<int>(((start_cost(a, u) + 1) * a.num_ctas + a.total_cost - 1) / a.total_cost) - 1;
-}
-// A CTA whose cost range falls strictly inside a bf16 tile u holds no unit.  It still
-// lies between the CTAs of u's item when tile u+1 belongs to the same item; it then
-// counts as one (empty) segment of that item.  Returns that item, or -1.
-__device__ __forceinline__ int empty_cta_item(const Int4DecodeArgs &a, int c) {
-  const int64_t x = static_cast<int64_t>(c) * a.total_cost / a.num_ctas;
-  if (x <= a.ur) return -1;  // every cost below ur starts a tile
-  const int64_t u = a.ur + (x - a.ur) / kWs;
-  if (u + 1 >= a.total_units) return -1;
-  const int item = unit_of(a, u).item;
-  return unit_of(a, u + 1).item == item ? item : -1;
-}
-// (batch, KV head, row of the per-kind arrays) of an item
-__device__ __forceinline__ void item_coords(const Int4DecodeArgs &a, int item, int &b, int &g, int &z) {
-  const DecodeParams &p = a.p;
-  if (item < a.n_items_r) {
-    b = item / p.Hr;
-    const int ri = item % p.Hr;
-    g = p.hm.retr_head[ri];
-    z = b * p.Hr + ri;
-  } else {
-    const int it = item - a.n_items_r;
-    b = it / p.Hs;
-    const int si = it % p.Hs;
-    g = p.hm.strm_head[si];
-    z = b * p.Hs + si;
-  }
+  return static_cast<int>(((u + 1) * a.num_ctas + a.total_units - 1) / a.total_units) - 1;
 }
 
-__device__ __forceinline__ int perm(int x) { return (x & ~7) | ((x & 7) >> 1) | ((x & 1) << 2); }
-
-// codes e0..e7 of one word -> pairs (c_0, c_4), (c_1, c_5), (c_2, c_6), (c_3, c_7), each code
-// OR-ed into the mantissa of kBase: 0x43004300 gives bf16 128 + c, 0x64006400 fp16 1024 + c
-template <uint32_t kBase>
-__device__ __forceinline__ uint4 expand8(uint32_t w) {
-  constexpr uint32_t kM = 0x000F000Fu;
-  return make_uint4((w & kM) | kBase, ((w >> 4) & kM) | kBase, ((w >> 8) & kM) | kBase, ((w >> 12) & kM) | kBase);
-}
-constexpr uint32_t kBf16Base = 0x43004300u;  // K codes: bf16 128 + c
-constexpr uint32_t kFp16Base = 0x64006400u;  // V codes: fp16 1024 + c
-
-// One warp copies the 16 query rows of an item from a raw stage to an expanded-query
-// buffer (both [16][128] bf16 in two 128-byte-swizzled atoms), reordering each 8-element
-// chunk by perm when `permute`, and writes the fp32 sum of every row.
-__device__ __forceinline__ void stage_queries(const char *src, char *dst, float *qsum, int lane, bool permute) {
-  const int r = lane >> 1, atom = lane & 1;
-  float s = 0.f;
+// One warp turns the G query rows of an item (bf16 [16][128], two 128-byte-swizzled
+// atoms) into the B operand of S^T: row 3q + l holds limb l of query head q's
+// coefficients, columns 0..63 those of U (q_{2j+1} / 16), 64..127 those of L
+// (q_{2j} - q_{2j+1} / 16).  Also writes sigma (coefficient = sigma * (l0 + l1 / 2^7 +
+// l2 / 2^14)) and sum(q) of every head.
+__device__ __forceinline__ void prep_queries(const char *qr, char *ql, float *qinfo, int G, int lane) {
+  for (int q = 0; q < G; ++q) {
+    float cu[2], cl[2], qs = 0.f;
 #pragma unroll
-  for (int ch = 0; ch < 8; ++ch) {
-    const int off = atom * 2048 + r * 128 + ((ch ^ (r & 7)) << 4);
-    const uint4 w = *reinterpret_cast<const uint4 *>(src + off);
-    s += (bf16lo(w.x) + bf16hi(w.x)) + (bf16lo(w.y) + bf16hi(w.y)) + (bf16lo(w.z) + bf16hi(w.z)) +
-         (bf16lo(w.w) + bf16hi(w.w));
-    uint4 o = w;
-    if (permute) {
-      o.x = __byte_perm(w.x, w.z, 0x5410);
-      o.y = __byte_perm(w.x, w.z, 0x7632);
-      o.z = __byte_perm(w.y, w.w, 0x5410);
-      o.w = __byte_perm(w.y, w.w, 0x7632);
+    for (int h = 0; h < 2; ++h) {
+      const int j = lane + 32 * h, c = 2 * j;  // columns c, c + 1 of atom h
+      const int off = h * 2048 + q * 128 + ((((c & 63) >> 3) ^ (q & 7)) << 4) + (c & 7) * 2;
+      const uint32_t w = *reinterpret_cast<const uint32_t *>(qr + off);
+      const float e = bf16lo(w), o = bf16hi(w);
+      cu[h] = o * 0.0625f;
+      cl[h] = e - cu[h];
+      qs += e + o;
     }
-    *reinterpret_cast<uint4 *>(dst + off) = o;
+    const float amax = warp_max(fmaxf(fmaxf(fabsf(cu[0]), fabsf(cu[1])), fmaxf(fabsf(cl[0]), fabsf(cl[1]))));
+    qs = warp_sum(qs);
+    const float inv = amax > 0.f ? 127.f / amax : 0.f;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const float x = (i < 2 ? cu[i] : cl[i - 2]) * inv;
+      const int k = (i < 2 ? 0 : 64) + lane + 32 * (i & 1);
+      const float l0 = rintf(x);
+      const float r1 = (x - l0) * 128.f;
+      const float l1 = rintf(r1);
+      const float l2 = rintf((r1 - l1) * 128.f);
+      ql[sw128(3 * q, k)] = static_cast<char>(static_cast<int>(l0));
+      ql[sw128(3 * q + 1, k)] = static_cast<char>(static_cast<int>(l1));
+      ql[sw128(3 * q + 2, k)] = static_cast<char>(static_cast<int>(l2));
+    }
+    if (lane == 0) {
+      qinfo[q] = amax * (1.f / 127.f);
+      qinfo[16 + q] = qs;
+    }
   }
-  s += __shfl_xor_sync(0xffffffffu, s, 1);
-  if (atom == 0) qsum[r] = s;
 }
 
 template <int NQ>
 __global__ void __launch_bounds__(kThreads, 1) decode_int4_kernel(const __grid_constant__ Int4DecodeArgs a) {
+  using C = Cols<NQ>;
   const DecodeParams &p = a.p;
   extern __shared__ char smem_raw[];
   char *smem = reinterpret_cast<char *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -206,10 +217,9 @@ __global__ void __launch_bounds__(kThreads, 1) decode_int4_kernel(const __grid_c
   volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + kSmMisc + 4);
   volatile int *last_flag = reinterpret_cast<volatile int *>(smem + kSmMisc + 8);
   float *red = reinterpret_cast<float *>(smem + kSmRed);
-  const float *qsum_all = reinterpret_cast<const float *>(smem + kSmQsum);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  // A decode launched next on the stream may start its set-up on the SMs this grid
+  // A kernel launched next on the stream may start its set-up on the SMs this grid
   // frees; it touches global memory only after its own griddepcontrol.wait, which
   // returns once this whole grid has completed.
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
@@ -218,27 +228,23 @@ __global__ void __launch_bounds__(kThreads, 1) decode_int4_kernel(const __grid_c
   const int G = p.G;
 
   if (tid == 0) {
-    for (int i = 0; i < kRaw; ++i) {
-      mbar_init(bar(kBarRawFull + i), 1);
-      mbar_init(bar(kBarRawEmpty + i), 256);
-    }
-    for (int i = 0; i < kCvt; ++i) {
-      mbar_init(bar(kBarCvtFull + i), 256);
-      mbar_init(bar(kBarCvtEmpty + i), 1);
+    for (int i = 0; i < kStages; ++i) {
+      mbar_init(bar(kBarFull + i), 1);
+      mbar_init(bar(kBarEmpty + i), 1);
+      mbar_init(bar(kBarCvt + i), 128);
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(bar(kBarSFull + i), 1);
       mbar_init(bar(kBarSFree + i), 128);
       mbar_init(bar(kBarPFull + i), 128);
       mbar_init(bar(kBarOFull + i), 1);
+      mbar_init(bar(kBarQFree + i), 2);  // the item's last S^T product (commit) + the softmax
     }
     mbar_init(bar(kBarDrain), 1);
     fence_mbar_init();
     *abort_flag = 0;
   }
-  // P'^T rows >= G stay zero for the whole kernel
-  for (int i = tid; i < 8192 / 16; i += kThreads) reinterpret_cast<uint4 *>(smem + kSmP)[i] = make_uint4(0, 0, 0, 0);
-  if (warp == 1) tc::tmem_alloc(smem_u32(tmem_slot), kTmemCols);
+  if (warp == 1) tc::tmem_alloc(smem_u32(tmem_slot), C::kAlloc);
   tc::fence_async_smem();
   tc::fence_before();
   __syncthreads();
@@ -248,110 +254,99 @@ __global__ void __launch_bounds__(kThreads, 1) decode_int4_kernel(const __grid_c
   if (warp == 0) {
     // ================= TMA producer =================
     if (lane == 0) {
+      for (const CUtensorMap *m : {&a.tm_q, &a.tm_kc, &a.tm_vc})
+        asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(m)) : "memory");
+      {  // L2 prefetch of the first tiles; no data is consumed before the wait below
+        UnitIter it(a, u0);
+        for (int j = 0; j < nu && j < kPrefetch; ++j, it.next()) {
+          const int64_t row = static_cast<int64_t>(it.un.item) * p.max_len + static_cast<int64_t>(it.un.tile) * kTile;
+          prefetch_l2(p.rk + row * (kD / 2), kTile * kD / 2);
+          prefetch_l2(p.rv + row * (kD / 2), kTile * kD / 2);
+          prefetch_l2(p.rk_sz + row * 4, kTile * 4);
+          prefetch_l2(p.rv_sz + row * 4, kTile * 4);
+        }
+      }
       // Launched as a programmatic dependent, this grid's set-up overlaps the previous
       // kernel on the stream; nothing is read from global memory before that kernel has
       // finished (every other read and every write of this grid follows these loads).
       asm volatile("griddepcontrol.wait;" ::: "memory");
-      int r = 0, prev_item = -1;
-      bool ok = true;
+      int prev_item = -1;
       UnitIter it(a, u0);
-      for (int j = 0; j < nu && ok; ++j, it.next(a)) {
+      for (int j = 0; j < nu; ++j, it.next()) {
+        const int s = j % kStages;
+        if (j >= kStages && !tc::wait_bar(bar(kBarEmpty + s), ((j / kStages) - 1) & 1, p.status, abort_flag)) break;
         const Unit un = it.un;
         const bool first = un.item != prev_item;
         prev_item = un.item;
-        int b, g, z;
-        item_coords(a, un.item, b, g, z);
-        const int qrow = b * p.Hq + g * G;  // rows beyond this group's G heads are never used
-        const int pieces = un.retr ? 1 : 4;
-        for (int c = 0; c < pieces; ++c, ++r) {
-          const int s = r % kRaw;
-          if (r >= kRaw && !tc::wait_bar(bar(kBarRawEmpty + s), ((r / kRaw) - 1) & 1, p.status, abort_flag)) {
-            ok = false;
-            break;
-          }
-          const uint32_t dst = sbase + kSmRaw + s * kRawStage;
-          const uint32_t fb = bar(kBarRawFull + s);
-          const bool with_q = first && c == 0;
-          if (un.retr) {
-            mbar_expect_tx(fb, 2 * 8192 + 2 * 512 + (with_q ? 4096 : 0));
-            const int y = un.tile * kTile;
-            tc::tma_3d(dst + kRawKc, &a.tm_kc, 0, y, z, fb);
-            tc::tma_3d(dst + kRawVc, &a.tm_vc, 0, y, z, fb);
-            const int64_t row = static_cast<int64_t>(z) * p.max_len + y;
-            bulk_g2s(dst + kRawKsz, p.rk_sz + row * 4, 512, fb);
-            bulk_g2s(dst + kRawVsz, p.rv_sz + row * 4, 512, fb);
-          } else {
-            mbar_expect_tx(fb, 4 * 4096 + (with_q ? 4096 : 0));
-            const int y = un.tile * kTile + 32 * c;  // rows past S+W read as zeros
-            tc::tma_3d(dst, &a.tm_ks, 0, y, z, fb);
-            tc::tma_3d(dst + 4096, &a.tm_ks, 64, y, z, fb);
-            tc::tma_3d(dst + 8192, &a.tm_vs, 0, y, z, fb);
-            tc::tma_3d(dst + 12288, &a.tm_vs, 64, y, z, fb);
-          }
-          if (with_q) {
-            tc::tma_2d(dst + kRawQ, &a.tm_q, 0, qrow, fb);
-            tc::tma_2d(dst + kRawQ + 2048, &a.tm_q, 64, qrow, fb);
-          }
+        const uint32_t dst = sbase + s * kStage;
+        const uint32_t fb = bar(kBarFull + s);
+        mbar_expect_tx(fb, 2 * 8192 + 2 * 512 + (first ? 4096 : 0));
+        const int y = un.tile * kTile;
+        const int z = un.item;  // = b * Hr + retrieval index
+        tc::tma_3d(dst + kStKc, &a.tm_kc, 0, y, z, fb);
+        tc::tma_3d(dst + kStVc, &a.tm_vc, 0, y, z, fb);
+        const int64_t row = static_cast<int64_t>(z) * p.max_len + y;
+        bulk_g2s(dst + kStKsz, p.rk_sz + row * 4, 512, fb);
+        bulk_g2s(dst + kStVsz, p.rv_sz + row * 4, 512, fb);
+        if (first) {
+          const int b = un.item / p.Hr;
+          const int g = p.hm.retr_head[un.item % p.Hr];
+          const int qrow = b * p.Hq + g * G;  // rows beyond this group's G heads are never used
+          tc::tma_2d(dst + kStQ, &a.tm_q, 0, qrow, fb);
+          tc::tma_2d(dst + kStQ + 2048, &a.tm_q, 64, qrow, fb);
         }
       }
     }
   } else if (warp == 1) {
     // ================= MMA issuer =================
-    // Event-driven: S(js) as soon as its expanded stage is ready and its S buffer free,
-    // O(jo) as soon as the softmax has written P'(jo), whichever comes first.
+    // Event-driven: S^T(js) as soon as its prep is done and its S buffer is free, O^T(jo)
+    // as soon as the softmax has written P'(jo), whichever comes first.
     if (lane == 0) {
-      constexpr uint32_t kIdS = tc::idesc_bf16(128, 16, false, false);
-      constexpr uint32_t kIdO = tc::idesc_bf16(128, 16, true, false);
-      constexpr uint32_t kIdO16 = tc::idesc_f16(128, 16, true, false, false);  // INT4 tiles: fp16 V" and P'
-      // descriptors of every operand base; a K step adds its byte offset >> 4
-      const uint64_t dq0 = tc::sdesc(sbase + kSmQ, 16, 1024);                         // Qpad, K-major
-      const uint64_t dv0 = tc::sdesc(sbase + kSmCvt + kCvtV, 16384, 1024);           // V"^T, MN-major
-      const uint64_t dp0 = tc::sdesc(sbase + kSmP, 16, 1024);                         // P'^T, K-major
+      constexpr uint32_t kIdS = idesc_i8(128, C::kS, true, false);   // [U | L] . Qx^T
+      constexpr uint32_t kIdO = idesc_i8(128, C::kO, true, true);    // [U_V | L_V]^T . P'^T
       int js = 0, jo = 0, nitem = -1, prev_item = -1;
-      UnitIter its(a, u0), ito(a, u0);
+      UnitIter its(a, u0);
       uint32_t idle = 0;
       unsigned long long t_idle = 0;
       while (jo < nu) {
         bool did = false;
         if (js < nu) {
-          const int cs = js % kCvt;
-          if (mbar_test_wait(bar(kBarCvtFull + cs), (js / kCvt) & 1) &&
+          const int s = js % kStages;
+          if (mbar_test_wait(bar(kBarCvt + s), (js / kStages) & 1) &&
               (js < 2 || mbar_test_wait(bar(kBarSFree + (js & 1)), ((js - 2) >> 1) & 1))) {
             const int item = its.un.item;
-            its.next(a);
+            its.next();
             if (item != prev_item) {
               prev_item = item;
               ++nitem;
             }
             tc::fence_after();
-            const uint64_t dq = dq0 + (nitem & 1) * (4096 >> 4);
-            const uint32_t d = tmem + kTmS + (js & 1) * kAcc * 16;
-            const uint32_t ka = tmem + kTmK + cs * 64;
-#pragma unroll
-            for (int i = 0; i < 8; ++i) {  // K = d 128 in steps of 16 (8 TMEM columns each)
-              const int kk = (i % kAcc) * (8 / kAcc) + i / kAcc;
-              tc::mma_ts(d + (i % kAcc) * 16, ka + kk * 8, dq + (kk >> 2) * 128 + (kk & 3) * 2, kIdS, i >= kAcc ? 1u : 0u);
-            }
+            const uint64_t ak = sdesc_l(sbase + s * kStage + kStKc, 16, 512, 4);
+            const uint32_t al = tmem + C::kLk + s * 16;
+            const uint64_t bq = sdesc_l(sbase + kSmQl + (nitem & 1) * kQlBytes, 16, 1024, 2);
+            const uint32_t d = tmem + (js & 1) * C::kS;
+            mma_i8(d, ak, bq, kIdS, 0u);             // bytes 0..31 of the code rows
+            mma_i8(d, ak + 2, bq + 2, kIdS, 1u);     // bytes 32..63
+            mma_i8_ts(d, al, bq + 4, kIdS, 1u);      // low nibbles 0..31 (TMEM)
+            mma_i8_ts(d, al + 8, bq + 6, kIdS, 1u);  // low nibbles 32..63
             tc::commit(bar(kBarSFull + (js & 1)));
             ++js;
+            // the item's query limbs are free once its last S^T product has run
+            if (js == nu || its.un.item != item) tc::commit(bar(kBarQFree + (nitem & 1)));
             did = true;
           }
         }
         if (jo < js && mbar_test_wait(bar(kBarPFull + (jo & 1)), (jo >> 1) & 1)) {
           tc::fence_after();
-          const int cs = jo % kCvt;
-          const uint32_t id = ito.un.retr ? kIdO16 : kIdO;
-          ito.next(a);
-          const uint64_t dv = dv0 + cs * (kCvtStage >> 4);
-          const uint64_t dp = dp0 + (jo & 1) * (4096 >> 4);
-          const uint32_t d = tmem + kTmO + (jo & 1) * kAcc * 16;
+          const int s = jo % kStages;
+          const uint64_t av = sdesc_l(sbase + s * kStage + kStVc, kStLv - kStVc, 512, 4);  // MN-major, 2 chunks
+          const uint64_t bp = sdesc_l(sbase + kSmP + (jo & 1) * 4096, 16, 1024, 2);
+          const uint32_t d = tmem + 2 * C::kS + (jo & 1) * C::kO;
 #pragma unroll
-          for (int i = 0; i < 8; ++i) {  // K = 128 tokens in steps of 16
-            const int kk = (i % kAcc) * (8 / kAcc) + i / kAcc;
-            tc::mma_ss(d + (i % kAcc) * 16, dv + kk * 128, dp + (kk >> 2) * 128 + (kk & 3) * 2, id, i >= kAcc ? 1u : 0u);
-          }
+          for (int k = 0; k < 4; ++k)  // 32 tokens per step
+            mma_i8(d, av + k * (2048 >> 4), bp + k * 2, kIdO, k > 0 ? 1u : 0u);
           tc::commit(bar(kBarOFull + (jo & 1)));
-          tc::commit(bar(kBarCvtEmpty + cs));  // V", K' and the stage's scales are no longer read
+          tc::commit(bar(kBarEmpty + s));  // the stage and its K low nibbles are no longer read
           ++jo;
           did = true;
         }
@@ -362,7 +357,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_int4_kernel(const __grid_c
           if (jo < js)
             mbar_try_wait_ns(bar(kBarPFull + (jo & 1)), (jo >> 1) & 1, 100);
           else
-            mbar_try_wait_ns(bar(kBarCvtFull + js % kCvt), (js / kCvt) & 1, 100);
+            mbar_try_wait_ns(bar(kBarCvt + js % kStages), (js / kStages) & 1, 100);
           if (++idle == 1) t_idle = globaltimer();
         }
         if (idle > 0 && (idle & 63) == 0) {
@@ -379,79 +374,92 @@ __global__ void __launch_bounds__(kThreads, 1) decode_int4_kernel(const __grid_c
     }
   } else if (warp < 6) {
     // ================= softmax warpgroup =================
-    // As in the bf16 kernel (lazy rescaling against a reference max, exact for INT4
-    // items), plus the scale and zero of every token: s = s_k (q . c') + (z_k - 128 s_k)
-    // sum(q); the MMA gets p' = fp16(p s_v) and zc accumulates p z_v - 1024 p' (bf16
-    // tiles: p' = bf16(p), zc = 0).
-    constexpr float kSlack = 8.0f;
+    // Exact running max (p <= 1, which bounds the P' limbs); s = s_k (q . c) + z_k sum(q);
+    // the MMA gets P' = p s_v as two signed limbs below the tile's largest s_v; zc
+    // accumulates p z_v.
     const int wq = warp & 3;
     const int t = (wq << 5) | lane;
     const uint32_t lane_base = tmem + (static_cast<uint32_t>(wq << 5) << 16);
     const float c = p.scale_log2;
-    float m[NQ], l[NQ], zc[NQ], o[NQ], qs[NQ];
+    float m[NQ], l[NQ], zc[NQ], o[NQ], sg[NQ], qs[NQ];
 #pragma unroll
     for (int q = 0; q < NQ; ++q) {
       m[q] = -INFINITY;
       l[q] = 0.f;
       zc[q] = 0.f;
       o[q] = 0.f;
+      sg[q] = 0.f;
       qs[q] = 0.f;
     }
-    bool ok = true, cur_int4 = false;
+    bool ok = true;
     int cur_item = -1, nitem = -1;
+    float sigp_prev = 0.f;  // P' limb scale of the previous tile
 
     // Writes this CTA's result for `item` (partial or final) and merges when last.
+    // Thread t < 64 ends with dimensions 2t, 2t + 1 of every head: its lane summed the
+    // code bytes of pair t, lane 64 + t the low nibbles.
     auto flush = [&](int item) {
 #pragma unroll
       for (int q = 0; q < NQ; ++q) {
         const float vl = warp_sum(l[q]);
         const float vz = warp_sum(zc[q]);
         if (lane == 0) {
-          red[wq * kN + q] = vl;
-          red[64 + wq * kN + q] = vz;
+          red[wq * 16 + q] = vl;
+          red[64 + wq * 16 + q] = vz;
         }
       }
-      tc::named_sync(1, 128);
-      float lt[NQ], zt[NQ];
-#pragma unroll
-      for (int q = 0; q < NQ; ++q) {
-        lt[q] = red[q] + red[kN + q] + red[2 * kN + q] + red[3 * kN + q];
-        zt[q] = red[64 + q] + red[64 + kN + q] + red[64 + 2 * kN + q] + red[64 + 3 * kN + q];
-      }
-      tc::named_sync(1, 128);
-      const bool retr = item < a.n_items_r;
-      const int units = retr ? a.units_r : a.units_s;
-      const int64_t ia = retr ? static_cast<int64_t>(item) * a.units_r
-                              : a.ur + static_cast<int64_t>(item - a.n_items_r) * a.units_s;
-      const int cfirst = cta_of(a, ia), clast = cta_of(a, ia + units - 1);
-      const int nseg = clast - cfirst + 1;
-      int b, g, z;
-      item_coords(a, item, b, g, z);
-      const int h0 = g * G;
-      const int e = cur_int4 ? perm(t) : t;  // output element held by this thread's O^T lane
-      if (nseg == 1) {
+      float *xch = reinterpret_cast<float *>(smem + kSmP);  // [16][64]; both P' buffers are idle here
+      if (t >= 64) {
 #pragma unroll
         for (int q = 0; q < NQ; ++q)
-          if (q < G) {
-            Elem<__nv_bfloat16>::store(p.out, (static_cast<int64_t>(b) * p.Hq + h0 + q) * kD + e,
-                                       (o[q] + zt[q]) / lt[q]);
-            if (t == 0 && p.lse) p.lse[b * p.Hq + h0 + q] = (m[q] + lg2(lt[q])) * kLn2;
-          }
+          if (q < G) xch[q * 64 + (t - 64)] = o[q];
+      }
+      tc::named_sync(1, 128);
+      float lt[NQ], zt[NQ], ev[NQ], od[NQ];
+#pragma unroll
+      for (int q = 0; q < NQ; ++q) {
+        lt[q] = red[q] + red[16 + q] + red[32 + q] + red[48 + q];
+        zt[q] = red[64 + q] + red[80 + q] + red[96 + q] + red[112 + q];
+        const float lo = t < 64 && q < G ? xch[q * 64 + t] : 0.f;
+        ev[q] = lo + zt[q];
+        od[q] = (o[q] - lo) * 0.0625f + zt[q];
+      }
+      tc::named_sync(1, 128);
+      const int units = a.units_r;
+      const int64_t ia = static_cast<int64_t>(item) * units;
+      const int cfirst = cta_of(a, ia), clast = cta_of(a, ia + units - 1);
+      const int nseg = clast - cfirst + 1;
+      const int b = item / p.Hr;
+      const int g = p.hm.retr_head[item % p.Hr];
+      const int h0 = g * G;
+      if (nseg == 1) {
+        if (t < 64) {
+#pragma unroll
+          for (int q = 0; q < NQ; ++q)
+            if (q < G) {
+              const float inv = 1.f / lt[q];
+              const __nv_bfloat162 pr = __floats2bfloat162_rn(ev[q] * inv, od[q] * inv);
+              *reinterpret_cast<__nv_bfloat162 *>(p.out + ((static_cast<int64_t>(b) * p.Hq + h0 + q) * kD + 2 * t) * 2) = pr;
+              if (t == 0 && p.lse) p.lse[b * p.Hq + h0 + q] = (m[q] + lg2(lt[q])) * kLn2;
+            }
+        }
         return;
       }
       const int seg = blockIdx.x - cfirst;
       const int64_t pitem = static_cast<int64_t>(b) * p.Hkv + g;
       float *part = p.partials + (pitem * p.max_splits) * G * kPartRow;
+      if (t < 64) {
 #pragma unroll
-      for (int q = 0; q < NQ; ++q)
-        if (q < G) {
-          float *dst = part + (static_cast<int64_t>(seg) * G + q) * kPartRow;
-          dst[e] = o[q] + zt[q];
-          if (t == 0) {
-            dst[kD] = m[q];
-            dst[kD + 1] = lt[q];
+        for (int q = 0; q < NQ; ++q)
+          if (q < G) {
+            float *dst = part + (static_cast<int64_t>(seg) * G + q) * kPartRow;
+            *reinterpret_cast<float2 *>(dst + 2 * t) = make_float2(ev[q], od[q]);
+            if (t == 0) {
+              dst[kD] = m[q];
+              dst[kD + 1] = lt[q];
+            }
           }
-        }
+      }
       __threadfence();
       tc::named_sync(1, 128);
       if (t == 0) {
@@ -465,14 +473,15 @@ __global__ void __launch_bounds__(kThreads, 1) decode_int4_kernel(const __grid_c
       if (t == 0) p.counters[pitem] = 0u;  // ready for the next call
     };
 
-    // o = (o + O^T(jj)) * alpha for this thread's position t
-    auto fold = [&](int jj, const float (&alpha)[NQ]) {
+    // o = (o + O^T(jj)) * alpha for this thread's row of O^T
+    auto fold = [&](int jj, float sigp, const float (&alpha)[NQ]) {
       if (ok) ok = tc::wait_bar(bar(kBarOFull + (jj & 1)), (jj >> 1) & 1, p.status, abort_flag);
       tc::fence_after();
-      float v[NQ];
-      tc::ld_sum<NQ, kAcc>(lane_base + kTmO + (jj & 1) * kAcc * 16, 16, v);
+      int r[C::kO];
+      ld_i32<C::kO>(lane_base + 2 * C::kS + (jj & 1) * C::kO, r);
 #pragma unroll
-      for (int q = 0; q < NQ; ++q) o[q] = (o[q] + v[q]) * alpha[q];
+      for (int q = 0; q < NQ; ++q)  // |R| < 2^22
+        o[q] = fmaf(sigp, fmaf(to_float(r[2 * q + 1]), 1.f / 254.f, to_float(r[2 * q])), o[q]) * alpha[q];
     };
     float one[NQ];
 #pragma unroll
@@ -480,61 +489,56 @@ __global__ void __launch_bounds__(kThreads, 1) decode_int4_kernel(const __grid_c
 
     bool pending = false;  // O^T of the previous unit still to be folded
     UnitIter it(a, u0);
-    for (int j = 0; j < nu; ++j, it.next(a)) {
+    for (int j = 0; j < nu; ++j, it.next()) {
       const Unit un = it.un;
-      const int cb = j & 1;
+      const int cb = j & 1, s = j % kStages;
       if (ok) ok = tc::wait_bar(bar(kBarSFull + cb), (j >> 1) & 1, p.status, abort_flag);
       tc::fence_after();
-      float sv[NQ];
-      tc::ld_sum<NQ, kAcc>(lane_base + kTmS + cb * kAcc * 16, 16, sv);
+      int sr[C::kS];
+      ld_i32<C::kS>(lane_base + cb * C::kS, sr);
       tc::fence_before();
       mbar_arrive(bar(kBarSFree + cb));  // S buffer j % 2 is free again
-      // the expanded stage of this tile (complete already: its MMA has run) holds the
-      // scales; waiting here orders the expansion warps' writes before these reads
-      const int cs = j % kCvt;
-      if (ok) ok = tc::wait_bar(bar(kBarCvtFull + cs), (j / kCvt) & 1, p.status, abort_flag);
-      const float4 mi = *reinterpret_cast<const float4 *>(smem + kSmCvt + cs * kCvtStage + kCvtMisc + t * 16);
-      // this token's validity
-      bool valid;
-      const int64_t tok = static_cast<int64_t>(un.tile) * kTile + t;
-      if (un.retr) {
-        valid = tok < p.len;
-      } else {
-        const int S = p.S, W = p.W;
-        const int64_t len = p.len;
-        const int64_t rstart = (len - W > S) ? len - W : S;
-        const int64_t rcount = len > rstart ? len - rstart : 0;
-        if (tok >= S + W) valid = false;
-        else if (tok < S) valid = tok < len;
-        else if (rcount >= W) valid = true;
-        else valid = (((tok - S) - (S % W)) % W + W) % W < rcount;
-      }
+      // the stage's prep is complete (its S^T product has run); waiting here orders the
+      // prep warps' writes before these reads
+      if (ok) ok = tc::wait_bar(bar(kBarCvt + s), (j / kStages) & 1, p.status, abort_flag);
+      const char *st = smem + s * kStage;
+      const float4 mi = *reinterpret_cast<const float4 *>(st + kStMisc + t * 16);  // s_k, z_k, s_v, z_v
+      const float4 tm4 = *reinterpret_cast<const float4 *>(st + kStTmax);
+      const float tmax = fmaxf(fmaxf(tm4.x, tm4.y), fmaxf(tm4.z, tm4.w));
+      const bool valid = static_cast<int64_t>(un.tile) * kTile + t < p.len;
       if (un.item != cur_item) {
         if (cur_item >= 0) {
-          if (pending) fold(j - 1, one);
+          if (pending) fold(j - 1, sigp_prev, one);
           flush(cur_item);
         }
         ++nitem;
+        const float *qi = reinterpret_cast<const float *>(smem + kSmQinfo) + (nitem & 1) * 32;
 #pragma unroll
         for (int q = 0; q < NQ; ++q) {
           m[q] = -INFINITY;
           l[q] = 0.f;
           zc[q] = 0.f;
           o[q] = 0.f;
-          qs[q] = qsum_all[(nitem & 1) * kN + q];
+          sg[q] = qi[q];
+          qs[q] = qi[16 + q];
         }
+        tc::named_sync(1, 128);
+        if (t == 0) mbar_arrive(bar(kBarQFree + (nitem & 1)));  // every thread has read the item's sigma and sum(q)
         pending = false;
         cur_item = un.item;
-        cur_int4 = un.retr;
       }
+      float sv[NQ];
 #pragma unroll
-      for (int q = 0; q < NQ; ++q) sv[q] = fmaf(mi.x, sv[q], mi.y * qs[q]);
-      const float slack = cur_int4 ? 0.f : kSlack;
-      // does any logit of this tile exceed the reference max by more than kSlack?
+      for (int q = 0; q < NQ; ++q) {  // S0 + S1 / 2^7 + S2 / 2^14, |S| < 2^22
+        const float x = fmaf(fmaf(to_float(sr[3 * q + 2]), 1.f / 128.f, to_float(sr[3 * q + 1])), 1.f / 128.f,
+                             to_float(sr[3 * q]));
+        sv[q] = fmaf(mi.x, sg[q] * x, mi.y * qs[q]);
+      }
+      // does any logit of this tile exceed the running max?
       int need = 0;
 #pragma unroll
       for (int q = 0; q < NQ; ++q)
-        if (q < G && valid && sv[q] * c > m[q] + slack) need = 1;
+        if (q < G && valid && sv[q] * c > m[q]) need = 1;
       need = tc::bar_or(1, 128, need);
       float alpha[NQ];
 #pragma unroll
@@ -543,166 +547,118 @@ __global__ void __launch_bounds__(kThreads, 1) decode_int4_kernel(const __grid_c
 #pragma unroll
         for (int q = 0; q < NQ; ++q) {
           const float x = warp_max((valid && q < G) ? sv[q] : -INFINITY);
-          if (lane == 0) red[wq * kN + q] = x;
+          if (lane == 0) red[wq * 16 + q] = x;
         }
         tc::named_sync(1, 128);
 #pragma unroll
         for (int q = 0; q < NQ; ++q) {
-          const float mt = fmaxf(fmaxf(red[q], red[kN + q]), fmaxf(red[2 * kN + q], red[3 * kN + q])) * c;
+          const float mt = fmaxf(fmaxf(red[q], red[16 + q]), fmaxf(red[32 + q], red[48 + q])) * c;
           const float mn = fmaxf(m[q], mt);
           alpha[q] = (mn == -INFINITY) ? 1.f : ex2(m[q] - mn);
           m[q] = mn;
         }
         tc::named_sync(1, 128);  // red is reused later
       }
-      uint16_t pb[NQ];
+      // P'^T limbs into buffer j % 2 (its previous reader, unit j-2, was folded at j-1):
+      // p s_v = sigp (l0 + l1 / 254) with l0 = rint(x) in [0, 127], x = p s_v / sigp, and
+      // l1 = rint(254 (x - l0)) in [-127, 127]; sigp = tmax / 126.99
+      const float invp = tmax > 0.f ? 126.99f / tmax : 0.f;
+      uint8_t *pb = reinterpret_cast<uint8_t *>(smem + kSmP + cb * 4096);
 #pragma unroll
       for (int q = 0; q < NQ; ++q) {
         const float pv = (valid && q < G && m[q] != -INFINITY) ? ex2(fmaf(sv[q], c, -m[q])) : 0.f;
         l[q] = fmaf(l[q], alpha[q], pv);
-        if (cur_int4) {
-          const __half hp = __float2half_rn(pv * mi.z);
-          zc[q] = fmaf(zc[q], alpha[q], fmaf(pv, mi.w, -1024.f * __half2float(hp)));
-          pb[q] = __half_as_ushort(hp);
-        } else {
-          const __nv_bfloat16 hb = __float2bfloat16_rn(pv);
-          pb[q] = *reinterpret_cast<const uint16_t *>(&hb);
+        zc[q] = fmaf(zc[q], alpha[q], pv * mi.w);
+        if (q < G) {
+          const float x = pv * mi.z * invp;
+          float r0, r1;
+          const uint32_t b0 = round_byte(x, r0);
+          const uint32_t b1 = round_byte((x - r0) * 254.f, r1);
+          pb[sw128(2 * q, t)] = static_cast<uint8_t>(b0);
+          pb[sw128(2 * q + 1, t)] = static_cast<uint8_t>(b1);
         }
-      }
-      // P'^T[q][t] into buffer j % 2 (its previous reader, unit j-2, was folded at j-1)
-      {
-        const int atom = t >> 6, col = t & 63;
-        char *pbase = smem + kSmP + cb * 4096 + atom * 2048;
-#pragma unroll
-        for (int q = 0; q < NQ; ++q)
-          if (q < G) {
-            const int chunk = (col >> 3) ^ (q & 7);
-            *reinterpret_cast<uint16_t *>(pbase + q * 128 + chunk * 16 + (col & 7) * 2) = pb[q];
-          }
       }
       tc::fence_async_smem();
       tc::fence_before();
       mbar_arrive(bar(kBarPFull + cb));
       // fold the previous unit of the same item, bringing it to this unit's scale
       if (pending) {
-        fold(j - 1, alpha);
+        fold(j - 1, sigp_prev, alpha);
       } else {
 #pragma unroll
         for (int q = 0; q < NQ; ++q) o[q] *= alpha[q];
       }
+      sigp_prev = tmax * (1.f / 126.99f);
       pending = true;
     }
     if (nu > 0) {
-      if (pending) fold(nu - 1, one);
+      if (pending) fold(nu - 1, sigp_prev, one);
       flush(cur_item);
-    } else {
-      const int item = empty_cta_item(a, blockIdx.x);
-      if (item >= 0) flush(item);  // m = -inf, l = 0, o = 0: a segment that sees nothing
     }
   } else {
-    // ================= expansion warps =================
+    // ================= prep warps =================
     const int wq = warp & 3;
-    const int h = (warp - 6) >> 2;    // half of the row: elements 64 h .. 64 h + 63
-    const int ct = (wq << 5) | lane;  // token row of the tile = TMEM lane
+    const int ct = (wq << 5) | lane;  // token row of the tile
+    const int rot = (ct >> 1) & 3;    // 64-byte swizzle of row ct: chunk i sits at i ^ rot
     const uint32_t tm_lane = tmem + (static_cast<uint32_t>(wq << 5) << 16);
-    const int rot = (ct >> 1) & 3;    // 64-byte swizzle of code row ct: chunk i sits at i ^ rot
-    int r = 0, prev_item = -1, nitem = -1;
+    int prev_item = -1, nitem = -1;
     UnitIter it(a, u0);
-    for (int j = 0; j < nu; ++j, it.next(a)) {
+    for (int j = 0; j < nu; ++j, it.next()) {
       const Unit un = it.un;
       const bool first = un.item != prev_item;
       if (first) {
         prev_item = un.item;
         ++nitem;
       }
-      const int cb = j % kCvt;
-      if (j >= kCvt && !tc::wait_bar(bar(kBarCvtEmpty + cb), ((j / kCvt) - 1) & 1, p.status, abort_flag)) break;
-      char *cv = smem + kSmCvt + cb * kCvtStage;
-      char *qdst = smem + kSmQ + (nitem & 1) * 4096;
-      float *qsum = reinterpret_cast<float *>(smem + kSmQsum) + (nitem & 1) * kN;
-      const uint32_t tk = tm_lane + kTmK + cb * 64 + h * 32;
-      if (un.retr) {
-        const int s = r % kRaw;
-        if (!tc::wait_bar(bar(kBarRawFull + s), (r / kRaw) & 1, p.status, abort_flag)) break;
-        const char *rs = smem + kSmRaw + s * kRawStage;
-        uint4 kw[2], vw[2];
+      const int s = j % kStages;
+      if (!tc::wait_bar(bar(kBarFull + s), (j / kStages) & 1, p.status, abort_flag)) break;
+      tc::fence_after();  // the TMEM columns written below were last read by an MMA
+      char *st = smem + s * kStage;
+      uint32_t lk[16];
 #pragma unroll
-        for (int i = 0; i < 2; ++i) {
-          const int off = ct * 64 + (((2 * h + i) ^ rot) << 4);
-          kw[i] = *reinterpret_cast<const uint4 *>(rs + kRawKc + off);
-          vw[i] = *reinterpret_cast<const uint4 *>(rs + kRawVc + off);
-        }
-#pragma unroll
-        for (int i = 0; i < 2; ++i) {  // K: 32 codes -> TMEM columns 32 h + 16 i ..
-          const uint4 e0 = expand8<kBf16Base>(kw[i].x), e1 = expand8<kBf16Base>(kw[i].y),
-                      e2 = expand8<kBf16Base>(kw[i].z), e3 = expand8<kBf16Base>(kw[i].w);
-          const uint32_t v[16] = {e0.x, e0.y, e0.z, e0.w, e1.x, e1.y, e1.z, e1.w,
-                                  e2.x, e2.y, e2.z, e2.w, e3.x, e3.y, e3.z, e3.w};
-          tc::st16(tk + i * 16, v);
-        }
-        char *vrow = cv + kCvtV + h * 16384 + ct * 128;
-#pragma unroll
-        for (int i = 0; i < 2; ++i) {  // V: 32 codes -> chunks 4 i .. 4 i + 3 of atom h
-          const uint32_t ws[4] = {vw[i].x, vw[i].y, vw[i].z, vw[i].w};
-#pragma unroll
-          for (int mm = 0; mm < 4; ++mm)
-            *reinterpret_cast<uint4 *>(vrow + (((4 * i + mm) ^ (ct & 7)) << 4)) = expand8<kFp16Base>(ws[mm]);
-        }
-        if (h == 0) {
-          const uint32_t ksz = *reinterpret_cast<const uint32_t *>(rs + kRawKsz + ct * 4);
-          const uint32_t vsz = *reinterpret_cast<const uint32_t *>(rs + kRawVsz + ct * 4);
-          const float ks = __half2float(__ushort_as_half(static_cast<unsigned short>(ksz & 0xffffu)));
-          const float kz = __half2float(__ushort_as_half(static_cast<unsigned short>(ksz >> 16)));
-          const float vs = __half2float(__ushort_as_half(static_cast<unsigned short>(vsz & 0xffffu)));
-          const float vz = __half2float(__ushort_as_half(static_cast<unsigned short>(vsz >> 16)));
-          *reinterpret_cast<float4 *>(cv + kCvtMisc + ct * 16) = make_float4(ks, fmaf(-128.f, ks, kz), vs, vz);
-        } else if (first && wq == 0) {
-          stage_queries(rs + kRawQ, qdst, qsum, lane, true);
-        }
-        mbar_arrive(bar(kBarRawEmpty + s));  // all 256 threads read this stage
-        ++r;
-      } else {
-        // the two warps of quarter wq expand piece wq (tokens 32 wq .. 32 wq + 31)
-        const int s = (r + wq) % kRaw;
-        if (!tc::wait_bar(bar(kBarRawFull + s), ((r + wq) / kRaw) & 1, p.status, abort_flag)) break;
-        const char *rs = smem + kSmRaw + s * kRawStage;
-#pragma unroll
-        for (int i = 0; i < 2; ++i) {  // K half h -> TMEM columns 32 h + 16 i ..
-          uint32_t v[16];
-#pragma unroll
-          for (int k = 0; k < 4; ++k) {
-            const int ch = 4 * i + k;
-            const uint4 w = *reinterpret_cast<const uint4 *>(rs + h * 4096 + lane * 128 + ((ch ^ (lane & 7)) << 4));
-            v[4 * k] = w.x;
-            v[4 * k + 1] = w.y;
-            v[4 * k + 2] = w.z;
-            v[4 * k + 3] = w.w;
-          }
-          tc::st16(tk + i * 16, v);
-        }
-        // V half h: the piece's swizzle matches the tile's (row ct = 32 wq + lane)
-#pragma unroll
-        for (int ch = 0; ch < 8; ++ch)
-          *reinterpret_cast<uint4 *>(cv + kCvtV + h * 16384 + ct * 128 + ch * 16) =
-              *reinterpret_cast<const uint4 *>(rs + 8192 + h * 4096 + lane * 128 + ch * 16);
-        if (h == 0)
-          *reinterpret_cast<float4 *>(cv + kCvtMisc + ct * 16) = make_float4(1.f, 0.f, 1.f, 0.f);
-        else if (first && wq == 0)
-          stage_queries(rs + kRawQ, qdst, qsum, lane, false);
-        mbar_arrive_n(bar(kBarRawEmpty + s), 4);  // the piece's only readers: 64 threads x 4
-        r += 4;
+      for (int i = 0; i < 4; ++i) {
+        const int off = ct * 64 + ((i ^ rot) << 4);
+        const uint4 kw = *reinterpret_cast<const uint4 *>(st + kStKc + off);
+        const uint4 vw = *reinterpret_cast<const uint4 *>(st + kStVc + off);
+        lk[4 * i] = kw.x & 0x0F0F0F0Fu;
+        lk[4 * i + 1] = kw.y & 0x0F0F0F0Fu;
+        lk[4 * i + 2] = kw.z & 0x0F0F0F0Fu;
+        lk[4 * i + 3] = kw.w & 0x0F0F0F0Fu;
+        *reinterpret_cast<uint4 *>(st + kStLv + off) =
+            make_uint4(vw.x & 0x0F0F0F0Fu, vw.y & 0x0F0F0F0Fu, vw.z & 0x0F0F0F0Fu, vw.w & 0x0F0F0F0Fu);
       }
-      tc::fence_async_smem();
+      tc::st16(tm_lane + C::kLk + s * 16, lk);  // K low nibbles: TMEM lane ct, bytes in order
+      // rows past len (the tail of the last tile) get zero scales: they then add nothing,
+      // and do not enter the tile's largest s_v
+      const bool tvalid = static_cast<int64_t>(un.tile) * kTile + ct < p.len;
+      const uint32_t ksz = tvalid ? *reinterpret_cast<const uint32_t *>(st + kStKsz + ct * 4) : 0u;
+      const uint32_t vsz = tvalid ? *reinterpret_cast<const uint32_t *>(st + kStVsz + ct * 4) : 0u;
+      const float vs = __half2float(__ushort_as_half(static_cast<unsigned short>(vsz & 0xffffu)));
+      *reinterpret_cast<float4 *>(st + kStMisc + ct * 16) =
+          make_float4(__half2float(__ushort_as_half(static_cast<unsigned short>(ksz & 0xffffu))),
+                      __half2float(__ushort_as_half(static_cast<unsigned short>(ksz >> 16))), vs,
+                      __half2float(__ushort_as_half(static_cast<unsigned short>(vsz >> 16))));
+      const float vmax = warp_max(vs);
+      if (lane == 0) reinterpret_cast<float *>(st + kStTmax)[wq] = vmax;
+      if (first && warp == 6) {
+        // the item's query limbs replace those of the item two before, once its last
+        // S^T product has run and the softmax has read its sigma and sum(q)
+        if (nitem >= 2 && !tc::wait_bar(bar(kBarQFree + (nitem & 1)), ((nitem - 2) >> 1) & 1, p.status, abort_flag))
+          break;
+        prep_queries(st + kStQ, smem + kSmQl + (nitem & 1) * kQlBytes,
+                     reinterpret_cast<float *>(smem + kSmQinfo) + (nitem & 1) * 32, G, lane);
+      }
       tc::st_wait();
+      tc::fence_async_smem();  // the low nibbles and query limbs are MMA operands
       tc::fence_before();
-      mbar_arrive(bar(kBarCvtFull + cb));
+      mbar_arrive(bar(kBarCvt + s));
     }
   }
 
   tc::fence_before();
   __syncthreads();
   tc::fence_after();
-  if (warp == 1) tc::tmem_free(tmem, kTmemCols);
+  if (warp == 1) tc::tmem_free(tmem, C::kAlloc);
 }
 
 template <int NQ>
@@ -732,50 +688,34 @@ cudaError_t launch_nq(const Int4DecodeArgs &a, bool overlap_previous, cudaStream
 }  // namespace
 
 bool decode_int4_tc_supported(const DecodeParams &p, duo_dtype dt) {
-  return dt == DUO_BF16 && p.D == kD && p.G >= 1 && p.G <= kN && tc::encode_fn() != nullptr;
+  return dt == DUO_BF16 && p.D == kD && p.G >= 1 && p.G <= 16 && tc::encode_fn() != nullptr;
 }
 
 cudaError_t launch_decode_int4_tc(const DecodeParams &p, int num_sms, bool overlap_previous, cudaStream_t st) {
+  if (p.Hr < 1 || p.len < 1) return cudaSuccess;  // no retrieval head: nothing to do here
   Int4DecodeArgs a{};
   a.p = p;
   a.units_r = static_cast<int>((p.len + kTile - 1) / kTile);
-  const int64_t slots = static_cast<int64_t>(p.S) + p.W;
-  // highest ring slot in use + 1: position p >= S sits in slot S + p mod W, so before the
-  // ring wraps (len <= W) the slots reach S + len - 1, beyond len itself
-  const int64_t reach = static_cast<int64_t>(p.S) + p.len;
-  const int64_t used = reach < slots ? reach : slots;
-  a.units_s = static_cast<int>((used + kTile - 1) / kTile);
-  a.n_items_r = p.B * p.Hr;
-  a.ur = static_cast<int64_t>(a.n_items_r) * a.units_r;
-  const int64_t us = static_cast<int64_t>(p.B) * p.Hs * a.units_s;
-  a.total_units = a.ur + us;
-  a.total_cost = a.ur + kWs * us;
+  a.n_items = p.B * p.Hr;
+  a.total_units = static_cast<int64_t>(a.n_items) * a.units_r;
   // at most one CTA per SM, and never more segments per item than partial slots
   int64_t ctas = num_sms;
-  if (ctas > a.ur + us) ctas = a.ur + us;
+  if (ctas > a.total_units) ctas = a.total_units;
   if (ctas > kMaxSplits) ctas = kMaxSplits;
   a.num_ctas = static_cast<int>(ctas);
   bool ok = true;
   {  // queries [B*Hq][d]
     const uint64_t d[2] = {kD, static_cast<uint64_t>(p.B) * p.Hq};
     const uint64_t s[1] = {kD * 2};
-    const uint32_t bx[2] = {64, kN};
+    const uint32_t bx[2] = {64, 16};
     ok &= tc::make_map(&a.tm_q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, p.q, 2, d, s, bx, CU_TENSOR_MAP_SWIZZLE_128B);
   }
   {  // retrieval codes [B*Hr][cap][64 B]
-    const uint64_t rows = static_cast<uint64_t>(p.B) * (p.Hr > 0 ? p.Hr : 1);
-    const uint64_t d[3] = {kD / 2, static_cast<uint64_t>(p.max_len), rows};
+    const uint64_t d[3] = {kD / 2, static_cast<uint64_t>(p.max_len), static_cast<uint64_t>(a.n_items)};
     const uint64_t s[2] = {kD / 2, static_cast<uint64_t>(kD / 2) * p.max_len};
     const uint32_t bx[3] = {kD / 2, kTile, 1};
     ok &= tc::make_map(&a.tm_kc, CU_TENSOR_MAP_DATA_TYPE_UINT8, p.rk, 3, d, s, bx, CU_TENSOR_MAP_SWIZZLE_64B);
     ok &= tc::make_map(&a.tm_vc, CU_TENSOR_MAP_DATA_TYPE_UINT8, p.rv, 3, d, s, bx, CU_TENSOR_MAP_SWIZZLE_64B);
-  }
-  {  // streaming [B*Hs][S+W][d] bf16, pieces of 32 rows
-    const uint64_t d[3] = {kD, static_cast<uint64_t>(slots), static_cast<uint64_t>(p.B) * (p.Hs > 0 ? p.Hs : 1)};
-    const uint64_t s[2] = {kD * 2, static_cast<uint64_t>(kD * 2) * slots};
-    const uint32_t bx[3] = {64, 32, 1};
-    ok &= tc::make_map(&a.tm_ks, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, p.sk, 3, d, s, bx, CU_TENSOR_MAP_SWIZZLE_128B);
-    ok &= tc::make_map(&a.tm_vs, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, p.sv, 3, d, s, bx, CU_TENSOR_MAP_SWIZZLE_128B);
   }
   if (!ok) return cudaErrorInvalidValue;
   if (p.G <= 1) return launch_nq<1>(a, overlap_previous, st);

@@ -400,7 +400,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
           bulk_g2s(sbase, part, bytes, bar(kBarMerge));
         }
         if (ok) ok = tc::wait_bar(bar(kBarMerge), 0, p.status, abort_flag);
-        merge_partials_smem(reinterpret_cast<float *>(smem), nseg, G, b, h0, p.Hq, p.out, p.lse, red + 4 * kN, t, 1);
+        merge_partials<true>(reinterpret_cast<const float *>(smem), nseg, G, b, h0, p.Hq, p.out, p.lse, red + 4 * kN, t, 1);
       } else {
         merge_partials(part, nseg, G, b, h0, p.Hq, p.out, p.lse, red + 4 * kN, t, 1);
       }
