@@ -21,12 +21,13 @@
 // and recombined in fp32 by exact magic-number adds (no conversion instructions).  Per token the scale and zero then give
 //   q . k_t = s_t (q . c_t) + z_t sum(q),   sum_t p_t v_t = sum_t p'_t c_t + sum_t p_t z_t.
 //
-// Roles of a CTA (one per SM, 320 threads):
+// Roles of a CTA (one per SM, 352 threads):
 //   warp 0     TMA producer: per 128-token tile the K and V code rows (64 B each,
 //              64-byte swizzle) and their scale/zero rows, at an item's first tile the
 //              group's bf16 queries; a ring of kStages stages.
-//   warp 1     MMA issuer and TMEM owner (4 MMAs for S^T and 4 for O^T per tile; the
-//              K low nibbles are read from tensor memory).
+//   warp 1     S^T issuer (4 MMAs per tile; the K low nibbles are read from tensor
+//              memory) and TMEM owner.
+//   warp 10    O^T issuer (4 MMAs per tile).
 //   warps 2-5  softmax: thread t owns token t of S^T and row t of O^T.
 //   warps 6-9  prep: a thread writes the low nibbles of token t's K row into TMEM lane
 //              t and those of its V row beside the V codes, and the token's {s_k, z_k,
@@ -42,7 +43,7 @@ namespace duo {
 
 namespace {
 
-constexpr int kThreads = 320;
+constexpr int kThreads = 352;
 constexpr int kTile = 128;
 constexpr int kD = 128;
 constexpr int kStages = 6;
@@ -67,7 +68,7 @@ static_assert(kSmemAlloc <= 232448, "shared memory");
 
 constexpr int kBarFull = 0, kBarEmpty = kStages, kBarCvt = 2 * kStages, kBarSFull = 3 * kStages,
               kBarSFree = kBarSFull + 2, kBarPFull = kBarSFull + 4, kBarOFull = kBarSFull + 6,
-              kBarQFree = kBarSFull + 8, kBarDrain = kBarSFull + 10, kNumBars = kBarSFull + 11;
+              kBarQFree = kBarSFull + 8, kBarDrain = kBarSFull + 10, kNumBars = kBarSFull + 12;
 static_assert(kNumBars * 8 <= 256, "barrier area");
 
 // tensor memory columns: S^T (three limbs per query head) x 2, O^T (two limbs) x 2, and
@@ -241,6 +242,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_int4_kernel(const __grid_c
       mbar_init(bar(kBarQFree + i), 2);  // the item's last S^T product (commit) + the softmax
     }
     mbar_init(bar(kBarDrain), 1);
+    mbar_init(bar(kBarDrain + 1), 1);
     fence_mbar_init();
     *abort_flag = 0;
   }
@@ -298,79 +300,61 @@ __global__ void __launch_bounds__(kThreads, 1) decode_int4_kernel(const __grid_c
       }
     }
   } else if (warp == 1) {
-    // ================= MMA issuer =================
-    // Event-driven: S^T(js) as soon as its prep is done and its S buffer is free, O^T(jo)
-    // as soon as the softmax has written P'(jo), whichever comes first.
+    // ================= S^T issuer =================
+    // Each tile's S^T once its prep is done and its S buffer is free.  The two products
+    // have issuers of their own (warps 1 and 10): a single thread that issued both had to
+    // watch two barriers at once and, blocked in one product's issue or asleep on the
+    // other's barrier, held up the next tile by a few hundred cycles.
     if (lane == 0) {
-      constexpr uint32_t kIdS = idesc_i8(128, C::kS, true, false);   // [U | L] . Qx^T
-      constexpr uint32_t kIdO = idesc_i8(128, C::kO, true, true);    // [U_V | L_V]^T . P'^T
-      int js = 0, jo = 0, nitem = -1, prev_item = -1;
+      constexpr uint32_t kIdS = idesc_i8(128, C::kS, true, false);  // [U | L] . Qx^T
+      int nitem = -1, prev_item = -1;
       UnitIter its(a, u0);
-      uint32_t idle = 0;
-      unsigned long long t_idle = 0;
-      while (jo < nu) {
-        bool did = false;
-        if (js < nu) {
-          const int s = js % kStages;
-          if (mbar_test_wait(bar(kBarCvt + s), (js / kStages) & 1) &&
-              (js < 2 || mbar_test_wait(bar(kBarSFree + (js & 1)), ((js - 2) >> 1) & 1))) {
-            const int item = its.un.item;
-            its.next();
-            if (item != prev_item) {
-              prev_item = item;
-              ++nitem;
-            }
-            tc::fence_after();
-            const uint64_t ak = sdesc_l(sbase + s * kStage + kStKc, 16, 512, 4);
-            const uint32_t al = tmem + C::kLk + s * 16;
-            const uint64_t bq = sdesc_l(sbase + kSmQl + (nitem & 1) * kQlBytes, 16, 1024, 2);
-            const uint32_t d = tmem + (js & 1) * C::kS;
-            mma_i8(d, ak, bq, kIdS, 0u);             // bytes 0..31 of the code rows
-            mma_i8(d, ak + 2, bq + 2, kIdS, 1u);     // bytes 32..63
-            mma_i8_ts(d, al, bq + 4, kIdS, 1u);      // low nibbles 0..31 (TMEM)
-            mma_i8_ts(d, al + 8, bq + 6, kIdS, 1u);  // low nibbles 32..63
-            tc::commit(bar(kBarSFull + (js & 1)));
-            ++js;
-            // the item's query limbs are free once its last S^T product has run
-            if (js == nu || its.un.item != item) tc::commit(bar(kBarQFree + (nitem & 1)));
-            did = true;
-          }
+      for (int js = 0; js < nu; ++js) {
+        const int s = js % kStages;
+        if (!tc::wait_bar(bar(kBarCvt + s), (js / kStages) & 1, p.status, abort_flag)) break;
+        if (js >= 2 && !tc::wait_bar(bar(kBarSFree + (js & 1)), ((js - 2) >> 1) & 1, p.status, abort_flag)) break;
+        const int item = its.un.item;
+        its.next();
+        if (item != prev_item) {
+          prev_item = item;
+          ++nitem;
         }
-        if (jo < js && mbar_test_wait(bar(kBarPFull + (jo & 1)), (jo >> 1) & 1)) {
-          tc::fence_after();
-          const int s = jo % kStages;
-          const uint64_t av = sdesc_l(sbase + s * kStage + kStVc, kStLv - kStVc, 512, 4);  // MN-major, 2 chunks
-          const uint64_t bp = sdesc_l(sbase + kSmP + (jo & 1) * 4096, 16, 1024, 2);
-          const uint32_t d = tmem + 2 * C::kS + (jo & 1) * C::kO;
-#pragma unroll
-          for (int k = 0; k < 4; ++k)  // 32 tokens per step
-            mma_i8(d, av + k * (2048 >> 4), bp + k * 2, kIdO, k > 0 ? 1u : 0u);
-          tc::commit(bar(kBarOFull + (jo & 1)));
-          tc::commit(bar(kBarEmpty + s));  // the stage and its K low nibbles are no longer read
-          ++jo;
-          did = true;
-        }
-        if (did) {
-          idle = 0;
-        } else {
-          // sleep on the event expected next rather than spin beside the other warps
-          if (jo < js)
-            mbar_try_wait_ns(bar(kBarPFull + (jo & 1)), (jo >> 1) & 1, 100);
-          else
-            mbar_try_wait_ns(bar(kBarCvt + js % kStages), (js / kStages) & 1, 100);
-          if (++idle == 1) t_idle = globaltimer();
-        }
-        if (idle > 0 && (idle & 63) == 0) {
-          if (*abort_flag) break;
-          if (globaltimer() - t_idle > kWaitLimitNs) {
-            flag_status(p.status, kDevTimeout);
-            *abort_flag = 1;
-            break;
-          }
-        }
+        tc::fence_after();
+        const uint64_t ak = sdesc_l(sbase + s * kStage + kStKc, 16, 512, 4);
+        const uint32_t al = tmem + C::kLk + s * 16;
+        const uint64_t bq = sdesc_l(sbase + kSmQl + (nitem & 1) * kQlBytes, 16, 1024, 2);
+        const uint32_t d = tmem + (js & 1) * C::kS;
+        mma_i8(d, ak, bq, kIdS, 0u);             // bytes 0..31 of the code rows
+        mma_i8(d, ak + 2, bq + 2, kIdS, 1u);     // bytes 32..63
+        mma_i8_ts(d, al, bq + 4, kIdS, 1u);      // low nibbles 0..31 (TMEM)
+        mma_i8_ts(d, al + 8, bq + 6, kIdS, 1u);  // low nibbles 32..63
+        tc::commit(bar(kBarSFull + (js & 1)));
+        // the item's query limbs are free once its last S^T product has run
+        if (js + 1 == nu || its.un.item != item) tc::commit(bar(kBarQFree + (nitem & 1)));
       }
       tc::commit(bar(kBarDrain));
       mbar_wait(bar(kBarDrain), 0, p.status);
+    }
+  } else if (warp == 10) {
+    // ================= O^T issuer =================
+    // Each tile's O^T once the softmax has written its P'; then the stage is released.
+    if (lane == 0) {
+      constexpr uint32_t kIdO = idesc_i8(128, C::kO, true, true);  // [U_V | L_V]^T . P'^T
+      for (int jo = 0; jo < nu; ++jo) {
+        if (!tc::wait_bar(bar(kBarPFull + (jo & 1)), (jo >> 1) & 1, p.status, abort_flag)) break;
+        tc::fence_after();
+        const int s = jo % kStages;
+        const uint64_t av = sdesc_l(sbase + s * kStage + kStVc, kStLv - kStVc, 512, 4);  // MN-major, 2 chunks
+        const uint64_t bp = sdesc_l(sbase + kSmP + (jo & 1) * 4096, 16, 1024, 2);
+        const uint32_t d = tmem + 2 * C::kS + (jo & 1) * C::kO;
+#pragma unroll
+        for (int k = 0; k < 4; ++k)  // 32 tokens per step
+          mma_i8(d, av + k * (2048 >> 4), bp + k * 2, kIdO, k > 0 ? 1u : 0u);
+        tc::commit(bar(kBarOFull + (jo & 1)));
+        tc::commit(bar(kBarEmpty + s));  // the stage and its K low nibbles are no longer read
+      }
+      tc::commit(bar(kBarDrain + 1));
+      mbar_wait(bar(kBarDrain + 1), 0, p.status);
     }
   } else if (warp < 6) {
     // ================= softmax warpgroup =================
@@ -595,7 +579,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_int4_kernel(const __grid_c
       if (pending) fold(nu - 1, sigp_prev, one);
       flush(cur_item);
     }
-  } else {
+  } else if (warp < 10) {
     // ================= prep warps =================
     const int wq = warp & 3;
     const int ct = (wq << 5) | lane;  // token row of the tile
@@ -633,13 +617,13 @@ __global__ void __launch_bounds__(kThreads, 1) decode_int4_kernel(const __grid_c
       const bool tvalid = static_cast<int64_t>(un.tile) * kTile + ct < p.len;
       const uint32_t ksz = tvalid ? *reinterpret_cast<const uint32_t *>(st + kStKsz + ct * 4) : 0u;
       const uint32_t vsz = tvalid ? *reinterpret_cast<const uint32_t *>(st + kStVsz + ct * 4) : 0u;
-      const float vs = __half2float(__ushort_as_half(static_cast<unsigned short>(vsz & 0xffffu)));
-      *reinterpret_cast<float4 *>(st + kStMisc + ct * 16) =
-          make_float4(__half2float(__ushort_as_half(static_cast<unsigned short>(ksz & 0xffffu))),
-                      __half2float(__ushort_as_half(static_cast<unsigned short>(ksz >> 16))), vs,
-                      __half2float(__ushort_as_half(static_cast<unsigned short>(vsz >> 16))));
-      const float vmax = warp_max(vs);
-      if (lane == 0) reinterpret_cast<float *>(st + kStTmax)[wq] = vmax;
+      const float2 kf = __half22float2(*reinterpret_cast<const __half2 *>(&ksz));
+      const float2 vf = __half22float2(*reinterpret_cast<const __half2 *>(&vsz));
+      *reinterpret_cast<float4 *>(st + kStMisc + ct * 16) = make_float4(kf.x, kf.y, vf.x, vf.y);
+      // the warp's largest s_v in one step: fp16 bits of non-negative values order as the values
+      const uint32_t vmax = __reduce_max_sync(0xffffffffu, vsz & 0xffffu);
+      if (lane == 0)
+        reinterpret_cast<float *>(st + kStTmax)[wq] = __half2float(__ushort_as_half(static_cast<unsigned short>(vmax)));
       if (first && warp == 6) {
         // the item's query limbs replace those of the item two before, once its last
         // S^T product has run and the softmax has read its sigma and sum(q)
