@@ -141,11 +141,14 @@ class ClockSampler:
                 "samples": len(sm)}
 
 
-def kernel_hash():
-    """Hash of the decode kernels' sources: recorded DRAM traffic is void once they change."""
+def kernel_hash(workload):
+    """Hash of the sources of the decode kernels a workload runs: recorded DRAM traffic
+    is void once they change."""
+    files = ["k_decode_tc.cu", "tcgen05.cuh", "decode_merge.cuh", "device_common.cuh", "duo_internal.h"]
+    if "int4" in workload:
+        files.append("k_decode_int4_tc.cu")
     h = hashlib.sha256()
-    for f in ("k_decode.cu", "k_decode_tc.cu", "k_decode_int4_tc.cu", "tcgen05.cuh", "decode_merge.cuh",
-              "device_common.cuh", "duo_internal.h"):
+    for f in files:
         h.update(open(os.path.join(ROOT, "head_split_kv_duo_b200", "csrc", f), "rb").read())
     return h.hexdigest()[:16]
 
@@ -157,7 +160,7 @@ def recorded_traffic(workload):
     if not os.path.exists(path):
         return None
     rec = json.load(open(path)).get(workload)
-    if not rec or rec.get("kernel_hash") != kernel_hash():
+    if not rec or rec.get("kernel_hash") != kernel_hash(workload):
         return None
     return rec.get("dram_bytes_per_launch")
 

@@ -21,17 +21,19 @@
 // and recombined in fp32 by exact magic-number adds (no conversion instructions).  Per token the scale and zero then give
 //   q . k_t = s_t (q . c_t) + z_t sum(q),   sum_t p_t v_t = sum_t p'_t c_t + sum_t p_t z_t.
 //
-// Roles of a CTA (one per SM, 352 threads):
+// Roles of a CTA (one per SM, 448 threads):
 //   warp 0     TMA producer: per 128-token tile the K and V code rows (64 B each,
 //              64-byte swizzle) and their scale/zero rows, at an item's first tile the
 //              group's bf16 queries; a ring of kStages stages.
-//   warp 1     S^T issuer (4 MMAs per tile; the K low nibbles are read from tensor
-//              memory) and TMEM owner.
-//   warp 10    O^T issuer (4 MMAs per tile).
-//   warps 2-5  softmax: thread t owns token t of S^T and row t of O^T.
-//   warps 6-9  prep: a thread writes the low nibbles of token t's K row into TMEM lane
+//   warp 1     MMA issuer and TMEM owner (4 MMAs for S^T and 4 for O^T per tile; the
+//              K low nibbles are read from tensor memory).
+//   warps 2-9  softmax, two warpgroups taking alternate tiles (each with its own running
+//              max and sums, combined when an item ends), so that the dependent chain
+//              of one tile overlaps the next: thread t owns token t of S^T and row t of
+//              O^T.
+//   warps 10-13 prep: a thread writes the low nibbles of token t's K row into TMEM lane
 //              t and those of its V row beside the V codes, and the token's {s_k, z_k,
-//              s_v, z_v}; warp 6 also turns an item's queries into limbs.
+//              s_v, z_v}; warp 10 also turns an item's queries into limbs.
 //
 // Work balance: every (batch, retrieval head) is an item of 128-token tiles; the tiles
 // of all items are laid end to end and cut into one equal range per CTA.  Split partials
@@ -43,7 +45,7 @@ namespace duo {
 
 namespace {
 
-constexpr int kThreads = 352;
+constexpr int kThreads = 448;
 constexpr int kTile = 128;
 constexpr int kD = 128;
 constexpr int kStages = 6;
@@ -56,28 +58,31 @@ constexpr int kStKc = 0, kStVc = 8192, kStLv = 16384, kStKsz = 24576, kStVsz = 2
               kStTmax = 27648, kStQ = 28672, kStage = 32768;
 constexpr int kQlBytes = 6144;                 // query limbs [48][128 B] s8, 128-byte swizzle
 constexpr int kSmQl = kStages * kStage;        // 2 x query limbs (item parity)
-constexpr int kSmP = kSmQl + 2 * kQlBytes;     // 2 x P' limbs [32][128 B] u8; flush exchange
-constexpr int kSmQinfo = kSmP + 8192;          // [2][32]: sigma[16], sum(q)[16] per query head
-constexpr int kSmRed = kSmQinfo + 256;         // [4][16] l, [4][16] zc, [128][6] merge
-constexpr int kSmBar = kSmRed + (2 * 4 * 16 + 128 * 6) * 4;
-constexpr int kSmMisc = kSmBar + 256;
+constexpr int kSmP = kSmQl + 2 * kQlBytes;     // 4 x P' limbs [32][128 B] s8; flush exchanges
+constexpr int kSmQinfo = kSmP + 4 * 4096;      // [2][32]: sigma[16], sum(q)[16] per query head
+constexpr int kSmRed = kSmQinfo + 256;         // per softmax group [4][16] l, [4][16] zc; [128][6] merge
+constexpr int kSmBar = kSmRed + (2 * 128 + 128 * 6) * 4;
+constexpr int kSmMisc = kSmBar + 512;
 constexpr int kSmemAlloc = kSmMisc + 64 + 1024;
 static_assert(kStage % 1024 == 0 && kStQ % 1024 == 0 && kSmQl % 1024 == 0 && kSmP % 1024 == 0 &&
                   kQlBytes % 1024 == 0, "alignment");
 static_assert(kSmemAlloc <= 232448, "shared memory");
 
+// P' and O^T have four buffers each, and so four barriers: with two groups a group
+// publishes P'(j + 2) before the issuer need have taken P'(j), so a barrier per
+// buffer pair would complete a second phase ahead of its waiter
 constexpr int kBarFull = 0, kBarEmpty = kStages, kBarCvt = 2 * kStages, kBarSFull = 3 * kStages,
-              kBarSFree = kBarSFull + 2, kBarPFull = kBarSFull + 4, kBarOFull = kBarSFull + 6,
-              kBarQFree = kBarSFull + 8, kBarDrain = kBarSFull + 10, kNumBars = kBarSFull + 12;
-static_assert(kNumBars * 8 <= 256, "barrier area");
+              kBarSFree = kBarSFull + 2, kBarPFull = kBarSFull + 4, kBarOFull = kBarSFull + 8,
+              kBarQFree = kBarSFull + 12, kBarDrain = kBarSFull + 14, kNumBars = kBarSFull + 15;
+static_assert(kNumBars * 8 <= 512, "barrier area");
 
-// tensor memory columns: S^T (three limbs per query head) x 2, O^T (two limbs) x 2, and
+// tensor memory columns: S^T (three limbs per query head) x 2, O^T (two limbs) x 4, and
 // per stage the K low nibbles (16 columns: 4 bytes each)
 template <int NQ>
 struct Cols {
   static constexpr int kS = (3 * NQ + 15) / 16 * 16;
   static constexpr int kO = (2 * NQ + 15) / 16 * 16;
-  static constexpr int kLk = 2 * kS + 2 * kO;
+  static constexpr int kLk = 2 * kS + 4 * kO;
   static constexpr int kUsed = kLk + kStages * 16;
   static constexpr int kAlloc = kUsed <= 128 ? 128 : kUsed <= 256 ? 256 : 512;
 };
@@ -237,12 +242,13 @@ __global__ void __launch_bounds__(kThreads, 1) decode_int4_kernel(const __grid_c
     for (int i = 0; i < 2; ++i) {
       mbar_init(bar(kBarSFull + i), 1);
       mbar_init(bar(kBarSFree + i), 128);
+      mbar_init(bar(kBarQFree + i), 3);  // the item's last S^T product (commit) + each softmax group
+    }
+    for (int i = 0; i < 4; ++i) {
       mbar_init(bar(kBarPFull + i), 128);
       mbar_init(bar(kBarOFull + i), 1);
-      mbar_init(bar(kBarQFree + i), 2);  // the item's last S^T product (commit) + the softmax
     }
     mbar_init(bar(kBarDrain), 1);
-    mbar_init(bar(kBarDrain + 1), 1);
     fence_mbar_init();
     *abort_flag = 0;
   }
@@ -300,70 +306,92 @@ __global__ void __launch_bounds__(kThreads, 1) decode_int4_kernel(const __grid_c
       }
     }
   } else if (warp == 1) {
-    // ================= S^T issuer =================
-    // Each tile's S^T once its prep is done and its S buffer is free.  The two products
-    // have issuers of their own (warps 1 and 10): a single thread that issued both had to
-    // watch two barriers at once and, blocked in one product's issue or asleep on the
-    // other's barrier, held up the next tile by a few hundred cycles.
+    // ================= MMA issuer =================
+    // Event-driven: S^T(js) as soon as its prep is done and its S buffer is free, O^T(jo)
+    // as soon as the softmax has written P'(jo), whichever comes first.
     if (lane == 0) {
-      constexpr uint32_t kIdS = idesc_i8(128, C::kS, true, false);  // [U | L] . Qx^T
-      int nitem = -1, prev_item = -1;
+      constexpr uint32_t kIdS = idesc_i8(128, C::kS, true, false);   // [U | L] . Qx^T
+      constexpr uint32_t kIdO = idesc_i8(128, C::kO, true, true);    // [U_V | L_V]^T . P'^T
+      int js = 0, jo = 0, nitem = -1, prev_item = -1;
       UnitIter its(a, u0);
-      for (int js = 0; js < nu; ++js) {
-        const int s = js % kStages;
-        if (!tc::wait_bar(bar(kBarCvt + s), (js / kStages) & 1, p.status, abort_flag)) break;
-        if (js >= 2 && !tc::wait_bar(bar(kBarSFree + (js & 1)), ((js - 2) >> 1) & 1, p.status, abort_flag)) break;
-        const int item = its.un.item;
-        its.next();
-        if (item != prev_item) {
-          prev_item = item;
-          ++nitem;
+      uint32_t idle = 0;
+      unsigned long long t_idle = 0;
+      while (jo < nu) {
+        bool did = false;
+        if (js < nu) {
+          const int s = js % kStages;
+          if (mbar_test_wait(bar(kBarCvt + s), (js / kStages) & 1) &&
+              (js < 2 || mbar_test_wait(bar(kBarSFree + (js & 1)), ((js - 2) >> 1) & 1))) {
+            const int item = its.un.item;
+            its.next();
+            if (item != prev_item) {
+              prev_item = item;
+              ++nitem;
+            }
+            tc::fence_after();
+            const uint64_t ak = sdesc_l(sbase + s * kStage + kStKc, 16, 512, 4);
+            const uint32_t al = tmem + C::kLk + s * 16;
+            const uint64_t bq = sdesc_l(sbase + kSmQl + (nitem & 1) * kQlBytes, 16, 1024, 2);
+            const uint32_t d = tmem + (js & 1) * C::kS;
+            mma_i8(d, ak, bq, kIdS, 0u);             // bytes 0..31 of the code rows
+            mma_i8(d, ak + 2, bq + 2, kIdS, 1u);     // bytes 32..63
+            mma_i8_ts(d, al, bq + 4, kIdS, 1u);      // low nibbles 0..31 (TMEM)
+            mma_i8_ts(d, al + 8, bq + 6, kIdS, 1u);  // low nibbles 32..63
+            tc::commit(bar(kBarSFull + (js & 1)));
+            ++js;
+            // the item's query limbs are free once its last S^T product has run
+            if (js == nu || its.un.item != item) tc::commit(bar(kBarQFree + (nitem & 1)));
+            did = true;
+          }
         }
-        tc::fence_after();
-        const uint64_t ak = sdesc_l(sbase + s * kStage + kStKc, 16, 512, 4);
-        const uint32_t al = tmem + C::kLk + s * 16;
-        const uint64_t bq = sdesc_l(sbase + kSmQl + (nitem & 1) * kQlBytes, 16, 1024, 2);
-        const uint32_t d = tmem + (js & 1) * C::kS;
-        mma_i8(d, ak, bq, kIdS, 0u);             // bytes 0..31 of the code rows
-        mma_i8(d, ak + 2, bq + 2, kIdS, 1u);     // bytes 32..63
-        mma_i8_ts(d, al, bq + 4, kIdS, 1u);      // low nibbles 0..31 (TMEM)
-        mma_i8_ts(d, al + 8, bq + 6, kIdS, 1u);  // low nibbles 32..63
-        tc::commit(bar(kBarSFull + (js & 1)));
-        // the item's query limbs are free once its last S^T product has run
-        if (js + 1 == nu || its.un.item != item) tc::commit(bar(kBarQFree + (nitem & 1)));
+        if (jo < js && mbar_test_wait(bar(kBarPFull + (jo & 3)), (jo >> 2) & 1)) {
+          tc::fence_after();
+          const int s = jo % kStages;
+          const uint64_t av = sdesc_l(sbase + s * kStage + kStVc, kStLv - kStVc, 512, 4);  // MN-major, 2 chunks
+          const uint64_t bp = sdesc_l(sbase + kSmP + (jo & 3) * 4096, 16, 1024, 2);
+          const uint32_t d = tmem + 2 * C::kS + (jo & 3) * C::kO;
+#pragma unroll
+          for (int k = 0; k < 4; ++k)  // 32 tokens per step
+            mma_i8(d, av + k * (2048 >> 4), bp + k * 2, kIdO, k > 0 ? 1u : 0u);
+          tc::commit(bar(kBarOFull + (jo & 3)));
+          tc::commit(bar(kBarEmpty + s));  // the stage and its K low nibbles are no longer read
+          ++jo;
+          did = true;
+        }
+        if (did) {
+          idle = 0;
+        } else {
+          // sleep on the event expected next rather than spin beside the other warps
+          if (jo < js)
+            mbar_try_wait_ns(bar(kBarPFull + (jo & 3)), (jo >> 2) & 1, 100);
+          else
+            mbar_try_wait_ns(bar(kBarCvt + js % kStages), (js / kStages) & 1, 100);
+          if (++idle == 1) t_idle = globaltimer();
+        }
+        if (idle > 0 && (idle & 63) == 0) {
+          if (*abort_flag) break;
+          if (globaltimer() - t_idle > kWaitLimitNs) {
+            flag_status(p.status, kDevTimeout);
+            *abort_flag = 1;
+            break;
+          }
+        }
       }
       tc::commit(bar(kBarDrain));
       mbar_wait(bar(kBarDrain), 0, p.status);
     }
-  } else if (warp == 10) {
-    // ================= O^T issuer =================
-    // Each tile's O^T once the softmax has written its P'; then the stage is released.
-    if (lane == 0) {
-      constexpr uint32_t kIdO = idesc_i8(128, C::kO, true, true);  // [U_V | L_V]^T . P'^T
-      for (int jo = 0; jo < nu; ++jo) {
-        if (!tc::wait_bar(bar(kBarPFull + (jo & 1)), (jo >> 1) & 1, p.status, abort_flag)) break;
-        tc::fence_after();
-        const int s = jo % kStages;
-        const uint64_t av = sdesc_l(sbase + s * kStage + kStVc, kStLv - kStVc, 512, 4);  // MN-major, 2 chunks
-        const uint64_t bp = sdesc_l(sbase + kSmP + (jo & 1) * 4096, 16, 1024, 2);
-        const uint32_t d = tmem + 2 * C::kS + (jo & 1) * C::kO;
-#pragma unroll
-        for (int k = 0; k < 4; ++k)  // 32 tokens per step
-          mma_i8(d, av + k * (2048 >> 4), bp + k * 2, kIdO, k > 0 ? 1u : 0u);
-        tc::commit(bar(kBarOFull + (jo & 1)));
-        tc::commit(bar(kBarEmpty + s));  // the stage and its K low nibbles are no longer read
-      }
-      tc::commit(bar(kBarDrain + 1));
-      mbar_wait(bar(kBarDrain + 1), 0, p.status);
-    }
-  } else if (warp < 6) {
-    // ================= softmax warpgroup =================
-    // Exact running max (p <= 1, which bounds the P' limbs); s = s_k (q . c) + z_k sum(q);
-    // the MMA gets P' = p s_v as two signed limbs below the tile's largest s_v; zc
-    // accumulates p z_v.
+  } else if (warp < 10) {
+    // ================= softmax warpgroups =================
+    // Group g takes the tiles j with j % 2 == g.  Exact running max (p <= 1, which bounds
+    // the P' limbs); s = s_k (q . c) + z_k sum(q); the MMA gets P' = p s_v as two signed
+    // limbs below the tile's largest s_v; zc accumulates p z_v.  When an item ends the two
+    // groups' states are combined (group 0 writes the result).
+    const int grp = (warp - 2) >> 2;
+    const int gbar = 1 + grp;  // the group's named barrier; barrier 3 joins both groups
     const int wq = warp & 3;
     const int t = (wq << 5) | lane;
     const uint32_t lane_base = tmem + (static_cast<uint32_t>(wq << 5) << 16);
+    float *gred = red + grp * 128;  // [4 warps][16] l (or maxima), [4][16] zc
     const float c = p.scale_log2;
     float m[NQ], l[NQ], zc[NQ], o[NQ], sg[NQ], qs[NQ];
 #pragma unroll
@@ -375,40 +403,73 @@ __global__ void __launch_bounds__(kThreads, 1) decode_int4_kernel(const __grid_c
       sg[q] = 0.f;
       qs[q] = 0.f;
     }
-    bool ok = true;
+    bool ok = true, qread = true;  // qread: this group has read (or released) the item's sigma, sum(q)
     int cur_item = -1, nitem = -1;
-    float sigp_prev = 0.f;  // P' limb scale of the previous tile
+    int jp = -1;            // this group's last tile, its O^T still to be folded
+    float sigp_prev = 0.f;  // P' limb scale of tile jp
 
-    // Writes this CTA's result for `item` (partial or final) and merges when last.
-    // Thread t < 64 ends with dimensions 2t, 2t + 1 of every head: its lane summed the
-    // code bytes of pair t, lane 64 + t the low nibbles.
+    // Both groups arrive here when an item ends, every tile of it folded.  Group 1 hands
+    // its state over; group 0 combines the two, writes this CTA's result for `item`
+    // (partial or final) and merges when last.  Thread t < 64 of group 0 ends with
+    // dimensions 2t, 2t + 1 of every head: its lane summed the code bytes of pair t,
+    // lane 64 + t the low nibbles.
     auto flush = [&](int item) {
 #pragma unroll
       for (int q = 0; q < NQ; ++q) {
         const float vl = warp_sum(l[q]);
         const float vz = warp_sum(zc[q]);
         if (lane == 0) {
-          red[wq * 16 + q] = vl;
-          red[64 + wq * 16 + q] = vz;
+          gred[wq * 16 + q] = vl;
+          gred[64 + wq * 16 + q] = vz;
         }
       }
-      float *xch = reinterpret_cast<float *>(smem + kSmP);  // [16][64]; both P' buffers are idle here
+      float *xo = reinterpret_cast<float *>(smem + kSmP);  // [16][128] o of group 1, then its m[16]
+      float *xch = xo + 16 * 128 + 16;                     // [16][64] low-nibble sums
+      tc::named_sync(3, 256);  // no P' buffer is in use: every product of the item has been folded
+      if (grp == 1) {
+#pragma unroll
+        for (int q = 0; q < NQ; ++q) xo[q * 128 + t] = o[q];
+        if (t == 0) {
+#pragma unroll
+          for (int q = 0; q < NQ; ++q) xo[16 * 128 + q] = m[q];
+        }
+      }
+      tc::named_sync(3, 256);
+      if (grp == 1) {
+        tc::named_sync(3, 256);  // group 0 has read the hand-over and the exchange area
+        return;
+      }
+      float lt[NQ], zt[NQ];
+      const float *r1 = red + 128;
+#pragma unroll
+      for (int q = 0; q < NQ; ++q) {
+        const float l0 = gred[q] + gred[16 + q] + gred[32 + q] + gred[48 + q];
+        const float z0 = gred[64 + q] + gred[80 + q] + gred[96 + q] + gred[112 + q];
+        const float l1 = r1[q] + r1[16 + q] + r1[32 + q] + r1[48 + q];
+        const float z1 = r1[64 + q] + r1[80 + q] + r1[96 + q] + r1[112 + q];
+        const float m1 = xo[16 * 128 + q];
+        const float mn = fmaxf(m[q], m1);
+        const float a0 = m[q] == -INFINITY ? 0.f : ex2(m[q] - mn);
+        const float a1 = m1 == -INFINITY ? 0.f : ex2(m1 - mn);
+        lt[q] = fmaf(l0, a0, l1 * a1);
+        zt[q] = fmaf(z0, a0, z1 * a1);
+        o[q] = fmaf(o[q], a0, xo[q * 128 + t] * a1);
+        m[q] = mn;
+      }
       if (t >= 64) {
 #pragma unroll
         for (int q = 0; q < NQ; ++q)
           if (q < G) xch[q * 64 + (t - 64)] = o[q];
       }
-      tc::named_sync(1, 128);
-      float lt[NQ], zt[NQ], ev[NQ], od[NQ];
+      tc::named_sync(gbar, 128);
+      float ev[NQ], od[NQ];
 #pragma unroll
       for (int q = 0; q < NQ; ++q) {
-        lt[q] = red[q] + red[16 + q] + red[32 + q] + red[48 + q];
-        zt[q] = red[64 + q] + red[80 + q] + red[96 + q] + red[112 + q];
         const float lo = t < 64 && q < G ? xch[q * 64 + t] : 0.f;
         ev[q] = lo + zt[q];
         od[q] = (o[q] - lo) * 0.0625f + zt[q];
       }
-      tc::named_sync(1, 128);
+      tc::named_sync(3, 256);  // release group 1: the shared-memory areas are read
       const int units = a.units_r;
       const int64_t ia = static_cast<int64_t>(item) * units;
       const int cfirst = cta_of(a, ia), clast = cta_of(a, ia + units - 1);
@@ -445,24 +506,24 @@ __global__ void __launch_bounds__(kThreads, 1) decode_int4_kernel(const __grid_c
           }
       }
       __threadfence();
-      tc::named_sync(1, 128);
+      tc::named_sync(gbar, 128);
       if (t == 0) {
         const uint32_t prev = atomicAdd(p.counters + pitem, 1u);
         *last_flag = (prev == static_cast<uint32_t>(nseg - 1)) ? 1 : 0;
       }
-      tc::named_sync(1, 128);
+      tc::named_sync(gbar, 128);
       if (!*last_flag) return;
       __threadfence();
-      merge_partials(part, nseg, G, b, h0, p.Hq, p.out, p.lse, red + 128, t, 1);
+      merge_partials(part, nseg, G, b, h0, p.Hq, p.out, p.lse, red + 256, t, gbar);
       if (t == 0) p.counters[pitem] = 0u;  // ready for the next call
     };
 
     // o = (o + O^T(jj)) * alpha for this thread's row of O^T
     auto fold = [&](int jj, float sigp, const float (&alpha)[NQ]) {
-      if (ok) ok = tc::wait_bar(bar(kBarOFull + (jj & 1)), (jj >> 1) & 1, p.status, abort_flag);
+      if (ok) ok = tc::wait_bar(bar(kBarOFull + (jj & 3)), (jj >> 2) & 1, p.status, abort_flag);
       tc::fence_after();
       int r[C::kO];
-      ld_i32<C::kO>(lane_base + 2 * C::kS + (jj & 1) * C::kO, r);
+      ld_i32<C::kO>(lane_base + 2 * C::kS + (jj & 3) * C::kO, r);
 #pragma unroll
       for (int q = 0; q < NQ; ++q)  // |R| < 2^22
         o[q] = fmaf(sigp, fmaf(to_float(r[2 * q + 1]), 1.f / 254.f, to_float(r[2 * q])), o[q]) * alpha[q];
@@ -470,12 +531,35 @@ __global__ void __launch_bounds__(kThreads, 1) decode_int4_kernel(const __grid_c
     float one[NQ];
 #pragma unroll
     for (int q = 0; q < NQ; ++q) one[q] = 1.f;
+    // the item's query information is released by a group that never reads it
+    auto release_unread = [&]() {
+      if (!qread && t == 0) mbar_arrive(bar(kBarQFree + (nitem & 1)));
+      qread = true;
+    };
 
-    bool pending = false;  // O^T of the previous unit still to be folded
     UnitIter it(a, u0);
     for (int j = 0; j < nu; ++j, it.next()) {
       const Unit un = it.un;
-      const int cb = j & 1, s = j % kStages;
+      if (un.item != cur_item) {
+        if (cur_item >= 0) {
+          if (jp >= 0) fold(jp, sigp_prev, one);
+          jp = -1;
+          release_unread();
+          flush(cur_item);
+        }
+        ++nitem;
+#pragma unroll
+        for (int q = 0; q < NQ; ++q) {
+          m[q] = -INFINITY;
+          l[q] = 0.f;
+          zc[q] = 0.f;
+          o[q] = 0.f;
+        }
+        qread = false;
+        cur_item = un.item;
+      }
+      if ((j & 1) != grp) continue;  // the other group's tile
+      const int cb = grp, s = j % kStages;
       if (ok) ok = tc::wait_bar(bar(kBarSFull + cb), (j >> 1) & 1, p.status, abort_flag);
       tc::fence_after();
       int sr[C::kS];
@@ -490,26 +574,16 @@ __global__ void __launch_bounds__(kThreads, 1) decode_int4_kernel(const __grid_c
       const float4 tm4 = *reinterpret_cast<const float4 *>(st + kStTmax);
       const float tmax = fmaxf(fmaxf(tm4.x, tm4.y), fmaxf(tm4.z, tm4.w));
       const bool valid = static_cast<int64_t>(un.tile) * kTile + t < p.len;
-      if (un.item != cur_item) {
-        if (cur_item >= 0) {
-          if (pending) fold(j - 1, sigp_prev, one);
-          flush(cur_item);
-        }
-        ++nitem;
+      if (!qread) {  // this group's first tile of the item: its sigma and sum(q)
         const float *qi = reinterpret_cast<const float *>(smem + kSmQinfo) + (nitem & 1) * 32;
 #pragma unroll
         for (int q = 0; q < NQ; ++q) {
-          m[q] = -INFINITY;
-          l[q] = 0.f;
-          zc[q] = 0.f;
-          o[q] = 0.f;
           sg[q] = qi[q];
           qs[q] = qi[16 + q];
         }
-        tc::named_sync(1, 128);
-        if (t == 0) mbar_arrive(bar(kBarQFree + (nitem & 1)));  // every thread has read the item's sigma and sum(q)
-        pending = false;
-        cur_item = un.item;
+        tc::named_sync(gbar, 128);
+        if (t == 0) mbar_arrive(bar(kBarQFree + (nitem & 1)));
+        qread = true;
       }
       float sv[NQ];
 #pragma unroll
@@ -518,12 +592,12 @@ __global__ void __launch_bounds__(kThreads, 1) decode_int4_kernel(const __grid_c
                              to_float(sr[3 * q]));
         sv[q] = fmaf(mi.x, sg[q] * x, mi.y * qs[q]);
       }
-      // does any logit of this tile exceed the running max?
+      // does any logit of this tile exceed the group's running max?
       int need = 0;
 #pragma unroll
       for (int q = 0; q < NQ; ++q)
         if (q < G && valid && sv[q] * c > m[q]) need = 1;
-      need = tc::bar_or(1, 128, need);
+      need = tc::bar_or(gbar, 128, need);
       float alpha[NQ];
 #pragma unroll
       for (int q = 0; q < NQ; ++q) alpha[q] = 1.f;
@@ -531,30 +605,31 @@ __global__ void __launch_bounds__(kThreads, 1) decode_int4_kernel(const __grid_c
 #pragma unroll
         for (int q = 0; q < NQ; ++q) {
           const float x = warp_max((valid && q < G) ? sv[q] : -INFINITY);
-          if (lane == 0) red[wq * 16 + q] = x;
+          if (lane == 0) gred[wq * 16 + q] = x;
         }
-        tc::named_sync(1, 128);
+        tc::named_sync(gbar, 128);
 #pragma unroll
         for (int q = 0; q < NQ; ++q) {
-          const float mt = fmaxf(fmaxf(red[q], red[16 + q]), fmaxf(red[32 + q], red[48 + q])) * c;
+          const float mt = fmaxf(fmaxf(gred[q], gred[16 + q]), fmaxf(gred[32 + q], gred[48 + q])) * c;
           const float mn = fmaxf(m[q], mt);
           alpha[q] = (mn == -INFINITY) ? 1.f : ex2(m[q] - mn);
           m[q] = mn;
         }
-        tc::named_sync(1, 128);  // red is reused later
+        tc::named_sync(gbar, 128);  // gred is reused later
       }
-      // P'^T limbs into buffer j % 2 (its previous reader, unit j-2, was folded at j-1):
-      // p s_v = sigp (l0 + l1 / 254) with l0 = rint(x) in [0, 127], x = p s_v / sigp, and
-      // l1 = rint(254 (x - l0)) in [-127, 127]; sigp = tmax / 126.99
+      // P'^T limbs into buffer j % 4 (its previous reader, tile j-4 of this group, was
+      // folded at tile j-2): p s_v = sigp (l0 + l1 / 254) with l0 = rint(x) in [0, 127],
+      // x = p s_v / sigp, l1 = rint(254 (x - l0)) in [-127, 127]; sigp = tmax / 126.99
       const float invp = tmax > 0.f ? 126.99f / tmax : 0.f;
-      uint8_t *pb = reinterpret_cast<uint8_t *>(smem + kSmP + cb * 4096);
+      const float zi = mi.z * invp;
+      uint8_t *pb = reinterpret_cast<uint8_t *>(smem + kSmP + (j & 3) * 4096);
 #pragma unroll
       for (int q = 0; q < NQ; ++q) {
         const float pv = (valid && q < G && m[q] != -INFINITY) ? ex2(fmaf(sv[q], c, -m[q])) : 0.f;
         l[q] = fmaf(l[q], alpha[q], pv);
         zc[q] = fmaf(zc[q], alpha[q], pv * mi.w);
         if (q < G) {
-          const float x = pv * mi.z * invp;
+          const float x = pv * zi;
           float r0, r1;
           const uint32_t b0 = round_byte(x, r0);
           const uint32_t b1 = round_byte((x - r0) * 254.f, r1);
@@ -564,23 +639,24 @@ __global__ void __launch_bounds__(kThreads, 1) decode_int4_kernel(const __grid_c
       }
       tc::fence_async_smem();
       tc::fence_before();
-      mbar_arrive(bar(kBarPFull + cb));
-      // fold the previous unit of the same item, bringing it to this unit's scale
-      if (pending) {
-        fold(j - 1, sigp_prev, alpha);
+      mbar_arrive(bar(kBarPFull + (j & 3)));
+      // fold this group's previous tile of the item, bringing it to this tile's scale
+      if (jp >= 0) {
+        fold(jp, sigp_prev, alpha);
       } else {
 #pragma unroll
         for (int q = 0; q < NQ; ++q) o[q] *= alpha[q];
       }
+      jp = j;
       sigp_prev = tmax * (1.f / 126.99f);
-      pending = true;
     }
     if (nu > 0) {
-      if (pending) fold(nu - 1, sigp_prev, one);
+      if (jp >= 0) fold(jp, sigp_prev, one);
+      release_unread();
       flush(cur_item);
     }
-  } else if (warp < 10) {
-    // ================= prep warps =================
+  } else {
+    // ================= prep warps (10-13) =================
     const int wq = warp & 3;
     const int ct = (wq << 5) | lane;  // token row of the tile
     const int rot = (ct >> 1) & 3;    // 64-byte swizzle of row ct: chunk i sits at i ^ rot
@@ -624,7 +700,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_int4_kernel(const __grid_c
       const uint32_t vmax = __reduce_max_sync(0xffffffffu, vsz & 0xffffu);
       if (lane == 0)
         reinterpret_cast<float *>(st + kStTmax)[wq] = __half2float(__ushort_as_half(static_cast<unsigned short>(vmax)));
-      if (first && warp == 6) {
+      if (first && warp == 10) {
         // the item's query limbs replace those of the item two before, once its last
         // S^T product has run and the softmax has read its sigma and sum(q)
         if (nitem >= 2 && !tc::wait_bar(bar(kBarQFree + (nitem & 1)), ((nitem - 2) >> 1) & 1, p.status, abort_flag))
