@@ -167,6 +167,19 @@ def recorded_traffic(workload):
 
 # ---------------------------------------------------------------- our arm
 
+def reduce_over_ranks(dist, ms, nbytes, device):
+    """Whole-job timing over the ranks: the slowest rank's time and the bytes of all
+    ranks (every rank takes both collectives, in the same order)."""
+    if not dist:
+        return ms, float(nbytes)
+    import torch
+    t = torch.tensor([ms], device=device, dtype=torch.float64)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    b = torch.tensor([float(nbytes)], device=device, dtype=torch.float64)
+    dist.all_reduce(b)
+    return float(t.item()), float(b.item())
+
+
 def run_ours(args, rank, world, dist):
     import torch
 
@@ -250,14 +263,7 @@ def run_ours(args, rank, world, dist):
     torch.cuda.synchronize()
     dec_ms = [a.elapsed_time(b) for a, b in kev[2]]
     assert cache.device_status() == 0, "device status word set"
-    ms_max, bytes_sum = ms, nbytes
-    if dist:
-        t = torch.tensor([ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms_max = float(t.item())
-        b = torch.tensor([float(nbytes)], device=dev, dtype=torch.float64)
-        dist.all_reduce(b)
-        bytes_sum = float(b.item())
+    ms_max, bytes_sum = reduce_over_ranks(dist, ms, nbytes, dev)
     value = bytes_sum / (ms_max * 1e-3) / 1e9
     us_per_token_layer = ms * 1e3 / (steps * nlayers)
     dec_avg_ms = statistics.mean(dec_ms)
