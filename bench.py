@@ -11,7 +11,9 @@ attention per step / step time (GB/s), the step timed with no events between its
 launches; each append + attend goes through duo_append_decode (one fused launch at
 batch 1).  roofline.achieved divides the same bytes by the timed region's time per
 decode call; a second pass of the same steps with an event pair around every call
-gives event_bracketed_call_us for reference.  The chunked pre-fill workload (256K
+gives event_bracketed_call_us for reference; roofline.traffic is the DRAM traffic per
+launch from the committed ncu capture, reported while the sources of the workload's
+kernels still hash to the recorded value.  The chunked pre-fill workload (256K
 prompt in 32K chunks, same shape) is timed after it and reported under "prefill",
 and the identification-phase gated forward (32K tokens) under "gated".
 
