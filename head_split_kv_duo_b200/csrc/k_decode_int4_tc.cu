@@ -18,7 +18,8 @@
 // head as three limbs (21 bits below the row's largest coefficient), P' per tile as two
 // (15 bits below the tile's largest s_v, which bounds p s_v since INT4 items keep the
 // running max exact, p <= 1).  The int32 accumulators are exact; the limbs are split
-// and recombined in fp32 by exact magic-number adds (no conversion instructions).  Per token the scale and zero then give
+// and recombined in fp32 by exact magic-number adds (no conversion instructions).  Per
+// token the scale and zero then give
 //   q . k_t = s_t (q . c_t) + z_t sum(q),   sum_t p_t v_t = sum_t p'_t c_t + sum_t p_t z_t.
 //
 // Roles of a CTA (one per SM, 448 threads):
