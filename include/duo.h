@@ -150,6 +150,9 @@ DUO_API duo_status duo_prefill_chunk(duo_cache *cache, int layer, const void *q,
  * cached token of its retrieval head, or to the sinks and ring of its streaming
  * head.  The token must have been appended first (it attends to itself).
  *   q, out  device [B][Hq][d];  lse device [B][Hq] fp32, or NULL
+ * With INT4 retrieval heads (bf16, head_dim 128) the streaming heads and the retrieval
+ * heads are two launches on the stream; each writes only its own heads' rows of out
+ * and lse.
  * DUO_ERR_INVALID if the layer is empty.
  */
 DUO_API duo_status duo_decode_attention(duo_cache *cache, int layer, const void *q, void *out, float *lse,
@@ -161,8 +164,9 @@ DUO_API duo_status duo_decode_attention(duo_cache *cache, int layer, const void 
  * duo_decode_attention ("Decoding Procedure", steps 2-4, in the order of reading R6).
  * For bf16 caches with head_dim 128 (not INT4) and batch 1 it is one launch: the decode
  * kernel writes the token's rows into the cache itself, each by the CTA that then reads
- * the tile holding it; other caches get the two launches (the faster choice measured).  The cache afterwards holds
- * exactly what duo_append_kv would have written, and len advances by one.
+ * the tile holding it; other caches get the append launch, then the decode launches
+ * (the faster choice measured).  The cache afterwards holds exactly what duo_append_kv
+ * would have written, and len advances by one.
  * DUO_ERR_CAPACITY if len + 1 > max_len.
  */
 DUO_API duo_status duo_append_decode(duo_cache *cache, int layer, const void *q, const void *k, const void *v,
