@@ -1,32 +1,41 @@
 #!/usr/bin/env python
 """Benchmark of the hybrid-head KV attention path on B200.
 
-Headline workload (N = 1): decode attention of a Llama-3-8B-shaped GQA layer (32 q /
-8 kv heads, d 128, 4 retrieval + 4 streaming kv heads, S 16, W 512, bf16) at a
-128K-token context, batch 1.  One step = for each of 4 layer caches in turn (4 x
-1.08 GB of K/V, larger than L2, so no L2 flush is needed): append the new token's
-K/V and run decode attention -- the whole decode path (append/evict, retrieval
-split-KV, streaming sink+ring, merge).  value = algorithmic HBM bytes of the decode
-attention per step / step time (GB/s), the step timed with no events between its
-launches; each append + attend goes through duo_append_decode (one fused launch at
-batch 1).  roofline.achieved divides the same bytes by the timed region's time per
-decode call; a second pass of the same steps with an event pair around every call
-gives event_bracketed_call_us for reference; roofline.traffic is the DRAM traffic per
-launch from the committed ncu capture, reported while the sources of the workload's
-kernels still hash to the recorded value.  The chunked pre-fill workload (256K
-prompt in 32K chunks, same shape) is timed after it and reported under "prefill",
-and the identification-phase gated forward (32K tokens) under "gated".
+Headline workload (N = 1): decode attention of a Llama-3-8B-shaped GQA model (32
+layers; per layer 32 q / 8 kv heads, d 128, 4 retrieval + 4 streaming kv heads, S 16,
+W 512, bf16) at a 128K-token context, batch 1.  One step = one new token through the
+32 layer caches (32 x 0.27 GB of K/V, far larger than L2, so no L2 flush is needed):
+per layer, append the token's K/V and run decode attention -- the whole decode path
+(append/evict, retrieval split-KV, streaming sink+ring, merge), through
+duo_append_decode (one fused launch per layer at batch 1).  value = algorithmic HBM
+bytes of the decode attention per step / step time (GB/s), the step timed with no
+events between its launches.  The K steps the driver asks for are timed as one region;
+the region is repeated (at least 5 times, and until about half a second of GPU time
+is covered) and value is the median region, with the spread reported beside it.
 
---impl reference times the fp64 CPU oracle on the host cores on a bounded sample of
-the same workload (the reference arm).  Under torchrun every rank runs an
-independent replica (the path does not shard); value sums the ranks' bytes over
-the slowest rank's time.
+"workloads" holds every decode configuration on the same footing (Llama-2-7B MHA 32K
+at batch 1 and 8, Llama-3-8B GQA 128K at batch 1 and 4, the 1M-token 32-layer stack
+with INT4 retrieval heads): 5 regions of at least 100 ms of GPU time each, median and
+spread, its roofline against the measured HBM peak, the clocks seen, and the fp64
+oracle timed on the host cores on a bounded sample of the same workload.  The chunked
+pre-fill (256K prompt in 32K chunks, same shape; at least 5 runs) is reported under
+"prefill" with an oracle baseline extrapolated from sampled query rows, and the
+identification-phase gated forward (32K tokens) under "gated".
+
+roofline.traffic is the DRAM traffic per launch from a committed ncu capture, reported
+while the sources of the kernels the workload runs still hash to the recorded value.
+
+--impl reference times the fp64 CPU oracle on the host cores, K steps after W warm-up
+steps, each step a bounded sample of the headline step (the oracle's decode of a few
+of its layers).  Under torchrun every rank runs an independent replica (the path does
+not shard); value sums the ranks' bytes over the slowest rank's time.
 """
 from __future__ import annotations
 
 import argparse
 import hashlib
 import json
+import math
 import os
 import statistics
 import subprocess
@@ -41,28 +50,39 @@ METRIC = "decode-attn achieved HBM GB/s + μs/token/layer at 128K; prefill TFLOP
 WORKLOAD = "llama3-8b-gqa-decode-128k-b1"
 HQ, HKV, D, NRET, S, W = 32, 8, 128, 4, 16, 512
 CTX = 131072
-ROT_LAYERS = 4
 PREFILL_LEN, PREFILL_CHUNK = 262144, 32768
+LAYERS = 32  # Llama-2-7B and Llama-3-8B both have 32 layers
 
 # decode workloads: (q heads, kv heads, retrieval kv heads, context, batch, layers, retrieval format);
-# `layers` caches are visited in turn each step (the headline rotates 4 so that a step
-# touches more K/V than L2 holds; the INT4 stack is the 32-layer model itself)
+# a step visits the `layers` caches in turn (one new token through the model)
 DECODE_WORKLOADS = {
-    "llama3-8b-gqa-decode-128k-b1": (32, 8, 4, 131072, 1, 4, "same"),
-    "llama3-8b-gqa-decode-128k-b4": (32, 8, 4, 131072, 4, 2, "same"),
-    "llama2-7b-mha-decode-32k-b1": (32, 32, 8, 32768, 1, 8, "same"),
-    "llama2-7b-mha-decode-32k-b8": (32, 32, 8, 32768, 8, 2, "same"),
-    "llama3-8b-gqa-decode-1m-int4-32l": (32, 8, 4, 1 << 20, 1, 32, "int4"),
+    "llama3-8b-gqa-decode-128k-b1": (32, 8, 4, 131072, 1, LAYERS, "same"),
+    "llama3-8b-gqa-decode-128k-b4": (32, 8, 4, 131072, 4, LAYERS, "same"),
+    "llama2-7b-mha-decode-32k-b1": (32, 32, 8, 32768, 1, LAYERS, "same"),
+    "llama2-7b-mha-decode-32k-b8": (32, 32, 8, 32768, 8, LAYERS, "same"),
+    "llama3-8b-gqa-decode-1m-int4-32l": (32, 8, 4, 1 << 20, 1, LAYERS, "int4"),
 }
+REGIONS = 5              # timed regions per workload (median and spread reported)
+REGION_MS = 100.0        # GPU time per region of a workload entry, at least
+HEADLINE_TOTAL_MS = 500.0  # headline: regions of K steps until about this much is timed
+MAX_HEADLINE_REGIONS = 25
+MAX_REGION_STEPS = 400
 
 
-def decode_bytes(len_, B=1, Hr=NRET, Hs=HKV - NRET, Hq=HQ, d=D, fmt="same"):
+def decode_bytes(len_, B=1, Hr=NRET, Hs=HKV - NRET, Hq=HQ, d=D, fmt="same", S=S, W=W):
     """Algorithmic HBM bytes of one decode-attention call: every visible K and V row
     once (bf16 rows, or INT4 codes plus fp16 scale/zero), the queries, the outputs and
     the lse."""
     kv = 2 * d * 2
     rkv = 2 * (d // 2 + 4) if fmt == "int4" else kv
     return B * (Hr * len_ * rkv + Hs * min(len_, S + W) * kv) + B * Hq * d * 2 * 2 + B * Hq * 4
+
+
+def visible_pairs(i, retrieval, S=S, W=W):
+    """Keys visible to the query at absolute position i (causal, or sinks + window)."""
+    if retrieval:
+        return i + 1
+    return min(i + 1, S) + min(W, max(0, i + 1 - S))
 
 
 def prefill_flops(L=PREFILL_LEN, Hq=HQ, d=D, G=HQ // HKV, nret=NRET):
@@ -89,6 +109,13 @@ def peaks():
         p = json.load(open(path))
         return p["hbm_gbs"], p["bf16_tflops"], p.get("bf16_tflops_sustained", p["bf16_tflops"]), "measured"
     return 6650.0, 1590.0, 1400.0, "fallback"
+
+
+def spread(values):
+    """Median, min, max and (max - min) / median in percent of a list of region values."""
+    med = statistics.median(values)
+    return {"median": round(med, 3), "min": round(min(values), 3), "max": round(max(values), 3),
+            "spread_pct": round(100.0 * (max(values) - min(values)) / med, 2) if med else None, "n": len(values)}
 
 
 class ClockSampler:
@@ -143,28 +170,47 @@ class ClockSampler:
                 "samples": len(sm)}
 
 
-def kernel_hash(workload):
-    """Hash of the sources of the decode kernels a workload runs: recorded DRAM traffic
-    is void once they change."""
-    files = ["k_decode_tc.cu", "tcgen05.cuh", "decode_merge.cuh", "device_common.cuh", "duo_internal.h"]
-    if "int4" in workload:
-        files.append("k_decode_int4_tc.cu")
+def _hash_files(files):
     h = hashlib.sha256()
     for f in files:
         h.update(open(os.path.join(ROOT, "head_split_kv_duo_b200", "csrc", f), "rb").read())
     return h.hexdigest()[:16]
 
 
+def kernel_hash(workload):
+    """Hash of the sources of the decode kernels a workload runs: recorded DRAM traffic
+    is void once they change."""
+    files = ["k_decode_tc.cu", "tcgen05.cuh", "decode_merge.cuh", "device_common.cuh", "duo_internal.h"]
+    if "int4" in workload:
+        files.append("k_decode_int4_tc.cu")
+    return _hash_files(files)
+
+
+def prefill_kernel_hash():
+    return _hash_files(["k_prefill_tc.cu", "tcgen05.cuh", "device_common.cuh", "duo_internal.h"])
+
+
+def _record(name):
+    path = os.path.join(ROOT, "profiles", name)
+    return json.load(open(path)) if os.path.exists(path) else {}
+
+
 def recorded_traffic(workload):
     """DRAM bytes (read + write) per decode launch from the committed ncu summary of
     this workload, when it was taken on the current kernel source."""
-    path = os.path.join(ROOT, "profiles", "decode_traffic.json")
-    if not os.path.exists(path):
-        return None
-    rec = json.load(open(path)).get(workload)
+    rec = _record("decode_traffic.json").get(workload)
     if not rec or rec.get("kernel_hash") != kernel_hash(workload):
         return None
     return rec.get("dram_bytes_per_launch")
+
+
+def recorded_prefill_counters():
+    """ncu counters of one pre-fill launch (tensor pipe, DRAM) recorded on the current
+    kernel source, or None."""
+    rec = _record("prefill_counters.json")
+    if not rec or rec.get("kernel_hash") != prefill_kernel_hash():
+        return None
+    return rec
 
 
 # ---------------------------------------------------------------- our arm
@@ -182,173 +228,232 @@ def reduce_over_ranks(dist, ms, nbytes, device):
     return float(t.item()), float(b.item())
 
 
-def run_ours(args, rank, world, dist):
-    import torch
+def launches_per_layer(B, fmt, Hs):
+    """Kernel launches of one duo_append_decode call (see include/duo.h)."""
+    if fmt == "same":
+        return (1, "fused append+decode") if B == 1 else (2, "append, then decode")
+    return (3 if Hs > 0 else 2), "append, bf16 streaming-head decode, INT4 retrieval-head decode"
 
-    from head_split_kv_duo_b200 import inputs
-    from head_split_kv_duo_b200.duo import DuoCache
 
-    dev = torch.device("cuda", int(os.environ.get("LOCAL_RANK", 0)))
-    torch.cuda.set_device(dev)
-    hbm_peak, tc_peak, tc_sust, peak_src = peaks()
-    steps, warmup = args.steps, args.warmup
-    Hq, Hkv, nret, ctx, B, nlayers, fmt = DECODE_WORKLOADS[args.workload]
-    if args.layers:
-        nlayers = args.layers
-    Hr, Hs = nret, Hkv - nret
-    max_len = ctx + warmup + 3 * steps + 16  # warm-up, timed and event passes, e2e pass
-    mask = inputs.retrieval_mask(nlayers, Hkv, nret, seed=1)
-    cache = DuoCache(nlayers, Hkv, D, mask, S, W, max_len, batch=B, q_heads=Hq, dtype=torch.bfloat16,
-                     retr_fmt=fmt, device=dev)
-    # fill each layer to `ctx` tokens (seeded N(0,1) K/V), in pieces of at most 2^18 tokens
-    piece = min(ctx, 1 << 18)
-    for layer in range(nlayers):
-        for t0 in range(0, ctx, piece):
-            n = min(piece, ctx - t0)
-            k = inputs.randn((B, n, Hkv, D), 100 + 1000 * layer + 2 * t0 // piece, device=dev)
-            v = inputs.randn((B, n, Hkv, D), 101 + 1000 * layer + 2 * t0 // piece, device=dev)
-            cache.append_kv(layer, k, v)
-            del k, v
-    torch.cuda.synchronize()
-    # per-step inputs: q, k, v of the new token for every layer
-    nstep_in = warmup + 2 * steps
-    qs = inputs.randn((nstep_in, nlayers, B, Hq, D), 7, device=dev)
-    ks = inputs.randn((nstep_in, nlayers, B, 1, Hkv, D), 8, device=dev)
-    vs = inputs.randn((nstep_in, nlayers, B, 1, Hkv, D), 9, device=dev)
-    out = torch.empty(nlayers, B, Hq, D, dtype=torch.bfloat16, device=dev)
-    lse = torch.empty(nlayers, B, Hq, dtype=torch.float32, device=dev)
-    stream = torch.cuda.current_stream()
+class DecodeRun:
+    """One decode workload: a cache of `layers` layers filled to `ctx` tokens and the
+    per-step inputs; step(i) appends token i to every layer and attends."""
 
-    def nbytes_of(n):
-        return decode_bytes(n, B=B, Hr=Hr, Hs=Hs, Hq=Hq, fmt=fmt)
+    def __init__(self, name, dev, extra_tokens, nstep_in):
+        import torch
 
-    def step(i, ev=None):
+        from head_split_kv_duo_b200 import inputs
+        from head_split_kv_duo_b200.duo import DuoCache
+
+        self.name = name
+        self.Hq, self.Hkv, self.nret, self.ctx, self.B, self.layers, self.fmt = DECODE_WORKLOADS[name]
+        self.Hr, self.Hs = self.nret, self.Hkv - self.nret
+        self.dev = dev
+        max_len = self.ctx + extra_tokens
+        mask = inputs.retrieval_mask(self.layers, self.Hkv, self.nret, seed=1)
+        self.cache = DuoCache(self.layers, self.Hkv, D, mask, S, W, max_len, batch=self.B, q_heads=self.Hq,
+                              dtype=torch.bfloat16, retr_fmt=self.fmt, device=dev)
+        # fill each layer to ctx tokens (seeded N(0,1) K/V), in pieces of at most 2^18 tokens
+        piece = min(self.ctx, 1 << 18)
+        for layer in range(self.layers):
+            for t0 in range(0, self.ctx, piece):
+                n = min(piece, self.ctx - t0)
+                k = inputs.randn((self.B, n, self.Hkv, D), 100 + 1000 * layer + 2 * t0 // piece, device=dev)
+                v = inputs.randn((self.B, n, self.Hkv, D), 101 + 1000 * layer + 2 * t0 // piece, device=dev)
+                self.cache.append_kv(layer, k, v)
+                del k, v
+        torch.cuda.synchronize()
+        # per-step inputs (q, k, v of the new token for every layer), reused cyclically
+        self.nin = nstep_in
+        self.qs = inputs.randn((nstep_in, self.layers, self.B, self.Hq, D), 7, device=dev)
+        self.ks = inputs.randn((nstep_in, self.layers, self.B, 1, self.Hkv, D), 8, device=dev)
+        self.vs = inputs.randn((nstep_in, self.layers, self.B, 1, self.Hkv, D), 9, device=dev)
+        self.out = torch.empty(self.layers, self.B, self.Hq, D, dtype=torch.bfloat16, device=dev)
+        self.lse = torch.empty(self.layers, self.B, self.Hq, dtype=torch.float32, device=dev)
+        self.stream = torch.cuda.current_stream()
+        self.lpl, self.launch_desc = launches_per_layer(self.B, self.fmt, self.Hs)
+
+    def nbytes_of(self, n):
+        return decode_bytes(n, B=self.B, Hr=self.Hr, Hs=self.Hs, Hq=self.Hq, fmt=self.fmt)
+
+    def step(self, i, ev=None):
+        import torch
+        j = i % self.nin
         nbytes = 0
-        for layer in range(nlayers):
-            n = cache.len(layer) + 1
+        for layer in range(self.layers):
+            n = self.cache.len(layer) + 1
             if ev is not None:
-                ev[0].record(stream)
-            # append the step's token and attend: one launch on the bf16 tcgen05 path
-            cache.append_decode(layer, qs[i, layer], ks[i, layer], vs[i, layer], out=out[layer], lse=lse[layer],
-                                stream=stream)
+                ev[0].record(self.stream)
+            self.cache.append_decode(layer, self.qs[j, layer], self.ks[j, layer], self.vs[j, layer],
+                                     out=self.out[layer], lse=self.lse[layer], stream=self.stream)
             if ev is not None:
-                ev[1].record(stream)
+                ev[1].record(self.stream)
                 ev[2].append((ev[0], ev[1]))
                 ev[0] = torch.cuda.Event(enable_timing=True)
                 ev[1] = torch.cuda.Event(enable_timing=True)
-            nbytes += nbytes_of(n)
+            nbytes += self.nbytes_of(n)
         return nbytes
 
-    for i in range(warmup):
-        step(i)
-    torch.cuda.synchronize()
-    if dist:
-        dist.barrier()
-    # timed region: the steps alone (no events between launches)
-    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    nbytes = 0
+    def region(self, first, steps, dist=None):
+        """Times `steps` steps as one region (synchronize and barrier on both sides);
+        returns (ms, bytes)."""
+        import torch
+        t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        torch.cuda.synchronize()
+        if dist:
+            dist.barrier()
+        t0.record(self.stream)
+        nbytes = 0
+        for i in range(first, first + steps):
+            nbytes += self.step(i)
+        t1.record(self.stream)
+        torch.cuda.synchronize()
+        if dist:
+            dist.barrier()
+        return t0.elapsed_time(t1), nbytes
+
+    def close(self):
+        import torch
+        assert self.cache.device_status() == 0, "device status word set"
+        self.cache.close()
+        del self.cache, self.qs, self.ks, self.vs
+        torch.cuda.empty_cache()
+
+
+def roofline_entry(name, per_launch_bytes, call_ms, hbm_peak, peak_src, launch_desc):
+    achieved = per_launch_bytes / (call_ms * 1e-3) / 1e9
+    return {"bound": "hbm", "kernel": "decode", "achieved": round(achieved, 1), "peak": hbm_peak,
+            "peak_source": f"{peak_src} hbm_gbs (burst copy)", "unit": "GB/s", "frac": round(achieved / hbm_peak, 4),
+            "frac_of_8tbs_spec": round(achieved / 8000.0, 4), "traffic": recorded_traffic(name),
+            "algorithmic_bytes_per_launch": int(per_launch_bytes), "avg_launch_us": round(call_ms * 1e3, 3),
+            "launch": launch_desc}
+
+
+def run_workload(name, dev, hbm_peak, peak_src):
+    """A decode workload entry: REGIONS regions of at least REGION_MS of GPU time."""
+    warm, calib = 3, 2
+    run = DecodeRun(name, dev, extra_tokens=warm + calib + REGIONS * MAX_REGION_STEPS + 16, nstep_in=64)
+    for i in range(warm):
+        run.step(i)
+    ms, _ = run.region(warm, calib)
+    steps = max(1, min(MAX_REGION_STEPS, math.ceil(REGION_MS / (ms / calib))))
+    first = warm + calib
+    ctx0 = run.cache.len(0)
+    regions = []
     with ClockSampler(dev.index) as clk:
-        torch.cuda.synchronize()
-        t0.record(stream)
-        for i in range(warmup, warmup + steps):
-            nbytes += step(i)
-        t1.record(stream)
-        torch.cuda.synchronize()
-    if dist:
-        dist.barrier()
-    ms = t0.elapsed_time(t1)
-    # per-call durations of the decode call for the roofline: the same steps again, with
-    # an event pair around every call (the events add a little time between launches)
+        for r in range(REGIONS):
+            ms, nbytes = run.region(first, steps)
+            first += steps
+            regions.append((ms, nbytes))
+    ctx1 = run.cache.len(0)
+    calls = steps * run.layers
+    gbs = [b / (m * 1e-3) / 1e9 for m, b in regions]
+    med = sorted(range(REGIONS), key=lambda r: gbs[r])[REGIONS // 2]
+    ms_med, bytes_med = regions[med]
+    entry = {
+        "workload": name,
+        "config": {"q_heads": run.Hq, "kv_heads": run.Hkv, "head_dim": D, "retrieval_kv_heads": run.nret, "S": S,
+                   "W": W, "context": run.ctx, "batch": run.B, "layers": run.layers, "retrieval_kv": run.fmt},
+        "gbs": round(gbs[med], 1),
+        "us_per_token_layer": round(ms_med * 1e3 / calls, 3),
+        "regions": dict(spread(gbs), unit="GB/s", steps_per_region=steps,
+                        region_ms_median=round(ms_med, 2), context_range=[ctx0, ctx1]),
+        "roofline": roofline_entry(name, bytes_med / calls, ms_med / calls, hbm_peak, peak_src, run.launch_desc),
+        "clocks": clk.summary(),
+        "gpu_launches": REGIONS * calls * run.lpl,
+    }
+    run.close()
+    return entry
+
+
+def run_headline(args, dev, dist, hbm_peak, peak_src):
+    import torch
+    K, warmup = args.steps, args.warmup
+    extra = warmup + 2 + MAX_HEADLINE_REGIONS * K + 2 * K + 16
+    run = DecodeRun(args.workload, dev, extra_tokens=extra, nstep_in=max(64, K))
+    for i in range(warmup):
+        run.step(i)
+    # regions of exactly K steps: at least REGIONS, and until about HEADLINE_TOTAL_MS
+    first = warmup
+    regions = []
+    with ClockSampler(dev.index) as clk:
+        ms, nbytes = run.region(first, K, dist)
+        first += K
+        regions.append((ms, nbytes))
+        nreg = max(REGIONS, min(MAX_HEADLINE_REGIONS, math.ceil(HEADLINE_TOTAL_MS / max(ms, 1e-3))))
+        if dist:  # every rank times the same number of regions (the slowest rank's need)
+            t = torch.tensor([nreg], device=dev, dtype=torch.int64)
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            nreg = int(t.item())
+        for r in range(1, nreg):
+            ms, nbytes = run.region(first, K, dist)
+            first += K
+            regions.append((ms, nbytes))
+    reduced = [reduce_over_ranks(dist, m, b, dev) for m, b in regions]
+    vals = [b / (m * 1e-3) / 1e9 for m, b in reduced]
+    med = sorted(range(len(vals)), key=lambda r: vals[r])[len(vals) // 2]
+    ms_max, bytes_sum = reduced[med]
+    ms_own, bytes_own = regions[med]
+    calls = K * run.layers
+    # per-call durations for reference: one more region with an event pair around every call
     kev = [torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True), []]
-    for i in range(warmup + steps, warmup + 2 * steps):
-        step(i, kev)
+    for i in range(first, first + K):
+        run.step(i, kev)
+    first += K
     torch.cuda.synchronize()
     dec_ms = [a.elapsed_time(b) for a, b in kev[2]]
-    assert cache.device_status() == 0, "device status word set"
-    ms_max, bytes_sum = reduce_over_ranks(dist, ms, nbytes, dev)
-    value = bytes_sum / (ms_max * 1e-3) / 1e9
-    us_per_token_layer = ms * 1e3 / (steps * nlayers)
-    dec_avg_ms = statistics.mean(dec_ms)
-    per_launch_bytes = nbytes / (steps * nlayers)
-    # the decode call's duration over the timed region: every launch in it belongs to a
-    # decode call (one fused launch at batch 1), so this includes the gaps between them
-    call_ms = ms / (steps * nlayers)
-    achieved = per_launch_bytes / (call_ms * 1e-3) / 1e9
+    roof = roofline_entry(args.workload, bytes_own / calls, ms_own / calls, hbm_peak, peak_src, run.launch_desc)
+    roof["event_bracketed_call_us"] = round(statistics.mean(dec_ms) * 1e3, 3)
 
     # ---- end-to-end through the public API with host buffers ----
     e2e = None
     if not args.skip_e2e:
-        hq = qs.cpu().pin_memory()
-        hk = ks.cpu().pin_memory()
-        hv = vs.cpu().pin_memory()
-        hout = torch.empty(nlayers, B, Hq, D, dtype=torch.bfloat16).pin_memory()
-        dq = torch.empty_like(qs[0])
-        dk = torch.empty_like(ks[0])
-        dv = torch.empty_like(vs[0])
-        # lengths cannot be rewound: this pass keeps appending (max_len has room for it)
+        hq = run.qs[:K].cpu().pin_memory()
+        hk = run.ks[:K].cpu().pin_memory()
+        hv = run.vs[:K].cpu().pin_memory()
+        hout = torch.empty(run.layers, run.B, run.Hq, D, dtype=torch.bfloat16).pin_memory()
+        dq = torch.empty_like(run.qs[0])
+        dk = torch.empty_like(run.ks[0])
+        dv = torch.empty_like(run.vs[0])
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         eb = 0
         torch.cuda.synchronize()
-        e0.record(stream)
-        for i in range(warmup, warmup + steps):
+        e0.record(run.stream)
+        for i in range(K):
             dq.copy_(hq[i], non_blocking=True)
             dk.copy_(hk[i], non_blocking=True)
             dv.copy_(hv[i], non_blocking=True)
-            for layer in range(nlayers):
-                eb += nbytes_of(cache.len(layer) + 1)
-                cache.append_decode(layer, dq[layer], dk[layer], dv[layer], out=out[layer], lse=lse[layer],
-                                    stream=stream)
-            hout.copy_(out, non_blocking=True)
-        e1.record(stream)
+            for layer in range(run.layers):
+                eb += run.nbytes_of(run.cache.len(layer) + 1)
+                run.cache.append_decode(layer, dq[layer], dk[layer], dv[layer], out=run.out[layer],
+                                        lse=run.lse[layer], stream=run.stream)
+            hout.copy_(run.out, non_blocking=True)
+        e1.record(run.stream)
         torch.cuda.synchronize()
         ems = e0.elapsed_time(e1)
         h2d = (dq.numel() + dk.numel() + dv.numel()) * 2
         e2e = {"value": round(eb / (ems * 1e-3) / 1e9, 1), "unit": "GB/s", "h2d_bytes_per_step": h2d,
-               "d2h_bytes_per_step": hout.numel() * 2, "ms_per_step": round(ems / steps, 4)}
-    cache.close()
-    del cache
-    torch.cuda.empty_cache()
-
-    # ---- chunked pre-fill (Llama-3-8B GQA, 256K in 32K chunks) ----
-    prefill = None
-    if not args.skip_prefill:
-        prefill = run_prefill(args, dev, tc_peak, tc_sust, peak_src)
-    gated = None
-    if not args.skip_gated:
-        gated = run_gated(args, dev, tc_peak, tc_sust, peak_src)
-
-    kv_gb = nlayers * nbytes_of(ctx) / 1e9
-    # per layer and step: one fused append + decode launch (bf16, batch 1), else the append
-    # then the decode; an INT4 layer decodes its bf16 streaming heads and its INT4
-    # retrieval heads in two launches
-    if fmt == "same":
-        launches_per_layer, launch_desc = (1, "fused append+decode") if B == 1 else (2, "append, then decode")
-    else:
-        launches_per_layer = 3 if Hkv > nret else 2
-        launch_desc = "append, bf16 streaming-head decode, INT4 retrieval-head decode"
-    res = {
-        "metric": METRIC, "value": round(value, 1), "unit": "GB/s", "n_gpus": world, "steps": steps,
-        "warmup": warmup, "ms_per_step": round(ms_max / steps, 4), "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": None, "dtype": "bf16" if fmt == "same" else "bf16+int4kv", "data": "synthetic",
-        "config": {"workload": args.workload, "q_heads": Hq, "kv_heads": Hkv, "head_dim": D, "retrieval_kv_heads": nret,
-                   "S": S, "W": W, "context": ctx, "batch": B, "layers": nlayers, "retrieval_kv": fmt,
-                   "l2": f"inputs larger than L2: {nlayers} layer caches of {kv_gb / nlayers:.2f} GB visited per step",
-                   "parallelism": f"replicas{world}"},
-        "us_per_token_layer": round(us_per_token_layer, 3),
-        "roofline": {"bound": "hbm", "kernel": "decode", "achieved": round(achieved, 1),
-                     "peak": hbm_peak, "peak_source": f"{peak_src} hbm_gbs (burst copy)", "unit": "GB/s",
-                     "frac": round(achieved / hbm_peak, 4), "frac_of_8tbs_spec": round(achieved / 8000.0, 4),
-                     "traffic": recorded_traffic(args.workload),
-                     "algorithmic_bytes_per_launch": int(per_launch_bytes), "avg_launch_us": round(call_ms * 1e3, 3),
-                     "event_bracketed_call_us": round(dec_avg_ms * 1e3, 3),
-                     "launch": launch_desc},
-        "gpu_launches": steps * nlayers * launches_per_layer,
+               "d2h_bytes_per_step": hout.numel() * 2, "ms_per_step": round(ems / K, 4)}
+    kv_gb = run.layers * run.nbytes_of(run.ctx) / 1e9
+    head = {
+        "value": round(vals[med], 1), "ms_per_step": round(ms_max / K, 4),
+        "regions": dict(spread(vals), unit="GB/s", steps_per_region=K,
+                        region_ms_median=round(ms_max, 2)),
+        "config": {"workload": args.workload, "q_heads": run.Hq, "kv_heads": run.Hkv, "head_dim": D,
+                   "retrieval_kv_heads": run.nret, "S": S, "W": W, "context": run.ctx, "batch": run.B,
+                   "layers": run.layers, "retrieval_kv": run.fmt,
+                   "l2": f"inputs larger than L2: {run.layers} layer caches of {kv_gb / run.layers:.2f} GB "
+                         f"visited per step",
+                   "parallelism": f"replicas{args.gpus}"},
+        "dtype": "bf16" if run.fmt == "same" else "bf16+int4kv",
+        "us_per_token_layer": round(ms_own * 1e3 / calls, 3),
+        "roofline": roof,
+        "gpu_launches": len(regions) * calls * run.lpl,
         "clocks": clk.summary(),
         "e2e": e2e,
-        "prefill": prefill,
-        "gated": gated,
     }
-    return res
+    run.close()
+    return head
 
 
 def run_prefill(args, dev, tc_peak, tc_sust, peak_src):
@@ -383,16 +488,28 @@ def run_prefill(args, dev, tc_peak, tc_sust, peak_src):
 
     for _ in range(args.prefill_warmup):
         one()
-    times = [one() for _ in range(args.prefill_steps)]
-    ms = statistics.mean(times)
+    with ClockSampler(dev.index) as clk:
+        times = [one() for _ in range(args.prefill_steps)]
     fl = prefill_flops(L)
+    tfl = [fl / (t * 1e-3) / 1e12 for t in times]
+    ms = statistics.median(times)
     tflops = fl / (ms * 1e-3) / 1e12
     name = f"llama3-8b-gqa-prefill-{L // 1024}k-chunk{C // 1024}k"
-    return {"workload": name, "tflops": round(tflops, 1), "ms": round(ms, 2),
-            "steps": args.prefill_steps, "algorithmic_tflop": round(fl / 1e12, 2),
-            "roofline": {"bound": "tensor", "achieved": round(tflops, 1), "peak": tc_peak,
-                         "peak_source": f"{peak_src} bf16_tflops (burst)", "unit": "TFLOP/s",
-                         "frac": round(tflops / tc_peak, 4), "frac_of_sustained": round(tflops / tc_sust, 4)}}
+    roof = {"bound": "tensor", "achieved": round(tflops, 1), "peak": tc_peak,
+            "peak_source": f"{peak_src} bf16_tflops (burst)", "unit": "TFLOP/s",
+            "frac": round(tflops / tc_peak, 4), "frac_of_sustained": round(tflops / tc_sust, 4),
+            "tensor_pipe_active": None, "traffic": None}
+    rec = recorded_prefill_counters() if L == PREFILL_LEN and C == PREFILL_CHUNK else None
+    if rec:
+        roof["tensor_pipe_active"] = rec.get("tensor_pipe_active")
+        roof["traffic"] = rec.get("dram_bytes_per_launch")
+        roof["counters_source"] = rec.get("source")
+    res = {"workload": name, "tflops": round(tflops, 1), "ms": round(ms, 2), "steps": args.prefill_steps,
+           "runs": dict(spread(tfl), unit="TFLOP/s"), "algorithmic_tflop": round(fl / 1e12, 2),
+           "roofline": roof, "clocks": clk.summary()}
+    if not args.skip_cpu_baseline:
+        res["cpu_baseline"] = oracle_prefill_sample(args, k.cpu(), v.cpu(), q.cpu(), mask, fl)
+    return res
 
 
 def run_gated(args, dev, tc_peak, tc_sust, peak_src):
@@ -411,7 +528,7 @@ def run_gated(args, dev, tc_peak, tc_sust, peak_src):
     out = torch.empty_like(q)
     stream = torch.cuda.current_stream()
     times = []
-    for i in range(4):
+    for i in range(6):
         a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         a.record(stream)
         gated_attention(q, k, v, alpha, S, W, out=out, stream=stream)
@@ -419,67 +536,154 @@ def run_gated(args, dev, tc_peak, tc_sust, peak_src):
         torch.cuda.synchronize()
         if i > 0:
             times.append(a.elapsed_time(b))
-    ms = statistics.mean(times)
+    ms = statistics.median(times)
     fl = gated_flops(L)
     tflops = fl / (ms * 1e-3) / 1e12
     return {"workload": f"llama3-8b-gqa-gated-{L // 1024}k", "tflops": round(tflops, 1), "ms": round(ms, 3),
-            "steps": len(times), "algorithmic_tflop": round(fl / 1e12, 3),
+            "steps": len(times), "runs": dict(spread([fl / (t * 1e-3) / 1e12 for t in times]), unit="TFLOP/s"),
+            "algorithmic_tflop": round(fl / 1e12, 3),
             "roofline": {"bound": "tensor", "achieved": round(tflops, 1), "peak": tc_peak,
                          "peak_source": f"{peak_src} bf16_tflops (burst)", "unit": "TFLOP/s",
                          "frac": round(tflops / tc_peak, 4), "frac_of_sustained": round(tflops / tc_sust, 4)}}
 
 
-# ---------------------------------------------------------- reference arm
+# ---------------------------------------------------------- the oracle on the host
 
-def oracle_sample(args):
-    """Time the fp64 oracle on decode steps of the headline workload (one layer at
-    128K context; each step = one query token, all 32 query heads)."""
+def _u16(t):
     import numpy as np
     import torch
+    return t.contiguous().view(torch.int16).numpy().view(np.uint16)
 
+
+class OracleDecode:
+    """The fp64 oracle's decode of one layer of a decode workload (the query of the
+    newest token at position ctx - 1, every query head of every sequence).  INT4
+    workloads go through the oracle's own quantiser and dequantiser, as the parity tests
+    do; `ctx_cap` bounds the context of the sample.  Inputs are the seeded N(0,1) draws
+    of the workload's first layer, drawn on `device` when given (faster) and copied to
+    the host."""
+
+    def __init__(self, name, ctx_cap=None, device="cpu"):
+        import numpy as np
+
+        import oracle
+        from head_split_kv_duo_b200 import inputs
+
+        self.oracle = oracle
+        Hq, Hkv, nret, ctx, B, _, fmt = DECODE_WORKLOADS[name]
+        self.ctx = min(ctx, ctx_cap) if ctx_cap else ctx
+        self.B, self.Hq, self.Hkv, self.nret, self.fmt = B, Hq, Hkv, nret, fmt
+        self.mask = inputs.retrieval_mask(1, Hkv, nret, seed=1)[0].numpy().astype(bool)
+        k = inputs.randn((B, self.ctx, Hkv, D), 100, device=device).cpu()
+        v = inputs.randn((B, self.ctx, Hkv, D), 101, device=device).cpu()
+        self.q = _u16(inputs.randn((B, 1, Hq, D), 7, device=device).cpu())
+        if fmt == "int4":
+            # fp64 K/V (the streaming heads' rows as they are); per retrieval head the codes
+            # and fp16 scale/zero from the oracle's quantiser, dequantised at every step
+            self.k = k.float().numpy().astype(np.float64)
+            self.v = v.float().numpy().astype(np.float64)
+            self.codes = [(g, oracle.int4_quantize(_u16(k[:, :, g])), oracle.int4_quantize(_u16(v[:, :, g])))
+                          for g in np.nonzero(self.mask)[0]]
+        else:
+            self.k, self.v = _u16(k), _u16(v)
+
+    def step(self):
+        if self.fmt == "int4":
+            for g, kc, vc in self.codes:
+                self.k[:, :, g] = self.oracle.int4_dequantize(*kc).reshape(self.B, self.ctx, D)
+                self.v[:, :, g] = self.oracle.int4_dequantize(*vc).reshape(self.B, self.ctx, D)
+        return self.oracle.attend(self.q, self.k, self.v, self.mask, S, W, pos0=self.ctx - 1)
+
+    def nbytes(self):
+        return decode_bytes(self.ctx, B=self.B, Hr=self.nret, Hs=self.Hkv - self.nret, Hq=self.Hq, fmt=self.fmt)
+
+
+def oracle_decode_sample(name, seconds, max_steps, ctx_cap=None, device="cpu"):
+    """cpu_baseline of a decode workload: oracle decode steps of one layer until
+    `seconds` of wall time (at least one)."""
     import oracle
-    from head_split_kv_duo_b200 import inputs
-
-    mask = inputs.retrieval_mask(1, HKV, NRET, seed=1)[0].numpy().astype(bool)
-    k = inputs.randn((1, CTX, HKV, D), 100).view(torch.int16).numpy().view(np.uint16)
-    v = inputs.randn((1, CTX, HKV, D), 101).view(torch.int16).numpy().view(np.uint16)
-    q = inputs.randn((1, 1, HQ, D), 7).view(torch.int16).numpy().view(np.uint16)
-    oracle.attend(q, k[:, :1024], v[:, :1024], mask, S, W, pos0=1023)  # load / warm
+    od = OracleDecode(name, ctx_cap, device)
     n, t_total = 0, 0.0
-    budget = args.oracle_seconds
-    while t_total < budget and n < args.oracle_max_steps:
+    while (t_total < seconds or n == 0) and n < max_steps:
         t = time.perf_counter()
-        oracle.attend(q, k, v, mask, S, W, pos0=CTX - 1)
+        od.step()
         t_total += time.perf_counter() - t
         n += 1
-    gbs = n * decode_bytes(CTX) / t_total / 1e9
+    gbs = n * od.nbytes() / t_total / 1e9
+    what = f"{n} oracle decode steps of one layer at context {od.ctx}"
+    if od.ctx != DECODE_WORKLOADS[name][3]:
+        what += f" (the workload's {DECODE_WORKLOADS[name][3]}-token context needs too much fp64 host memory)"
+    if od.fmt == "int4":
+        what += ", each step dequantising the oracle's INT4 codes of the retrieval heads, then attending"
     return {"value": round(gbs, 3), "unit": "GB/s", "cores": oracle.num_threads(), "kind": "oracle",
-            "sample": f"{n} decode steps of one layer at context {CTX} (all 32 query heads), "
-                      f"{t_total:.1f} s wall on {oracle.num_threads()} threads",
-            "seconds": round(t_total, 2), "steps": n}
+            "sample": f"{what}, batch {od.B}, all {od.Hq} query heads; {t_total:.1f} s wall on "
+                      f"{oracle.num_threads()} threads", "seconds": round(t_total, 2), "steps": n}
 
+
+def oracle_prefill_sample(args, k, v, q, mask, flops_total):
+    """cpu_baseline of the pre-fill: the oracle on sampled query rows of every chunk (the
+    first and last rows, rows around S and W, and random rows), all 32 query heads; the
+    whole prompt's time is extrapolated by the count of visible (query, key) pairs."""
+    import numpy as np
+
+    import oracle
+    L, C = args.prefill_len, args.prefill_chunk
+    kb, vb, qb = _u16(k), _u16(v), _u16(q)
+    m = mask[0].numpy().astype(bool)
+    G = HQ // HKV
+    rng = np.random.default_rng(0)
+    nchunks = L // C
+    per_chunk = {c: set([0, C - 1] + [x for x in (S - 1, S, S + 1, W - 1, W, W + 1) if 0 <= x < C])
+                 for c in range(nchunks)}
+    for r in rng.integers(0, L, args.prefill_oracle_rows):
+        per_chunk[int(r) // C].add(int(r) % C)
+    pairs_sample, t_total, nrows = 0, 0.0, 0
+    for c in range(nchunks):
+        rows = sorted(per_chunk[c])
+        ids = [r * HQ + h for r in rows for h in range(HQ)]
+        t = time.perf_counter()
+        oracle.attend(qb, kb[:, :(c + 1) * C], vb[:, :(c + 1) * C], m, S, W, pos0=c * C, rows=ids)
+        t_total += time.perf_counter() - t
+        nrows += len(ids)
+        for r in rows:
+            i = c * C + r
+            pairs_sample += sum(visible_pairs(i, m[h // G]) for h in range(HQ))
+    pairs_total = flops_total // (4 * D)
+    est_s = t_total * pairs_total / pairs_sample
+    return {"value": round(flops_total / est_s / 1e12, 6), "unit": "TFLOP/s", "cores": oracle.num_threads(),
+            "kind": "oracle", "extrapolated": True, "seconds_sampled": round(t_total, 2),
+            "seconds_extrapolated": round(est_s, 1),
+            "sample": f"{nrows} (query row, head) pairs of the {L // 1024}K prompt ({pairs_sample} of the "
+                      f"{pairs_total} visible (query, key) pairs), {t_total:.1f} s wall on "
+                      f"{oracle.num_threads()} threads; time extrapolated by visible-pair count"}
+
+
+# ---------------------------------------------------------------- main
 
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--workload", default=WORKLOAD, choices=sorted(DECODE_WORKLOADS))
-    ap.add_argument("--layers", type=int, default=0,
-                    help="layer caches to rotate through instead of the workload's (small profiling captures)")
-    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workloads", default="all",
+                    help="comma-separated decode workloads for the 'workloads' entries, 'all' or 'none'")
     ap.add_argument("--skip-prefill", action="store_true")
     ap.add_argument("--skip-decode", action="store_true", help="time only the pre-fill workload")
     ap.add_argument("--prefill-len", type=int, default=PREFILL_LEN)
     ap.add_argument("--prefill-chunk", type=int, default=PREFILL_CHUNK)
+    ap.add_argument("--prefill-steps", type=int, default=5)
+    ap.add_argument("--prefill-warmup", type=int, default=1)
+    ap.add_argument("--prefill-oracle-rows", type=int, default=256)
     ap.add_argument("--skip-e2e", action="store_true")
     ap.add_argument("--skip-gated", action="store_true", help="skip the gated (identification-phase) forward")
     ap.add_argument("--gated-len", type=int, default=32768)
     ap.add_argument("--skip-cpu-baseline", action="store_true")
-    ap.add_argument("--prefill-steps", type=int, default=2)
-    ap.add_argument("--prefill-warmup", type=int, default=1)
-    ap.add_argument("--oracle-seconds", type=float, default=6.0)
+    ap.add_argument("--oracle-seconds", type=float, default=4.0)
     ap.add_argument("--oracle-max-steps", type=int, default=40)
+    ap.add_argument("--ref-layers", type=int, default=4,
+                    help="reference arm: layers of the headline step the oracle decodes per step")
     args = ap.parse_args()
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -488,21 +692,9 @@ def main():
     if args.impl == "reference":
         if rank != 0:
             return 0
-        t0 = time.perf_counter()
-        for _ in range(args.warmup):
-            pass
-        cb = oracle_sample(args)
-        res = {"impl": "reference", "metric": METRIC, "value": cb["value"], "unit": "GB/s", "n_gpus": args.gpus,
-               "steps": cb["steps"], "warmup": args.warmup, "ms_per_step": round(cb["seconds"] * 1e3 / max(cb["steps"], 1), 3),
-               "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-               "config": {"workload": WORKLOAD, "q_heads": HQ, "kv_heads": HKV, "head_dim": D,
-                          "retrieval_kv_heads": NRET, "S": S, "W": W, "context": CTX, "batch": 1},
-               "cpu_baseline": cb,
-               "e2e": {"value": cb["value"], "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
-               "wall_s": round(time.perf_counter() - t0, 1)}
-        print(json.dumps(res))
-        return 0
+        return run_reference(args)
 
+    import torch
     dist = None
     if world > 1:
         import datetime
@@ -510,25 +702,85 @@ def main():
         import torch.distributed as tdist
         tdist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
         dist = tdist
+    dev = torch.device("cuda", int(os.environ.get("LOCAL_RANK", 0)))
+    torch.cuda.set_device(dev)
+    hbm_peak, tc_peak, tc_sust, peak_src = peaks()
     if args.skip_decode:
-        import torch
-        dev = torch.device("cuda", int(os.environ.get("LOCAL_RANK", 0)))
-        torch.cuda.set_device(dev)
-        _, tc_peak, tc_sust, src = peaks()
         if rank == 0:
-            res = {"prefill": run_prefill(args, dev, tc_peak, tc_sust, src)}
+            res = {"prefill": run_prefill(args, dev, tc_peak, tc_sust, peak_src)}
             if not args.skip_gated:
-                res["gated"] = run_gated(args, dev, tc_peak, tc_sust, src)
+                res["gated"] = run_gated(args, dev, tc_peak, tc_sust, peak_src)
             print(json.dumps(res))
+        if dist:
+            dist.barrier()
+            dist.destroy_process_group()
         return 0
-    res = run_ours(args, rank, world, dist)
-    if rank == 0 and not args.skip_cpu_baseline:
-        res["cpu_baseline"] = oracle_sample(args)
+
+    head = run_headline(args, dev, dist, hbm_peak, peak_src)
+    res = {"metric": METRIC, "value": head["value"], "unit": "GB/s", "n_gpus": world, "steps": args.steps,
+           "warmup": args.warmup, "ms_per_step": head["ms_per_step"], "higher_is_better": True, "scaling": "weak",
+           "vs_baseline": None, "dtype": head["dtype"], "data": "synthetic", "config": head["config"],
+           "us_per_token_layer": head["us_per_token_layer"], "regions": head["regions"],
+           "roofline": head["roofline"], "gpu_launches": head["gpu_launches"], "clocks": head["clocks"],
+           "e2e": head["e2e"]}
+    # the remaining configurations run on rank 0 only (each rank is an independent replica)
+    if rank == 0:
+        if args.workloads != "none":
+            names = sorted(DECODE_WORKLOADS) if args.workloads == "all" else args.workloads.split(",")
+            res["workloads"] = {}
+            for name in names:
+                e = run_workload(name, dev, hbm_peak, peak_src)
+                if not args.skip_cpu_baseline:
+                    cap = 1 << 17 if DECODE_WORKLOADS[name][6] == "int4" else None
+                    e["cpu_baseline"] = oracle_decode_sample(name, args.oracle_seconds, args.oracle_max_steps, cap, dev)
+                res["workloads"][name] = e
+        if not args.skip_prefill:
+            res["prefill"] = run_prefill(args, dev, tc_peak, tc_sust, peak_src)
+        if not args.skip_gated:
+            res["gated"] = run_gated(args, dev, tc_peak, tc_sust, peak_src)
+        if not args.skip_cpu_baseline:
+            res["cpu_baseline"] = oracle_decode_sample(args.workload, args.oracle_seconds, args.oracle_max_steps,
+                                                       device=dev)
     if dist:
         dist.barrier()
         dist.destroy_process_group()
     if rank == 0:
         print(json.dumps(res))
+    return 0
+
+
+def run_reference(args):
+    """The reference arm: the fp64 oracle on the host cores, W warm-up steps then K
+    timed steps; a step is the oracle's decode of `ref_layers` layers of the headline
+    step (one layer's seeded K/V stands in for each of them: the oracle's time does not
+    depend on the values)."""
+    import oracle
+    t_wall = time.perf_counter()
+    od = OracleDecode(args.workload, 1 << 17 if DECODE_WORKLOADS[args.workload][6] == "int4" else None)
+    for _ in range(args.warmup):
+        for _ in range(args.ref_layers):
+            od.step()
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        for _ in range(args.ref_layers):
+            od.step()
+    secs = time.perf_counter() - t0
+    nbytes = args.steps * args.ref_layers * od.nbytes()
+    gbs = nbytes / secs / 1e9
+    Hq, Hkv, nret, ctx, B, layers, fmt = DECODE_WORKLOADS[args.workload]
+    cb = {"value": round(gbs, 3), "unit": "GB/s", "cores": oracle.num_threads(), "kind": "oracle",
+          "sample": f"{args.steps} steps, each the oracle's decode of {args.ref_layers} of the {layers} layers of "
+                    f"the step at context {od.ctx}; {secs:.1f} s wall on {oracle.num_threads()} threads"}
+    res = {"impl": "reference", "metric": METRIC, "value": cb["value"], "unit": "GB/s", "n_gpus": args.gpus,
+           "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(secs * 1e3 / args.steps, 3),
+           "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+           "config": {"workload": args.workload, "q_heads": Hq, "kv_heads": Hkv, "head_dim": D,
+                      "retrieval_kv_heads": nret, "S": S, "W": W, "context": ctx, "batch": B, "layers": layers,
+                      "retrieval_kv": fmt},
+           "cpu_baseline": cb,
+           "e2e": {"value": cb["value"], "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+           "wall_s": round(time.perf_counter() - t_wall, 1)}
+    print(json.dumps(res))
     return 0
 
 
