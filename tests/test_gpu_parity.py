@@ -566,3 +566,63 @@ def test_append_decode_equals_append_then_decode(Hq, Hkv, mask_row, S, W, B, ctx
     want, want_lse = _decode_oracle(q[:, steps - 1:], k, v, mask[0], S, W, T - 1, 1)
     if fmt == "same":
         assert_close(o2.float().cpu().numpy()[:, None], want, dtype, l2.cpu().numpy()[:, None], want_lse, "append_decode")
+
+
+# ------------------------------------------- the 1M-token INT4 stack at its own size
+
+def test_int4_decode_1m_llama3_one_layer():
+    """One layer of the 1M-token Llama-3-8B stack at its own size (32 q / 8 kv heads, 4
+    INT4 retrieval + 4 bf16 streaming heads chosen by the seed, S 16, W 512, batch 1):
+    2^20 - 2 tokens appended, then two decode steps.  Every INT4 code and fp16
+    scale/zero is bit-exact with the oracle's quantiser; the outputs and lse of all 32
+    query heads match the oracle over its own dequantisation.  The oracle runs one KV
+    head (and its four query heads) at a time to bound host memory."""
+    Hq, Hkv, d, S, W, G = 32, 8, 128, 16, 512, 4
+    T, steps = 1 << 20, 2
+    ctx = T - steps
+    mask = inputs.retrieval_mask(1, Hkv, 4, seed=1)
+    q = inputs.randn((1, steps, Hq, d), 150, device=DEV)
+    k = inputs.randn((1, T, Hkv, d), 151, device=DEV)
+    v = inputs.randn((1, T, Hkv, d), 152, device=DEV)
+    cache = DuoCache(1, Hkv, d, mask, S, W, T, q_heads=Hq, dtype=torch.bfloat16, retr_fmt="int4")
+    for t0 in range(0, ctx, 1 << 18):
+        t1 = min(ctx, t0 + (1 << 18))
+        cache.append_kv(0, k[:, t0:t1].contiguous(), v[:, t0:t1].contiguous())
+    outs, lses = [], []
+    for t in range(steps):
+        cache.append_kv(0, k[:, ctx + t:ctx + t + 1].contiguous(), v[:, ctx + t:ctx + t + 1].contiguous())
+        o, l = cache.decode_attention(0, q[:, t].contiguous())
+        outs.append(o.float()[0].cpu().numpy())
+        lses.append(l[0].cpu().numpy())
+    torch.cuda.synchronize()
+    assert cache.device_status() == 0 and cache.len(0) == T
+    got, got_lse = np.stack(outs), np.stack(lses)          # [steps][Hq][d], [steps][Hq]
+    ridx = [g for g in range(Hkv) if mask[0, g]]
+    rk, cap = cache.region(0, duo.DUO_REGION_RETR_K)
+    rv, _ = cache.region(0, duo.DUO_REGION_RETR_V)
+    ks, _ = cache.region(0, duo.DUO_REGION_RETR_KSZ)
+    vs, _ = cache.region(0, duo.DUO_REGION_RETR_VSZ)
+    qb = bits(q)
+    want = np.zeros_like(got, dtype=np.float64)
+    want_lse = np.zeros_like(got_lse, dtype=np.float64)
+    for g in range(Hkv):
+        kg, vg = bits(k[:, :, g:g + 1]), bits(v[:, :, g:g + 1])   # [1][T][1][d] bf16 bits
+        if mask[0, g]:
+            i = ridx.index(g)
+            kd, vd = [], []
+            for src, codes_r, sz_r in ((kg, rk, ks), (vg, rv, vs)):
+                codes, sb, zb = oracle.int4_quantize(src.reshape(T, d))
+                dev_codes = codes_r.view(1, len(ridx), cap, 64)[0, i, :T].cpu().numpy()
+                dev_sz = sz_r.view(torch.int16).view(1, len(ridx), cap, 2)[0, i, :T].cpu().numpy().view(np.uint16)
+                assert np.array_equal(dev_codes, codes), f"INT4 codes of kv head {g} differ"
+                assert np.array_equal(dev_sz[:, 0], sb) and np.array_equal(dev_sz[:, 1], zb), f"scale/zero of {g}"
+                (kd if src is kg else vd).append(oracle.int4_dequantize(codes, sb, zb).reshape(1, T, 1, d))
+            kg, vg = kd[0], vd[0]
+            del kd, vd
+        for t in range(steps):
+            w, l = oracle.attend(qb[:, t:t + 1, g * G:(g + 1) * G], kg[:, :ctx + t + 1], vg[:, :ctx + t + 1],
+                                 [bool(mask[0, g])], S, W, pos0=ctx + t)
+            want[t, g * G:(g + 1) * G] = w[0, 0]
+            want_lse[t, g * G:(g + 1) * G] = l[0, 0]
+        del kg, vg
+    assert_close(got, want, torch.bfloat16, got_lse, want_lse, "int4 decode at 1M")
