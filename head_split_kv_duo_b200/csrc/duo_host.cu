@@ -131,8 +131,17 @@ bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) ==
 
 bool layer_ok(const duo_cache *c, int layer) { return c && layer >= 0 && layer < c->layers; }
 
+// Test controls (duo_debug_launch_controls): process-wide.
+std::atomic<int> g_dry_run{0};
+std::atomic<int64_t> g_fail_countdown{-1};
+
 duo_status ensure_init(duo_cache *c, cudaStream_t st) {
   if (c->initialised) return DUO_OK;
+  if (duo::dry_run()) {  // no device: the count of a full B200 for the work split
+    c->num_sms = 148;
+    c->initialised = true;
+    return DUO_OK;
+  }
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return DUO_ERR_CUDA;
   int sms = 0;
@@ -264,7 +273,8 @@ duo_status duo_append_kv(duo_cache *c, int layer, const void *k, const void *v, 
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   duo_status s = ensure_init(c, st);
   if (s != DUO_OK) return s;
-  if (launch_append(append_params(c, ly, k, v, n), c->dtype, st) != cudaSuccess) return DUO_ERR_CUDA;
+  const AppendParams ap = append_params(c, ly, k, v, n);
+  if (launch_via_hook([&] { return launch_append(ap, c->dtype, st); }) != cudaSuccess) return DUO_ERR_CUDA;
   ly.len += n;
   return DUO_OK;
 }
@@ -282,7 +292,7 @@ duo_status duo_prefill_chunk(duo_cache *c, int layer, const void *q, const void 
   duo_status s = ensure_init(c, st);
   if (s != DUO_OK) return s;
 
-  // 1. stage the streaming history the chunk may see (before the ring is overwritten)
+  // 1. stage the streaming history the chunk may see, in position order
   const int64_t len = ly.len;
   HistParams hp{};
   hp.sk = ly.sk;
@@ -298,13 +308,8 @@ duo_status duo_prefill_chunk(duo_cache *c, int layer, const void *q, const void 
   hp.hs = static_cast<int>(std::min<int64_t>(c->S, len));
   hp.wstart = std::max<int64_t>(c->S, len - c->W + 1);
   hp.hw = static_cast<int>(std::max<int64_t>(0, len - hp.wstart));
-  if (ly.Hs > 0 && hp.hs + hp.hw > 0)
-    if (launch_hist(hp, c->dtype, st) != cudaSuccess) return DUO_ERR_CUDA;
 
-  // 2. append the chunk (retrieval rows are then read back by the attention)
-  if (launch_append(append_params(c, ly, k, v, n), c->dtype, st) != cudaSuccess) return DUO_ERR_CUDA;
-
-  // 3. attention
+  // 2. attention: cached positions from the cache, the chunk from k and v
   PrefillParams p{};
   p.q = static_cast<const char *>(q);
   p.k = static_cast<const char *>(k);
@@ -334,8 +339,22 @@ duo_status duo_prefill_chunk(duo_cache *c, int layer, const void *q, const void 
   p.wstart = hp.wstart;
   p.scale_log2 = c->scale * 1.4426950408889634f;
   p.hm = ly.hm;
-  cudaError_t e = prefill_tc_supported(p, c->dtype) ? launch_prefill_tc(p, st) : launch_prefill_simt(p, c->dtype, st);
-  if (e != cudaSuccess) return DUO_ERR_CUDA;
+  p.mix_alpha = nullptr;
+
+  // 3. append the chunk (the only launch that changes the cache, so it goes last: a call
+  // that fails leaves the cache as it was)
+  const AppendParams ap = append_params(c, ly, k, v, n);
+
+  // every fallible set-up step comes before the first launch
+  const bool tc = prefill_tc_supported(p, c->dtype) && !dry_run();
+  PrefillTcLaunch tl;
+  if (tc && prepare_prefill_tc(p, &tl) != cudaSuccess) return DUO_ERR_CUDA;
+  if (ly.Hs > 0 && hp.hs + hp.hw > 0)
+    if (launch_via_hook([&] { return launch_hist(hp, c->dtype, st); }) != cudaSuccess) return DUO_ERR_CUDA;
+  if (launch_via_hook([&] { return tc ? launch_prefill_tc(tl, st) : launch_prefill_simt(p, c->dtype, st); }) !=
+      cudaSuccess)
+    return DUO_ERR_CUDA;
+  if (launch_via_hook([&] { return launch_append(ap, c->dtype, st); }) != cudaSuccess) return DUO_ERR_CUDA;
   ly.len += n;
   return DUO_OK;
 }
@@ -413,6 +432,19 @@ cudaError_t launch_decode_any(const duo_cache *c, const DecodeParams &p, cudaStr
   return launch_decode(p, c->dtype, int4, st);
 }
 
+// The decode launches of `p`, each through the test controls.
+cudaError_t decode_any(const duo_cache *c, const DecodeParams &p, cudaStream_t st) {
+  if (dry_run() || c->fmt != DUO_KV_INT4_G128 || !decode_int4_tc_supported(p, c->dtype) || p.Hs == 0)
+    return launch_via_hook([&] { return launch_decode_any(c, p, st); });
+  // INT4 layer with streaming heads: two launches (each counted by the test controls)
+  DecodeParams ps = p;
+  ps.Hr = 0;
+  cudaError_t e = launch_via_hook([&] { return launch_decode_tc(ps, c->num_sms, true, st); });
+  if (e != cudaSuccess) return e;
+  DecodeParams pr = p;
+  return launch_via_hook([&] { return launch_decode_int4_tc(pr, c->num_sms, true, st); });
+}
+
 bool decode_args_ok(const void *q, const void *out, const float *lse) {
   return q && out && aligned16(q) && aligned16(out) && !(reinterpret_cast<uintptr_t>(lse) & 3u);
 }
@@ -428,7 +460,7 @@ duo_status duo_decode_attention(duo_cache *c, int layer, const void *q, void *ou
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   duo_status s = ensure_init(c, st);
   if (s != DUO_OK) return s;
-  if (launch_decode_any(c, decode_params(c, ly, q, out, lse), st) != cudaSuccess) return DUO_ERR_CUDA;
+  if (decode_any(c, decode_params(c, ly, q, out, lse), st) != cudaSuccess) return DUO_ERR_CUDA;
   return DUO_OK;
 }
 
@@ -448,17 +480,21 @@ duo_status duo_append_decode(duo_cache *c, int layer, const void *q, const void 
   // One launch where it measured faster (batch 1: 53.1 against 55.4 us per Llama-3 128K
   // layer step); at batch 4 the append kernel ahead of a dependent decode measured
   // faster (169.5 against 177.6 us), so larger batches keep the two launches.
-  if (!int4 && c->B == 1 && decode_tc_supported(p, c->dtype, int4)) {
+  if (!int4 && c->B == 1 && !dry_run() && decode_tc_supported(p, c->dtype, int4)) {
     // one launch: the decode kernel writes the token's rows before it reads their tiles
     p.nk = static_cast<const char *>(k);
     p.nv = static_cast<const char *>(v);
     p.npos = ly.len;
-    if (launch_decode_tc(p, c->num_sms, true, st) != cudaSuccess) return DUO_ERR_CUDA;
-  } else {
-    if (launch_append(append_params(c, ly, k, v, 1), c->dtype, st) != cudaSuccess) return DUO_ERR_CUDA;
-    if (launch_decode_any(c, p, st) != cudaSuccess) return DUO_ERR_CUDA;
+    if (launch_via_hook([&] { return launch_decode_tc(p, c->num_sms, true, st); }) != cudaSuccess) return DUO_ERR_CUDA;
+    ly.len += 1;
+    return DUO_OK;
   }
+  const AppendParams ap = append_params(c, ly, k, v, 1);
+  if (launch_via_hook([&] { return launch_append(ap, c->dtype, st); }) != cudaSuccess) return DUO_ERR_CUDA;
+  // the token is in the cache now: len follows what the cache holds, even if the
+  // attention launch below fails
   ly.len += 1;
+  if (decode_any(c, p, st) != cudaSuccess) return DUO_ERR_CUDA;
   return DUO_OK;
 }
 
@@ -535,7 +571,7 @@ duo_status duo_debug_region(const duo_cache *c, int layer, duo_region which, voi
 
 duo_status duo_get_device_status(duo_cache *c, void *stream) {
   if (!c) return DUO_ERR_INVALID;
-  if (!c->initialised) return DUO_OK;
+  if (!c->initialised || dry_run()) return DUO_OK;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   if (cudaStreamSynchronize(st) != cudaSuccess) return DUO_ERR_CUDA;
   uint32_t word = 0;
@@ -545,4 +581,35 @@ duo_status duo_get_device_status(duo_cache *c, void *stream) {
   return (word & kDevTimeout) ? DUO_ERR_TIMEOUT : DUO_ERR_CUDA;
 }
 
+duo_status duo_debug_launch_controls(int dry_run, int64_t fail_after) {
+  if ((dry_run != 0 && dry_run != 1) || fail_after < -1) return DUO_ERR_INVALID;
+  g_dry_run.store(dry_run);
+  g_fail_countdown.store(fail_after);
+  return DUO_OK;
+}
+
 }  // extern "C"
+
+namespace duo {
+
+bool dry_run() { return g_dry_run.load(std::memory_order_relaxed) != 0; }
+
+bool launch_intercepted(cudaError_t *e) {
+  int64_t left = g_fail_countdown.load(std::memory_order_relaxed);
+  while (left >= 0) {
+    if (g_fail_countdown.compare_exchange_weak(left, left - 1)) {
+      if (left == 0) {  // this launch is the one that fails; nothing is launched
+        *e = cudaErrorLaunchFailure;
+        return true;
+      }
+      break;
+    }
+  }
+  if (dry_run()) {
+    *e = cudaSuccess;
+    return true;
+  }
+  return false;
+}
+
+}  // namespace duo

@@ -2,10 +2,12 @@
 // Not part of the public ABI (include/duo.h is).
 #pragma once
 
+#include <atomic>
 #include <cstddef>
 #include <cstdint>
 #include <vector>
 
+#include <cuda.h>
 #include <cuda_runtime.h>
 
 #include "duo.h"
@@ -112,7 +114,7 @@ struct PrefillParams {
   const char *q, *k, *v;  // q [B][n][Hq][d]; k, v [B][n][Hkv][d] (the chunk)
   char *out;
   float *lse;
-  const char *rk, *rv;    // retrieval cache (chunk already appended)
+  const char *rk, *rv;    // retrieval cache: positions 0 .. len-1 (the chunk itself is read from k, v)
   const char *hk, *hv;    // streaming history staging
   uint32_t *status;
   int B, n, Hq, Hkv, G, D, Hr, Hs, HsMax, S, W;
@@ -121,16 +123,54 @@ struct PrefillParams {
   int64_t wstart;
   float scale_log2;
   HeadMap hm;
+  // gated mixing (identification-phase forward): when set, every output row becomes
+  // mix_alpha[g] * (the row already in out) + (1 - mix_alpha[g]) * (this attention)
+  const float *mix_alpha;
 };
+
+// Raises the dynamic shared-memory limit of `kernel` to `bytes` on the current device.
+// The attribute belongs to the device, so `done` keeps one bit per device (devices 0-63)
+// that already has it; a device past 63 sets it at every call (harmless, only slower).
+template <typename Kernel>
+cudaError_t opt_in_smem(Kernel kernel, int bytes, std::atomic<uint64_t> &done) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  const uint64_t bit = (dev >= 0 && dev < 64) ? (1ull << dev) : 0ull;
+  if (bit && (done.load(std::memory_order_acquire) & bit)) return cudaSuccess;
+  e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (e == cudaSuccess && bit) done.fetch_or(bit, std::memory_order_acq_rel);
+  return e;
+}
 
 // ---- launchers (return cudaSuccess or the launch error) ----
 cudaError_t launch_append(const AppendParams &p, duo_dtype dt, cudaStream_t st);
 cudaError_t launch_hist(const HistParams &p, duo_dtype dt, cudaStream_t st);
 cudaError_t launch_decode(const DecodeParams &p, duo_dtype dt, bool int4, cudaStream_t st);
 cudaError_t launch_prefill_simt(const PrefillParams &p, duo_dtype dt, cudaStream_t st);
-// tcgen05 pre-fill (bf16, d = 128); returns cudaErrorNotSupported when it does not apply
-cudaError_t launch_prefill_tc(const PrefillParams &p, cudaStream_t st);
+// tcgen05 pre-fill (bf16, d = 128).  prepare_prefill_tc does every host step that can
+// fail (tensor maps, the shared-memory limit), so that a call can finish its set-up
+// before its first launch; launch_prefill_tc then only launches.
+struct PrefillTcLaunch {
+  PrefillParams p;
+  CUtensorMap tm_q, tm_kc, tm_vc, tm_kh, tm_vh, tm_kn, tm_vn;
+};
 bool prefill_tc_supported(const PrefillParams &p, duo_dtype dt);
+cudaError_t prepare_prefill_tc(const PrefillParams &p, PrefillTcLaunch *l);
+cudaError_t launch_prefill_tc(const PrefillTcLaunch &l, cudaStream_t st);
+
+// Test controls of the host bookkeeping (duo_debug_launch_controls): true when the launch
+// about to be made must be skipped, with *e the result to report for it.
+bool launch_intercepted(cudaError_t *e);
+bool dry_run();
+// Runs one launch (a callable returning its cudaError_t) unless the test controls
+// intercept it.
+template <typename F>
+cudaError_t launch_via_hook(F &&launch) {
+  cudaError_t e;
+  if (launch_intercepted(&e)) return e;
+  return launch();
+}
 
 // tcgen05 decode (bf16, d = 128, up to 16 query heads per KV head), one CTA per SM.
 // overlap_previous: launch as a programmatic dependent of the previous kernel on the

@@ -559,12 +559,9 @@ cudaError_t launch_t(const DecodeParams &p, cudaStream_t st) {
   using C = RowCfg<T, D>;
   constexpr int STAGE = (INT4 && I4Cfg::STAGE > C::STAGE) ? I4Cfg::STAGE : C::STAGE;
   constexpr int smem = kStages * STAGE + 8 * kStages + 16;
-  static bool attr_set = false;
-  if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(decode_kernel<T, D, QG, INT4>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-    if (e != cudaSuccess) return e;
-    attr_set = true;
-  }
+  static std::atomic<uint64_t> attr{0};
+  const cudaError_t e = opt_in_smem(decode_kernel<T, D, QG, INT4>, smem, attr);
+  if (e != cudaSuccess) return e;
   const int grid = p.n_retr_ctas + p.B * p.Hs * p.nqg;
   decode_kernel<T, D, QG, INT4><<<grid, kThreads, smem, st>>>(p);
   return cudaGetLastError();

@@ -279,7 +279,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_int4_kernel(const __grid_c
       // kernel on the stream; nothing is read from global memory before that kernel has
       // finished (every other read and every write of this grid follows these loads).
       asm volatile("griddepcontrol.wait;" ::: "memory");
-      int prev_item = -1;
+      int prev_item = -1, issued = 0;
       UnitIter it(a, u0);
       for (int j = 0; j < nu; ++j, it.next()) {
         const int s = j % kStages;
@@ -304,7 +304,10 @@ __global__ void __launch_bounds__(kThreads, 1) decode_int4_kernel(const __grid_c
           tc::tma_2d(dst + kStQ, &a.tm_q, 0, qrow, fb);
           tc::tma_2d(dst + kStQ + 2048, &a.tm_q, 64, qrow, fb);
         }
+        ++issued;
       }
+      // after an abort, loads may still be landing: none may outlive the CTA
+      tc::drain_loads(bar(kBarFull), kStages, issued, p.status);
     }
   } else if (warp == 1) {
     // ================= MMA issuer =================
@@ -724,12 +727,10 @@ __global__ void __launch_bounds__(kThreads, 1) decode_int4_kernel(const __grid_c
 
 template <int NQ>
 cudaError_t launch_nq(const Int4DecodeArgs &a, bool overlap_previous, cudaStream_t st) {
-  static bool attr = false;
-  if (!attr) {
-    const cudaError_t e =
-        cudaFuncSetAttribute(decode_int4_kernel<NQ>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemAlloc);
+  static std::atomic<uint64_t> attr{0};
+  {
+    const cudaError_t e = opt_in_smem(decode_int4_kernel<NQ>, kSmemAlloc, attr);
     if (e != cudaSuccess) return e;
-    attr = true;
   }
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(a.num_ctas);

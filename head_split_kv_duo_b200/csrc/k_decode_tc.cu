@@ -173,6 +173,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
       // append warp (retrieval: row npos; streaming: the row's slot)
       const int64_t tile_r = p.npos / kTile, tile_s = (p.npos < p.S ? p.npos : p.S + p.npos % p.W) / kTile;
       bool appended = p.nk == nullptr;
+      int issued = 0;
       UnitIter it(a, u0);
       for (int j = 0; j < nu; ++j, it.next(a)) {
         const int s = j % kStages;
@@ -212,7 +213,10 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
         const int qrow = b * p.Hq + g * G;  // rows beyond this group's G heads are never used
         tc::tma_2d(dst + kStQ, &a.tm_q, 0, qrow, fb);
         tc::tma_2d(dst + kStQ + 2048, &a.tm_q, 64, qrow, fb);
+        ++issued;
       }
+      // after an abort, loads may still be landing: none may outlive the CTA
+      tc::drain_loads(bar(kBarFull), kStages, issued, p.status);
     }
   } else if (warp == 1) {
     // ================= MMA issuer =================
@@ -399,7 +403,8 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
           mbar_expect_tx(bar(kBarMerge), bytes);
           bulk_g2s(sbase, part, bytes, bar(kBarMerge));
         }
-        if (ok) ok = tc::wait_bar(bar(kBarMerge), 0, p.status, abort_flag);
+        // waited for even after an abort (bounded): the copy must not outlive the CTA
+        if (!mbar_wait(bar(kBarMerge), 0, p.status)) ok = false;
         merge_partials<true>(reinterpret_cast<const float *>(smem), nseg, G, b, h0, p.Hq, p.out, p.lse, red + 4 * kN, t, 1);
       } else {
         merge_partials(part, nseg, G, b, h0, p.Hq, p.out, p.lse, red + 4 * kN, t, 1);
@@ -529,11 +534,10 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
 
 template <int NQ>
 cudaError_t launch_nq(const TcDecodeArgs &a, bool overlap_previous, cudaStream_t st) {
-  static bool attr = false;
-  if (!attr) {
-    cudaError_t e = cudaFuncSetAttribute(decode_tc_kernel<NQ>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemAlloc);
+  static std::atomic<uint64_t> attr{0};
+  {
+    const cudaError_t e = opt_in_smem(decode_tc_kernel<NQ>, kSmemAlloc, attr);
     if (e != cudaSuccess) return e;
-    attr = true;
   }
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(a.num_ctas);

@@ -4,7 +4,8 @@
 // Used for fp32 caches and for head_dim 64; bf16 / head_dim 128 pre-fill runs on the
 // tensor cores (k_prefill_tc.cu).  One warp owns one query row (b, r, h) at position
 // i = len + r; lanes split head_dim.  Keys come from two places:
-//   * retrieval heads: the full cache, rows 0..i (the chunk was appended first);
+//   * retrieval heads: the full cache for positions 0..len-1, then the chunk's own rows
+//     0..r from the chunk input (the caller appends the chunk after the attention);
 //   * streaming heads: the staged history (sinks 0..hs-1 and positions wstart..len-1)
 //     and then the chunk's own rows, each filtered by the Lambda mask
 //     (j < S or i - j < W) -- tiles of keys outside the mask are never touched.
@@ -58,7 +59,11 @@ __global__ void __launch_bounds__(256) prefill_simt_kernel(const PrefillParams p
   const int idx = p.hm.kind_idx[g];
   if (p.hm.is_retr[g]) {
     const int64_t base = (static_cast<int64_t>(b) * p.Hr + idx) * p.max_len;
-    for (int64_t j = 0; j <= i; ++j) st.key(p.rk + (base + j) * RB, p.rv + (base + j) * RB, lane);
+    for (int64_t j = 0; j < p.len; ++j) st.key(p.rk + (base + j) * RB, p.rv + (base + j) * RB, lane);
+    for (int t = 0; t <= r; ++t) {  // positions len..i, causal
+      const int64_t off = ((static_cast<int64_t>(b) * p.n + t) * p.Hkv + g) * RB;
+      st.key(p.k + off, p.v + off, lane);
+    }
   } else {
     const int64_t hbase = (static_cast<int64_t>(b) * p.HsMax + idx) * (p.S + p.W);
     // history rows: sinks (always visible) then the window rows still within W of i
@@ -77,8 +82,15 @@ __global__ void __launch_bounds__(256) prefill_simt_kernel(const PrefillParams p
   }
   const float inv = 1.f / st.l;
   char *orow = p.out + ((static_cast<int64_t>(b) * p.n + r) * p.Hq + h) * RB;
+  // gated mixing: blend with the row already in out (each lane reads what it rewrites)
+  const float mixa = p.mix_alpha ? p.mix_alpha[g] : 0.f;
 #pragma unroll
-  for (int e = 0; e < WarpRow<T, D>::E; ++e) Elem<T>::store(orow, lane * WarpRow<T, D>::E + e, st.o[e] * inv);
+  for (int e = 0; e < WarpRow<T, D>::E; ++e) {
+    const int col = lane * WarpRow<T, D>::E + e;
+    float x = st.o[e] * inv;
+    if (p.mix_alpha) x = fmaf(mixa, Elem<T>::load(orow, col) - x, x);
+    Elem<T>::store(orow, col, x);
+  }
   if (lane == 0 && p.lse) p.lse[(static_cast<int64_t>(b) * p.n + r) * p.Hq + h] = (st.m + lg2(st.l)) * kLn2;
 }
 

@@ -3,8 +3,9 @@
 //
 // Operation ("Chunked Pre-filling", masks of "The Full and Streaming Attention
 // Masks"): the n chunk queries at positions len .. len+n-1 attend to
-//   * retrieval heads: every key 0 .. i (causal), read from the full cache, into
-//     which the chunk has already been appended;
+//   * retrieval heads: every key 0 .. i (causal): positions before len from the full
+//     cache, the chunk's own positions from the chunk input (so the attention does not
+//     depend on the chunk having been appended: the caller appends after it);
 //   * streaming heads: the staged history (sinks, then positions wstart..len-1) and
 //     the chunk's own keys, with the Lambda mask j < S or i - j < W.  Key tiles that
 //     hold no visible key for any row of a query tile are never loaded (tile skip).
@@ -26,11 +27,8 @@
 // softmax warps work.
 //
 // Every mbarrier wait is bounded; a wait that runs out latches kDevTimeout in the
-// status word and sets an abort flag so that every role drains and exits.
-#include <cuda.h>
-#include <cudaTypedefs.h>
-
-#include "device_common.cuh"
+// status word and sets an abort flag so that every role drains and exits (the
+// producers first wait, bounded, for the loads they issued).
 #include "tcgen05.cuh"
 
 namespace duo {
@@ -75,127 +73,13 @@ struct TileDesc {
   int y;        // first row in the source
 };
 
-struct TcArgs {
-  PrefillParams p;
-  CUtensorMap tm_q, tm_kc, tm_vc, tm_kh, tm_vh, tm_kn, tm_vn;
-};
-
-// ---------------------------------------------------------------- PTX wrappers
-
-__device__ __forceinline__ void tma_3d(uint32_t dst, const CUtensorMap *m, int x, int y, int z, uint32_t bar) {
-  asm volatile(
-      "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4}], [%5];" ::"r"(dst),
-      "l"(reinterpret_cast<uint64_t>(m)), "r"(x), "r"(y), "r"(z), "r"(bar)
-      : "memory");
-}
-__device__ __forceinline__ void tma_4d(uint32_t dst, const CUtensorMap *m, int x, int y, int z, int w, uint32_t bar) {
-  asm volatile(
-      "cp.async.bulk.tensor.4d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4, %5}], [%6];" ::"r"(dst),
-      "l"(reinterpret_cast<uint64_t>(m)), "r"(x), "r"(y), "r"(z), "r"(w), "r"(bar)
-      : "memory");
-}
-__device__ __forceinline__ void prefetch_map(const CUtensorMap *m) {
-  asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(m)) : "memory");
-}
-
-__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
-__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
-
-__device__ __forceinline__ void tc_commit(uint32_t bar) {
-  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar) : "memory");
-}
-
-__device__ __forceinline__ void tc_mma(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc, uint32_t acc) {
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
-      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(acc)
-      : "memory");
-}
-
-// 32 consecutive fp32 columns of this thread's TMEM lane
-__device__ __forceinline__ void tc_ld32(uint32_t taddr, float (&v)[32]) {
-  uint32_t r[32];
-  asm volatile(
-      "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
-      "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, "
-      "%16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];"
-      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]), "=r"(r[8]),
-        "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]), "=r"(r[16]),
-        "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]),
-        "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
-      : "r"(taddr));
-  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
-#pragma unroll
-  for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
-}
-
-// MMA with A read from tensor memory (bf16 pairs per 32-bit column, K-major)
-__device__ __forceinline__ void tc_mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
-                                          uint32_t acc) {
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
-      "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(acc)
-      : "memory");
-}
-
-// store 32 consecutive fp32 columns of this thread's TMEM lane, and wait for it
-__device__ __forceinline__ void tc_st32(uint32_t taddr, const float (&v)[32]) {
-  asm volatile(
-      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "
-      "{%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16, "
-      "%17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31, %32};" ::"r"(taddr),
-      "r"(__float_as_uint(v[0])), "r"(__float_as_uint(v[1])), "r"(__float_as_uint(v[2])), "r"(__float_as_uint(v[3])),
-      "r"(__float_as_uint(v[4])), "r"(__float_as_uint(v[5])), "r"(__float_as_uint(v[6])), "r"(__float_as_uint(v[7])),
-      "r"(__float_as_uint(v[8])), "r"(__float_as_uint(v[9])), "r"(__float_as_uint(v[10])), "r"(__float_as_uint(v[11])),
-      "r"(__float_as_uint(v[12])), "r"(__float_as_uint(v[13])), "r"(__float_as_uint(v[14])), "r"(__float_as_uint(v[15])),
-      "r"(__float_as_uint(v[16])), "r"(__float_as_uint(v[17])), "r"(__float_as_uint(v[18])), "r"(__float_as_uint(v[19])),
-      "r"(__float_as_uint(v[20])), "r"(__float_as_uint(v[21])), "r"(__float_as_uint(v[22])), "r"(__float_as_uint(v[23])),
-      "r"(__float_as_uint(v[24])), "r"(__float_as_uint(v[25])), "r"(__float_as_uint(v[26])), "r"(__float_as_uint(v[27])),
-      "r"(__float_as_uint(v[28])), "r"(__float_as_uint(v[29])), "r"(__float_as_uint(v[30])), "r"(__float_as_uint(v[31]))
-      : "memory");
-  asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
-}
-__device__ __forceinline__ void named_sync(int id, int n) { asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory"); }
-
-// Shared-memory matrix descriptor, 128-byte swizzle (sm_100 layout: start >> 4 at
-// bit 0, leading byte offset >> 4 at bit 16, stride byte offset >> 4 at bit 32,
-// version 1 at bit 46, swizzle mode 2 at bit 61).
-__device__ __forceinline__ uint64_t sdesc(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
-  return static_cast<uint64_t>((saddr >> 4) & 0x3FFFu) | (static_cast<uint64_t>((lbo >> 4) & 0x3FFFu) << 16) |
-         (static_cast<uint64_t>((sbo >> 4) & 0x3FFFu) << 32) | (1ull << 46) | (2ull << 61);
-}
-
-// Instruction descriptor of kind::f16: fp32 accumulator, bf16 A and B, M 128, N 128.
-constexpr uint32_t idesc_bf16(bool b_mn_major) {
-  return (1u << 4) | (1u << 7) | (1u << 10) | ((b_mn_major ? 1u : 0u) << 16) | ((128u >> 3) << 17) | ((128u >> 4) << 24);
-}
-
-// Bounded wait that also gives up at once after another role aborted; the thread
-// sleeps inside try_wait (woken when the phase completes) instead of spinning.
-__device__ __forceinline__ bool wait_bar(uint32_t bar, uint32_t parity, uint32_t *status, volatile int *abort_flag) {
-  if (mbar_try_wait_ns(bar, parity, 20000)) return true;
-  const unsigned long long t0 = globaltimer();
-#pragma unroll 1
-  while (true) {
-    if (mbar_try_wait_ns(bar, parity, 20000)) return true;
-    if (*abort_flag) return false;
-    if (globaltimer() - t0 > kWaitLimitNs) {
-      flag_status(status, kDevTimeout);
-      *abort_flag = 1;
-      return false;
-    }
-  }
-}
+using TcArgs = PrefillTcLaunch;  // the kernel's parameter block (host-prepared tensor maps)
 
 // ---------------------------------------------------------------- tile lists
 
 struct Plan {
   bool retr;
-  int nt;          // key tiles to visit
+  int nh;          // retrieval: tiles of cached positions 0 .. len-1 (then chunk tiles)
   int64_t q0;      // absolute position of query row 0 of this tile
   int kvrow;       // retrieval: z index of the head in the cache map / streaming: in the hist map
 };
@@ -306,8 +190,11 @@ __device__ __forceinline__ void probabilities(const float (&v)[N], float c, floa
 // A key offset relative to a tile start, clamped to [-1, 127].
 __device__ __forceinline__ int clamp_col(int64_t x) { return static_cast<int>(x < -1 ? -1 : (x > kBN - 1 ? kBN - 1 : x)); }
 
+// Tile j of the query tile's key sequence: retrieval heads visit the cached positions
+// 0 .. len-1 (nh tiles, the last one possibly partial), then the chunk from its start;
+// streaming heads follow their tile list.
 __device__ __forceinline__ TileDesc tile_of(const Plan &pl, const TileDesc *tl, int j) {
-  if (pl.retr) return {0, j * kBN};
+  if (pl.retr) return j < pl.nh ? TileDesc{0, j * kBN} : TileDesc{2, (j - pl.nh) * kBN};
   return tl[j];
 }
 
@@ -316,16 +203,16 @@ __device__ __forceinline__ void load_tile(const TcArgs &a, const TileDesc &t, co
                                           uint32_t dst, uint32_t fb, bool is_k) {
   if (t.src == 0) {
     const CUtensorMap *m = is_k ? &a.tm_kc : &a.tm_vc;
-    tma_3d(dst, m, 0, t.y, pl.kvrow, fb);
-    tma_3d(dst + 16384, m, 64, t.y, pl.kvrow, fb);
+    tc::tma_3d(dst, m, 0, t.y, pl.kvrow, fb);
+    tc::tma_3d(dst + 16384, m, 64, t.y, pl.kvrow, fb);
   } else if (t.src == 1) {
     const CUtensorMap *m = is_k ? &a.tm_kh : &a.tm_vh;
-    tma_3d(dst, m, 0, t.y, pl.kvrow, fb);
-    tma_3d(dst + 16384, m, 64, t.y, pl.kvrow, fb);
+    tc::tma_3d(dst, m, 0, t.y, pl.kvrow, fb);
+    tc::tma_3d(dst + 16384, m, 64, t.y, pl.kvrow, fb);
   } else {
     const CUtensorMap *m = is_k ? &a.tm_kn : &a.tm_vn;
-    tma_4d(dst, m, 0, g, t.y, b, fb);
-    tma_4d(dst + 16384, m, 64, g, t.y, b, fb);
+    tc::tma_4d(dst, m, 0, g, t.y, b, fb);
+    tc::tma_4d(dst + 16384, m, 64, g, t.y, b, fb);
   }
 }
 
@@ -358,6 +245,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) prefill_tc_kernel(const __grid_
   const int r0 = qt * npos;  // first chunk row (position offset) of the block
   Plan pl;
   pl.retr = p.hm.is_retr[g] != 0;
+  pl.nh = pl.retr ? static_cast<int>((p.len + kBN - 1) / kBN) : 0;
   pl.q0 = p.len + r0;
   pl.kvrow = b * (pl.retr ? p.Hr : p.HsMax) + p.hm.kind_idx[g];
 
@@ -369,58 +257,62 @@ __global__ void __launch_bounds__(kTcThreads, 1) prefill_tc_kernel(const __grid_
     *abort_flag = 0;
     int nt;
     if (pl.retr) {
-      const int64_t last = pl.q0 + ((r0 + npos < p.n) ? npos : p.n - r0) - 1;  // last key position needed
-      nt = static_cast<int>(last / kBN) + 1;
+      const int rows = (r0 + npos < p.n) ? r0 + npos : p.n;  // chunk rows 0 .. rows-1 are needed
+      nt = pl.nh + (rows + kBN - 1) / kBN;
     } else {
       nt = streaming_tiles(p, r0, npos, tl);
     }
     *ntiles_sm = nt;
   }
-  if (warp == 1) {  // TMEM: 512 columns
-    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_slot)),
-                 "r"(512));
-    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
-  }
-  tc_fence_before();
+  if (warp == 1) tc::tmem_alloc(smem_u32(tmem_slot), 512);
+  tc::fence_before();
   __syncthreads();
-  tc_fence_after();
+  tc::fence_after();
   const uint32_t tmem = *tmem_slot;
   const int nt = *ntiles_sm;
 
   if (warp == 0) {
     // ================= TMA producer: Q, then the K ring =================
     if (lane == 0) {
-      prefetch_map(&a.tm_q);
+      tc::prefetch_map(&a.tm_q);
       mbar_expect_tx(bar(kBarQ), 32768);
-      tma_4d(sbase + kSmQ, &a.tm_q, 0, g * G, r0, b, bar(kBarQ));  // box: 64 dims x G heads x npos positions
-      tma_4d(sbase + kSmQ + 16384, &a.tm_q, 64, g * G, r0, b, bar(kBarQ));
+      tc::tma_4d(sbase + kSmQ, &a.tm_q, 0, g * G, r0, b, bar(kBarQ));  // box: 64 dims x G heads x npos positions
+      tc::tma_4d(sbase + kSmQ + 16384, &a.tm_q, 64, g * G, r0, b, bar(kBarQ));
+      int issued = 0;
       for (int j = 0; j < nt; ++j) {
         const int s = j % kKStages;
-        if (j >= kKStages && !wait_bar(bar(kBarKEmpty + s), ((j / kKStages) - 1) & 1, p.status, abort_flag)) break;
+        if (j >= kKStages && !tc::wait_bar(bar(kBarKEmpty + s), ((j / kKStages) - 1) & 1, p.status, abort_flag)) break;
         const TileDesc t = tile_of(pl, tl, j);
         const uint32_t dst = sbase + kSmK + s * 32768, fb = bar(kBarKFull + s);
         mbar_expect_tx(fb, 32768);
         load_tile(a, t, pl, g, b, dst, fb, true);
+        ++issued;
       }
+      // nothing may still be landing in shared memory when the CTA ends
+      mbar_wait(bar(kBarQ), 0, p.status);
+      tc::drain_loads(bar(kBarKFull), kKStages, issued, p.status);
     }
   } else if (warp == kVWarp) {
     // ================= TMA producer: the V ring =================
     if (lane == 0) {
+      int issued = 0;
       for (int j = 0; j < nt; ++j) {
         const int s = j % kVStages;
-        if (j >= kVStages && !wait_bar(bar(kBarVEmpty + s), ((j / kVStages) - 1) & 1, p.status, abort_flag)) break;
+        if (j >= kVStages && !tc::wait_bar(bar(kBarVEmpty + s), ((j / kVStages) - 1) & 1, p.status, abort_flag)) break;
         const TileDesc t = tile_of(pl, tl, j);
         const uint32_t dst = sbase + kSmV + s * 32768, fb = bar(kBarVFull + s);
         mbar_expect_tx(fb, 32768);
         load_tile(a, t, pl, g, b, dst, fb, false);
+        ++issued;
       }
+      tc::drain_loads(bar(kBarVFull), kVStages, issued, p.status);
     }
   } else if (warp == 1) {
     // ================= MMA issuer =================
     if (lane == 0) {
-      constexpr uint32_t kIdS = idesc_bf16(false);
-      constexpr uint32_t kIdPV = idesc_bf16(true);
-      bool ok = wait_bar(bar(kBarQ), 0, p.status, abort_flag);
+      constexpr uint32_t kIdS = tc::idesc_bf16(kBM, kBN, false, false);
+      constexpr uint32_t kIdPV = tc::idesc_bf16(kBM, kD, false, true);
+      bool ok = tc::wait_bar(bar(kBarQ), 0, p.status, abort_flag);
       auto issue_pv = [&](int jj) {
         // O += P_jj V_jj : K = 128 keys in 8 steps of 16; P from TMEM (bf16 pairs, K-major),
         // V from shared memory (d contiguous, MN-major)
@@ -428,40 +320,40 @@ __global__ void __launch_bounds__(kTcThreads, 1) prefill_tc_kernel(const __grid_
         const uint32_t vbase = sbase + kSmV + sv * 32768;
         const uint32_t pcol = tmem + kTmP + (jj & 1) * 64;
         for (int kk = 0; kk < 8; ++kk) {
-          const uint64_t bd = sdesc(vbase + kk * 2048, 16384, 1024);
-          tc_mma_ts(tmem + kTmO, pcol + kk * 8, bd, kIdPV, (jj > 0 || kk > 0) ? 1u : 0u);
+          const uint64_t bd = tc::sdesc(vbase + kk * 2048, 16384, 1024);
+          tc::mma_ts(tmem + kTmO, pcol + kk * 8, bd, kIdPV, (jj > 0 || kk > 0) ? 1u : 0u);
         }
-        tc_commit(bar(kBarOFull));
-        tc_commit(bar(kBarVEmpty + sv));
+        tc::commit(bar(kBarOFull));
+        tc::commit(bar(kBarVEmpty + sv));
       };
       for (int j = 0; j < nt && ok; ++j) {
         const int sk = j % kKStages;
-        if (!wait_bar(bar(kBarKFull + sk), (j / kKStages) & 1, p.status, abort_flag)) { ok = false; break; }
-        if (j >= 2 && !wait_bar(bar(kBarSFree + (j & 1)), ((j - 2) >> 1) & 1, p.status, abort_flag)) { ok = false; break; }
-        tc_fence_after();
+        if (!tc::wait_bar(bar(kBarKFull + sk), (j / kKStages) & 1, p.status, abort_flag)) { ok = false; break; }
+        if (j >= 2 && !tc::wait_bar(bar(kBarSFree + (j & 1)), ((j - 2) >> 1) & 1, p.status, abort_flag)) { ok = false; break; }
+        tc::fence_after();
         // S_j = Q K_j^T : K = d 128 in 8 steps of 16; Q and K are K-major
         const uint32_t kbase = sbase + kSmK + sk * 32768;
         for (int kk = 0; kk < 8; ++kk) {
           const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
-          tc_mma(tmem + kTmS + (j & 1) * 128, sdesc(sbase + kSmQ + off, 16, 1024), sdesc(kbase + off, 16, 1024), kIdS,
-                 kk > 0 ? 1u : 0u);
+          tc::mma_ss(tmem + kTmS + (j & 1) * 128, tc::sdesc(sbase + kSmQ + off, 16, 1024),
+                     tc::sdesc(kbase + off, 16, 1024), kIdS, kk > 0 ? 1u : 0u);
         }
-        tc_commit(bar(kBarSFull + (j & 1)));
-        tc_commit(bar(kBarKEmpty + sk));
+        tc::commit(bar(kBarSFull + (j & 1)));
+        tc::commit(bar(kBarKEmpty + sk));
         if (j >= 1) {
-          if (!wait_bar(bar(kBarPFull + ((j - 1) & 1)), ((j - 1) >> 1) & 1, p.status, abort_flag)) { ok = false; break; }
-          if (!wait_bar(bar(kBarVFull + ((j - 1) % kVStages)), ((j - 1) / kVStages) & 1, p.status, abort_flag)) { ok = false; break; }
-          tc_fence_after();
+          if (!tc::wait_bar(bar(kBarPFull + ((j - 1) & 1)), ((j - 1) >> 1) & 1, p.status, abort_flag)) { ok = false; break; }
+          if (!tc::wait_bar(bar(kBarVFull + ((j - 1) % kVStages)), ((j - 1) / kVStages) & 1, p.status, abort_flag)) { ok = false; break; }
+          tc::fence_after();
           issue_pv(j - 1);
         }
       }
-      if (ok && nt > 0 && wait_bar(bar(kBarPFull + ((nt - 1) & 1)), ((nt - 1) >> 1) & 1, p.status, abort_flag) &&
-          wait_bar(bar(kBarVFull + ((nt - 1) % kVStages)), ((nt - 1) / kVStages) & 1, p.status, abort_flag)) {
-        tc_fence_after();
+      if (ok && nt > 0 && tc::wait_bar(bar(kBarPFull + ((nt - 1) & 1)), ((nt - 1) >> 1) & 1, p.status, abort_flag) &&
+          tc::wait_bar(bar(kBarVFull + ((nt - 1) % kVStages)), ((nt - 1) / kVStages) & 1, p.status, abort_flag)) {
+        tc::fence_after();
         issue_pv(nt - 1);
       }
       // drain: every MMA this thread issued has completed before TMEM is freed
-      tc_commit(bar(kBarDrain));
+      tc::commit(bar(kBarDrain));
       mbar_wait(bar(kBarDrain), 0, p.status);
     }
   } else {
@@ -489,8 +381,8 @@ __global__ void __launch_bounds__(kTcThreads, 1) prefill_tc_kernel(const __grid_
       // Mask of this row over the tile's 128 keys, as three column bounds: key col is
       // visible iff col <= hi && (col < sink_c || col > win_c).
       int hi, sink_c = kBN, win_c = -1;
-      if (t.src == 0) {  // retrieval cache: positions y + col, causal only
-        hi = clamp_col(i - t.y);
+      if (t.src == 0) {  // retrieval cache: positions y + col < len, all before the query
+        hi = clamp_col(p.len - 1 - t.y);
       } else {
         int64_t base, sink_rel, win_rel;
         int valid;
@@ -507,17 +399,19 @@ __global__ void __launch_bounds__(kTcThreads, 1) prefill_tc_kernel(const __grid_
           win_rel = i - p.W - p.wstart + p.hs - t.y;
         }
         hi = min(hi, valid - 1);
-        sink_c = static_cast<int>(sink_rel < 0 ? 0 : (sink_rel > kBN ? kBN : sink_rel));
-        win_c = clamp_col(win_rel);
+        if (!pl.retr) {  // retrieval heads see every key up to the query (causal only)
+          sink_c = static_cast<int>(sink_rel < 0 ? 0 : (sink_rel > kBN ? kBN : sink_rel));
+          win_c = clamp_col(win_rel);
+        }
       }
       const bool full_vis = hi >= kBN - 1 && (sink_c >= kBN || win_c < 0);
 
-      if (ok) ok = wait_bar(bar(kBarSFull + (j & 1)), (j >> 1) & 1, p.status, abort_flag);
-      tc_fence_after();
+      if (ok) ok = tc::wait_bar(bar(kBarSFull + (j & 1)), (j >> 1) & 1, p.status, abort_flag);
+      tc::fence_after();
       // this thread's kCols logits of S_j, then the S buffer is released
       float v[kCols];
-      tc_ld32(lane_base + kTmS + (j & 1) * 128 + part * kCols, v);
-      tc_fence_before();
+      tc::ld<kCols>(lane_base + kTmS + (j & 1) * 128 + part * kCols, v);
+      tc::fence_before();
       mbar_arrive(bar(kBarSFree + (j & 1)));
       if (!full_vis) {
 #pragma unroll
@@ -534,7 +428,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) prefill_tc_kernel(const __grid_
       for (int e = 8; e < kCols; e += 2) mx4[(e >> 1) & 3] = fmax3(mx4[(e >> 1) & 3], v[e], v[e + 1]);
       float mx = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3]));
       xch[((j & 1) * kSplit + part) * kBM + row] = mx;
-      named_sync(1, kSoft);
+      tc::named_sync(1, kSoft);
 #pragma unroll
       for (int o = 1; o < kSplit; ++o) mx = fmaxf(mx, xch[((j & 1) * kSplit + ((part + o) % kSplit)) * kBM + row]);
       const float tmax = mx * c;  // -inf when nothing in the tile is visible
@@ -548,14 +442,14 @@ __global__ void __launch_bounds__(kTcThreads, 1) prefill_tc_kernel(const __grid_
       bool waited = false;
       if (j >= 1 && __any_sync(0xffffffffu, need)) {
         // rescale this thread's kCols columns of O once P_{j-1} V_{j-1} has landed
-        if (ok) ok = wait_bar(bar(kBarOFull), (j - 1) & 1, p.status, abort_flag);
-        tc_fence_after();
+        if (ok) ok = tc::wait_bar(bar(kBarOFull), (j - 1) & 1, p.status, abort_flag);
+        tc::fence_after();
         float w[kCols];
         const uint32_t oa = lane_base + kTmO + part * kCols;
-        tc_ld32(oa, w);
+        tc::ld<kCols>(oa, w);
 #pragma unroll
         for (int e = 0; e < kCols; ++e) w[e] *= alpha;
-        tc_st32(oa, w);
+        tc::st32(oa, w);
         waited = true;
       }
       // probabilities (masked logits are -inf and give 0), row sum, bf16 pairs of P_j
@@ -570,35 +464,47 @@ __global__ void __launch_bounds__(kTcThreads, 1) prefill_tc_kernel(const __grid_
       tc::st_wait();
       // one wait per P V product, in order (here unless the rescale already waited)
       if (j >= 1 && !waited) {
-        if (ok) ok = wait_bar(bar(kBarOFull), (j - 1) & 1, p.status, abort_flag);
+        if (ok) ok = tc::wait_bar(bar(kBarOFull), (j - 1) & 1, p.status, abort_flag);
       }
       l += rsum;
-      tc_fence_before();
+      tc::fence_before();
       mbar_arrive(bar(kBarPFull + (j & 1)));
     }
     // the last product, then the row's normaliser from all parts
-    if (nt > 0 && ok) ok = wait_bar(bar(kBarOFull), (nt - 1) & 1, p.status, abort_flag);
-    tc_fence_after();
+    if (nt > 0 && ok) ok = tc::wait_bar(bar(kBarOFull), (nt - 1) & 1, p.status, abort_flag);
+    tc::fence_after();
     float *xl = xch + 2 * kSplit * kBM;  // [part][row]
     xl[part * kBM + row] = l;
-    named_sync(1, kSoft);
+    tc::named_sync(1, kSoft);
     float lrow = 0.f;
 #pragma unroll
     for (int o = 0; o < kSplit; ++o) lrow += xl[o * kBM + row];
-    // epilogue: normalise and store this thread's kCols dims of the row (bf16) and its lse
+    // epilogue: normalise and store this thread's kCols dims of the row (bf16) and its lse;
+    // in gated mixing, blend with the row already in out
     const bool store = r0 + rpos < p.n;
     char *orow = p.out + ((static_cast<int64_t>(b) * p.n + r0 + rpos) * p.Hq + h) * (kD * 2) + part * (kCols * 2);
     const float inv = 1.f / lrow;
+    const float mixa = p.mix_alpha ? p.mix_alpha[g] : 0.f;
     {
       float w[kCols];
-      tc_ld32(lane_base + kTmO + part * kCols, w);
+      tc::ld<kCols>(lane_base + kTmO + part * kCols, w);
       if (store) {
 #pragma unroll
         for (int q = 0; q < kCols / 8; ++q) {
+          float x[8];
+#pragma unroll
+          for (int e = 0; e < 8; ++e) x[e] = w[8 * q + e] * inv;
+          if (p.mix_alpha) {
+            const uint4 old = *reinterpret_cast<const uint4 *>(orow + q * 16);
+            float f[8];
+            Elem<__nv_bfloat16>::unpack(old, f);
+#pragma unroll
+            for (int e = 0; e < 8; ++e) x[e] = fmaf(mixa, f[e] - x[e], x[e]);
+          }
           uint32_t wd[4];
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
-            const __nv_bfloat162 pb = __floats2bfloat162_rn(w[8 * q + 2 * e] * inv, w[8 * q + 2 * e + 1] * inv);
+            const __nv_bfloat162 pb = __floats2bfloat162_rn(x[2 * e], x[2 * e + 1]);
             wd[e] = *reinterpret_cast<const uint32_t *>(&pb);
           }
           *reinterpret_cast<uint4 *>(orow + q * 16) = make_uint4(wd[0], wd[1], wd[2], wd[3]);
@@ -608,44 +514,10 @@ __global__ void __launch_bounds__(kTcThreads, 1) prefill_tc_kernel(const __grid_
     if (store && part == 0 && p.lse) p.lse[(static_cast<int64_t>(b) * p.n + r0 + rpos) * p.Hq + h] = (m + lg2(lrow)) * kLn2;
   }
 
-  tc_fence_before();
+  tc::fence_before();
   __syncthreads();
-  tc_fence_after();
-  if (warp == 1) asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(512));
-}
-
-// ---------------------------------------------------------------- host side
-
-PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
-  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-  static bool tried = false;
-  if (!tried) {
-    tried = true;
-    void *ptr = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
-  }
-  return fn;
-}
-
-// bf16 map of `rank` dims (innermost first), box {64, ...}, 128-byte swizzle.
-bool make_map(CUtensorMap *m, const void *base, int rank, const uint64_t *dims, const uint64_t *strides_bytes,
-              const uint32_t *box) {
-  auto fn = encode_fn();
-  if (!fn) return false;
-  cuuint64_t gd[5], gs[4];
-  cuuint32_t bx[5], es[5];
-  for (int r = 0; r < rank; ++r) {
-    gd[r] = dims[r];
-    bx[r] = box[r];
-    es[r] = 1;
-  }
-  for (int r = 0; r < rank - 1; ++r) gs[r] = strides_bytes[r];
-  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, rank, const_cast<void *>(base), gd, gs, bx, es,
-            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+  tc::fence_after();
+  if (warp == 1) tc::tmem_free(tmem, 512);
 }
 
 }  // namespace
@@ -653,7 +525,7 @@ bool make_map(CUtensorMap *m, const void *base, int rank, const uint64_t *dims, 
 bool prefill_tc_supported(const PrefillParams &p, duo_dtype dt) {
   if (dt != DUO_BF16 || p.D != kD) return false;
   if (p.G < 1 || p.G > kBM || (p.G & (p.G - 1)) != 0) return false;  // the group must tile 128 rows
-  if (encode_fn() == nullptr) return false;
+  if (tc::encode_fn() == nullptr) return false;
   // streaming tile list must fit: history tiles + window tiles + a sink tile
   const int hist_tiles = (p.hs + p.hw + kBN - 1) / kBN;
   const int win_tiles = (p.W + 2 * kBN - 2) / kBN + 1;
@@ -661,49 +533,55 @@ bool prefill_tc_supported(const PrefillParams &p, duo_dtype dt) {
   return hist_tiles + win_tiles + sink_tiles <= kMaxStrmTiles;
 }
 
-cudaError_t launch_prefill_tc(const PrefillParams &p, cudaStream_t st) {
-  static TcArgs a;  // host staging only; copied into the launch's parameter buffer
+cudaError_t prepare_prefill_tc(const PrefillParams &p, PrefillTcLaunch *l) {
+  TcArgs &a = *l;
   a.p = p;
   const uint64_t row = kD * 2;
+  const CUtensorMapDataType bf = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+  const CUtensorMapSwizzle sw = CU_TENSOR_MAP_SWIZZLE_128B;
+  // maps of sources this launch never reads (no cached positions, no streaming history)
+  // still need a valid description: they point at the chunk input
+  const void *rk = p.len > 0 && p.Hr > 0 ? p.rk : p.k, *rv = p.len > 0 && p.Hr > 0 ? p.rv : p.v;
+  const void *hk = p.hs + p.hw > 0 ? p.hk : p.k, *hv = p.hs + p.hw > 0 ? p.hv : p.v;
   bool ok = true;
   {  // q [B][n][Hq][d]; box = 64 dims x G heads x 128/G positions (one GQA group)
     const uint64_t d[4] = {kD, static_cast<uint64_t>(p.Hq), static_cast<uint64_t>(p.n), static_cast<uint64_t>(p.B)};
     const uint64_t s[3] = {row, row * p.Hq, row * p.Hq * p.n};
     const uint32_t bx[4] = {64, static_cast<uint32_t>(p.G), static_cast<uint32_t>(kBM / p.G), 1};
-    ok &= make_map(&a.tm_q, p.q, 4, d, s, bx);
+    ok &= tc::make_map(&a.tm_q, bf, p.q, 4, d, s, bx, sw);
   }
   {  // chunk k, v [B][n][Hkv][d]
     const uint64_t d[4] = {kD, static_cast<uint64_t>(p.Hkv), static_cast<uint64_t>(p.n), static_cast<uint64_t>(p.B)};
     const uint64_t s[3] = {row, row * p.Hkv, row * p.Hkv * p.n};
     const uint32_t bx[4] = {64, 1, kBN, 1};
-    ok &= make_map(&a.tm_kn, p.k, 4, d, s, bx);
-    ok &= make_map(&a.tm_vn, p.v, 4, d, s, bx);
+    ok &= tc::make_map(&a.tm_kn, bf, p.k, 4, d, s, bx, sw);
+    ok &= tc::make_map(&a.tm_vn, bf, p.v, 4, d, s, bx, sw);
   }
   {  // retrieval cache [B*Hr][cap][d]
     const uint64_t d[3] = {kD, static_cast<uint64_t>(p.max_len), static_cast<uint64_t>(p.B) * (p.Hr > 0 ? p.Hr : 1)};
     const uint64_t s[2] = {row, row * p.max_len};
     const uint32_t bx[3] = {64, kBN, 1};
-    ok &= make_map(&a.tm_kc, p.rk, 3, d, s, bx);
-    ok &= make_map(&a.tm_vc, p.rv, 3, d, s, bx);
+    ok &= tc::make_map(&a.tm_kc, bf, rk, 3, d, s, bx, sw);
+    ok &= tc::make_map(&a.tm_vc, bf, rv, 3, d, s, bx, sw);
   }
   {  // streaming history [B*HsMax][S+W][d]
     const uint64_t d[3] = {kD, static_cast<uint64_t>(p.S + p.W), static_cast<uint64_t>(p.B) * (p.HsMax > 0 ? p.HsMax : 1)};
     const uint64_t s[2] = {row, row * (p.S + p.W)};
     const uint32_t bx[3] = {64, kBN, 1};
-    ok &= make_map(&a.tm_kh, p.hk, 3, d, s, bx);
-    ok &= make_map(&a.tm_vh, p.hv, 3, d, s, bx);
+    ok &= tc::make_map(&a.tm_kh, bf, hk, 3, d, s, bx, sw);
+    ok &= tc::make_map(&a.tm_vh, bf, hv, 3, d, s, bx, sw);
   }
   if (!ok) return cudaErrorInvalidValue;
-  static bool attr = false;
-  if (!attr) {
-    cudaError_t e = cudaFuncSetAttribute(prefill_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemAlloc);
-    if (e != cudaSuccess) return e;
-    attr = true;
-  }
+  static std::atomic<uint64_t> attr{0};
+  return opt_in_smem(prefill_tc_kernel, kSmemAlloc, attr);
+}
+
+cudaError_t launch_prefill_tc(const PrefillTcLaunch &l, cudaStream_t st) {
+  const PrefillParams &p = l.p;
   const int npos = kBM / p.G;
   const int ntq = (p.n + npos - 1) / npos;
   const int grid = ntq * p.B * p.Hkv;
-  prefill_tc_kernel<<<grid, kTcThreads, kSmemAlloc, st>>>(a);
+  prefill_tc_kernel<<<grid, kTcThreads, kSmemAlloc, st>>>(l);
   return cudaGetLastError();
 }
 

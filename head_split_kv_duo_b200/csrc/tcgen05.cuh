@@ -1,4 +1,5 @@
-// tcgen05.cuh -- sm_100a tensor-core plumbing shared by the tcgen05 decode kernels:
+// tcgen05.cuh -- sm_100a tensor-core plumbing shared by the tcgen05 kernels (decode and
+// pre-fill):
 // tiled TMA loads, tensor-memory loads and stores, MMA issue and commit, shared-memory
 // matrix descriptors (128-byte swizzle), instruction descriptors, bounded barrier
 // waits, and the host-side tensor-map encoder.
@@ -24,6 +25,15 @@ __device__ __forceinline__ void tma_3d(uint32_t dst, const CUtensorMap *m, int x
       "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4}], [%5];" ::"r"(dst),
       "l"(reinterpret_cast<uint64_t>(m)), "r"(x), "r"(y), "r"(z), "r"(bar)
       : "memory");
+}
+__device__ __forceinline__ void tma_4d(uint32_t dst, const CUtensorMap *m, int x, int y, int z, int w, uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.4d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4, %5}], [%6];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(m)), "r"(x), "r"(y), "r"(z), "r"(w), "r"(bar)
+      : "memory");
+}
+__device__ __forceinline__ void prefetch_map(const CUtensorMap *m) {
+  asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(m)) : "memory");
 }
 
 // ---- ordering between the generic proxy, the async proxy and tcgen05 operations ----
@@ -83,7 +93,7 @@ constexpr uint32_t idesc_bf16(int M, int N, bool a_mn_major, bool b_mn_major) {
 }
 
 // ---- tensor memory <-> registers (warp-collective; a warp reaches lanes 32*(warp%4)..+31) ----
-// N (1, 2, 4, 8 or 16) consecutive 32-bit columns of this thread's lane
+// N (1, 2, 4, 8, 16 or 32) consecutive 32-bit columns of this thread's lane
 template <int N>
 __device__ __forceinline__ void ld(uint32_t taddr, float (&v)[N]) {
   uint32_t r[N];
@@ -99,8 +109,18 @@ __device__ __forceinline__ void ld(uint32_t taddr, float (&v)[N]) {
     asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];"
                  : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7])
                  : "r"(taddr));
+  } else if constexpr (N == 32) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+        "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, "
+        "%16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]), "=r"(r[8]),
+          "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]), "=r"(r[16]),
+          "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]),
+          "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+        : "r"(taddr));
   } else {
-    static_assert(N == 16, "1, 2, 4, 8 or 16 columns");
+    static_assert(N == 16, "1, 2, 4, 8, 16 or 32 columns");
     asm volatile(
         "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
         "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15}, [%16];"
@@ -165,6 +185,23 @@ __device__ __forceinline__ void st16(uint32_t taddr, const uint32_t (&v)[16]) {
       : "memory");
 }
 __device__ __forceinline__ void st_wait() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
+// 32 consecutive fp32 columns of this thread's lane, stored and waited for
+__device__ __forceinline__ void st32(uint32_t taddr, const float (&v)[32]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "
+      "{%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16, "
+      "%17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31, %32};" ::"r"(taddr),
+      "r"(__float_as_uint(v[0])), "r"(__float_as_uint(v[1])), "r"(__float_as_uint(v[2])), "r"(__float_as_uint(v[3])),
+      "r"(__float_as_uint(v[4])), "r"(__float_as_uint(v[5])), "r"(__float_as_uint(v[6])), "r"(__float_as_uint(v[7])),
+      "r"(__float_as_uint(v[8])), "r"(__float_as_uint(v[9])), "r"(__float_as_uint(v[10])), "r"(__float_as_uint(v[11])),
+      "r"(__float_as_uint(v[12])), "r"(__float_as_uint(v[13])), "r"(__float_as_uint(v[14])), "r"(__float_as_uint(v[15])),
+      "r"(__float_as_uint(v[16])), "r"(__float_as_uint(v[17])), "r"(__float_as_uint(v[18])), "r"(__float_as_uint(v[19])),
+      "r"(__float_as_uint(v[20])), "r"(__float_as_uint(v[21])), "r"(__float_as_uint(v[22])), "r"(__float_as_uint(v[23])),
+      "r"(__float_as_uint(v[24])), "r"(__float_as_uint(v[25])), "r"(__float_as_uint(v[26])), "r"(__float_as_uint(v[27])),
+      "r"(__float_as_uint(v[28])), "r"(__float_as_uint(v[29])), "r"(__float_as_uint(v[30])), "r"(__float_as_uint(v[31]))
+      : "memory");
+  asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+}
 
 // ---- CTA-level helpers ----
 __device__ __forceinline__ void named_sync(int id, int n) { asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory"); }
@@ -201,28 +238,39 @@ __device__ __forceinline__ bool wait_bar(uint32_t bar, uint32_t parity, uint32_t
   }
 }
 
+// Before a producer thread exits: waits, bounded but regardless of an abort, until the
+// last loads it issued into a ring of `stages` stages have landed, so that no async copy
+// still writes this CTA's shared memory when it ends.  Load j went to stage j % stages
+// and completes phase j / stages of that stage's full barrier (at full_bar0 + 8 * stage);
+// no later phase can complete, as the producer issued nothing after it.
+__device__ __forceinline__ void drain_loads(uint32_t full_bar0, int stages, int issued, uint32_t *status) {
+#pragma unroll 1
+  for (int j = issued > stages ? issued - stages : 0; j < issued; ++j)
+    mbar_wait(full_bar0 + 8u * static_cast<uint32_t>(j % stages), static_cast<uint32_t>(j / stages) & 1u, status);
+}
+
 // ---- host: tensor maps ----
+// cuTensorMapEncodeTiled from the driver (the runtime hands out the entry point), or
+// nullptr when the driver does not offer it; looked up once per process.
 inline PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
-  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-  static bool tried = false;
-  if (!tried) {
-    tried = true;
+  static const PFN_cuTensorMapEncodeTiled_v12000 fn = []() -> PFN_cuTensorMapEncodeTiled_v12000 {
     void *ptr = nullptr;
     cudaDriverEntryPointQueryResult q;
     if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
         q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
-  }
+      return reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+    return nullptr;
+  }();
   return fn;
 }
-// A tiled map of `rank` (<= 3) dimensions: dims innermost first, strides in bytes of
+// A tiled map of `rank` (<= 5) dimensions: dims innermost first, strides in bytes of
 // dimensions 1.., box sizes in elements; out-of-range elements read as zero.
 inline bool make_map(CUtensorMap *m, CUtensorMapDataType type, const void *base, int rank, const uint64_t *dims,
                      const uint64_t *strides, const uint32_t *box, CUtensorMapSwizzle swizzle) {
   auto fn = encode_fn();
-  if (!fn || rank < 1 || rank > 3) return false;
-  cuuint64_t gd[3], gs[2];
-  cuuint32_t bx[3], es[3] = {1, 1, 1};
+  if (!fn || rank < 1 || rank > 5) return false;
+  cuuint64_t gd[5], gs[4];
+  cuuint32_t bx[5], es[5] = {1, 1, 1, 1, 1};
   for (int r = 0; r < rank; ++r) {
     gd[r] = dims[r];
     bx[r] = box[r];

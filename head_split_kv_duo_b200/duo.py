@@ -76,11 +76,11 @@ def lib() -> ctypes.CDLL:
             L.duo_get_device_status.argtypes = [vp, vp]
             L.duo_status_str.restype = ctypes.c_char_p
             L.duo_status_str.argtypes = [i32]
-            L.duo_gated_workspace_bytes.restype = ctypes.c_size_t
-            L.duo_gated_workspace_bytes.argtypes = [i32, i32, i32, i32, i32, i32, i32, i32]
             L.duo_gated_attention.restype = i32
             L.duo_gated_attention.argtypes = [vp, vp, vp, i32, i32, i32, i32, i32, i32, vp, i32, i32,
-                                              ctypes.c_float, vp, vp, ctypes.c_size_t, vp]
+                                              ctypes.c_float, vp, vp]
+            L.duo_debug_launch_controls.restype = i32
+            L.duo_debug_launch_controls.argtypes = [i32, i64]
             _lib = L
     return _lib
 
@@ -176,15 +176,14 @@ def duo_get_device_status(handle, stream=None) -> int:
     return lib().duo_get_device_status(handle, _ptr(stream))
 
 
-def duo_gated_workspace_bytes(batch, seq_len, q_heads, kv_heads, head_dim, dtype, S, W) -> int:
-    return lib().duo_gated_workspace_bytes(batch, seq_len, q_heads, kv_heads, head_dim, dtype, S, W)
-
-
 def duo_gated_attention(q, k, v, batch, seq_len, q_heads, kv_heads, head_dim, dtype, alpha, S, W, softmax_scale,
-                        out, workspace, workspace_bytes, stream=None) -> int:
+                        out, stream=None) -> int:
     return lib().duo_gated_attention(_ptr(q), _ptr(k), _ptr(v), batch, seq_len, q_heads, kv_heads, head_dim, dtype,
-                                     _ptr(alpha), S, W, float(softmax_scale), _ptr(out), _ptr(workspace),
-                                     workspace_bytes, _ptr(stream))
+                                     _ptr(alpha), S, W, float(softmax_scale), _ptr(out), _ptr(stream))
+
+
+def duo_debug_launch_controls(dry_run: int, fail_after: int) -> int:
+    return lib().duo_debug_launch_controls(int(dry_run), int(fail_after))
 
 
 # ---- torch-owned cache ----
@@ -319,8 +318,7 @@ class DuoCache:
 
 def gated_attention(q, k, v, alpha, S, W, softmax_scale=0.0, out=None, stream=None):
     """Gated mixed attention over whole sequences (duo_gated_attention): q [B][L][Hq][d],
-    k, v [B][L][Hkv][d] (bf16 or fp32, CUDA), alpha [Hkv] fp32 on the same device.
-    The workspace is a torch buffer allocated here."""
+    k, v [B][L][Hkv][d] (bf16 or fp32, CUDA), alpha [Hkv] fp32 on the same device."""
     B, L, Hq, d = q.shape
     Hkv = k.shape[2]
     dt = {torch.bfloat16: DUO_BF16, torch.float32: DUO_FP32}.get(q.dtype)
@@ -329,15 +327,9 @@ def gated_attention(q, k, v, alpha, S, W, softmax_scale=0.0, out=None, stream=No
     for t in (q, k, v, alpha):
         if not t.is_contiguous() or t.device != q.device:
             raise DuoError(DUO_ERR_INVALID, "gated_attention inputs must be contiguous on one device")
-    nbytes = duo_gated_workspace_bytes(B, L, Hq, Hkv, d, dt, S, W)
-    if nbytes == 0:
-        raise DuoError(DUO_ERR_INVALID, "gated_attention shape")
-    ws = torch.empty(nbytes + 256, dtype=torch.uint8, device=q.device)
-    off = (-ws.data_ptr()) % 256
     if out is None:
         out = torch.empty_like(q)
-    st = duo_gated_attention(q, k, v, B, L, Hq, Hkv, d, dt, alpha, S, W, softmax_scale, out, ws[off:], nbytes,
-                             _stream_ptr(stream))
+    st = duo_gated_attention(q, k, v, B, L, Hq, Hkv, d, dt, alpha, S, W, softmax_scale, out, _stream_ptr(stream))
     if st != DUO_OK:
         raise DuoError(st, "duo_gated_attention")
     return out

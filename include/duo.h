@@ -38,11 +38,16 @@
  * stream).  Calls on one handle must be ordered on one stream (or externally
  * synchronised): they share the cache's scratch space.  A handle is not thread-safe.
  *
- * Errors: every argument is checked before any launch; on error nothing is
- * launched and the cache (lengths included) is unchanged.  len advances only when
- * every launch of the call was accepted.  A failed launch returns DUO_ERR_CUDA.
- * Conditions detected on the device (a bounded wait that ran out) are latched in a
- * status word and reported by duo_get_device_status().
+ * Errors: every argument is checked, and every fallible host step of a call (tensor
+ * map encoding, kernel attributes) is done, before its first launch; on such an error
+ * nothing is launched and the cache (lengths included) is unchanged.  A launch that
+ * fails returns DUO_ERR_CUDA.  len always describes what the cache holds: it advances
+ * exactly when the launch that writes the new rows was accepted.  Each call writes the
+ * cache in its last launch, so a call that fails leaves it unchanged -- except
+ * duo_append_decode on its two-launch path, whose token stays appended (len advanced)
+ * when the attention launch after the append fails.  Conditions detected on the device
+ * (a bounded wait that ran out) are latched in a status word and reported by
+ * duo_get_device_status().
  */
 #ifndef DUO_H
 #define DUO_H
@@ -136,7 +141,9 @@ DUO_API duo_status duo_append_kv(duo_cache *cache, int layer, const void *k, con
  * Chunked pre-fill of one layer ("Chunked Pre-filling", Figure 5 right): the n
  * queries at positions len .. len+n-1 attend to the layer's cache plus the
  * chunk itself -- causal mask for retrieval heads, Lambda mask for streaming heads
- * -- and the chunk is then appended as by duo_append_kv.
+ * -- and the chunk is then appended as by duo_append_kv.  Launches: the staging copy
+ * of the streaming heads' history (when there is any), the attention (cached positions
+ * from the cache, the chunk's own keys from k and v), then the append.
  *   q, out  device [B][n][Hq][d];  k, v device [B][n][Hkv][d]
  *   lse     device [B][n][Hq] fp32, or NULL
  * DUO_ERR_UNSUPPORTED for an INT4 retrieval cache.
@@ -166,7 +173,9 @@ DUO_API duo_status duo_decode_attention(duo_cache *cache, int layer, const void 
  * kernel writes the token's rows into the cache itself, each by the CTA that then reads
  * the tile holding it; other caches get the append launch, then the decode launches
  * (the faster choice measured).  The cache afterwards holds exactly what duo_append_kv
- * would have written, and len advances by one.
+ * would have written, and len advances by one.  On the two-launch path, a failure of
+ * the attention launch after the append was accepted returns DUO_ERR_CUDA with the
+ * token appended and len advanced (outputs not written).
  * DUO_ERR_CAPACITY if len + 1 > max_len.
  */
 DUO_API duo_status duo_append_decode(duo_cache *cache, int layer, const void *q, const void *k, const void *v,
@@ -221,10 +230,10 @@ DUO_API duo_status duo_get_device_status(duo_cache *cache, void *cuda_stream);
 
 /*
  * duo_decode_attention for callers that cannot allocate device memory when they
- * decode -- for instance code running while a CUDA graph is being captured, where
- * cudaMalloc is not allowed, or a runtime whose device memory belongs to a pool sized
- * once at start-up.  The paper has no counterpart: this is a property of the library,
- * not of the method.
+ * decode -- for instance a serving runtime whose device memory belongs to a pool it
+ * sized once at start-up (every further cudaMalloc fails or fragments that pool), or
+ * a caller with a fixed memory budget that must not grow while it runs.  The paper has
+ * no counterpart: this is a property of the library, not of the method.
  *
  * Same arguments, layouts and result as duo_decode_attention.  It calls no cudaMalloc,
  * cudaFree or allocating library routine and does not use the scratch area of the
@@ -234,12 +243,17 @@ DUO_API duo_status duo_get_device_status(duo_cache *cache, void *cuda_stream);
  * call; the rest of the array keeps the previous call's contents, so calls that
  * overlap on the GPU (other streams, other threads) race and must be ordered by the
  * caller.  The first call on each device looks up the array's device address with
- * cudaGetSymbolAddress, with that device current; make that first call before any
- * stream capture.
+ * cudaGetSymbolAddress, with that device current, and keeps it for the life of the
+ * process; make that first call before any stream capture.  After cudaDeviceReset on
+ * a device the kept address is stale: do not call this entry point on that device again
+ * in the same process.
  * Limits: bf16 caches with head_dim 128, not INT4, at most 16 query heads per KV head
  * (else DUO_ERR_UNSUPPORTED).  The partials of B*kv_heads heads must fit the array at
  * one CTA: B*kv_heads*G*(head_dim+4)*4 bytes <= 4 MiB less the tickets, else
- * DUO_ERR_CAPACITY; larger head counts still fit but run on fewer CTAs.
+ * DUO_ERR_CAPACITY; larger head counts still fit but run on fewer CTAs.  The refusal is
+ * kept even though a single CTA would need no scratch: such a cache would decode on one
+ * SM, over a hundred times slower than duo_decode_attention, and the caller should know
+ * the size is past what this entry point serves.
  */
 DUO_API duo_status duo_decode_attention_static_scratch(duo_cache *cache, int layer, const void *q, void *out,
                                                        float *lse, void *cuda_stream);
@@ -256,19 +270,28 @@ DUO_API duo_status duo_decode_attention_static_scratch(duo_cache *cache, int lay
  *   alpha    device [Hkv] fp32, one gate per KV head (values outside [0, 1] are used
  *            as given)
  *   softmax_scale  0 means 1/sqrt(head_dim)
- *   workspace      caller-owned device buffer of >= duo_gated_workspace_bytes() bytes,
- *                  256-byte aligned; its contents are scratch (the K/V copy and the
- *                  streaming term); it must not be used by another call meanwhile.
- * The causal term is written to `out`, the Lambda term to the workspace, and one
- * elementwise kernel mixes them in place.  Launches on `cuda_stream`; arguments are
- * checked before any launch (DUO_ERR_INVALID; DUO_ERR_CAPACITY for a short workspace).
+ * Two launches on `cuda_stream`, both reading q, k and v where they are (no copy, no
+ * scratch): the causal term is written to `out`, then the Lambda term is computed and
+ * each row of `out` becomes alpha * out + (1 - alpha) * streaming.  Arguments are
+ * checked before any launch (DUO_ERR_INVALID).
  */
-DUO_API size_t duo_gated_workspace_bytes(int batch, int seq_len, int q_heads, int kv_heads, int head_dim,
-                                         duo_dtype dtype, int S, int W);
 DUO_API duo_status duo_gated_attention(const void *q, const void *k, const void *v, int batch, int seq_len,
                                        int q_heads, int kv_heads, int head_dim, duo_dtype dtype, const float *alpha,
-                                       int S, int W, float softmax_scale, void *out, void *workspace,
-                                       size_t workspace_bytes, void *cuda_stream);
+                                       int S, int W, float softmax_scale, void *out, void *cuda_stream);
+
+/*
+ * Test controls of the host-side bookkeeping, process-wide and not thread-safe (tests
+ * only; the paper has no counterpart).
+ *   dry_run     1: no call touches a device -- the first-use clear of a cache buffer and
+ *               every kernel launch are skipped and reported as accepted -- so that
+ *               argument checks, lengths and the error contract above can be exercised
+ *               on a machine without a GPU; 0: normal operation.
+ *   fail_after  >= 0: the launch attempt number fail_after + 1, counted from this call,
+ *               is not made and reports a launch failure (the call returns
+ *               DUO_ERR_CUDA); -1: off.
+ * DUO_ERR_INVALID for other values.
+ */
+DUO_API duo_status duo_debug_launch_controls(int dry_run, int64_t fail_after);
 
 /* Static description of a status code. */
 DUO_API const char *duo_status_str(duo_status status);

@@ -165,37 +165,25 @@ def test_status_strings():
 
 # ------------------------------------------------------- gated mixed attention
 
-def test_gated_workspace_bytes():
-    """Two one-layer caches (all retrieval, all streaming) plus the streaming term."""
-    B, L, Hq, Hkv, d, S, W = 2, 1000, 8, 4, 128, 4, 16
-    n = duo.duo_gated_workspace_bytes(B, L, Hq, Hkv, d, duo.DUO_BF16, S, W)
-    full = duo.duo_cache_bytes(1, Hkv, d, np.ones(Hkv, np.uint8), S, W, L, duo._opts(batch=B, q_heads=Hq))
-    strm = duo.duo_cache_bytes(1, Hkv, d, np.zeros(Hkv, np.uint8), S, W, L, duo._opts(batch=B, q_heads=Hq))
-    assert n >= full + strm + B * L * Hq * d * 2
-    assert duo.duo_gated_workspace_bytes(B, L, Hq, Hkv, 96, duo.DUO_BF16, S, W) == 0  # head_dim
-    assert duo.duo_gated_workspace_bytes(B, L, 6, 4, d, duo.DUO_BF16, S, W) == 0       # Hq % Hkv
-    assert duo.duo_gated_workspace_bytes(B, 0, Hq, Hkv, d, duo.DUO_BF16, S, W) == 0    # empty sequence
-    assert duo.duo_gated_workspace_bytes(B, L, Hq, Hkv, d, duo.DUO_BF16, S, 0) == 0    # W >= 1
-
-
 def test_gated_checks_arguments_before_any_launch():
     B, L, Hq, Hkv, d, S, W = 1, 100, 4, 2, 64, 2, 8
-    n = duo.duo_gated_workspace_bytes(B, L, Hq, Hkv, d, duo.DUO_FP32, S, W)
     p = FAKE
 
     def call(**kw):
-        a = dict(q=p, k=p, v=p, alpha=p, out=p, ws=p, nb=n, scale=0.0, L=L)
+        a = dict(q=p, k=p, v=p, alpha=p, out=p, scale=0.0, L=L, d=d, Hq=Hq, W=W)
         a.update(kw)
-        return duo.duo_gated_attention(a["q"], a["k"], a["v"], B, a["L"], Hq, Hkv, d, duo.DUO_FP32, a["alpha"], S, W,
-                                       a["scale"], a["out"], a["ws"], a["nb"])
+        return duo.duo_gated_attention(a["q"], a["k"], a["v"], B, a["L"], a["Hq"], Hkv, a["d"], duo.DUO_FP32,
+                                       a["alpha"], S, a["W"], a["scale"], a["out"])
 
     assert call(q=0) == duo.DUO_ERR_INVALID
     assert call(alpha=0) == duo.DUO_ERR_INVALID
     assert call(out=p + 8) == duo.DUO_ERR_INVALID       # 16-byte alignment
-    assert call(ws=p + 16) == duo.DUO_ERR_INVALID       # 256-byte alignment
+    assert call(alpha=p + 2) == duo.DUO_ERR_INVALID     # 4-byte alignment
     assert call(scale=-1.0) == duo.DUO_ERR_INVALID
-    assert call(L=0) == duo.DUO_ERR_INVALID
-    assert call(nb=n - 1) == duo.DUO_ERR_CAPACITY
+    assert call(L=0) == duo.DUO_ERR_INVALID             # empty sequence
+    assert call(d=96) == duo.DUO_ERR_INVALID            # head_dim
+    assert call(Hq=5) == duo.DUO_ERR_INVALID            # Hq % Hkv
+    assert call(W=0) == duo.DUO_ERR_INVALID             # W >= 1
 
 
 def test_append_decode_checks_arguments_before_any_launch():
@@ -211,3 +199,96 @@ def test_append_decode_checks_arguments_before_any_launch():
         assert duo.duo_cache_len(h, 0) == (duo.DUO_OK, 0)
     finally:
         duo.duo_cache_destroy(h)
+
+
+# ------------------------------------- host bookkeeping under the test launch controls
+
+@pytest.fixture
+def dry_run():
+    """Launches skipped and reported as accepted (duo_debug_launch_controls)."""
+    assert duo.duo_debug_launch_controls(1, -1) == duo.DUO_OK
+    yield
+    assert duo.duo_debug_launch_controls(0, -1) == duo.DUO_OK
+
+
+def test_launch_controls_reject_bad_values():
+    assert duo.duo_debug_launch_controls(2, -1) == duo.DUO_ERR_INVALID
+    assert duo.duo_debug_launch_controls(0, -2) == duo.DUO_ERR_INVALID
+    assert duo.duo_debug_launch_controls(0, -1) == duo.DUO_OK
+
+
+def test_dry_run_lengths_and_slots_follow_the_slot_rule(dry_run):
+    """Appends and pre-fill chunks of assorted sizes: len advances by n, and every
+    streaming slot reports the position the oracle's replay of the slot rule puts there."""
+    S, W = 3, 7
+    mask = np.array([[1, 0, 0, 1]], dtype=np.uint8)
+    st, h, _ = _create(layers=1, mask=mask, S=S, W=W, max_len=200)
+    assert st == duo.DUO_OK
+    chunks, n_total = [1, 5, 2, 9, 1, 30, 4], 0
+    for i, n in enumerate(chunks):
+        if i % 2:
+            assert duo.duo_prefill_chunk(h, 0, FAKE, FAKE, FAKE, n, FAKE, None) == duo.DUO_OK
+        else:
+            assert duo.duo_append_kv(h, 0, FAKE, FAKE, n) == duo.DUO_OK
+        n_total += n
+        assert duo.duo_cache_len(h, 0) == (duo.DUO_OK, n_total)
+        replay = oracle.ring_replay(S, W, chunks[:i + 1])[-1]
+        for slot in range(S + W):
+            assert duo.duo_debug_slot_position(h, 0, 1, slot) == (duo.DUO_OK, int(replay[slot]))
+    assert duo.duo_decode_attention(h, 0, FAKE, FAKE, None) == duo.DUO_OK
+    assert duo.duo_get_device_status(h) == duo.DUO_OK
+    duo.duo_cache_destroy(h)
+
+
+def _fail_nth(h, call, n):
+    """Runs `call` with launch attempt n (0-based) failing; returns its status and len."""
+    assert duo.duo_debug_launch_controls(1, n) == duo.DUO_OK
+    st = call()
+    assert duo.duo_debug_launch_controls(1, -1) == duo.DUO_OK
+    return st, duo.duo_cache_len(h, 0)[1]
+
+
+@pytest.mark.parametrize("call,launches,appends_at", [
+    # (call, its launches here, index of the launch that writes the cache)
+    ("append_kv", 1, 0),
+    ("prefill_first", 2, 1),      # attention, append (no streaming history yet)
+    ("prefill_later", 3, 2),      # history staging, attention, append
+    ("decode", 1, None),
+    ("append_decode", 2, 0),      # append, then attention (the two-launch path)
+])
+def test_failed_launch_keeps_the_length_contract(dry_run, call, launches, appends_at):
+    """Each launch of each call fails in turn: the call returns DUO_ERR_CUDA, and len
+    advances exactly when the launch that writes the cache was accepted -- which, the
+    cache being written by the last launch of every call but duo_append_decode's
+    two-launch path, means a failed call leaves the cache unchanged."""
+    mask = np.array([[1, 0, 0, 1]], dtype=np.uint8)
+    n = 6
+    for k in range(launches + 1):
+        st, h, _ = _create(layers=1, mask=mask, S=2, W=4, max_len=100)
+        if call in ("prefill_later", "decode", "append_decode"):
+            assert duo.duo_append_kv(h, 0, FAKE, FAKE, 10) == duo.DUO_OK
+        len0 = duo.duo_cache_len(h, 0)[1]
+        fns = {
+            "append_kv": lambda: duo.duo_append_kv(h, 0, FAKE, FAKE, n),
+            "prefill_first": lambda: duo.duo_prefill_chunk(h, 0, FAKE, FAKE, FAKE, n, FAKE, None),
+            "prefill_later": lambda: duo.duo_prefill_chunk(h, 0, FAKE, FAKE, FAKE, n, FAKE, None),
+            "decode": lambda: duo.duo_decode_attention(h, 0, FAKE, FAKE, None),
+            "append_decode": lambda: duo.duo_append_decode(h, 0, FAKE, FAKE, FAKE, FAKE, None),
+        }
+        st, len1 = _fail_nth(h, fns[call], k)
+        grew = {"append_decode": 1, "decode": 0}.get(call, n)
+        if k == launches:  # no launch failed
+            assert st == duo.DUO_OK and len1 == len0 + grew
+        else:
+            assert st == duo.DUO_ERR_CUDA
+            appended = appends_at is not None and k > appends_at
+            assert len1 == len0 + (grew if appended else 0), (call, k)
+        duo.duo_cache_destroy(h)
+
+
+def test_gated_launch_failure_is_reported(dry_run):
+    for k, want in [(0, duo.DUO_ERR_CUDA), (1, duo.DUO_ERR_CUDA), (2, duo.DUO_OK)]:
+        assert duo.duo_debug_launch_controls(1, k) == duo.DUO_OK
+        st = duo.duo_gated_attention(FAKE, FAKE, FAKE, 1, 100, 4, 2, 64, duo.DUO_FP32, FAKE, 2, 8, 0.0, FAKE)
+        assert st == want, k
+    assert duo.duo_debug_launch_controls(1, -1) == duo.DUO_OK
