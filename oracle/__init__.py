@@ -73,6 +73,14 @@ def _load():
             lib.oracle_int4_quantize.argtypes = [i64, i32, vp, i32, vp, vp, vp]
             lib.oracle_int4_dequantize.restype = None
             lib.oracle_int4_dequantize.argtypes = [i64, i32, vp, vp, vp, vp]
+            lib.oracle_fp8_quantize.restype = None
+            lib.oracle_fp8_quantize.argtypes = [i64, i32, vp, i32, vp, vp]
+            lib.oracle_fp8_dequantize.restype = None
+            lib.oracle_fp8_dequantize.argtypes = [i64, i32, vp, vp, vp]
+            lib.oracle_e4m3_value.restype = dbl
+            lib.oracle_e4m3_value.argtypes = [ctypes.c_uint8]
+            lib.oracle_e4m3_encode.restype = ctypes.c_uint8
+            lib.oracle_e4m3_encode.argtypes = [ctypes.c_float]
             lib.oracle_layer_kv_elems.restype = dbl
             lib.oracle_layer_kv_elems.argtypes = [i64, i64, i64, i64, i64, i64]
             lib.oracle_budget_ratio.restype = dbl
@@ -222,6 +230,41 @@ def int4_dequantize(codes, scale_bits, zero_bits) -> np.ndarray:
     out = np.empty((nrows, 2 * half), dtype=np.float64)
     _load().oracle_int4_dequantize(nrows, 2 * half, _ptr(c), _ptr(sb), _ptr(zb), _ptr(out))
     return out
+
+
+def fp8_quantize(x):
+    """Rows [nrows][gs] (float32 or bf16 bits as uint16) -> (codes uint8 [nrows][gs] in OCP
+    E4M3, scales float32 [nrows] = amax / 448); reading R14 of oracle.c."""
+    xa, xt = _as_input(x)
+    if xt == F64:
+        raise TypeError("fp8_quantize takes float32 or bf16 rows")
+    xa = xa.reshape(-1, xa.shape[-1])
+    nrows, gs = xa.shape
+    codes = np.empty((nrows, gs), dtype=np.uint8)
+    scales = np.empty((nrows,), dtype=np.float32)
+    _load().oracle_fp8_quantize(nrows, gs, _ptr(np.ascontiguousarray(xa)), xt, _ptr(codes), _ptr(scales))
+    return codes, scales
+
+
+def fp8_dequantize(codes, scales) -> np.ndarray:
+    """codes [nrows][gs] E4M3 + fp32 scales [nrows] -> float64 [nrows][gs] (value * scale)."""
+    c = np.ascontiguousarray(codes, dtype=np.uint8)
+    c = c.reshape(-1, c.shape[-1])
+    nrows, gs = c.shape
+    sc = np.ascontiguousarray(scales, dtype=np.float32).reshape(nrows)
+    out = np.empty((nrows, gs), dtype=np.float64)
+    _load().oracle_fp8_dequantize(nrows, gs, _ptr(c), _ptr(sc), _ptr(out))
+    return out
+
+
+def e4m3_value(code: int) -> float:
+    """Value of one OCP E4M3 code."""
+    return float(_load().oracle_e4m3_value(int(code)))
+
+
+def e4m3_encode(y: float) -> int:
+    """Nearest OCP E4M3 code of a float (ties to even, held at +-448)."""
+    return int(_load().oracle_e4m3_encode(float(y)))
 
 
 def layer_kv_elems(Hr: int, Hs: int, L: int, S: int, W: int, d: int) -> float:

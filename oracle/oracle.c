@@ -33,6 +33,10 @@
  *   R9 INT4: one group = one token's row of a head; fp32 min/max; scale =
  *      fp16((max-min)/15), zero = fp16(min); code = clamp(rint((x-zero)/scale),0,15);
  *      element 2t in the low nibble of byte t; dequant = code*scale + zero.
+ *   R14 FP8: one group = one token's row of a head; amax = fp32 max |x|; scale =
+ *      amax / 448 in IEEE fp32 (kept as fp32); code = the OCP E4M3 value nearest to
+ *      x / scale (fp32 division), ties to even mantissa, magnitudes past 448 held at
+ *      448; amax = 0 gives scale 0 and zero codes; dequant = value(code) * scale.
  *
  * Build: gcc -O2 -ffp-contract=off -fopenmp -fPIC -shared (no fast-math).
  */
@@ -343,6 +347,74 @@ void oracle_int4_dequantize(int64_t nrows, int gs, const uint8_t *codes, const u
       out[r * gs + e] = (double)code * sc + z;
     }
   }
+}
+
+/* ---- FP8 (E4M3) quantisation with a per-row scale, reading R14 ---- */
+
+/* OCP 8-bit floating point E4M3 ("OFP8" specification): 1 sign bit, 4 exponent bits
+ * with bias 7, 3 mantissa bits; exponent field 0 holds subnormals m * 2^-9; no
+ * infinities, and S.1111.111 is NaN, so the largest finite magnitude is 1.75 * 2^8 =
+ * 448 (S.1111.110).  This encodes a finite float by round to nearest, ties to the
+ * even mantissa, holding magnitudes >= 448 at 448. */
+static uint8_t e4m3_encode(float y) {
+  const uint8_t sign = signbit(y) ? 0x80 : 0x00;
+  const double a = fabs((double)y);
+  if (a >= 448.0) return sign | 0x7E;
+  if (a == 0.0) return sign;
+  int e2;
+  frexp(a, &e2); /* a = f 2^e2 with f in [0.5, 1): a lies in [2^(e2-1), 2^e2) */
+  int E = e2 - 1;
+  if (E < -6) E = -6;                   /* subnormal range shares the step of binade -6 */
+  const double step = ldexp(1.0, E - 3); /* 3 mantissa bits: 8 steps per binade */
+  const double r = rint(a / step);       /* a / step is exact; rint rounds half to even */
+  const double v = r * step;             /* may carry into the next binade: still <= 448 */
+  if (v == 0.0) return sign;
+  int ev;
+  frexp(v, &ev);
+  const int Ev = ev - 1;
+  if (Ev < -6) return sign | (uint8_t)(v / ldexp(1.0, -9)); /* subnormal: m * 2^-9, m in 1..7 */
+  const int mant = (int)(v / ldexp(1.0, Ev - 3)) - 8;       /* 1.mmm -> mmm */
+  return sign | (uint8_t)((Ev + 7) << 3) | (uint8_t)mant;
+}
+
+/* value of an E4M3 code (exact in fp64); NaN codes are never produced here */
+static double e4m3_value(uint8_t c) {
+  const int s = c >> 7, e = (c >> 3) & 15, m = c & 7;
+  const double mag = e == 0 ? ldexp((double)m, -9) : ldexp(1.0 + m / 8.0, e - 7);
+  return s ? -mag : mag;
+}
+
+double oracle_e4m3_value(uint8_t c) { return e4m3_value(c); }
+uint8_t oracle_e4m3_encode(float y) { return e4m3_encode(y); }
+
+/* x [nrows][gs] (bf16 or f32) -> codes [nrows][gs] E4M3, scales [nrows] fp32 */
+void oracle_fp8_quantize(int64_t nrows, int gs, const void *x, int dtype, uint8_t *codes, float *scales) {
+#pragma omp parallel for schedule(static)
+  for (int64_t r = 0; r < nrows; ++r) {
+    const int64_t base = r * gs;
+    float amax = 0.0f;
+    for (int e = 0; e < gs; ++e) {
+      const float f = fabsf(load_f32(x, dtype, base + e));
+      if (f > amax) amax = f;
+    }
+    volatile float scale = amax / 448.0f; /* volatile: one IEEE fp32 division */
+    scales[r] = scale;
+    for (int e = 0; e < gs; ++e) {
+      uint8_t c = 0;
+      if (scale != 0.0f) {
+        volatile float y = load_f32(x, dtype, base + e) / scale;
+        c = e4m3_encode(y);
+      }
+      codes[base + e] = c;
+    }
+  }
+}
+
+/* codes [nrows][gs] E4M3 + scales [nrows] fp32 -> out [nrows][gs] fp64, value(code) * scale */
+void oracle_fp8_dequantize(int64_t nrows, int gs, const uint8_t *codes, const float *scales, double *out) {
+#pragma omp parallel for schedule(static)
+  for (int64_t r = 0; r < nrows; ++r)
+    for (int e = 0; e < gs; ++e) out[r * gs + e] = e4m3_value(codes[r * gs + e]) * (double)scales[r];
 }
 
 /* ---- memory closed forms ---- */

@@ -361,6 +361,66 @@ def test_int4_constant_row():
     np.testing.assert_array_equal(oracle.int4_dequantize(codes, sb, zb), row.astype(np.float64))
 
 
+# ------------------------------------------------------------------ FP8 pins
+
+def test_fp8_worked_example():
+    """amax 3.5 gives the scale 3.5 / 448 = 2^-7, so y = 128 x: values worked out by hand
+    from the OCP E4M3 layout (bias 7, 3 mantissa bits, 448 the largest finite value):
+    1 -> 128 = 0x70, -2 -> -256 = 0xF8, 0.5 -> 64 = 0x68, 3.5 -> 448 = 0x7E; ties go to
+    the even mantissa (8.5 -> 8 = 0x50, 9.5 -> 10 = 0x52); 3 * 2^-9 is the subnormal
+    0x03; 0 -> 0x00."""
+    vals = [1.0, -2.0, 0.5, 3.5, 8.5 * 2.0 ** -7, 9.5 * 2.0 ** -7, 3 * 2.0 ** -16, 0.0]
+    row = np.zeros((1, 128), dtype=np.float32)
+    row[0, :len(vals)] = vals
+    codes, scales = oracle.fp8_quantize(row)
+    assert scales[0] == np.float32(2.0 ** -7)
+    assert codes[0, :8].tolist() == [0x70, 0xF8, 0x68, 0x7E, 0x50, 0x52, 0x03, 0x00]
+    deq = oracle.fp8_dequantize(codes, scales)[0, :8]
+    np.testing.assert_array_equal(deq, [1.0, -2.0, 0.5, 3.5, 8 * 2.0 ** -7, 10 * 2.0 ** -7, 3 * 2.0 ** -16, 0.0])
+
+
+def test_fp8_encoder_matches_torch_float8_e4m3fn():
+    """The oracle's E4M3 rounding equals torch's float32 -> float8_e4m3fn conversion (an
+    independent implementation of the same format) on random values, exact ties and
+    subnormals within +-448, and its decoding equals torch's for every finite code."""
+    rng = np.random.default_rng(11)
+    y = np.concatenate([rng.uniform(-448, 448, 4000), rng.standard_normal(2000) * 2.0 ** rng.integers(-12, 6, 2000),
+                        (np.arange(-64, 64) + 0.5) * 2.0 ** -3, (np.arange(0, 16) + 0.5) * 2.0 ** -9]).astype(np.float32)
+    y = y[np.abs(y) <= 448]
+    want = torch.from_numpy(y).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    got = np.array([oracle.e4m3_encode(float(v)) for v in y], dtype=np.uint8)
+    np.testing.assert_array_equal(got, want)
+    finite = [c for c in range(256) if (c & 0x7F) != 0x7F]
+    tv = torch.tensor(finite, dtype=torch.uint8).view(torch.float8_e4m3fn).to(torch.float64).numpy()
+    np.testing.assert_array_equal([oracle.e4m3_value(c) for c in finite], tv)
+
+
+def test_fp8_round_trip_bound_and_order():
+    """Dequantised values stay within half an E4M3 step of x (relative 2^-4 in the normal
+    range, 2^-10 of the scale below it); codes are monotone in x; a row's largest
+    magnitude lands on +-448; no NaN code is produced."""
+    x = torch.randn(500, 128, generator=torch.Generator().manual_seed(6)).to(torch.bfloat16)
+    bits = x.view(torch.int16).numpy().view(np.uint16)
+    xf = x.to(torch.float64).numpy()
+    codes, scales = oracle.fp8_quantize(bits)
+    deq = oracle.fp8_dequantize(codes, scales)
+    sc = scales.astype(np.float64)[:, None]
+    bound = sc * np.maximum(np.abs(xf) / sc * 2.0 ** -4, 2.0 ** -10) * (1 + 1e-6)
+    assert np.all(np.abs(deq - xf) <= bound)
+    assert not np.any((codes & 0x7F) == 0x7F)
+    for r in range(500):
+        order = np.argsort(xf[r], kind="stable")
+        assert np.all(np.diff(deq[r][order]) >= 0)
+        i = np.argmax(np.abs(xf[r]))
+        assert codes[r, i] == (0xFE if xf[r, i] < 0 else 0x7E)
+
+
+def test_fp8_zero_row():
+    codes, scales = oracle.fp8_quantize(np.zeros((2, 128), dtype=np.float32))
+    assert np.all(scales == 0) and np.all(codes == 0)
+    assert np.all(oracle.fp8_dequantize(codes, scales) == 0)
+
+
 # ------------------------------------------------------------- mutation check
 
 def _pin_failures(mutant):
