@@ -61,6 +61,7 @@ DECODE_WORKLOADS = {
     "llama2-7b-mha-decode-32k-b1": (32, 32, 8, 32768, 1, LAYERS, "same"),
     "llama2-7b-mha-decode-32k-b8": (32, 32, 8, 32768, 8, LAYERS, "same"),
     "llama3-8b-gqa-decode-1m-int4-32l": (32, 8, 4, 1 << 20, 1, LAYERS, "int4"),
+    "llama3-8b-gqa-decode-128k-fp8-b1": (32, 8, 4, 131072, 1, LAYERS, "fp8"),
 }
 REGIONS = 5              # timed regions per workload (median and spread reported)
 REGION_MS = 100.0        # GPU time per region of a workload entry, at least
@@ -71,10 +72,10 @@ MAX_REGION_STEPS = 400
 
 def decode_bytes(len_, B=1, Hr=NRET, Hs=HKV - NRET, Hq=HQ, d=D, fmt="same", S=S, W=W):
     """Algorithmic HBM bytes of one decode-attention call: every visible K and V row
-    once (bf16 rows, or INT4 codes plus fp16 scale/zero), the queries, the outputs and
-    the lse."""
+    once (bf16 rows, INT4 codes plus fp16 scale/zero, or FP8 codes plus an fp32 scale),
+    the queries, the outputs and the lse."""
     kv = 2 * d * 2
-    rkv = 2 * (d // 2 + 4) if fmt == "int4" else kv
+    rkv = {"int4": 2 * (d // 2 + 4), "fp8": 2 * (d + 4)}.get(fmt, kv)
     return B * (Hr * len_ * rkv + Hs * min(len_, S + W) * kv) + B * Hq * d * 2 * 2 + B * Hq * 4
 
 
@@ -183,6 +184,8 @@ def kernel_hash(workload):
     files = ["k_decode_tc.cu", "tcgen05.cuh", "decode_merge.cuh", "device_common.cuh", "duo_internal.h"]
     if "int4" in workload:
         files.append("k_decode_int4_tc.cu")
+    if "fp8" in workload:
+        files.append("k_decode_fp8_tc.cu")
     return _hash_files(files)
 
 
@@ -232,14 +235,14 @@ def launches_per_layer(B, fmt, Hs):
     """Kernel launches of one duo_append_decode call (see include/duo.h)."""
     if fmt == "same":
         return (1, "fused append+decode") if B == 1 else (2, "append, then decode")
-    return (3 if Hs > 0 else 2), "append, bf16 streaming-head decode, INT4 retrieval-head decode"
+    return (3 if Hs > 0 else 2), f"append, bf16 streaming-head decode, {fmt.upper()} retrieval-head decode"
 
 
 class DecodeRun:
     """One decode workload: a cache of `layers` layers filled to `ctx` tokens and the
     per-step inputs; step(i) appends token i to every layer and attends."""
 
-    def __init__(self, name, dev, extra_tokens, nstep_in):
+    def __init__(self, name, dev, extra_tokens, nstep_in, layers=0):
         import torch
 
         from head_split_kv_duo_b200 import inputs
@@ -247,6 +250,8 @@ class DecodeRun:
 
         self.name = name
         self.Hq, self.Hkv, self.nret, self.ctx, self.B, self.layers, self.fmt = DECODE_WORKLOADS[name]
+        if layers:
+            self.layers = layers
         self.Hr, self.Hs = self.nret, self.Hkv - self.nret
         self.dev = dev
         max_len = self.ctx + extra_tokens
@@ -370,7 +375,7 @@ def run_headline(args, dev, dist, hbm_peak, peak_src):
     import torch
     K, warmup = args.steps, args.warmup
     extra = warmup + 2 + MAX_HEADLINE_REGIONS * K + 2 * K + 16
-    run = DecodeRun(args.workload, dev, extra_tokens=extra, nstep_in=max(64, K))
+    run = DecodeRun(args.workload, dev, extra_tokens=extra, nstep_in=max(64, K), layers=args.layers)
     for i in range(warmup):
         run.step(i)
     # regions of exactly K steps: at least REGIONS, and until about HEADLINE_TOTAL_MS
@@ -445,7 +450,7 @@ def run_headline(args, dev, dist, hbm_peak, peak_src):
                    "l2": f"inputs larger than L2: {run.layers} layer caches of {kv_gb / run.layers:.2f} GB "
                          f"visited per step",
                    "parallelism": f"replicas{args.gpus}"},
-        "dtype": "bf16" if run.fmt == "same" else "bf16+int4kv",
+        "dtype": "bf16" if run.fmt == "same" else f"bf16+{run.fmt}kv",
         "us_per_token_layer": round(ms_own * 1e3 / calls, 3),
         "roofline": roof,
         "gpu_launches": len(regions) * calls * run.lpl,
@@ -577,21 +582,23 @@ class OracleDecode:
         k = inputs.randn((B, self.ctx, Hkv, D), 100, device=device).cpu()
         v = inputs.randn((B, self.ctx, Hkv, D), 101, device=device).cpu()
         self.q = _u16(inputs.randn((B, 1, Hq, D), 7, device=device).cpu())
-        if fmt == "int4":
+        if fmt in ("int4", "fp8"):
             # fp64 K/V (the streaming heads' rows as they are); per retrieval head the codes
-            # and fp16 scale/zero from the oracle's quantiser, dequantised at every step
+            # and scales from the oracle's quantiser, dequantised at every step
             self.k = k.float().numpy().astype(np.float64)
             self.v = v.float().numpy().astype(np.float64)
-            self.codes = [(g, oracle.int4_quantize(_u16(k[:, :, g])), oracle.int4_quantize(_u16(v[:, :, g])))
+            quant = oracle.int4_quantize if fmt == "int4" else oracle.fp8_quantize
+            self.codes = [(g, quant(_u16(k[:, :, g]).reshape(-1, D)), quant(_u16(v[:, :, g]).reshape(-1, D)))
                           for g in np.nonzero(self.mask)[0]]
         else:
             self.k, self.v = _u16(k), _u16(v)
 
     def step(self):
-        if self.fmt == "int4":
+        if self.fmt in ("int4", "fp8"):
+            deq = self.oracle.int4_dequantize if self.fmt == "int4" else self.oracle.fp8_dequantize
             for g, kc, vc in self.codes:
-                self.k[:, :, g] = self.oracle.int4_dequantize(*kc).reshape(self.B, self.ctx, D)
-                self.v[:, :, g] = self.oracle.int4_dequantize(*vc).reshape(self.B, self.ctx, D)
+                self.k[:, :, g] = deq(*kc).reshape(self.B, self.ctx, D)
+                self.v[:, :, g] = deq(*vc).reshape(self.B, self.ctx, D)
         return self.oracle.attend(self.q, self.k, self.v, self.mask, S, W, pos0=self.ctx - 1)
 
     def nbytes(self):
@@ -613,8 +620,8 @@ def oracle_decode_sample(name, seconds, max_steps, ctx_cap=None, device="cpu"):
     what = f"{n} oracle decode steps of one layer at context {od.ctx}"
     if od.ctx != DECODE_WORKLOADS[name][3]:
         what += f" (the workload's {DECODE_WORKLOADS[name][3]}-token context needs too much fp64 host memory)"
-    if od.fmt == "int4":
-        what += ", each step dequantising the oracle's INT4 codes of the retrieval heads, then attending"
+    if od.fmt in ("int4", "fp8"):
+        what += f", each step dequantising the oracle's {od.fmt.upper()} codes of the retrieval heads, then attending"
     return {"value": round(gbs, 3), "unit": "GB/s", "cores": oracle.num_threads(), "kind": "oracle",
             "sample": f"{what}, batch {od.B}, all {od.Hq} query heads; {t_total:.1f} s wall on "
                       f"{oracle.num_threads()} threads", "seconds": round(t_total, 2), "steps": n}
@@ -664,6 +671,8 @@ def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--workload", default=WORKLOAD, choices=sorted(DECODE_WORKLOADS))
+    ap.add_argument("--layers", type=int, default=0,
+                    help="layer caches of the headline workload (0: the model's 32); small profiling captures only")
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])

@@ -52,9 +52,10 @@ duo_status make_cfg(int layers, int kv_heads, int head_dim, const uint8_t *mask,
   if (o.q_heads == 0) o.q_heads = kv_heads;
   if (o.q_heads < kv_heads || o.q_heads % kv_heads != 0 || o.q_heads > 4096) return DUO_ERR_INVALID;
   if (o.dtype != DUO_BF16 && o.dtype != DUO_FP32) return DUO_ERR_INVALID;
-  if (o.retr_fmt != DUO_KV_SAME && o.retr_fmt != DUO_KV_INT4_G128) return DUO_ERR_INVALID;
+  if (o.retr_fmt != DUO_KV_SAME && o.retr_fmt != DUO_KV_INT4_G128 && o.retr_fmt != DUO_KV_FP8_E4M3)
+    return DUO_ERR_INVALID;
   if (!(o.softmax_scale >= 0.f) || !std::isfinite(o.softmax_scale)) return DUO_ERR_INVALID;
-  if (o.retr_fmt == DUO_KV_INT4_G128 && (o.dtype != DUO_BF16 || head_dim != 128)) return DUO_ERR_UNSUPPORTED;
+  if (o.retr_fmt != DUO_KV_SAME && (o.dtype != DUO_BF16 || head_dim != 128)) return DUO_ERR_UNSUPPORTED;
   for (int i = 0; i < layers * kv_heads; ++i)
     if (mask[i] > 1) return DUO_ERR_INVALID;
   c->layers = layers;
@@ -84,7 +85,10 @@ bool make_layout(const Cfg &c, const uint8_t *mask, Layout *L) {
   const int64_t units = std::max<int64_t>((c.max_len + 127) / 128, (static_cast<int64_t>(c.S) + c.W + 127) / 128);
   L->max_splits = static_cast<int>(std::min<int64_t>(kMaxSplits, std::max<int64_t>(1, units)));
   const size_t row = static_cast<size_t>(c.D) * c.esize;
-  const size_t rrow = c.fmt == DUO_KV_INT4_G128 ? static_cast<size_t>(c.D / 2) : row;
+  // retrieval row bytes: d elements, d/2 INT4 code bytes, or d FP8 code bytes
+  const size_t rrow = c.fmt == DUO_KV_INT4_G128 ? static_cast<size_t>(c.D / 2)
+                      : c.fmt == DUO_KV_FP8_E4M3 ? static_cast<size_t>(c.D)
+                                                 : row;
   const size_t nslots = static_cast<size_t>(c.S) + c.W;
   size_t off = 0;
   auto take = [&](size_t bytes) {
@@ -112,7 +116,7 @@ bool make_layout(const Cfg &c, const uint8_t *mask, Layout *L) {
     const size_t rbytes = static_cast<size_t>(c.B) * lo.Hr * L->cap * rrow;
     lo.rk = take(rbytes);
     lo.rv = take(rbytes);
-    if (c.fmt == DUO_KV_INT4_G128) {
+    if (c.fmt != DUO_KV_SAME) {  // INT4 fp16 scale + zero, or FP8 fp32 scale: 4 bytes per row
       const size_t zbytes = static_cast<size_t>(c.B) * lo.Hr * L->cap * 4 + 16;
       lo.rk_sz = take(zbytes);
       lo.rv_sz = take(zbytes);
@@ -174,6 +178,7 @@ AppendParams append_params(const duo_cache *c, const Layer &ly, const void *k, c
   p.max_len = c->cap;
   p.ring_from = std::max<int64_t>(c->S, ly.len + n - c->W);
   p.int4 = c->fmt == DUO_KV_INT4_G128 ? 1 : 0;
+  p.fp8 = c->fmt == DUO_KV_FP8_E4M3 ? 1 : 0;
   p.hm = ly.hm;
   return p;
 }
@@ -254,8 +259,8 @@ duo_status duo_cache_create(int layers, int kv_heads, int head_dim, const uint8_
     }
     ly.rk = h->buf + lo.rk;
     ly.rv = h->buf + lo.rv;
-    ly.rk_sz = c.fmt == DUO_KV_INT4_G128 ? h->buf + lo.rk_sz : nullptr;
-    ly.rv_sz = c.fmt == DUO_KV_INT4_G128 ? h->buf + lo.rv_sz : nullptr;
+    ly.rk_sz = c.fmt != DUO_KV_SAME ? h->buf + lo.rk_sz : nullptr;
+    ly.rv_sz = c.fmt != DUO_KV_SAME ? h->buf + lo.rv_sz : nullptr;
     ly.sk = h->buf + lo.sk;
     ly.sv = h->buf + lo.sv;
     ly.len = 0;
@@ -285,7 +290,7 @@ duo_status duo_prefill_chunk(duo_cache *c, int layer, const void *q, const void 
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) ||
       (reinterpret_cast<uintptr_t>(lse) & 3u))
     return DUO_ERR_INVALID;
-  if (c->fmt == DUO_KV_INT4_G128) return DUO_ERR_UNSUPPORTED;
+  if (c->fmt != DUO_KV_SAME) return DUO_ERR_UNSUPPORTED;  // quantised caches: decode only
   Layer &ly = c->L[layer];
   if (ly.len + n > c->max_len) return DUO_ERR_CAPACITY;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
@@ -415,6 +420,17 @@ DecodeParams decode_params(const duo_cache *c, const Layer &ly, const void *q, v
 
 cudaError_t launch_decode_any(const duo_cache *c, const DecodeParams &p, cudaStream_t st) {
   const bool int4 = c->fmt == DUO_KV_INT4_G128;
+  if (c->fmt == DUO_KV_FP8_E4M3) {
+    // bf16 streaming heads on the bf16 kernel, then the FP8 retrieval heads
+    if (!decode_fp8_tc_supported(p, c->dtype)) return cudaErrorNotSupported;
+    if (p.Hs > 0) {
+      DecodeParams ps = p;
+      ps.Hr = 0;
+      const cudaError_t e = launch_decode_tc(ps, c->num_sms, true, st);
+      if (e != cudaSuccess) return e;
+    }
+    return launch_decode_fp8_tc(p, c->num_sms, true, st);
+  }
   // the tcgen05 decodes overlap their start-up with the previous kernel on the stream
   if (int4 && decode_int4_tc_supported(p, c->dtype)) {
     // the bf16 streaming heads on the bf16 kernel (a few tiles), then the INT4 retrieval
@@ -434,15 +450,18 @@ cudaError_t launch_decode_any(const duo_cache *c, const DecodeParams &p, cudaStr
 
 // The decode launches of `p`, each through the test controls.
 cudaError_t decode_any(const duo_cache *c, const DecodeParams &p, cudaStream_t st) {
-  if (dry_run() || c->fmt != DUO_KV_INT4_G128 || !decode_int4_tc_supported(p, c->dtype) || p.Hs == 0)
-    return launch_via_hook([&] { return launch_decode_any(c, p, st); });
-  // INT4 layer with streaming heads: two launches (each counted by the test controls)
+  const bool int4 = c->fmt == DUO_KV_INT4_G128 && decode_int4_tc_supported(p, c->dtype);
+  const bool fp8 = c->fmt == DUO_KV_FP8_E4M3 && decode_fp8_tc_supported(p, c->dtype);
+  if (dry_run() || (!int4 && !fp8) || p.Hs == 0) return launch_via_hook([&] { return launch_decode_any(c, p, st); });
+  // quantised layer with streaming heads: two launches (each counted by the test controls)
   DecodeParams ps = p;
   ps.Hr = 0;
   cudaError_t e = launch_via_hook([&] { return launch_decode_tc(ps, c->num_sms, true, st); });
   if (e != cudaSuccess) return e;
   DecodeParams pr = p;
-  return launch_via_hook([&] { return launch_decode_int4_tc(pr, c->num_sms, true, st); });
+  return launch_via_hook([&] {
+    return int4 ? launch_decode_int4_tc(pr, c->num_sms, true, st) : launch_decode_fp8_tc(pr, c->num_sms, true, st);
+  });
 }
 
 bool decode_args_ok(const void *q, const void *out, const float *lse) {
@@ -473,7 +492,7 @@ duo_status duo_append_decode(duo_cache *c, int layer, const void *q, const void 
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   duo_status s = ensure_init(c, st);
   if (s != DUO_OK) return s;
-  const bool int4 = c->fmt == DUO_KV_INT4_G128;
+  const bool int4 = c->fmt != DUO_KV_SAME;  // quantised caches take the two-launch path
   Layer next = ly;
   next.len = ly.len + 1;
   DecodeParams p = decode_params(c, next, q, out, lse);
@@ -507,7 +526,9 @@ duo_status duo_cache_len(const duo_cache *c, int layer, int64_t *len) {
 duo_status duo_kv_bytes(const duo_cache *c, int64_t Lq, uint64_t *retained, uint64_t *full) {
   if (!c || Lq < 0) return DUO_ERR_INVALID;
   const uint64_t row = static_cast<uint64_t>(c->D) * c->esize;
-  const uint64_t rrow = c->fmt == DUO_KV_INT4_G128 ? static_cast<uint64_t>(c->D / 2 + 4) : row;
+  const uint64_t rrow = c->fmt == DUO_KV_INT4_G128   ? static_cast<uint64_t>(c->D / 2 + 4)
+                        : c->fmt == DUO_KV_FP8_E4M3 ? static_cast<uint64_t>(c->D + 4)
+                                                    : row;
   const uint64_t keep = static_cast<uint64_t>(std::min<int64_t>(Lq, static_cast<int64_t>(c->S) + c->W));
   uint64_t r = 0;
   for (const Layer &ly : c->L) r += static_cast<uint64_t>(ly.Hr) * Lq * rrow + static_cast<uint64_t>(ly.Hs) * keep * row;
@@ -547,9 +568,11 @@ duo_status duo_debug_region(const duo_cache *c, int layer, duo_region which, voi
                             int64_t *cap) {
   if (!layer_ok(c, layer)) return DUO_ERR_INVALID;
   const Layer &ly = c->L[layer];
-  const bool int4 = c->fmt == DUO_KV_INT4_G128;
+  const bool quant = c->fmt != DUO_KV_SAME;
   const uint64_t row = static_cast<uint64_t>(c->D) * c->esize;
-  const uint64_t rrow = int4 ? static_cast<uint64_t>(c->D / 2) : row;
+  const uint64_t rrow = c->fmt == DUO_KV_INT4_G128   ? static_cast<uint64_t>(c->D / 2)
+                        : c->fmt == DUO_KV_FP8_E4M3 ? static_cast<uint64_t>(c->D)
+                                                    : row;
   const uint64_t rrows = static_cast<uint64_t>(c->B) * ly.Hr * c->cap;
   const uint64_t srows = static_cast<uint64_t>(c->B) * ly.Hs * (static_cast<uint64_t>(c->S) + c->W);
   char *p = nullptr;
@@ -557,8 +580,8 @@ duo_status duo_debug_region(const duo_cache *c, int layer, duo_region which, voi
   switch (which) {
     case DUO_REGION_RETR_K: p = ly.rk; n = rrows * rrow; break;
     case DUO_REGION_RETR_V: p = ly.rv; n = rrows * rrow; break;
-    case DUO_REGION_RETR_KSZ: if (!int4) return DUO_ERR_INVALID; p = ly.rk_sz; n = rrows * 4; break;
-    case DUO_REGION_RETR_VSZ: if (!int4) return DUO_ERR_INVALID; p = ly.rv_sz; n = rrows * 4; break;
+    case DUO_REGION_RETR_KSZ: if (!quant) return DUO_ERR_INVALID; p = ly.rk_sz; n = rrows * 4; break;
+    case DUO_REGION_RETR_VSZ: if (!quant) return DUO_ERR_INVALID; p = ly.rv_sz; n = rrows * 4; break;
     case DUO_REGION_STRM_K: p = ly.sk; n = srows * row; break;
     case DUO_REGION_STRM_V: p = ly.sv; n = srows * row; break;
     default: return DUO_ERR_INVALID;

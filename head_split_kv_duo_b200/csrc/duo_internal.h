@@ -77,6 +77,7 @@ struct AppendParams {
   int64_t len, max_len;  // max_len: row stride of retrieval arrays (capacity rounded up to 256)
   int64_t ring_from;  // first non-sink position that reaches the ring
   int int4;           // retrieval rows stored INT4
+  int fp8;            // retrieval rows stored FP8 (E4M3 + fp32 scale)
   HeadMap hm;
 };
 
@@ -180,6 +181,10 @@ cudaError_t launch_decode_tc(const DecodeParams &p, int num_sms, bool overlap_pr
 // tcgen05 decode over an INT4 retrieval cache (bf16, head_dim 128, G <= 16)
 bool decode_int4_tc_supported(const DecodeParams &p, duo_dtype dt);
 cudaError_t launch_decode_int4_tc(const DecodeParams &p, int num_sms, bool overlap_previous, cudaStream_t st);
+
+// tcgen05 decode over an FP8 (E4M3) retrieval cache (bf16, head_dim 128, G <= 16)
+bool decode_fp8_tc_supported(const DecodeParams &p, duo_dtype dt);
+cudaError_t launch_decode_fp8_tc(const DecodeParams &p, int num_sms, bool overlap_previous, cudaStream_t st);
 
 // decode tiling shared by host (split sizing) and device
 int decode_tokens_per_stage(duo_dtype dt, int D, bool int4);

@@ -53,6 +53,27 @@ __device__ __forceinline__ void quantize_row_int4(const char *src, uint8_t *code
   }
 }
 
+// FP8 (OCP E4M3) quantisation of one bf16 row of 128 elements by one warp (format of
+// duo.h: fp32 max |x|, scale = max / 448 and x / scale in IEEE fp32, nearest E4M3 value
+// with ties to even, held at +-448).
+__device__ __forceinline__ void quantize_row_fp8(const char *src, uint8_t *codes, float *scale_out, int lane) {
+  const uint2 u = __ldg(reinterpret_cast<const uint2 *>(src) + lane);  // elements 4*lane .. 4*lane+3
+  const float x[4] = {bf16lo(u.x), bf16hi(u.x), bf16lo(u.y), bf16hi(u.y)};
+  float amax = fmaxf(fmaxf(fabsf(x[0]), fabsf(x[1])), fmaxf(fabsf(x[2]), fabsf(x[3])));
+  amax = warp_max(amax);
+  const float scale = __fdiv_rn(amax, 448.0f);
+  float y[4] = {0.f, 0.f, 0.f, 0.f};
+  if (scale != 0.f) {
+#pragma unroll
+    for (int e = 0; e < 4; ++e) y[e] = __fdiv_rn(x[e], scale);
+  }
+  uint16_t lo, hi;  // the first source lands in the upper byte
+  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(lo) : "f"(y[1]), "f"(y[0]));
+  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(hi) : "f"(y[3]), "f"(y[2]));
+  reinterpret_cast<uint32_t *>(codes)[lane] = static_cast<uint32_t>(lo) | (static_cast<uint32_t>(hi) << 16);
+  if (lane == 0) *scale_out = scale;
+}
+
 template <typename T>
 __global__ void __launch_bounds__(256) append_kernel(const AppendParams p) {
   // a decode launched right after may start its set-up now; it waits for this grid to
@@ -72,7 +93,13 @@ __global__ void __launch_bounds__(256) append_kernel(const AppendParams p) {
   const int idx = p.hm.kind_idx[g];
   if (p.hm.is_retr[g]) {
     const int64_t row = (static_cast<int64_t>(b) * p.Hr + idx) * p.max_len + pos;
-    if (!p.int4) {
+    if (p.fp8) {
+      const int CB = p.D;  // code bytes per row
+      quantize_row_fp8(p.k + src_off, reinterpret_cast<uint8_t *>(p.rk) + row * CB,
+                       reinterpret_cast<float *>(p.rk_sz) + row, lane);
+      quantize_row_fp8(p.v + src_off, reinterpret_cast<uint8_t *>(p.rv) + row * CB,
+                       reinterpret_cast<float *>(p.rv_sz) + row, lane);
+    } else if (!p.int4) {
       copy_row(p.rk + row * RB, p.k + src_off, RB, lane);
       copy_row(p.rv + row * RB, p.v + src_off, RB, lane);
     } else {

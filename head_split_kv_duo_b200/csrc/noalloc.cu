@@ -82,8 +82,8 @@ extern "C" duo_status duo_decode_attention_static_scratch(duo_cache *c, int laye
   p.nqg = 1;
   p.scale_log2 = c->scale * 1.4426950408889634f;
   p.hm = ly.hm;
-  const bool int4 = c->fmt == DUO_KV_INT4_G128;
-  if (!decode_tc_supported(p, c->dtype, int4)) return DUO_ERR_UNSUPPORTED;
+  // quantised retrieval caches (INT4, FP8) are not served here
+  if (c->fmt != DUO_KV_SAME || !decode_tc_supported(p, c->dtype, false)) return DUO_ERR_UNSUPPORTED;
 
   // Scratch layout: tickets [B][Hkv] (256-byte padded), then partials
   // [B][Hkv][ctas][G][d+4] floats.  Fewer CTAs are used when the partials of one

@@ -224,6 +224,9 @@ __device__ __forceinline__ int bar_or(int id, int n, int v) {
 // The thread sleeps inside try_wait (woken when the phase completes, or after the
 // hint) instead of spinning, so waiting warps leave the issue slots to working ones.
 __device__ __forceinline__ bool wait_bar(uint32_t bar, uint32_t parity, uint32_t *status, volatile int *abort_flag) {
+  // a phase that has already completed is seen by one non-blocking test (a sleeping
+  // try_wait costs about a tenth of a microsecond even then)
+  if (mbar_test_wait(bar, parity)) return true;
   if (mbar_try_wait_ns(bar, parity, 20000)) return true;
   const unsigned long long t0 = globaltimer();
 #pragma unroll 1

@@ -18,12 +18,12 @@ from . import build as _build
 
 DUO_OK, DUO_ERR_INVALID, DUO_ERR_CAPACITY, DUO_ERR_CUDA, DUO_ERR_TIMEOUT, DUO_ERR_UNSUPPORTED = range(6)
 DUO_BF16, DUO_FP32 = 0, 1
-DUO_KV_SAME, DUO_KV_INT4_G128 = 0, 1
+DUO_KV_SAME, DUO_KV_INT4_G128, DUO_KV_FP8_E4M3 = 0, 1, 2
 (DUO_REGION_RETR_K, DUO_REGION_RETR_V, DUO_REGION_RETR_KSZ, DUO_REGION_RETR_VSZ, DUO_REGION_STRM_K,
  DUO_REGION_STRM_V) = range(6)
 
 _DTYPES = {torch.bfloat16: DUO_BF16, torch.float32: DUO_FP32}
-_FMTS = {"same": DUO_KV_SAME, "int4": DUO_KV_INT4_G128}
+_FMTS = {"same": DUO_KV_SAME, "int4": DUO_KV_INT4_G128, "fp8": DUO_KV_FP8_E4M3}
 
 
 class duo_opts(ctypes.Structure):

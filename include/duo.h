@@ -82,8 +82,14 @@ typedef enum { DUO_BF16 = 0, DUO_FP32 = 1 } duo_dtype;
  * group per token row of a head (head_dim must be 128), fp16 scale and zero per
  * group: scale = fp16((max-min)/15), zero = fp16(min), code = clamp(rint((x - zero)
  * / scale), 0, 15) in fp32, element 2t in the low nibble of byte t, value =
- * code*scale + zero.  bf16 only.  Streaming heads always keep the working dtype. */
-typedef enum { DUO_KV_SAME = 0, DUO_KV_INT4_G128 = 1 } duo_kv_fmt;
+ * code*scale + zero.  DUO_KV_FP8_E4M3: 8-bit floating point codes (OCP E4M3: bias 7,
+ * 3 mantissa bits, largest finite 448), one fp32 scale per token row of a head (head_dim
+ * 128): scale = max|x| / 448, code = x / scale rounded to the nearest E4M3 value (ties
+ * to even, held at +-448), value = code * scale ("Integration with Existing
+ * Optimizations": 8-bit KV).  Both: bf16 only; caches of these formats are filled with
+ * duo_append_kv / duo_append_decode and read by decode (pre-fill of them is
+ * DUO_ERR_UNSUPPORTED).  Streaming heads always keep the working dtype. */
+typedef enum { DUO_KV_SAME = 0, DUO_KV_INT4_G128 = 1, DUO_KV_FP8_E4M3 = 2 } duo_kv_fmt;
 
 typedef struct {
   int batch;           /* B >= 1                                               */
@@ -157,9 +163,9 @@ DUO_API duo_status duo_prefill_chunk(duo_cache *cache, int layer, const void *q,
  * cached token of its retrieval head, or to the sinks and ring of its streaming
  * head.  The token must have been appended first (it attends to itself).
  *   q, out  device [B][Hq][d];  lse device [B][Hq] fp32, or NULL
- * With INT4 retrieval heads (bf16, head_dim 128) the streaming heads and the retrieval
- * heads are two launches on the stream; each writes only its own heads' rows of out
- * and lse.
+ * With INT4 or FP8 retrieval heads (bf16, head_dim 128) the streaming heads and the
+ * retrieval heads are two launches on the stream; each writes only its own heads' rows
+ * of out and lse.
  * DUO_ERR_INVALID if the layer is empty.
  */
 DUO_API duo_status duo_decode_attention(duo_cache *cache, int layer, const void *q, void *out, float *lse,
@@ -169,7 +175,7 @@ DUO_API duo_status duo_decode_attention(duo_cache *cache, int layer, const void 
  * duo_append_kv of one token followed by duo_decode_attention, as one call: k, v
  * device [B][1][Hkv][d] (the token at position len), q / out / lse as for
  * duo_decode_attention ("Decoding Procedure", steps 2-4, in the order of reading R6).
- * For bf16 caches with head_dim 128 (not INT4) and batch 1 it is one launch: the decode
+ * For bf16 caches with head_dim 128 (not INT4 or FP8) and batch 1 it is one launch: the decode
  * kernel writes the token's rows into the cache itself, each by the CTA that then reads
  * the tile holding it; other caches get the append launch, then the decode launches
  * (the faster choice measured).  The cache afterwards holds exactly what duo_append_kv
@@ -204,8 +210,9 @@ DUO_API duo_status duo_debug_slot_position(const duo_cache *cache, int layer, in
  * Device address and size of one storage array of a layer, for inspection and
  * tests (no device access).  which:
  *   DUO_REGION_RETR_K / _RETR_V   retrieval heads [B][H_r][cap][row], row = d
- *                                 elements, or d/2 code bytes for INT4
- *   DUO_REGION_RETR_KSZ / _VSZ    INT4 only: [B][H_r][cap][2] fp16 (scale, zero)
+ *                                 elements, or d/2 code bytes for INT4, d for FP8
+ *   DUO_REGION_RETR_KSZ / _VSZ    INT4: [B][H_r][cap][2] fp16 (scale, zero);
+ *                                 FP8: [B][H_r][cap] fp32 scale
  *   DUO_REGION_STRM_K / _STRM_V   streaming heads [B][H_s][S+W][d]
  * Heads of a kind are in increasing KV-head order.  *cap receives the token stride
  * of retrieval arrays (max_len rounded up to a multiple of 256).  Any output
@@ -247,7 +254,7 @@ DUO_API duo_status duo_get_device_status(duo_cache *cache, void *cuda_stream);
  * process; make that first call before any stream capture.  After cudaDeviceReset on
  * a device the kept address is stale: do not call this entry point on that device again
  * in the same process.
- * Limits: bf16 caches with head_dim 128, not INT4, at most 16 query heads per KV head
+ * Limits: bf16 caches with head_dim 128, not INT4 or FP8, at most 16 query heads per KV head
  * (else DUO_ERR_UNSUPPORTED).  The partials of B*kv_heads heads must fit the array at
  * one CTA: B*kv_heads*G*(head_dim+4)*4 bytes <= 4 MiB less the tickets, else
  * DUO_ERR_CAPACITY; larger head counts still fit but run on fewer CTAs.  The refusal is

@@ -100,11 +100,30 @@ def test_calls_check_arguments_before_any_launch():
     duo.duo_cache_destroy(h)
 
 
-def test_int4_prefill_is_unsupported():
-    st, h, _ = _create(opts=duo._opts(retr_fmt=duo.DUO_KV_INT4_G128))
+@pytest.mark.parametrize("fmt", [duo.DUO_KV_INT4_G128, duo.DUO_KV_FP8_E4M3])
+def test_quantised_prefill_is_unsupported(fmt):
+    st, h, _ = _create(opts=duo._opts(retr_fmt=fmt))
     assert st == duo.DUO_OK
     assert duo.duo_prefill_chunk(h, 0, FAKE, FAKE, FAKE, 4, FAKE, None) == duo.DUO_ERR_UNSUPPORTED
     duo.duo_cache_destroy(h)
+
+
+def test_fp8_layout_and_bytes():
+    """FP8 retrieval rows are d code bytes plus a 4-byte fp32 scale; fp32 or head_dim 64
+    caches cannot take the format; an unknown format is invalid."""
+    st, h, need = _create(layers=1, Hkv=4, mask=np.array([[1, 1, 0, 0]], np.uint8), S=16, W=512, max_len=1 << 20,
+                          opts=duo._opts(retr_fmt=duo.DUO_KV_FP8_E4M3))
+    assert st == duo.DUO_OK
+    st, r, f = duo.duo_kv_bytes(h, 1 << 20)
+    assert r == 2 * (2 * (1 << 20) * (128 + 4) + 2 * 528 * 256)
+    st, ptr, nb, cap = duo.duo_debug_region(h, 0, duo.DUO_REGION_RETR_K)
+    assert nb == 2 * cap * 128
+    st, ptr, nb, cap = duo.duo_debug_region(h, 0, duo.DUO_REGION_RETR_VSZ)
+    assert st == duo.DUO_OK and nb == 2 * cap * 4
+    duo.duo_cache_destroy(h)
+    assert _create(opts=duo._opts(dtype=duo.DUO_FP32, retr_fmt=duo.DUO_KV_FP8_E4M3))[0] == duo.DUO_ERR_UNSUPPORTED
+    assert _create(d=64, opts=duo._opts(retr_fmt=duo.DUO_KV_FP8_E4M3))[0] == duo.DUO_ERR_UNSUPPORTED
+    assert _create(opts=duo._opts(retr_fmt=3))[0] == duo.DUO_ERR_INVALID
 
 
 @pytest.mark.skipif(torch.cuda.is_available(), reason="checks the no-device failure path")

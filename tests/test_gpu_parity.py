@@ -626,3 +626,124 @@ def test_int4_decode_1m_llama3_one_layer():
             want_lse[t, g * G:(g + 1) * G] = l[0, 0]
         del kg, vg
     assert_close(got, want, torch.bfloat16, got_lse, want_lse, "int4 decode at 1M")
+
+
+# ------------------------------------------------------------------- FP8
+
+def _fp8_decode_check(Hq, Hkv, mask_row, S, W, B, ctx, steps, seed, plant=False, k_gain=1.0, v_gain=1.0, q_gain=1.0):
+    """Append ctx tokens, then `steps` decode steps, on an FP8 (E4M3) retrieval cache.
+    Every retrieval code byte and fp32 scale must equal the oracle's quantiser bit for
+    bit; outputs are compared with the oracle over its own dequantisation of the
+    retrieval rows (streaming heads keep bf16).  k_gain, v_gain and q_gain scale the
+    N(0,1) draws (then rounded to bf16) to exercise the kernel's query and value-scale
+    normalisation."""
+    d, T, G = 128, ctx + steps, Hq // Hkv
+    mask = torch.tensor([mask_row], dtype=torch.uint8)
+    q = (inputs.randn((B, steps, Hq, d), seed, torch.float32, DEV) * q_gain).to(torch.bfloat16)
+    k = (inputs.randn((B, T, Hkv, d), seed + 1, torch.float32, DEV) * k_gain).to(torch.bfloat16)
+    v = (inputs.randn((B, T, Hkv, d), seed + 2, torch.float32, DEV) * v_gain).to(torch.bfloat16)
+    ridx = [g for g in range(Hkv) if mask_row[g]]
+    if plant and ctx > 2:
+        P = ctx // 2
+        ramp = torch.linspace(-2.0, 2.0, d, device=DEV).to(torch.bfloat16)
+        for g in ridx:
+            k[:, P, g] = (3.0 * q[:, 0, g * G].float()).to(torch.bfloat16)
+            v[:, P, g] = ramp
+    cache = DuoCache(1, Hkv, d, mask, S, W, T, batch=B, q_heads=Hq, dtype=torch.bfloat16, retr_fmt="fp8")
+    if ctx > 0:
+        cache.append_kv(0, k[:, :ctx].contiguous(), v[:, :ctx].contiguous())
+    outs, lses = [], []
+    for t in range(steps):
+        cache.append_kv(0, k[:, ctx + t:ctx + t + 1].contiguous(), v[:, ctx + t:ctx + t + 1].contiguous())
+        o, l = cache.decode_attention(0, q[:, t].contiguous())
+        outs.append(o.float()[:, None])
+        lses.append(l[:, None])
+    torch.cuda.synchronize()
+    assert cache.device_status() == 0
+    got, got_lse = torch.cat(outs, 1).cpu().numpy(), torch.cat(lses, 1).cpu().numpy()
+    rk, cap = cache.region(0, duo.DUO_REGION_RETR_K)
+    rv, _ = cache.region(0, duo.DUO_REGION_RETR_V)
+    ks, _ = cache.region(0, duo.DUO_REGION_RETR_KSZ)
+    vs, _ = cache.region(0, duo.DUO_REGION_RETR_VSZ)
+    kq = k.float().cpu().numpy().astype(np.float64)
+    vq = v.float().cpu().numpy().astype(np.float64)
+    for i, g in enumerate(ridx):
+        for src, C, Z, dst in ((k, rk, ks, kq), (v, rv, vs, vq)):
+            codes, scales = oracle.fp8_quantize(bits(src[:, :, g]).reshape(-1, d))
+            dev_codes = C.view(B, len(ridx), cap, d)[:, i, :T].cpu().numpy().reshape(-1, d)
+            dev_sc = Z.view(torch.float32).view(B, len(ridx), cap)[:, i, :T].cpu().numpy().reshape(-1)
+            assert np.array_equal(dev_codes, codes), f"FP8 codes of kv head {g} differ"
+            assert np.array_equal(dev_sc.view(np.uint32), scales.view(np.uint32)), f"FP8 scales of kv head {g} differ"
+            dst[:, :, g] = oracle.fp8_dequantize(codes, scales).reshape(B, T, d)
+    ws, ls = [], []
+    for t in range(steps):
+        w, l = oracle.attend(bits(q[:, t:t + 1]), kq[:, :ctx + t + 1], vq[:, :ctx + t + 1],
+                             np.asarray(mask_row, dtype=bool), S, W, pos0=ctx + t)
+        ws.append(w)
+        ls.append(l)
+    want, want_lse = np.concatenate(ws, 1), np.concatenate(ls, 1)
+    scale = max(1.0, float(np.abs(want).max()))
+    assert_close(got / scale, want / scale, torch.bfloat16, got_lse, want_lse,
+                 f"fp8 decode Hq{Hq} Hkv{Hkv} B{B} ctx{ctx} gains {k_gain},{v_gain},{q_gain}")
+    return got, want
+
+
+@pytest.mark.parametrize("Hq,Hkv,mask_row,S,W,B,ctx", [
+    (8, 8, [1, 0, 1, 0, 0, 0, 0, 1], 4, 32, 1, 0),        # first token: sees only itself
+    (8, 8, [1, 0, 1, 0, 0, 0, 0, 1], 4, 32, 2, 37),       # MHA, one ragged tile
+    (16, 8, [1] * 8, 16, 64, 1, 3000),                     # all retrieval, group 2
+    (32, 4, [0, 0, 0, 0], 16, 512, 2, 2000),               # all streaming (bf16 pieces only)
+    (64, 4, [1, 0, 1, 1], 16, 512, 1, 5000),               # group 16
+    (32, 4, [0, 1, 1, 0], 0, 100, 3, 1000),                # group 8, no sinks
+    (32, 8, [0, 1, 0, 1, 1, 0, 0, 1], 16, 512, 1, 1 << 17),  # Llama-3 shape, 128K
+    (32, 8, [0, 1, 0, 1, 1, 0, 0, 1], 16, 512, 4, 20000),    # batch 4
+    (32, 8, [1, 0, 1, 0, 1, 0, 1, 0], 16, 512, 2, 118),      # ring slots past len (tile 1)
+])
+def test_fp8_tc_decode_shapes(Hq, Hkv, mask_row, S, W, B, ctx):
+    _fp8_decode_check(Hq, Hkv, mask_row, S, W, B, ctx, 2, 160)
+
+
+@pytest.mark.parametrize("k_gain,v_gain,q_gain", [(1000.0, 1000.0, 1e-3), (1e-4, 1e-4, 1e4), (1 / 300, 1.0, 300.0),
+                                                   (100.0, 1.0, 1e-2)])
+def test_fp8_tc_decode_value_ranges(k_gain, v_gain, q_gain):
+    """K and V far above or below 1 (the per-row scales and the tile's largest V scale
+    carry them) and queries far from 1 (the power-of-two query prescale keeps them in
+    fp16); the logits keep their N(0,1) size (k_gain * q_gain = 1)."""
+    _fp8_decode_check(32, 8, [1, 0, 0, 1, 1, 0, 0, 1], 16, 512, 1, 3000, 1, 165, k_gain=k_gain, v_gain=v_gain,
+                      q_gain=q_gain)
+
+
+@pytest.mark.parametrize("Hq,Hkv,B,ctx", [(32, 8, 1, 20000), (8, 8, 2, 5000)])
+def test_fp8_tc_decode_planted_needle(Hq, Hkv, B, ctx):
+    mask_row = [1, 0] * (Hkv // 2)
+    got, want = _fp8_decode_check(Hq, Hkv, mask_row, 16, 512, B, ctx, 1, 170, plant=True)
+    G = Hq // Hkv
+    ramp = np.linspace(-2.0, 2.0, 128)
+    for g in range(0, Hkv, 2):  # retrieval heads recover the planted ramp
+        assert np.abs(want[:, 0, g * G] - ramp).max() < 0.3
+        assert np.abs(got[:, 0, g * G] - ramp).max() < 0.3
+
+
+def test_fp8_append_decode_equals_append_then_decode():
+    """duo_append_decode on an FP8 cache (two launches) leaves the same cache and returns
+    the same outputs as duo_append_kv followed by duo_decode_attention."""
+    Hq, Hkv, d, S, W, B, ctx, steps = 32, 8, 128, 16, 64, 1, 400, 20
+    mask = torch.tensor([[0, 1, 1, 0, 0, 1, 0, 1]], dtype=torch.uint8)
+    T = ctx + steps
+    q = inputs.randn((B, steps, Hq, d), 175, device=DEV)
+    k = inputs.randn((B, T, Hkv, d), 176, device=DEV)
+    v = inputs.randn((B, T, Hkv, d), 177, device=DEV)
+    c1 = DuoCache(1, Hkv, d, mask, S, W, T, batch=B, q_heads=Hq, dtype=torch.bfloat16, retr_fmt="fp8")
+    c2 = DuoCache(1, Hkv, d, mask, S, W, T, batch=B, q_heads=Hq, dtype=torch.bfloat16, retr_fmt="fp8")
+    for c in (c1, c2):
+        c.append_kv(0, k[:, :ctx].contiguous(), v[:, :ctx].contiguous())
+    for t in range(steps):
+        kt, vt = k[:, ctx + t:ctx + t + 1].contiguous(), v[:, ctx + t:ctx + t + 1].contiguous()
+        c1.append_kv(0, kt, vt)
+        o1, l1 = c1.decode_attention(0, q[:, t].contiguous())
+        o2, l2 = c2.append_decode(0, q[:, t].contiguous(), kt, vt)
+        assert torch.equal(o1, o2) and torch.equal(l1, l2), f"step {t}"
+    torch.cuda.synchronize()
+    for r in [duo.DUO_REGION_RETR_K, duo.DUO_REGION_RETR_V, duo.DUO_REGION_RETR_KSZ, duo.DUO_REGION_RETR_VSZ,
+              duo.DUO_REGION_STRM_K, duo.DUO_REGION_STRM_V]:
+        assert torch.equal(c1.region(0, r)[0], c2.region(0, r)[0]), f"region {r}"
