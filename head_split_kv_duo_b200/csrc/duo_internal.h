@@ -186,6 +186,65 @@ cudaError_t launch_decode_int4_tc(const DecodeParams &p, int num_sms, bool overl
 bool decode_fp8_tc_supported(const DecodeParams &p, duo_dtype dt);
 cudaError_t launch_decode_fp8_tc(const DecodeParams &p, int num_sms, bool overlap_previous, cudaStream_t st);
 
+// ---- paged pool of sequences (ragged batching) ----
+constexpr int kPoolTile = 128;       // tokens per retrieval page (= one decode tile)
+constexpr int kPoolMaxSeqs = 128;    // sequences in one pool decode call
+constexpr int kPoolMaxSuper = 1024;  // (layer, sequence) pairs in one pool decode call
+
+// One layer of a pool as the kernels see it, kept in device memory (written once):
+// the tensor maps of its retrieval pages [pages][Hr][128][d] and of its streaming
+// arrays [max_seqs][Hs][S+W][d], its head partition and its array bases.
+struct alignas(64) PoolLayerDesc {
+  CUtensorMap tm_kr, tm_vr, tm_ks, tm_vs;
+  HeadMap hm;
+  int Hr, Hs;
+  char *rk, *rv, *sk, *sv;
+};
+
+// A pool decode call: layers layer0 .. layer0+nlayers-1 of the listed sequences.
+struct PoolDecodeCall {
+  const PoolLayerDesc *layers;  // device, every layer of the pool
+  const int *table;             // device block table [max_seqs][pages_per_seq]
+  int pages_per_seq;
+  int layer0, nlayers, nseq;
+  int slot[kPoolMaxSeqs];       // sequence slots
+  int len[kPoolMaxSeqs];        // tokens per sequence, the step's token included
+};
+
+// tcgen05 decode over a pool (bf16, d 128, G <= 16): every (layer, sequence, KV head)
+// of the call in one launch; p supplies q / out / lse ([nlayers][nseq][Hq][...]), the
+// scratch (partials for num_sms + items segments, one ticket per item), status, the
+// shape (Hq, Hkv, G, D, S, W) and the logit scale.
+cudaError_t launch_decode_pool_tc(const DecodeParams &p, const PoolDecodeCall &c, const int *layer_hr,
+                                  const int *layer_hs, int num_sms, cudaStream_t st);
+
+// Append of one token per listed sequence on every layer of a pool call (rows of the
+// retrieval pages and the sink / ring slots), also writing the block-table entries of
+// pages the step opens.  k, v [nlayers][nseq][Hkv][d].
+struct PoolAppendCall {
+  const PoolLayerDesc *layers;
+  int *table;
+  int pages_per_seq;
+  int layer0, nlayers, nseq, Hkv, D, S, W;
+  const char *k, *v;
+  int slot[kPoolMaxSeqs];
+  int pos[kPoolMaxSeqs];        // position of the token (tokens before it)
+  int page[kPoolMaxSeqs];       // physical page holding it
+  int new_page[kPoolMaxSeqs];   // 1: the step opens that page (write the table entry)
+};
+cudaError_t launch_pool_append(const PoolAppendCall &c, cudaStream_t st);
+// Append of n tokens of one sequence on one layer; pages[i] is the physical page of
+// logical page first_page + i (entries written to the table too).
+struct PoolChunkAppend {
+  const PoolLayerDesc *layer;
+  int *table;
+  int pages_per_seq, slot, Hkv, D, S, W, n, first_page, npages;
+  int64_t pos0, ring_from;
+  const char *k, *v;            // [n][Hkv][d]
+  int pages[256];
+};
+cudaError_t launch_pool_chunk_append(const PoolChunkAppend &c, int Hr, int Hs, cudaStream_t st);
+
 // decode tiling shared by host (split sizing) and device
 int decode_tokens_per_stage(duo_dtype dt, int D, bool int4);
 

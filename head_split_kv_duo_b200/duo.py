@@ -81,6 +81,31 @@ def lib() -> ctypes.CDLL:
                                               ctypes.c_float, vp, vp]
             L.duo_debug_launch_controls.restype = i32
             L.duo_debug_launch_controls.argtypes = [i32, i64]
+            L.duo_pool_bytes.restype = ctypes.c_size_t
+            L.duo_pool_bytes.argtypes = [i32, i32, i32, vp, i32, i32, i32, i64, i64, ctypes.POINTER(duo_opts)]
+            L.duo_pool_create.restype = i32
+            L.duo_pool_create.argtypes = [i32, i32, i32, vp, i32, i32, i32, i64, i64, ctypes.POINTER(duo_opts), vp,
+                                          ctypes.c_size_t, ctypes.POINTER(vp)]
+            L.duo_pool_destroy.restype = None
+            L.duo_pool_destroy.argtypes = [vp]
+            L.duo_pool_open.restype = i32
+            L.duo_pool_open.argtypes = [vp, vp, ctypes.POINTER(i32)]
+            L.duo_pool_close.restype = i32
+            L.duo_pool_close.argtypes = [vp, i32]
+            L.duo_pool_len.restype = i32
+            L.duo_pool_len.argtypes = [vp, i32, i32, ctypes.POINTER(i64)]
+            L.duo_pool_free_pages.restype = i32
+            L.duo_pool_free_pages.argtypes = [vp, ctypes.POINTER(i64)]
+            L.duo_pool_append_kv.restype = i32
+            L.duo_pool_append_kv.argtypes = [vp, i32, i32, vp, vp, i32, vp]
+            L.duo_pool_decode_step.restype = i32
+            L.duo_pool_decode_step.argtypes = [vp, i32, i32, i32, ctypes.POINTER(i32), vp, vp, vp, vp, vp, vp]
+            L.duo_pool_page.restype = i32
+            L.duo_pool_page.argtypes = [vp, i32, i32, ctypes.POINTER(i32)]
+            L.duo_pool_region.restype = i32
+            L.duo_pool_region.argtypes = [vp, i32, i32, ctypes.POINTER(vp), u64p]
+            L.duo_pool_device_status.restype = i32
+            L.duo_pool_device_status.argtypes = [vp, vp]
             _lib = L
     return _lib
 
@@ -184,6 +209,76 @@ def duo_gated_attention(q, k, v, batch, seq_len, q_heads, kv_heads, head_dim, dt
 
 def duo_debug_launch_controls(dry_run: int, fail_after: int) -> int:
     return lib().duo_debug_launch_controls(int(dry_run), int(fail_after))
+
+
+def duo_pool_bytes(layers, kv_heads, head_dim, retrieval_head_mask, S, W, max_seqs, max_len, num_pages,
+                   opts=None) -> int:
+    m = _mask_buf(retrieval_head_mask)
+    return int(lib().duo_pool_bytes(layers, kv_heads, head_dim, m, S, W, max_seqs, max_len, num_pages,
+                                    ctypes.byref(opts) if opts is not None else None))
+
+
+def duo_pool_create(layers, kv_heads, head_dim, retrieval_head_mask, S, W, max_seqs, max_len, num_pages, opts,
+                    dev_buf, dev_bytes):
+    """Returns (status, handle)."""
+    m = _mask_buf(retrieval_head_mask)
+    h = ctypes.c_void_p()
+    st = lib().duo_pool_create(layers, kv_heads, head_dim, m, S, W, max_seqs, max_len, num_pages,
+                               ctypes.byref(opts) if opts is not None else None, _ptr(dev_buf), int(dev_bytes),
+                               ctypes.byref(h))
+    return st, h
+
+
+def duo_pool_destroy(handle):
+    lib().duo_pool_destroy(handle)
+
+
+def duo_pool_open(handle, stream=None):
+    s = ctypes.c_int()
+    st = lib().duo_pool_open(handle, _ptr(stream), ctypes.byref(s))
+    return st, s.value
+
+
+def duo_pool_close(handle, seq) -> int:
+    return lib().duo_pool_close(handle, seq)
+
+
+def duo_pool_len(handle, seq, layer):
+    n = ctypes.c_int64()
+    st = lib().duo_pool_len(handle, seq, layer, ctypes.byref(n))
+    return st, n.value
+
+
+def duo_pool_free_pages(handle):
+    n = ctypes.c_int64()
+    st = lib().duo_pool_free_pages(handle, ctypes.byref(n))
+    return st, n.value
+
+
+def duo_pool_append_kv(handle, layer, seq, k, v, n, stream=None) -> int:
+    return lib().duo_pool_append_kv(handle, layer, seq, _ptr(k), _ptr(v), n, _ptr(stream))
+
+
+def duo_pool_decode_step(handle, layer0, nlayers, seqs, q, k, v, out, lse, stream=None) -> int:
+    arr = (ctypes.c_int * len(seqs))(*[int(x) for x in seqs])
+    return lib().duo_pool_decode_step(handle, layer0, nlayers, len(seqs), arr, _ptr(q), _ptr(k), _ptr(v), _ptr(out),
+                                      _ptr(lse), _ptr(stream))
+
+
+def duo_pool_page(handle, seq, logical_page):
+    p = ctypes.c_int()
+    st = lib().duo_pool_page(handle, seq, logical_page, ctypes.byref(p))
+    return st, p.value
+
+
+def duo_pool_region(handle, layer, which):
+    p, n = ctypes.c_void_p(), ctypes.c_uint64()
+    st = lib().duo_pool_region(handle, layer, which, ctypes.byref(p), ctypes.byref(n))
+    return st, (p.value or 0), n.value
+
+
+def duo_pool_device_status(handle, stream=None) -> int:
+    return lib().duo_pool_device_status(handle, _ptr(stream))
 
 
 # ---- torch-owned cache ----
@@ -314,6 +409,97 @@ class DuoCache:
         self._check(st, "duo_debug_region")
         off = ptr - self.buffer.data_ptr()
         return self.buffer[off:off + nbytes], cap
+
+
+class DuoPool:
+    """A paged pool of sequences (ragged batching) whose device storage is one torch uint8
+    buffer: bf16, head_dim 128."""
+
+    def __init__(self, layers, kv_heads, retrieval_mask, S, W, max_seqs, max_len, num_pages, *, q_heads=0,
+                 softmax_scale=0.0, device="cuda"):
+        self.layers, self.kv_heads, self.head_dim = layers, kv_heads, 128
+        self.S, self.W, self.max_seqs, self.max_len, self.num_pages = S, W, max_seqs, max_len, num_pages
+        self.q_heads = q_heads or kv_heads
+        self.mask = torch.as_tensor(retrieval_mask, dtype=torch.uint8).reshape(layers, kv_heads).clone()
+        self.opts = _opts(1, q_heads, DUO_BF16, DUO_KV_SAME, softmax_scale)
+        nbytes = duo_pool_bytes(layers, kv_heads, 128, self.mask, S, W, max_seqs, max_len, num_pages, self.opts)
+        if nbytes == 0:
+            raise DuoError(DUO_ERR_INVALID, "duo_pool_bytes")
+        self.buffer = torch.empty(nbytes + 256, dtype=torch.uint8, device=device)
+        base = (self.buffer.data_ptr() + 255) // 256 * 256
+        st, self.handle = duo_pool_create(layers, kv_heads, 128, self.mask, S, W, max_seqs, max_len, num_pages,
+                                          self.opts, base, nbytes)
+        if st != DUO_OK:
+            raise DuoError(st, "duo_pool_create")
+
+    def close(self):
+        if getattr(self, "handle", None):
+            duo_pool_destroy(self.handle)
+            self.handle = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+    def _check(self, st, what):
+        if st != DUO_OK:
+            raise DuoError(st, what)
+
+    def open(self, stream=None) -> int:
+        st, s = duo_pool_open(self.handle, _stream_ptr(stream))
+        self._check(st, "duo_pool_open")
+        return s
+
+    def close_seq(self, seq):
+        self._check(duo_pool_close(self.handle, seq), "duo_pool_close")
+
+    def len(self, seq, layer) -> int:
+        st, n = duo_pool_len(self.handle, seq, layer)
+        self._check(st, "duo_pool_len")
+        return n
+
+    def free_pages(self) -> int:
+        st, n = duo_pool_free_pages(self.handle)
+        self._check(st, "duo_pool_free_pages")
+        return n
+
+    def append_kv(self, layer, seq, k, v, stream=None):
+        """k, v [n][Hkv][128] bf16."""
+        n = k.shape[0]
+        for t, name in ((k, "k"), (v, "v")):
+            if t.dtype != torch.bfloat16 or tuple(t.shape) != (n, self.kv_heads, 128) or not t.is_contiguous():
+                raise ValueError(f"{name}: expected contiguous bf16 [{n}][{self.kv_heads}][128]")
+        self._check(duo_pool_append_kv(self.handle, layer, seq, k, v, n, _stream_ptr(stream)), "duo_pool_append_kv")
+
+    def decode_step(self, layer0, nlayers, seqs, q, k, v, out=None, lse=None, want_lse=True, stream=None):
+        """q [nlayers][nseq][Hq][128], k, v [nlayers][nseq][Hkv][128] bf16 -> (out, lse)."""
+        ns = len(seqs)
+        for t, name, h in ((q, "q", self.q_heads), (k, "k", self.kv_heads), (v, "v", self.kv_heads)):
+            if t.dtype != torch.bfloat16 or tuple(t.shape) != (nlayers, ns, h, 128) or not t.is_contiguous():
+                raise ValueError(f"{name}: expected contiguous bf16 [{nlayers}][{ns}][{h}][128]")
+        if out is None:
+            out = torch.empty_like(q)
+        if lse is None and want_lse:
+            lse = torch.empty(nlayers, ns, self.q_heads, dtype=torch.float32, device=q.device)
+        self._check(duo_pool_decode_step(self.handle, layer0, nlayers, seqs, q, k, v, out, lse, _stream_ptr(stream)),
+                    "duo_pool_decode_step")
+        return out, lse
+
+    def page(self, seq, logical_page) -> int:
+        st, p = duo_pool_page(self.handle, seq, logical_page)
+        self._check(st, "duo_pool_page")
+        return p
+
+    def region(self, layer, which):
+        st, ptr, nbytes = duo_pool_region(self.handle, layer, which)
+        self._check(st, "duo_pool_region")
+        off = ptr - self.buffer.data_ptr()
+        return self.buffer[off:off + nbytes]
+
+    def device_status(self, stream=None) -> int:
+        return duo_pool_device_status(self.handle, _stream_ptr(stream))
 
 
 def gated_attention(q, k, v, alpha, S, W, softmax_scale=0.0, out=None, stream=None):

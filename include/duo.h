@@ -266,6 +266,80 @@ DUO_API duo_status duo_decode_attention_static_scratch(duo_cache *cache, int lay
                                                        float *lse, void *cuda_stream);
 
 /*
+ * ---- Paged pool of sequences: ragged batching ----
+ *
+ * Sequences of different lengths share one caller-owned buffer (the pages name batched
+ * serving, and how the dual cache fits paged memory management, as open questions:
+ * "Critical Assessment").  Retrieval heads keep K/V in pages of 128 tokens: page p of
+ * layer l is [H_r(l)][128][d] and holds the same 128 positions of one sequence for all
+ * of the layer's retrieval heads; a sequence's logical page i is physical page
+ * table[slot][i] on every layer (a block table in the buffer, kept by the library).
+ * Streaming heads keep their sinks + ring per sequence slot, [slot][H_s][S+W][d], with
+ * the slot rule of duo_append_kv.  The host keeps every sequence's length per layer.
+ * bf16, head_dim 128, retrieval format DUO_KV_SAME, at most 16 query heads per KV head
+ * (else DUO_ERR_UNSUPPORTED).  Sequences are filled with duo_pool_append_kv and decoded
+ * with duo_pool_decode_step; pre-fill attention over a pool is not provided.  Calls on
+ * one pool must be ordered on one stream.  Errors follow the cache's contract: checked
+ * before any launch, lengths follow what the cache holds.
+ */
+typedef struct duo_pool duo_pool;
+
+/* Bytes of the pool buffer: max_seqs sequence slots, num_pages pages per layer, every
+ * sequence at most max_len tokens.  0 for invalid arguments. */
+DUO_API size_t duo_pool_bytes(int layers, int kv_heads, int head_dim, const uint8_t *retrieval_head_mask, int S, int W,
+                              int max_seqs, int64_t max_len, int64_t num_pages, const duo_opts *opts);
+
+/* Creates a pool over caller-owned device memory (>= duo_pool_bytes(), 256-byte
+ * aligned; the first launching call clears it).  opts->batch is ignored.  No device
+ * work happens here. */
+DUO_API duo_status duo_pool_create(int layers, int kv_heads, int head_dim, const uint8_t *retrieval_head_mask, int S,
+                                   int W, int max_seqs, int64_t max_len, int64_t num_pages, const duo_opts *opts,
+                                   void *dev_buf, size_t dev_bytes, duo_pool **out);
+DUO_API void duo_pool_destroy(duo_pool *pool); /* host handle only */
+
+/* Opens a sequence in a free slot (*seq), length 0 on every layer; its sink / ring rows
+ * are cleared on `cuda_stream`.  DUO_ERR_CAPACITY when every slot is open. */
+DUO_API duo_status duo_pool_open(duo_pool *pool, void *cuda_stream, int *seq);
+/* Closes a sequence: its pages return to the pool, its slot can be opened again. */
+DUO_API duo_status duo_pool_close(duo_pool *pool, int seq);
+DUO_API duo_status duo_pool_len(const duo_pool *pool, int seq, int layer, int64_t *len);
+DUO_API duo_status duo_pool_free_pages(const duo_pool *pool, int64_t *pages);
+
+/* Appends n >= 1 tokens (k, v [n][Hkv][d]) to one sequence on one layer, as
+ * duo_append_kv does for a cache: every retrieval row into the sequence's pages (new
+ * pages are taken from the pool; the rest of a page the call opens is cleared), sinks and
+ * the last min(n, W) positions into the ring.  DUO_ERR_CAPACITY past max_len or when
+ * the pool has too few free pages. */
+DUO_API duo_status duo_pool_append_kv(duo_pool *pool, int layer, int seq, const void *k, const void *v, int n,
+                                      void *cuda_stream);
+
+/*
+ * One decode step of a ragged batch: for each of the nseq listed sequences (host array
+ * `seqs`, distinct, open) and each layer layer0 .. layer0+nlayers-1, append the token
+ * (k, v [nlayers][nseq][Hkv][d]) at the sequence's length, then attend with its query
+ * (q [nlayers][nseq][Hq][d]) over that layer's cache ("Decoding Procedure", steps 2-5),
+ * writing out [nlayers][nseq][Hq][d] and lse [nlayers][nseq][Hq] (fp32, or NULL).  Two
+ * launches whatever nlayers and nseq: the append of every (layer, sequence, KV head),
+ * then one tcgen05 decode over all of them, each sequence at its own length.  Several
+ * layers in one call serve callers that hold the queries of those layers together (in
+ * a model, layer l+1's query depends on layer l's output, so a model step makes one call
+ * per layer).  A listed sequence must have the same length on every listed layer.
+ * nseq <= 128, nlayers * nseq <= 1024.  DUO_ERR_CAPACITY past max_len or without free
+ * pages; as for duo_append_decode, a failed attention launch leaves the tokens appended.
+ */
+DUO_API duo_status duo_pool_decode_step(duo_pool *pool, int layer0, int nlayers, int nseq, const int *seqs,
+                                        const void *q, const void *k, const void *v, void *out, float *lse,
+                                        void *cuda_stream);
+
+/* Physical page of a sequence's logical page (host bookkeeping, for inspection). */
+DUO_API duo_status duo_pool_page(const duo_pool *pool, int seq, int logical_page, int *physical_page);
+/* Device address and size of a layer's page array (DUO_REGION_RETR_K / _V,
+ * [pages][H_r][128][d]) or streaming array (DUO_REGION_STRM_K / _V, [slots][H_s][S+W][d]). */
+DUO_API duo_status duo_pool_region(const duo_pool *pool, int layer, duo_region which, void **ptr, uint64_t *bytes);
+/* Synchronises `cuda_stream`, reads and clears the pool's device status word. */
+DUO_API duo_status duo_pool_device_status(duo_pool *pool, void *cuda_stream);
+
+/*
  * Gated mixed attention of the identification phase ("Gate Parameterization"): over
  * whole sequences (positions 0..L-1, no cache), the output of every query head of KV
  * head g is
