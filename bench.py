@@ -15,9 +15,11 @@ is covered) and value is the median region, with the spread reported beside it.
 
 "workloads" holds every decode configuration on the same footing (Llama-2-7B MHA 32K
 at batch 1 and 8, Llama-3-8B GQA 128K at batch 1 and 4, the 1M-token 32-layer stack
-with INT4 retrieval heads): 5 regions of at least 100 ms of GPU time each, median and
-spread, its roofline against the measured HBM peak, the clocks seen, and the fp64
-oracle timed on the host cores on a bounded sample of the same workload.  The chunked
+with INT4 retrieval heads, Llama-3 128K with FP8 retrieval heads, a ragged batch of 8
+Llama-3 sequences from 2K to 128K tokens in the paged pool, and Llama-2 32K with the
+pool's 32-layers-per-launch step): 5 regions of at least 100 ms of GPU time each,
+median and spread, its roofline against the measured HBM peak, the clocks seen, and
+the fp64 oracle timed on the host cores on a bounded sample of the same workload.  The chunked
 pre-fill (256K prompt in 32K chunks, same shape; at least 5 runs) is reported under
 "prefill" with an oracle baseline extrapolated from sampled query rows, and the
 identification-phase gated forward (32K tokens) under "gated".
@@ -62,6 +64,14 @@ DECODE_WORKLOADS = {
     "llama2-7b-mha-decode-32k-b8": (32, 32, 8, 32768, 8, LAYERS, "same"),
     "llama3-8b-gqa-decode-1m-int4-32l": (32, 8, 4, 1 << 20, 1, LAYERS, "int4"),
     "llama3-8b-gqa-decode-128k-fp8-b1": (32, 8, 4, 131072, 1, LAYERS, "fp8"),
+}
+# pool (ragged batch) workloads: (q heads, kv heads, retrieval kv heads, contexts of the
+# sequences, layers, layers per decode_step call); every step appends one token to every
+# sequence on every layer and attends
+POOL_WORKLOADS = {
+    "llama3-8b-gqa-decode-ragged-8seq-32l": (32, 8, 4, [2048, 4096, 8192, 16384, 32768, 65536, 98304, 131072],
+                                             LAYERS, 1),
+    "llama2-7b-mha-decode-32k-b1-pool-32l-per-launch": (32, 32, 8, [32768], LAYERS, LAYERS),
 }
 REGIONS = 5              # timed regions per workload (median and spread reported)
 REGION_MS = 100.0        # GPU time per region of a workload entry, at least
@@ -369,6 +379,144 @@ def run_workload(name, dev, hbm_peak, peak_src):
     }
     run.close()
     return entry
+
+
+class PoolRun:
+    """A pool workload: every sequence filled to its context on every layer (one seeded
+    K/V draw per sequence, appended to each layer: the values do not change the work),
+    then steps of duo_pool_decode_step over all sequences."""
+
+    def __init__(self, name, dev, extra_tokens, nstep_in):
+        import torch
+
+        from head_split_kv_duo_b200 import inputs
+        from head_split_kv_duo_b200.duo import DuoPool
+
+        self.Hq, self.Hkv, self.nret, self.ctxs, self.layers, self.per_call = POOL_WORKLOADS[name]
+        self.Hr, self.Hs = self.nret, self.Hkv - self.nret
+        self.nseq = len(self.ctxs)
+        pages = sum((c + extra_tokens + 127) // 128 + 1 for c in self.ctxs)
+        mask = inputs.retrieval_mask(self.layers, self.Hkv, self.nret, seed=1)
+        self.pool = DuoPool(self.layers, self.Hkv, mask, S, W, self.nseq, max(self.ctxs) + extra_tokens, pages,
+                            q_heads=self.Hq, device=dev)
+        self.seqs = [self.pool.open() for _ in self.ctxs]
+        for i, c in enumerate(self.ctxs):
+            k = inputs.randn((c, self.Hkv, D), 400 + 2 * i, device=dev)
+            v = inputs.randn((c, self.Hkv, D), 401 + 2 * i, device=dev)
+            for layer in range(self.layers):
+                self.pool.append_kv(layer, self.seqs[i], k, v)
+            del k, v
+        torch.cuda.synchronize()
+        self.nin = nstep_in
+        self.qs = inputs.randn((nstep_in, self.layers, self.nseq, self.Hq, D), 17, device=dev)
+        self.ks = inputs.randn((nstep_in, self.layers, self.nseq, self.Hkv, D), 18, device=dev)
+        self.vs = inputs.randn((nstep_in, self.layers, self.nseq, self.Hkv, D), 19, device=dev)
+        self.out = torch.empty(self.layers, self.nseq, self.Hq, D, dtype=torch.bfloat16, device=dev)
+        self.lse = torch.empty(self.layers, self.nseq, self.Hq, dtype=torch.float32, device=dev)
+        self.stream = torch.cuda.current_stream()
+
+    def step(self, i, per_call=None):
+        per_call = per_call or self.per_call
+        j = i % self.nin
+        nbytes = 0
+        for l0 in range(0, self.layers, per_call):
+            sl = slice(l0, l0 + per_call)
+            for s in self.seqs:
+                nbytes += per_call * decode_bytes(self.pool.len(s, l0) + 1, B=1, Hr=self.Hr, Hs=self.Hs, Hq=self.Hq)
+            self.pool.decode_step(l0, per_call, self.seqs, self.qs[j, sl], self.ks[j, sl], self.vs[j, sl],
+                                  out=self.out[sl], lse=self.lse[sl], stream=self.stream)
+        return nbytes
+
+    def region(self, first, steps, per_call=None):
+        import torch
+        t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        torch.cuda.synchronize()
+        t0.record(self.stream)
+        nbytes = 0
+        for i in range(first, first + steps):
+            nbytes += self.step(i, per_call)
+        t1.record(self.stream)
+        torch.cuda.synchronize()
+        return t0.elapsed_time(t1), nbytes
+
+    def close(self):
+        import torch
+        assert self.pool.device_status() == 0, "device status word set"
+        self.pool.close()
+        del self.pool, self.qs, self.ks, self.vs
+        torch.cuda.empty_cache()
+
+
+def run_pool_workload(name, dev, hbm_peak, peak_src):
+    """A pool workload entry: REGIONS regions of at least REGION_MS, and the same steps
+    with all layers in one decode_step call when the workload makes one call per layer."""
+    warm, calib = 3, 2
+    extra = warm + calib + 2 * REGIONS * MAX_REGION_STEPS + 16
+    run = PoolRun(name, dev, extra, nstep_in=64)
+    for i in range(warm):
+        run.step(i)
+    ms, _ = run.region(warm, calib)
+    steps = max(1, min(MAX_REGION_STEPS, math.ceil(REGION_MS / (ms / calib))))
+    first = warm + calib
+    variants = [("per_call", run.per_call)] + ([("all_layers_one_call", run.layers)] if run.per_call < run.layers else [])
+    res = {}
+    with ClockSampler(dev.index) as clk:
+        for vname, per_call in variants:
+            regions = []
+            for r in range(REGIONS):
+                regions.append(run.region(first, steps, per_call))
+                first += steps
+            gbs = [b / (m * 1e-3) / 1e9 for m, b in regions]
+            med = sorted(range(REGIONS), key=lambda r: gbs[r])[REGIONS // 2]
+            calls = steps * (run.layers // per_call)
+            ms_med, bytes_med = regions[med]
+            res[vname] = {"layers_per_call": per_call, "gbs": round(gbs[med], 1),
+                          "us_per_token_layer": round(ms_med * 1e3 / (steps * run.layers), 3),
+                          "regions": dict(spread(gbs), unit="GB/s", steps_per_region=steps,
+                                          region_ms_median=round(ms_med, 2)),
+                          "roofline": roofline_entry(name, bytes_med / calls, ms_med / calls, hbm_peak, peak_src,
+                                                     "pool append, then pool decode (all sequences, "
+                                                     f"{per_call} layer(s) per launch)"),
+                          "gpu_launches": REGIONS * calls * 2}
+    entry = {"workload": name,
+             "config": {"q_heads": run.Hq, "kv_heads": run.Hkv, "head_dim": D, "retrieval_kv_heads": run.nret, "S": S,
+                        "W": W, "contexts": run.ctxs, "sequences": run.nseq, "layers": run.layers,
+                        "retrieval_kv": "same (paged)"},
+             "gbs": res["per_call"]["gbs"], "us_per_token_layer": res["per_call"]["us_per_token_layer"],
+             "regions": res["per_call"]["regions"], "roofline": res["per_call"]["roofline"],
+             "gpu_launches": res["per_call"]["gpu_launches"], "clocks": clk.summary()}
+    if "all_layers_one_call" in res:
+        entry["all_layers_one_call"] = res["all_layers_one_call"]
+    run.close()
+    return entry
+
+
+def oracle_pool_sample(name, seconds, device="cpu"):
+    """cpu_baseline of a pool workload: the oracle's decode of one layer of every
+    sequence (each at its own context) until `seconds` of wall time (at least one)."""
+    import numpy as np
+
+    import oracle
+    from head_split_kv_duo_b200 import inputs
+    Hq, Hkv, nret, ctxs, layers, _ = POOL_WORKLOADS[name]
+    mask = inputs.retrieval_mask(1, Hkv, nret, seed=1)[0].numpy().astype(bool)
+    data = []
+    for i, c in enumerate(ctxs):
+        k = _u16(inputs.randn((1, c, Hkv, D), 400 + 2 * i, device=device).cpu())
+        v = _u16(inputs.randn((1, c, Hkv, D), 401 + 2 * i, device=device).cpu())
+        q = _u16(inputs.randn((1, 1, Hq, D), 17 + i, device=device).cpu())
+        data.append((q, k, v, c))
+    n, t_total, nbytes = 0, 0.0, 0
+    while t_total < seconds or n == 0:
+        t = time.perf_counter()
+        for q, k, v, c in data:
+            oracle.attend(q, k, v, mask, S, W, pos0=c - 1)
+        t_total += time.perf_counter() - t
+        nbytes += sum(decode_bytes(c, B=1, Hr=nret, Hs=Hkv - nret, Hq=Hq) for c in ctxs)
+        n += 1
+    return {"value": round(nbytes / t_total / 1e9, 3), "unit": "GB/s", "cores": oracle.num_threads(), "kind": "oracle",
+            "sample": f"{n} oracle decode steps of one layer of all {len(ctxs)} sequences (contexts {ctxs}); "
+                      f"{t_total:.1f} s wall on {oracle.num_threads()} threads", "seconds": round(t_total, 2)}
 
 
 def run_headline(args, dev, dist, hbm_peak, peak_src):
@@ -735,13 +883,20 @@ def main():
     # the remaining configurations run on rank 0 only (each rank is an independent replica)
     if rank == 0:
         if args.workloads != "none":
-            names = sorted(DECODE_WORKLOADS) if args.workloads == "all" else args.workloads.split(",")
+            names = sorted(DECODE_WORKLOADS) + sorted(POOL_WORKLOADS) if args.workloads == "all" \
+                else args.workloads.split(",")
             res["workloads"] = {}
             for name in names:
-                e = run_workload(name, dev, hbm_peak, peak_src)
-                if not args.skip_cpu_baseline:
-                    cap = 1 << 17 if DECODE_WORKLOADS[name][6] == "int4" else None
-                    e["cpu_baseline"] = oracle_decode_sample(name, args.oracle_seconds, args.oracle_max_steps, cap, dev)
+                if name in POOL_WORKLOADS:
+                    e = run_pool_workload(name, dev, hbm_peak, peak_src)
+                    if not args.skip_cpu_baseline:
+                        e["cpu_baseline"] = oracle_pool_sample(name, args.oracle_seconds, dev)
+                else:
+                    e = run_workload(name, dev, hbm_peak, peak_src)
+                    if not args.skip_cpu_baseline:
+                        cap = 1 << 17 if DECODE_WORKLOADS[name][6] == "int4" else None
+                        e["cpu_baseline"] = oracle_decode_sample(name, args.oracle_seconds, args.oracle_max_steps,
+                                                                 cap, dev)
                 res["workloads"][name] = e
         if not args.skip_prefill:
             res["prefill"] = run_prefill(args, dev, tc_peak, tc_sust, peak_src)
