@@ -8,23 +8,27 @@
 //     depend on the chunk having been appended: the caller appends after it);
 //   * streaming heads: the staged history (sinks, then positions wstart..len-1) and
 //     the chunk's own keys, with the Lambda mask j < S or i - j < W.  Key tiles that
-//     hold no visible key for any row of a query tile are never loaded (tile skip).
+//     hold no visible key for any row of the CTA's query tiles are never loaded (tile
+//     skip).
 //
-// One CTA = one 128-row query tile (a GQA group of heads x 128/G positions); 19 warps:
-//   warp 0      TMA producer: Q once, then K tiles of 128 keys into a 3-stage ring
-//   warp 18     TMA producer: V tiles into a 2-stage ring
+// One CTA = two 128-row query tiles (each a GQA group of heads x 128/G positions, the
+// second following the first) that share every K/V tile it loads; 12 warps:
+//   warp 0      TMA producer: both Q tiles once, then K tiles of 128 keys (2-stage ring)
 //   warp 1      TMEM allocator; lane 0 issues every tcgen05.mma
-//   warps 2..17 softmax: four threads per query row (TMEM lane), 32 columns each, so
-//               that 16 warps hide the latency of the tensor-memory loads
-// TMEM (512 columns): S double buffer at 0 and 128, O accumulator at 256, P (bf16
-// pairs) double buffer at 384 and 448.
-//   S_j = Q K_j^T      (M 128, N 128, K 128: 8 MMAs of K 16), into S[j % 2]
-//   O += P_j V_j       (M 128, N 128, K 128 keys), A = P_j from TMEM, B = V_j (smem)
-// The softmax warps read S_j once from TMEM, release it, and write P_j (bf16) back
-// into TMEM; O stays in TMEM and is rescaled there only when a row's maximum grows
-// past its reference by 2^8.  K stages are released as soon as S_j is computed and V
-// stages once P_j V_j is, so the tensor core computes S_{j+1} and P_j V_j while the
-// softmax warps work.
+//   warp 2      TMA producer: V tiles (2-stage ring)
+//   warps 4..7  softmax of query tile 0, warps 8..11 of query tile 1: one thread per
+//               query row (TMEM lane), all 128 logits of a key tile in registers
+// TMEM (512 columns): S_t at 128 t, O_t at 256 + 128 t for query tile t; the softmax
+// writes P_t (bf16 pairs) over the first 64 columns of S_t.
+//   S_t(j) = Q_t K_j^T   (M 128, N 128, K 128: 8 MMAs of K 16), into S_t
+//   O_t += P_t(j) V_j    (M 128, N 128, K 128 keys), A = P_t(j) from TMEM, B = V_j (smem)
+// The MMA thread issues PV_0(j), S_0(j+1), PV_1(j), S_1(j+1), ...: the tensor core
+// works on one query tile while the other tile's softmax runs (ping-pong).  tcgen05.mma
+// operations of one thread complete in issue order, so S_t(j+1) overwrites P_t(j) only
+// after PV_t(j) has read it, and when S_t(j) has landed PV_t(j-1) has too: O_t may then
+// be rescaled in place.  The running max m is a reference: P = exp2(s*c - m) may exceed
+// 1 by up to 2^kSlack, and m (with O and l) is rescaled only when a row's tile maximum
+// passes m + kSlack.
 //
 // Every mbarrier wait is bounded; a wait that runs out latches kDevTimeout in the
 // status word and sets an abort flag so that every role drains and exits (the
@@ -37,36 +41,34 @@ namespace {
 
 constexpr int kBM = 128;  // query rows per tile
 constexpr int kBN = 128;  // keys per tile
-constexpr int kSplit = 4;                      // softmax threads per query row
-constexpr int kCols = kBN / kSplit;            // S, P and O columns per softmax thread
-constexpr int kVWarp = 2 + 4 * kSplit;         // the V producer follows the softmax warps
-constexpr int kTcThreads = 32 * (kVWarp + 1);  // warp 0 K/Q TMA, warp 1 MMA + TMEM, softmax, V TMA
+constexpr int kQT = 2;    // query tiles per CTA
+constexpr int kSoftWarp0 = 4;                       // first softmax warp (tile t: warps 4 + 4t .. 7 + 4t)
+constexpr int kTcThreads = 32 * (kSoftWarp0 + 4 * kQT);
 constexpr int kD = 128;
-constexpr int kKStages = 3;  // K ring: a stage is free once S_j is computed
-constexpr int kVStages = 2;  // V ring: a stage is free once P_j V_j is computed
+constexpr int kKStages = 2;  // K ring: a stage is free once S_1(j) is computed
+constexpr int kVStages = 2;  // V ring: a stage is free once P_1(j) V_j is computed
 constexpr int kMaxStrmTiles = 48;
+constexpr int kPolyExp = 12;  // exponentials of every 32 (interior tiles) on the FMA pipe
 
 // shared memory map (bytes from the 1 KiB-aligned base); every tile is two 128B-swizzled
 // [128][64] bf16 halves of 16 KiB
-constexpr int kSmQ = 0;
-constexpr int kSmK = 32768;                         // K stage s at kSmK + s * 32 KiB
+constexpr int kSmQ = 0;                             // query tile t at kSmQ + t * 32 KiB
+constexpr int kSmK = kQT * 32768;                   // K stage s at kSmK + s * 32 KiB
 constexpr int kSmV = kSmK + kKStages * 32768;       // V stage s at kSmV + s * 32 KiB
 constexpr int kSmBar = kSmV + kVStages * 32768;
 constexpr int kSmMisc = kSmBar + 256;
-constexpr int kSmXchg = kSmMisc + 1024 + kMaxStrmTiles * 16;  // row max / sum exchange, 3 kSplit x 128 floats
-constexpr int kSmTotal = kSmXchg + 3 * kSplit * 128 * 4;
+constexpr int kSmTotal = kSmMisc + 1024 + kMaxStrmTiles * 16;
 constexpr int kSmemAlloc = kSmTotal + 1024;  // slack for aligning the base to 1 KiB
 
-// TMEM columns: S double buffer, O accumulator, P double buffer (bf16 pairs, A operand)
-constexpr int kTmS = 0, kTmO = 256, kTmP = 384;
+// TMEM columns of query tile t: S_t (P_t over its first 64) and O_t
+constexpr int kTmS = 0, kTmO = 256;
 
-// barrier indices (8 bytes each).  Double-buffered resources (S, P) have one barrier
-// per buffer, so that no barrier can complete two phases ahead of a thread waiting on
-// it (parity waits).
+// barrier indices (8 bytes each)
 constexpr int kBarQ = 0, kBarKFull = 1, kBarKEmpty = kBarKFull + kKStages, kBarVFull = kBarKEmpty + kKStages,
-              kBarVEmpty = kBarVFull + kVStages, kBarSFull = kBarVEmpty + kVStages, kBarSFree = kBarSFull + 2,
-              kBarPFull = kBarSFree + 2, kBarOFull = kBarPFull + 2, kBarDrain = kBarOFull + 1, kNumBars = kBarDrain + 1;
+              kBarVEmpty = kBarVFull + kVStages, kBarSFull = kBarVEmpty + kVStages, kBarPFull = kBarSFull + kQT,
+              kBarOFull = kBarPFull + kQT, kBarDrain = kBarOFull + kQT, kNumBars = kBarDrain + 1;
 static_assert(kNumBars * 8 <= 256, "barrier area");
+static_assert(kSmemAlloc <= 227 * 1024, "shared memory");
 
 struct TileDesc {
   int src;      // 0 retrieval cache, 1 streaming history, 2 chunk input
@@ -157,17 +159,18 @@ __device__ __forceinline__ void exp2_poly2(uint64_t x2, float &r0, float &r1) {
   r1 = __int_as_float(__float_as_int(q1) + (__float_as_int(t1) << 23));
 }
 
-// exp2(v*c - mc) of N logits, their sum into rowsum and bf16 pairs into pk; logits
+// exp2(v*c - mc) of the N logits v[B .. B+N), their sum into rowsum and bf16 pairs into pk; logits
 // [P0, P0+PN) use the FMA-pipe polynomial (which needs finite arguments), the rest MUFU.
 // The scaling and the sums run on packed fp32 pairs.
-template <int N, int P0, int PN>
-__device__ __forceinline__ void probabilities(const float (&v)[N], float c, float mc, float &rowsum,
+template <int N, int P0, int PN, int B = 0, int M>
+__device__ __forceinline__ void probabilities(const float (&v)[M], float c, float mc, float &rowsum,
                                               uint32_t (&pk)[N / 2]) {
+  static_assert(B + N <= M, "logit range");
   const uint64_t cc = pack2(c, c), mm = pack2(-mc, -mc);
   uint64_t acc[2] = {pack2(0.f, 0.f), pack2(0.f, 0.f)};
 #pragma unroll
   for (int e = 0; e < N; e += 2) {
-    const uint64_t x = ffma2(pack2(v[e], v[e + 1]), cc, mm);
+    const uint64_t x = ffma2(pack2(v[B + e], v[B + e + 1]), cc, mm);
     float p0, p1;
     if (e >= P0 && e < P0 + PN) {
       exp2_poly2(x, p0, p1);
@@ -218,6 +221,48 @@ __device__ __forceinline__ void load_tile(const TcArgs &a, const TileDesc &t, co
 
 // ---------------------------------------------------------------- the kernel
 
+// 128 consecutive fp32 columns of this thread's lane: four loads, one wait that names
+// every destination register (so that no use is scheduled before it)
+#define DUO_R4(x) "+r"(r[(x)]), "+r"(r[(x) + 1]), "+r"(r[(x) + 2]), "+r"(r[(x) + 3])
+#define DUO_R16(x) DUO_R4(x), DUO_R4((x) + 4), DUO_R4((x) + 8), DUO_R4((x) + 12)
+#define DUO_O4(x) "=r"(r[(x)]), "=r"(r[(x) + 1]), "=r"(r[(x) + 2]), "=r"(r[(x) + 3])
+#define DUO_O16(x) DUO_O4(x), DUO_O4((x) + 4), DUO_O4((x) + 8), DUO_O4((x) + 12)
+__device__ __forceinline__ void ld128(uint32_t taddr, float (&v)[128]) {
+  uint32_t r[128];
+#pragma unroll
+  for (int c = 0; c < 4; ++c) {
+    uint32_t *q = r + 32 * c;
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+        "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, "
+        "%16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];"
+        : "=r"(q[0]), "=r"(q[1]), "=r"(q[2]), "=r"(q[3]), "=r"(q[4]), "=r"(q[5]), "=r"(q[6]), "=r"(q[7]), "=r"(q[8]),
+          "=r"(q[9]), "=r"(q[10]), "=r"(q[11]), "=r"(q[12]), "=r"(q[13]), "=r"(q[14]), "=r"(q[15]), "=r"(q[16]),
+          "=r"(q[17]), "=r"(q[18]), "=r"(q[19]), "=r"(q[20]), "=r"(q[21]), "=r"(q[22]), "=r"(q[23]), "=r"(q[24]),
+          "=r"(q[25]), "=r"(q[26]), "=r"(q[27]), "=r"(q[28]), "=r"(q[29]), "=r"(q[30]), "=r"(q[31])
+        : "r"(taddr + 32 * c));
+  }
+  asm volatile("tcgen05.wait::ld.sync.aligned;"
+               : DUO_R16(0), DUO_R16(16), DUO_R16(32), DUO_R16(48), DUO_R16(64), DUO_R16(80), DUO_R16(96), DUO_R16(112)
+               :
+               : "memory");
+#pragma unroll
+  for (int i = 0; i < 128; ++i) v[i] = __uint_as_float(r[i]);
+}
+#undef DUO_R4
+#undef DUO_R16
+#undef DUO_O4
+#undef DUO_O16
+
+// P of logits v[B .. B+32) as 16 bf16 pairs into TMEM columns B/2 .. B/2+15 of s_cols
+// (no wait), their sum into rs; PN of the 32 exponentials on the FMA pipe
+template <int B, int PN>
+__device__ __forceinline__ void p_chunk(const float (&v)[128], float c, float mc, float &rs, uint32_t s_cols) {
+  uint32_t pk[16];
+  probabilities<32, 0, PN, B>(v, c, mc, rs, pk);
+  tc::st16(s_cols + B / 2, pk);
+}
+
 __global__ void __launch_bounds__(kTcThreads, 1) prefill_tc_kernel(const __grid_constant__ TcArgs a) {
   const PrefillParams &p = a.p;
   extern __shared__ char smem_raw[];
@@ -232,17 +277,19 @@ __global__ void __launch_bounds__(kTcThreads, 1) prefill_tc_kernel(const __grid_
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
 
-  // ---- which query tile ----
-  // GQA packing: the 128 rows of the tile are npos = 128 / G consecutive positions x the
-  // G query heads of one KV head (row r = position r / G, head r % G), so every K/V tile
-  // a CTA loads serves the whole group.
+  // ---- which query tiles ----
+  // GQA packing: the 128 rows of a query tile are npos = 128 / G consecutive positions x
+  // the G query heads of one KV head (row r = position r / G, head r % G), so every K/V
+  // tile a CTA loads serves the whole group, for both of its query tiles.
   const int G = p.G;
   const int npos = kBM / G;
-  const int ntq = (p.n + npos - 1) / npos;
+  const int ntq = (p.n + npos - 1) / npos;         // query tiles of one (sequence, KV head)
+  const int ncta = (ntq + kQT - 1) / kQT;
   const int bg = blockIdx.x % (p.B * p.Hkv);
-  const int qt = ntq - 1 - blockIdx.x / (p.B * p.Hkv);  // heaviest (latest) blocks first
+  const int qc = ncta - 1 - blockIdx.x / (p.B * p.Hkv);  // heaviest (latest) blocks first
   const int b = bg / p.Hkv, g = bg % p.Hkv;
-  const int r0 = qt * npos;  // first chunk row (position offset) of the block
+  const int r0 = qc * kQT * npos;                   // first chunk row (position offset) of the CTA
+  const int nq = (ntq - qc * kQT) < kQT ? (ntq - qc * kQT) : kQT;  // query tiles present (1 or 2)
   Plan pl;
   pl.retr = p.hm.is_retr[g] != 0;
   pl.nh = pl.retr ? static_cast<int>((p.len + kBN - 1) / kBN) : 0;
@@ -250,17 +297,16 @@ __global__ void __launch_bounds__(kTcThreads, 1) prefill_tc_kernel(const __grid_
   pl.kvrow = b * (pl.retr ? p.Hr : p.HsMax) + p.hm.kind_idx[g];
 
   if (tid == 0) {
-    for (int i = 0; i < kNumBars; ++i)
-      mbar_init(bar(i), (i == kBarSFree || i == kBarSFree + 1 || i == kBarPFull || i == kBarPFull + 1) ? 128 * kSplit : 1);
+    for (int i = 0; i < kNumBars; ++i) mbar_init(bar(i), (i >= kBarPFull && i < kBarPFull + kQT) ? kBM : 1);
     if (smem_u32(smem) & 1023u) flag_status(p.status, kDevTimeout);  // layout assumption (never expected)
     fence_mbar_init();
     *abort_flag = 0;
     int nt;
+    const int rows = (r0 + nq * npos < p.n) ? r0 + nq * npos : p.n;  // chunk rows 0 .. rows-1 are needed
     if (pl.retr) {
-      const int rows = (r0 + npos < p.n) ? r0 + npos : p.n;  // chunk rows 0 .. rows-1 are needed
       nt = pl.nh + (rows + kBN - 1) / kBN;
     } else {
-      nt = streaming_tiles(p, r0, npos, tl);
+      nt = streaming_tiles(p, r0, rows - r0, tl);
     }
     *ntiles_sm = nt;
   }
@@ -272,12 +318,14 @@ __global__ void __launch_bounds__(kTcThreads, 1) prefill_tc_kernel(const __grid_
   const int nt = *ntiles_sm;
 
   if (warp == 0) {
-    // ================= TMA producer: Q, then the K ring =================
+    // ================= TMA producer: the Q tiles, then the K ring =================
     if (lane == 0) {
       tc::prefetch_map(&a.tm_q);
-      mbar_expect_tx(bar(kBarQ), 32768);
-      tc::tma_4d(sbase + kSmQ, &a.tm_q, 0, g * G, r0, b, bar(kBarQ));  // box: 64 dims x G heads x npos positions
-      tc::tma_4d(sbase + kSmQ + 16384, &a.tm_q, 64, g * G, r0, b, bar(kBarQ));
+      mbar_expect_tx(bar(kBarQ), 32768 * nq);
+      for (int t = 0; t < nq; ++t) {  // box: 64 dims x G heads x npos positions
+        tc::tma_4d(sbase + kSmQ + t * 32768, &a.tm_q, 0, g * G, r0 + t * npos, b, bar(kBarQ));
+        tc::tma_4d(sbase + kSmQ + t * 32768 + 16384, &a.tm_q, 64, g * G, r0 + t * npos, b, bar(kBarQ));
+      }
       int issued = 0;
       for (int j = 0; j < nt; ++j) {
         const int s = j % kKStages;
@@ -292,7 +340,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) prefill_tc_kernel(const __grid_
       mbar_wait(bar(kBarQ), 0, p.status);
       tc::drain_loads(bar(kBarKFull), kKStages, issued, p.status);
     }
-  } else if (warp == kVWarp) {
+  } else if (warp == 2) {
     // ================= TMA producer: the V ring =================
     if (lane == 0) {
       int issued = 0;
@@ -312,68 +360,76 @@ __global__ void __launch_bounds__(kTcThreads, 1) prefill_tc_kernel(const __grid_
     if (lane == 0) {
       constexpr uint32_t kIdS = tc::idesc_bf16(kBM, kBN, false, false);
       constexpr uint32_t kIdPV = tc::idesc_bf16(kBM, kD, false, true);
-      bool ok = tc::wait_bar(bar(kBarQ), 0, p.status, abort_flag);
-      auto issue_pv = [&](int jj) {
-        // O += P_jj V_jj : K = 128 keys in 8 steps of 16; P from TMEM (bf16 pairs, K-major),
-        // V from shared memory (d contiguous, MN-major)
-        const int sv = jj % kVStages;
-        const uint32_t vbase = sbase + kSmV + sv * 32768;
-        const uint32_t pcol = tmem + kTmP + (jj & 1) * 64;
-        for (int kk = 0; kk < 8; ++kk) {
-          const uint64_t bd = tc::sdesc(vbase + kk * 2048, 16384, 1024);
-          tc::mma_ts(tmem + kTmO, pcol + kk * 8, bd, kIdPV, (jj > 0 || kk > 0) ? 1u : 0u);
-        }
-        tc::commit(bar(kBarOFull));
-        tc::commit(bar(kBarVEmpty + sv));
-      };
-      for (int j = 0; j < nt && ok; ++j) {
-        const int sk = j % kKStages;
-        if (!tc::wait_bar(bar(kBarKFull + sk), (j / kKStages) & 1, p.status, abort_flag)) { ok = false; break; }
-        if (j >= 2 && !tc::wait_bar(bar(kBarSFree + (j & 1)), ((j - 2) >> 1) & 1, p.status, abort_flag)) { ok = false; break; }
-        tc::fence_after();
-        // S_j = Q K_j^T : K = d 128 in 8 steps of 16; Q and K are K-major
-        const uint32_t kbase = sbase + kSmK + sk * 32768;
+      // S_t(j) = Q_t K_j^T : K = d 128 in 8 steps of 16; Q and K are K-major
+      auto issue_s = [&](int t, int j) {
+        const uint32_t kbase = sbase + kSmK + (j % kKStages) * 32768, qbase = sbase + kSmQ + t * 32768;
         for (int kk = 0; kk < 8; ++kk) {
           const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
-          tc::mma_ss(tmem + kTmS + (j & 1) * 128, tc::sdesc(sbase + kSmQ + off, 16, 1024),
-                     tc::sdesc(kbase + off, 16, 1024), kIdS, kk > 0 ? 1u : 0u);
+          tc::mma_ss(tmem + kTmS + t * 128, tc::sdesc(qbase + off, 16, 1024), tc::sdesc(kbase + off, 16, 1024), kIdS,
+                     kk > 0 ? 1u : 0u);
         }
-        tc::commit(bar(kBarSFull + (j & 1)));
-        tc::commit(bar(kBarKEmpty + sk));
-        if (j >= 1) {
-          if (!tc::wait_bar(bar(kBarPFull + ((j - 1) & 1)), ((j - 1) >> 1) & 1, p.status, abort_flag)) { ok = false; break; }
-          if (!tc::wait_bar(bar(kBarVFull + ((j - 1) % kVStages)), ((j - 1) / kVStages) & 1, p.status, abort_flag)) { ok = false; break; }
-          tc::fence_after();
-          issue_pv(j - 1);
+        tc::commit(bar(kBarSFull + t));
+      };
+      // O_t += P_t(j) V_j : K = 128 keys in 8 steps of 16; P from TMEM (bf16 pairs,
+      // K-major), V from shared memory (d contiguous, MN-major)
+      auto issue_pv = [&](int t, int j) {
+        const uint32_t vbase = sbase + kSmV + (j % kVStages) * 32768;
+        for (int kk = 0; kk < 8; ++kk) {
+          const uint64_t bd = tc::sdesc(vbase + kk * 2048, 16384, 1024);
+          tc::mma_ts(tmem + kTmO + t * 128, tmem + kTmS + t * 128 + kk * 8, bd, kIdPV, (j > 0 || kk > 0) ? 1u : 0u);
         }
-      }
-      if (ok && nt > 0 && tc::wait_bar(bar(kBarPFull + ((nt - 1) & 1)), ((nt - 1) >> 1) & 1, p.status, abort_flag) &&
-          tc::wait_bar(bar(kBarVFull + ((nt - 1) % kVStages)), ((nt - 1) / kVStages) & 1, p.status, abort_flag)) {
+      };
+      bool ok = nt > 0 && tc::wait_bar(bar(kBarQ), 0, p.status, abort_flag) &&
+                tc::wait_bar(bar(kBarKFull), 0, p.status, abort_flag);
+      if (ok) {
         tc::fence_after();
-        issue_pv(nt - 1);
+        for (int t = 0; t < nq; ++t) issue_s(t, 0);
+        tc::commit(bar(kBarKEmpty));
+      }
+      for (int j = 0; j < nt && ok; ++j) {
+        for (int t = 0; t < nq && ok; ++t) {
+          if (!tc::wait_bar(bar(kBarPFull + t), j & 1, p.status, abort_flag)) { ok = false; break; }
+          if (t == 0 &&
+              !tc::wait_bar(bar(kBarVFull + (j % kVStages)), (j / kVStages) & 1, p.status, abort_flag)) {
+            ok = false;
+            break;
+          }
+          tc::fence_after();
+          issue_pv(t, j);
+          if (t == nq - 1) tc::commit(bar(kBarVEmpty + (j % kVStages)));
+          if (j + 1 < nt) {
+            if (t == 0) {
+              if (!tc::wait_bar(bar(kBarKFull + ((j + 1) % kKStages)), ((j + 1) / kKStages) & 1, p.status,
+                                abort_flag)) {
+                ok = false;
+                break;
+              }
+              tc::fence_after();
+            }
+            issue_s(t, j + 1);
+            if (t == nq - 1) tc::commit(bar(kBarKEmpty + ((j + 1) % kKStages)));
+          } else {
+            tc::commit(bar(kBarOFull + t));
+          }
+        }
       }
       // drain: every MMA this thread issued has completed before TMEM is freed
       tc::commit(bar(kBarDrain));
       mbar_wait(bar(kBarDrain), 0, p.status);
     }
-  } else {
-    // ================= softmax: 4 kSplit warps, kSplit threads per query row =================
-    // Warp w reads TMEM lanes 32*(w%4).. (rows) and columns [kCols*part, kCols*part+kCols)
-    // of S, O and P.  The running max m is a reference: P = exp2(s*c - m) may exceed 1 by
-    // up to 2^kSlack, and m (with O in TMEM and l) is rescaled only when a row's tile
-    // maximum passes m + kSlack.  S is read from TMEM once per tile.
+  } else if (warp >= kSoftWarp0 && (warp - kSoftWarp0) / 4 < nq) {
+    // ================= softmax of query tile qt: one thread per query row =================
     constexpr float kSlack = 8.0f;
-    constexpr int kSoft = 128 * kSplit;  // softmax threads (named barrier 1)
+    const int qt = (warp - kSoftWarp0) >> 2;
     const int wq = warp & 3;
-    const int part = (warp - 2) >> 2;
     const int row = (wq << 5) | lane;
     const uint32_t lane_base = tmem + (static_cast<uint32_t>(wq << 5) << 16);
-    const int rpos = row / G;                  // position offset of this row within the block
+    const uint32_t s_cols = lane_base + kTmS + qt * 128, o_cols = lane_base + kTmO + qt * 128;
+    const int rpos = qt * npos + row / G;      // position offset of this row within the CTA
     const int h = g * G + row % G;             // its query head
     const int64_t i = pl.q0 + rpos;            // absolute query position
     const float c = p.scale_log2;
     float m = -INFINITY, l = 0.f;
-    float *xch = reinterpret_cast<float *>(smem + kSmXchg);  // [tile parity][part][row] partial maxima
     bool ok = true;
 
     for (int j = 0; j < nt; ++j) {
@@ -404,33 +460,27 @@ __global__ void __launch_bounds__(kTcThreads, 1) prefill_tc_kernel(const __grid_
           win_c = clamp_col(win_rel);
         }
       }
-      const bool full_vis = hi >= kBN - 1 && (sink_c >= kBN || win_c < 0);
+      // warp-uniform (the branches below issue warp-collective TMEM stores): a warp
+      // with any masked row takes the masked path, a no-op for its other rows
+      const bool full_vis = __all_sync(0xffffffffu, hi >= kBN - 1 && (sink_c >= kBN || win_c < 0));
 
-      if (ok) ok = tc::wait_bar(bar(kBarSFull + (j & 1)), (j >> 1) & 1, p.status, abort_flag);
+      if (ok) ok = tc::wait_bar(bar(kBarSFull + qt), j & 1, p.status, abort_flag);
       tc::fence_after();
-      // this thread's kCols logits of S_j, then the S buffer is released
-      float v[kCols];
-      tc::ld<kCols>(lane_base + kTmS + (j & 1) * 128 + part * kCols, v);
-      tc::fence_before();
-      mbar_arrive(bar(kBarSFree + (j & 1)));
+      float v[128];
+      ld128(s_cols, v);
       if (!full_vis) {
 #pragma unroll
-        for (int e = 0; e < kCols; ++e) {
-          const int col = part * kCols + e;
-          const bool vis = col <= hi && (col < sink_c || col > win_c);
+        for (int e = 0; e < 128; ++e) {
+          const bool vis = e <= hi && (e < sink_c || e > win_c);
           v[e] = vis ? v[e] : -INFINITY;
         }
       }
-      float mx4[4];  // four independent chains of three-input maxima
+      float mx8[8];  // eight independent chains of three-input maxima
 #pragma unroll
-      for (int u = 0; u < 4; ++u) mx4[u] = fmaxf(v[2 * u], v[2 * u + 1]);
+      for (int u = 0; u < 8; ++u) mx8[u] = fmaxf(v[2 * u], v[2 * u + 1]);
 #pragma unroll
-      for (int e = 8; e < kCols; e += 2) mx4[(e >> 1) & 3] = fmax3(mx4[(e >> 1) & 3], v[e], v[e + 1]);
-      float mx = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3]));
-      xch[((j & 1) * kSplit + part) * kBM + row] = mx;
-      tc::named_sync(1, kSoft);
-#pragma unroll
-      for (int o = 1; o < kSplit; ++o) mx = fmaxf(mx, xch[((j & 1) * kSplit + ((part + o) % kSplit)) * kBM + row]);
+      for (int e = 16; e < 128; e += 2) mx8[(e >> 1) & 7] = fmax3(mx8[(e >> 1) & 7], v[e], v[e + 1]);
+      const float mx = fmaxf(fmaxf(fmax3(mx8[0], mx8[1], mx8[2]), fmax3(mx8[3], mx8[4], mx8[5])), fmaxf(mx8[6], mx8[7]));
       const float tmax = mx * c;  // -inf when nothing in the tile is visible
       const bool need = tmax > m + kSlack;
       float alpha = 1.f;
@@ -438,64 +488,59 @@ __global__ void __launch_bounds__(kTcThreads, 1) prefill_tc_kernel(const __grid_
         alpha = ex2(m - tmax);  // 0 while m is -inf
         m = tmax;
       }
-      l *= alpha;
-      bool waited = false;
       if (j >= 1 && __any_sync(0xffffffffu, need)) {
-        // rescale this thread's kCols columns of O once P_{j-1} V_{j-1} has landed
-        if (ok) ok = tc::wait_bar(bar(kBarOFull), (j - 1) & 1, p.status, abort_flag);
-        tc::fence_after();
-        float w[kCols];
-        const uint32_t oa = lane_base + kTmO + part * kCols;
-        tc::ld<kCols>(oa, w);
+        // rescale this row of O_t: S_t(j) has landed, so P_t(j-1) V_{j-1} has too
+#pragma unroll 1
+        for (int q = 0; q < 4; ++q) {
+          float w[32];
+          tc::ld<32>(o_cols + 32 * q, w);
 #pragma unroll
-        for (int e = 0; e < kCols; ++e) w[e] *= alpha;
-        tc::st32(oa, w);
-        waited = true;
+          for (int e = 0; e < 32; ++e) w[e] *= alpha;
+          tc::st32(o_cols + 32 * q, w);
+        }
       }
-      // probabilities (masked logits are -inf and give 0), row sum, bf16 pairs of P_j
-      float rsum;
+      // probabilities (masked logits are -inf and give 0), row sum, bf16 pairs of P_t(j)
+      // over the first 64 columns of S_t
       const float mc = (m == -INFINITY) ? 0.f : m;
-      uint32_t pk[kCols / 2];
-      // 3/8 of the exponentials of interior tiles on the FMA pipe, the rest on MUFU
-      if (!full_vis) probabilities<kCols, 0, 0>(v, c, mc, rsum, pk);
-      else probabilities<kCols, 0, kCols * 3 / 8>(v, c, mc, rsum, pk);
-      // P_j into TMEM buffer j % 2 (its previous reader P_{j-2} V_{j-2} was waited for at j-1)
-      tc::st16(lane_base + kTmP + (j & 1) * 64 + part * (kCols / 2), pk);
-      tc::st_wait();
-      // one wait per P V product, in order (here unless the rescale already waited)
-      if (j >= 1 && !waited) {
-        if (ok) ok = tc::wait_bar(bar(kBarOFull), (j - 1) & 1, p.status, abort_flag);
+      float rs[4];
+      if (!full_vis) {
+        p_chunk<0, 0>(v, c, mc, rs[0], s_cols);
+        p_chunk<32, 0>(v, c, mc, rs[1], s_cols);
+        p_chunk<64, 0>(v, c, mc, rs[2], s_cols);
+        p_chunk<96, 0>(v, c, mc, rs[3], s_cols);
+      } else {
+        p_chunk<0, kPolyExp>(v, c, mc, rs[0], s_cols);
+        p_chunk<32, kPolyExp>(v, c, mc, rs[1], s_cols);
+        p_chunk<64, kPolyExp>(v, c, mc, rs[2], s_cols);
+        p_chunk<96, kPolyExp>(v, c, mc, rs[3], s_cols);
       }
-      l += rsum;
+      const float rsum = (rs[0] + rs[1]) + (rs[2] + rs[3]);
+      tc::st_wait();
       tc::fence_before();
-      mbar_arrive(bar(kBarPFull + (j & 1)));
+      mbar_arrive(bar(kBarPFull + qt));
+      l = l * alpha + rsum;
     }
-    // the last product, then the row's normaliser from all parts
-    if (nt > 0 && ok) ok = tc::wait_bar(bar(kBarOFull), (nt - 1) & 1, p.status, abort_flag);
+    // the last product, then the epilogue: normalise and store the row (bf16) and its
+    // lse; in gated mixing, blend with the row already in out
+    if (nt > 0 && ok) ok = tc::wait_bar(bar(kBarOFull + qt), 0, p.status, abort_flag);
     tc::fence_after();
-    float *xl = xch + 2 * kSplit * kBM;  // [part][row]
-    xl[part * kBM + row] = l;
-    tc::named_sync(1, kSoft);
-    float lrow = 0.f;
-#pragma unroll
-    for (int o = 0; o < kSplit; ++o) lrow += xl[o * kBM + row];
-    // epilogue: normalise and store this thread's kCols dims of the row (bf16) and its lse;
-    // in gated mixing, blend with the row already in out
     const bool store = r0 + rpos < p.n;
-    char *orow = p.out + ((static_cast<int64_t>(b) * p.n + r0 + rpos) * p.Hq + h) * (kD * 2) + part * (kCols * 2);
-    const float inv = 1.f / lrow;
+    char *orow = p.out + ((static_cast<int64_t>(b) * p.n + r0 + rpos) * p.Hq + h) * (kD * 2);
+    const float inv = 1.f / l;
     const float mixa = p.mix_alpha ? p.mix_alpha[g] : 0.f;
-    {
-      float w[kCols];
-      tc::ld<kCols>(lane_base + kTmO + part * kCols, w);
+#pragma unroll 1
+    for (int q = 0; q < 4; ++q) {
+      float w[32];
+      tc::ld<32>(o_cols + 32 * q, w);
       if (store) {
 #pragma unroll
-        for (int q = 0; q < kCols / 8; ++q) {
+        for (int u = 0; u < 4; ++u) {
           float x[8];
 #pragma unroll
-          for (int e = 0; e < 8; ++e) x[e] = w[8 * q + e] * inv;
+          for (int e = 0; e < 8; ++e) x[e] = w[8 * u + e] * inv;
+          char *dst = orow + q * 64 + u * 16;
           if (p.mix_alpha) {
-            const uint4 old = *reinterpret_cast<const uint4 *>(orow + q * 16);
+            const uint4 old = *reinterpret_cast<const uint4 *>(dst);
             float f[8];
             Elem<__nv_bfloat16>::unpack(old, f);
 #pragma unroll
@@ -507,11 +552,11 @@ __global__ void __launch_bounds__(kTcThreads, 1) prefill_tc_kernel(const __grid_
             const __nv_bfloat162 pb = __floats2bfloat162_rn(x[2 * e], x[2 * e + 1]);
             wd[e] = *reinterpret_cast<const uint32_t *>(&pb);
           }
-          *reinterpret_cast<uint4 *>(orow + q * 16) = make_uint4(wd[0], wd[1], wd[2], wd[3]);
+          *reinterpret_cast<uint4 *>(dst) = make_uint4(wd[0], wd[1], wd[2], wd[3]);
         }
       }
     }
-    if (store && part == 0 && p.lse) p.lse[(static_cast<int64_t>(b) * p.n + r0 + rpos) * p.Hq + h] = (m + lg2(lrow)) * kLn2;
+    if (store && p.lse) p.lse[(static_cast<int64_t>(b) * p.n + r0 + rpos) * p.Hq + h] = (m + lg2(l)) * kLn2;
   }
 
   tc::fence_before();
@@ -528,7 +573,7 @@ bool prefill_tc_supported(const PrefillParams &p, duo_dtype dt) {
   if (tc::encode_fn() == nullptr) return false;
   // streaming tile list must fit: history tiles + window tiles + a sink tile
   const int hist_tiles = (p.hs + p.hw + kBN - 1) / kBN;
-  const int win_tiles = (p.W + 2 * kBN - 2) / kBN + 1;
+  const int win_tiles = (p.W + 3 * kBN - 2) / kBN + 1;  // window of two query tiles
   const int sink_tiles = (p.S + kBN - 1) / kBN;
   return hist_tiles + win_tiles + sink_tiles <= kMaxStrmTiles;
 }
@@ -580,7 +625,7 @@ cudaError_t launch_prefill_tc(const PrefillTcLaunch &l, cudaStream_t st) {
   const PrefillParams &p = l.p;
   const int npos = kBM / p.G;
   const int ntq = (p.n + npos - 1) / npos;
-  const int grid = ntq * p.B * p.Hkv;
+  const int grid = (ntq + kQT - 1) / kQT * p.B * p.Hkv;
   prefill_tc_kernel<<<grid, kTcThreads, kSmemAlloc, st>>>(l);
   return cudaGetLastError();
 }
