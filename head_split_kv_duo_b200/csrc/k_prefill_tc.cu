@@ -48,7 +48,7 @@ constexpr int kD = 128;
 constexpr int kKStages = 2;  // K ring: a stage is free once S_1(j) is computed
 constexpr int kVStages = 2;  // V ring: a stage is free once P_1(j) V_j is computed
 constexpr int kMaxStrmTiles = 48;
-constexpr int kPolyExp = 12;  // exponentials of every 32 (interior tiles) on the FMA pipe
+constexpr int kPolyExp = 0;   // exponentials of every 32 (interior tiles) on the FMA pipe
 
 // shared memory map (bytes from the 1 KiB-aligned base); every tile is two 128B-swizzled
 // [128][64] bf16 halves of 16 KiB
@@ -360,24 +360,32 @@ __global__ void __launch_bounds__(kTcThreads, 1) prefill_tc_kernel(const __grid_
     if (lane == 0) {
       constexpr uint32_t kIdS = tc::idesc_bf16(kBM, kBN, false, false);
       constexpr uint32_t kIdPV = tc::idesc_bf16(kBM, kD, false, true);
-      // S_t(j) = Q_t K_j^T : K = d 128 in 8 steps of 16; Q and K are K-major
+      // Shared-memory descriptors are built once: the start address sits in the low 14
+      // bits as addr >> 4 and every operand lies below 256 KiB, so an operand at byte
+      // offset o from a base is the base's descriptor + (o >> 4).  A single thread issues
+      // every MMA; keeping its per-MMA work to an add keeps the tensor pipe fed.
+      const uint64_t qd0 = tc::sdesc(sbase + kSmQ, 16, 1024), kd0 = tc::sdesc(sbase + kSmK, 16, 1024);
+      const uint64_t vd0 = tc::sdesc(sbase + kSmV, 16384, 1024);
+      // S_t(j) = Q_t K_j^T : K = d 128 in 8 steps of 16 (16 dims = 32 bytes within a
+      // 128-byte swizzled row, the second 64 dims in the other half); Q and K K-major
       auto issue_s = [&](int t, int j) {
-        const uint32_t kbase = sbase + kSmK + (j % kKStages) * 32768, qbase = sbase + kSmQ + t * 32768;
+        const uint64_t qd = qd0 + t * (32768 >> 4), kd = kd0 + (j % kKStages) * (32768 >> 4);
+        const uint32_t d = tmem + kTmS + t * 128;
+#pragma unroll
         for (int kk = 0; kk < 8; ++kk) {
-          const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
-          tc::mma_ss(tmem + kTmS + t * 128, tc::sdesc(qbase + off, 16, 1024), tc::sdesc(kbase + off, 16, 1024), kIdS,
-                     kk > 0 ? 1u : 0u);
+          const uint32_t o = ((kk >> 2) * 16384 + (kk & 3) * 32) >> 4;
+          tc::mma_ss(d, qd + o, kd + o, kIdS, kk > 0 ? 1u : 0u);
         }
         tc::commit(bar(kBarSFull + t));
       };
-      // O_t += P_t(j) V_j : K = 128 keys in 8 steps of 16; P from TMEM (bf16 pairs,
-      // K-major), V from shared memory (d contiguous, MN-major)
+      // O_t += P_t(j) V_j : K = 128 keys in 8 steps of 16 (16 keys = 2 KiB of V); P from
+      // TMEM (bf16 pairs, K-major), V from shared memory (d contiguous, MN-major)
       auto issue_pv = [&](int t, int j) {
-        const uint32_t vbase = sbase + kSmV + (j % kVStages) * 32768;
-        for (int kk = 0; kk < 8; ++kk) {
-          const uint64_t bd = tc::sdesc(vbase + kk * 2048, 16384, 1024);
-          tc::mma_ts(tmem + kTmO + t * 128, tmem + kTmS + t * 128 + kk * 8, bd, kIdPV, (j > 0 || kk > 0) ? 1u : 0u);
-        }
+        const uint64_t vd = vd0 + (j % kVStages) * (32768 >> 4);
+        const uint32_t d = tmem + kTmO + t * 128, pa = tmem + kTmS + t * 128;
+        const uint32_t acc0 = j > 0 ? 1u : 0u;
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) tc::mma_ts(d, pa + kk * 8, vd + kk * (2048 >> 4), kIdPV, kk > 0 ? 1u : acc0);
       };
       bool ok = nt > 0 && tc::wait_bar(bar(kBarQ), 0, p.status, abort_flag) &&
                 tc::wait_bar(bar(kBarKFull), 0, p.status, abort_flag);
@@ -491,13 +499,15 @@ __global__ void __launch_bounds__(kTcThreads, 1) prefill_tc_kernel(const __grid_
       if (j >= 1 && __any_sync(0xffffffffu, need)) {
         // rescale this row of O_t: S_t(j) has landed, so P_t(j-1) V_{j-1} has too
 #pragma unroll 1
-        for (int q = 0; q < 4; ++q) {
-          float w[32];
-          tc::ld<32>(o_cols + 32 * q, w);
+        for (int q = 0; q < 8; ++q) {  // 16 columns at a time: the logits stay in registers
+          float w[16];
+          tc::ld<16>(o_cols + 16 * q, w);
+          uint32_t u[16];
 #pragma unroll
-          for (int e = 0; e < 32; ++e) w[e] *= alpha;
-          tc::st32(o_cols + 32 * q, w);
+          for (int e = 0; e < 16; ++e) u[e] = __float_as_uint(w[e] * alpha);
+          tc::st16(o_cols + 16 * q, u);
         }
+        tc::st_wait();
       }
       // probabilities (masked logits are -inf and give 0), row sum, bf16 pairs of P_t(j)
       // over the first 64 columns of S_t
