@@ -98,6 +98,15 @@ __device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes) {
 __device__ __forceinline__ void mbar_arrive(uint32_t bar) {
   asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
 }
+// One arrival per warp, for a barrier initialised with a count of warps: the warp's
+// lanes synchronise first (which orders each lane's earlier stores and fences before the
+// elected lane's arrive), then lane 0 arrives.  Every lane of the warp must call it.
+// A role of 128 threads arriving one by one would make 128 atomic updates of one
+// shared-memory word per phase, which the thread polling that barrier queues behind.
+__device__ __forceinline__ void mbar_arrive_warp(uint32_t bar) {
+  __syncwarp();
+  if ((threadIdx.x & 31) == 0) mbar_arrive(bar);
+}
 // non-blocking: has the phase of `bar` with this parity completed?
 __device__ __forceinline__ bool mbar_test_wait(uint32_t bar, uint32_t parity) {
   uint32_t done;

@@ -73,8 +73,8 @@ static_assert(kSmemAlloc <= 232448, "shared memory");
 // publishes P'(j + 2) before the issuer need have taken P'(j), so a barrier per
 // buffer pair would complete a second phase ahead of its waiter
 constexpr int kBarFull = 0, kBarEmpty = kStages, kBarCvt = 2 * kStages, kBarSFull = 3 * kStages,
-              kBarSFree = kBarSFull + 2, kBarPFull = kBarSFull + 4, kBarOFull = kBarSFull + 8,
-              kBarQFree = kBarSFull + 12, kBarDrain = kBarSFull + 14, kNumBars = kBarSFull + 15;
+              kBarPFull = kBarSFull + 2, kBarOFull = kBarSFull + 6, kBarQFree = kBarSFull + 10,
+              kBarDrain = kBarSFull + 12, kNumBars = kBarSFull + 13;
 static_assert(kNumBars * 8 <= 512, "barrier area");
 
 // tensor memory columns: S^T (three limbs per query head) x 2, O^T (two limbs) x 4, and
@@ -238,15 +238,14 @@ __global__ void __launch_bounds__(kThreads, 1) decode_int4_kernel(const __grid_c
     for (int i = 0; i < kStages; ++i) {
       mbar_init(bar(kBarFull + i), 1);
       mbar_init(bar(kBarEmpty + i), 1);
-      mbar_init(bar(kBarCvt + i), 128);
+      mbar_init(bar(kBarCvt + i), 4);   // one arrival per prep warp
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(bar(kBarSFull + i), 1);
-      mbar_init(bar(kBarSFree + i), 128);
       mbar_init(bar(kBarQFree + i), 3);  // the item's last S^T product (commit) + each softmax group
     }
     for (int i = 0; i < 4; ++i) {
-      mbar_init(bar(kBarPFull + i), 128);
+      mbar_init(bar(kBarPFull + i), 4);  // one arrival per warp of a softmax group
       mbar_init(bar(kBarOFull + i), 1);
     }
     mbar_init(bar(kBarDrain), 1);
@@ -311,75 +310,65 @@ __global__ void __launch_bounds__(kThreads, 1) decode_int4_kernel(const __grid_c
     }
   } else if (warp == 1) {
     // ================= MMA issuer =================
-    // Event-driven: S^T(js) as soon as its prep is done and its S buffer is free, O^T(jo)
-    // as soon as the softmax has written P'(jo), whichever comes first.
+    // One bounded wait per tile: P'(j) written (which also means S^T(j) has been read and
+    // the prep of tile j + 2 is done), then S^T(j + 2) and O^T(j).  Waiting costs this
+    // thread a shared-memory round trip, and a single thread issuing dependent
+    // instructions sets the pace of the pipeline, so its per-tile work is kept small:
+    // one wait, descriptors as a base plus a constant, stage and phase as counters.
     if (lane == 0) {
       constexpr uint32_t kIdS = idesc_i8(128, C::kS, true, false);   // [U | L] . Qx^T
       constexpr uint32_t kIdO = idesc_i8(128, C::kO, true, true);    // [U_V | L_V]^T . P'^T
-      int js = 0, jo = 0, nitem = -1, prev_item = -1;
+      constexpr uint32_t kStDesc = kStage >> 4;                       // one stage in descriptor units
+      const uint64_t ak0 = sdesc_l(sbase + kStKc, 16, 512, 4);
+      const uint64_t av0 = sdesc_l(sbase + kStVc, kStLv - kStVc, 512, 4);  // MN-major, 2 chunks
+      const uint64_t bq0 = sdesc_l(sbase + kSmQl, 16, 1024, 2);
+      const uint64_t bp0 = sdesc_l(sbase + kSmP, 16, 1024, 2);
+      int nitem = -1, prev_item = -1;
       UnitIter its(a, u0);
-      uint32_t idle = 0;
-      unsigned long long t_idle = 0;
-      while (jo < nu) {
-        bool did = false;
-        if (js < nu) {
-          const int s = js % kStages;
-          if (mbar_test_wait(bar(kBarCvt + s), (js / kStages) & 1) &&
-              (js < 2 || mbar_test_wait(bar(kBarSFree + (js & 1)), ((js - 2) >> 1) & 1))) {
-            const int item = its.un.item;
-            its.next();
-            if (item != prev_item) {
-              prev_item = item;
-              ++nitem;
-            }
-            tc::fence_after();
-            const uint64_t ak = sdesc_l(sbase + s * kStage + kStKc, 16, 512, 4);
-            const uint32_t al = tmem + C::kLk + s * 16;
-            const uint64_t bq = sdesc_l(sbase + kSmQl + (nitem & 1) * kQlBytes, 16, 1024, 2);
-            const uint32_t d = tmem + (js & 1) * C::kS;
-            mma_i8(d, ak, bq, kIdS, 0u);             // bytes 0..31 of the code rows
-            mma_i8(d, ak + 2, bq + 2, kIdS, 1u);     // bytes 32..63
-            mma_i8_ts(d, al, bq + 4, kIdS, 1u);      // low nibbles 0..31 (TMEM)
-            mma_i8_ts(d, al + 8, bq + 6, kIdS, 1u);  // low nibbles 32..63
-            tc::commit(bar(kBarSFull + (js & 1)));
-            ++js;
-            // the item's query limbs are free once its last S^T product has run
-            if (js == nu || its.un.item != item) tc::commit(bar(kBarQFree + (nitem & 1)));
-            did = true;
-          }
+      int ss = 0, sph = 0;  // stage of S^T(js) and the phase of its prep barrier
+      int os = 0;           // stage of O^T(jo)
+      bool ok = true;
+      auto issue_s = [&](int js) {  // S^T(js), its prep and S buffer ready
+        const int item = its.un.item;
+        its.next();
+        if (item != prev_item) {
+          prev_item = item;
+          ++nitem;
         }
-        if (jo < js && mbar_test_wait(bar(kBarPFull + (jo & 3)), (jo >> 2) & 1)) {
-          tc::fence_after();
-          const int s = jo % kStages;
-          const uint64_t av = sdesc_l(sbase + s * kStage + kStVc, kStLv - kStVc, 512, 4);  // MN-major, 2 chunks
-          const uint64_t bp = sdesc_l(sbase + kSmP + (jo & 3) * 4096, 16, 1024, 2);
-          const uint32_t d = tmem + 2 * C::kS + (jo & 3) * C::kO;
+        tc::fence_after();
+        const uint64_t ak = ak0 + ss * kStDesc;
+        const uint64_t bq = bq0 + (nitem & 1) * (kQlBytes >> 4);
+        const uint32_t al = tmem + C::kLk + ss * 16;
+        const uint32_t d = tmem + (js & 1) * C::kS;
+        mma_i8(d, ak, bq, kIdS, 0u);             // bytes 0..31 of the code rows
+        mma_i8(d, ak + 2, bq + 2, kIdS, 1u);     // bytes 32..63
+        mma_i8_ts(d, al, bq + 4, kIdS, 1u);      // low nibbles 0..31 (TMEM)
+        mma_i8_ts(d, al + 8, bq + 6, kIdS, 1u);  // low nibbles 32..63
+        tc::commit(bar(kBarSFull + (js & 1)));
+        // the item's query limbs are free once its last S^T product has run
+        if (js + 1 == nu || its.un.item != item) tc::commit(bar(kBarQFree + (nitem & 1)));
+        if (++ss == kStages) {
+          ss = 0;
+          sph ^= 1;
+        }
+      };
+      for (int js = 0; js < 2 && js < nu && ok; ++js) {  // the first two after their prep
+        ok = tc::wait_bar(bar(kBarCvt + ss), sph, p.status, abort_flag);
+        if (ok) issue_s(js);
+      }
+      for (int jo = 0; jo < nu && ok; ++jo) {
+        if (!(ok = tc::wait_bar(bar(kBarPFull + (jo & 3)), (jo >> 2) & 1, p.status, abort_flag))) break;
+        if (jo + 2 < nu) issue_s(jo + 2);  // first: the softmax needs S^T(jo + 2) before O^T(jo)
+        tc::fence_after();
+        const uint64_t av = av0 + os * kStDesc;
+        const uint64_t bp = bp0 + (jo & 3) * (4096 >> 4);
+        const uint32_t d = tmem + 2 * C::kS + (jo & 3) * C::kO;
 #pragma unroll
-          for (int k = 0; k < 4; ++k)  // 32 tokens per step
-            mma_i8(d, av + k * (2048 >> 4), bp + k * 2, kIdO, k > 0 ? 1u : 0u);
-          tc::commit(bar(kBarOFull + (jo & 3)));
-          tc::commit(bar(kBarEmpty + s));  // the stage and its K low nibbles are no longer read
-          ++jo;
-          did = true;
-        }
-        if (did) {
-          idle = 0;
-        } else {
-          // sleep on the event expected next rather than spin beside the other warps
-          if (jo < js)
-            mbar_try_wait_ns(bar(kBarPFull + (jo & 3)), (jo >> 2) & 1, 100);
-          else
-            mbar_try_wait_ns(bar(kBarCvt + js % kStages), (js / kStages) & 1, 100);
-          if (++idle == 1) t_idle = globaltimer();
-        }
-        if (idle > 0 && (idle & 63) == 0) {
-          if (*abort_flag) break;
-          if (globaltimer() - t_idle > kWaitLimitNs) {
-            flag_status(p.status, kDevTimeout);
-            *abort_flag = 1;
-            break;
-          }
-        }
+        for (int k = 0; k < 4; ++k)  // 32 tokens per step
+          mma_i8(d, av + k * (2048 >> 4), bp + k * 2, kIdO, k > 0 ? 1u : 0u);
+        tc::commit(bar(kBarOFull + (jo & 3)));
+        tc::commit(bar(kBarEmpty + os));  // the stage and its K low nibbles are no longer read
+        if (++os == kStages) os = 0;
       }
       tc::commit(bar(kBarDrain));
       mbar_wait(bar(kBarDrain), 0, p.status);
@@ -568,8 +557,6 @@ __global__ void __launch_bounds__(kThreads, 1) decode_int4_kernel(const __grid_c
       tc::fence_after();
       int sr[C::kS];
       ld_i32<C::kS>(lane_base + cb * C::kS, sr);
-      tc::fence_before();
-      mbar_arrive(bar(kBarSFree + cb));  // S buffer j % 2 is free again
       // the stage's prep is complete (its S^T product has run); waiting here orders the
       // prep warps' writes before these reads
       if (ok) ok = tc::wait_bar(bar(kBarCvt + s), (j / kStages) & 1, p.status, abort_flag);
@@ -641,9 +628,13 @@ __global__ void __launch_bounds__(kThreads, 1) decode_int4_kernel(const __grid_c
           pb[sw128(2 * q + 1, t)] = static_cast<uint8_t>(b1);
         }
       }
+      // P'(j) also vouches to the MMA thread that S^T(j) has been read (its buffer takes
+      // S^T(j + 2)) and that the prep of tile j + 2 is done: one wait there per tile
+      if (j + 2 < nu && ok)
+        ok = tc::wait_bar(bar(kBarCvt + (j + 2) % kStages), ((j + 2) / kStages) & 1, p.status, abort_flag);
       tc::fence_async_smem();
       tc::fence_before();
-      mbar_arrive(bar(kBarPFull + (j & 3)));
+      mbar_arrive_warp(bar(kBarPFull + (j & 3)));
       // fold this group's previous tile of the item, bringing it to this tile's scale
       if (jp >= 0) {
         fold(jp, sigp_prev, alpha);
@@ -675,7 +666,8 @@ __global__ void __launch_bounds__(kThreads, 1) decode_int4_kernel(const __grid_c
         ++nitem;
       }
       const int s = j % kStages;
-      if (!tc::wait_bar(bar(kBarFull + s), (j / kStages) & 1, p.status, abort_flag)) break;
+      // the warp leaves together (its arrive below is warp-collective)
+      if (!__all_sync(0xffffffffu, tc::wait_bar(bar(kBarFull + s), (j / kStages) & 1, p.status, abort_flag))) break;
       tc::fence_after();  // the TMEM columns written below were last read by an MMA
       char *st = smem + s * kStage;
       uint32_t lk[16];
@@ -707,7 +699,8 @@ __global__ void __launch_bounds__(kThreads, 1) decode_int4_kernel(const __grid_c
       if (first && warp == 10) {
         // the item's query limbs replace those of the item two before, once its last
         // S^T product has run and the softmax has read its sigma and sum(q)
-        if (nitem >= 2 && !tc::wait_bar(bar(kBarQFree + (nitem & 1)), ((nitem - 2) >> 1) & 1, p.status, abort_flag))
+        if (nitem >= 2 &&
+            !__all_sync(0xffffffffu, tc::wait_bar(bar(kBarQFree + (nitem & 1)), ((nitem - 2) >> 1) & 1, p.status, abort_flag)))
           break;
         prep_queries(st + kStQ, smem + kSmQl + (nitem & 1) * kQlBytes,
                      reinterpret_cast<float *>(smem + kSmQinfo) + (nitem & 1) * 32, G, lane);
@@ -715,7 +708,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_int4_kernel(const __grid_c
       tc::st_wait();
       tc::fence_async_smem();  // the low nibbles and query limbs are MMA operands
       tc::fence_before();
-      mbar_arrive(bar(kBarCvt + s));
+      mbar_arrive_warp(bar(kBarCvt + s));
     }
   }
 

@@ -297,7 +297,8 @@ __global__ void __launch_bounds__(kTcThreads, 1) prefill_tc_kernel(const __grid_
   pl.kvrow = b * (pl.retr ? p.Hr : p.HsMax) + p.hm.kind_idx[g];
 
   if (tid == 0) {
-    for (int i = 0; i < kNumBars; ++i) mbar_init(bar(i), (i >= kBarPFull && i < kBarPFull + kQT) ? kBM : 1);
+    // P_t is published by one arrival per softmax warp
+    for (int i = 0; i < kNumBars; ++i) mbar_init(bar(i), (i >= kBarPFull && i < kBarPFull + kQT) ? kBM / 32 : 1);
     if (smem_u32(smem) & 1023u) flag_status(p.status, kDevTimeout);  // layout assumption (never expected)
     fence_mbar_init();
     *abort_flag = 0;
@@ -527,7 +528,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) prefill_tc_kernel(const __grid_
       const float rsum = (rs[0] + rs[1]) + (rs[2] + rs[3]);
       tc::st_wait();
       tc::fence_before();
-      mbar_arrive(bar(kBarPFull + qt));
+      mbar_arrive_warp(bar(kBarPFull + qt));
       l = l * alpha + rsum;
     }
     // the last product, then the epilogue: normalise and store the row (bf16) and its
