@@ -22,12 +22,12 @@
 // token the scale and zero then give
 //   q . k_t = s_t (q . c_t) + z_t sum(q),   sum_t p_t v_t = sum_t p'_t c_t + sum_t p_t z_t.
 //
-// Roles of a CTA (one per SM, 448 threads):
+// Roles of a CTA (one per SM, 480 threads):
 //   warp 0     TMA producer: per 128-token tile the K and V code rows (64 B each,
 //              64-byte swizzle) and their scale/zero rows, at an item's first tile the
 //              group's bf16 queries; a ring of kStages stages.
-//   warp 1     MMA issuer and TMEM owner (4 MMAs for S^T and 4 for O^T per tile; the
-//              K low nibbles are read from tensor memory).
+//   warp 1     TMEM owner and S^T issuer (4 MMAs per tile; the K low nibbles are read
+//              from tensor memory); warp 14 issues O^T (4 MMAs per tile).
 //   warps 2-9  softmax, two warpgroups taking alternate tiles (each with its own running
 //              max and sums, combined when an item ends), so that the dependent chain
 //              of one tile overlaps the next: thread t owns token t of S^T and row t of
@@ -46,7 +46,7 @@ namespace duo {
 
 namespace {
 
-constexpr int kThreads = 448;
+constexpr int kThreads = 480;
 constexpr int kTile = 128;
 constexpr int kD = 128;
 constexpr int kStages = 6;
@@ -74,7 +74,7 @@ static_assert(kSmemAlloc <= 232448, "shared memory");
 // buffer pair would complete a second phase ahead of its waiter
 constexpr int kBarFull = 0, kBarEmpty = kStages, kBarCvt = 2 * kStages, kBarSFull = 3 * kStages,
               kBarPFull = kBarSFull + 2, kBarOFull = kBarSFull + 6, kBarQFree = kBarSFull + 10,
-              kBarDrain = kBarSFull + 12, kNumBars = kBarSFull + 13;
+              kBarDrain = kBarSFull + 12, kNumBars = kBarSFull + 14;  // a drain barrier per issuer
 static_assert(kNumBars * 8 <= 512, "barrier area");
 
 // tensor memory columns: S^T (three limbs per query head) x 2, O^T (two limbs) x 4, and
@@ -249,6 +249,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_int4_kernel(const __grid_c
       mbar_init(bar(kBarOFull + i), 1);
     }
     mbar_init(bar(kBarDrain), 1);
+    mbar_init(bar(kBarDrain + 1), 1);
     fence_mbar_init();
     *abort_flag = 0;
   }
@@ -308,70 +309,81 @@ __global__ void __launch_bounds__(kThreads, 1) decode_int4_kernel(const __grid_c
       // after an abort, loads may still be landing: none may outlive the CTA
       tc::drain_loads(bar(kBarFull), kStages, issued, p.status);
     }
-  } else if (warp == 1) {
-    // ================= MMA issuer =================
-    // One bounded wait per tile: P'(j) written (which also means S^T(j) has been read and
-    // the prep of tile j + 2 is done), then S^T(j + 2) and O^T(j).  Waiting costs this
-    // thread a shared-memory round trip, and a single thread issuing dependent
-    // instructions sets the pace of the pipeline, so its per-tile work is kept small:
-    // one wait, descriptors as a base plus a constant, stage and phase as counters.
+  } else if (warp == 1 || warp == 14) {
+    // ================= MMA issuers: S^T on warp 1, O^T on warp 14 =================
+    // Each waits once per tile, on P'(j) (which also means S^T(j) has been read and the
+    // prep of tile j + 2 is done), then issues S^T(j + 2) (warp 1) or O^T(j) (warp 14).
+    // A barrier wait and an MMA issue each cost a thread hundreds of cycles on a loaded
+    // SM, and one thread issuing dependent instructions sets the pace of the pipeline:
+    // two issuers halve it, and their per-tile work is kept small (one wait, descriptors
+    // as a base plus a constant, stage and phase as running counters).  tcgen05.commit
+    // tracks the committing thread's own MMAs; the stage is released after O^T(j), and
+    // S^T(j) has completed by then (the softmax saw it land before writing P'(j)).
     if (lane == 0) {
       constexpr uint32_t kIdS = idesc_i8(128, C::kS, true, false);   // [U | L] . Qx^T
       constexpr uint32_t kIdO = idesc_i8(128, C::kO, true, true);    // [U_V | L_V]^T . P'^T
       constexpr uint32_t kStDesc = kStage >> 4;                       // one stage in descriptor units
-      const uint64_t ak0 = sdesc_l(sbase + kStKc, 16, 512, 4);
-      const uint64_t av0 = sdesc_l(sbase + kStVc, kStLv - kStVc, 512, 4);  // MN-major, 2 chunks
-      const uint64_t bq0 = sdesc_l(sbase + kSmQl, 16, 1024, 2);
-      const uint64_t bp0 = sdesc_l(sbase + kSmP, 16, 1024, 2);
-      int nitem = -1, prev_item = -1;
-      UnitIter its(a, u0);
-      int ss = 0, sph = 0;  // stage of S^T(js) and the phase of its prep barrier
-      int os = 0;           // stage of O^T(jo)
       bool ok = true;
-      auto issue_s = [&](int js) {  // S^T(js), its prep and S buffer ready
-        const int item = its.un.item;
-        its.next();
-        if (item != prev_item) {
-          prev_item = item;
-          ++nitem;
+      if (warp == 1) {
+        const uint64_t ak0 = sdesc_l(sbase + kStKc, 16, 512, 4);
+        const uint64_t bq0 = sdesc_l(sbase + kSmQl, 16, 1024, 2);
+        int nitem = -1, prev_item = -1;
+        UnitIter its(a, u0);
+        int ss = 0, sph = 0;  // stage of S^T(js) and the phase of its prep barrier
+        auto issue_s = [&](int js) {  // S^T(js), its prep and S buffer ready
+          const int item = its.un.item;
+          its.next();
+          if (item != prev_item) {
+            prev_item = item;
+            ++nitem;
+          }
+          tc::fence_after();
+          const uint64_t ak = ak0 + ss * kStDesc;
+          const uint64_t bq = bq0 + (nitem & 1) * (kQlBytes >> 4);
+          const uint32_t al = tmem + C::kLk + ss * 16;
+          const uint32_t d = tmem + (js & 1) * C::kS;
+          mma_i8(d, ak, bq, kIdS, 0u);             // bytes 0..31 of the code rows
+          mma_i8(d, ak + 2, bq + 2, kIdS, 1u);     // bytes 32..63
+          mma_i8_ts(d, al, bq + 4, kIdS, 1u);      // low nibbles 0..31 (TMEM)
+          mma_i8_ts(d, al + 8, bq + 6, kIdS, 1u);  // low nibbles 32..63
+          tc::commit(bar(kBarSFull + (js & 1)));
+          // the item's query limbs are free once its last S^T product has run
+          if (js + 1 == nu || its.un.item != item) tc::commit(bar(kBarQFree + (nitem & 1)));
+          if (++ss == kStages) {
+            ss = 0;
+            sph ^= 1;
+          }
+        };
+        for (int js = 0; js < 2 && js < nu && ok; ++js) {  // the first two after their prep
+          ok = tc::wait_bar(bar(kBarCvt + ss), sph, p.status, abort_flag);
+          if (ok) issue_s(js);
         }
-        tc::fence_after();
-        const uint64_t ak = ak0 + ss * kStDesc;
-        const uint64_t bq = bq0 + (nitem & 1) * (kQlBytes >> 4);
-        const uint32_t al = tmem + C::kLk + ss * 16;
-        const uint32_t d = tmem + (js & 1) * C::kS;
-        mma_i8(d, ak, bq, kIdS, 0u);             // bytes 0..31 of the code rows
-        mma_i8(d, ak + 2, bq + 2, kIdS, 1u);     // bytes 32..63
-        mma_i8_ts(d, al, bq + 4, kIdS, 1u);      // low nibbles 0..31 (TMEM)
-        mma_i8_ts(d, al + 8, bq + 6, kIdS, 1u);  // low nibbles 32..63
-        tc::commit(bar(kBarSFull + (js & 1)));
-        // the item's query limbs are free once its last S^T product has run
-        if (js + 1 == nu || its.un.item != item) tc::commit(bar(kBarQFree + (nitem & 1)));
-        if (++ss == kStages) {
-          ss = 0;
-          sph ^= 1;
+        for (int jo = 0; jo + 2 < nu && ok; ++jo) {
+          if (!(ok = tc::wait_bar(bar(kBarPFull + (jo & 3)), (jo >> 2) & 1, p.status, abort_flag))) break;
+          issue_s(jo + 2);
         }
-      };
-      for (int js = 0; js < 2 && js < nu && ok; ++js) {  // the first two after their prep
-        ok = tc::wait_bar(bar(kBarCvt + ss), sph, p.status, abort_flag);
-        if (ok) issue_s(js);
-      }
-      for (int jo = 0; jo < nu && ok; ++jo) {
-        if (!(ok = tc::wait_bar(bar(kBarPFull + (jo & 3)), (jo >> 2) & 1, p.status, abort_flag))) break;
-        if (jo + 2 < nu) issue_s(jo + 2);  // first: the softmax needs S^T(jo + 2) before O^T(jo)
-        tc::fence_after();
-        const uint64_t av = av0 + os * kStDesc;
-        const uint64_t bp = bp0 + (jo & 3) * (4096 >> 4);
-        const uint32_t d = tmem + 2 * C::kS + (jo & 3) * C::kO;
+      } else {
+        const uint64_t av0 = sdesc_l(sbase + kStVc, kStLv - kStVc, 512, 4);  // MN-major, 2 chunks
+        const uint64_t bp0 = sdesc_l(sbase + kSmP, 16, 1024, 2);
+        int os = 0;  // stage of O^T(jo)
+        for (int jo = 0; jo < nu && ok; ++jo) {
+          if (!(ok = tc::wait_bar(bar(kBarPFull + (jo & 3)), (jo >> 2) & 1, p.status, abort_flag))) break;
+          tc::fence_after();
+          const uint64_t av = av0 + os * kStDesc;
+          const uint64_t bp = bp0 + (jo & 3) * (4096 >> 4);
+          const uint32_t d = tmem + 2 * C::kS + (jo & 3) * C::kO;
 #pragma unroll
-        for (int k = 0; k < 4; ++k)  // 32 tokens per step
-          mma_i8(d, av + k * (2048 >> 4), bp + k * 2, kIdO, k > 0 ? 1u : 0u);
-        tc::commit(bar(kBarOFull + (jo & 3)));
-        tc::commit(bar(kBarEmpty + os));  // the stage and its K low nibbles are no longer read
-        if (++os == kStages) os = 0;
+          for (int k = 0; k < 4; ++k)  // 32 tokens per step
+            mma_i8(d, av + k * (2048 >> 4), bp + k * 2, kIdO, k > 0 ? 1u : 0u);
+          tc::commit(bar(kBarOFull + (jo & 3)));
+          tc::commit(bar(kBarEmpty + os));  // the stage and its K low nibbles are no longer read
+          if (++os == kStages) os = 0;
+        }
       }
-      tc::commit(bar(kBarDrain));
-      mbar_wait(bar(kBarDrain), 0, p.status);
+      // drain: every MMA this thread issued has completed before TMEM is freed
+      const uint32_t drain = bar(kBarDrain + (warp == 1 ? 0 : 1));
+      tc::commit(drain);
+      mbar_wait(drain, 0, p.status);
     }
   } else if (warp < 10) {
     // ================= softmax warpgroups =================
