@@ -73,8 +73,9 @@ static_assert(kSmemAlloc <= 232448, "shared memory");
 // publishes P'(j + 2) before the issuer need have taken P'(j), so a barrier per
 // buffer pair would complete a second phase ahead of its waiter
 constexpr int kBarFull = 0, kBarEmpty = kStages, kBarCvt = 2 * kStages, kBarSFull = 3 * kStages,
-              kBarPFull = kBarSFull + 2, kBarOFull = kBarSFull + 6, kBarQFree = kBarSFull + 10,
-              kBarDrain = kBarSFull + 12, kNumBars = kBarSFull + 14;  // a drain barrier per issuer
+              kBarSFree = kBarSFull + 2, kBarPFull = kBarSFull + 4, kBarOFull = kBarSFull + 8,
+              kBarQFree = kBarSFull + 12, kBarDrain = kBarSFull + 14,
+              kNumBars = kBarSFull + 16;  // a drain barrier per issuer
 static_assert(kNumBars * 8 <= 512, "barrier area");
 
 // tensor memory columns: S^T (three limbs per query head) x 2, O^T (two limbs) x 4, and
@@ -242,6 +243,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_int4_kernel(const __grid_c
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(bar(kBarSFull + i), 1);
+      mbar_init(bar(kBarSFree + i), 4);  // one arrival per warp of a softmax group
       mbar_init(bar(kBarQFree + i), 3);  // the item's last S^T product (commit) + each softmax group
     }
     for (int i = 0; i < 4; ++i) {
@@ -311,14 +313,14 @@ __global__ void __launch_bounds__(kThreads, 1) decode_int4_kernel(const __grid_c
     }
   } else if (warp == 1 || warp == 14) {
     // ================= MMA issuers: S^T on warp 1, O^T on warp 14 =================
-    // Each waits once per tile, on P'(j) (which also means S^T(j) has been read and the
-    // prep of tile j + 2 is done), then issues S^T(j + 2) (warp 1) or O^T(j) (warp 14).
-    // A barrier wait and an MMA issue each cost a thread hundreds of cycles on a loaded
-    // SM, and one thread issuing dependent instructions sets the pace of the pipeline:
-    // two issuers halve it, and their per-tile work is kept small (one wait, descriptors
-    // as a base plus a constant, stage and phase as running counters).  tcgen05.commit
-    // tracks the committing thread's own MMAs; the stage is released after O^T(j), and
-    // S^T(j) has completed by then (the softmax saw it land before writing P'(j)).
+    // Warp 1 issues S^T(j) once the prep of tile j is done and the softmax has read
+    // S^T(j - 2) (its buffer); warp 14 issues O^T(j) once P'(j) is written.  A barrier
+    // wait and an MMA issue each cost a thread hundreds of cycles on a loaded SM, and a
+    // thread issuing dependent instructions sets the pace of the pipeline: two issuers,
+    // each with little per-tile work (descriptors as a base plus a constant, stage and
+    // phase as running counters), keep S^T ahead of the softmax.  tcgen05.commit tracks
+    // the committing thread's own MMAs; the stage is released after O^T(j), and S^T(j)
+    // has completed by then (the softmax saw it land before writing P'(j)).
     if (lane == 0) {
       constexpr uint32_t kIdS = idesc_i8(128, C::kS, true, false);   // [U | L] . Qx^T
       constexpr uint32_t kIdO = idesc_i8(128, C::kO, true, true);    // [U_V | L_V]^T . P'^T
@@ -330,7 +332,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_int4_kernel(const __grid_c
         int nitem = -1, prev_item = -1;
         UnitIter its(a, u0);
         int ss = 0, sph = 0;  // stage of S^T(js) and the phase of its prep barrier
-        auto issue_s = [&](int js) {  // S^T(js), its prep and S buffer ready
+        auto issue_s = [&](int js) {  // S^T(js), its prep done and its S buffer read
           const int item = its.un.item;
           its.next();
           if (item != prev_item) {
@@ -354,13 +356,10 @@ __global__ void __launch_bounds__(kThreads, 1) decode_int4_kernel(const __grid_c
             sph ^= 1;
           }
         };
-        for (int js = 0; js < 2 && js < nu && ok; ++js) {  // the first two after their prep
-          ok = tc::wait_bar(bar(kBarCvt + ss), sph, p.status, abort_flag);
+        for (int js = 0; js < nu && ok; ++js) {
+          ok = tc::wait_bar(bar(kBarCvt + ss), sph, p.status, abort_flag) &&
+               (js < 2 || tc::wait_bar(bar(kBarSFree + (js & 1)), ((js - 2) >> 1) & 1, p.status, abort_flag));
           if (ok) issue_s(js);
-        }
-        for (int jo = 0; jo + 2 < nu && ok; ++jo) {
-          if (!(ok = tc::wait_bar(bar(kBarPFull + (jo & 3)), (jo >> 2) & 1, p.status, abort_flag))) break;
-          issue_s(jo + 2);
         }
       } else {
         const uint64_t av0 = sdesc_l(sbase + kStVc, kStLv - kStVc, 512, 4);  // MN-major, 2 chunks
@@ -569,6 +568,8 @@ __global__ void __launch_bounds__(kThreads, 1) decode_int4_kernel(const __grid_c
       tc::fence_after();
       int sr[C::kS];
       ld_i32<C::kS>(lane_base + cb * C::kS, sr);
+      tc::fence_before();
+      mbar_arrive_warp(bar(kBarSFree + cb));  // S buffer j % 2 is free again
       // the stage's prep is complete (its S^T product has run); waiting here orders the
       // prep warps' writes before these reads
       if (ok) ok = tc::wait_bar(bar(kBarCvt + s), (j / kStages) & 1, p.status, abort_flag);
@@ -640,10 +641,6 @@ __global__ void __launch_bounds__(kThreads, 1) decode_int4_kernel(const __grid_c
           pb[sw128(2 * q + 1, t)] = static_cast<uint8_t>(b1);
         }
       }
-      // P'(j) also vouches to the MMA thread that S^T(j) has been read (its buffer takes
-      // S^T(j + 2)) and that the prep of tile j + 2 is done: one wait there per tile
-      if (j + 2 < nu && ok)
-        ok = tc::wait_bar(bar(kBarCvt + (j + 2) % kStages), ((j + 2) / kStages) & 1, p.status, abort_flag);
       tc::fence_async_smem();
       tc::fence_before();
       mbar_arrive_warp(bar(kBarPFull + (j & 3)));
