@@ -15,10 +15,10 @@
 // 2^14, so no query overflows or loses bits in fp16), and smax is the tile's largest
 // V scale (P' stays in [0, 2^8] whatever the scales); both factors are undone in fp32.
 //
-// Roles of a CTA (one per SM, 320 threads):
+// Roles of a CTA (one per SM, 352 threads):
 //   warp 0     TMA producer: per 128-token tile the K and V code rows (128 B each,
 //              128-byte swizzle), their scale rows, the group's bf16 queries.
-//   warp 1     MMA issuer and TMEM owner.
+//   warp 1     TMEM owner and S^T issuer; warp 10 issues O^T.
 //   warps 2-5  softmax: thread t owns token t of S^T and dimension t of O^T.
 //   warps 6-9  convert: thread t widens token t's K row into TMEM lane t (the A
 //              operand of S^T) and its V row into the swizzled shared-memory V tile,
@@ -38,7 +38,7 @@ namespace duo {
 
 namespace {
 
-constexpr int kThreads = 320;
+constexpr int kThreads = 352;
 constexpr int kTile = 128;
 constexpr int kD = 128;
 constexpr int kN = 16;  // padded query heads per item
@@ -79,7 +79,7 @@ static_assert(kTmK + kBufs * 64 <= kTmemCols, "tensor memory");
 constexpr int kBarFull = 0, kBarEmpty = kStages, kBarCvtK = 2 * kStages, kBarCvtV = kBarCvtK + kBufs,
               kBarKFree = kBarCvtV + kBufs, kBarVFree = kBarKFree + kBufs, kBarSclFree = kBarVFree + kBufs,
               kBarSFull = kBarSclFree + kBufs, kBarSFree = kBarSFull + 2, kBarPFull = kBarSFree + 2,
-              kBarOFull = kBarPFull + 2, kBarDrain = kBarOFull + 2, kBarMerge = kBarDrain + 1,
+              kBarOFull = kBarPFull + 2, kBarDrain = kBarOFull + 2, kBarMerge = kBarDrain + 2,  // a drain per issuer
               kNumBars = kBarMerge + 1;
 static_assert(kNumBars * 8 <= 256, "barrier area");
 
@@ -154,7 +154,9 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fp8_kernel(const __grid_co
       const bool many = (i >= kBarCvtK && i < kBarKFree) || (i >= kBarSclFree && i < kBarSclFree + kBufs) ||
                         i == kBarSFree || i == kBarSFree + 1 || i == kBarPFull || i == kBarPFull + 1;
       const bool empty = i >= kBarEmpty && i < kBarEmpty + kStages;
-      mbar_init(bar(i), empty ? 129 : (many ? 128 : 1));
+      // the convert and softmax warps arrive once per warp; a code stage is also released
+      // by the S^T issuer's commit
+      mbar_init(bar(i), empty ? 5 : (many ? 4 : 1));
     }
     fence_mbar_init();
     *abort_flag = 0;
@@ -209,60 +211,67 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fp8_kernel(const __grid_co
       }
       tc::drain_loads(bar(kBarFull), kStages, issued, p.status);
     }
-  } else if (warp == 1) {
-    // ================= MMA issuer =================
+  } else if (warp == 1 || warp == 10) {
+    // ================= MMA issuers: S^T on warp 1, O^T on warp 10 =================
+    // A barrier wait and an MMA issue each cost a thread hundreds of cycles on a loaded
+    // SM, and a thread issuing dependent instructions sets the pace of the pipeline, so
+    // the two products have an issuer each.  tcgen05.commit tracks the committing
+    // thread's own MMAs.
     if (lane == 0) {
       constexpr uint32_t kIdS = tc::idesc_f16(128, kN, false, false, false);  // fp16, A from TMEM
       constexpr uint32_t kIdO = tc::idesc_f16(128, kN, true, false, false);   // V16^T MN-major
       bool ok = true;
-      const uint64_t dq0 = tc::sdesc(sbase + kStQ, 16, 1024);    // Q16, K-major
-      const uint64_t dv0 = tc::sdesc(sbase + kSmV, 16384, 1024);  // V16^T, MN-major
-      const uint64_t dp0 = tc::sdesc(sbase + kSmP, 16, 1024);    // P'^T, K-major
-      auto issue_o = [&](int jj) {
-        const int pb = jj & 1, vb = jj % kBufs;
-        const uint64_t dv = dv0 + vb * (32768 >> 4);
-        const uint64_t dp = dp0 + pb * (4096 >> 4);
-        const uint32_t d = tmem + kTmO + pb * kAcc * 16;
+      if (warp == 1) {
+        // S^T(j) once K16(j) is widened and the softmax has read S^T(j - 2) (its buffer)
+        const uint64_t dq0 = tc::sdesc(sbase + kStQ, 16, 1024);  // Q16, K-major
+        for (int j = 0; j < nu && ok; ++j) {
+          const int s = j % kStages, pb = j & 1, kb = j % kBufs;
+          if (!tc::wait_bar(bar(kBarCvtK + kb), (j / kBufs) & 1, p.status, abort_flag)) { ok = false; break; }
+          if (j >= 2 && !tc::wait_bar(bar(kBarSFree + pb), ((j - 2) >> 1) & 1, p.status, abort_flag)) { ok = false; break; }
+          tc::fence_after();
+          const uint64_t dq = dq0 + s * (kStage >> 4);
+          const uint32_t d = tmem + kTmS + pb * kAcc * 16;
+          const uint32_t ka = tmem + kTmK + kb * 64;
 #pragma unroll
-        for (int i = 0; i < 8; ++i) {  // K = 128 tokens in steps of 16
-          const int kk = (i % kAcc) * (8 / kAcc) + i / kAcc;
-          tc::mma_ss(d + (i % kAcc) * 16, dv + kk * 128, dp + (kk >> 2) * 128 + (kk & 3) * 2, kIdO, i >= kAcc ? 1u : 0u);
+          for (int i = 0; i < 8; ++i) {  // K = d 128 in steps of 16 (8 TMEM columns each)
+            const int kk = (i % kAcc) * (8 / kAcc) + i / kAcc;
+            tc::mma_ts(d + (i % kAcc) * 16, ka + kk * 8, dq + (kk >> 2) * 128 + (kk & 3) * 2, kIdS, i >= kAcc ? 1u : 0u);
+          }
+          tc::commit(bar(kBarSFull + pb));
+          tc::commit(bar(kBarKFree + kb));  // K16 of this buffer is free again
+          tc::commit(bar(kBarEmpty + s));   // the stage's queries are read (its codes: the convert warps)
         }
-        tc::commit(bar(kBarOFull + pb));
-        tc::commit(bar(kBarVFree + vb));  // V16 of this buffer is free again
-      };
-      // O^T(jj) once the softmax has written P'(jj) and V16(jj) is widened
-      auto try_o = [&](int jj) {
-        if (!tc::wait_bar(bar(kBarPFull + (jj & 1)), (jj >> 1) & 1, p.status, abort_flag)) return false;
-        if (!tc::wait_bar(bar(kBarCvtV + jj % kBufs), (jj / kBufs) & 1, p.status, abort_flag)) return false;
-        tc::fence_after();
-        issue_o(jj);
-        return true;
-      };
-      for (int j = 0; j < nu && ok; ++j) {
-        const int s = j % kStages, pb = j & 1, kb = j % kBufs;
-        if (!tc::wait_bar(bar(kBarCvtK + kb), (j / kBufs) & 1, p.status, abort_flag)) { ok = false; break; }
-        if (j >= 2 && !tc::wait_bar(bar(kBarSFree + pb), ((j - 2) >> 1) & 1, p.status, abort_flag)) { ok = false; break; }
-        tc::fence_after();
-        const uint64_t dq = dq0 + s * (kStage >> 4);
-        const uint32_t d = tmem + kTmS + pb * kAcc * 16;
-        const uint32_t ka = tmem + kTmK + kb * 64;
+      } else {
+        // O^T(j) once the softmax has written P'(j) and V16(j) is widened
+        const uint64_t dv0 = tc::sdesc(sbase + kSmV, 16384, 1024);  // V16^T, MN-major
+        const uint64_t dp0 = tc::sdesc(sbase + kSmP, 16, 1024);    // P'^T, K-major
+        for (int j = 0; j < nu && ok; ++j) {
+          const int pb = j & 1, vb = j % kBufs;
+          if (!tc::wait_bar(bar(kBarPFull + pb), (j >> 1) & 1, p.status, abort_flag) ||
+              !tc::wait_bar(bar(kBarCvtV + vb), (j / kBufs) & 1, p.status, abort_flag)) {
+            ok = false;
+            break;
+          }
+          tc::fence_after();
+          const uint64_t dv = dv0 + vb * (32768 >> 4);
+          const uint64_t dp = dp0 + pb * (4096 >> 4);
+          const uint32_t d = tmem + kTmO + pb * kAcc * 16;
 #pragma unroll
-        for (int i = 0; i < 8; ++i) {  // K = d 128 in steps of 16 (8 TMEM columns each)
-          const int kk = (i % kAcc) * (8 / kAcc) + i / kAcc;
-          tc::mma_ts(d + (i % kAcc) * 16, ka + kk * 8, dq + (kk >> 2) * 128 + (kk & 3) * 2, kIdS, i >= kAcc ? 1u : 0u);
+          for (int i = 0; i < 8; ++i) {  // K = 128 tokens in steps of 16
+            const int kk = (i % kAcc) * (8 / kAcc) + i / kAcc;
+            tc::mma_ss(d + (i % kAcc) * 16, dv + kk * 128, dp + (kk >> 2) * 128 + (kk & 3) * 2, kIdO, i >= kAcc ? 1u : 0u);
+          }
+          tc::commit(bar(kBarOFull + pb));
+          tc::commit(bar(kBarVFree + vb));  // V16 of this buffer is free again
         }
-        tc::commit(bar(kBarSFull + pb));
-        tc::commit(bar(kBarKFree + kb));  // K16 of this buffer is free again
-        tc::commit(bar(kBarEmpty + s));   // the stage's queries are read (its codes: the convert warps)
-        if (j >= 1 && !try_o(j - 1)) { ok = false; break; }
       }
-      if (ok && nu > 0) try_o(nu - 1);
-      tc::commit(bar(kBarDrain));
-      mbar_wait(bar(kBarDrain), 0, p.status);
+      // drain: every MMA this thread issued has completed before TMEM is freed
+      const uint32_t drain = bar(kBarDrain + (warp == 1 ? 0 : 1));
+      tc::commit(drain);
+      mbar_wait(drain, 0, p.status);
     }
   } else if (warp >= 6) {
-    // ================= convert warps =================
+    // ================= convert warps (6-9) =================
     const int wq = warp & 3;
     const int t = (wq << 5) | lane;
     const uint32_t tm_lane = tmem + (static_cast<uint32_t>(wq << 5) << 16);
@@ -353,7 +362,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fp8_kernel(const __grid_co
       tc::st_wait();
       tc::fence_async_smem();  // Q16 is read by the MMA (async proxy)
       tc::fence_before();
-      mbar_arrive(bar(kBarCvtK + b));
+      mbar_arrive_warp(bar(kBarCvtK + b));
       // V row t -> V16 [half][token t][64 dims], 128-byte swizzle (the layout a TMA of a
       // bf16 tile would write): dims 8m .. 8m+7 of a half form 16-byte chunk m
       if (ok && j >= kBufs) ok = tc::wait_bar(bar(kBarVFree + b), ph, p.status, abort_flag);
@@ -372,8 +381,8 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fp8_kernel(const __grid_co
         *reinterpret_cast<uint4 *>(rowp + (((m0 + 1) ^ rot) << 4)) = o1;
       }
       tc::fence_async_smem();  // V16 is read by the MMA (async proxy)
-      mbar_arrive(bar(kBarCvtV + b));
-      mbar_arrive(bar(kBarEmpty + s));  // this thread has read the stage's codes
+      mbar_arrive_warp(bar(kBarCvtV + b));
+      mbar_arrive_warp(bar(kBarEmpty + s));  // the warp has read the stage's codes
     }
   } else {
     // ================= softmax warpgroup (warps 2-5) =================
@@ -480,13 +489,13 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fp8_kernel(const __grid_co
       float sv[NQ];
       tc::ld_sum<NQ, kAcc>(lane_base + kTmS + b * kAcc * 16, 16, sv);
       tc::fence_before();
-      mbar_arrive(bar(kBarSFree + b));
+      mbar_arrive_warp(bar(kBarSFree + b));
       // the convert warps' factors of this tile (ordered before these reads by its barrier)
       const int kb = j % kBufs;
       if (ok) ok = tc::wait_bar(bar(kBarCvtK + kb), (j / kBufs) & 1, p.status, abort_flag);
       const float *scl = reinterpret_cast<const float *>(smem + kSmScl + kb * kSclBytes);
       const float fk = scl[t], fv = scl[128 + t], smax = scl[256];
-      mbar_arrive(bar(kBarSclFree + kb));
+      mbar_arrive_warp(bar(kBarSclFree + kb));
       const bool valid = static_cast<int64_t>(un.tile) * kTile + t < p.len;
       if (un.item != cur_item) {
         if (cur_item >= 0) {
@@ -549,7 +558,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fp8_kernel(const __grid_co
       }
       tc::fence_async_smem();
       tc::fence_before();
-      mbar_arrive(bar(kBarPFull + b));
+      mbar_arrive_warp(bar(kBarPFull + b));
       if (pending) {
         fold(j - 1, smax_prev, alpha);
       } else {
