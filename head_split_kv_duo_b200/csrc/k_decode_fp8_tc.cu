@@ -15,15 +15,15 @@
 // 2^14, so no query overflows or loses bits in fp16), and smax is the tile's largest
 // V scale (P' stays in [0, 2^8] whatever the scales); both factors are undone in fp32.
 //
-// Roles of a CTA (one per SM, 352 threads):
+// Roles of a CTA (one per SM, 480 threads):
 //   warp 0     TMA producer: per 128-token tile the K and V code rows (128 B each,
 //              128-byte swizzle), their scale rows, the group's bf16 queries.
 //   warp 1     TMEM owner and S^T issuer; warp 10 issues O^T.
 //   warps 2-5  softmax: thread t owns token t of S^T and dimension t of O^T.
-//   warps 6-9  convert: thread t widens token t's K row into TMEM lane t (the A
-//              operand of S^T) and its V row into the swizzled shared-memory V tile,
-//              converts its share of the queries in place, and writes the token's
-//              scales for the softmax.
+//   warps 6-9, 11-14  convert: thread t of either group widens half of token t's K
+//              row into TMEM lane t (the A operand of S^T) and half of its V row into
+//              the swizzled shared-memory V tile, converts its share of the queries in
+//              place, and (first group) writes the token's scales for the softmax.
 // A widened tile lives from its conversion until its O^T product, so there are three
 // widened buffers; the K half is released after S^T, the V half after O^T, and the
 // codes' stage once both are widened and S^T has read the queries.
@@ -38,11 +38,11 @@ namespace duo {
 
 namespace {
 
-constexpr int kThreads = 352;
+constexpr int kThreads = 480;
 constexpr int kTile = 128;
 constexpr int kD = 128;
 constexpr int kN = 16;  // padded query heads per item
-constexpr int kStages = 2;   // code stages (TMA ring)
+constexpr int kStages = 3;   // code stages (TMA ring): three hide the HBM latency of a tile
 constexpr int kBufs = 3;     // widened K16 / V16 / scale buffers
 constexpr int kPrefetch = 4;
 constexpr int kAcc = 4;  // independent accumulator chains per contraction
@@ -54,8 +54,8 @@ constexpr int kSmV = kStages * kStage;     // kBufs x V16 [2 halves][128 tokens]
 constexpr int kSmP = kSmV + kBufs * 32768; // 2 x P'^T [16][128] fp16 (2 atoms of 2 KiB)
 constexpr int kSmScl = kSmP + 8192;        // kBufs x {s_k' [128], s_v' [128], smax, pad}
 constexpr int kSclBytes = 2 * 128 * 4 + 64;
-constexpr int kSmCred = kSmScl + kBufs * kSclBytes;  // convert reductions: kBufs x [4 warps][2]
-constexpr int kSmRed = kSmCred + 128;      // softmax reductions [4][16] + merge exchange [128][6]
+constexpr int kSmCred = kSmScl + kBufs * kSclBytes;  // convert reductions: kBufs x [8 warps][2]
+constexpr int kSmRed = kSmCred + 256;      // softmax reductions [4][16] + merge exchange [128][6]
 constexpr int kSmBar = kSmRed + (4 * 16 + 128 * 6) * 4;
 constexpr int kSmMisc = kSmBar + 256;
 constexpr int kSmemAlloc = kSmMisc + 64 + 1024;
@@ -67,15 +67,15 @@ constexpr int kTmS = 0, kTmO = 2 * kAcc * 16, kTmK = 4 * kAcc * 16, kTmemCols = 
 static_assert(kTmK + kBufs * 64 <= kTmemCols, "tensor memory");
 
 // Per widened buffer b (tile j uses b = j % kBufs, phase j / kBufs):
-//   CvtK   K16, Q16 and the scales of the tile are written    (128 convert threads)
-//   CvtV   V16 of the tile is written                         (128 convert threads)
+//   CvtK   K16, Q16 and the scales of the tile are written    (8 convert warps)
+//   CvtV   V16 of the tile is written                         (8 convert warps)
 //   KFree  S^T of the tile has run (K16 free)                 (MMA commit)
 //   VFree  O^T of the tile has run (V16 free)                 (MMA commit)
-//   SclFree the softmax has read the tile's scales            (128 softmax threads)
+//   SclFree the softmax has read the tile's scales            (4 softmax warps)
 // The convert warps rewrite buffer b for tile j + kBufs only after KFree, SclFree and
 // VFree of tile j, so no waiter on CvtK or CvtV can find its barrier two phases ahead.
-// A code stage s (tile j, phase j / kStages) is free (Empty) once the 128 convert
-// threads have read its codes and S^T has read its queries.
+// A code stage s (tile j, phase j / kStages) is free (Empty) once the 8 convert warps
+// have read its codes and S^T has read its queries.
 constexpr int kBarFull = 0, kBarEmpty = kStages, kBarCvtK = 2 * kStages, kBarCvtV = kBarCvtK + kBufs,
               kBarKFree = kBarCvtV + kBufs, kBarVFree = kBarKFree + kBufs, kBarSclFree = kBarVFree + kBufs,
               kBarSFull = kBarSclFree + kBufs, kBarSFree = kBarSFull + 2, kBarPFull = kBarSFree + 2,
@@ -154,9 +154,10 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fp8_kernel(const __grid_co
       const bool many = (i >= kBarCvtK && i < kBarKFree) || (i >= kBarSclFree && i < kBarSclFree + kBufs) ||
                         i == kBarSFree || i == kBarSFree + 1 || i == kBarPFull || i == kBarPFull + 1;
       const bool empty = i >= kBarEmpty && i < kBarEmpty + kStages;
-      // the convert and softmax warps arrive once per warp; a code stage is also released
-      // by the S^T issuer's commit
-      mbar_init(bar(i), empty ? 5 : (many ? 4 : 1));
+      // the convert (8) and softmax (4) warps arrive once per warp; a code stage is also
+      // released by the S^T issuer's commit
+      const bool cvt = i >= kBarCvtK && i < kBarKFree;
+      mbar_init(bar(i), empty ? 9 : (cvt ? 8 : (many ? 4 : 1)));
     }
     fence_mbar_init();
     *abort_flag = 0;
@@ -271,13 +272,15 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fp8_kernel(const __grid_co
       mbar_wait(drain, 0, p.status);
     }
   } else if (warp >= 6) {
-    // ================= convert warps (6-9) =================
+    // ================= convert warps (6-9: dims 0-63, 11-14: dims 64-127) =================
     const int wq = warp & 3;
     const int t = (wq << 5) | lane;
+    const int hf = warp >= 11 ? 1 : 0;                     // which half of the row
+    const int cw = hf * 4 + ((warp - (hf ? 11 : 6)) & 3);  // convert warp 0..7
     const uint32_t tm_lane = tmem + (static_cast<uint32_t>(wq << 5) << 16);
-    float *cred = reinterpret_cast<float *>(smem + kSmCred);  // [parity][4 warps][2]
+    float *cred = reinterpret_cast<float *>(smem + kSmCred);  // [buffer][8 warps][2]
     // After an abort the loop still runs to its end (on whatever the buffers hold): the
-    // four warps meet at a named barrier every tile, so none may leave early.
+    // eight warps meet at a named barrier every tile, so none may leave early.
     bool ok = true;
     UnitIter it(a, u0);
     for (int j = 0; j < nu; ++j, it.next()) {
@@ -291,31 +294,29 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fp8_kernel(const __grid_co
       const bool valid = static_cast<int64_t>(it.un.tile) * kTile + t < p.len;
       const float sk = valid ? reinterpret_cast<const float *>(st + kStKs)[t] : 0.f;
       const float sv = valid ? reinterpret_cast<const float *>(st + kStVs)[t] : 0.f;
-      // this thread's 16 query elements: half h, row r, 16-byte chunks c0, c0 + 1
+      // this thread's 8 query elements: half qh, row qr, 16-byte chunk qc + hf
       const int qh = t >> 6, qr = (t & 63) >> 2, qc = (t & 3) * 2;
       char *qrow = st + kStQ + qh * 2048 + qr * 128;
-      uint4 qw[2];
+      uint4 *pq = reinterpret_cast<uint4 *>(qrow + (((qc + hf) ^ (qr & 7)) << 4));
+      const uint4 qw = qr < G ? *pq : make_uint4(0, 0, 0, 0);
       float qmax = 0.f;
-#pragma unroll
-      for (int u = 0; u < 2; ++u) {
-        uint4 *pq = reinterpret_cast<uint4 *>(qrow + (((qc + u) ^ (qr & 7)) << 4));
-        qw[u] = qr < G ? *pq : make_uint4(0, 0, 0, 0);
-        const uint32_t w4[4] = {qw[u].x, qw[u].y, qw[u].z, qw[u].w};
+      {
+        const uint32_t w4[4] = {qw.x, qw.y, qw.z, qw.w};
 #pragma unroll
         for (int e = 0; e < 4; ++e) qmax = fmaxf(qmax, fmaxf(fabsf(bf16lo(w4[e])), fabsf(bf16hi(w4[e]))));
       }
-      // tile-wide largest |q| and largest V scale, over the 128 convert threads
+      // tile-wide largest |q| and largest V scale, over the 256 convert threads
       const float wqm = warp_max(qmax), wsm = warp_max(sv);
       if (lane == 0) {
-        cred[(b * 4 + wq) * 2] = wqm;
-        cred[(b * 4 + wq) * 2 + 1] = wsm;
+        cred[(b * 8 + cw) * 2] = wqm;
+        cred[(b * 8 + cw) * 2 + 1] = wsm;
       }
-      tc::named_sync(2, 128);
+      tc::named_sync(2, 256);
       float qm = 0.f, smax = 0.f;
 #pragma unroll
-      for (int w = 0; w < 4; ++w) {
-        qm = fmaxf(qm, cred[(b * 4 + w) * 2]);
-        smax = fmaxf(smax, cred[(b * 4 + w) * 2 + 1]);
+      for (int w = 0; w < 8; ++w) {
+        qm = fmaxf(qm, cred[(b * 8 + w) * 2]);
+        smax = fmaxf(smax, cred[(b * 8 + w) * 2 + 1]);
       }
       // 2^e with the largest |q| in [2^13, 2^14): every query element fits fp16 exactly
       // unless it is 2^24 times smaller than the largest (then it only rounds)
@@ -326,21 +327,21 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fp8_kernel(const __grid_co
         e = e < -100 ? -100 : (e > 100 ? 100 : e);
       }
       const float qs = __int_as_float((127 + e) << 23);  // 2^e, exact
-#pragma unroll
-      for (int u = 0; u < 2; ++u) {
-        const uint32_t w4[4] = {qw[u].x, qw[u].y, qw[u].z, qw[u].w};
+      {
+        const uint32_t w4[4] = {qw.x, qw.y, qw.z, qw.w};
         uint4 o;
         o.x = f16x2_bits(bf16lo(w4[0]) * qs, bf16hi(w4[0]) * qs);
         o.y = f16x2_bits(bf16lo(w4[1]) * qs, bf16hi(w4[1]) * qs);
         o.z = f16x2_bits(bf16lo(w4[2]) * qs, bf16hi(w4[2]) * qs);
         o.w = f16x2_bits(bf16lo(w4[3]) * qs, bf16hi(w4[3]) * qs);
-        *reinterpret_cast<uint4 *>(qrow + (((qc + u) ^ (qr & 7)) << 4)) = o;
+        *pq = o;
       }
       // K row t -> TMEM lane t, 64 columns of fp16 pairs (dims 2c, 2c+1 in column c);
-      // 8 chunks of 16 codes: chunk c holds dims 16c .. 16c+15 = columns 8c .. 8c+7
+      // 8 chunks of 16 codes: chunk c holds dims 16c .. 16c+15 = columns 8c .. 8c+7.
+      // This thread widens chunks 4 hf .. 4 hf + 3.
       const int rot = t & 7;
 #pragma unroll
-      for (int q4 = 0; q4 < 4; ++q4) {  // 2 chunks -> 16 columns per store
+      for (int q4 = 2 * hf; q4 < 2 * hf + 2; ++q4) {  // 2 chunks -> 16 columns per store
         uint32_t cols[16];
 #pragma unroll
         for (int cc = 0; cc < 2; ++cc) {
@@ -355,10 +356,12 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fp8_kernel(const __grid_co
       }
       // the token's factors for the softmax: logit = S * s_k * 2^-e * scale * log2(e),
       // P' = p * s_v / smax
-      float *scl = reinterpret_cast<float *>(smem + kSmScl + b * kSclBytes);
-      scl[t] = sk * __int_as_float((127 - e) << 23) * p.scale_log2;
-      scl[128 + t] = smax > 0.f ? sv / smax : 0.f;
-      if (t == 0) scl[256] = smax;
+      if (hf == 0) {
+        float *scl = reinterpret_cast<float *>(smem + kSmScl + b * kSclBytes);
+        scl[t] = sk * __int_as_float((127 - e) << 23) * p.scale_log2;
+        scl[128 + t] = smax > 0.f ? sv / smax : 0.f;
+        if (t == 0) scl[256] = smax;
+      }
       tc::st_wait();
       tc::fence_async_smem();  // Q16 is read by the MMA (async proxy)
       tc::fence_before();
@@ -368,7 +371,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fp8_kernel(const __grid_co
       if (ok && j >= kBufs) ok = tc::wait_bar(bar(kBarVFree + b), ph, p.status, abort_flag);
       char *vbuf = smem + kSmV + b * 32768;
 #pragma unroll
-      for (int c = 0; c < 8; ++c) {
+      for (int c = 4 * hf; c < 4 * hf + 4; ++c) {
         const uint4 w = *reinterpret_cast<const uint4 *>(st + kStVc + t * 128 + ((c ^ rot) << 4));
         uint4 o0, o1;
         widen4(w.x, o0.x, o0.y);
