@@ -418,32 +418,55 @@ DecodeParams decode_params(const duo_cache *c, const Layer &ly, const void *q, v
   return p;
 }
 
+// SMs for a quantised layer's bf16 streaming heads, decoded beside its retrieval heads:
+// a share in proportion to their bytes (1.5 times, a lone CTA hides less latency), at
+// least one, at most an eighth of the SMs, and no more than their tiles.
+static int streaming_ctas(const DecodeParams &p, int num_sms, bool int4) {
+  const int64_t slots = static_cast<int64_t>(p.S) + p.W, reach = static_cast<int64_t>(p.S) + p.len;
+  const int64_t used = reach < slots ? reach : slots;
+  const int64_t units_s = static_cast<int64_t>(p.B) * p.Hs * ((used + 127) / 128);
+  const int64_t units_r = static_cast<int64_t>(p.B) * p.Hr * ((p.len + 127) / 128);
+  const double bs = static_cast<double>(units_s) * 128 * p.D * 2 * 2;                 // bf16 K and V
+  const double br = static_cast<double>(units_r) * 128 * (int4 ? 2 * (p.D / 2 + 4) : 2 * (p.D + 4));
+  int k = static_cast<int>(1.5 * num_sms * bs / (bs + br) + 0.999);
+  const int hi = num_sms / 8 > 1 ? num_sms / 8 : 1;
+  k = k < 1 ? 1 : (k > hi ? hi : k);
+  return static_cast<int>(units_s < k ? (units_s > 0 ? units_s : 1) : k);
+}
+
+// A quantised layer: its bf16 streaming heads on the bf16 kernel (a few CTAs, leading)
+// and its retrieval heads on the INT4 or FP8 kernel beside it on the other SMs; the two
+// write disjoint heads, partial rows and tickets.  Each launch goes through the test
+// controls when `hooked`.
+static cudaError_t launch_quantised_layer(const duo_cache *c, const DecodeParams &p, bool int4, bool hooked,
+                                          cudaStream_t st) {
+  auto run = [&](auto &&f) { return hooked ? launch_via_hook(f) : f(); };
+  int rest = c->num_sms;
+  DecodeParams pr = p;
+  if (p.Hs > 0) {
+    DecodeParams ps = p;
+    ps.Hr = 0;
+    ps.pdl_mode = 1;
+    const int k = streaming_ctas(p, c->num_sms, int4);
+    const cudaError_t e = run([&] { return launch_decode_tc(ps, k, true, st); });
+    if (e != cudaSuccess) return e;
+    rest -= k;
+    pr.pdl_mode = 2;
+  }
+  return run([&] {
+    return int4 ? launch_decode_int4_tc(pr, rest, true, st) : launch_decode_fp8_tc(pr, rest, true, st);
+  });
+}
+
 cudaError_t launch_decode_any(const duo_cache *c, const DecodeParams &p, cudaStream_t st) {
   const bool int4 = c->fmt == DUO_KV_INT4_G128;
   if (c->fmt == DUO_KV_FP8_E4M3) {
-    // bf16 streaming heads on the bf16 kernel, then the FP8 retrieval heads
     if (!decode_fp8_tc_supported(p, c->dtype)) return cudaErrorNotSupported;
-    if (p.Hs > 0) {
-      DecodeParams ps = p;
-      ps.Hr = 0;
-      const cudaError_t e = launch_decode_tc(ps, c->num_sms, true, st);
-      if (e != cudaSuccess) return e;
-    }
-    return launch_decode_fp8_tc(p, c->num_sms, true, st);
+    return launch_quantised_layer(c, p, false, false, st);
   }
   // the tcgen05 decodes overlap their start-up with the previous kernel on the stream
-  if (int4 && decode_int4_tc_supported(p, c->dtype)) {
-    // the bf16 streaming heads on the bf16 kernel (a few tiles), then the INT4 retrieval
-    // heads; the two write disjoint heads, partial rows and tickets
-    // (decode_int4_tc_supported implies decode_tc_supported for that view)
-    if (p.Hs > 0) {
-      DecodeParams ps = p;
-      ps.Hr = 0;
-      const cudaError_t e = launch_decode_tc(ps, c->num_sms, true, st);
-      if (e != cudaSuccess) return e;
-    }
-    return launch_decode_int4_tc(p, c->num_sms, true, st);
-  }
+  // (decode_int4_tc_supported implies decode_tc_supported for the streaming view)
+  if (int4 && decode_int4_tc_supported(p, c->dtype)) return launch_quantised_layer(c, p, true, false, st);
   if (decode_tc_supported(p, c->dtype, int4)) return launch_decode_tc(p, c->num_sms, true, st);
   return launch_decode(p, c->dtype, int4, st);
 }
@@ -454,14 +477,7 @@ cudaError_t decode_any(const duo_cache *c, const DecodeParams &p, cudaStream_t s
   const bool fp8 = c->fmt == DUO_KV_FP8_E4M3 && decode_fp8_tc_supported(p, c->dtype);
   if (dry_run() || (!int4 && !fp8) || p.Hs == 0) return launch_via_hook([&] { return launch_decode_any(c, p, st); });
   // quantised layer with streaming heads: two launches (each counted by the test controls)
-  DecodeParams ps = p;
-  ps.Hr = 0;
-  cudaError_t e = launch_via_hook([&] { return launch_decode_tc(ps, c->num_sms, true, st); });
-  if (e != cudaSuccess) return e;
-  DecodeParams pr = p;
-  return launch_via_hook([&] {
-    return int4 ? launch_decode_int4_tc(pr, c->num_sms, true, st) : launch_decode_fp8_tc(pr, c->num_sms, true, st);
-  });
+  return launch_quantised_layer(c, p, int4, true, st);
 }
 
 bool decode_args_ok(const void *q, const void *out, const float *lse) {

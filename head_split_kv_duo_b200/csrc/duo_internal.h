@@ -109,6 +109,16 @@ struct DecodeParams {
   // position npos = len - 1; the CTA that reads a row's tile writes it first
   const char *nk, *nv;
   int64_t npos;
+  // Programmatic dependent launch of a quantised layer's two decodes (the bf16 streaming
+  // heads and the quantised retrieval heads, disjoint heads, partial rows and tickets):
+  //   0  alone: dependents are released at once; global memory is touched only after the
+  //      previous grid on the stream has completed
+  //   1  leading (the streaming heads, on a few CTAs): dependents are released only once
+  //      the previous grid has completed, so that the next grid may start at once
+  //   2  beside the leader (the retrieval heads, on the other SMs): no wait at the start
+  //      (the leader's release implies the grid before it has completed); the grid waits
+  //      for the leader before it ends, so that whatever follows it sees both complete
+  int pdl_mode;
 };
 
 struct PrefillParams {

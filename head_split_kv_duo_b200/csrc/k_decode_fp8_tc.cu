@@ -185,8 +185,9 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fp8_kernel(const __grid_co
           prefetch_l2(p.rv_sz + row * 4, kTile * 4);
         }
       }
-      // launched as a programmatic dependent: no global read before the previous kernel ends
-      asm volatile("griddepcontrol.wait;" ::: "memory");
+      // launched as a programmatic dependent: no global read before the previous kernel
+      // ends (beside a leading grid, that grid's release already implies it)
+      if (p.pdl_mode != 2) asm volatile("griddepcontrol.wait;" ::: "memory");
       int issued = 0;
       UnitIter it(a, u0);
       for (int j = 0; j < nu; ++j, it.next()) {
@@ -580,6 +581,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fp8_kernel(const __grid_co
   tc::fence_before();
   __syncthreads();
   tc::fence_after();
+  if (p.pdl_mode == 2 && tid == 0) asm volatile("griddepcontrol.wait;" ::: "memory");  // the leader has ended
   if (warp == 1) tc::tmem_free(tmem, kTmemCols);
 }
 

@@ -280,7 +280,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_int4_kernel(const __grid_c
       // Launched as a programmatic dependent, this grid's set-up overlaps the previous
       // kernel on the stream; nothing is read from global memory before that kernel has
       // finished (every other read and every write of this grid follows these loads).
-      asm volatile("griddepcontrol.wait;" ::: "memory");
+      if (p.pdl_mode != 2) asm volatile("griddepcontrol.wait;" ::: "memory");  // (beside a leader: implied)
       int prev_item = -1, issued = 0;
       UnitIter it(a, u0);
       for (int j = 0; j < nu; ++j, it.next()) {
@@ -724,6 +724,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_int4_kernel(const __grid_c
   tc::fence_before();
   __syncthreads();
   tc::fence_after();
+  if (p.pdl_mode == 2 && tid == 0) asm volatile("griddepcontrol.wait;" ::: "memory");  // the leader has ended
   if (warp == 1) tc::tmem_free(tmem, C::kAlloc);
 }
 

@@ -267,8 +267,9 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   // A decode launched next on the stream may start its set-up on the SMs this grid
   // frees; it touches global memory only after its own griddepcontrol.wait, which
-  // returns once this whole grid has completed.
-  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  // returns once this whole grid has completed.  A leading grid (pdl_mode 1) releases
+  // its dependent only after its own wait (below).
+  if (p.pdl_mode != 1) asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   const int64_t u0 = cta_begin(a, blockIdx.x), u1 = cta_begin(a, blockIdx.x + 1);
   const int nu = static_cast<int>(u1 - u0);
   const int G = p.G;
@@ -314,6 +315,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
       // finished (every other read and every write of this grid follows this wait or the
       // append warp's).
       asm volatile("griddepcontrol.wait;" ::: "memory");
+      if (p.pdl_mode == 1) asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     }
     if (lane == 0) {
       // contiguous cache, fused append: the tile of each item that holds the appended row
