@@ -138,6 +138,7 @@ bool layer_ok(const duo_cache *c, int layer) { return c && layer >= 0 && layer <
 // Test controls (duo_debug_launch_controls): process-wide.
 std::atomic<int> g_dry_run{0};
 std::atomic<int64_t> g_fail_countdown{-1};
+std::atomic<int> g_device_stall{0};
 
 duo_status ensure_init(duo_cache *c, cudaStream_t st) {
   if (c->initialised) return DUO_OK;
@@ -372,6 +373,7 @@ namespace {
 DecodeParams decode_params(const duo_cache *c, const Layer &ly, const void *q, void *out, float *lse) {
   const bool int4 = c->fmt == DUO_KV_INT4_G128;
   DecodeParams p{};
+  p.debug_stall = g_device_stall.load(std::memory_order_relaxed);
   p.q = static_cast<const char *>(q);
   p.out = static_cast<char *>(out);
   p.lse = lse;
@@ -624,6 +626,12 @@ duo_status duo_debug_launch_controls(int dry_run, int64_t fail_after) {
   if ((dry_run != 0 && dry_run != 1) || fail_after < -1) return DUO_ERR_INVALID;
   g_dry_run.store(dry_run);
   g_fail_countdown.store(fail_after);
+  return DUO_OK;
+}
+
+duo_status duo_debug_device_stall(int on) {
+  if (on != 0 && on != 1) return DUO_ERR_INVALID;
+  g_device_stall.store(on);
   return DUO_OK;
 }
 

@@ -119,6 +119,9 @@ struct DecodeParams {
   //      (the leader's release implies the grid before it has completed); the grid waits
   //      for the leader before it ends, so that whatever follows it sees both complete
   int pdl_mode;
+  // test control (duo_debug_device_stall): the bf16 decode's softmax first waits for a
+  // barrier that nothing arrives at, so that its bounded wait runs out
+  int debug_stall;
 };
 
 struct PrefillParams {

@@ -50,7 +50,9 @@ constexpr int kSmemAlloc = kSmMisc + 64 + 1024;
 // Double-buffered resources (S, P, O) each have one barrier per buffer, so that no
 // barrier can complete two phases ahead of the thread waiting on it (parity waits).
 constexpr int kBarFull = 0, kBarEmpty = 3, kBarSFull = 6, kBarSFree = 8, kBarPFull = 10, kBarOFull = 12,
-              kBarDrain = 14, kBarAppend = 15, kBarMerge = 16, kNumBars = 17;
+              kBarDrain = 14, kBarAppend = 15, kBarMerge = 16,
+              kBarStall = 17,  // test control: nothing ever arrives here
+              kNumBars = 18;
 
 // ---- work plans: how the flattened 128-token units of a launch map onto items ----
 //
@@ -543,6 +545,8 @@ __global__ void __launch_bounds__(kThreads, 1) decode_tc_kernel(const __grid_con
     UnitIter<Plan> iter(a, u0);
     for (int j = 0; j < nu; ++j, iter.next(a)) {
       const Item &un = iter.it;
+      // test control: a wait that runs out (the bounded-wait and abort paths on a GPU)
+      if (j == 0 && p.debug_stall && ok) ok = tc::wait_bar(bar(kBarStall), 0, p.status, abort_flag);
       if (ok) ok = tc::wait_bar(bar(kBarSFull + (j & 1)), (j >> 1) & 1, p.status, abort_flag);
       tc::fence_after();
       float sv[NQ];

@@ -48,7 +48,6 @@ constexpr int kD = 128;
 constexpr int kKStages = 2;  // K ring: a stage is free once S_1(j) is computed
 constexpr int kVStages = 2;  // V ring: a stage is free once P_1(j) V_j is computed
 constexpr int kMaxStrmTiles = 48;
-constexpr int kPolyExp = 0;   // exponentials of every 32 (interior tiles) on the FMA pipe
 
 // shared memory map (bytes from the 1 KiB-aligned base); every tile is two 128B-swizzled
 // [128][64] bf16 halves of 16 KiB
@@ -138,31 +137,11 @@ __device__ __forceinline__ float fmax3(float a, float b, float c) {
   return d;
 }
 
-// 2^x of a pair on the FMA pipe: x = n + f with n the nearest integer (|f| <= 1/2),
-// 2^f by a cubic fitted for this kernel by weighted least squares on [-1/2, 1/2]
-// (maximum relative error 1.0e-4, below bf16's 2^-9), and n added to the exponent
-// field.  Arguments below -126 give 2^-126 (the callers' tiles hold no -inf).
-__device__ __forceinline__ void exp2_poly2(uint64_t x2, float &r0, float &r1) {
-  float x0, x1;
-  unpack2(x2, x0, x1);
-  x2 = pack2(fmaxf(x0, -126.0f), fmaxf(x1, -126.0f));
-  const uint64_t t = fadd2(x2, pack2(12582912.0f, 12582912.0f));  // 1.5 * 2^23: rounds to an integer
-  const uint64_t n = fadd2(t, pack2(-12582912.0f, -12582912.0f));
-  const uint64_t f = ffma2(n, pack2(-1.0f, -1.0f), x2);  // x - n, exact
-  uint64_t q = ffma2(pack2(0.05500858f, 0.05500858f), f, pack2(0.24221036f, 0.24221036f));
-  q = ffma2(q, f, pack2(0.6932829f, 0.6932829f));
-  q = ffma2(q, f, pack2(1.0f, 1.0f));
-  float q0, q1, t0, t1;
-  unpack2(q, q0, q1);
-  unpack2(t, t0, t1);
-  r0 = __int_as_float(__float_as_int(q0) + (__float_as_int(t0) << 23));
-  r1 = __int_as_float(__float_as_int(q1) + (__float_as_int(t1) << 23));
-}
-
-// exp2(v*c - mc) of the N logits v[B .. B+N), their sum into rowsum and bf16 pairs into pk; logits
-// [P0, P0+PN) use the FMA-pipe polynomial (which needs finite arguments), the rest MUFU.
-// The scaling and the sums run on packed fp32 pairs.
-template <int N, int P0, int PN, int B = 0, int M>
+// exp2(v*c - mc) of the N logits v[B .. B+N) on MUFU, their sum into rowsum and bf16
+// pairs into pk.  The scaling and the sums run on packed fp32 pairs.  (With two query
+// tiles in ping-pong, moving part of the exponentials to an FMA-pipe polynomial only
+// added instructions.)
+template <int N, int B = 0, int M>
 __device__ __forceinline__ void probabilities(const float (&v)[M], float c, float mc, float &rowsum,
                                               uint32_t (&pk)[N / 2]) {
   static_assert(B + N <= M, "logit range");
@@ -171,15 +150,9 @@ __device__ __forceinline__ void probabilities(const float (&v)[M], float c, floa
 #pragma unroll
   for (int e = 0; e < N; e += 2) {
     const uint64_t x = ffma2(pack2(v[B + e], v[B + e + 1]), cc, mm);
-    float p0, p1;
-    if (e >= P0 && e < P0 + PN) {
-      exp2_poly2(x, p0, p1);
-    } else {
-      float x0, x1;
-      unpack2(x, x0, x1);
-      p0 = ex2(x0);
-      p1 = ex2(x1);
-    }
+    float x0, x1;
+    unpack2(x, x0, x1);
+    const float p0 = ex2(x0), p1 = ex2(x1);
     acc[(e >> 1) & 1] = fadd2(acc[(e >> 1) & 1], pack2(p0, p1));
     const __nv_bfloat162 pb = __floats2bfloat162_rn(p0, p1);
     pk[e >> 1] = *reinterpret_cast<const uint32_t *>(&pb);
@@ -255,11 +228,11 @@ __device__ __forceinline__ void ld128(uint32_t taddr, float (&v)[128]) {
 #undef DUO_O16
 
 // P of logits v[B .. B+32) as 16 bf16 pairs into TMEM columns B/2 .. B/2+15 of s_cols
-// (no wait), their sum into rs; PN of the 32 exponentials on the FMA pipe
-template <int B, int PN>
+// (no wait), their sum into rs
+template <int B>
 __device__ __forceinline__ void p_chunk(const float (&v)[128], float c, float mc, float &rs, uint32_t s_cols) {
   uint32_t pk[16];
-  probabilities<32, 0, PN, B>(v, c, mc, rs, pk);
+  probabilities<32, B>(v, c, mc, rs, pk);
   tc::st16(s_cols + B / 2, pk);
 }
 
@@ -469,9 +442,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) prefill_tc_kernel(const __grid_
           win_c = clamp_col(win_rel);
         }
       }
-      // warp-uniform (the branches below issue warp-collective TMEM stores): a warp
-      // with any masked row takes the masked path, a no-op for its other rows
-      const bool full_vis = __all_sync(0xffffffffu, hi >= kBN - 1 && (sink_c >= kBN || win_c < 0));
+      const bool full_vis = hi >= kBN - 1 && (sink_c >= kBN || win_c < 0);
 
       if (ok) ok = tc::wait_bar(bar(kBarSFull + qt), j & 1, p.status, abort_flag);
       tc::fence_after();
@@ -514,17 +485,10 @@ __global__ void __launch_bounds__(kTcThreads, 1) prefill_tc_kernel(const __grid_
       // over the first 64 columns of S_t
       const float mc = (m == -INFINITY) ? 0.f : m;
       float rs[4];
-      if (!full_vis) {
-        p_chunk<0, 0>(v, c, mc, rs[0], s_cols);
-        p_chunk<32, 0>(v, c, mc, rs[1], s_cols);
-        p_chunk<64, 0>(v, c, mc, rs[2], s_cols);
-        p_chunk<96, 0>(v, c, mc, rs[3], s_cols);
-      } else {
-        p_chunk<0, kPolyExp>(v, c, mc, rs[0], s_cols);
-        p_chunk<32, kPolyExp>(v, c, mc, rs[1], s_cols);
-        p_chunk<64, kPolyExp>(v, c, mc, rs[2], s_cols);
-        p_chunk<96, kPolyExp>(v, c, mc, rs[3], s_cols);
-      }
+      p_chunk<0>(v, c, mc, rs[0], s_cols);
+      p_chunk<32>(v, c, mc, rs[1], s_cols);
+      p_chunk<64>(v, c, mc, rs[2], s_cols);
+      p_chunk<96>(v, c, mc, rs[3], s_cols);
       const float rsum = (rs[0] + rs[1]) + (rs[2] + rs[3]);
       tc::st_wait();
       tc::fence_before();

@@ -81,6 +81,8 @@ def lib() -> ctypes.CDLL:
                                               ctypes.c_float, vp, vp]
             L.duo_debug_launch_controls.restype = i32
             L.duo_debug_launch_controls.argtypes = [i32, i64]
+            L.duo_debug_device_stall.restype = i32
+            L.duo_debug_device_stall.argtypes = [i32]
             L.duo_pool_bytes.restype = ctypes.c_size_t
             L.duo_pool_bytes.argtypes = [i32, i32, i32, vp, i32, i32, i32, i64, i64, ctypes.POINTER(duo_opts)]
             L.duo_pool_create.restype = i32
@@ -209,6 +211,10 @@ def duo_gated_attention(q, k, v, batch, seq_len, q_heads, kv_heads, head_dim, dt
 
 def duo_debug_launch_controls(dry_run: int, fail_after: int) -> int:
     return lib().duo_debug_launch_controls(int(dry_run), int(fail_after))
+
+
+def duo_debug_device_stall(on: int) -> int:
+    return lib().duo_debug_device_stall(int(on))
 
 
 def duo_pool_bytes(layers, kv_heads, head_dim, retrieval_head_mask, S, W, max_seqs, max_len, num_pages,

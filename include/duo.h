@@ -374,6 +374,19 @@ DUO_API duo_status duo_gated_attention(const void *q, const void *k, const void 
  */
 DUO_API duo_status duo_debug_launch_controls(int dry_run, int64_t fail_after);
 
+/*
+ * Test control of the device-side timeout path, process-wide (tests only; the paper has
+ * no counterpart).  on = 1: every bf16 tensor-core decode of a contiguous cache
+ * (duo_decode_attention, duo_append_decode, and the streaming heads of an INT4 or FP8
+ * layer) makes its softmax warps wait first for a barrier that nothing arrives at.  That
+ * bounded wait runs out after about 2 s; the kernel latches DUO_ERR_TIMEOUT in the
+ * cache's status word (read by duo_get_device_status), every role of every CTA stops
+ * waiting, drains its copies and products and exits, and the call's outputs are
+ * undefined.  The CUDA context stays usable.  on = 0: normal operation.
+ * DUO_ERR_INVALID for other values.
+ */
+DUO_API duo_status duo_debug_device_stall(int on);
+
 /* Static description of a status code. */
 DUO_API const char *duo_status_str(duo_status status);
 

@@ -230,6 +230,13 @@ def dry_run():
     assert duo.duo_debug_launch_controls(0, -1) == duo.DUO_OK
 
 
+def test_device_stall_control_checks_its_argument():
+    assert duo.duo_debug_device_stall(2) == duo.DUO_ERR_INVALID
+    assert duo.duo_debug_device_stall(-1) == duo.DUO_ERR_INVALID
+    assert duo.duo_debug_device_stall(1) == duo.DUO_OK
+    assert duo.duo_debug_device_stall(0) == duo.DUO_OK
+
+
 def test_launch_controls_reject_bad_values():
     assert duo.duo_debug_launch_controls(2, -1) == duo.DUO_ERR_INVALID
     assert duo.duo_debug_launch_controls(0, -2) == duo.DUO_ERR_INVALID
