@@ -147,6 +147,41 @@ __device__ __forceinline__ void ld_i32(uint32_t taddr, int (&v)[N]) {
     for (int i = 0; i < 16; ++i) v[c + i] = __float_as_int(f[i]);
   }
 }
+// N (a multiple of 16) int32 columns of this thread's TMEM lane, loads issued only:
+// ld_i32_wait names every destination register, so that no use precedes the wait
+template <int N>
+__device__ __forceinline__ void ld_i32_issue(uint32_t taddr, uint32_t (&r)[N]) {
+#pragma unroll
+  for (int c = 0; c < N; c += 16) {
+    uint32_t *q = r + c;
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+        "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15}, [%16];"
+        : "=r"(q[0]), "=r"(q[1]), "=r"(q[2]), "=r"(q[3]), "=r"(q[4]), "=r"(q[5]), "=r"(q[6]), "=r"(q[7]), "=r"(q[8]),
+          "=r"(q[9]), "=r"(q[10]), "=r"(q[11]), "=r"(q[12]), "=r"(q[13]), "=r"(q[14]), "=r"(q[15])
+        : "r"(taddr + c));
+  }
+}
+template <int N>
+__device__ __forceinline__ void ld_i32_wait(uint32_t (&r)[N]) {
+  static_assert(N == 16 || N == 32, "16 or 32 columns");
+  if constexpr (N == 16) {
+    asm volatile("tcgen05.wait::ld.sync.aligned;"
+                 : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]), "+r"(r[6]), "+r"(r[7]),
+                   "+r"(r[8]), "+r"(r[9]), "+r"(r[10]), "+r"(r[11]), "+r"(r[12]), "+r"(r[13]), "+r"(r[14]), "+r"(r[15])
+                 :
+                 : "memory");
+  } else {
+    asm volatile("tcgen05.wait::ld.sync.aligned;"
+                 : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]), "+r"(r[6]), "+r"(r[7]),
+                   "+r"(r[8]), "+r"(r[9]), "+r"(r[10]), "+r"(r[11]), "+r"(r[12]), "+r"(r[13]), "+r"(r[14]), "+r"(r[15]),
+                   "+r"(r[16]), "+r"(r[17]), "+r"(r[18]), "+r"(r[19]), "+r"(r[20]), "+r"(r[21]), "+r"(r[22]),
+                   "+r"(r[23]), "+r"(r[24]), "+r"(r[25]), "+r"(r[26]), "+r"(r[27]), "+r"(r[28]), "+r"(r[29]),
+                   "+r"(r[30]), "+r"(r[31])
+                 :
+                 : "memory");
+  }
+}
 // byte (row n, column k) of a [rows][128 B] K-major operand with 128-byte swizzle
 __device__ __forceinline__ int sw128(int n, int k) { return (n >> 3) * 1024 + (n & 7) * 128 + (((k >> 4) ^ (n & 7)) << 4) + (k & 15); }
 
@@ -522,15 +557,26 @@ __global__ void __launch_bounds__(kThreads, 1) decode_int4_kernel(const __grid_c
       if (t == 0) p.counters[pitem] = 0u;  // ready for the next call
     };
 
-    // o = (o + O^T(jj)) * alpha for this thread's row of O^T
-    auto fold = [&](int jj, float sigp, const float (&alpha)[NQ]) {
+    // o = (o + O^T(jj)) * alpha for this thread's row of O^T, in two halves: the load of
+    // O^T(jj) is issued at the start of the group's next tile (its product has long run)
+    // and the rows are added once that tile's alpha is known, so that the load's
+    // latency overlaps the tile's arithmetic
+    uint32_t orow[C::kO];
+    auto fold_issue = [&](int jj) {
       if (ok) ok = tc::wait_bar(bar(kBarOFull + (jj & 3)), (jj >> 2) & 1, p.status, abort_flag);
       tc::fence_after();
-      int r[C::kO];
-      ld_i32<C::kO>(lane_base + 2 * C::kS + (jj & 3) * C::kO, r);
+      ld_i32_issue<C::kO>(lane_base + 2 * C::kS + (jj & 3) * C::kO, orow);
+    };
+    auto fold_finish = [&](float sigp, const float (&alpha)[NQ]) {
+      ld_i32_wait<C::kO>(orow);
 #pragma unroll
       for (int q = 0; q < NQ; ++q)  // |R| < 2^22
-        o[q] = fmaf(sigp, fmaf(to_float(r[2 * q + 1]), 1.f / 254.f, to_float(r[2 * q])), o[q]) * alpha[q];
+        o[q] = fmaf(sigp, fmaf(to_float(static_cast<int>(orow[2 * q + 1])), 1.f / 254.f,
+                               to_float(static_cast<int>(orow[2 * q]))), o[q]) * alpha[q];
+    };
+    auto fold = [&](int jj, float sigp, const float (&alpha)[NQ]) {
+      fold_issue(jj);
+      fold_finish(sigp, alpha);
     };
     float one[NQ];
 #pragma unroll
@@ -570,6 +616,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_int4_kernel(const __grid_c
       ld_i32<C::kS>(lane_base + cb * C::kS, sr);
       tc::fence_before();
       mbar_arrive_warp(bar(kBarSFree + cb));  // S buffer j % 2 is free again
+      if (jp >= 0) fold_issue(jp);  // finished below, once alpha is known
       // the stage's prep is complete (its S^T product has run); waiting here orders the
       // prep warps' writes before these reads
       if (ok) ok = tc::wait_bar(bar(kBarCvt + s), (j / kStages) & 1, p.status, abort_flag);
@@ -624,7 +671,8 @@ __global__ void __launch_bounds__(kThreads, 1) decode_int4_kernel(const __grid_c
       // P'^T limbs into buffer j % 4 (its previous reader, tile j-4 of this group, was
       // folded at tile j-2): p s_v = sigp (l0 + l1 / 254) with l0 = rint(x) in [0, 127],
       // x = p s_v / sigp, l1 = rint(254 (x - l0)) in [-127, 127]; sigp = tmax / 126.99
-      const float invp = tmax > 0.f ? 126.99f / tmax : 0.f;
+      // (approximate division: the limbs only need x <= 126.99 (1 + 2^-21) < 127.5)
+      const float invp = tmax > 0.f ? __fdividef(126.99f, tmax) : 0.f;
       const float zi = mi.z * invp;
       uint8_t *pb = reinterpret_cast<uint8_t *>(smem + kSmP + (j & 3) * 4096);
 #pragma unroll
@@ -646,7 +694,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_int4_kernel(const __grid_c
       mbar_arrive_warp(bar(kBarPFull + (j & 3)));
       // fold this group's previous tile of the item, bringing it to this tile's scale
       if (jp >= 0) {
-        fold(jp, sigp_prev, alpha);
+        fold_finish(sigp_prev, alpha);
       } else {
 #pragma unroll
         for (int q = 0; q < NQ; ++q) o[q] *= alpha[q];
