@@ -59,7 +59,7 @@ constexpr int kStKc = 0, kStVc = 8192, kStLv = 16384, kStKsz = 24576, kStVsz = 2
               kStTmax = 27648, kStQ = 28672, kStage = 32768;
 constexpr int kQlBytes = 6144;                 // query limbs [48][128 B] s8, 128-byte swizzle
 constexpr int kSmQl = kStages * kStage;        // 2 x query limbs (item parity)
-constexpr int kSmP = kSmQl + 2 * kQlBytes;     // 4 x P' limbs [32][128 B] s8; flush exchanges
+constexpr int kSmP = kSmQl + 2 * kQlBytes;     // 4 x P'^T limbs (MN-major, 4 KiB each); flush exchanges
 constexpr int kSmQinfo = kSmP + 4 * 4096;      // [2][32]: sigma[16], sum(q)[16] per query head
 constexpr int kSmRed = kSmQinfo + 256;         // per softmax group [4][16] l, [4][16] zc; [128][6] merge
 constexpr int kSmBar = kSmRed + (2 * 128 + 128 * 6) * 4;
@@ -104,8 +104,8 @@ __device__ __forceinline__ uint64_t sdesc_l(uint32_t saddr, uint32_t lbo, uint32
          (static_cast<uint64_t>((sbo >> 4) & 0x3FFFu) << 32) | (1ull << 46) | (static_cast<uint64_t>(layout) << 61);
 }
 // kind::i8 instruction descriptor: int32 accumulator, A unsigned, B signed or unsigned
-constexpr uint32_t idesc_i8(int M, int N, bool b_signed, bool a_mn_major) {
-  return (2u << 4) | ((b_signed ? 1u : 0u) << 10) | ((a_mn_major ? 1u : 0u) << 15) |
+constexpr uint32_t idesc_i8(int M, int N, bool b_signed, bool a_mn_major, bool b_mn_major = false) {
+  return (2u << 4) | ((b_signed ? 1u : 0u) << 10) | ((a_mn_major ? 1u : 0u) << 15) | ((b_mn_major ? 1u : 0u) << 16) |
          ((static_cast<uint32_t>(N) >> 3) << 17) | ((static_cast<uint32_t>(M) >> 4) << 24);
 }
 __device__ __forceinline__ void mma_i8(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc, uint32_t acc) {
@@ -358,7 +358,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_int4_kernel(const __grid_c
     // has completed by then (the softmax saw it land before writing P'(j)).
     if (lane == 0) {
       constexpr uint32_t kIdS = idesc_i8(128, C::kS, true, false);   // [U | L] . Qx^T
-      constexpr uint32_t kIdO = idesc_i8(128, C::kO, true, true);    // [U_V | L_V]^T . P'^T
+      constexpr uint32_t kIdO = idesc_i8(128, C::kO, true, true, true);  // [U_V | L_V]^T . P'^T (both MN-major)
       constexpr uint32_t kStDesc = kStage >> 4;                       // one stage in descriptor units
       bool ok = true;
       if (warp == 1) {
@@ -398,7 +398,10 @@ __global__ void __launch_bounds__(kThreads, 1) decode_int4_kernel(const __grid_c
         }
       } else {
         const uint64_t av0 = sdesc_l(sbase + kStVc, kStLv - kStVc, 512, 4);  // MN-major, 2 chunks
-        const uint64_t bp0 = sdesc_l(sbase + kSmP, 16, 1024, 2);
+        // P'^T MN-major without swizzle: 16 limb bytes of a token per row, 8 tokens per
+        // 128-byte core matrix (the leading byte offset steps along the tokens), blocks of
+        // 16 limb rows 2 KiB apart
+        const uint64_t bp0 = sdesc_l(sbase + kSmP, 128, 2048, 0);
         int os = 0;  // stage of O^T(jo)
         for (int jo = 0; jo < nu && ok; ++jo) {
           if (!(ok = tc::wait_bar(bar(kBarPFull + (jo & 3)), (jo >> 2) & 1, p.status, abort_flag))) break;
@@ -408,7 +411,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_int4_kernel(const __grid_c
           const uint32_t d = tmem + 2 * C::kS + (jo & 3) * C::kO;
 #pragma unroll
           for (int k = 0; k < 4; ++k)  // 32 tokens per step
-            mma_i8(d, av + k * (2048 >> 4), bp + k * 2, kIdO, k > 0 ? 1u : 0u);
+            mma_i8(d, av + k * (2048 >> 4), bp + k * (512 >> 4), kIdO, k > 0 ? 1u : 0u);
           tc::commit(bar(kBarOFull + (jo & 3)));
           tc::commit(bar(kBarEmpty + os));  // the stage and its K low nibbles are no longer read
           if (++os == kStages) os = 0;
@@ -674,20 +677,37 @@ __global__ void __launch_bounds__(kThreads, 1) decode_int4_kernel(const __grid_c
       // (approximate division: the limbs only need x <= 126.99 (1 + 2^-21) < 127.5)
       const float invp = tmax > 0.f ? __fdividef(126.99f, tmax) : 0.f;
       const float zi = mi.z * invp;
-      uint8_t *pb = reinterpret_cast<uint8_t *>(smem + kSmP + (j & 3) * 4096);
+      // limb bytes of this token, row n = 2q + limb of P'^T, four to a word (heads q >= G
+      // have p = 0 and give zero bytes)
+      constexpr int kPB = 2 * NQ;
+      uint32_t pw[(kPB + 3) / 4];
+#pragma unroll
+      for (int w = 0; w < (kPB + 3) / 4; ++w) pw[w] = 0u;
 #pragma unroll
       for (int q = 0; q < NQ; ++q) {
         const float pv = (valid && q < G && m[q] != -INFINITY) ? ex2(fmaf(sv[q], c, -m[q])) : 0.f;
         l[q] = fmaf(l[q], alpha[q], pv);
         zc[q] = fmaf(zc[q], alpha[q], pv * mi.w);
-        if (q < G) {
-          const float x = pv * zi;
-          float r0, r1;
-          const uint32_t b0 = round_byte(x, r0);
-          const uint32_t b1 = round_byte((x - r0) * 254.f, r1);
-          pb[sw128(2 * q, t)] = static_cast<uint8_t>(b0);
-          pb[sw128(2 * q + 1, t)] = static_cast<uint8_t>(b1);
-        }
+        const float x = pv * zi;
+        float r0, r1;
+        const uint32_t b0 = round_byte(x, r0);
+        const uint32_t b1 = round_byte((x - r0) * 254.f, r1);
+        pw[(2 * q) >> 2] |= b0 << (8 * ((2 * q) & 3));
+        pw[(2 * q + 1) >> 2] |= b1 << (8 * ((2 * q + 1) & 3));
+      }
+      // P'^T is MN-major without swizzle: token t's limb bytes are contiguous, 16 per
+      // 2 KiB block (byte (n, t) at (n / 16) * 2048 + 16 t + n % 16): one store
+      char *pt = smem + kSmP + (j & 3) * 4096 + 16 * t;
+      if constexpr (kPB == 2) {
+        *reinterpret_cast<uint16_t *>(pt) = static_cast<uint16_t>(pw[0]);
+      } else if constexpr (kPB == 4) {
+        *reinterpret_cast<uint32_t *>(pt) = pw[0];
+      } else if constexpr (kPB == 8) {
+        *reinterpret_cast<uint2 *>(pt) = make_uint2(pw[0], pw[1]);
+      } else {
+#pragma unroll
+        for (int b = 0; b < kPB / 16; ++b)
+          *reinterpret_cast<uint4 *>(pt + 2048 * b) = make_uint4(pw[4 * b], pw[4 * b + 1], pw[4 * b + 2], pw[4 * b + 3]);
       }
       tc::fence_async_smem();
       tc::fence_before();
