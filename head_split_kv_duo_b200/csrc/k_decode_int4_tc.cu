@@ -640,11 +640,23 @@ __global__ void __launch_bounds__(kThreads, 1) decode_int4_kernel(const __grid_c
         qread = true;
       }
       float sv[NQ];
+      if constexpr (NQ >= 2) {
+        // two heads per packed fp32 instruction; the same roundings as one head at a time
+        const uint64_t nmag = pack2(-kMagic, -kMagic), r128 = pack2(1.f / 128.f, 1.f / 128.f);
+        const uint64_t kx = pack2(mi.x, mi.x), ky = pack2(mi.y, mi.y);
+        auto limbs = [&](int i, int q) {  // exact int -> float of limb i of heads q, q + 1
+          return fadd2(pack2(__int_as_float(sr[3 * q + i] + kMagicBits), __int_as_float(sr[3 * q + 3 + i] + kMagicBits)),
+                       nmag);
+        };
 #pragma unroll
-      for (int q = 0; q < NQ; ++q) {  // S0 + S1 / 2^7 + S2 / 2^14, |S| < 2^22
-        const float x = fmaf(fmaf(to_float(sr[3 * q + 2]), 1.f / 128.f, to_float(sr[3 * q + 1])), 1.f / 128.f,
-                             to_float(sr[3 * q]));
-        sv[q] = fmaf(mi.x, sg[q] * x, mi.y * qs[q]);
+        for (int q = 0; q < NQ; q += 2) {  // S0 + S1 / 2^7 + S2 / 2^14, |S| < 2^22
+          const uint64_t x = ffma2(ffma2(limbs(2, q), r128, limbs(1, q)), r128, limbs(0, q));
+          const uint64_t v = ffma2(kx, fmul2(pack2(sg[q], sg[q + 1]), x), fmul2(ky, pack2(qs[q], qs[q + 1])));
+          unpack2(v, sv[q], sv[q + 1]);
+        }
+      } else {
+        const float x = fmaf(fmaf(to_float(sr[2]), 1.f / 128.f, to_float(sr[1])), 1.f / 128.f, to_float(sr[0]));
+        sv[0] = fmaf(mi.x, sg[0] * x, mi.y * qs[0]);
       }
       // does any logit of this tile exceed the group's running max?
       int need = 0;
@@ -683,17 +695,41 @@ __global__ void __launch_bounds__(kThreads, 1) decode_int4_kernel(const __grid_c
       uint32_t pw[(kPB + 3) / 4];
 #pragma unroll
       for (int w = 0; w < (kPB + 3) / 4; ++w) pw[w] = 0u;
+      float pv[NQ];
 #pragma unroll
-      for (int q = 0; q < NQ; ++q) {
-        const float pv = (valid && q < G && m[q] != -INFINITY) ? ex2(fmaf(sv[q], c, -m[q])) : 0.f;
-        l[q] = fmaf(l[q], alpha[q], pv);
-        zc[q] = fmaf(zc[q], alpha[q], pv * mi.w);
-        const float x = pv * zi;
+      for (int q = 0; q < NQ; ++q) pv[q] = (valid && q < G && m[q] != -INFINITY) ? ex2(fmaf(sv[q], c, -m[q])) : 0.f;
+      // l, zc and the limb bytes, two heads per packed instruction where NQ >= 2 (the same
+      // roundings: (x - r0) * 254 is exact before its one rounding, as x * 254 - 254 r0 is)
+      auto limb_bytes = [&](int q, float x) {
         float r0, r1;
         const uint32_t b0 = round_byte(x, r0);
         const uint32_t b1 = round_byte((x - r0) * 254.f, r1);
         pw[(2 * q) >> 2] |= b0 << (8 * ((2 * q) & 3));
         pw[(2 * q + 1) >> 2] |= b1 << (8 * ((2 * q + 1) & 3));
+      };
+      if constexpr (NQ >= 2) {
+        const uint64_t mag = pack2(kMagic, kMagic), nmag = pack2(-kMagic, -kMagic), f254 = pack2(254.f, 254.f),
+                       n254 = pack2(-254.f, -254.f), w2 = pack2(mi.w, mi.w), zi2 = pack2(zi, zi);
+#pragma unroll
+        for (int q = 0; q < NQ; q += 2) {
+          const uint64_t p2 = pack2(pv[q], pv[q + 1]), a2 = pack2(alpha[q], alpha[q + 1]);
+          unpack2(ffma2(pack2(l[q], l[q + 1]), a2, p2), l[q], l[q + 1]);
+          unpack2(ffma2(pack2(zc[q], zc[q + 1]), a2, fmul2(p2, w2)), zc[q], zc[q + 1]);
+          const uint64_t x2 = fmul2(p2, zi2);
+          const uint64_t t2 = fadd2(x2, mag);                       // x + 1.5 * 2^23: rint(x) in the low bits
+          const uint64_t u2 = fadd2(ffma2(x2, f254, fmul2(fadd2(t2, nmag), n254)), mag);
+          float t0, t1, u0, u1;
+          unpack2(t2, t0, t1);
+          unpack2(u2, u0, u1);
+          pw[(2 * q) >> 2] |= (static_cast<uint32_t>(__float_as_int(t0)) & 0xFFu) << (8 * ((2 * q) & 3));
+          pw[(2 * q + 1) >> 2] |= (static_cast<uint32_t>(__float_as_int(u0)) & 0xFFu) << (8 * ((2 * q + 1) & 3));
+          pw[(2 * q + 2) >> 2] |= (static_cast<uint32_t>(__float_as_int(t1)) & 0xFFu) << (8 * ((2 * q + 2) & 3));
+          pw[(2 * q + 3) >> 2] |= (static_cast<uint32_t>(__float_as_int(u1)) & 0xFFu) << (8 * ((2 * q + 3) & 3));
+        }
+      } else {
+        l[0] = fmaf(l[0], alpha[0], pv[0]);
+        zc[0] = fmaf(zc[0], alpha[0], pv[0] * mi.w);
+        limb_bytes(0, pv[0] * zi);
       }
       // P'^T is MN-major without swizzle: token t's limb bytes are contiguous, 16 per
       // 2 KiB block (byte (n, t) at (n / 16) * 2048 + 16 t + n % 16): one store
