@@ -67,7 +67,7 @@ static_assert(kSmemAlloc <= 232448, "shared memory");
 constexpr int kBarFull = 0, kBarEmpty = kStages, kBarSFull = 2 * kStages, kBarSFree = kBarSFull + 2,
               kBarPFull = kBarSFull + 4, kBarOFull = kBarSFull + 8, kBarQFree = kBarSFull + 12,
               kBarQInfo = kBarSFull + 14, kBarDrain = kBarSFull + 16,  // a drain barrier per issuer
-              kNumBars = kBarSFull + 18;
+              kBarMerge = kBarSFull + 18, kNumBars = kBarSFull + 19;
 static_assert(kNumBars * 8 <= 256, "barrier area");
 
 // tensor memory columns: S^T x 2 and O^T x 4, three limb columns per query head each
@@ -264,6 +264,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fp8_kernel(const __grid_co
       mbar_init(bar(kBarPFull + i), 4);  // one arrival per warp of a softmax group
       mbar_init(bar(kBarOFull + i), 1);
     }
+    mbar_init(bar(kBarMerge), 1);  // partial rows copied in for the final merge
     fence_mbar_init();
     *abort_flag = 0;
   }
@@ -445,7 +446,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fp8_kernel(const __grid_co
     // Both groups arrive here when an item ends, every tile of it folded.  Group 1 hands
     // its state over; group 0 combines the two, writes this CTA's result for `item`
     // (partial or final) and merges when last.
-    auto flush = [&](int item) {
+    auto flush = [&](int item, bool final_flush) {
 #pragma unroll
       for (int q = 0; q < NQ; ++q) {
         const float vl = warp_sum(l[q]);
@@ -511,14 +512,32 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fp8_kernel(const __grid_co
         }
       __threadfence();
       tc::named_sync(gbar, 128);
+      // at the CTA's last item the code stages are idle (every load consumed, every
+      // product run): the merging CTA copies the item's partial rows in with one bulk
+      // copy and merges from shared memory (1: merge from global memory, 2: from here)
+      const uint32_t bytes = static_cast<uint32_t>(nseg) * G * kPartRow * 4;
       if (t == 0) {
         const uint32_t prev = atomicAdd(p.counters + pitem, 1u);
-        *last_flag = (prev == static_cast<uint32_t>(nseg - 1)) ? 1 : 0;
+        const bool here = final_flush && bytes <= static_cast<uint32_t>(kSmQl) && *abort_flag == 0;
+        *last_flag = (prev == static_cast<uint32_t>(nseg - 1)) ? (here ? 2 : 1) : 0;
       }
       tc::named_sync(gbar, 128);
-      if (!*last_flag) return;
+      const int how = *last_flag;
+      if (!how) return;
       __threadfence();
-      merge_partials(part, nseg, G, b, h0, p.Hq, p.out, p.lse, red + 128, t, gbar);
+      if (how == 2) {
+        if (t == 0) {
+          asm volatile("fence.proxy.async.global;" ::: "memory");  // the rows were written by other CTAs
+          mbar_expect_tx(bar(kBarMerge), bytes);
+          bulk_g2s(sbase, part, bytes, bar(kBarMerge));
+        }
+        // waited for even after an abort (bounded): the copy must not outlive the CTA
+        if (!mbar_wait(bar(kBarMerge), 0, p.status)) ok = false;
+        merge_partials<true>(reinterpret_cast<const float *>(smem), nseg, G, b, h0, p.Hq, p.out, p.lse, red + 128, t,
+                             gbar);
+      } else {
+        merge_partials(part, nseg, G, b, h0, p.Hq, p.out, p.lse, red + 128, t, gbar);
+      }
       if (t == 0) p.counters[pitem] = 0u;  // ready for the next call
     };
 
@@ -561,7 +580,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fp8_kernel(const __grid_co
           if (jp >= 0) fold(jp, sigp_prev, one);
           jp = -1;
           release_unread();
-          flush(cur_item);
+          flush(cur_item, false);
         }
         ++nitem;
 #pragma unroll
@@ -698,7 +717,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_fp8_kernel(const __grid_co
     if (nu > 0) {
       if (jp >= 0) fold(jp, sigp_prev, one);
       release_unread();
-      flush(cur_item);
+      flush(cur_item, true);
     }
   }
 
