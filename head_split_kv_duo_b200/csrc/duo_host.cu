@@ -6,6 +6,7 @@
 #include <new>
 
 #include "duo_internal.h"
+#include "nvtx_range.h"
 
 using namespace duo;
 
@@ -211,6 +212,7 @@ size_t duo_cache_bytes(int layers, int kv_heads, int head_dim, const uint8_t *ma
 
 duo_status duo_cache_create(int layers, int kv_heads, int head_dim, const uint8_t *mask, int S, int W,
                             int64_t max_len, const duo_opts *opts, void *dev_buf, size_t dev_bytes, duo_cache **out) {
+  DUO_NVTX_RANGE("duo_cache_create");
   if (!out) return DUO_ERR_INVALID;
   *out = nullptr;
   Cfg c;
@@ -273,6 +275,7 @@ duo_status duo_cache_create(int layers, int kv_heads, int head_dim, const uint8_
 void duo_cache_destroy(duo_cache *cache) { delete cache; }
 
 duo_status duo_append_kv(duo_cache *c, int layer, const void *k, const void *v, int n, void *stream) {
+  DUO_NVTX_RANGE("duo_append_kv");
   if (!layer_ok(c, layer) || !k || !v || n < 1 || !aligned16(k) || !aligned16(v)) return DUO_ERR_INVALID;
   Layer &ly = c->L[layer];
   if (ly.len + n > c->max_len) return DUO_ERR_CAPACITY;
@@ -287,6 +290,7 @@ duo_status duo_append_kv(duo_cache *c, int layer, const void *k, const void *v, 
 
 duo_status duo_prefill_chunk(duo_cache *c, int layer, const void *q, const void *k, const void *v, int n, void *out,
                              float *lse, void *stream) {
+  DUO_NVTX_RANGE("duo_prefill_chunk");
   if (!layer_ok(c, layer) || !q || !k || !v || !out || n < 1) return DUO_ERR_INVALID;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) ||
       (reinterpret_cast<uintptr_t>(lse) & 3u))
@@ -491,6 +495,7 @@ bool decode_args_ok(const void *q, const void *out, const float *lse) {
 extern "C" {
 
 duo_status duo_decode_attention(duo_cache *c, int layer, const void *q, void *out, float *lse, void *stream) {
+  DUO_NVTX_RANGE("duo_decode_attention");
   if (!layer_ok(c, layer) || !decode_args_ok(q, out, lse)) return DUO_ERR_INVALID;
   Layer &ly = c->L[layer];
   if (ly.len < 1) return DUO_ERR_INVALID;
@@ -503,6 +508,7 @@ duo_status duo_decode_attention(duo_cache *c, int layer, const void *q, void *ou
 
 duo_status duo_append_decode(duo_cache *c, int layer, const void *q, const void *k, const void *v, void *out,
                              float *lse, void *stream) {
+  DUO_NVTX_RANGE("duo_append_decode");
   if (!layer_ok(c, layer) || !decode_args_ok(q, out, lse) || !k || !v || !aligned16(k) || !aligned16(v))
     return DUO_ERR_INVALID;
   Layer &ly = c->L[layer];
@@ -611,6 +617,7 @@ duo_status duo_debug_region(const duo_cache *c, int layer, duo_region which, voi
 }
 
 duo_status duo_get_device_status(duo_cache *c, void *stream) {
+  DUO_NVTX_RANGE("duo_get_device_status");
   if (!c) return DUO_ERR_INVALID;
   if (!c->initialised || dry_run()) return DUO_OK;
   cudaStream_t st = static_cast<cudaStream_t>(stream);

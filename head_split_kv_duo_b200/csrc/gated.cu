@@ -14,6 +14,7 @@
 #include <cmath>
 
 #include "duo_internal.h"
+#include "nvtx_range.h"
 
 namespace duo {
 
@@ -67,6 +68,7 @@ extern "C" duo_status duo_gated_attention(const void *q, const void *k, const vo
                                           int q_heads, int kv_heads, int head_dim, duo_dtype dtype,
                                           const float *alpha, int S, int W, float softmax_scale, void *out,
                                           void *stream) {
+  DUO_NVTX_RANGE("duo_gated_attention");
   using namespace duo;
   if (!gated_args_ok(batch, seq_len, q_heads, kv_heads, head_dim, dtype, S, W)) return DUO_ERR_INVALID;
   if (!q || !k || !v || !alpha || !out || !(softmax_scale >= 0.f) || !std::isfinite(softmax_scale))

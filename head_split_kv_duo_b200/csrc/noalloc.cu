@@ -11,6 +11,7 @@
 #include <mutex>
 
 #include "duo_internal.h"
+#include "nvtx_range.h"
 
 namespace {
 
@@ -48,6 +49,7 @@ duo_status scratch_for_current_device(unsigned char **out) {
 
 extern "C" duo_status duo_decode_attention_static_scratch(duo_cache *c, int layer, const void *q, void *out,
                                                           float *lse, void *stream) {
+  DUO_NVTX_RANGE("duo_decode_attention_static_scratch");
   using namespace duo;
   if (!c || layer < 0 || layer >= c->layers || !q || !out) return DUO_ERR_INVALID;
   if ((reinterpret_cast<uintptr_t>(q) & 15u) || (reinterpret_cast<uintptr_t>(out) & 15u) ||

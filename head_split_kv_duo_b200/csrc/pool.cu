@@ -21,6 +21,7 @@
 
 #include "decode_merge.cuh"
 #include "tcgen05.cuh"
+#include "nvtx_range.h"
 
 struct duo_pool {
   int layers = 0, Hkv = 0, Hq = 0, G = 0, D = 0, S = 0, W = 0, max_seqs = 0, pages_per_seq = 0;
@@ -303,6 +304,7 @@ size_t duo_pool_bytes(int layers, int kv_heads, int head_dim, const uint8_t *mas
 duo_status duo_pool_create(int layers, int kv_heads, int head_dim, const uint8_t *mask, int S, int W, int max_seqs,
                            int64_t max_len, int64_t num_pages, const duo_opts *opts, void *dev_buf, size_t dev_bytes,
                            duo_pool **out) {
+  DUO_NVTX_RANGE("duo_pool_create");
   if (!out) return DUO_ERR_INVALID;
   *out = nullptr;
   int Hq = 0;
@@ -368,6 +370,7 @@ duo_status duo_pool_create(int layers, int kv_heads, int head_dim, const uint8_t
 void duo_pool_destroy(duo_pool *pool) { delete pool; }
 
 duo_status duo_pool_open(duo_pool *P, void *stream, int *seq) {
+  DUO_NVTX_RANGE("duo_pool_open");
   if (!P || !seq) return DUO_ERR_INVALID;
   int s = -1;
   for (int i = 0; i < P->max_seqs; ++i)
@@ -441,6 +444,7 @@ duo_status duo_pool_region(const duo_pool *P, int layer, duo_region which, void 
 }
 
 duo_status duo_pool_append_kv(duo_pool *P, int layer, int seq, const void *k, const void *v, int n, void *stream) {
+  DUO_NVTX_RANGE("duo_pool_append_kv");
   if (!seq_ok(P, seq) || layer < 0 || layer >= P->layers || !k || !v || n < 1) return DUO_ERR_INVALID;
   if ((reinterpret_cast<uintptr_t>(k) | reinterpret_cast<uintptr_t>(v)) & 15u) return DUO_ERR_INVALID;
   const int64_t len = P->len[seq][layer];
@@ -506,6 +510,7 @@ duo_status duo_pool_append_kv(duo_pool *P, int layer, int seq, const void *k, co
 
 duo_status duo_pool_decode_step(duo_pool *P, int layer0, int nlayers, int nseq, const int *seqs, const void *q,
                                 const void *k, const void *v, void *out, float *lse, void *stream) {
+  DUO_NVTX_RANGE("duo_pool_decode_step");
   if (!P || nlayers < 1 || layer0 < 0 || layer0 + nlayers > P->layers || nseq < 1 || nseq > kPoolMaxSeqs ||
       nlayers * nseq > kPoolMaxSuper || !seqs || !q || !k || !v || !out)
     return DUO_ERR_INVALID;
@@ -603,6 +608,7 @@ duo_status duo_pool_decode_step(duo_pool *P, int layer0, int nlayers, int nseq, 
 }
 
 duo_status duo_pool_device_status(duo_pool *P, void *stream) {
+  DUO_NVTX_RANGE("duo_pool_device_status");
   if (!P) return DUO_ERR_INVALID;
   if (!P->initialised || dry_run()) return DUO_OK;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
