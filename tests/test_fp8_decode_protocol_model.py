@@ -20,85 +20,16 @@ can run and some role is unfinished is a deadlock.
 
 The model runs on the CPU and no GPU fault can come from it.  It checks the protocol
 the kernel implements, including items of a single tile, where one softmax group
-releases an item's queries unread.  It does not check the kernel itself.
+releases an item's queries unread.  It does not check the kernel itself.  It is
+sequentially consistent.  A wait that exists for memory visibility cannot be shown
+necessary here: the QInfo wait, before the softmax reads 2^-e_q, is already implied by
+S^T having landed.
 """
-import random
-
 import pytest
 
+from protocol_sim import Sim, units_of, wait
+
 K_STAGES = 5
-
-
-class Barrier:
-    def __init__(self, name, count):
-        self.name, self.count, self.pending, self.phases = name, count, 0, 0
-
-    def arrive(self, sim):
-        self.pending += 1
-        assert self.pending <= self.count, f"{self.name}: too many arrivals"
-        if self.pending == self.count:
-            self.pending = 0
-            self.phases += 1
-            for (b, k) in sim.blocked_on():
-                if b is self:
-                    assert self.phases <= k + 1, f"{self.name}: phase {k} overrun by a waiter's barrier"
-
-
-class Sim:
-    def __init__(self, seed):
-        self.rng = random.Random(seed)
-        self.bars = {}
-        self.buf = {}
-        self.actors = []  # [generator, pending wait (bar, phase) or None, name]
-
-    def bar(self, name, count=1):
-        if name not in self.bars:
-            self.bars[name] = Barrier(name, count)
-        return self.bars[name]
-
-    def write(self, buf, version):
-        self.buf[buf] = version
-
-    def read(self, buf, version):
-        assert self.buf.get(buf) == version, f"read of {buf}: expected {version}, found {self.buf.get(buf)}"
-
-    def arrive(self, name):
-        self.bars[name].arrive(self)
-
-    def spawn(self, gen, name):
-        self.actors.append([gen, None, name])
-
-    def blocked_on(self):
-        return [a[1] for a in self.actors if a[1] is not None]
-
-    def run(self, limit=200000):
-        steps = 0
-        while self.actors:
-            steps += 1
-            assert steps < limit, "no progress"
-            runnable = []
-            for a in self.actors:
-                w = a[1]
-                if w is None or (w[0].phases & 1) != (w[1] & 1):
-                    runnable.append(a)
-            assert runnable, "deadlock: " + ", ".join(f"{a[2]} waits {a[1][0].name} phase {a[1][1]}"
-                                                      for a in self.actors)
-            a = self.rng.choice(runnable)
-            if a[1] is not None:
-                b, k = a[1]
-                assert b.phases == k + 1, f"{a[2]}: wait on {b.name} for phase {k} passed at phase count {b.phases}"
-                a[1] = None
-            try:
-                req = next(a[0])
-            except StopIteration:
-                self.actors.remove(a)
-                continue
-            if req is not None:  # ('wait', barrier name, phase index)
-                a[1] = (self.bars[req[1]], req[2])
-
-
-def wait(name, k):
-    return ("wait", name, k)
 
 
 def fp8_cta(sim, units, ring=4, sfree_wait=True):
@@ -271,14 +202,6 @@ def fp8_cta(sim, units, ring=4, sfree_wait=True):
     sim.spawn(mma_engine(o_queue, "o"), "o_mma")
     sim.spawn(softmax(0), "softmax0")
     sim.spawn(softmax(1), "softmax1")
-
-
-def units_of(tiles_per_item, first_tile=0):
-    out = []
-    for i, n in enumerate(tiles_per_item):
-        t0 = first_tile if i == 0 else 0
-        out += [(i, t0 + t) for t in range(n)]
-    return out
 
 
 CASES = [
