@@ -163,6 +163,17 @@ def test_bf16_protocol_random_interleavings(tiles):
         sim.run()
 
 
+@pytest.mark.parametrize("tiles", [[5], [1, 2, 3, 4], [8, 8, 1]], ids=["5", "1.2.3.4", "8.8.1"])
+def test_bf16_protocol_pool_plan(tiles):
+    """The pooled cache's plan: the same roles with no fused append (the pool appends
+    in a launch of its own before the decode)."""
+    units = units_of(tiles)
+    for seed in range(300):
+        sim = Sim(seed)
+        bf16_cta(sim, units, set())
+        sim.run()
+
+
 def _caught(tiles, seeds=300, **mistake):
     units = units_of(tiles)
     n = 0
